@@ -1,0 +1,391 @@
+// C ABI of libpi (declared in include/pi.h): argument validation, workspace
+// layout and the stream-ordered launch sequences of each entry point.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "pi.h"
+#include "pi_common.cuh"
+#include "pi_kernels.cuh"
+
+namespace pi {
+namespace {
+
+thread_local char g_err[512] = "";
+
+pi_status fail(pi_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+pi_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PI_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int words_of(int F) { return (F + 31) / 32; }
+
+// Validates one layer descriptor.
+pi_status check_layer(const pi_layer* L, int i) {
+  if (!L) return fail(PI_ERR_INVALID, "layer %d: null descriptor", i);
+  const int d = L->d_model, F = L->d_ff, r = L->rank, H = L->hot;
+  if (d < 1 || d > PI_MAX_D_MODEL) return fail(PI_ERR_INVALID, "layer %d: d_model %d out of range", i, d);
+  if (F < 1 || F > PI_MAX_D_FF) return fail(PI_ERR_INVALID, "layer %d: d_ff %d out of range", i, F);
+  if (r < 1 || r > PI_MAX_RANK) return fail(PI_ERR_INVALID, "layer %d: rank %d out of range", i, r);
+  if (H < 0 || H > F) return fail(PI_ERR_INVALID, "layer %d: hot %d not in [0, d_ff]", i, H);
+  if (L->act != PI_RELU && L->act != PI_REGLU)
+    return fail(PI_ERR_INVALID, "layer %d: unknown activation %d", i, L->act);
+  if (L->w_dtype != PI_F32 && L->w_dtype != PI_F16 && L->w_dtype != PI_Q4_0)
+    return fail(PI_ERR_INVALID, "layer %d: unknown weight dtype %d", i, L->w_dtype);
+  if (L->p_dtype == PI_Q4_0)
+    return fail(PI_ERR_UNSUPPORTED, "layer %d: Q4_0 predictor weights are not supported", i);
+  if (L->p_dtype != PI_F32 && L->p_dtype != PI_F16)
+    return fail(PI_ERR_INVALID, "layer %d: unknown predictor dtype %d", i, L->p_dtype);
+  const int dmul = L->w_dtype == PI_Q4_0 ? 32 : 8;
+  if (d % dmul) return fail(PI_ERR_INVALID, "layer %d: d_model %d not a multiple of %d", i, d, dmul);
+  if (L->p_dtype == PI_F32 ? (d % 4) : (d % 8))
+    return fail(PI_ERR_INVALID, "layer %d: d_model %d not a multiple of the predictor chunk", i, d);
+  if (L->p_dtype == PI_F32 ? (r % 4) : (r % 8))
+    return fail(PI_ERR_INVALID, "layer %d: rank %d not a multiple of %d", i, r,
+                L->p_dtype == PI_F32 ? 4 : 8);
+  const bool reglu = L->act == PI_REGLU, q4 = L->w_dtype == PI_Q4_0;
+  if (!L->w_up || !L->w_down_t || !L->p1 || !L->p2 || (reglu && !L->w_gate))
+    return fail(PI_ERR_INVALID, "layer %d: null weight pointer", i);
+  if (q4 && (!L->w_up_scales || !L->w_down_t_scales || (reglu && !L->w_gate_scales)))
+    return fail(PI_ERR_INVALID, "layer %d: Q4_0 weights need scale arrays", i);
+  const void* w16[] = {L->w_up, L->w_down_t, L->p1, L->p2, reglu ? L->w_gate : L->w_up};
+  for (const void* p : w16)
+    if (!aligned(p, 16)) return fail(PI_ERR_INVALID, "layer %d: weight pointer not 16-byte aligned", i);
+  if (q4) {
+    const void* s2[] = {L->w_up_scales, L->w_down_t_scales, reglu ? L->w_gate_scales : L->w_up_scales};
+    for (const void* p : s2)
+      if (!aligned(p, 2)) return fail(PI_ERR_INVALID, "layer %d: scale pointer not 2-byte aligned", i);
+  }
+  if ((L->bias && !aligned(L->bias, 4)) || (L->p_bias && !aligned(L->p_bias, 4)))
+    return fail(PI_ERR_INVALID, "layer %d: bias pointer not 4-byte aligned", i);
+  return PI_OK;
+}
+
+WsLayout layout_for(int d, int F, int r, int batch) {
+  WsLayout w{};
+  size_t off = sizeof(WsHeader);
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  w.splits = down_splits(batch, d);
+  w.xh = take((size_t)batch * d * 4);
+  w.u = take((size_t)batch * r * 4);
+  w.mask = take((size_t)batch * words_of(F) * 4);
+  w.idx = take((size_t)F * 4);
+  w.count = take(16);
+  w.h = take((size_t)F * batch * 4);
+  w.part = take((size_t)w.splits * batch * d * 4);
+  w.y = take((size_t)batch * d * 4);
+  w.total = off;
+  return w;
+}
+
+WsLayout layout_for_layers(const pi_layer* layers, int n, int batch) {
+  int d = 0, F = 0, r = 0;
+  for (int l = 0; l < n; ++l) {
+    d = d > layers[l].d_model ? d : layers[l].d_model;
+    F = F > layers[l].d_ff ? F : layers[l].d_ff;
+    r = r > layers[l].rank ? r : layers[l].rank;
+  }
+  return layout_for(d, F, r, batch);
+}
+
+pi_status check_ws(void* ws, size_t ws_bytes, const WsLayout& lay) {
+  if (!ws) return fail(PI_ERR_INVALID, "null workspace");
+  if (!aligned(ws, 256)) return fail(PI_ERR_INVALID, "workspace not 256-byte aligned");
+  if (ws_bytes < lay.total)
+    return fail(PI_ERR_INVALID, "workspace too small: %zu < %zu bytes", ws_bytes, lay.total);
+  return PI_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>((char*)ws + off); }
+
+WsHeader* header(void* ws) { return reinterpret_cast<WsHeader*>(ws); }
+uint32_t* status_word(void* ws) { return &header(ws)->status; }
+
+float logit32(float tau) { return (float)std::log((double)tau / (1.0 - (double)tau)); }
+
+// Optional per-launch event recorder used by pi_ffn_stack_profile.
+struct Prof {
+  cudaEvent_t* ev = nullptr;  // 2 per launch
+  int* kind = nullptr;
+  int cap = 0, n = 0;
+  cudaStream_t s = nullptr;
+  void before(int k) {
+    if (!ev || n >= cap) return;
+    kind[n] = k;
+    cudaEventRecord(ev[2 * n], s);
+  }
+  void after() {
+    if (!ev || n >= cap) return;
+    cudaEventRecord(ev[2 * n + 1], s);
+    ++n;
+  }
+};
+
+pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                   int per_token, const int32_t* idx, const int32_t* count, const float* resid,
+                   float* out, void* ws, const WsLayout& lay, cudaStream_t s,
+                   Prof* prof = nullptr) {
+  Prof none;
+  Prof& P = prof ? *prof : none;
+  P.before(PI_KIND_FFN_UP);
+  cudaError_t e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h),
+                                header(ws), s);
+  P.after();
+  if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
+  const int S = down_splits(batch, L.d_model);
+  P.before(PI_KIND_FFN_DOWN);
+  e = launch_ffn_down(L, batch, idx, count, at<float>(ws, lay.h), at<float>(ws, lay.part), S,
+                      header(ws), s);
+  P.after();
+  if (e != cudaSuccess) return cuda_fail(e, "ffn_down launch");
+  P.before(PI_KIND_REDUCE);
+  e = launch_reduce(at<float>(ws, lay.part), S, batch, L.d_model, resid, out, s);
+  P.after();
+  if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
+  return PI_OK;
+}
+
+pi_status stack_check(const pi_layer* layers, int n_layers, float* x, int batch, float tau,
+                      int mode, uint32_t* mask_trace, void* ws, size_t ws_bytes, WsLayout* lay) {
+  if (!layers || n_layers < 1) return fail(PI_ERR_INVALID, "need at least one layer");
+  pi_status st;
+  for (int l = 0; l < n_layers; ++l) {
+    if ((st = check_layer(&layers[l], l)) != PI_OK) return st;
+    if (layers[l].d_model != layers[0].d_model || layers[l].d_ff != layers[0].d_ff)
+      return fail(PI_ERR_INVALID, "layer %d: all layers must share d_model and d_ff", l);
+  }
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID, "batch %d not in [1, 64]", batch);
+  if (!(tau > 0.f && tau < 1.f)) return fail(PI_ERR_INVALID, "tau must lie in (0, 1)");
+  if (mode != PI_MASK_PER_TOKEN && mode != PI_MASK_UNION) return fail(PI_ERR_INVALID, "unknown mask mode %d", mode);
+  if (!x || !aligned(x, 16)) return fail(PI_ERR_INVALID, "x null or not 16-byte aligned");
+  if (mask_trace && !aligned(mask_trace, 4)) return fail(PI_ERR_INVALID, "mask_trace misaligned");
+  *lay = layout_for_layers(layers, n_layers, batch);
+  return check_ws(ws, ws_bytes, *lay);
+}
+
+pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, float tau,
+                    int mode, uint32_t* mask_trace, void* ws, const WsLayout& lay,
+                    cudaStream_t s, Prof* prof) {
+  Prof none;
+  Prof& P = prof ? *prof : none;
+  pi_status st;
+  const float theta = logit32(tau);
+  const int d = layers[0].d_model, words = words_of(layers[0].d_ff);
+  const int per_token = (mode == PI_MASK_PER_TOKEN && batch > 1);
+  float* xh = at<float>(ws, lay.xh);
+  int32_t* idx = at<int32_t>(ws, lay.idx);
+  int32_t* cnt = at<int32_t>(ws, lay.count);
+  for (int l = 0; l < n_layers; ++l) {
+    const pi_layer& L = layers[l];
+    uint32_t* mask = mask_trace ? mask_trace + (size_t)l * batch * words : at<uint32_t>(ws, lay.mask);
+    P.before(PI_KIND_RMSNORM);
+    cudaError_t e = launch_rmsnorm(x, batch, d, xh, s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
+    P.before(PI_KIND_PRED_U);
+    e = launch_pred_u(L, xh, batch, at<float>(ws, lay.u), s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
+    P.before(PI_KIND_PRED_Z);
+    e = launch_pred_z(L, at<float>(ws, lay.u), batch, theta, mask, s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "pred_z launch");
+    P.before(PI_KIND_COMPACT);
+    e = launch_compact(mask, batch, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "compact launch");
+    if ((st = ffn_body(L, xh, batch, per_token ? mask : nullptr, per_token, idx, cnt, x, x, ws,
+                       lay, s, prof)) != PI_OK)
+      return st;
+  }
+  return PI_OK;
+}
+
+}  // namespace
+}  // namespace pi
+
+using namespace pi;
+
+extern "C" {
+
+int pi_version(void) { return PI_VERSION; }
+
+const char* pi_last_error(void) { return g_err; }
+
+const char* pi_status_string(int status) {
+  switch (status) {
+    case PI_OK: return "PI_OK";
+    case PI_ERR_INVALID: return "PI_ERR_INVALID";
+    case PI_ERR_UNSUPPORTED: return "PI_ERR_UNSUPPORTED";
+    case PI_ERR_CUDA: return "PI_ERR_CUDA";
+    case PI_ERR_TIMEOUT: return "PI_ERR_TIMEOUT";
+    case PI_ERR_DEVICE_CHECK: return "PI_ERR_DEVICE_CHECK";
+    default: return "PI_ERR_UNKNOWN";
+  }
+}
+
+size_t pi_workspace_bytes(const pi_layer* layers, int n_layers, int batch) {
+  if (!layers || n_layers < 1 || batch < 1 || batch > PI_MAX_BATCH) return 0;
+  for (int l = 0; l < n_layers; ++l)
+    if (check_layer(&layers[l], l) != PI_OK) return 0;
+  return layout_for_layers(layers, n_layers, batch).total;
+}
+
+pi_status pi_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < sizeof(WsHeader))
+    return fail(PI_ERR_INVALID, "workspace must be 256-byte aligned and >= 256 bytes");
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream);
+  return e == cudaSuccess ? PI_OK : cuda_fail(e, "workspace init");
+}
+
+pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float tau,
+                     uint32_t* mask, void* ws, size_t ws_bytes, void* stream) {
+  pi_status st = check_layer(layer, 0);
+  if (st != PI_OK) return st;
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID, "batch %d not in [1, 64]", batch);
+  if (!(tau > 0.f && tau < 1.f)) return fail(PI_ERR_INVALID, "tau must lie in (0, 1)");
+  if (!xh || !aligned(xh, 16)) return fail(PI_ERR_INVALID, "xh null or not 16-byte aligned");
+  if (!mask || !aligned(mask, 4)) return fail(PI_ERR_INVALID, "mask null or misaligned");
+  const WsLayout lay = layout_for_layers(layer, 1, batch);
+  if ((st = check_ws(ws, ws_bytes, lay)) != PI_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_pred_u(*layer, xh, batch, at<float>(ws, lay.u), s);
+  if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
+  e = launch_pred_z(*layer, at<float>(ws, lay.u), batch, logit32(tau), mask, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pred_z launch");
+  return PI_OK;
+}
+
+pi_status pi_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,
+                     int32_t* idx, int32_t* count, void* stream) {
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID, "batch %d not in [1, 64]", batch);
+  if (d_ff < 1 || d_ff > PI_MAX_D_FF) return fail(PI_ERR_INVALID, "d_ff %d out of range", d_ff);
+  if (begin < 0 || begin > d_ff) return fail(PI_ERR_INVALID, "begin %d not in [0, d_ff]", begin);
+  if (mode != PI_MASK_PER_TOKEN && mode != PI_MASK_UNION) return fail(PI_ERR_INVALID, "unknown mask mode %d", mode);
+  if (!mask || !idx || !count || !aligned(mask, 4) || !aligned(idx, 4) || !aligned(count, 4))
+    return fail(PI_ERR_INVALID, "null or misaligned mask/idx/count");
+  cudaError_t e = launch_compact(mask, batch, d_ff, begin, mode, idx, count, (cudaStream_t)stream);
+  return e == cudaSuccess ? PI_OK : cuda_fail(e, "compact launch");
+}
+
+pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch, const uint32_t* mask,
+                        const int32_t* idx, const int32_t* count, int mode, float* y, void* ws,
+                        size_t ws_bytes, void* stream) {
+  pi_status st = check_layer(layer, 0);
+  if (st != PI_OK) return st;
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID, "batch %d not in [1, 64]", batch);
+  if (mode != PI_MASK_PER_TOKEN && mode != PI_MASK_UNION) return fail(PI_ERR_INVALID, "unknown mask mode %d", mode);
+  if (!xh || !aligned(xh, 16)) return fail(PI_ERR_INVALID, "xh null or not 16-byte aligned");
+  if (!y || !aligned(y, 16)) return fail(PI_ERR_INVALID, "y null or not 16-byte aligned");
+  if (!idx || !count || !aligned(idx, 4) || !aligned(count, 4))
+    return fail(PI_ERR_INVALID, "null or misaligned idx/count");
+  const int per_token = (mode == PI_MASK_PER_TOKEN && batch > 1);
+  if (per_token && (!mask || !aligned(mask, 4)))
+    return fail(PI_ERR_INVALID, "per-token mode with batch > 1 needs the mask");
+  const WsLayout lay = layout_for_layers(layer, 1, batch);
+  if ((st = check_ws(ws, ws_bytes, lay)) != PI_OK) return st;
+  return ffn_body(*layer, xh, batch, per_token ? mask : nullptr, per_token, idx, count, nullptr, y,
+                  ws, lay, (cudaStream_t)stream);
+}
+
+pi_status pi_ffn_stack(const pi_layer* layers, int n_layers, float* x, int batch, float tau,
+                       int mode, uint32_t* mask_trace, void* ws, size_t ws_bytes, void* stream) {
+  WsLayout lay;
+  pi_status st = stack_check(layers, n_layers, x, batch, tau, mode, mask_trace, ws, ws_bytes, &lay);
+  if (st != PI_OK) return st;
+  return stack_run(layers, n_layers, x, batch, tau, mode, mask_trace, ws, lay,
+                   (cudaStream_t)stream, nullptr);
+}
+
+const char* pi_kind_name(int kind) {
+  static const char* names[PI_KINDS] = {"rmsnorm", "pred_u", "pred_z", "compact",
+                                        "ffn_up",  "ffn_down", "reduce"};
+  return (kind >= 0 && kind < PI_KINDS) ? names[kind] : "unknown";
+}
+
+pi_status pi_ffn_stack_profile(const pi_layer* layers, int n_layers, float* x, int batch,
+                               float tau, int mode, uint32_t* mask_trace, void* ws,
+                               size_t ws_bytes, void* stream, float* kind_ms,
+                               int* kind_launches) {
+  WsLayout lay;
+  pi_status st = stack_check(layers, n_layers, x, batch, tau, mode, mask_trace, ws, ws_bytes, &lay);
+  if (st != PI_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  Prof P;
+  P.cap = n_layers * 8;
+  P.s = s;
+  P.ev = new cudaEvent_t[2 * P.cap];
+  P.kind = new int[P.cap];
+  int made = 0;
+  cudaError_t e = cudaSuccess;
+  for (; made < 2 * P.cap && e == cudaSuccess; ++made) e = cudaEventCreate(&P.ev[made]);
+  if (e == cudaSuccess) e = launch_delay(2000000ull, s);
+  if (e != cudaSuccess) st = cuda_fail(e, "profile setup");
+  if (st == PI_OK) st = stack_run(layers, n_layers, x, batch, tau, mode, mask_trace, ws, lay, s, &P);
+  if (st == PI_OK && (e = cudaStreamSynchronize(s)) != cudaSuccess) st = cuda_fail(e, "profile sync");
+  if (st == PI_OK) {
+    float ms[PI_KINDS] = {0};
+    int cnt[PI_KINDS] = {0};
+    for (int i = 0; i < P.n; ++i) {
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, P.ev[2 * i], P.ev[2 * i + 1]) == cudaSuccess) {
+        ms[P.kind[i]] += t;
+        cnt[P.kind[i]] += 1;
+      }
+    }
+    for (int k = 0; k < PI_KINDS; ++k) {
+      if (kind_ms) kind_ms[k] = ms[k];
+      if (kind_launches) kind_launches[k] = cnt[k];
+    }
+  }
+  for (int i = 0; i < made; ++i) cudaEventDestroy(P.ev[i]);
+  delete[] P.ev;
+  delete[] P.kind;
+  return st;
+}
+
+pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {
+  if (!ws || !aligned(ws, 256) || !out) return fail(PI_ERR_INVALID, "workspace or output null");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned long long v[2];
+  e = cudaMemcpy(v, &header(ws)->rows_listed, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "counter read");
+  if (clear && (e = cudaMemset(&header(ws)->rows_listed, 0, sizeof v)) != cudaSuccess)
+    return cuda_fail(e, "counter clear");
+  out[0] = v[0];
+  out[1] = v[1];
+  return PI_OK;
+}
+
+pi_status pi_get_device_status(void* ws, void* stream, int clear, uint32_t* detail) {
+  if (!ws || !aligned(ws, 256)) return fail(PI_ERR_INVALID, "workspace null or misaligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, status_word(ws), sizeof word, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  if (clear) {
+    e = cudaMemset(status_word(ws), 0, sizeof word);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  }
+  if (detail) *detail = word;
+  if (word & DEV_TIMEOUT) return fail(PI_ERR_TIMEOUT, "a bounded device wait gave up (status 0x%x)", word);
+  if (word) return fail(PI_ERR_DEVICE_CHECK, "device-side range check failed (status 0x%x)", word);
+  return PI_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,662 @@
+// libpi kernels, sm_100a.
+//
+// The hot path of one FFN layer (see pi.h for the operation definitions):
+//   rmsnorm -> predictor u = p1 xh -> predictor logits + threshold -> mask
+//   -> compaction -> gathered up/gate rows + activation -> gathered split-K
+//   down projection -> fixed-order reduction (+ residual).
+//
+// All weight traffic is 16-byte streaming loads of whole neuron rows (a row
+// per warp for the dot products, a row per CTA for the down projection),
+// with the reused vectors (xh, u) staged in shared memory.  Accumulation is
+// fp32 throughout.
+#include <algorithm>
+#include <mutex>
+#include <unordered_map>
+
+#include "pi_kernels.cuh"
+
+namespace pi {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
+  if (status) atomicOr(status, bit);
+}
+
+// Stage xh[t0 .. t0+TB) (fp32 [B][d]) into shared memory, zero past B.
+template <int TB>
+__device__ __forceinline__ void stage_x(float* sx, const float* xh, int B, int d, int t0) {
+  const int n4 = d / 4;
+  for (int e = threadIdx.x; e < TB * n4; e += blockDim.x) {
+    const int b = e / n4, i = e % n4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t0 + b < B) v = reinterpret_cast<const float4*>(xh + (size_t)(t0 + b) * d)[i];
+    reinterpret_cast<float4*>(sx + (size_t)b * d)[i] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dot products of NR weight rows against TB staged vectors, one 16-byte chunk
+// (chunk c covers columns [c*CC, (c+1)*CC)) at a time.
+template <int WT, int NR, int TB>
+struct RowDot {
+  __device__ __forceinline__ static void chunk(const char* const* rows,
+                                               const uint16_t* const* scales, int c,
+                                               const float* sx, int d,
+                                               float (&acc)[NR][TB]) {
+    if constexpr (WT == PI_F32) {
+      uint4 v[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) v[r] = ld_stream16(rows[r] + (size_t)c * 16);
+#pragma unroll
+      for (int b = 0; b < TB; ++b) {
+        const float4 x = *reinterpret_cast<const float4*>(sx + (size_t)b * d + c * 4);
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          float a = acc[r][b];
+          a = fmaf(__uint_as_float(v[r].x), x.x, a);
+          a = fmaf(__uint_as_float(v[r].y), x.y, a);
+          a = fmaf(__uint_as_float(v[r].z), x.z, a);
+          a = fmaf(__uint_as_float(v[r].w), x.w, a);
+          acc[r][b] = a;
+        }
+      }
+    } else if constexpr (WT == PI_F16) {
+      float w[NR][8];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) f16x8_to_f32(ld_stream16(rows[r] + (size_t)c * 16), w[r]);
+#pragma unroll
+      for (int b = 0; b < TB; ++b) {
+        const float4 x0 = *reinterpret_cast<const float4*>(sx + (size_t)b * d + c * 8);
+        const float4 x1 = *reinterpret_cast<const float4*>(sx + (size_t)b * d + c * 8 + 4);
+        const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          float a = acc[r][b];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) a = fmaf(w[r][e], xv[e], a);
+          acc[r][b] = a;
+        }
+      }
+    } else {  // Q4_0: chunk c = block c of the row
+      uint4 v[NR];
+      float s[NR];
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        v[r] = ld_stream16(rows[r] + (size_t)c * 16);
+        s[r] = h2f(ld_stream_u16(scales[r] + c));
+      }
+#pragma unroll
+      for (int b = 0; b < TB; ++b) {
+        const float* xp = sx + (size_t)b * d + c * 32;
+        float xv[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 t = reinterpret_cast<const float4*>(xp)[q];
+          xv[4 * q] = t.x; xv[4 * q + 1] = t.y; xv[4 * q + 2] = t.z; xv[4 * q + 3] = t.w;
+        }
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const uint32_t wd[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+          float a = 0.f;
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint32_t byte = (wd[k >> 2] >> (8 * (k & 3))) & 0xFFu;
+            a = fmaf(q4_centered(byte & 0xFu), xv[k], a);
+            a = fmaf(q4_centered(byte >> 4), xv[k + 16], a);
+          }
+          acc[r][b] = fmaf(a, s[r], acc[r][b]);
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+template <int TB>
+__global__ void __launch_bounds__(1024) k_rmsnorm(const float* __restrict__ x, int d,
+                                                  float* __restrict__ xh) {
+  const float* xr = x + (size_t)blockIdx.x * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+  ss = warp_sum(ss);
+  __shared__ float red[32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float inv = 1.0f / sqrtf(red[0] / (float)d + 1e-6f);
+  for (int i = threadIdx.x; i < d; i += blockDim.x) xh[(size_t)blockIdx.x * d + i] = xr[i] * inv;
+}
+
+// u[b][k] = p1[k] . xh[b]; one warp per predictor row.
+template <int PT, int TB>
+__global__ void __launch_bounds__(kThreads) k_pred_u(const char* __restrict__ p1,
+                                                     const float* __restrict__ xh, int B,
+                                                     int d, int r, float* __restrict__ u) {
+  extern __shared__ __align__(16) float sx[];
+  const int t0 = blockIdx.y * TB;
+  stage_x<TB>(sx, xh, B, d, t0);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int CC = WTraits<PT>::CHUNK_COLS;
+  const int nch = d / CC;
+  const int64_t rb = row_bytes(PT, d);
+  for (int k = blockIdx.x * kWarps + warp; k < r; k += gridDim.x * kWarps) {
+    float acc[1][TB];
+#pragma unroll
+    for (int b = 0; b < TB; ++b) acc[0][b] = 0.f;
+    const char* rows[1] = {p1 + (size_t)k * rb};
+    const uint16_t* sc[1] = {nullptr};
+#pragma unroll 4
+    for (int c = lane; c < nch; c += 32) RowDot<PT, 1, TB>::chunk(rows, sc, c, sx, d, acc);
+#pragma unroll
+    for (int b = 0; b < TB; ++b) {
+      const float v = warp_sum(acc[0][b]);
+      if (lane == 0 && t0 + b < B) u[(size_t)(t0 + b) * r + k] = v;
+    }
+  }
+}
+
+// Predictor logits and threshold: one warp per mask word (32 neurons).
+template <int PT, int TB>
+__global__ void __launch_bounds__(kThreads) k_pred_z(const char* __restrict__ p2,
+                                                     const float* __restrict__ pbias,
+                                                     const float* __restrict__ u, int B, int r,
+                                                     int F, int H, float theta,
+                                                     uint32_t* __restrict__ mask, int words) {
+  extern __shared__ __align__(16) float su[];
+  const int t0 = blockIdx.y * TB;
+  stage_x<TB>(su, u, B, r, t0);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int CC = WTraits<PT>::CHUNK_COLS;
+  const int nch = r / CC;
+  const int64_t rb = row_bytes(PT, r);
+  for (int w = blockIdx.x * kWarps + warp; w < words; w += gridDim.x * kWarps) {
+    const int j0 = w * 32;
+    float zl[TB];
+#pragma unroll
+    for (int b = 0; b < TB; ++b) zl[b] = 0.f;
+    if (j0 + 32 > H) {
+      for (int jj = 0; jj < 32; jj += 2) {
+        // two neurons per pass for more loads in flight
+        const int ja = j0 + jj, jb = j0 + jj + 1;
+        const bool va = ja >= H && ja < F, vb = jb >= H && jb < F;
+        if (!va && !vb) continue;
+        float acc[2][TB];
+#pragma unroll
+        for (int b = 0; b < TB; ++b) acc[0][b] = acc[1][b] = 0.f;
+        const char* rows[2] = {p2 + (size_t)(va ? ja : jb) * rb, p2 + (size_t)(vb ? jb : ja) * rb};
+        const uint16_t* sc[2] = {nullptr, nullptr};
+#pragma unroll 2
+        for (int c = lane; c < nch; c += 32) RowDot<PT, 2, TB>::chunk(rows, sc, c, su, r, acc);
+#pragma unroll
+        for (int b = 0; b < TB; ++b) {
+          const float za = warp_sum(acc[0][b]);
+          const float zb = warp_sum(acc[1][b]);
+          if (lane == jj && va) zl[b] = za + (pbias ? pbias[ja] : 0.f);
+          if (lane == jj + 1 && vb) zl[b] = zb + (pbias ? pbias[jb] : 0.f);
+        }
+      }
+    }
+    const int j = j0 + lane;
+#pragma unroll
+    for (int b = 0; b < TB; ++b) {
+      const bool on = j < F && (j < H || zl[b] > theta);
+      const uint32_t bits = __ballot_sync(0xffffffffu, on);
+      if (lane == 0 && t0 + b < B) mask[(size_t)(t0 + b) * words + w] = bits;
+    }
+  }
+}
+
+// Compaction: one CTA per list; block-wide exclusive scan of per-word
+// popcounts, each thread then writes its word's set bits in order.
+__global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ mask, int B,
+                                                  int words, int F, int begin, int unite,
+                                                  int32_t* __restrict__ idx, int idx_stride,
+                                                  int32_t* __restrict__ count) {
+  __shared__ int wsum[32];
+  __shared__ int s_base;
+  const int list = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  if (tid == 0) s_base = 0;
+  __syncthreads();
+  int32_t* out = idx + (size_t)list * idx_stride;
+  for (int w0 = 0; w0 < words; w0 += blockDim.x) {
+    const int w = w0 + tid;
+    uint32_t m = 0;
+    if (w < words) {
+      if (unite) {
+        for (int b = 0; b < B; ++b) m |= mask[(size_t)b * words + w];
+      } else {
+        m = mask[(size_t)list * words + w];
+      }
+      const int lo = w * 32;
+      if (begin > lo) m = (begin - lo >= 32) ? 0u : (m & (~0u << (begin - lo)));
+      if (F < lo + 32) m = (F <= lo) ? 0u : (m & ((1u << (F - lo)) - 1u));
+    }
+    const int c = __popc(m);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      int v = lane < nw ? wsum[lane] : 0;
+      int vi = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, vi, o);
+        if (lane >= o) vi += t;
+      }
+      if (lane < nw) wsum[lane] = vi - v;  // exclusive warp offsets
+      if (lane == 31) wsum[31] = vi;       // (nw <= 31 here) total of this tile
+    }
+    __syncthreads();
+    int pos = s_base + wsum[warp] + incl - c;
+    const int lo = w * 32;
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      out[pos++] = lo + bit;
+      m &= m - 1u;
+    }
+    const int tile_total = wsum[31];
+    __syncthreads();
+    if (tid == 0) s_base += tile_total;
+    __syncthreads();
+  }
+  if (tid == 0) count[list] = s_base;
+}
+
+// Gathered up/gate rows + activation: one warp per listed row.
+template <int WT, int ACT, int TB>
+__global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __restrict__ xh,
+                                                     int B, const uint32_t* __restrict__ mask,
+                                                     int per_token, int words,
+                                                     const int32_t* __restrict__ idx,
+                                                     const int32_t* __restrict__ count,
+                                                     float* __restrict__ h, WsHeader* hdr) {
+  extern __shared__ __align__(16) float sx[];
+  uint32_t* status = hdr ? &hdr->status : nullptr;
+  const int d = L.d_model, F = L.d_ff, H = L.hot;
+  const int t0 = blockIdx.y * TB;
+  stage_x<TB>(sx, xh, B, d, t0);
+  __syncthreads();
+  int cnt = *count;
+  if (cnt < 0 || cnt > F - H) {
+    if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) flag(status, DEV_BAD_COUNT);
+    cnt = cnt < 0 ? 0 : F - H;
+  }
+  const int N = H + cnt;
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&hdr->rows_listed, (unsigned long long)N);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int NR = (ACT == PI_REGLU) ? 2 : 1;
+  constexpr int CC = WTraits<WT>::CHUNK_COLS;
+  const int nch = d / CC;
+  const int64_t rb = row_bytes(WT, d);
+  const int nb = d / 32;
+  for (int n = blockIdx.x * kWarps + warp; n < N; n += gridDim.x * kWarps) {
+    const int j = n < H ? n : idx[n - H];
+    if (j < H && n >= H || j >= F || j < 0) {
+      if (lane == 0) {
+        flag(status, DEV_BAD_INDEX);
+        for (int b = 0; b < TB; ++b)
+          if (t0 + b < B) h[(size_t)n * B + t0 + b] = 0.f;
+      }
+      continue;
+    }
+    const char* rows[NR];
+    const uint16_t* sc[NR];
+    if constexpr (ACT == PI_REGLU) {
+      rows[0] = (const char*)L.w_gate + (size_t)j * rb;
+      rows[1] = (const char*)L.w_up + (size_t)j * rb;
+      sc[0] = (const uint16_t*)L.w_gate_scales + (size_t)j * nb;
+      sc[1] = (const uint16_t*)L.w_up_scales + (size_t)j * nb;
+    } else {
+      rows[0] = (const char*)L.w_up + (size_t)j * rb;
+      sc[0] = (const uint16_t*)L.w_up_scales + (size_t)j * nb;
+    }
+    float acc[NR][TB];
+#pragma unroll
+    for (int r = 0; r < NR; ++r)
+#pragma unroll
+      for (int b = 0; b < TB; ++b) acc[r][b] = 0.f;
+#pragma unroll 2
+    for (int c = lane; c < nch; c += 32) RowDot<WT, NR, TB>::chunk(rows, sc, c, sx, d, acc);
+    const float bj = L.bias ? L.bias[j] : 0.f;
+#pragma unroll
+    for (int b = 0; b < TB; ++b) {
+      float g = warp_sum(acc[0][b]) + bj;
+      float hv = g > 0.f ? g : 0.f;
+      if constexpr (ACT == PI_REGLU) hv *= warp_sum(acc[NR - 1][b]);
+      if (per_token && n >= H && mask && t0 + b < B) {
+        const uint32_t bit = (mask[(size_t)(t0 + b) * words + (j >> 5)] >> (j & 31)) & 1u;
+        if (!bit) hv = 0.f;
+      }
+      if (lane == 0 && t0 + b < B) h[(size_t)n * B + t0 + b] = hv;
+    }
+  }
+}
+
+// Split-K gathered down projection.  Grid (column tiles, S, token chunks):
+// CTA (x, s, z) accumulates rows [s*N/S, (s+1)*N/S) of the list for 8
+// columns per thread and TB tokens, skipping rows whose h is 0 for all of
+// its tokens, and writes its partial sums.
+template <int WT, int TB>
+__global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ wd,
+                                                       const uint16_t* __restrict__ wsc, int d,
+                                                       int F, int H,
+                                                       const int32_t* __restrict__ idx,
+                                                       const int32_t* __restrict__ count,
+                                                       const float* __restrict__ h, int B,
+                                                       int S, float* __restrict__ part,
+                                                       WsHeader* hdr) {
+  const int s = blockIdx.y, t0 = blockIdx.z * TB;
+  const int col0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  int cnt = *count;
+  cnt = cnt < 0 ? 0 : (cnt > F - H ? F - H : cnt);
+  const int N = H + cnt;
+  const int n0 = (int)((int64_t)s * N / S), n1 = (int)((int64_t)(s + 1) * N / S);
+  float acc[TB][8];
+#pragma unroll
+  for (int b = 0; b < TB; ++b)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
+  const int64_t rb = row_bytes(WT, d);
+  const int nb = d / 32;
+  unsigned long long nread = 0;
+  if (col0 < d) {
+#pragma unroll 4
+    for (int n = n0; n < n1; ++n) {
+      float hv[TB];
+      bool any = false;
+#pragma unroll
+      for (int b = 0; b < TB; ++b) {
+        hv[b] = (t0 + b < B) ? h[(size_t)n * B + t0 + b] : 0.f;
+        any |= hv[b] != 0.f;
+      }
+      if (!any) continue;
+      const int j = n < H ? n : idx[n - H];
+      if (j < 0 || j >= F) continue;
+      ++nread;
+      float w[8];
+      const char* row = wd + (size_t)j * rb;
+      if constexpr (WT == PI_F32) {
+        const uint4 a = ld_stream16(row + (size_t)col0 * 4);
+        const uint4 c = ld_stream16(row + (size_t)col0 * 4 + 16);
+        w[0] = __uint_as_float(a.x); w[1] = __uint_as_float(a.y);
+        w[2] = __uint_as_float(a.z); w[3] = __uint_as_float(a.w);
+        w[4] = __uint_as_float(c.x); w[5] = __uint_as_float(c.y);
+        w[6] = __uint_as_float(c.z); w[7] = __uint_as_float(c.w);
+      } else if constexpr (WT == PI_F16) {
+        f16x8_to_f32(ld_stream16(row + (size_t)col0 * 2), w);
+      } else {
+        const int blk = col0 >> 5, k0 = col0 & 31;
+        const uint2 q = *reinterpret_cast<const uint2*>(row + (size_t)blk * 16 + (k0 & 15));
+        const float sc = h2f(wsc[(size_t)j * nb + blk]);
+        const int sh = k0 >= 16 ? 4 : 0;
+        const uint32_t qq[2] = {q.x, q.y};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          w[e] = q4_centered((qq[e >> 2] >> (8 * (e & 3) + sh)) & 0xFu) * sc;
+      }
+#pragma unroll
+      for (int b = 0; b < TB; ++b)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(hv[b], w[e], acc[b][e]);
+    }
+#pragma unroll
+    for (int b = 0; b < TB; ++b) {
+      if (t0 + b >= B) continue;
+      float* o = part + ((size_t)s * B + t0 + b) * d + col0;
+      reinterpret_cast<float4*>(o)[0] = make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
+      reinterpret_cast<float4*>(o)[1] = make_float4(acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
+    }
+  }
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0 && nread) atomicAdd(&hdr->rows_down, nread);
+}
+
+__global__ void __launch_bounds__(kThreads) k_reduce(const float* __restrict__ part, int S,
+                                                     int64_t n, const float* resid,
+                                                     float* out) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part[(size_t)s * n + e];
+    out[e] = (resid ? resid[e] : 0.f) + acc;
+  }
+}
+
+__global__ void k_delay(unsigned long long ns) {
+  unsigned long long t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  do {
+    __nanosleep(1000);
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  } while (t - t0 < ns && t >= t0);
+}
+
+// Shared-memory opt-in: raises a kernel's dynamic shared-memory limit on the
+// current device the first time a launch needs more than 48 KB (keyed by the
+// kernel's address), so a warm-up call leaves nothing but launches for a
+// later graph capture.
+cudaError_t allow_smem_fn(const void* fn, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  static std::unordered_map<uint64_t, size_t> granted;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const uint64_t key = (uint64_t)(uintptr_t)fn * 131u + (uint64_t)dev;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = granted.find(key);
+  if (it != granted.end() && it->second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) granted[key] = bytes;
+  return e;
+}
+
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+  return allow_smem_fn(reinterpret_cast<const void*>(kernel), bytes);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ policy
+
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+int pick_tb(int batch, int d) {
+  int tb = batch <= 1 ? 1 : (batch <= 2 ? 2 : (batch <= 4 ? 4 : 8));
+  while (tb > 1 && (size_t)tb * d * 4 > 200 * 1024) tb >>= 1;
+  return tb;
+}
+
+int down_tb(int batch) { return batch <= 1 ? 1 : (batch <= 2 ? 2 : (batch <= 4 ? 4 : 8)); }
+
+int down_splits(int batch, int d) {
+  const int sms = device_sms();
+  const int tiles = (d + 8 * kThreads - 1) / (8 * kThreads);
+  const int chunks = (batch + down_tb(batch) - 1) / down_tb(batch);
+  int s = (2 * sms + tiles * chunks - 1) / (tiles * chunks);
+  return std::max(1, std::min(s, sms));
+}
+
+// ---------------------------------------------------------------- launches
+
+cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s) {
+  k_rmsnorm<1><<<batch, 1024, 0, s>>>(x, d, xh);
+  return cudaGetLastError();
+}
+
+template <int PT, int TB>
+static cudaError_t pred_u_t(const pi_layer& L, const float* xh, int batch, float* u,
+                            cudaStream_t s) {
+  const size_t smem = (size_t)TB * L.d_model * 4;
+  auto kern = k_pred_u<PT, TB>;
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(std::min((L.rank + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
+  kern<<<grid, kThreads, smem, s>>>((const char*)L.p1, xh, batch, L.d_model, L.rank, u);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pred_u(const pi_layer& L, const float* xh, int batch, float* u,
+                          cudaStream_t s) {
+  const int tb = pick_tb(batch, L.d_model);
+#define PI_PU(PT)                                                         \
+  switch (tb) {                                                           \
+    case 1: return pred_u_t<PT, 1>(L, xh, batch, u, s);                   \
+    case 2: return pred_u_t<PT, 2>(L, xh, batch, u, s);                   \
+    case 4: return pred_u_t<PT, 4>(L, xh, batch, u, s);                   \
+    default: return pred_u_t<PT, 8>(L, xh, batch, u, s);                  \
+  }
+  if (L.p_dtype == PI_F32) { PI_PU(PI_F32) } else { PI_PU(PI_F16) }
+#undef PI_PU
+}
+
+template <int PT, int TB>
+static cudaError_t pred_z_t(const pi_layer& L, const float* u, int batch, float theta,
+                            uint32_t* mask, cudaStream_t s) {
+  const size_t smem = (size_t)TB * L.rank * 4;
+  auto kern = k_pred_z<PT, TB>;
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const int words = (L.d_ff + 31) / 32;
+  dim3 grid(std::min((words + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
+  kern<<<grid, kThreads, smem, s>>>((const char*)L.p2, L.p_bias, u, batch, L.rank, L.d_ff,
+                                    L.hot, theta, mask, words);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pred_z(const pi_layer& L, const float* u, int batch, float theta,
+                          uint32_t* mask, cudaStream_t s) {
+  const int tb = pick_tb(batch, L.rank);
+#define PI_PZ(PT)                                                         \
+  switch (tb) {                                                           \
+    case 1: return pred_z_t<PT, 1>(L, u, batch, theta, mask, s);          \
+    case 2: return pred_z_t<PT, 2>(L, u, batch, theta, mask, s);          \
+    case 4: return pred_z_t<PT, 4>(L, u, batch, theta, mask, s);          \
+    default: return pred_z_t<PT, 8>(L, u, batch, theta, mask, s);         \
+  }
+  if (L.p_dtype == PI_F32) { PI_PZ(PI_F32) } else { PI_PZ(PI_F16) }
+#undef PI_PZ
+}
+
+cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,
+                           int32_t* idx, int32_t* count, cudaStream_t s) {
+  const int words = (d_ff + 31) / 32;
+  const int unite = (mode == PI_MASK_UNION);
+  const int lists = unite ? 1 : batch;
+  const int threads = std::min(992, std::max(32, ((words + 31) / 32) * 32));
+  k_compact<<<lists, threads, 0, s>>>(mask, batch, words, d_ff, begin, unite, idx, d_ff, count);
+  return cudaGetLastError();
+}
+
+template <int WT, int ACT, int TB>
+static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                            int per_token, const int32_t* idx, const int32_t* count, float* h,
+                            WsHeader* status, cudaStream_t s) {
+  const size_t smem = (size_t)TB * L.d_model * 4;
+  auto kern = k_ffn_up<WT, ACT, TB>;
+  cudaError_t e = allow_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(std::min((L.d_ff + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
+  kern<<<grid, kThreads, smem, s>>>(L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
+                                    count, h, status);
+  return cudaGetLastError();
+}
+
+template <int WT, int ACT>
+static cudaError_t ffn_up_a(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                            int per_token, const int32_t* idx, const int32_t* count, float* h,
+                            WsHeader* status, cudaStream_t s) {
+  switch (pick_tb(batch, L.d_model)) {
+    case 1: return ffn_up_t<WT, ACT, 1>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+    case 2: return ffn_up_t<WT, ACT, 2>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+    case 4: return ffn_up_t<WT, ACT, 4>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+    default: return ffn_up_t<WT, ACT, 8>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+  }
+}
+
+cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                          int per_token, const int32_t* idx, const int32_t* count, float* h,
+                          WsHeader* status, cudaStream_t s) {
+#define PI_UP(WT)                                                                              \
+  return L.act == PI_REGLU                                                                     \
+             ? ffn_up_a<WT, PI_REGLU>(L, xh, batch, mask, per_token, idx, count, h, status, s) \
+             : ffn_up_a<WT, PI_RELU>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+  if (L.w_dtype == PI_F32) { PI_UP(PI_F32) }
+  if (L.w_dtype == PI_F16) { PI_UP(PI_F16) }
+  PI_UP(PI_Q4_0)
+#undef PI_UP
+}
+
+template <int WT, int TB>
+static cudaError_t ffn_down_t(const pi_layer& L, int batch, const int32_t* idx,
+                              const int32_t* count, const float* h, float* part, int S,
+                              WsHeader* hdr, cudaStream_t s) {
+  const int tiles = (L.d_model + 8 * kThreads - 1) / (8 * kThreads);
+  dim3 grid(tiles, S, (batch + TB - 1) / TB);
+  k_ffn_down<WT, TB><<<grid, kThreads, 0, s>>>((const char*)L.w_down_t,
+                                              (const uint16_t*)L.w_down_t_scales, L.d_model,
+                                              L.d_ff, L.hot, idx, count, h, batch, S, part, hdr);
+  return cudaGetLastError();
+}
+
+template <int WT>
+static cudaError_t ffn_down_w(const pi_layer& L, int batch, const int32_t* idx,
+                              const int32_t* count, const float* h, float* part, int S,
+                              WsHeader* hdr, cudaStream_t s) {
+  switch (down_tb(batch)) {
+    case 1: return ffn_down_t<WT, 1>(L, batch, idx, count, h, part, S, hdr, s);
+    case 2: return ffn_down_t<WT, 2>(L, batch, idx, count, h, part, S, hdr, s);
+    case 4: return ffn_down_t<WT, 4>(L, batch, idx, count, h, part, S, hdr, s);
+    default: return ffn_down_t<WT, 8>(L, batch, idx, count, h, part, S, hdr, s);
+  }
+}
+
+cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,
+                            const int32_t* count, const float* h, float* part, int splits,
+                            WsHeader* hdr, cudaStream_t s) {
+  if (L.w_dtype == PI_F32) return ffn_down_w<PI_F32>(L, batch, idx, count, h, part, splits, hdr, s);
+  if (L.w_dtype == PI_F16) return ffn_down_w<PI_F16>(L, batch, idx, count, h, part, splits, hdr, s);
+  return ffn_down_w<PI_Q4_0>(L, batch, idx, count, h, part, splits, hdr, s);
+}
+
+cudaError_t launch_delay(unsigned long long ns, cudaStream_t s) {
+  k_delay<<<1, 32, 0, s>>>(ns);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce(const float* part, int splits, int batch, int d, const float* resid,
+                          float* out, cudaStream_t s) {
+  const int64_t n = (int64_t)batch * d;
+  const int grid = (int)std::min<int64_t>((n + kThreads - 1) / kThreads, device_sms() * 8);
+  k_reduce<<<grid, kThreads, 0, s>>>(part, splits, n, resid, out);
+  return cudaGetLastError();
+}
+
+}  // namespace pi

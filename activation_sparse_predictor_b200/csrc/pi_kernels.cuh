@@ -1,0 +1,50 @@
+// Launchers of the libpi kernels (host side, internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pi.h"
+#include "pi_common.cuh"
+
+namespace pi {
+
+int device_sms();                 // SM count of the current device (cached)
+int pick_tb(int batch, int d);    // tokens per pass of the x-staged kernels
+int down_tb(int batch);           // tokens per pass of the down projection
+int down_splits(int batch, int d);// split-K slices of the down projection
+
+// xh[b] = x[b] / sqrt(mean(x[b]^2) + 1e-6), b < batch.
+cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s);
+
+// u[b][k] = p1[k] . xh[b]
+cudaError_t launch_pred_u(const pi_layer& L, const float* xh, int batch, float* u,
+                          cudaStream_t s);
+
+// mask[b] from z = p2 u + p_bias (rows >= hot), bits < hot set.
+cudaError_t launch_pred_z(const pi_layer& L, const float* u, int batch, float theta,
+                          uint32_t* mask, cudaStream_t s);
+
+// ascending set-bit lists (see pi_compact)
+cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,
+                           int32_t* idx, int32_t* count, cudaStream_t s);
+
+// h[n][b] for rows n of [0,hot) U idx[0..count)
+cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                          int per_token, const int32_t* idx, const int32_t* count, float* h,
+                          WsHeader* hdr, cudaStream_t s);
+
+// part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n]
+cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,
+                            const int32_t* count, const float* h, float* part, int splits,
+                            WsHeader* hdr, cudaStream_t s);
+
+// out[b][i] = (resid ? resid[b][i] : 0) + sum_s part[s][b][i], s ascending.
+cudaError_t launch_reduce(const float* part, int splits, int batch, int d, const float* resid,
+                          float* out, cudaStream_t s);
+
+// A kernel that waits about `ns` nanoseconds of device time and exits
+// (lets the host enqueue a timed sequence before the device reaches it).
+cudaError_t launch_delay(unsigned long long ns, cudaStream_t s);
+
+}  // namespace pi

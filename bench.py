@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Decode benchmark of the predictor-gated sparse FFN stack.
+
+One step = one decode token through the whole stack (every layer: rmsnorm,
+predictor, compaction, gathered up/gate + activation, gathered split-K down
+projection, residual) of the Llama2-70B-shaped ReGLU Q4_0 workload (80
+layers, d_model 8192, d_ff 28672, batch 1) on seeded synthetic weights
+generated in place on the GPU.  Prints one JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl pi|reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU; every rank
+decodes its own token stream through its own copy of the stack (the decode
+step has no data-path exchange), so scaling is weak and `value` sums the
+ranks' tokens over the slowest rank's time.
+
+--impl reference times the CPU oracle on the host cores instead: the same
+workload and metric, each step one token through a bounded sample of the
+layers, extrapolated to the whole stack.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-FFN decode tokens/s (Llama2-70B Q4_0 shape)"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "llama2_70b_reglu_8192x28672_q4_0"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="pi", choices=["pi", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--mode", default="per_token", choices=["per_token", "union"])
+    ap.add_argument("--cpu-sample-layers", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clock, power and clock-event reasons through NVML while
+    the timed region runs."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, torch_dev: int, interval=0.02):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.interval = interval
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(torch_dev)
+            try:
+                bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(torch_dev)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report it, keep running
+            self.err = repr(e)
+
+    def _sample(self):
+        nv = self.nv
+        mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.samples.append(mhz)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": getattr(self, "err", "no samples")}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if (args.impl == "pi" and torch.cuda.is_available()) else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------ accounting
+
+def weight_row_bytes(dtype: str, d: int) -> float:
+    return {"f32": 4.0 * d, "f16": 2.0 * d, "q4_0": d / 2 + (d // 32) * 2}[dtype]
+
+
+def predictor_bytes(w) -> float:
+    pb = {"f32": 4.0, "f16": 2.0}[w.p_dtype]
+    return (w.rank * w.d_model + (w.d_ff - w.hot) * w.rank) * pb + (w.d_ff - w.hot) * 4
+
+
+def layer_algorithmic_bytes(w, rows_listed: int, rows_down: int, n_layers: int) -> dict:
+    """Algorithmic bytes of each kernel kind summed over a run in which the
+    FFN launches processed `rows_listed` up/gate rows and read `rows_down`
+    w_down_t rows, over `n_layers` layer evaluations (batch 1)."""
+    rb = weight_row_bytes(w.w_dtype, w.d_model)
+    d4 = 4.0 * w.d_model
+    words = (w.d_ff + 31) // 32
+    return {
+        "rmsnorm": n_layers * 2 * d4,
+        "pred_u": n_layers * (w.rank * w.d_model * {"f32": 4, "f16": 2}[w.p_dtype] + d4 + 4 * w.rank),
+        "pred_z": n_layers * ((w.d_ff - w.hot) * w.rank * {"f32": 4, "f16": 2}[w.p_dtype]
+                              + (w.d_ff - w.hot) * 4 + 4 * w.rank + 4 * words),
+        "compact": n_layers * 4.0 * words,
+        "ffn_up": rows_listed * ((w.nm - 1) * rb + 4 + 4) + n_layers * (d4 + 4 * words),
+        "ffn_down": rows_down * rb,
+        "reduce": 0.0,  # partials live in L2; counted as traffic only by ncu
+    }
+
+
+# ---------------------------------------------------------------- CPU leg
+
+def cpu_oracle_tokens_per_s(w, n_sample_layers: int, reps: int, step0: int = 0):
+    """Times the CPU oracle (as it stands) on one token through
+    `n_sample_layers` layers `reps` times; returns (tokens/s extrapolated to
+    the whole stack, threads used, seconds per layer, description)."""
+    from activation_sparse_predictor_b200 import synth
+    from oracle import Oracle
+    orc = Oracle()
+    layers = [synth.layer_host(w, l) for l in range(n_sample_layers)]
+    x = synth.x_host(w, step0, 1)[0]
+    per_layer = []
+    for r in range(reps):
+        xr = x.copy()
+        for L in layers:
+            t0 = time.perf_counter()
+            xo, _, _ = orc.layer_forward(L, xr, w.tau)
+            per_layer.append(time.perf_counter() - t0)
+            xr = xo.astype("float32")
+    s = statistics.median(per_layer)
+    tps = 1.0 / (s * w.n_layers)
+    desc = (f"oracle (plain C, double accumulation, OpenMP) on one token through "
+            f"{n_sample_layers} of {w.n_layers} layers x {reps}; median seconds per layer "
+            f"{s:.3f} extrapolated to the {w.n_layers}-layer stack")
+    return tps, orc.num_threads(), s, desc
+
+
+def run_reference(args, world, rank):
+    """CPU oracle arm: rank 0 only, bounded sample per step."""
+    if rank != 0:
+        return
+    from activation_sparse_predictor_b200 import build, synth
+    build.build_synth()
+    w = synth.WORKLOADS[args.workload]
+    from oracle import Oracle
+    from oracle.build import build as build_oracle
+    build_oracle()
+    orc = Oracle()
+    layers = [synth.layer_host(w, l) for l in range(args.cpu_sample_layers)]
+    per_step = []
+    for step in range(args.warmup + args.steps):
+        x = synth.x_host(w, step, 1)[0]
+        t0 = time.perf_counter()
+        for L in layers:
+            xo, _, _ = orc.layer_forward(L, x, w.tau)
+            x = xo.astype("float32")
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            per_step.append(dt)
+    sec_per_layer = sum(per_step) / (len(per_step) * len(layers))
+    tps = 1.0 / (sec_per_layer * w.n_layers)
+    sample = (f"each step: one token through {len(layers)} of {w.n_layers} layers "
+              f"(host-generated, resident); tokens/s extrapolated to all {w.n_layers} layers")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tps, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * sec_per_layer * w.n_layers, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded generator; no weights or datasets)",
+        "config": workload_config(w, 1, "per_token"),
+        "cpu_baseline": {"value": tps, "unit": UNIT, "cores": orc.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": tps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(w, batch, mode):
+    return {"workload": w.name, "layers": w.n_layers, "d_model": w.d_model, "d_ff": w.d_ff,
+            "hot_prefix": w.hot, "predictor_rank": w.rank, "activation": w.act,
+            "weights": w.w_dtype, "predictor_weights": w.p_dtype, "batch": batch,
+            "mask_mode": mode, "tau": w.tau,
+            "l2": "inputs larger than L2: every step streams the whole stack's weights "
+                  "and predictors from HBM (no flush needed)"}
+
+
+# ---------------------------------------------------------------- GPU leg
+
+def run_pi(args, world, rank, local):
+    import torch
+
+    from activation_sparse_predictor_b200 import pi, synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = synth.WORKLOADS[args.workload]
+    B = args.batch
+    mode = pi.MODES[args.mode]
+    layers = []
+    for l in range(w.n_layers):
+        t = synth.layer_device(w, l, dev)
+        layers.append(pi.Layer.from_workload(
+            w, {k: t[k] for k in ("w_gate", "w_up", "w_down_t", "bias", "p1", "p2", "p_bias")
+                if k in t}))
+    arr = pi.layer_array(layers)
+    K, W = args.steps, max(3, args.warmup)
+    xs = torch.stack([synth.x_device(w, rank * 1_000_003 + s, B, dev) for s in range(K + W)])
+    stream = torch.cuda.Stream(dev)
+    ws = pi.workspace(layers, B, dev, stream)
+    x = torch.empty((B, w.d_model), dtype=torch.float32, device=dev)
+    torch.cuda.synchronize(dev)
+
+    with torch.cuda.stream(stream):
+        # eager warm-up: also settles shared-memory attributes before capture
+        for i in range(2):
+            x.copy_(xs[i])
+            pi.pi_ffn_stack(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            pi.pi_ffn_stack(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
+        for i in range(W):
+            x.copy_(xs[i])
+            g.replay()
+    stream.synchronize()
+    st, word = pi.pi_get_device_status(ws, stream=stream)
+    assert st == pi.PI_OK, f"device status {word:#x} after warm-up"
+    pi.pi_read_counters(ws, clear=True, stream=stream)
+
+    # ---- timed region: K graph replays, inputs already in HBM
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with sampler:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for i in range(K):
+                x.copy_(xs[W + i])
+                g.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    rows_listed, rows_down = pi.pi_read_counters(ws, clear=True, stream=stream)
+    ms_max = max_over_ranks(ms, world, dev)
+    value = world * K * B / (ms_max / 1000.0)
+
+    # bytes actually read per step (predictor + listed rows + nonzero down rows)
+    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * w.n_layers)
+    step_bytes = sum(by.values()) / K
+    peak, peak_kind = hbm_peak()
+    step_gbs = step_bytes / (ms / K / 1000.0) / 1e9
+
+    # ---- per-kernel device times: one profiled pass over the same step inputs
+    x.copy_(xs[W])
+    pi.pi_read_counters(ws, clear=True, stream=stream)
+    prof = pi.pi_ffn_stack_profile(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
+    pr_listed, pr_down = pi.pi_read_counters(ws, clear=True, stream=stream)
+    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, w.n_layers)
+    dom = max(prof, key=lambda k: prof[k][0])
+    dom_ms, dom_n = prof[dom]
+    achieved = pby[dom] / dom_n / (dom_ms / dom_n / 1000.0) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
+                "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
+                "traffic": None,
+                "algorithmic_bytes_per_launch": pby[dom] / dom_n,
+                "avg_launch_us": 1000.0 * dom_ms / dom_n,
+                "per_kind_ms_per_step": {k: v[0] for k, v in prof.items()},
+                "launches_per_step": {k: v[1] for k, v in prof.items()}}
+
+    # ---- end to end through the C ABI with host buffers: pinned H2D of the
+    # step's input, the stack, D2H of the step's output, every step
+    hx = torch.empty((K, B, w.d_model), dtype=torch.float32).pin_memory()
+    hx.copy_(xs[W:W + K].cpu())
+    hy = torch.empty((K, B, w.d_model), dtype=torch.float32).pin_memory()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(K):
+            x.copy_(hx[i], non_blocking=True)
+            g.replay()
+            hy[i].copy_(x, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e = {"value": world * K * B / (e2e_ms / 1000.0), "unit": UNIT,
+           "h2d_bytes_per_step": B * w.d_model * 4, "d2h_bytes_per_step": B * w.d_model * 4}
+    assert bool(torch.isfinite(hy).all())
+
+    st, word = pi.pi_get_device_status(ws, stream=stream)
+    assert st == pi.PI_OK, f"device status {word:#x}"
+    del g
+    if rank != 0:
+        return
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        tps, cores, s, desc = cpu_oracle_tokens_per_s(w, args.cpu_sample_layers, 2)
+        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded generator, weights generated on the GPU; no datasets)",
+        "config": dict(workload_config(w, B, args.mode),
+                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "hbm_gbs_actual": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
+        "bytes_per_step": step_bytes,
+        "rows_per_step": {"listed": rows_listed / K, "down_read": rows_down / K},
+        "clocks": sampler.summary(),
+        "e2e": e2e,
+        "gpu_launches": K * sum(v[1] for v in prof.values()),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_pi(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

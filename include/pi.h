@@ -1,0 +1,223 @@
+/*
+ * pi.h — C ABI of the predictor-gated, neuron-aware sparse FFN decode step
+ * (libpi.so, CUDA kernels for sm_100a).
+ *
+ * What the operations are, from the PowerInfer write-ups:
+ *  - Before a layer's FFN runs, a small per-layer predictor decides which
+ *    neurons the input activates, and only those neurons are computed
+ *    (QbitAI article, r-manual.ru, §"Что такое «разреженная активация»?").
+ *  - Neurons split into a small always-active ("hot") group and a large
+ *    input-dependent ("cold") group; each group's partial result is summed
+ *    into the layer output (same article, §"Гибридный дизайн вывода
+ *    CPU/GPU", the example in which an input activates neurons 3, 4 and 5;
+ *    aibars.net "SJTU-IPADS/PowerInfer", §"Mecanismo de Neurônios Quentes e
+ *    Frios").  Here the hot group is a frequency-sorted prefix [0, hot) of
+ *    the neuron order and both groups run on the same GPU.
+ *  - Activations ReLU and ReGLU (hada.io summary, §"Hạn chế và FAQ"),
+ *    weights optionally INT4 Q4_0 (same page, §"Lượng tử hóa và tương
+ *    thích").
+ *
+ * Conventions shared by every call
+ *  - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *    never allocates, frees or synchronises (except pi_get_device_status).
+ *    Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL = the
+ *    legacy default stream) and runs asynchronously.
+ *  - Matrices are row-major.  FFN weights are NEURON-MAJOR: row j of
+ *    w_gate, w_up and w_down_t is neuron j's d_model weights, so every
+ *    active neuron is one contiguous row per matrix.
+ *  - Q4_0 weights: a [d_ff][d_model/32][16]-byte array of 4-bit codes and a
+ *    [d_ff][d_model/32] array of binary16 scales.  Weight (j, c) is
+ *    (q - 8) * s with s the scale of block c/32 of row j and q the nibble for
+ *    element k = c % 32: the low nibble of byte k for k < 16, the high nibble
+ *    of byte k - 16 otherwise.
+ *  - Masks: bit j of a token's mask is bit (j % 32) of 32-bit word j / 32;
+ *    a token's mask has ceil(d_ff / 32) words; bits at or beyond d_ff are 0.
+ *  - Synchronous argument errors return PI_ERR_INVALID (null or misaligned
+ *    pointer, bad size, workspace too small) or PI_ERR_UNSUPPORTED (a dtype /
+ *    activation / size combination this build does not implement) before
+ *    anything is enqueued.  A failed launch returns PI_ERR_CUDA.  Problems
+ *    only the device can see (an index out of range, a bounded wait that ran
+ *    out) set sticky bits in the workspace's status word and skip the bad
+ *    access; read them with pi_get_device_status.
+ *  - pi_last_error() describes the last failure of the calling thread.
+ */
+#ifndef PI_H
+#define PI_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PI_VERSION 1
+#define PI_MAX_BATCH 64        /* tokens per call                           */
+#define PI_MAX_D_MODEL 16384   /* d_model upper bound                       */
+#define PI_MAX_RANK 8192       /* predictor rank upper bound                */
+#define PI_MAX_D_FF (1 << 20)  /* d_ff upper bound                          */
+
+typedef enum pi_status {
+  PI_OK = 0,
+  PI_ERR_INVALID = 1,      /* bad argument, nothing enqueued                */
+  PI_ERR_UNSUPPORTED = 2,  /* valid but not implemented, nothing enqueued   */
+  PI_ERR_CUDA = 3,         /* a CUDA call or launch failed                  */
+  PI_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out            */
+  PI_ERR_DEVICE_CHECK = 5  /* a device-side range check failed              */
+} pi_status;
+
+typedef enum pi_dtype { PI_F32 = 0, PI_F16 = 1, PI_Q4_0 = 2 } pi_dtype;
+typedef enum pi_act { PI_RELU = 0, PI_REGLU = 1 } pi_act;
+
+/* How a batch's tokens share the predicted neuron set.
+ *  PER_TOKEN: each token's FFN runs over its own predicted set; rows
+ *             listed for any token are read once and a token whose own
+ *             mask bit is 0 gets h = 0 for that neuron.
+ *  UNION:     every token's FFN runs over the union of the batch's
+ *             predicted sets (prefill). */
+typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_mode;
+
+/* One FFN layer and its predictor.  All pointers are device pointers.
+ *  d_model, d_ff, rank : sizes d, F, r.  hot : H, 0 <= H <= F, the
+ *                        always-active prefix [0, H) of the neuron order.
+ *  act        : PI_RELU  h_j = max(0, w_up[j].xh + bias[j])
+ *               PI_REGLU h_j = max(0, w_gate[j].xh + bias[j]) * (w_up[j].xh)
+ *  w_dtype    : PI_F32, PI_F16 or PI_Q4_0 for w_gate / w_up / w_down_t.
+ *  p_dtype    : PI_F32 or PI_F16 for p1 / p2.
+ *  w_gate     : [F][d] (ReGLU only; NULL for ReLU).   w_up : [F][d].
+ *  w_down_t   : [F][d], row j = column j of W_down, so y = sum_j h_j w_down_t[j].
+ *  *_scales   : Q4_0 only, [F][d/32] binary16; NULL otherwise.
+ *  bias       : [F] fp32 on the first matrix (gate for ReGLU, up for ReLU); NULL = 0.
+ *  p1         : [r][d], p2 : [F][r]; predictor logits z = p2 (p1 xh) + p_bias.
+ *  p_bias     : [F] fp32; NULL = 0.
+ * Alignment: every weight pointer 16-byte aligned; d % 8 (F32, F16),
+ * d % 32 (Q4_0) == 0; r % 4 (F32 predictor) / r % 8 (F16 predictor) == 0. */
+typedef struct pi_layer {
+  int32_t d_model, d_ff, rank, hot;
+  int32_t act, w_dtype, p_dtype;
+  const void* w_gate;
+  const void* w_up;
+  const void* w_down_t;
+  const void* w_gate_scales;
+  const void* w_up_scales;
+  const void* w_down_t_scales;
+  const float* bias;
+  const void* p1;
+  const void* p2;
+  const float* p_bias;
+} pi_layer;
+
+/* Bytes of workspace the calls below need for these layers at this batch
+ * size, on the current CUDA device (the split of the down projection
+ * follows the device's SM count).  Returns 0 on invalid arguments. */
+size_t pi_workspace_bytes(const pi_layer* layers, int n_layers, int batch);
+
+/* Clears the workspace's status word and wait counters; call once after
+ * allocating a workspace (256-byte aligned) and before its first use. */
+pi_status pi_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* The activation predictor (QbitAI article, §"Что такое «разреженная
+ * активация»?": a small per-layer model predicts the neurons the input
+ * activates).  For each token b of xh [batch][d] (the FFN input, fp32):
+ *   u = p1 xh_b (fp32 accumulation),  z_j = p2[j] . u + p_bias[j],
+ *   bit j of mask[b] = 1  if j < hot, or if sigmoid(z_j) > tau, i.e.
+ *                         z_j > logit(tau) (logit taken in double, rounded
+ *                         to fp32); 0 otherwise.  Rows j < hot of p2 are not read.
+ * mask: [batch][ceil(d_ff/32)] uint32.  tau in (0, 1).  batch in [1, 64].
+ * Workspace: pi_workspace_bytes(layer, 1, batch). */
+pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float tau,
+                     uint32_t* mask, void* ws, size_t ws_bytes, void* stream);
+
+/* Mask compaction: neuron ids j in [begin, d_ff) whose bit is set, in
+ * ascending order, int32.  mask: [batch][ceil(d_ff/32)].
+ *   PI_MASK_UNION    : one list over the OR of the batch's masks;
+ *                      idx [d_ff] (first count[0] entries valid), count [1].
+ *   PI_MASK_PER_TOKEN: one list per token; token b's list at idx + b*d_ff,
+ *                      its length in count[b]; idx [batch][d_ff], count [batch].
+ * count stays on the device.  0 <= begin <= d_ff. */
+pi_status pi_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,
+                     int32_t* idx, int32_t* count, void* stream);
+
+/* The FFN over the neuron set S = [0, hot) U idx[0 .. *count) for a batch of
+ * FFN inputs xh [batch][d]:
+ *   y[b] = sum over j in S, of h_bj * w_down_t[j]   (fp32, [batch][d])
+ * with h_bj the activation of `act`.  idx: ascending neuron ids in
+ * [hot, d_ff) (e.g. pi_compact with begin = hot and PI_MASK_UNION); count: a
+ * device int32.  mode PI_MASK_PER_TOKEN with batch > 1 also needs `mask`
+ * ([batch][ceil(d_ff/32)]) and sets h_bj = 0 when token b's bit j is 0 for
+ * a cold neuron j; otherwise mask may be NULL.  Rows whose h is 0 for every
+ * token of the batch are not read from w_down_t.  The down projection is a
+ * split-K sum whose split and order are fixed for a given device, batch
+ * and count, so results are bitwise reproducible.  Out-of-range ids or
+ * count are skipped and flagged in the status word.
+ * Workspace: pi_workspace_bytes(layer, 1, batch). */
+pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch,
+                        const uint32_t* mask, const int32_t* idx, const int32_t* count,
+                        int mode, float* y, void* ws, size_t ws_bytes, void* stream);
+
+/* A stack of n_layers sparse FFN layers on the residual stream
+ * x [batch][d] (fp32, updated in place), each layer l being
+ *   xh = x / sqrt(mean(x^2) + 1e-6);  mask = pi_predict(layer l, xh, tau);
+ *   S  = [0, hot) U (compaction of the mask over [hot, d_ff));
+ *   x  = x + FFN_S(xh)
+ * (the pre-norm residual chaining is this library's reading; the pages do
+ * not describe how layers chain).  All layers must share d_model and d_ff;
+ * `layers`
+ * is a HOST array of n_layers descriptors.  mode: PI_MASK_PER_TOKEN or
+ * PI_MASK_UNION as in pi_sparse_ffn.  mask_trace: NULL, or device
+ * [n_layers][batch][ceil(d_ff/32)] receiving every layer's predicted masks
+ * (d_ff of the largest layer).  No host synchronisation; capturable in a
+ * CUDA graph.  Workspace: pi_workspace_bytes(layers, n_layers, batch). */
+pi_status pi_ffn_stack(const pi_layer* layers, int n_layers, float* x, int batch, float tau,
+                       int mode, uint32_t* mask_trace, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Kernel kinds timed by pi_ffn_stack_profile, in launch order per layer. */
+enum {
+  PI_KIND_RMSNORM = 0,
+  PI_KIND_PRED_U = 1,    /* u = p1 xh                                     */
+  PI_KIND_PRED_Z = 2,    /* logits, threshold, mask                        */
+  PI_KIND_COMPACT = 3,   /* mask -> ascending list                          */
+  PI_KIND_FFN_UP = 4,    /* gathered gate/up rows + activation              */
+  PI_KIND_FFN_DOWN = 5,  /* gathered split-K down projection                */
+  PI_KIND_REDUCE = 6,    /* fixed-order partial sum + residual              */
+  PI_KINDS = 7
+};
+
+/* Measurement variant of pi_ffn_stack (same arguments, same launches and
+ * results) that records a CUDA event on `stream` before and after every
+ * launch.  A short delay kernel (about 2 ms, ends on its own) runs first so
+ * the host has enqueued the whole sequence before the device reaches it,
+ * and event intervals hold device time only.  Synchronises `stream` at the
+ * end.  kind_ms[PI_KINDS] receives each kind's total milliseconds,
+ * kind_launches[PI_KINDS] its number of launches (both nullable). */
+pi_status pi_ffn_stack_profile(const pi_layer* layers, int n_layers, float* x, int batch,
+                               float tau, int mode, uint32_t* mask_trace, void* ws,
+                               size_t ws_bytes, void* stream, float* kind_ms,
+                               int* kind_launches);
+
+const char* pi_kind_name(int kind);
+
+/* Synchronises `stream` and reads the workspace's two row counters, which
+ * every FFN launch advances on the device: out[0] = neuron rows whose
+ * gate/up (ReGLU) or up (ReLU) weights were read, out[1] = rows of w_down_t
+ * read (rows whose h was nonzero for some token).  Each pass over a row by a
+ * token chunk of at most 8 tokens counts once.  Together with the
+ * predictor's fixed size they give the bytes the path actually read.
+ * `clear` != 0 resets both. */
+pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out);
+
+/* Synchronises `stream`, reads the workspace's status word and returns
+ * PI_OK, PI_ERR_DEVICE_CHECK or PI_ERR_TIMEOUT (timeout wins).  `detail`
+ * (nullable) receives the raw word; `clear` != 0 resets it. */
+pi_status pi_get_device_status(void* ws, void* stream, int clear, uint32_t* detail);
+
+const char* pi_status_string(int status);
+const char* pi_last_error(void);
+int pi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PI_H */

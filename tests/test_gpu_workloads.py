@@ -1,0 +1,112 @@
+"""CUDA path vs the CPU oracle at the five workloads' full layer shapes, in
+the launch configuration the benchmark times (pi_ffn_stack), plus the
+headline 80-layer Llama2-70B-shaped Q4_0 stack.  Where the oracle would be
+too slow (64-token union batches) it checks a sample of tokens one by one;
+masks of every token are checked."""
+import numpy as np
+import pytest
+
+from activation_sparse_predictor_b200 import synth
+from gpu_helpers import TOL, check_mask, device_layer, pi_mod, words_np
+from oracle import rel_l2
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+NAMES = synth.WORKLOAD_ORDER
+
+
+@pytest.fixture(scope="module")
+def pi():
+    return pi_mod()
+
+
+def _run_layer_stack(pi, L, x0, mode, words):
+    batch = x0.shape[0]
+    x = torch.from_numpy(x0).cuda()
+    trace = torch.zeros((1, batch, words), dtype=torch.int32, device="cuda")
+    pi.pi_ffn_stack([L], x, 0.5, mode, mask_trace=trace)
+    return x.cpu().numpy(), words_np(trace)[0]
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_workload_layer_decode(pi, orc, name):
+    w = synth.WORKLOADS[name]
+    layer = w.n_layers - 1
+    L, _ = device_layer(w, layer)
+    H = synth.layer_host(w, layer)
+    words = (w.d_ff + 31) // 32
+    for batch in w.batches:
+        x0 = synth.x_host(w, 0, batch)
+        xg, tr = _run_layer_stack(pi, L, x0, pi.PI_MASK_PER_TOKEN, words)
+        for b in range(batch):
+            xo, m, z = orc.layer_forward(H, x0[b], w.tau)
+            flips = check_mask(tr[b], z, w.d_ff, w.hot, synth.threshold_logit(w.tau))
+            if flips:
+                continue  # a band neuron decided differently: this token's y is not comparable
+            assert rel_l2(xg[b] - x0[b], xo - x0[b]) <= TOL[w.w_dtype], (name, batch, b)
+        # the separate entry points on the oracle's own mask
+        xh = np.stack([orc.rmsnorm(x0[b]) for b in range(batch)]).astype(np.float32)
+        _, z0 = orc.predict(H, xh[0].astype(np.float64))
+        m0 = orc.mask(z0, w.d_ff, w.hot, 0.0)
+        dm = torch.from_numpy(m0.view(np.int32)[None]).cuda()
+        idx, cnt = pi.pi_compact(dm, w.d_ff, w.hot, pi.PI_MASK_UNION)
+        lst = orc.compact(m0, w.d_ff, w.hot)
+        assert int(cnt.cpu()[0]) == len(lst)
+        assert np.array_equal(idx.cpu().numpy()[0, :len(lst)], lst)
+        y = pi.pi_sparse_ffn(L, torch.from_numpy(xh[:1]).cuda(), None, idx, cnt,
+                             pi.PI_MASK_UNION).cpu().numpy()[0]
+        assert rel_l2(y, orc.sparse_ffn(H, xh[0].astype(np.float64), lst)) <= TOL[w.w_dtype]
+
+
+@pytest.mark.parametrize("name", [n for n in NAMES if synth.WORKLOADS[n].union_batches])
+def test_workload_layer_union(pi, orc, name):
+    w = synth.WORKLOADS[name]
+    L, _ = device_layer(w, 0)
+    H = synth.layer_host(w, 0)
+    words = (w.d_ff + 31) // 32
+    for batch in w.union_batches:
+        x0 = synth.x_host(w, 1, batch)
+        xg, tr = _run_layer_stack(pi, L, x0, pi.PI_MASK_UNION, words)
+        ms, xh, flips = [], [], 0
+        for b in range(batch):
+            xhb = orc.rmsnorm(x0[b])
+            _, z = orc.predict(H, xhb)
+            flips += check_mask(tr[b], z, w.d_ff, w.hot, 0.0)
+            ms.append(orc.mask(z, w.d_ff, w.hot, 0.0))
+            xh.append(xhb)
+        union = orc.compact(np.stack(ms), w.d_ff, w.hot)
+        if flips:
+            pytest.skip("a band neuron decided differently; union set not comparable")
+        for b in (0, batch // 2 + 5, batch - 1):
+            ref = orc.sparse_ffn(H, xh[b], union)
+            assert rel_l2(xg[b] - x0[b], ref) <= TOL[w.w_dtype], (name, b)
+
+
+def test_headline_stack_80_layers(pi, orc):
+    """Llama2-70B-shaped Q4_0 ReGLU stack, 80 layers, batch 1: masks of the
+    first layers match the oracle chain, a 2-layer chain matches end to end,
+    and the whole stack is bitwise reproducible."""
+    w = synth.WORKLOADS["llama2_70b_reglu_8192x28672_q4_0"]
+    layers = [device_layer(w, l)[0] for l in range(w.n_layers)]
+    words = (w.d_ff + 31) // 32
+    x0 = synth.x_host(w, 0, 1)
+    outs, trace = [], None
+    for rep in range(2):
+        x = torch.from_numpy(x0).cuda()
+        tr = torch.zeros((w.n_layers, 1, words), dtype=torch.int32, device="cuda")
+        pi.pi_ffn_stack(layers, x, 0.5, pi.PI_MASK_UNION, mask_trace=tr)
+        outs.append(x.cpu().numpy())
+        trace = words_np(tr)
+    assert np.array_equal(outs[0], outs[1])
+    assert np.all(np.isfinite(outs[0]))
+    # oracle chain over the first two layers
+    xr = x0[0].astype(np.float64)
+    for l in range(2):
+        H = synth.layer_host(w, l)
+        xo, m, z = orc.layer_forward(H, xr.astype(np.float32), 0.5)
+        assert check_mask(trace[l, 0], z, w.d_ff, w.hot, 0.0) == 0
+        xr = xo
+    x = torch.from_numpy(x0).cuda()
+    pi.pi_ffn_stack(layers[:2], x, 0.5, pi.PI_MASK_UNION)
+    assert rel_l2(x.cpu().numpy()[0] - x0[0], xr - x0[0]) <= TOL["q4_0"]
