@@ -8,6 +8,7 @@
 #include "pi.h"
 #include "pi_common.cuh"
 #include "pi_kernels.cuh"
+#include "pi_stack.cuh"
 
 namespace pi {
 namespace {
@@ -68,6 +69,12 @@ pi_status check_layer(const pi_layer* L, int i) {
   }
   if ((L->bias && !aligned(L->bias, 4)) || (L->p_bias && !aligned(L->p_bias, 4)))
     return fail(PI_ERR_INVALID, "layer %d: bias pointer not 4-byte aligned", i);
+  const int64_t codes = row_bytes(L->w_dtype, d);
+  const int64_t strides[2] = {L->w_row_stride, L->w_down_row_stride};
+  for (int64_t st : strides)
+    if (st != 0 && (st < codes || st % 16 != 0))
+      return fail(PI_ERR_INVALID, "layer %d: row stride %lld must be 0 or a multiple of 16 >= %lld",
+                  i, (long long)st, (long long)codes);
   return PI_OK;
 }
 
@@ -82,7 +89,12 @@ WsLayout layout_for(int d, int F, int r, int batch) {
   w.idx = take((size_t)F * 4);
   w.count = take(16);
   w.h = take((size_t)F * batch * 4);
-  w.part = take((size_t)w.splits * batch * d * 4);
+  // split-K partials: the multi-kernel split, or one slice per SM for the
+  // fused single-token stack
+  const size_t parts = (size_t)w.splits * batch > 2 * (size_t)device_sms()
+                           ? (size_t)w.splits * batch
+                           : 2 * (size_t)device_sms();
+  w.part = take(parts * d * 4);
   w.y = take((size_t)batch * d * 4);
   w.total = off;
   return w;
@@ -176,11 +188,26 @@ pi_status stack_check(const pi_layer* layers, int n_layers, float* x, int batch,
 
 pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, float tau,
                     int mode, uint32_t* mask_trace, void* ws, const WsLayout& lay,
-                    cudaStream_t s, Prof* prof) {
+                    cudaStream_t s, Prof* prof, unsigned long long* trace = nullptr,
+                    unsigned long long* utrace = nullptr) {
   Prof none;
   Prof& P = prof ? *prof : none;
   pi_status st;
   const float theta = logit32(tau);
+  if (stack1_supported(layers, n_layers, batch)) {
+    const int words = words_of(layers[0].d_ff), chunk = stack1_chunk();
+    for (int l0 = 0; l0 < n_layers; l0 += chunk) {
+      const int n = n_layers - l0 < chunk ? n_layers - l0 : chunk;
+      P.before(PI_KIND_FUSED);
+      cudaError_t e = launch_stack1(layers + l0, n, x,
+                                    mask_trace ? mask_trace + (size_t)l0 * words : nullptr, ws,
+                                    lay, theta, s, trace ? trace + (size_t)l0 * device_sms() * 16 : nullptr,
+                                    utrace ? utrace + (size_t)l0 * stack1_unit_trace_len() * 4 : nullptr);
+      P.after();
+      if (e != cudaSuccess) return cuda_fail(e, "fused stack launch");
+    }
+    return PI_OK;
+  }
   const int d = layers[0].d_model, words = words_of(layers[0].d_ff);
   const int per_token = (mode == PI_MASK_PER_TOKEN && batch > 1);
   float* xh = at<float>(ws, lay.xh);
@@ -309,8 +336,8 @@ pi_status pi_ffn_stack(const pi_layer* layers, int n_layers, float* x, int batch
 }
 
 const char* pi_kind_name(int kind) {
-  static const char* names[PI_KINDS] = {"rmsnorm", "pred_u", "pred_z", "compact",
-                                        "ffn_up",  "ffn_down", "reduce"};
+  static const char* names[PI_KINDS] = {"rmsnorm", "pred_u",   "pred_z", "compact",
+                                        "ffn_up",  "ffn_down", "reduce", "fused_stack"};
   return (kind >= 0 && kind < PI_KINDS) ? names[kind] : "unknown";
 }
 
@@ -354,6 +381,21 @@ pi_status pi_ffn_stack_profile(const pi_layer* layers, int n_layers, float* x, i
   delete[] P.kind;
   return st;
 }
+
+pi_status pi_ffn_stack_timeline(const pi_layer* layers, int n_layers, float* x, float tau,
+                                void* ws, size_t ws_bytes, void* stream,
+                                unsigned long long* timeline, unsigned long long* unit_timeline) {
+  WsLayout lay;
+  pi_status st = stack_check(layers, n_layers, x, 1, tau, PI_MASK_UNION, nullptr, ws, ws_bytes, &lay);
+  if (st != PI_OK) return st;
+  if (!timeline || !aligned(timeline, 8)) return fail(PI_ERR_INVALID, "timeline null or misaligned");
+  if (!stack1_supported(layers, n_layers, 1))
+    return fail(PI_ERR_UNSUPPORTED, "these layers do not run on the persistent kernel");
+  return stack_run(layers, n_layers, x, 1, tau, PI_MASK_UNION, nullptr, ws, lay,
+                   (cudaStream_t)stream, nullptr, timeline, unit_timeline);
+}
+
+int pi_device_sms(void) { return device_sms(); }
 
 pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {
   if (!ws || !aligned(ws, 256) || !out) return fail(PI_ERR_INVALID, "workspace or output null");

@@ -86,6 +86,14 @@ __host__ __device__ __forceinline__ int64_t row_bytes(int dt, int d) {
   return dt == PI_F32 ? 4LL * d : (dt == PI_F16 ? 2LL * d : (int64_t)d / 2);
 }
 
+// Row-to-row distance of a weight matrix's codes, and of its Q4_0 scales.
+__host__ __device__ __forceinline__ int64_t code_stride(int dt, int d, int64_t stride) {
+  return stride ? stride : row_bytes(dt, d);
+}
+__host__ __device__ __forceinline__ int64_t scale_stride(int d, int64_t stride) {
+  return stride ? stride : (int64_t)(d / 32) * 2;
+}
+
 // ----------------------------------------------------------- workspace
 // Offsets (bytes from the workspace base) of the buffers a call uses.
 struct WsLayout {

@@ -304,8 +304,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
   constexpr int NR = (ACT == PI_REGLU) ? 2 : 1;
   constexpr int CC = WTraits<WT>::CHUNK_COLS;
   const int nch = d / CC;
-  const int64_t rb = row_bytes(WT, d);
-  const int nb = d / 32;
+  const int64_t rb = code_stride(WT, d, L.w_row_stride);
+  const int64_t sbs = scale_stride(d, L.w_row_stride);
   for (int n = blockIdx.x * kWarps + warp; n < N; n += gridDim.x * kWarps) {
     const int j = n < H ? n : idx[n - H];
     if (j < H && n >= H || j >= F || j < 0) {
@@ -321,11 +321,11 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
     if constexpr (ACT == PI_REGLU) {
       rows[0] = (const char*)L.w_gate + (size_t)j * rb;
       rows[1] = (const char*)L.w_up + (size_t)j * rb;
-      sc[0] = (const uint16_t*)L.w_gate_scales + (size_t)j * nb;
-      sc[1] = (const uint16_t*)L.w_up_scales + (size_t)j * nb;
+      sc[0] = (const uint16_t*)((const char*)L.w_gate_scales + (size_t)j * sbs);
+      sc[1] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs);
     } else {
       rows[0] = (const char*)L.w_up + (size_t)j * rb;
-      sc[0] = (const uint16_t*)L.w_up_scales + (size_t)j * nb;
+      sc[0] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs);
     }
     float acc[NR][TB];
 #pragma unroll
@@ -361,7 +361,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
                                                        const int32_t* __restrict__ count,
                                                        const float* __restrict__ h, int B,
                                                        int S, float* __restrict__ part,
-                                                       WsHeader* hdr) {
+                                                       WsHeader* hdr, int64_t stride) {
   const int s = blockIdx.y, t0 = blockIdx.z * TB;
   const int col0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   int cnt = *count;
@@ -373,8 +373,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
   for (int b = 0; b < TB; ++b)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
-  const int64_t rb = row_bytes(WT, d);
-  const int nb = d / 32;
+  const int64_t rb = code_stride(WT, d, stride);
+  const int64_t sbs = scale_stride(d, stride);
   unsigned long long nread = 0;
   if (col0 < d) {
 #pragma unroll 4
@@ -404,7 +404,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
       } else {
         const int blk = col0 >> 5, k0 = col0 & 31;
         const uint2 q = *reinterpret_cast<const uint2*>(row + (size_t)blk * 16 + (k0 & 15));
-        const float sc = h2f(wsc[(size_t)j * nb + blk]);
+        const float sc = h2f(reinterpret_cast<const uint16_t*>(
+            reinterpret_cast<const char*>(wsc) + (size_t)j * sbs)[blk]);
         const int sh = k0 >= 16 ? 4 : 0;
         const uint32_t qq[2] = {q.x, q.y};
 #pragma unroll
@@ -447,6 +448,15 @@ __global__ void k_delay(unsigned long long ns) {
   } while (t - t0 < ns && t >= t0);
 }
 
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+  return allow_smem_fn(reinterpret_cast<const void*>(kernel), bytes);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ policy
+
 // Shared-memory opt-in: raises a kernel's dynamic shared-memory limit on the
 // current device the first time a launch needs more than 48 KB (keyed by the
 // kernel's address), so a warm-up call leaves nothing but launches for a
@@ -466,14 +476,6 @@ cudaError_t allow_smem_fn(const void* fn, size_t bytes) {
   return e;
 }
 
-template <typename K>
-cudaError_t allow_smem(K kernel, size_t bytes) {
-  return allow_smem_fn(reinterpret_cast<const void*>(kernel), bytes);
-}
-
-}  // namespace
-
-// ------------------------------------------------------------------ policy
 
 int device_sms() {
   static int cache[64] = {0};
@@ -622,7 +624,8 @@ static cudaError_t ffn_down_t(const pi_layer& L, int batch, const int32_t* idx,
   dim3 grid(tiles, S, (batch + TB - 1) / TB);
   k_ffn_down<WT, TB><<<grid, kThreads, 0, s>>>((const char*)L.w_down_t,
                                               (const uint16_t*)L.w_down_t_scales, L.d_model,
-                                              L.d_ff, L.hot, idx, count, h, batch, S, part, hdr);
+                                              L.d_ff, L.hot, idx, count, h, batch, S, part, hdr,
+                                              L.w_down_row_stride);
   return cudaGetLastError();
 }
 

@@ -10,6 +10,9 @@
 namespace pi {
 
 int device_sms();                 // SM count of the current device (cached)
+
+// Raises a kernel's dynamic shared-memory limit on the current device once.
+cudaError_t allow_smem_fn(const void* fn, size_t bytes);
 int pick_tb(int batch, int d);    // tokens per pass of the x-staged kernels
 int down_tb(int batch);           // tokens per pass of the down projection
 int down_splits(int batch, int d);// split-K slices of the down projection

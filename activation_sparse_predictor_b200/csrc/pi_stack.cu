@@ -1,0 +1,1389 @@
+// Persistent single-token decode kernel for the whole FFN stack (sm_100a).
+//
+// One cooperative launch runs a chunk of layers with one CTA per SM.  Each
+// CTA has a producer warp that streams every weight row the CTA will use
+// through a ring of shared-memory stages with 1-D bulk copies
+// (cp.async.bulk, completion counted on an mbarrier per stage), and eight
+// consumer warps that share every stage: each consumer thread owns a slice
+// of the row's columns, so a stage is held only briefly and the ring keeps
+// many rows in flight.  Per layer:
+//
+//   x^  : every CTA normalises the full residual vector (rmsnorm) itself
+//   A   : predictor rows of P1 (a static share per CTA)   -> u      | grid barrier 1
+//   B   : predictor rows of P2 for the CTA's mask words   -> mask   | grid barrier 2 (arrive)
+//   C   : the CTA's hot neurons (j = s, s + SMs, ...)      -> h
+//         grid barrier 2 (wait), compaction of the mask in every CTA, the
+//         CTA's share of the ascending cold list (positions s, s + SMs, ...) -> h
+//   D   : down rows of the CTA's neurons whose h != 0     -> partial y | grid barrier 3
+//   E   : fixed-order reduction of the CTA's column slice, residual add | grid barrier 4
+//
+// The producer runs ahead across phases for every row whose address does
+// not depend on this layer's data (P1, P2, hot rows, the next layer's rows),
+// so HBM keeps streaming through the grid barriers; only cold rows wait for
+// the compaction and down rows for their h.  Every wait (mbarrier, grid
+// barrier, flag) is bounded by %globaltimer; a wait that runs out sets
+// DEV_TIMEOUT and an abort flag, after which every thread runs the rest of
+// its loops without waiting or computing and the producer waits (bounded)
+// for its own copies in flight before exiting.
+//
+// Q4_0 gate/up dot products are exact integer sums: the normalised input is
+// rounded once per layer to int16 on a per-vector scale, each block's
+// sum_k (q_k - 8) x_k is formed with dp2a in int32 (no rounding), then
+// scaled in fp32.  Everything else accumulates in fp32.
+#include <cstdlib>
+#include <cstring>
+
+#include "pi_kernels.cuh"
+#include "pi_stack.cuh"
+
+namespace pi {
+namespace {
+
+constexpr int NCW = 16;             // consumer warps
+constexpr int NCT = NCW * 32;       // consumer threads
+constexpr int NPMAX = 4;            // producer warps at most (after the consumers)
+constexpr int NTHR = NCT + 32 * NPMAX;
+constexpr int NSMAX = 24;           // ring stages at most
+constexpr int MAXL = 24;            // layers per launch
+constexpr int GRP = 32;             // items per cross-warp finalisation group
+constexpr int MAXA = 16;            // P1 rows per CTA at most
+constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
+constexpr int UTR = 512;            // units per layer recorded by the unit trace
+
+struct LayerPtrs {
+  const char* first;            // W_gate (ReGLU) or W_up (ReLU): codes / rows
+  const char* second;           // W_up (ReGLU only)
+  const char* down;             // W_down^T
+  const char* first_scales;     // Q4_0 scales
+  const char* second_scales;
+  const char* down_scales;
+  const float* bias;
+  const char* p1;
+  const char* p2;
+  const float* pbias;
+};
+static_assert(sizeof(LayerPtrs) == 80, "compact layer pointers");
+
+// Shape and shared-memory plan, identical for every CTA.
+struct Plan {
+  int d, F, r, H;
+  int ns, G, maxc, maxi, nsms;
+  int np;                           // producer warps (divides ns)
+  int gw, gd;                       // consumer warp groups: up-projection / down phases
+  int hp;                           // hot neurons per unit (adjacent records)
+  int dr;                           // down rows per unit at most (adjacent records)
+  int packed_up, packed_down;       // neuron records contiguous in memory
+  long long up_stride, down_stride; // bytes between consecutive neurons' rows (codes)
+  long long up_sstride, down_sstride; // the same for Q4_0 scales
+  uint32_t sb;                      // stage bytes
+  uint32_t rowb, scb;               // weight row bytes (codes), Q4_0 scale row bytes
+  uint32_t p1_bytes, p2_row;        // predictor row bytes
+  uint32_t item_bytes, down_bytes;  // bytes copied per item / per down row
+  uint32_t o_first_s, o_second, o_second_s, o_down_s;  // offsets inside a stage
+  uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_mw, o_scan, o_cold, o_hval, o_flag,
+      o_dlist, o_runs, o_pbs, o_hbs, o_redA, o_redC, o_redE, o_ring, total;
+};
+
+struct StackParams {
+  Plan pl;
+  int n_layers;
+  float theta;
+  float* x;              // [d] residual stream, in/out
+  uint32_t* mask;        // this chunk's first layer's mask words
+  long long mask_stride; // words between consecutive layers' masks (0: reused)
+  float* u;              // [r]
+  float* part;           // [nsms][d]
+  int32_t* count;        // cold-list length of the last layer
+  WsHeader* hdr;
+  unsigned long long* trace;  // nullable [n_layers][nsms][16] timeline
+  unsigned long long* utrace; // nullable [n_layers][UTR][4]: CTA 0's units
+  LayerPtrs L[MAXL];
+};
+static_assert(sizeof(StackParams) < 4000, "kernel parameter block under 4 KB");
+
+// -------------------------------------------------------------- primitives
+
+__device__ __forceinline__ uint32_t sa(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint64_t gtime() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(sa(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(sa(b)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(sa(b)), "r"(count)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(sa(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait that lets the hardware suspend the warp until the phase completes
+// or `hint_ns` passes, so waiting warps do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(sa(b)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// 1-D bulk copy global -> shared, completion counted on `bar` (bytes % 16 == 0,
+// both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
+                                         uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(sa(dst)),
+      "l"(src), "r"(bytes), "r"(sa(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+
+__device__ __forceinline__ void csync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-barrier arrival (after a CTA-wide bar.sync): release at gpu scope,
+// cumulative over the writes the CTA's threads made before the bar.sync.
+__device__ __forceinline__ void grid_arrive(uint32_t* ctr) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+
+__device__ __forceinline__ float4 f4add(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+// ------------------------------------------------------ vector layouts
+// Vectors dotted with fp16 rows (x^ and u when the predictor is fp16) are
+// staged "split-half": element i at ((i & 7) >> 2) * n/2 + (i >> 3) * 4 + (i & 3),
+// so the two float4 halves of 16-byte chunk c are float4 number c and
+// n/8 + c, and consecutive threads read consecutive 16-byte words (no bank
+// conflicts).  fp32 rows use the natural order.  The int16 copy of x^ for
+// Q4_0 rows is sub-chunk-major: element 32k + 8q + o at (q * nb + k) * 8 + o.
+template <int DT>
+__device__ __forceinline__ int vpos(int i, int n) {
+  if constexpr (DT == PI_F16) return ((i & 7) >> 2) * (n >> 1) + ((i >> 3) << 2) + (i & 3);
+  return i;
+}
+
+__device__ __forceinline__ int qpos(int i, int nb) {
+  return ((((i >> 3) & 3) * nb + (i >> 5)) << 3) + (i & 7);
+}
+
+// Dot product of 16-byte chunk c of a DT row with the staged vector v (length n).
+template <int DT>
+__device__ __forceinline__ float chunk_dot(const uint4 w, const float* v, int c, int n) {
+  const float4* v4 = reinterpret_cast<const float4*>(v);
+  if constexpr (DT == PI_F32) {
+    const float4 x = v4[c];
+    float a = __uint_as_float(w.x) * x.x;
+    a = fmaf(__uint_as_float(w.y), x.y, a);
+    a = fmaf(__uint_as_float(w.z), x.z, a);
+    return fmaf(__uint_as_float(w.w), x.w, a);
+  } else {
+    float f[8];
+    f16x8_to_f32(w, f);
+    const float4 lo = v4[c], hi = v4[(n >> 3) + c];
+    float a = f[0] * lo.x, b = f[4] * hi.x;
+    a = fmaf(f[1], lo.y, a);
+    b = fmaf(f[5], hi.y, b);
+    a = fmaf(f[2], lo.z, a);
+    b = fmaf(f[6], hi.z, b);
+    a = fmaf(f[3], lo.w, a);
+    b = fmaf(f[7], hi.w, b);
+    return a + b;
+  }
+}
+
+// sum_k (q_k - 8) * x_k over one Q4_0 block in exact int32 arithmetic:
+// xw[m] holds the int16 pair (x[2m], x[2m+1]); `base` = -8 * sum_k x_k.
+__device__ __forceinline__ int q4_block_dot(const uint4 v, const int (&xw)[16], int base) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  int lo_acc = base, hi_acc = 0;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int lo = (int)(w[m] & 0x0F0F0F0Fu);         // elements 4m .. 4m+3
+    const int hi = (int)((w[m] >> 4) & 0x0F0F0F0Fu);  // elements 4m+16 .. 4m+19
+    lo_acc = __dp2a_lo(xw[2 * m], lo, lo_acc);
+    lo_acc = __dp2a_hi(xw[2 * m + 1], lo, lo_acc);
+    hi_acc = __dp2a_lo(xw[8 + 2 * m], hi, hi_acc);
+    hi_acc = __dp2a_hi(xw[9 + 2 * m], hi, hi_acc);
+  }
+  return lo_acc + hi_acc;
+}
+
+// -------------------------------------------------------- shared carving
+
+struct Smem {
+  uint64_t* full;
+  uint64_t* empty;
+  uint64_t* listbar;
+  volatile int* abort;        // CTA-wide: stop waiting and computing
+  volatile int* nc;           // this CTA's cold items (current layer)
+  float* xscale;              // int16 scale of xh (Q4_0)
+  float* xf;
+  int16_t* xi;
+  int* bsum;
+  float* us;
+  uint32_t* bw;
+  uint32_t* mw;
+  int* scan;
+  int* cold;
+  float* hval;
+  volatile int* flag;
+  int* dlist;
+  int* runs;                  // down-row units: first dlist position, row count
+  float* pbs;                 // predictor biases of the CTA's mask words
+  float* hbs;                 // activation biases of the CTA's items
+  float* redA;
+  float* redC;
+  float4* redE;
+  char* ring;
+};
+
+__device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
+  Smem S;
+  S.full = reinterpret_cast<uint64_t*>(base);
+  S.empty = S.full + NSMAX;
+  S.listbar = S.empty + NSMAX;
+  int* misc = reinterpret_cast<int*>(base + pl.o_misc);
+  S.abort = misc;
+  S.nc = misc + 1;
+  S.xscale = reinterpret_cast<float*>(misc + 2);
+  S.xf = reinterpret_cast<float*>(base + pl.o_xf);
+  S.xi = reinterpret_cast<int16_t*>(base + pl.o_xi);
+  S.bsum = reinterpret_cast<int*>(base + pl.o_bsum);
+  S.us = reinterpret_cast<float*>(base + pl.o_u);
+  S.bw = reinterpret_cast<uint32_t*>(base + pl.o_bw);
+  S.mw = reinterpret_cast<uint32_t*>(base + pl.o_mw);
+  S.scan = reinterpret_cast<int*>(base + pl.o_scan);
+  S.cold = reinterpret_cast<int*>(base + pl.o_cold);
+  S.hval = reinterpret_cast<float*>(base + pl.o_hval);
+  S.flag = reinterpret_cast<volatile int*>(base + pl.o_flag);
+  S.dlist = reinterpret_cast<int*>(base + pl.o_dlist);
+  S.runs = reinterpret_cast<int*>(base + pl.o_runs);
+  S.pbs = reinterpret_cast<float*>(base + pl.o_pbs);
+  S.hbs = reinterpret_cast<float*>(base + pl.o_hbs);
+  S.redA = reinterpret_cast<float*>(base + pl.o_redA);
+  S.redC = reinterpret_cast<float*>(base + pl.o_redC);
+  S.redE = reinterpret_cast<float4*>(base + pl.o_redE);
+  S.ring = reinterpret_cast<char*>(base + pl.o_ring);
+  return S;
+}
+
+// Marks this CTA (and the grid) as aborted after a wait ran out.
+__device__ void raise_abort(const Smem& S, WsHeader* hdr) {
+  *S.abort = 1;
+  atomicOr(&hdr->status, DEV_TIMEOUT);
+  atomicExch(&hdr->counters[1], 1u);
+}
+
+// Bounded mbarrier wait; false on abort or timeout (timeout raises abort).
+// The warp sleeps in the hardware wait between checks.
+__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Smem& S, WsHeader* hdr) {
+  if (mbar_try(bar, parity)) return true;
+  if (*S.abort) return false;
+  const uint64_t t0 = gtime();
+  while (true) {
+    if (mbar_try_sleep(bar, parity, 50000u)) return true;
+    if (*S.abort) return false;
+    if (gtime() - t0 > kTimeoutNs) {
+      raise_abort(S, hdr);
+      return false;
+    }
+  }
+}
+
+// Bounded grid-barrier wait by one thread: counter >= target.
+__device__ bool grid_wait(WsHeader* hdr, uint32_t target, const Smem& S) {
+  if (*S.abort) return false;
+  if (ld_acquire(&hdr->counters[0]) >= target) return true;
+  const uint64_t t0 = gtime();
+  while (true) {
+    __nanosleep(64);
+    if (ld_acquire(&hdr->counters[0]) >= target) return true;
+    if (ld_acquire(&hdr->counters[1]) != 0u) {
+      *S.abort = 1;
+      return false;
+    }
+    if (gtime() - t0 > kTimeoutNs) {
+      raise_abort(S, hdr);
+      return false;
+    }
+  }
+}
+
+// Timeline stamp, when a trace buffer is given.
+__device__ __forceinline__ void tstamp(const StackParams& P, int l, int slot,
+                                       unsigned long long v) {
+  if (P.trace) P.trace[((size_t)l * gridDim.x + blockIdx.x) * 16 + slot] = v;
+}
+
+// Unit trace of CTA 0 (slot 0 armed, 1 data seen by consumer warp 0,
+// 2 released by consumer warp 0, 3 bytes).
+__device__ __forceinline__ void utstamp(const StackParams& P, int l, uint32_t u, int slot,
+                                        unsigned long long v) {
+  if (P.utrace && blockIdx.x == 0 && u < (uint32_t)UTR)
+    P.utrace[((size_t)l * UTR + u) * 4 + slot] = v;
+}
+
+// ------------------------------------------------------------ per-CTA shares
+
+struct Ranges {
+  int kA0, kA1;   // P1 rows
+  int wB0, wB1;   // mask words evaluated here
+  int Wlo, W;     // first word holding a cold neuron, words per mask
+  int ngh;        // hot groups g = s, s + SMs, ... of hp adjacent neurons
+  int nh;         // hot neurons in them
+};
+
+__device__ __forceinline__ Ranges ranges(const Plan& pl) {
+  Ranges R;
+  const int S = gridDim.x, s = blockIdx.x;
+  R.kA0 = (int)((long long)s * pl.r / S);
+  R.kA1 = (int)((long long)(s + 1) * pl.r / S);
+  R.W = (pl.F + 31) / 32;
+  R.Wlo = pl.H / 32;
+  const int Wc = R.W - R.Wlo;
+  R.wB0 = R.Wlo + (int)((long long)s * Wc / S);
+  R.wB1 = R.Wlo + (int)((long long)(s + 1) * Wc / S);
+  const int G = (pl.H + pl.hp - 1) / pl.hp;
+  R.ngh = s < G ? (G - 1 - s) / S + 1 : 0;
+  R.nh = 0;
+  if (R.ngh > 0) {
+    const int gl = s + S * (R.ngh - 1);
+    R.nh = (R.ngh - 1) * pl.hp + min(pl.hp, pl.H - gl * pl.hp);
+  }
+  return R;
+}
+
+// First neuron of this CTA's hot group gi.
+__device__ __forceinline__ int hot_group_first(int gi, const Plan& pl) {
+  return ((int)blockIdx.x + (int)gridDim.x * gi) * pl.hp;
+}
+
+__device__ __forceinline__ int item_neuron(int i, const Ranges& R, const Plan& pl, const Smem& S) {
+  if (i < R.nh) return hot_group_first(i / pl.hp, pl) + i % pl.hp;
+  return S.cold[i - R.nh];
+}
+
+// Down-row units: runs of consecutive nonzero items whose neurons are
+// adjacent (when down records are packed), at most pl.dr rows each.  The
+// producers and the consumers apply this rule to the same sequence.
+__device__ __forceinline__ bool run_extends(int jprev, int jnext, int len, const Plan& pl) {
+  return pl.packed_down && jnext == jprev + 1 && len < pl.dr;
+}
+
+// ---------------------------------------------------------------- producer
+
+template <int WT, int ACT, int PT>
+__device__ void producer(const StackParams& P, const Smem& S, const int p) {
+  const Plan& pl = P.pl;
+  WsHeader* hdr = P.hdr;
+  const Ranges R = ranges(pl);
+  uint32_t uc = 0;  // unit sequence number, identical on every producer and consumer
+  uint32_t last[NSMAX];
+#pragma unroll
+  for (int i = 0; i < NSMAX; ++i) last[i] = 0xFFFFFFFFu;
+  bool ok = true;
+  unsigned long long w_empty = 0, w_list = 0, w_flag = 0;  // stall time (ns)
+  int cur_l = 0;
+  uint32_t l_uc0 = 0;  // first unit of the current layer
+
+  // Stage uc % ns belongs to producer (uc % ns) % np == uc % np (np divides ns).
+  auto mine = [&]() { return (int)(uc % (uint32_t)pl.np) == p; };
+  // Claims unit uc's stage (one of ours) and arms its full barrier for `bytes`.
+  auto claim = [&](uint32_t bytes) -> char* {
+    const int st = (int)(uc % (uint32_t)pl.ns);
+    const uint32_t k = uc / (uint32_t)pl.ns;
+    if (k > 0 && !mbar_try(&S.empty[st], (k - 1) & 1u)) {
+      const unsigned long long t0 = P.trace ? gtime() : 0ull;
+      if (!wait_mbar(&S.empty[st], (k - 1) & 1u, S, hdr)) {
+        ok = false;
+        return nullptr;
+      }
+      if (P.trace) w_empty += gtime() - t0;
+    }
+    mbar_arrive_tx(&S.full[st], bytes);
+    last[st] = uc;
+    if (P.utrace) {
+      utstamp(P, cur_l, uc - l_uc0, 0, gtime());
+      utstamp(P, cur_l, uc - l_uc0, 3, bytes);
+    }
+    return S.ring + (size_t)st * pl.sb;
+  };
+  auto bar_of = [&]() { return &S.full[uc % (uint32_t)pl.ns]; };
+
+  // Up-projection records of neurons j0 .. j0+n-1 (n > 1 only when packed).
+  auto items = [&](const LayerPtrs& L, int j0, int n) {
+    if (mine()) {
+      char* dst = claim(pl.item_bytes * (uint32_t)n);
+      if (dst) {
+        uint64_t* b = bar_of();
+        if (pl.packed_up) {
+          bulk_g2s(dst, L.first + (size_t)j0 * pl.up_stride, pl.item_bytes * (uint32_t)n, b);
+        } else {
+          bulk_g2s(dst, L.first + (size_t)j0 * pl.up_stride, pl.rowb, b);
+          if constexpr (WT == PI_Q4_0)
+            bulk_g2s(dst + pl.o_first_s, L.first_scales + (size_t)j0 * pl.up_sstride, pl.scb, b);
+          if constexpr (ACT == PI_REGLU) {
+            bulk_g2s(dst + pl.o_second, L.second + (size_t)j0 * pl.up_stride, pl.rowb, b);
+            if constexpr (WT == PI_Q4_0)
+              bulk_g2s(dst + pl.o_second_s, L.second_scales + (size_t)j0 * pl.up_sstride, pl.scb, b);
+          }
+        }
+      }
+    }
+    ++uc;
+  };
+  // Down records of neurons j0 .. j0+n-1.
+  auto downs = [&](const LayerPtrs& L, int j0, int n) {
+    if (mine()) {
+      char* dst = claim(pl.down_bytes * (uint32_t)n);
+      if (dst) {
+        uint64_t* b = bar_of();
+        if (pl.packed_down) {
+          bulk_g2s(dst, L.down + (size_t)j0 * pl.down_stride, pl.down_bytes * (uint32_t)n, b);
+        } else {
+          bulk_g2s(dst, L.down + (size_t)j0 * pl.down_stride, pl.rowb, b);
+          if constexpr (WT == PI_Q4_0)
+            bulk_g2s(dst + pl.o_down_s, L.down_scales + (size_t)j0 * pl.down_sstride, pl.scb, b);
+        }
+      }
+    }
+    ++uc;
+  };
+
+  for (int l = 0; l < P.n_layers && ok; ++l) {
+    const LayerPtrs& L = P.L[l];
+    cur_l = l;
+    l_uc0 = uc;
+    // A: predictor rows of P1
+    for (int k = R.kA0; k < R.kA1 && ok; ++k, ++uc) {
+      if (!mine()) continue;
+      char* dst = claim(pl.p1_bytes);
+      if (!dst) break;
+      bulk_g2s(dst, L.p1 + (size_t)k * pl.p1_bytes, pl.p1_bytes, bar_of());
+    }
+    // B: predictor rows of P2, G per unit
+    for (int w = R.wB0; w < R.wB1 && ok; ++w) {
+      for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F && ok; ja += pl.G, ++uc) {
+        if (!mine()) continue;
+        const int jb = min(ja + pl.G, pl.F);
+        const uint32_t bytes = (uint32_t)(jb - ja) * pl.p2_row;
+        char* dst = claim(bytes);
+        if (!dst) break;
+        bulk_g2s(dst, L.p2 + (size_t)ja * pl.p2_row, bytes, bar_of());
+      }
+    }
+    // C: hot groups, then (after the consumers' compaction) cold neurons
+    for (int gi = 0; gi < R.ngh && ok; ++gi) {
+      const int j0 = hot_group_first(gi, pl);
+      items(L, j0, min(pl.hp, pl.H - j0));
+    }
+    {
+      const unsigned long long t0 = P.trace ? gtime() : 0ull;
+      if (!ok || !wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr)) break;
+      if (P.trace) w_list += gtime() - t0;
+    }
+    const int nc = *S.nc;
+    for (int i = 0; i < nc && ok; ++i) items(L, S.cold[i], 1);
+    // D: down rows of items whose h != 0, in item order, as runs
+    const int tag = (l + 1) << 2;
+    int rj = -1, rlen = 0;  // open run: first neuron, rows
+    for (int i = 0; i < R.nh + nc && ok; ++i) {
+      int f = S.flag[i];
+      if ((f & ~3) != tag) {
+        const uint64_t t0 = gtime();
+        while (((f = S.flag[i]) & ~3) != tag) {
+          if (*S.abort) { ok = false; break; }
+          if (gtime() - t0 > kTimeoutNs) { raise_abort(S, hdr); ok = false; break; }
+          __nanosleep(128);
+        }
+        if (P.trace) w_flag += gtime() - t0;
+        if (!ok) break;
+      }
+      if ((f & 3) != 2) continue;
+      const int j = item_neuron(i, R, pl, S);
+      if (rlen > 0 && run_extends(rj + rlen - 1, j, rlen, pl)) {
+        ++rlen;
+        continue;
+      }
+      if (rlen > 0) downs(L, rj, rlen);
+      rj = j;
+      rlen = 1;
+    }
+    if (ok && rlen > 0) downs(L, rj, rlen);
+    if (P.trace && p == 0) {
+      tstamp(P, l, 12, w_empty);
+      tstamp(P, l, 13, w_list);
+      tstamp(P, l, 14, w_flag);
+      tstamp(P, l, 15, gtime());
+      w_empty = w_list = w_flag = 0;
+    }
+  }
+  // Drain: wait (bounded) until every copy this thread issued has landed.
+  for (int st = 0; st < pl.ns; ++st) {
+    if (last[st] == 0xFFFFFFFFu) continue;
+    const uint32_t par = (last[st] / (uint32_t)pl.ns) & 1u;
+    const uint64_t t0 = gtime();
+    while (!mbar_try(&S.full[st], par)) {
+      if (gtime() - t0 > kTimeoutNs) {
+        atomicOr(&hdr->status, DEV_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- consumers
+
+template <int WT, int ACT, int PT>
+__device__ void consumers(const StackParams& P, const Smem& S) {
+  constexpr bool two = (ACT == PI_REGLU);
+  const Plan& pl = P.pl;
+  WsHeader* hdr = P.hdr;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nS = gridDim.x, s = blockIdx.x;
+  const Ranges R = ranges(pl);
+  const int d = pl.d, nb = d / 32;
+  // Units of the predictor and up-projection phases are shared by groups of
+  // WPG warps; unit uc goes to group uc % GW.  GW divides the ring depth, so
+  // a stage is always consumed by the same group and every warp has seen the
+  // previous phase of each stage it waits on (exact parity test).
+  const int GW = pl.gw, WPG = NCW / GW, grp = warp / WPG, wg = warp % WPG;
+  const int gtid = wg * 32 + lane, GT = WPG * 32;
+  // The down-projection phase uses GD groups of NCW / GD warps.
+  const int GD = pl.gd, WPD = NCW / GD, dgrp = warp / WPD;
+  const int dtid = (warp % WPD) * 32 + lane, DT = WPD * 32;
+  uint32_t uc = 0, nbar = 0;
+  int cur_l = 0;
+  uint32_t l_uc0 = 0;
+
+  auto ready = [&](int st) -> bool {
+    const bool ok = wait_mbar(&S.full[st], (uc / (uint32_t)pl.ns) & 1u, S, hdr);
+    if (P.utrace && tid == 0) utstamp(P, cur_l, uc - l_uc0, 1, gtime());
+    return __all_sync(0xffffffffu, ok);
+  };
+  auto stage = [&](int st) { return S.ring + (size_t)st * pl.sb; };
+  // each of the `warps` warps that shared a unit releases its part of it
+  auto release = [&](int st, int warps) {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.empty[st], (uint32_t)(NCW / warps));
+    if (P.utrace && tid == 0) utstamp(P, cur_l, uc - l_uc0, 2, gtime());
+  };
+  auto gsync_arrive = [&]() {
+    csync();
+    ++nbar;
+    if (tid == 0 && !*S.abort) grid_arrive(&hdr->counters[0]);
+  };
+  auto gsync_wait = [&]() {
+    if (tid == 0) grid_wait(hdr, nbar * (uint32_t)nS, S);
+    csync();
+  };
+
+  for (int l = 0; l < P.n_layers; ++l) {
+    const LayerPtrs& L = P.L[l];
+    uint32_t* mask = P.mask + (size_t)l * P.mask_stride;
+    const int tag = (l + 1) << 2;
+    cur_l = l;
+    l_uc0 = uc;
+
+    // ---- x^ = x / sqrt(mean(x^2) + 1e-6); all loads issued at once
+    if (tid == 0) tstamp(P, l, 0, gtime());
+    {
+      constexpr int MX = 6;   // float4 per thread, d <= 12288
+      const float4* x4 = reinterpret_cast<const float4*>(P.x);
+      float4 xv[MX];
+      float ss = 0.f;
+#pragma unroll
+      for (int m = 0; m < MX; ++m) {
+        const int q = tid + m * NCT;
+        xv[m] = q < d / 4 ? __ldcg(x4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int m = 0; m < MX; ++m)
+        ss += xv[m].x * xv[m].x + xv[m].y * xv[m].y + xv[m].z * xv[m].z + xv[m].w * xv[m].w;
+      ss = warp_sum(ss);
+      if (lane == 0) S.redA[warp] = ss;
+      csync();
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) tot += S.redA[w];
+      const float inv = 1.0f / sqrtf(tot / (float)d + 1e-6f);
+      float amax = 0.f;
+#pragma unroll
+      for (int m = 0; m < MX; ++m) {
+        const int q = tid + m * NCT;
+        if (q >= d / 4) break;
+        const float e[4] = {xv[m].x * inv, xv[m].y * inv, xv[m].z * inv, xv[m].w * inv};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          S.xf[vpos<PT>(4 * q + k, d)] = e[k];
+          amax = fmaxf(amax, fabsf(e[k]));
+        }
+      }
+      if constexpr (WT == PI_Q4_0) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        csync();  // everyone has read redA
+        if (lane == 0) S.redA[warp] = amax;
+        csync();
+        float mx = 0.f;
+#pragma unroll
+        for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, S.redA[w]);
+        const float xs = mx > 0.f ? mx / 32767.0f : 1.0f;
+        const float ixs = 1.0f / xs;
+        if (tid == 0) *S.xscale = xs;
+#pragma unroll
+        for (int m = 0; m < MX; ++m) {
+          const int q = tid + m * NCT;
+          if (q >= d / 4) break;
+          const float e[4] = {xv[m].x * inv, xv[m].y * inv, xv[m].z * inv, xv[m].w * inv};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            int v = __float2int_rn(e[k] * ixs);
+            v = v > 32767 ? 32767 : (v < -32767 ? -32767 : v);
+            S.xi[qpos(4 * q + k, nb)] = (int16_t)v;
+          }
+        }
+        csync();
+        const int4* xb = reinterpret_cast<const int4*>(S.xi);
+        for (int k = tid; k < nb; k += NCT) {
+          int t = 0;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int4 v = xb[q * nb + k];
+            const int w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) t += (int)(int16_t)(w4[e] & 0xFFFF) + (w4[e] >> 16);
+          }
+          S.bsum[k] = t;
+        }
+      }
+      csync();
+    }
+    if (tid == 0) tstamp(P, l, 1, gtime());
+
+    // ---- A: u = P1 xh; each row shared by one warp group
+    const int nA = R.kA1 - R.kA0;
+    {
+      constexpr int CCP = WTraits<PT>::CHUNK_COLS;
+      const int nch = d / CCP;
+      const uint32_t ua0 = uc;
+      for (int a = 0; a < nA; ++a, ++uc) {
+        if ((int)(uc % (uint32_t)GW) != grp) continue;
+        const int st = (int)(uc % (uint32_t)pl.ns);
+        if (!ready(st)) continue;
+        const char* row = stage(st);
+        float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+        int c = gtid;
+        for (; c + 3 * GT < nch; c += 4 * GT) {
+          v0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.xf, c, d);
+          v1 += chunk_dot<PT>(lds128(row + (size_t)(c + GT) * 16), S.xf, c + GT, d);
+          v2 += chunk_dot<PT>(lds128(row + (size_t)(c + 2 * GT) * 16), S.xf, c + 2 * GT, d);
+          v3 += chunk_dot<PT>(lds128(row + (size_t)(c + 3 * GT) * 16), S.xf, c + 3 * GT, d);
+        }
+        for (; c < nch; c += GT) v0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.xf, c, d);
+        release(st, WPG);
+        float v = warp_sum((v0 + v1) + (v2 + v3));
+        if (lane == 0) S.redA[MAXA + a * NCW + wg] = v;
+      }
+      csync();
+      for (int a = tid; a < nA; a += NCT) {
+        const int wpg = NCW / (int)(pl.gw);
+        float v = 0.f;
+        for (int w = 0; w < wpg; ++w) v += S.redA[MAXA + a * NCW + w];
+        __stcg(P.u + R.kA0 + a, v);
+      }
+      (void)ua0;
+    }
+    if (tid == 0) tstamp(P, l, 2, gtime());
+    gsync_arrive();  // 1: u complete
+    // biases used later in this layer: their load latency overlaps the barrier
+    for (int k = tid; k < (R.wB1 - R.wB0) * 32; k += NCT) {
+      const int j = 32 * R.wB0 + k;
+      S.pbs[k] = (L.pbias && j < pl.F) ? L.pbias[j] : 0.f;
+    }
+    for (int i = tid; i < R.nh; i += NCT) S.hbs[i] = L.bias ? L.bias[item_neuron(i, R, pl, S)] : 0.f;
+    gsync_wait();
+    if (tid == 0) tstamp(P, l, 3, gtime());
+
+    // ---- B: logits of the CTA's mask words; the group's warps take the rows
+    for (int k = tid; k < pl.r; k += NCT) S.us[vpos<PT>(k, pl.r)] = __ldcg(P.u + k);
+    for (int k = tid; k < R.wB1 - R.wB0; k += NCT) S.bw[k] = 0u;
+    csync();
+    {
+      constexpr int CCP = WTraits<PT>::CHUNK_COLS;
+      const int nch = pl.r / CCP;
+      for (int w = R.wB0; w < R.wB1; ++w) {
+        for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F; ja += pl.G, ++uc) {
+          if ((int)(uc % (uint32_t)GW) != grp) continue;
+          const int st = (int)(uc % (uint32_t)pl.ns);
+          if (!ready(st)) continue;
+          const char* buf = stage(st);
+          const int jb = min(ja + pl.G, pl.F);
+          uint32_t bits = 0u;
+          for (int j = ja + wg; j < jb; j += WPG) {
+            const char* row = buf + (size_t)(j - ja) * pl.p2_row;
+            float z0 = 0.f, z1 = 0.f;
+            int c = lane;
+            for (; c + 32 < nch; c += 64) {
+              z0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.us, c, pl.r);
+              z1 += chunk_dot<PT>(lds128(row + (size_t)(c + 32) * 16), S.us, c + 32, pl.r);
+            }
+            if (c < nch) z0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.us, c, pl.r);
+            const float z = warp_sum(z0 + z1) + S.pbs[j - 32 * R.wB0];
+            if (j >= pl.H && z > P.theta) bits |= 1u << (j & 31);
+          }
+          release(st, WPG);
+          if (lane == 0 && bits) atomicOr(&S.bw[w - R.wB0], bits);
+        }
+      }
+    }
+    csync();
+    for (int k = tid; k < R.wB1 - R.wB0; k += NCT) {
+      const int w = R.wB0 + k;
+      uint32_t word = S.bw[k];
+      const int lo = 32 * w;
+      if (pl.H > lo) word |= (pl.H - lo >= 32) ? 0xFFFFFFFFu : ((1u << (pl.H - lo)) - 1u);
+      __stcg(mask + w, word);
+    }
+    for (int w = (int)((long long)s * R.Wlo / nS) + tid; w < (int)((long long)(s + 1) * R.Wlo / nS);
+         w += NCT)
+      __stcg(mask + w, 0xFFFFFFFFu);
+    if (tid == 0) tstamp(P, l, 4, gtime());
+    gsync_arrive();  // 2: mask complete (waited for after the hot items)
+
+    // ---- C: items (hot, then cold); each unit shared by one warp group,
+    // per-warp partial sums combined in fixed order per group of GRP items
+    int fin = 0;  // next item to finalise
+    auto finalise = [&](int upto) {  // items [fin, upto)
+      csync();
+      const int i = fin + tid;
+      if (i < upto) {
+        const float* r = S.redC + ((i / GRP) & 1) * (GRP * NCW * 2) + (i % GRP) * NCW * 2;
+        float a = 0.f, b = 0.f;
+        for (int w = 0; w < WPG; ++w) {
+          a += r[2 * w];
+          b += r[2 * w + 1];
+        }
+        if constexpr (WT == PI_Q4_0) {
+          a *= *S.xscale;
+          b *= *S.xscale;
+        }
+        const float g = a + S.hbs[i];
+        float h = g > 0.f ? g : 0.f;
+        if constexpr (two) h *= b;
+        S.hval[i] = h;
+        __threadfence_block();
+        S.flag[i] = tag | (h != 0.f ? 2 : 1);
+      }
+      fin = upto;
+    };
+    // one unit: items i0 .. i0+n-1, record r of the stage for item i0 + r
+    auto unit_items = [&](int i0, int n) {
+      if ((int)(uc % (uint32_t)GW) == grp) {
+        const int st = (int)(uc % (uint32_t)pl.ns);
+        const bool ok = ready(st);
+        float a[8], b[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
+        if (ok) {
+          const char* base = stage(st);
+          if constexpr (WT == PI_Q4_0) {
+            const int4* xb = reinterpret_cast<const int4*>(S.xi);
+            for (int k = gtid; k < nb; k += GT) {
+              const int4 x0 = xb[k], x1 = xb[nb + k], x2 = xb[2 * nb + k], x3 = xb[3 * nb + k];
+              const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                  x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+              const int bs = -8 * S.bsum[k];
+#pragma unroll
+              for (int r = 0; r < 8; ++r) {
+                if (r >= n) break;
+                const char* buf = base + (size_t)r * pl.item_bytes;
+                const uint4 cf = lds128(buf + (size_t)k * 16);
+                const float sf = h2f(reinterpret_cast<const uint16_t*>(buf + pl.o_first_s)[k]);
+                a[r] = fmaf((float)q4_block_dot(cf, xw, bs), sf, a[r]);
+                if constexpr (two) {
+                  const uint4 cs = lds128(buf + pl.o_second + (size_t)k * 16);
+                  const float sg = h2f(reinterpret_cast<const uint16_t*>(buf + pl.o_second_s)[k]);
+                  b[r] = fmaf((float)q4_block_dot(cs, xw, bs), sg, b[r]);
+                }
+              }
+            }
+          } else {
+            constexpr int CCW = WTraits<WT>::CHUNK_COLS;
+            const int nch = d / CCW;
+            for (int c = gtid; c < nch; c += GT) {
+#pragma unroll
+              for (int r = 0; r < 8; ++r) {
+                if (r >= n) break;
+                const char* buf = base + (size_t)r * pl.item_bytes;
+                a[r] += chunk_dot<WT>(lds128(buf + (size_t)c * 16), S.xf, c, d);
+                if constexpr (two)
+                  b[r] += chunk_dot<WT>(lds128(buf + pl.o_second + (size_t)c * 16), S.xf, c, d);
+              }
+            }
+          }
+          release(st, WPG);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int r = 0; r < 8; ++r) {
+            if (r >= n) break;
+            a[r] += __shfl_xor_sync(0xffffffffu, a[r], o);
+            if constexpr (two) b[r] += __shfl_xor_sync(0xffffffffu, b[r], o);
+          }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          if (r >= n) break;
+          const float av = a[r];
+          const float bv = two ? b[r] : 0.f;
+          if (lane == 0) {
+            const int i = i0 + r;
+            float* rr = S.redC + ((i / GRP) & 1) * (GRP * NCW * 2) + (i % GRP) * NCW * 2 + 2 * wg;
+            rr[0] = av;
+            rr[1] = bv;
+          }
+        }
+      }
+      ++uc;
+      // finalise every group of GRP items completed by this unit
+      const int i1 = i0 + n;
+      if (i1 / GRP != i0 / GRP) finalise((i1 / GRP) * GRP);
+    };
+    for (int gi = 0; gi < R.ngh; ++gi) {
+      const int j0 = hot_group_first(gi, pl);
+      unit_items(gi * pl.hp, min(pl.hp, pl.H - j0));
+    }
+    if (fin < R.nh) finalise(R.nh);
+    if (tid == 0) tstamp(P, l, 5, gtime());
+
+    // ---- compaction (every CTA, after barrier 2): its share of the list
+    gsync_wait();
+    if (tid == 0) tstamp(P, l, 6, gtime());
+    {
+      const int Wc = R.W - R.Wlo;
+      const int per = (Wc + NCT - 1) / NCT;
+      const int wa = R.Wlo + tid * per, wb = min(R.Wlo + (tid + 1) * per, R.W);
+      int cnt = 0;
+      for (int w = wa; w < wb; ++w) {
+        uint32_t m = __ldcg(mask + w);
+        const int lo = 32 * w;
+        if (pl.H > lo) m &= (pl.H - lo >= 32) ? 0u : (~0u << (pl.H - lo));
+        S.mw[w - R.Wlo] = m;
+        cnt += __popc(m);
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      if (lane == 31) S.scan[warp] = incl;
+      csync();
+      int wpre = 0, total = 0;
+#pragma unroll
+      for (int w = 0; w < NCW; ++w) {
+        const int v = S.scan[w];
+        if (w < warp) wpre += v;
+        total += v;
+      }
+      int p = wpre + incl - cnt;  // list position of this thread's first neuron
+      for (int w = wa; w < wb; ++w) {
+        uint32_t m = S.mw[w - R.Wlo];
+        while (m) {
+          const int bit = __ffs(m) - 1;
+          m &= m - 1u;
+          if (p % nS == s) {
+            const int j = 32 * w + bit;
+            S.cold[p / nS] = j;
+            S.hbs[R.nh + p / nS] = L.bias ? L.bias[j] : 0.f;
+          }
+          ++p;
+        }
+      }
+      if (tid == 0) {
+        *S.nc = total > s ? (total - s + nS - 1) / nS : 0;
+        if (s == 0) __stcg(P.count, total);
+      }
+      csync();
+      if (lane == 0) mbar_arrive(S.listbar, 1u);
+    }
+    const int nc = *S.nc;
+    for (int i = R.nh; i < R.nh + nc; ++i) unit_items(i, 1);
+    if (fin < R.nh + nc) finalise(R.nh + nc);
+    csync();
+    if (tid == 0) tstamp(P, l, 7, gtime());
+
+    // ---- D: down rows of items with h != 0; each unit (a run of adjacent
+    // neurons' rows) shared by one of GD warp groups, each group covering
+    // every column with its own accumulators
+    const int ni = R.nh + nc;
+    if (warp == 0) {
+      int base = 0;
+      for (int i0 = 0; i0 < ni; i0 += 32) {
+        const int i = i0 + lane;
+        const bool nz = i < ni && S.hval[i] != 0.f;
+        const uint32_t bal = __ballot_sync(0xffffffffu, nz);
+        if (nz) S.dlist[base + __popc(bal & ((1u << lane) - 1u))] = i;
+        base += __popc(bal);
+      }
+      __syncwarp();
+      if (lane == 0) {
+        int nr = 0, jp = -1, len = 0;
+        for (int q = 0; q < base; ++q) {
+          const int j = item_neuron(S.dlist[q], R, pl, S);
+          if (len > 0 && run_extends(jp, j, len, pl)) {
+            ++len;
+          } else {
+            if (len > 0) S.runs[2 * nr++ + 1] = len;
+            S.runs[2 * nr] = q;
+            len = 1;
+          }
+          jp = j;
+        }
+        if (len > 0) S.runs[2 * nr++ + 1] = len;
+        S.scan[NCW] = base;
+        S.scan[NCW + 1] = nr;
+      }
+    }
+    csync();
+    const int nd = S.scan[NCW], nruns = S.scan[NCW + 1];
+    {
+      constexpr int CC = WTraits<WT>::CHUNK_COLS;
+      constexpr int MAXK = (CC == 32) ? 1 : 48 / CC;  // chunks per thread of a D group
+      const int nch = d / CC;
+      float acc[MAXK][CC];
+#pragma unroll
+      for (int k = 0; k < MAXK; ++k)
+#pragma unroll
+        for (int e = 0; e < CC; ++e) acc[k][e] = 0.f;
+      for (int q = 0; q < nruns; ++q, ++uc) {
+        if ((int)(uc % (uint32_t)GD) != dgrp) continue;
+        const int st = (int)(uc % (uint32_t)pl.ns);
+        if (!ready(st)) continue;
+        const int q0 = S.runs[2 * q], len = S.runs[2 * q + 1];
+        for (int rr = 0; rr < len; ++rr) {
+          const char* row = stage(st) + (size_t)rr * pl.down_bytes;
+          const float hv = S.hval[S.dlist[q0 + rr]];
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int c = dtid + k * DT;
+            if (c >= nch) break;
+            const uint4 v = lds128(row + (size_t)c * 16);
+            if constexpr (WT == PI_Q4_0) {
+              const float hs = hv * h2f(reinterpret_cast<const uint16_t*>(row + pl.o_down_s)[c]);
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const uint32_t byte = (wv[e >> 2] >> (8 * (e & 3))) & 0xFFu;
+                acc[k][e] = fmaf(hs, q4_centered(byte & 0xFu), acc[k][e]);
+                acc[k][e + 16] = fmaf(hs, q4_centered(byte >> 4), acc[k][e + 16]);
+              }
+            } else if constexpr (WT == PI_F16) {
+              float f[8];
+              f16x8_to_f32(v, f);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(hv, f[e], acc[k][e]);
+            } else {
+              acc[k][0] = fmaf(hv, __uint_as_float(v.x), acc[k][0]);
+              acc[k][1] = fmaf(hv, __uint_as_float(v.y), acc[k][1]);
+              acc[k][2] = fmaf(hv, __uint_as_float(v.z), acc[k][2]);
+              acc[k][3] = fmaf(hv, __uint_as_float(v.w), acc[k][3]);
+            }
+          }
+        }
+        release(st, WPD);
+      }
+      // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
+      float* part = P.part + ((size_t)s * GD + dgrp) * d;
+#pragma unroll
+      for (int k = 0; k < MAXK; ++k) {
+        const int c = dtid + k * DT;
+        if (c >= nch) break;
+#pragma unroll
+        for (int e = 0; e < CC; e += 4)
+          __stcg(reinterpret_cast<float4*>(part + c * CC + e),
+                 make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]));
+      }
+    }
+    if (tid == 0) {
+      atomicAdd(&hdr->rows_listed, (unsigned long long)ni);
+      atomicAdd(&hdr->rows_down, (unsigned long long)nd);
+      tstamp(P, l, 8, gtime());
+    }
+    gsync_arrive();  // 3: partials complete
+    gsync_wait();
+    if (tid == 0) tstamp(P, l, 9, gtime());
+
+    // ---- E: reduce this CTA's float4 column slice over the nS * GD partial
+    // rows in a fixed order (rows in interleaved groups, then the groups in
+    // order), residual add.
+    {
+      const int q4n = d / 4, nP = nS * GD;
+      const int cq0 = (int)((long long)s * q4n / nS), cq1 = (int)((long long)(s + 1) * q4n / nS);
+      const int nq = cq1 - cq0;  // <= 32
+      const int g = nq > 0 ? NCT / nq : 0;
+      const float4* pp = reinterpret_cast<const float4*>(P.part);
+      if (nq > 0 && tid < nq * g) {
+        const int q = tid % nq, gi = tid / nq;
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp0 = gi; sp0 < nP; sp0 += 8 * g) {
+          float4 v[8];
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int sp = sp0 + m * g;
+            v[m] = sp < nP ? __ldcg(pp + (size_t)sp * q4n + cq0 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int m = 0; m < 8; ++m) t = f4add(t, v[m]);
+        }
+        S.redE[gi * nq + q] = t;
+      }
+      csync();
+      if (tid < nq) {
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int gi = 0; gi < g; ++gi) y = f4add(y, S.redE[gi * nq + tid]);
+        float4* x4 = reinterpret_cast<float4*>(P.x) + cq0 + tid;
+        __stcg(x4, f4add(__ldcg(x4), y));
+      }
+    }
+    csync();
+    if (tid == 0) tstamp(P, l, 10, gtime());
+    if (l + 1 < P.n_layers) {
+      gsync_arrive();  // 4: x complete
+      gsync_wait();
+    }
+    if (tid == 0) tstamp(P, l, 11, gtime());
+  }
+}
+
+template <int WT, int ACT, int PT>
+__global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ StackParams P) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const Smem S = carve(smem, P.pl);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < P.pl.ns; ++i) {
+      mbar_init(&S.full[i], 1u);
+      mbar_init(&S.empty[i], (uint32_t)NCW);
+    }
+    mbar_init(S.listbar, (uint32_t)NCW);
+    *S.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  for (int i = threadIdx.x; i < P.pl.maxi; i += NTHR) S.flag[i] = 0;
+  __syncthreads();
+  if (threadIdx.x >= NCT) {
+    const int p = (threadIdx.x - NCT) >> 5;
+    if ((threadIdx.x & 31) == 0 && p < P.pl.np) producer<WT, ACT, PT>(P, S, p);
+    return;
+  }
+  consumers<WT, ACT, PT>(P, S);
+}
+
+// ------------------------------------------------------------------- host
+
+int smem_optin() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) v = 0;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+uint32_t up16(uint32_t v) { return (v + 15u) & ~15u; }
+uint32_t up128(uint32_t v) { return (v + 127u) & ~127u; }
+
+// Whether every layer stores each neuron's up-projection record (and each
+// down row with its scales) contiguously, with the record as row stride.
+void packing(const pi_layer* layers, int n, uint32_t rowb, uint32_t scb, int* up, int* down) {
+  *up = *down = 1;
+  for (int l = 0; l < n; ++l) {
+    const pi_layer& L = layers[l];
+    const bool two = L.act == PI_REGLU, q4 = L.w_dtype == PI_Q4_0;
+    const uintptr_t rec = (uintptr_t)rowb + scb;
+    const uintptr_t first = (uintptr_t)(two ? L.w_gate : L.w_up);
+    const uintptr_t first_s = (uintptr_t)(two ? L.w_gate_scales : L.w_up_scales);
+    const int64_t item = (two ? 2 : 1) * (int64_t)rec;
+    bool ok = code_stride(L.w_dtype, L.d_model, L.w_row_stride) == item;
+    if (q4) ok = ok && first_s == first + rowb;
+    if (two) {
+      ok = ok && (uintptr_t)L.w_up == first + rec;
+      if (q4) ok = ok && (uintptr_t)L.w_up_scales == (uintptr_t)L.w_up + rowb;
+    }
+    if (!ok) *up = 0;
+    bool dk = code_stride(L.w_dtype, L.d_model, L.w_down_row_stride) == (int64_t)rec;
+    if (q4) dk = dk && (uintptr_t)L.w_down_t_scales == (uintptr_t)L.w_down_t + rowb;
+    if (!dk) *down = 0;
+  }
+}
+
+bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
+  const pi_layer& L0 = layers[0];
+  Plan pl{};
+  pl.d = L0.d_model;
+  pl.F = L0.d_ff;
+  pl.r = L0.rank;
+  pl.H = L0.hot;
+  pl.nsms = nsms;
+  const int d = pl.d, F = pl.F, r = pl.r, H = pl.H;
+  const bool q4 = L0.w_dtype == PI_Q4_0, two = L0.act == PI_REGLU;
+  const uint32_t pb = L0.p_dtype == PI_F32 ? 4u : 2u;
+  pl.rowb = (uint32_t)row_bytes(L0.w_dtype, d);
+  pl.scb = q4 ? (uint32_t)(d / 32) * 2u : 0u;
+  pl.p1_bytes = (uint32_t)d * pb;
+  pl.p2_row = (uint32_t)r * pb;
+  // record layout inside a stage: [first codes | first scales | second codes | second scales]
+  pl.o_first_s = pl.rowb;
+  pl.o_second = pl.rowb + pl.scb;
+  pl.o_second_s = 2 * pl.rowb + pl.scb;
+  pl.item_bytes = (two ? 2u : 1u) * (pl.rowb + pl.scb);
+  pl.o_down_s = pl.rowb;
+  pl.down_bytes = pl.rowb + pl.scb;
+  packing(layers, n_layers, pl.rowb, pl.scb, &pl.packed_up, &pl.packed_down);
+  pl.up_stride = code_stride(L0.w_dtype, d, L0.w_row_stride);
+  pl.up_sstride = scale_stride(d, L0.w_row_stride);
+  pl.down_stride = code_stride(L0.w_dtype, d, L0.w_down_row_stride);
+  pl.down_sstride = scale_stride(d, L0.w_down_row_stride);
+  for (int l = 1; l < n_layers; ++l)
+    if (layers[l].w_row_stride != L0.w_row_stride || layers[l].w_down_row_stride != L0.w_down_row_stride)
+      return false;
+  // adjacent hot records per unit (packed): units of at least 16 KB
+  pl.hp = 1;
+  if (pl.packed_up)
+    while (pl.hp < 8 && (uint32_t)pl.hp * pl.item_bytes < 16384u) ++pl.hp;
+  uint32_t sb = pl.p1_bytes;
+  sb = sb > (uint32_t)pl.hp * pl.item_bytes ? sb : (uint32_t)pl.hp * pl.item_bytes;
+  sb = sb > pl.down_bytes ? sb : pl.down_bytes;
+  sb = sb > pl.p2_row ? sb : pl.p2_row;
+  sb = up128(sb);
+  pl.sb = sb;
+  pl.dr = pl.packed_down ? (int)(sb / pl.down_bytes) : 1;
+  if (pl.dr < 1) pl.dr = 1;
+  int G = 32;
+  while (G > 1 && (uint32_t)G * pl.p2_row > sb) G >>= 1;
+  pl.G = G;
+  const int W = (F + 31) / 32, Wlo = H / 32, Wc = W - Wlo;
+  pl.maxc = (F - H + nsms - 1) / nsms + 1;
+  pl.maxi = (H + nsms - 1) / nsms + pl.hp + pl.maxc + 1;
+  const int bw = Wc / nsms + 2;
+  uint32_t o = 8 * (2 * NSMAX + 1);  // mbarriers
+  o = up16(o);
+  pl.o_misc = o;       o = up16(o + 16);
+  pl.o_xf = o;         o = up16(o + 4u * d);
+  pl.o_xi = o;         o = up16(o + (q4 ? 2u * d : 0u));
+  pl.o_bsum = o;       o = up16(o + (q4 ? 4u * (d / 32) : 0u));
+  pl.o_u = o;          o = up16(o + 4u * r);
+  pl.o_bw = o;         o = up16(o + 4u * bw);
+  pl.o_mw = o;         o = up16(o + 4u * Wc);
+  pl.o_scan = o;       o = up16(o + 4u * (NCW + 4));
+  pl.o_cold = o;       o = up16(o + 4u * pl.maxc);
+  pl.o_hval = o;       o = up16(o + 4u * pl.maxi);
+  pl.o_flag = o;       o = up16(o + 4u * pl.maxi);
+  pl.o_dlist = o;      o = up16(o + 4u * pl.maxi);
+  pl.o_runs = o;       o = up16(o + 8u * pl.maxi);
+  pl.o_pbs = o;        o = up16(o + 4u * 32u * bw);
+  pl.o_hbs = o;        o = up16(o + 4u * pl.maxi);
+  pl.o_redA = o;       o = up16(o + 4u * (MAXA + MAXA * NCW));
+  pl.o_redC = o;       o = up16(o + 4u * (2 * GRP * NCW * 2));
+  pl.o_redE = o;       o = up16(o + 16u * NCT);
+  pl.o_ring = up128(o);
+  const int avail = smem_optin() - (int)pl.o_ring;
+  if (avail <= 0) return false;
+  int ns = avail / (int)sb;
+  if (ns > NSMAX) ns = NSMAX;
+  // producer warps own every np-th stage: np must divide ns
+  if (ns >= 8) {
+    pl.np = 4;
+    ns -= ns % 4;
+  } else if (ns >= 4) {
+    pl.np = 2;
+    ns -= ns % 2;
+  } else if (ns >= 3) {
+    pl.np = 1;
+  } else {
+    return false;
+  }
+  pl.ns = ns;
+  // consumer groups must divide the ring depth (a stage is always consumed
+  // by the same group); the down phase also needs every column to fit one
+  // group's accumulators (64 floats per thread)
+  pl.gw = ns % 4 == 0 ? 4 : (ns % 2 == 0 ? 2 : 1);
+  {
+    // chunks per consumer thread in the down phase must fit its accumulators
+    // (one Q4_0 block, or 48 fp16 / fp32 values)
+    const int cc = L0.w_dtype == PI_Q4_0 ? 32 : (L0.w_dtype == PI_F16 ? 8 : 4);
+    const int cap = cc == 32 ? 1 : 48 / cc;
+    const int per2 = (d / cc + NCT / 2 - 1) / (NCT / 2);
+    const int per1 = (d / cc + NCT - 1) / NCT;
+    if (ns % 2 == 0 && per2 <= cap) pl.gd = 2;
+    else if (per1 <= cap) pl.gd = 1;
+    else return false;
+  }
+  pl.total = pl.o_ring + (uint32_t)ns * sb;
+  *out = pl;
+  return true;
+}
+
+bool fused_disabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("PI_DISABLE_FUSED");
+    v = (e && e[0] && e[0] != '0') ? 1 : 0;
+  }
+  return v == 1;
+}
+
+template <int WT, int ACT, int PT>
+cudaError_t launch_t(const StackParams& P, cudaStream_t s) {
+  auto kern = k_stack1<WT, ACT, PT>;
+  cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(kern), P.pl.total);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(P.pl.nsms);
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = P.pl.total;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, P);
+}
+
+cudaError_t launch_any(const StackParams& P, int wt, int act, int pt, cudaStream_t s) {
+  // weight / predictor dtype pairs that share one staged-vector layout
+  if (wt == PI_Q4_0) {
+    if (act == PI_REGLU)
+      return pt == PI_F32 ? launch_t<PI_Q4_0, PI_REGLU, PI_F32>(P, s)
+                          : launch_t<PI_Q4_0, PI_REGLU, PI_F16>(P, s);
+    return pt == PI_F32 ? launch_t<PI_Q4_0, PI_RELU, PI_F32>(P, s)
+                        : launch_t<PI_Q4_0, PI_RELU, PI_F16>(P, s);
+  }
+  if (wt == PI_F16)
+    return act == PI_REGLU ? launch_t<PI_F16, PI_REGLU, PI_F16>(P, s)
+                           : launch_t<PI_F16, PI_RELU, PI_F16>(P, s);
+  return act == PI_REGLU ? launch_t<PI_F32, PI_REGLU, PI_F32>(P, s)
+                         : launch_t<PI_F32, PI_RELU, PI_F32>(P, s);
+}
+
+}  // namespace
+
+int stack1_chunk() { return MAXL; }
+int stack1_unit_trace_len() { return UTR; }
+
+bool stack1_supported(const pi_layer* layers, int n_layers, int batch) {
+  if (batch != 1 || n_layers < 1 || fused_disabled()) return false;
+  const pi_layer& a = layers[0];
+  for (int l = 1; l < n_layers; ++l) {
+    const pi_layer& b = layers[l];
+    if (b.d_model != a.d_model || b.d_ff != a.d_ff || b.rank != a.rank || b.hot != a.hot ||
+        b.act != a.act || b.w_dtype != a.w_dtype || b.p_dtype != a.p_dtype)
+      return false;
+  }
+  // fp16 weights go with an fp16 predictor, fp32 with fp32 (one staged layout)
+  if ((a.w_dtype == PI_F16 && a.p_dtype != PI_F16) || (a.w_dtype == PI_F32 && a.p_dtype != PI_F32))
+    return false;
+  if (a.d_model > 12288 || a.rank > 2048) return false;
+  if (a.w_dtype == PI_Q4_0) {
+    if (a.d_model % 256) return false;
+    for (int l = 0; l < n_layers; ++l) {
+      const pi_layer& b = layers[l];
+      if (((uintptr_t)b.w_up_scales | (uintptr_t)b.w_down_t_scales |
+           (uintptr_t)(b.act == PI_REGLU ? b.w_gate_scales : b.w_up_scales)) & 15u)
+        return false;
+    }
+  }
+  const int nsms = device_sms();
+  if (nsms < 128) return false;                                // slice bounds below
+  if ((a.d_model / 4 + nsms - 1) / nsms > 32) return false;    // reduce slice <= 32 float4
+  if ((a.rank + nsms - 1) / nsms > MAXA) return false;         // P1 rows per CTA
+  Plan pl;
+  return make_plan(layers, n_layers, nsms, &pl);
+}
+
+cudaError_t launch_stack1(const pi_layer* layers, int n_layers, float* x, uint32_t* mask_trace,
+                          void* ws, const WsLayout& lay, float theta, cudaStream_t s,
+                          unsigned long long* trace, unsigned long long* utrace) {
+  const int nsms = device_sms();
+  if (n_layers < 1 || n_layers > MAXL) return cudaErrorInvalidValue;
+  StackParams P;
+  memset(&P, 0, sizeof P);
+  if (!make_plan(layers, n_layers, nsms, &P.pl)) return cudaErrorInvalidConfiguration;
+  const pi_layer& a = layers[0];
+  const int words = (a.d_ff + 31) / 32;
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  P.theta = theta;
+  P.x = x;
+  P.u = reinterpret_cast<float*>((char*)ws + lay.u);
+  P.part = reinterpret_cast<float*>((char*)ws + lay.part);
+  P.count = reinterpret_cast<int32_t*>((char*)ws + lay.count);
+  P.hdr = hdr;
+  P.trace = trace;
+  P.utrace = utrace;
+  P.n_layers = n_layers;
+  if (mask_trace) {
+    P.mask = mask_trace;
+    P.mask_stride = words;
+  } else {
+    P.mask = reinterpret_cast<uint32_t*>((char*)ws + lay.mask);
+    P.mask_stride = 0;
+  }
+  for (int i = 0; i < n_layers; ++i) {
+    const pi_layer& L = layers[i];
+    const bool two = L.act == PI_REGLU;
+    LayerPtrs& p = P.L[i];
+    p.first = (const char*)(two ? L.w_gate : L.w_up);
+    p.first_scales = (const char*)(two ? L.w_gate_scales : L.w_up_scales);
+    p.second = (const char*)(two ? L.w_up : nullptr);
+    p.second_scales = (const char*)(two ? L.w_up_scales : nullptr);
+    p.down = (const char*)L.w_down_t;
+    p.down_scales = (const char*)L.w_down_t_scales;
+    p.bias = L.bias;
+    p.p1 = (const char*)L.p1;
+    p.p2 = (const char*)L.p2;
+    p.pbias = L.p_bias;
+  }
+  cudaError_t e = cudaMemsetAsync(hdr->counters, 0, 2 * sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  return launch_any(P, a.w_dtype, a.act, a.p_dtype, s);
+}
+
+}  // namespace pi

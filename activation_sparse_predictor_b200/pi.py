@@ -39,6 +39,7 @@ class pi_layer(ctypes.Structure):
         ("w_gate_scales", ctypes.c_void_p), ("w_up_scales", ctypes.c_void_p),
         ("w_down_t_scales", ctypes.c_void_p), ("bias", ctypes.c_void_p),
         ("p1", ctypes.c_void_p), ("p2", ctypes.c_void_p), ("p_bias", ctypes.c_void_p),
+        ("w_row_stride", ctypes.c_int64), ("w_down_row_stride", ctypes.c_int64),
     ]
 
 
@@ -60,6 +61,8 @@ def _load():
                                        ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
         "pi_kind_name": (ctypes.c_char_p, [i32]),
         "pi_read_counters": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_uint64)]),
+        "pi_ffn_stack_timeline": (i32, [L, i32, vp, f32, vp, sz, vp, vp, vp]),
+        "pi_device_sms": (i32, []),
         "pi_status_string": (ctypes.c_char_p, [i32]),
         "pi_last_error": (ctypes.c_char_p, []),
         "pi_version": (i32, []),
@@ -108,7 +111,8 @@ class Layer:
     `tensors` keys: w_gate (ReGLU), w_up, w_down_t (tensors, or (codes,
     scales) pairs for q4_0), bias, p1, p2, p_bias."""
 
-    def __init__(self, *, d_model, d_ff, rank, hot, act, w_dtype, p_dtype, tensors: dict):
+    def __init__(self, *, d_model, d_ff, rank, hot, act, w_dtype, p_dtype, tensors: dict,
+                 w_row_stride: int = 0, w_down_row_stride: int = 0):
         self.tensors = tensors
         self.d_model, self.d_ff, self.rank, self.hot = d_model, d_ff, rank, hot
         self.act, self.w_dtype, self.p_dtype = act, w_dtype, p_dtype
@@ -126,16 +130,65 @@ class Layer:
         dn, ds = w("w_down_t")
         self.c = pi_layer(d_model, d_ff, rank, hot, ACTS[act], DTYPES[w_dtype], DTYPES[p_dtype],
                           g, u, dn, gs, us, ds, _ptr(tensors.get("bias")), _ptr(tensors["p1"]),
-                          _ptr(tensors["p2"]), _ptr(tensors.get("p_bias")))
+                          _ptr(tensors["p2"]), _ptr(tensors.get("p_bias")), w_row_stride,
+                          w_down_row_stride)
 
     @classmethod
-    def from_workload(cls, w, tensors: dict) -> "Layer":
+    def from_workload(cls, w, tensors: dict, **strides) -> "Layer":
         return cls(d_model=w.d_model, d_ff=w.d_ff, rank=w.rank, hot=w.hot, act=w.act,
-                   w_dtype=w.w_dtype, p_dtype=w.p_dtype, tensors=tensors)
+                   w_dtype=w.w_dtype, p_dtype=w.p_dtype, tensors=tensors, **strides)
+
+    @classmethod
+    def packed(cls, w, tensors: dict) -> "Layer":
+        """A layer whose neuron records are packed (see pack_records): each
+        neuron's gate/up weights, and each down row with its scales, are one
+        contiguous span.  Returns the Layer; the packed buffers live in it."""
+        packed, strides = pack_records(w, tensors)
+        return cls.from_workload(w, packed, **strides)
 
     @property
     def words(self) -> int:
         return (self.d_ff + 31) // 32
+
+
+def pack_records(w, tensors: dict):
+    """Rearranges a layer's FFN weights (dense matrices as produced by the
+    input generator) into per-neuron records on the same device:
+      up record j  : [gate row j | up row j]  (ReGLU) or [up row j] (ReLU),
+                     Q4_0 rows as [codes (d/2 B) | scales (d/16 B)];
+      down record j: [w_down_t row j] (Q4_0: codes | scales).
+    Returns (tensor dict with views into the packed buffers, strides)."""
+    import torch
+    def q4rows(pair):
+        codes, scales = pair
+        F = codes.shape[0]
+        return torch.cat([codes.reshape(F, -1), scales.contiguous().view(torch.uint8).reshape(F, -1)], 1)
+    def pad16(b):  # each record a multiple of 16 bytes (16-byte aligned rows)
+        extra = (-b.shape[1]) % 16
+        return b if extra == 0 else torch.cat([b, b.new_zeros((b.shape[0], extra))], 1)
+    def asbytes(t):
+        b = q4rows(t) if isinstance(t, tuple) else t.contiguous().view(torch.uint8).reshape(t.shape[0], -1)
+        return pad16(b)
+    F = tensors["w_up"][0].shape[0] if isinstance(tensors["w_up"], tuple) else tensors["w_up"].shape[0]
+    first = [tensors["w_gate"], tensors["w_up"]] if w.act == "reglu" else [tensors["w_up"]]
+    up = torch.cat([asbytes(t) for t in first], 1).contiguous()
+    down = asbytes(tensors["w_down_t"]).contiguous()
+    out = {k: v for k, v in tensors.items() if k not in ("w_gate", "w_up", "w_down_t")}
+    rb = {"f32": 4 * w.d_model, "f16": 2 * w.d_model, "q4_0": w.d_model // 2}[w.w_dtype]
+    sc = w.d_model // 16 if w.w_dtype == "q4_0" else 0
+    rec = rb + sc + (-(rb + sc)) % 16
+    def view(buf, off, n):
+        return buf[:, off:off + n]
+    names = ["w_gate", "w_up"] if w.act == "reglu" else ["w_up"]
+    for i, name in enumerate(names):
+        base = i * rec
+        if w.w_dtype == "q4_0":
+            out[name] = (view(up, base, rb), view(up, base + rb, sc))
+        else:
+            out[name] = view(up, base, rb)
+    out["w_down_t"] = (view(down, 0, rb), view(down, rb, sc)) if w.w_dtype == "q4_0" else view(down, 0, rb)
+    out["_packed_up"], out["_packed_down"] = up, down
+    return out, {"w_row_stride": up.shape[1], "w_down_row_stride": down.shape[1]}
 
 
 def _layer_array(layers):
@@ -220,7 +273,7 @@ def pi_ffn_stack(layers, x, tau: float, mode: int, mask_trace=None, ws=None, str
     return x
 
 
-PI_KINDS = 7
+PI_KINDS = 8
 
 
 def pi_ffn_stack_profile(layers, x, tau: float, mode: int, mask_trace=None, ws=None,
@@ -244,6 +297,25 @@ def pi_read_counters(ws, clear: bool = False, stream=None):
     out = (ctypes.c_uint64 * 2)()
     _check(_lib.pi_read_counters(_ptr(ws), _stream(stream), int(clear), out))
     return int(out[0]), int(out[1])
+
+
+def pi_ffn_stack_timeline(layers, x, tau: float, ws=None, stream=None, _arr=None):
+    """Runs the stack (batch 1, persistent kernel) and returns (timeline
+    [n_layers][SMs][16], unit timeline [n_layers][512][4]) as device int64
+    tensors (see include/pi.h)."""
+    import torch
+    if ws is None:
+        ws = workspace(layers, 1, x.device, stream)
+    arr = _arr if _arr is not None else _layer_array(layers)
+    tl = torch.zeros((len(layers), pi_device_sms(), 16), dtype=torch.int64, device=x.device)
+    ut = torch.zeros((len(layers), 512, 4), dtype=torch.int64, device=x.device)
+    _check(_lib.pi_ffn_stack_timeline(arr, len(layers), _ptr(x), tau, _ptr(ws), ws.numel(),
+                                      _stream(stream), _ptr(tl), _ptr(ut)))
+    return tl, ut
+
+
+def pi_device_sms() -> int:
+    return int(_lib.pi_device_sms())
 
 
 def pi_kind_name(kind: int) -> str:

@@ -286,9 +286,10 @@ def run_pi(args, world, rank, local):
     layers = []
     for l in range(w.n_layers):
         t = synth.layer_device(w, l, dev)
-        layers.append(pi.Layer.from_workload(
+        layers.append(pi.Layer.packed(
             w, {k: t[k] for k in ("w_gate", "w_up", "w_down_t", "bias", "p1", "p2", "p_bias")
                 if k in t}))
+        del t
     arr = pi.layer_array(layers)
     K, W = args.steps, max(3, args.warmup)
     xs = torch.stack([synth.x_device(w, rank * 1_000_003 + s, B, dev) for s in range(K + W)])
@@ -345,6 +346,8 @@ def run_pi(args, world, rank, local):
     prof = pi.pi_ffn_stack_profile(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
     pr_listed, pr_down = pi.pi_read_counters(ws, clear=True, stream=stream)
     pby = layer_algorithmic_bytes(w, pr_listed, pr_down, w.n_layers)
+    pby["fused_stack"] = sum(pby.values())  # the fused kernel runs every step
+    prof = {k: v for k, v in prof.items() if v[1] > 0}
     dom = max(prof, key=lambda k: prof[k][0])
     dom_ms, dom_n = prof[dom]
     achieved = pby[dom] / dom_n / (dom_ms / dom_n / 1000.0) / 1e9

@@ -90,8 +90,16 @@ typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_m
  *  bias       : [F] fp32 on the first matrix (gate for ReGLU, up for ReLU); NULL = 0.
  *  p1         : [r][d], p2 : [F][r]; predictor logits z = p2 (p1 xh) + p_bias.
  *  p_bias     : [F] fp32; NULL = 0.
+ *  w_row_stride     : bytes from row j to row j+1 of w_gate and w_up, and (Q4_0)
+ *                     of their scale arrays; 0 = dense rows (codes d/2 bytes,
+ *                     scales d/16 bytes apart for Q4_0).  A stride lets one
+ *                     buffer hold each neuron's record [gate | up] (Q4_0:
+ *                     [gate codes | gate scales | up codes | up scales]) so the
+ *                     neuron's up-projection weights are one contiguous read.
+ *  w_down_row_stride: the same for w_down_t and its scales.
  * Alignment: every weight pointer 16-byte aligned; d % 8 (F32, F16),
- * d % 32 (Q4_0) == 0; r % 4 (F32 predictor) / r % 8 (F16 predictor) == 0. */
+ * d % 32 (Q4_0) == 0; r % 4 (F32 predictor) / r % 8 (F16 predictor) == 0;
+ * strides multiples of 16 and at least one row's codes. */
 typedef struct pi_layer {
   int32_t d_model, d_ff, rank, hot;
   int32_t act, w_dtype, p_dtype;
@@ -105,6 +113,8 @@ typedef struct pi_layer {
   const void* p1;
   const void* p2;
   const float* p_bias;
+  int64_t w_row_stride;
+  int64_t w_down_row_stride;
 } pi_layer;
 
 /* Bytes of workspace the calls below need for these layers at this batch
@@ -161,7 +171,11 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch,
  *   S  = [0, hot) U (compaction of the mask over [hot, d_ff));
  *   x  = x + FFN_S(xh)
  * (the pre-norm residual chaining is this library's reading; the pages do
- * not describe how layers chain).  All layers must share d_model and d_ff;
+ * not describe how layers chain).  With batch 1 and layers of one shape
+ * (d_model <= 12288, rank <= 2048; Q4_0 also d_model % 256 == 0 and 16-byte
+ * aligned scale arrays) the whole stack runs in one persistent cooperative
+ * kernel per 24 layers; otherwise as a sequence of per-step kernels.
+ * Setting the environment variable PI_DISABLE_FUSED=1 forces the sequence.  All layers must share d_model and d_ff;
  * `layers`
  * is a HOST array of n_layers descriptors.  mode: PI_MASK_PER_TOKEN or
  * PI_MASK_UNION as in pi_sparse_ffn.  mask_trace: NULL, or device
@@ -181,7 +195,8 @@ enum {
   PI_KIND_FFN_UP = 4,    /* gathered gate/up rows + activation              */
   PI_KIND_FFN_DOWN = 5,  /* gathered split-K down projection                */
   PI_KIND_REDUCE = 6,    /* fixed-order partial sum + residual              */
-  PI_KINDS = 7
+  PI_KIND_FUSED = 7,     /* persistent single-token stack kernel (all steps) */
+  PI_KINDS = 8
 };
 
 /* Measurement variant of pi_ffn_stack (same arguments, same launches and
@@ -197,6 +212,29 @@ pi_status pi_ffn_stack_profile(const pi_layer* layers, int n_layers, float* x, i
                                int* kind_launches);
 
 const char* pi_kind_name(int kind);
+
+/* Measurement variant of pi_ffn_stack for the persistent single-token
+ * kernel (batch 1; PI_ERR_UNSUPPORTED otherwise): the same launches and
+ * results, plus a timeline.  timeline: device [n_layers][pi_device_sms()][16]
+ * of unsigned 64-bit values per layer and CTA: slots 0-11 are %globaltimer
+ * stamps (ns) taken by the CTA's first consumer thread at the layer's phase
+ * boundaries: 0 layer start, 1 input normalised, 2 predictor rows of P1
+ * done, 3 grid barrier 1 passed, 4 mask words done, 5 hot items done,
+ * 6 grid barrier 2 passed, 7 compaction and cold items done, 8 down rows
+ * done, 9 grid barrier 3 passed, 10 column slice reduced, 11 grid barrier 4
+ * passed; slots 12-14 are the producer warp's stall times in ns (waiting for
+ * a free stage, for the cold list, for activations) and slot 15
+ * the producer's end-of-layer stamp.  unit_timeline: NULL, or device
+ * [n_layers][512][4] receiving, for the first CTA's first 512 streamed units
+ * of each layer, the times the unit's copy was armed, its data seen by the
+ * first consumer warp and its stage released, and its byte count.
+ * Asynchronous like pi_ffn_stack. */
+pi_status pi_ffn_stack_timeline(const pi_layer* layers, int n_layers, float* x, float tau,
+                                void* ws, size_t ws_bytes, void* stream,
+                                unsigned long long* timeline, unsigned long long* unit_timeline);
+
+/* Number of SMs of the current device (the persistent kernel's grid). */
+int pi_device_sms(void);
 
 /* Synchronises `stream` and reads the workspace's two row counters, which
  * every FFN launch advances on the device: out[0] = neuron rows whose

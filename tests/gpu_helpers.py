@@ -15,11 +15,14 @@ def pi_mod():
     return pi
 
 
-def device_layer(w, layer: int, device="cuda"):
-    """(pi.Layer, raw tensors) of layer `layer`, generated in place on the GPU."""
+def device_layer(w, layer: int, device="cuda", packed: bool = False):
+    """(pi.Layer, raw tensors) of layer `layer`, generated in place on the GPU;
+    packed=True stores each neuron's weights as one record (row strides)."""
     pi = pi_mod()
     t = synth.layer_device(w, layer, device)
     keep = {k: t[k] for k in ("w_gate", "w_up", "w_down_t", "bias", "p1", "p2", "p_bias") if k in t}
+    if packed:
+        return pi.Layer.packed(w, keep), t
     return pi.Layer.from_workload(w, keep), t
 
 

@@ -131,11 +131,12 @@ def _oracle_masks(orc, H, w, xh):
 
 @pytest.mark.parametrize("shape", SHAPES)
 @pytest.mark.parametrize("act,wdt", KINDS)
-@pytest.mark.parametrize("batch,mode", [(1, "union"), (3, "per_token"), (16, "per_token"),
-                                        (64, "union"), (5, "union")])
-def test_sparse_ffn(pi, orc, shape, act, wdt, batch, mode):
+@pytest.mark.parametrize("batch,mode,packed", [(1, "union", False), (3, "per_token", True),
+                                               (16, "per_token", False), (64, "union", True),
+                                               (5, "union", False), (1, "union", True)])
+def test_sparse_ffn(pi, orc, shape, act, wdt, batch, mode, packed):
     w = _wl(act, wdt, shape)
-    L, _ = device_layer(w, 0)
+    L, _ = device_layer(w, 0, packed=packed)
     H = synth.layer_host(w, 0)
     xh = _xh(w.d_model, batch, 3)
     masks, _ = _oracle_masks(orc, H, w, xh)
@@ -213,11 +214,12 @@ def test_device_checks_flag_bad_lists(pi, orc):
 # -------------------------------------------------------------------- stack
 
 @pytest.mark.parametrize("act,wdt", [("relu", "f32"), ("reglu", "f16"), ("reglu", "q4_0"),
-                                     ("relu", "q4_0")])
+                                     ("relu", "q4_0"), ("relu", "f16")])
 @pytest.mark.parametrize("batch,mode", [(1, "union"), (4, "per_token"), (8, "union")])
-def test_stack(pi, orc, act, wdt, batch, mode):
+@pytest.mark.parametrize("packed", [False, True])
+def test_stack(pi, orc, act, wdt, batch, mode, packed):
     w = _wl(act, wdt, (512, 1500, 64, 256), seed=43, mean=0.15).scaled(3)
-    dev = [device_layer(w, l) for l in range(w.n_layers)]
+    dev = [device_layer(w, l, packed=packed) for l in range(w.n_layers)]
     host = [synth.layer_host(w, l) for l in range(w.n_layers)]
     x0 = synth.x_host(w, 0, batch)
     x = torch.from_numpy(x0).cuda()
@@ -260,9 +262,10 @@ def _check_union_stack(orc, host, x0, xg, tr, w):
         assert rel_l2(xg[b] - x0[b], xs[b] - x0[b]) <= TOL[w.w_dtype]
 
 
-def test_stack_is_deterministic(pi):
+@pytest.mark.parametrize("packed", [False, True])
+def test_stack_is_deterministic(pi, packed):
     w = _wl("reglu", "q4_0", (512, 1500, 64, 256), seed=44).scaled(4)
-    layers = [device_layer(w, l)[0] for l in range(4)]
+    layers = [device_layer(w, l, packed=packed)[0] for l in range(4)]
     x0 = torch.from_numpy(synth.x_host(w, 0, 1)).cuda()
     outs = []
     for _ in range(2):

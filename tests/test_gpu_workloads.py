@@ -33,7 +33,7 @@ def _run_layer_stack(pi, L, x0, mode, words):
 def test_workload_layer_decode(pi, orc, name):
     w = synth.WORKLOADS[name]
     layer = w.n_layers - 1
-    L, _ = device_layer(w, layer)
+    L, _ = device_layer(w, layer, packed=True)
     H = synth.layer_host(w, layer)
     words = (w.d_ff + 31) // 32
     for batch in w.batches:
@@ -62,7 +62,7 @@ def test_workload_layer_decode(pi, orc, name):
 @pytest.mark.parametrize("name", [n for n in NAMES if synth.WORKLOADS[n].union_batches])
 def test_workload_layer_union(pi, orc, name):
     w = synth.WORKLOADS[name]
-    L, _ = device_layer(w, 0)
+    L, _ = device_layer(w, 0, packed=True)
     H = synth.layer_host(w, 0)
     words = (w.d_ff + 31) // 32
     for batch in w.union_batches:
@@ -88,7 +88,7 @@ def test_headline_stack_80_layers(pi, orc):
     first layers match the oracle chain, a 2-layer chain matches end to end,
     and the whole stack is bitwise reproducible."""
     w = synth.WORKLOADS["llama2_70b_reglu_8192x28672_q4_0"]
-    layers = [device_layer(w, l)[0] for l in range(w.n_layers)]
+    layers = [device_layer(w, l, packed=True)[0] for l in range(w.n_layers)]
     words = (w.d_ff + 31) // 32
     x0 = synth.x_host(w, 0, 1)
     outs, trace = [], None
