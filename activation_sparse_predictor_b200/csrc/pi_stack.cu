@@ -1,11 +1,13 @@
 // Persistent single-token decode kernel for the whole FFN stack (sm_100a).
 //
 // One cooperative launch runs a chunk of layers with one CTA per SM.  Each
-// CTA has a producer warp that streams every weight row the CTA will use
-// through a ring of shared-memory stages with 1-D bulk copies
-// (cp.async.bulk, completion counted on an mbarrier per stage), and eight
-// consumer warps that share every stage: each consumer thread owns a slice
-// of the row's columns, so a stage is held only briefly and the ring keeps
+// CTA has four producer warps (one thread each) that stream every weight row
+// the CTA will use through a ring of shared-memory stages with 1-D bulk
+// copies (cp.async.bulk, completion counted on an mbarrier per stage; each
+// copy costs its thread a few hundred ns to issue, so the copies of
+// consecutive stages are issued by different threads), and sixteen consumer
+// warps in groups: a unit (stage) goes to one group, whose threads each take
+// a slice of its columns, so a stage is held only briefly and the ring keeps
 // many rows in flight.  Per layer:
 //
 //   x^  : every CTA normalises the full residual vector (rmsnorm) itself
@@ -17,11 +19,13 @@
 //   D   : down rows of the CTA's neurons whose h != 0     -> partial y | grid barrier 3
 //   E   : fixed-order reduction of the CTA's column slice, residual add | grid barrier 4
 //
-// The producer runs ahead across phases for every row whose address does
-// not depend on this layer's data (P1, P2, hot rows, the next layer's rows),
-// so HBM keeps streaming through the grid barriers; only cold rows wait for
-// the compaction and down rows for their h.  Every wait (mbarrier, grid
-// barrier, flag) is bounded by %globaltimer; a wait that runs out sets
+// The producers run ahead across phases for every row whose address does
+// not depend on this layer's data (P1, P2, hot rows, the next layer's rows);
+// only cold rows wait for the compaction and down rows for their h.  (L2
+// prefetching of the static rows ahead of the ring, by bulk or per-line
+// prefetches, measured slower at every distance tried, 256 KB to 1 MB per
+// CTA, and is not used.)  Every wait (mbarrier, grid barrier, flag) is
+// bounded by %globaltimer; a wait that runs out sets
 // DEV_TIMEOUT and an abort flag, after which every thread runs the rest of
 // its loops without waiting or computing and the producer waits (bounded)
 // for its own copies in flight before exiting.
@@ -41,8 +45,9 @@ namespace {
 
 constexpr int NCW = 16;             // consumer warps
 constexpr int NCT = NCW * 32;       // consumer threads
-constexpr int NPMAX = 4;            // producer warps at most (after the consumers)
+constexpr int NPMAX = 4;            // producer warps (after the consumers)
 constexpr int NTHR = NCT + 32 * NPMAX;
+static_assert((NPMAX & (NPMAX - 1)) == 0, "stage owner is st & (NPMAX - 1)");
 constexpr int NSMAX = 24;           // ring stages at most
 constexpr int MAXL = 24;            // layers per launch
 constexpr int GRP = 32;             // items per cross-warp finalisation group
@@ -68,7 +73,7 @@ static_assert(sizeof(LayerPtrs) == 80, "compact layer pointers");
 struct Plan {
   int d, F, r, H;
   int ns, G, maxc, maxi, nsms;
-  int np;                           // producer warps (divides ns)
+  int np;                           // producer warps
   int gw, gd;                       // consumer warp groups: up-projection / down phases
   int hp;                           // hot neurons per unit (adjacent records)
   int dr;                           // down rows per unit at most (adjacent records)
@@ -80,7 +85,7 @@ struct Plan {
   uint32_t p1_bytes, p2_row;        // predictor row bytes
   uint32_t item_bytes, down_bytes;  // bytes copied per item / per down row
   uint32_t o_first_s, o_second, o_second_s, o_down_s;  // offsets inside a stage
-  uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_mw, o_scan, o_cold, o_hval, o_flag,
+  uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_mw, o_scan, o_items, o_hval, o_flag,
       o_dlist, o_runs, o_pbs, o_hbs, o_redA, o_redC, o_redE, o_ring, total;
 };
 
@@ -199,20 +204,33 @@ __device__ __forceinline__ int qpos(int i, int nb) {
   return ((((i >> 3) & 3) * nb + (i >> 5)) << 3) + (i & 7);
 }
 
-// Dot product of 16-byte chunk c of a DT row with the staged vector v (length n).
+// The staged-vector elements that chunk c of a DT row multiplies.
+struct VFrag {
+  float4 lo, hi;  // hi only for fp16 rows
+};
+
 template <int DT>
-__device__ __forceinline__ float chunk_dot(const uint4 w, const float* v, int c, int n) {
+__device__ __forceinline__ VFrag vfrag(const float* v, int c, int n) {
   const float4* v4 = reinterpret_cast<const float4*>(v);
+  VFrag f;
+  f.lo = v4[c];
+  if constexpr (DT == PI_F16) f.hi = v4[(n >> 3) + c];
+  else f.hi = f.lo;
+  return f;
+}
+
+// Dot product of a 16-byte chunk of a DT row with its vector fragment.
+template <int DT>
+__device__ __forceinline__ float frag_dot(const uint4 w, const VFrag& x) {
   if constexpr (DT == PI_F32) {
-    const float4 x = v4[c];
-    float a = __uint_as_float(w.x) * x.x;
-    a = fmaf(__uint_as_float(w.y), x.y, a);
-    a = fmaf(__uint_as_float(w.z), x.z, a);
-    return fmaf(__uint_as_float(w.w), x.w, a);
+    float a = __uint_as_float(w.x) * x.lo.x;
+    a = fmaf(__uint_as_float(w.y), x.lo.y, a);
+    a = fmaf(__uint_as_float(w.z), x.lo.z, a);
+    return fmaf(__uint_as_float(w.w), x.lo.w, a);
   } else {
     float f[8];
     f16x8_to_f32(w, f);
-    const float4 lo = v4[c], hi = v4[(n >> 3) + c];
+    const float4 lo = x.lo, hi = x.hi;
     float a = f[0] * lo.x, b = f[4] * hi.x;
     a = fmaf(f[1], lo.y, a);
     b = fmaf(f[5], hi.y, b);
@@ -222,6 +240,20 @@ __device__ __forceinline__ float chunk_dot(const uint4 w, const float* v, int c,
     b = fmaf(f[7], hi.w, b);
     return a + b;
   }
+}
+
+// Dot product of 16-byte chunk c of a DT row with the staged vector v (length n).
+template <int DT>
+__device__ __forceinline__ float chunk_dot(const uint4 w, const float* v, int c, int n) {
+  return frag_dot<DT>(w, vfrag<DT>(v, c, n));
+}
+
+// Two nibbles of a Q4_0 word as floats 1 + q/16: x holds 0x80 | q << 3 in
+// each byte (q = the nibble), and the byte permute places byte b (and b+1)
+// as bits 16..23 under the exponent byte 0x3F.
+__device__ __forceinline__ float2 nib_pair(uint32_t x, int b) {
+  return make_float2(__uint_as_float(__byte_perm(x, 0x3F00u, 0x5044u | ((uint32_t)b << 8))),
+                     __uint_as_float(__byte_perm(x, 0x3F00u, 0x5044u | ((uint32_t)(b + 1) << 8))));
 }
 
 // sum_k (q_k - 8) * x_k over one Q4_0 block in exact int32 arithmetic:
@@ -257,7 +289,7 @@ struct Smem {
   uint32_t* bw;
   uint32_t* mw;
   int* scan;
-  int* cold;
+  int* items;                 // neuron of each item: hot items, then this layer's cold list
   float* hval;
   volatile int* flag;
   int* dlist;
@@ -286,7 +318,7 @@ __device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
   S.bw = reinterpret_cast<uint32_t*>(base + pl.o_bw);
   S.mw = reinterpret_cast<uint32_t*>(base + pl.o_mw);
   S.scan = reinterpret_cast<int*>(base + pl.o_scan);
-  S.cold = reinterpret_cast<int*>(base + pl.o_cold);
+  S.items = reinterpret_cast<int*>(base + pl.o_items);
   S.hval = reinterpret_cast<float*>(base + pl.o_hval);
   S.flag = reinterpret_cast<volatile int*>(base + pl.o_flag);
   S.dlist = reinterpret_cast<int*>(base + pl.o_dlist);
@@ -308,8 +340,10 @@ __device__ void raise_abort(const Smem& S, WsHeader* hdr) {
 }
 
 // Bounded mbarrier wait; false on abort or timeout (timeout raises abort).
-// The warp sleeps in the hardware wait between checks.
-__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Smem& S, WsHeader* hdr) {
+// The first try usually succeeds; the warp sleeps in the hardware wait
+// between later checks.
+__device__ __forceinline__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Smem& S,
+                                          WsHeader* hdr) {
   if (mbar_try(bar, parity)) return true;
   if (*S.abort) return false;
   const uint64_t t0 = gtime();
@@ -391,10 +425,20 @@ __device__ __forceinline__ int hot_group_first(int gi, const Plan& pl) {
   return ((int)blockIdx.x + (int)gridDim.x * gi) * pl.hp;
 }
 
-__device__ __forceinline__ int item_neuron(int i, const Ranges& R, const Plan& pl, const Smem& S) {
-  if (i < R.nh) return hot_group_first(i / pl.hp, pl) + i % pl.hp;
-  return S.cold[i - R.nh];
-}
+// Position in the unit sequence: unit number, its stage (uc % ns) and the
+// stage's use count (uc / ns), advanced without divisions.
+struct Cursor {
+  uint32_t uc = 0;
+  int st = 0;
+  uint32_t gen = 0;
+  __device__ __forceinline__ void next(int ns) {
+    ++uc;
+    if (++st == ns) {
+      st = 0;
+      ++gen;
+    }
+  }
+};
 
 // Down-row units: runs of consecutive nonzero items whose neurons are
 // adjacent (when down records are packed), at most pl.dr rows each.  The
@@ -410,8 +454,8 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   const Plan& pl = P.pl;
   WsHeader* hdr = P.hdr;
   const Ranges R = ranges(pl);
-  uint32_t uc = 0;  // unit sequence number, identical on every producer and consumer
-  uint32_t last[NSMAX];
+  Cursor cu;  // unit sequence, identical on every producer and consumer
+  uint32_t last[NSMAX];  // use count of each stage's last copy issued here
 #pragma unroll
   for (int i = 0; i < NSMAX; ++i) last[i] = 0xFFFFFFFFu;
   bool ok = true;
@@ -419,12 +463,12 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   int cur_l = 0;
   uint32_t l_uc0 = 0;  // first unit of the current layer
 
-  // Stage uc % ns belongs to producer (uc % ns) % np == uc % np (np divides ns).
-  auto mine = [&]() { return (int)(uc % (uint32_t)pl.np) == p; };
-  // Claims unit uc's stage (one of ours) and arms its full barrier for `bytes`.
+  // Stage st belongs to producer st % NPMAX.
+  auto mine = [&]() { return (cu.st & (NPMAX - 1)) == p; };
+  // Claims the current unit's stage (one of ours) and arms its full barrier for `bytes`.
   auto claim = [&](uint32_t bytes) -> char* {
-    const int st = (int)(uc % (uint32_t)pl.ns);
-    const uint32_t k = uc / (uint32_t)pl.ns;
+    const int st = cu.st;
+    const uint32_t k = cu.gen;
     if (k > 0 && !mbar_try(&S.empty[st], (k - 1) & 1u)) {
       const unsigned long long t0 = P.trace ? gtime() : 0ull;
       if (!wait_mbar(&S.empty[st], (k - 1) & 1u, S, hdr)) {
@@ -434,14 +478,14 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       if (P.trace) w_empty += gtime() - t0;
     }
     mbar_arrive_tx(&S.full[st], bytes);
-    last[st] = uc;
+    last[st] = k;
     if (P.utrace) {
-      utstamp(P, cur_l, uc - l_uc0, 0, gtime());
-      utstamp(P, cur_l, uc - l_uc0, 3, bytes);
+      utstamp(P, cur_l, cu.uc - l_uc0, 0, gtime());
+      utstamp(P, cur_l, cu.uc - l_uc0, 3, bytes);
     }
     return S.ring + (size_t)st * pl.sb;
   };
-  auto bar_of = [&]() { return &S.full[uc % (uint32_t)pl.ns]; };
+  auto bar_of = [&]() { return &S.full[cu.st]; };
 
   // Up-projection records of neurons j0 .. j0+n-1 (n > 1 only when packed).
   auto items = [&](const LayerPtrs& L, int j0, int n) {
@@ -463,7 +507,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         }
       }
     }
-    ++uc;
+    cu.next(pl.ns);
   };
   // Down records of neurons j0 .. j0+n-1.
   auto downs = [&](const LayerPtrs& L, int j0, int n) {
@@ -480,35 +524,38 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         }
       }
     }
-    ++uc;
+    cu.next(pl.ns);
   };
 
   for (int l = 0; l < P.n_layers && ok; ++l) {
     const LayerPtrs& L = P.L[l];
     cur_l = l;
-    l_uc0 = uc;
+    l_uc0 = cu.uc;
     // A: predictor rows of P1
-    for (int k = R.kA0; k < R.kA1 && ok; ++k, ++uc) {
-      if (!mine()) continue;
-      char* dst = claim(pl.p1_bytes);
-      if (!dst) break;
-      bulk_g2s(dst, L.p1 + (size_t)k * pl.p1_bytes, pl.p1_bytes, bar_of());
+    for (int k = R.kA0; k < R.kA1 && ok; ++k, cu.next(pl.ns)) {
+      if (mine()) {
+        char* dst = claim(pl.p1_bytes);
+        if (!dst) break;
+        bulk_g2s(dst, L.p1 + (size_t)k * pl.p1_bytes, pl.p1_bytes, bar_of());
+      }
     }
     // B: predictor rows of P2, G per unit
     for (int w = R.wB0; w < R.wB1 && ok; ++w) {
-      for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F && ok; ja += pl.G, ++uc) {
-        if (!mine()) continue;
+      for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F && ok; ja += pl.G, cu.next(pl.ns)) {
         const int jb = min(ja + pl.G, pl.F);
         const uint32_t bytes = (uint32_t)(jb - ja) * pl.p2_row;
-        char* dst = claim(bytes);
-        if (!dst) break;
-        bulk_g2s(dst, L.p2 + (size_t)ja * pl.p2_row, bytes, bar_of());
+        if (mine()) {
+          char* dst = claim(bytes);
+          if (!dst) break;
+          bulk_g2s(dst, L.p2 + (size_t)ja * pl.p2_row, bytes, bar_of());
+        }
       }
     }
     // C: hot groups, then (after the consumers' compaction) cold neurons
     for (int gi = 0; gi < R.ngh && ok; ++gi) {
       const int j0 = hot_group_first(gi, pl);
-      items(L, j0, min(pl.hp, pl.H - j0));
+      const int n = min(pl.hp, pl.H - j0);
+      items(L, j0, n);
     }
     {
       const unsigned long long t0 = P.trace ? gtime() : 0ull;
@@ -516,7 +563,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       if (P.trace) w_list += gtime() - t0;
     }
     const int nc = *S.nc;
-    for (int i = 0; i < nc && ok; ++i) items(L, S.cold[i], 1);
+    for (int i = 0; i < nc && ok; ++i) items(L, S.items[R.nh + i], 1);
     // D: down rows of items whose h != 0, in item order, as runs
     const int tag = (l + 1) << 2;
     int rj = -1, rlen = 0;  // open run: first neuron, rows
@@ -533,7 +580,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         if (!ok) break;
       }
       if ((f & 3) != 2) continue;
-      const int j = item_neuron(i, R, pl, S);
+      const int j = S.items[i];
       if (rlen > 0 && run_extends(rj + rlen - 1, j, rlen, pl)) {
         ++rlen;
         continue;
@@ -554,7 +601,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   // Drain: wait (bounded) until every copy this thread issued has landed.
   for (int st = 0; st < pl.ns; ++st) {
     if (last[st] == 0xFFFFFFFFu) continue;
-    const uint32_t par = (last[st] / (uint32_t)pl.ns) & 1u;
+    const uint32_t par = last[st] & 1u;
     const uint64_t t0 = gtime();
     while (!mbar_try(&S.full[st], par)) {
       if (gtime() - t0 > kTimeoutNs) {
@@ -585,21 +632,24 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
   // The down-projection phase uses GD groups of NCW / GD warps.
   const int GD = pl.gd, WPD = NCW / GD, dgrp = warp / WPD;
   const int dtid = (warp % WPD) * 32 + lane, DT = WPD * 32;
-  uint32_t uc = 0, nbar = 0;
+  Cursor cu;  // the unit sequence (every warp walks all of it)
+  uint32_t nbar = 0;
   int cur_l = 0;
   uint32_t l_uc0 = 0;
+  const uint32_t gwm = (uint32_t)GW - 1u, gdm = (uint32_t)GD - 1u;  // GW, GD: powers of 2
 
-  auto ready = [&](int st) -> bool {
-    const bool ok = wait_mbar(&S.full[st], (uc / (uint32_t)pl.ns) & 1u, S, hdr);
-    if (P.utrace && tid == 0) utstamp(P, cur_l, uc - l_uc0, 1, gtime());
+  // the current unit's data has landed (false on abort / timeout)
+  auto ready = [&]() -> bool {
+    const bool ok = wait_mbar(&S.full[cu.st], cu.gen & 1u, S, hdr);
+    if (P.utrace && tid == 0) utstamp(P, cur_l, cu.uc - l_uc0, 1, gtime());
     return __all_sync(0xffffffffu, ok);
   };
-  auto stage = [&](int st) { return S.ring + (size_t)st * pl.sb; };
-  // each of the `warps` warps that shared a unit releases its part of it
-  auto release = [&](int st, int warps) {
+  auto stage = [&]() { return S.ring + (size_t)cu.st * pl.sb; };
+  // each of the `warps` warps that shared the current unit releases its part of it
+  auto release = [&](int warps) {
     __syncwarp();
-    if (lane == 0) mbar_arrive(&S.empty[st], (uint32_t)(NCW / warps));
-    if (P.utrace && tid == 0) utstamp(P, cur_l, uc - l_uc0, 2, gtime());
+    if (lane == 0) mbar_arrive(&S.empty[cu.st], (uint32_t)(NCW / warps));
+    if (P.utrace && tid == 0) utstamp(P, cur_l, cu.uc - l_uc0, 2, gtime());
   };
   auto gsync_arrive = [&]() {
     csync();
@@ -616,78 +666,91 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     uint32_t* mask = P.mask + (size_t)l * P.mask_stride;
     const int tag = (l + 1) << 2;
     cur_l = l;
-    l_uc0 = uc;
+    l_uc0 = cu.uc;
 
-    // ---- x^ = x / sqrt(mean(x^2) + 1e-6); all loads issued at once
+    // ---- x^ = x / sqrt(mean(x^2) + 1e-6): each thread takes 8-element
+    // chunks c = tid, tid + NCT, ... (all loads issued at once); one CTA-wide
+    // reduction gives sum(x^2) and max|x|; 16-byte stores of x^ (and of its
+    // int16 copy) are conflict-free
     if (tid == 0) tstamp(P, l, 0, gtime());
     {
-      constexpr int MX = 6;   // float4 per thread, d <= 12288
+      constexpr int MC = 3;  // chunks per thread, d <= 12288
+      const int nc8 = d / 8;
       const float4* x4 = reinterpret_cast<const float4*>(P.x);
-      float4 xv[MX];
-      float ss = 0.f;
+      float4 xa[MC], xb[MC];
 #pragma unroll
-      for (int m = 0; m < MX; ++m) {
-        const int q = tid + m * NCT;
-        xv[m] = q < d / 4 ? __ldcg(x4 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int m = 0; m < MC; ++m) {
+        const int c = tid + m * NCT;
+        const bool in = c < nc8;
+        xa[m] = in ? __ldcg(x4 + 2 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        xb[m] = in ? __ldcg(x4 + 2 * c + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      float ss = 0.f, mx = 0.f;
+#pragma unroll
+      for (int m = 0; m < MC; ++m) {
+        const float e[8] = {xa[m].x, xa[m].y, xa[m].z, xa[m].w, xb[m].x, xb[m].y, xb[m].z, xb[m].w};
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          ss = fmaf(e[k], e[k], ss);
+          mx = fmaxf(mx, fabsf(e[k]));
+        }
       }
 #pragma unroll
-      for (int m = 0; m < MX; ++m)
-        ss += xv[m].x * xv[m].x + xv[m].y * xv[m].y + xv[m].z * xv[m].z + xv[m].w * xv[m].w;
-      ss = warp_sum(ss);
-      if (lane == 0) S.redA[warp] = ss;
+      for (int o = 16; o > 0; o >>= 1) {
+        ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      if (lane == 0) {
+        S.redA[warp] = ss;
+        S.redA[NCW + warp] = mx;
+      }
       csync();
-      float tot = 0.f;
+      float tot = 0.f, amax = 0.f;
 #pragma unroll
-      for (int w = 0; w < NCW; ++w) tot += S.redA[w];
-      const float inv = 1.0f / sqrtf(tot / (float)d + 1e-6f);
-      float amax = 0.f;
-#pragma unroll
-      for (int m = 0; m < MX; ++m) {
-        const int q = tid + m * NCT;
-        if (q >= d / 4) break;
-        const float e[4] = {xv[m].x * inv, xv[m].y * inv, xv[m].z * inv, xv[m].w * inv};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          S.xf[vpos<PT>(4 * q + k, d)] = e[k];
-          amax = fmaxf(amax, fabsf(e[k]));
-        }
+      for (int w = 0; w < NCW; ++w) {
+        tot += S.redA[w];
+        amax = fmaxf(amax, S.redA[NCW + w]);
       }
+      const float inv = 1.0f / sqrtf(tot / (float)d + 1e-6f);
+      float ixs = 1.f;
       if constexpr (WT == PI_Q4_0) {
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-        csync();  // everyone has read redA
-        if (lane == 0) S.redA[warp] = amax;
-        csync();
-        float mx = 0.f;
-#pragma unroll
-        for (int w = 0; w < NCW; ++w) mx = fmaxf(mx, S.redA[w]);
-        const float xs = mx > 0.f ? mx / 32767.0f : 1.0f;
-        const float ixs = 1.0f / xs;
+        const float xm = amax * inv;  // max |x^|: scaling by inv > 0 keeps the order
+        const float xs = xm > 0.f ? xm / 32767.0f : 1.0f;
+        ixs = 1.0f / xs;
         if (tid == 0) *S.xscale = xs;
+      }
+      float4* xf4 = reinterpret_cast<float4*>(S.xf);
 #pragma unroll
-        for (int m = 0; m < MX; ++m) {
-          const int q = tid + m * NCT;
-          if (q >= d / 4) break;
-          const float e[4] = {xv[m].x * inv, xv[m].y * inv, xv[m].z * inv, xv[m].w * inv};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            int v = __float2int_rn(e[k] * ixs);
-            v = v > 32767 ? 32767 : (v < -32767 ? -32767 : v);
-            S.xi[qpos(4 * q + k, nb)] = (int16_t)v;
-          }
+      for (int m = 0; m < MC; ++m) {
+        const int c = tid + m * NCT;
+        if (c >= nc8) break;  // warp-uniform for Q4_0 (d % 256 == 0)
+        const float4 lo = make_float4(xa[m].x * inv, xa[m].y * inv, xa[m].z * inv, xa[m].w * inv);
+        const float4 hi = make_float4(xb[m].x * inv, xb[m].y * inv, xb[m].z * inv, xb[m].w * inv);
+        if constexpr (PT == PI_F16) {
+          xf4[c] = lo;  // split-half layout
+          xf4[nc8 + c] = hi;
+        } else {
+          xf4[2 * c] = lo;
+          xf4[2 * c + 1] = hi;
         }
-        csync();
-        const int4* xb = reinterpret_cast<const int4*>(S.xi);
-        for (int k = tid; k < nb; k += NCT) {
-          int t = 0;
+        if constexpr (WT == PI_Q4_0) {
+          const float e[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          int v[8], t = 0;
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int4 v = xb[q * nb + k];
-            const int w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) t += (int)(int16_t)(w4[e] & 0xFFFF) + (w4[e] >> 16);
+          for (int k = 0; k < 8; ++k) {
+            int q = __float2int_rn(e[k] * ixs);
+            q = q > 32767 ? 32767 : (q < -32767 ? -32767 : q);
+            v[k] = q;
+            t += q;
           }
-          S.bsum[k] = t;
+          // chunk c = 4 * block + sub-chunk: sub-chunk-major int16 layout
+          reinterpret_cast<int4*>(S.xi)[(c & 3) * nb + (c >> 2)] =
+              make_int4((v[0] & 0xFFFF) | (v[1] << 16), (v[2] & 0xFFFF) | (v[3] << 16),
+                        (v[4] & 0xFFFF) | (v[5] << 16), (v[6] & 0xFFFF) | (v[7] << 16));
+          // block sum over the block's 4 chunks (4 adjacent lanes)
+          t += __shfl_xor_sync(0xffffffffu, t, 1);
+          t += __shfl_xor_sync(0xffffffffu, t, 2);
+          if ((lane & 3) == 0) S.bsum[c >> 2] = t;
         }
       }
       csync();
@@ -699,12 +762,10 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     {
       constexpr int CCP = WTraits<PT>::CHUNK_COLS;
       const int nch = d / CCP;
-      const uint32_t ua0 = uc;
-      for (int a = 0; a < nA; ++a, ++uc) {
-        if ((int)(uc % (uint32_t)GW) != grp) continue;
-        const int st = (int)(uc % (uint32_t)pl.ns);
-        if (!ready(st)) continue;
-        const char* row = stage(st);
+      for (int a = 0; a < nA; ++a, cu.next(pl.ns)) {
+        if ((int)(cu.uc & gwm) != grp) continue;
+        if (!ready()) continue;
+        const char* row = stage();
         float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
         int c = gtid;
         for (; c + 3 * GT < nch; c += 4 * GT) {
@@ -714,7 +775,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
           v3 += chunk_dot<PT>(lds128(row + (size_t)(c + 3 * GT) * 16), S.xf, c + 3 * GT, d);
         }
         for (; c < nch; c += GT) v0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.xf, c, d);
-        release(st, WPG);
+        release(WPG);
         float v = warp_sum((v0 + v1) + (v2 + v3));
         if (lane == 0) S.redA[MAXA + a * NCW + wg] = v;
       }
@@ -725,7 +786,6 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         for (int w = 0; w < wpg; ++w) v += S.redA[MAXA + a * NCW + w];
         __stcg(P.u + R.kA0 + a, v);
       }
-      (void)ua0;
     }
     if (tid == 0) tstamp(P, l, 2, gtime());
     gsync_arrive();  // 1: u complete
@@ -734,7 +794,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       const int j = 32 * R.wB0 + k;
       S.pbs[k] = (L.pbias && j < pl.F) ? L.pbias[j] : 0.f;
     }
-    for (int i = tid; i < R.nh; i += NCT) S.hbs[i] = L.bias ? L.bias[item_neuron(i, R, pl, S)] : 0.f;
+    for (int i = tid; i < R.nh; i += NCT) S.hbs[i] = L.bias ? L.bias[S.items[i]] : 0.f;
     gsync_wait();
     if (tid == 0) tstamp(P, l, 3, gtime());
 
@@ -746,26 +806,38 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       constexpr int CCP = WTraits<PT>::CHUNK_COLS;
       const int nch = pl.r / CCP;
       for (int w = R.wB0; w < R.wB1; ++w) {
-        for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F; ja += pl.G, ++uc) {
-          if ((int)(uc % (uint32_t)GW) != grp) continue;
-          const int st = (int)(uc % (uint32_t)pl.ns);
-          if (!ready(st)) continue;
-          const char* buf = stage(st);
+        for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F; ja += pl.G, cu.next(pl.ns)) {
+          if ((int)(cu.uc & gwm) != grp) continue;
+          if (!ready()) continue;
+          const char* buf = stage();
           const int jb = min(ja + pl.G, pl.F);
           uint32_t bits = 0u;
-          for (int j = ja + wg; j < jb; j += WPG) {
+          // a warp takes rows j and j + WPG together (one u load for both)
+          for (int j = ja + wg; j < jb; j += 2 * WPG) {
+            const int j2 = j + WPG;
+            const bool pair = j2 < jb;  // warp-uniform
             const char* row = buf + (size_t)(j - ja) * pl.p2_row;
+            const char* row2 = row + (size_t)WPG * pl.p2_row;
             float z0 = 0.f, z1 = 0.f;
-            int c = lane;
-            for (; c + 32 < nch; c += 64) {
-              z0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.us, c, pl.r);
-              z1 += chunk_dot<PT>(lds128(row + (size_t)(c + 32) * 16), S.us, c + 32, pl.r);
+#pragma unroll 4
+            for (int c = lane; c < nch; c += 32) {
+              const VFrag uf = vfrag<PT>(S.us, c, pl.r);
+              z0 += frag_dot<PT>(lds128(row + (size_t)c * 16), uf);
+              if (pair) z1 += frag_dot<PT>(lds128(row2 + (size_t)c * 16), uf);
             }
-            if (c < nch) z0 += chunk_dot<PT>(lds128(row + (size_t)c * 16), S.us, c, pl.r);
-            const float z = warp_sum(z0 + z1) + S.pbs[j - 32 * R.wB0];
-            if (j >= pl.H && z > P.theta) bits |= 1u << (j & 31);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+              z0 += __shfl_xor_sync(0xffffffffu, z0, o);
+              z1 += __shfl_xor_sync(0xffffffffu, z1, o);
+            }
+            const float za = z0 + S.pbs[j - 32 * R.wB0];
+            if (j >= pl.H && za > P.theta) bits |= 1u << (j & 31);
+            if (pair) {
+              const float zb = z1 + S.pbs[j2 - 32 * R.wB0];
+              if (j2 >= pl.H && zb > P.theta) bits |= 1u << (j2 & 31);
+            }
           }
-          release(st, WPG);
+          release(WPG);
           if (lane == 0 && bits) atomicOr(&S.bw[w - R.wB0], bits);
         }
       }
@@ -812,14 +884,13 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     };
     // one unit: items i0 .. i0+n-1, record r of the stage for item i0 + r
     auto unit_items = [&](int i0, int n) {
-      if ((int)(uc % (uint32_t)GW) == grp) {
-        const int st = (int)(uc % (uint32_t)pl.ns);
-        const bool ok = ready(st);
+      if ((int)(cu.uc & gwm) == grp) {
+        const bool ok = ready();
         float a[8], b[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
         if (ok) {
-          const char* base = stage(st);
+          const char* base = stage();
           if constexpr (WT == PI_Q4_0) {
             const int4* xb = reinterpret_cast<const int4*>(S.xi);
             for (int k = gtid; k < nb; k += GT) {
@@ -855,7 +926,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
               }
             }
           }
-          release(st, WPG);
+          release(WPG);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1)
@@ -878,7 +949,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
           }
         }
       }
-      ++uc;
+      cu.next(pl.ns);
       // finalise every group of GRP items completed by this unit
       const int i1 = i0 + n;
       if (i1 / GRP != i0 / GRP) finalise((i1 / GRP) * GRP);
@@ -920,18 +991,24 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         if (w < warp) wpre += v;
         total += v;
       }
-      int p = wpre + incl - cnt;  // list position of this thread's first neuron
+      // list position p = wpre + incl - cnt of this thread's first neuron goes
+      // to CTA p % nS, slot p / nS; both advance without dividing again
+      const int p = wpre + incl - cnt;
+      int r = p % nS, q = p / nS;
       for (int w = wa; w < wb; ++w) {
         uint32_t m = S.mw[w - R.Wlo];
         while (m) {
           const int bit = __ffs(m) - 1;
           m &= m - 1u;
-          if (p % nS == s) {
+          if (r == s) {
             const int j = 32 * w + bit;
-            S.cold[p / nS] = j;
-            S.hbs[R.nh + p / nS] = L.bias ? L.bias[j] : 0.f;
+            S.items[R.nh + q] = j;
+            S.hbs[R.nh + q] = L.bias ? L.bias[j] : 0.f;
           }
-          ++p;
+          if (++r == nS) {
+            r = 0;
+            ++q;
+          }
         }
       }
       if (tid == 0) {
@@ -964,7 +1041,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       if (lane == 0) {
         int nr = 0, jp = -1, len = 0;
         for (int q = 0; q < base; ++q) {
-          const int j = item_neuron(S.dlist[q], R, pl, S);
+          const int j = S.items[S.dlist[q]];
           if (len > 0 && run_extends(jp, j, len, pl)) {
             ++len;
           } else {
@@ -981,38 +1058,78 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     }
     csync();
     const int nd = S.scan[NCW], nruns = S.scan[NCW + 1];
-    {
+    if constexpr (WT == PI_Q4_0) {
+      // one Q4_0 block (32 columns) per thread (the plan keeps d / 32 within
+      // a group).  sum_j hs_j (q - 8), hs_j = h_j * scale, is accumulated as
+      // sum_j 16 hs_j (1 + q/16) with packed fp32x2 FMAs on floats built from
+      // the nibbles by byte permutes, minus 24 sum_j hs_j at the end.
+      const int nch = d / 32, c = dtid;
+      float2 acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] = make_float2(0.f, 0.f);
+      float corr = 0.f;
+      for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+        if ((int)(cu.uc & gdm) != dgrp) continue;
+        if (!ready()) continue;
+        const int q0 = S.runs[2 * q], len = S.runs[2 * q + 1];
+        if (c < nch) {
+#pragma unroll 2
+          for (int rr = 0; rr < len; ++rr) {
+            const char* row = stage() + (size_t)rr * pl.down_bytes;
+            const uint4 v = lds128(row + (size_t)c * 16);
+            const float hs =
+                S.hval[S.dlist[q0 + rr]] * h2f(reinterpret_cast<const uint16_t*>(row + pl.o_down_s)[c]);
+            corr += hs;
+            const float2 h2 = make_float2(16.f * hs, 16.f * hs);
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+              // byte b: 0x80 | q << 3 for element 4m + b (low nibbles) / 16 + 4m + b (high)
+              const uint32_t lo = ((wv[m] << 3) & 0x78787878u) | 0x80808080u;
+              const uint32_t hi = ((wv[m] >> 1) & 0x78787878u) | 0x80808080u;
+#pragma unroll
+              for (int b = 0; b < 4; b += 2) {
+                acc[(4 * m + b) >> 1] = __ffma2_rn(nib_pair(lo, b), h2, acc[(4 * m + b) >> 1]);
+                acc[(16 + 4 * m + b) >> 1] =
+                    __ffma2_rn(nib_pair(hi, b), h2, acc[(16 + 4 * m + b) >> 1]);
+              }
+            }
+          }
+        }
+        release(WPD);
+      }
+      // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
+      if (c < nch) {
+        float* part = P.part + ((size_t)s * GD + dgrp) * d + (size_t)c * 32;
+        const float k24 = 24.f * corr;
+#pragma unroll
+        for (int e = 0; e < 16; e += 2)
+          __stcg(reinterpret_cast<float4*>(part + 2 * e),
+                 make_float4(acc[e].x - k24, acc[e].y - k24, acc[e + 1].x - k24, acc[e + 1].y - k24));
+      }
+    } else {
+      // fp16 / fp32 rows: up to 48 columns per thread
       constexpr int CC = WTraits<WT>::CHUNK_COLS;
-      constexpr int MAXK = (CC == 32) ? 1 : 48 / CC;  // chunks per thread of a D group
+      constexpr int MAXK = 48 / CC;  // chunks per thread of a D group
       const int nch = d / CC;
       float acc[MAXK][CC];
 #pragma unroll
       for (int k = 0; k < MAXK; ++k)
 #pragma unroll
         for (int e = 0; e < CC; ++e) acc[k][e] = 0.f;
-      for (int q = 0; q < nruns; ++q, ++uc) {
-        if ((int)(uc % (uint32_t)GD) != dgrp) continue;
-        const int st = (int)(uc % (uint32_t)pl.ns);
-        if (!ready(st)) continue;
+      for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+        if ((int)(cu.uc & gdm) != dgrp) continue;
+        if (!ready()) continue;
         const int q0 = S.runs[2 * q], len = S.runs[2 * q + 1];
         for (int rr = 0; rr < len; ++rr) {
-          const char* row = stage(st) + (size_t)rr * pl.down_bytes;
+          const char* row = stage() + (size_t)rr * pl.down_bytes;
           const float hv = S.hval[S.dlist[q0 + rr]];
 #pragma unroll
           for (int k = 0; k < MAXK; ++k) {
             const int c = dtid + k * DT;
             if (c >= nch) break;
             const uint4 v = lds128(row + (size_t)c * 16);
-            if constexpr (WT == PI_Q4_0) {
-              const float hs = hv * h2f(reinterpret_cast<const uint16_t*>(row + pl.o_down_s)[c]);
-              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int e = 0; e < 16; ++e) {
-                const uint32_t byte = (wv[e >> 2] >> (8 * (e & 3))) & 0xFFu;
-                acc[k][e] = fmaf(hs, q4_centered(byte & 0xFu), acc[k][e]);
-                acc[k][e + 16] = fmaf(hs, q4_centered(byte >> 4), acc[k][e + 16]);
-              }
-            } else if constexpr (WT == PI_F16) {
+            if constexpr (WT == PI_F16) {
               float f[8];
               f16x8_to_f32(v, f);
 #pragma unroll
@@ -1025,7 +1142,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
             }
           }
         }
-        release(st, WPD);
+        release(WPD);
       }
       // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
       float* part = P.part + ((size_t)s * GD + dgrp) * d;
@@ -1057,18 +1174,22 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       const int nq = cq1 - cq0;  // <= 32
       const int g = nq > 0 ? NCT / nq : 0;
       const float4* pp = reinterpret_cast<const float4*>(P.part);
+      float4* x4 = reinterpret_cast<float4*>(P.x) + cq0 + tid;
+      const float4 xo = tid < nq ? __ldcg(x4) : make_float4(0.f, 0.f, 0.f, 0.f);
       if (nq > 0 && tid < nq * g) {
+        // rows gi, gi + g, ... summed in that order; 12 loads in flight
+        constexpr int ER = 12;
         const int q = tid % nq, gi = tid / nq;
         float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int sp0 = gi; sp0 < nP; sp0 += 8 * g) {
-          float4 v[8];
+        for (int sp0 = gi; sp0 < nP; sp0 += ER * g) {
+          float4 v[ER];
 #pragma unroll
-          for (int m = 0; m < 8; ++m) {
+          for (int m = 0; m < ER; ++m) {
             const int sp = sp0 + m * g;
             v[m] = sp < nP ? __ldcg(pp + (size_t)sp * q4n + cq0 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
           }
 #pragma unroll
-          for (int m = 0; m < 8; ++m) t = f4add(t, v[m]);
+          for (int m = 0; m < ER; ++m) t = f4add(t, v[m]);
         }
         S.redE[gi * nq + q] = t;
       }
@@ -1076,8 +1197,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       if (tid < nq) {
         float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int gi = 0; gi < g; ++gi) y = f4add(y, S.redE[gi * nq + tid]);
-        float4* x4 = reinterpret_cast<float4*>(P.x) + cq0 + tid;
-        __stcg(x4, f4add(__ldcg(x4), y));
+        __stcg(x4, f4add(xo, y));
       }
     }
     csync();
@@ -1104,6 +1224,12 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int i = threadIdx.x; i < P.pl.maxi; i += NTHR) S.flag[i] = 0;
+  {
+    // the CTA's hot items: groups g = s, s + SMs, ... of hp adjacent neurons
+    const Ranges R = ranges(P.pl);
+    for (int i = threadIdx.x; i < R.nh; i += NTHR)
+      S.items[i] = hot_group_first(i / P.pl.hp, P.pl) + i % P.pl.hp;
+  }
   __syncthreads();
   if (threadIdx.x >= NCT) {
     const int p = (threadIdx.x - NCT) >> 5;
@@ -1213,7 +1339,7 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.o_bw = o;         o = up16(o + 4u * bw);
   pl.o_mw = o;         o = up16(o + 4u * Wc);
   pl.o_scan = o;       o = up16(o + 4u * (NCW + 4));
-  pl.o_cold = o;       o = up16(o + 4u * pl.maxc);
+  pl.o_items = o;      o = up16(o + 4u * pl.maxi);
   pl.o_hval = o;       o = up16(o + 4u * pl.maxi);
   pl.o_flag = o;       o = up16(o + 4u * pl.maxi);
   pl.o_dlist = o;      o = up16(o + 4u * pl.maxi);
@@ -1228,19 +1354,12 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   if (avail <= 0) return false;
   int ns = avail / (int)sb;
   if (ns > NSMAX) ns = NSMAX;
-  // producer warps own every np-th stage: np must divide ns
-  if (ns >= 8) {
-    pl.np = 4;
-    ns -= ns % 4;
-  } else if (ns >= 4) {
-    pl.np = 2;
-    ns -= ns % 2;
-  } else if (ns >= 3) {
-    pl.np = 1;
-  } else {
-    return false;
-  }
+  if (ns < 3) return false;
+  // an even ring (a multiple of 4 when deep) lets the consumer groups divide it
+  if (ns >= 8) ns -= ns % 4;
+  else if (ns >= 4) ns -= ns % 2;
   pl.ns = ns;
+  pl.np = NPMAX;  // producer warp p owns the stages st with st % np == p
   // consumer groups must divide the ring depth (a stage is always consumed
   // by the same group); the down phase also needs every column to fit one
   // group's accumulators (64 floats per thread)
