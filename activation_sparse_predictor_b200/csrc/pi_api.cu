@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "pi.h"
 #include "pi_common.cuh"
@@ -242,6 +243,37 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
 }  // namespace
 }  // namespace pi
 
+// Scratch of pi_predict_noalloc: the predictor's hidden vector u for
+// batch * rank <= PI_PREDICT_NOALLOC_MAX_FLOATS, one copy per device (part of
+// the module image, so it takes no allocation at run time).
+static __device__ __align__(256) float g_predict_u[PI_PREDICT_NOALLOC_MAX_FLOATS];
+
+namespace pi {
+namespace {
+
+// Device address of g_predict_u on the current device.  Looked up once per
+// device, by the first pi_predict_noalloc call made with that device current.
+pi_status predict_scratch(float** out) {
+  static std::mutex mu;
+  static float* addr[64] = {};
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(PI_ERR_UNSUPPORTED, "device %d: at most 64 devices", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_predict_u);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress of the predictor scratch");
+    addr[dev] = static_cast<float*>(p);
+  }
+  *out = addr[dev];
+  return PI_OK;
+}
+
+}  // namespace
+}  // namespace pi
+
 using namespace pi;
 
 extern "C" {
@@ -290,6 +322,30 @@ pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float ta
   cudaError_t e = launch_pred_u(*layer, xh, batch, at<float>(ws, lay.u), s);
   if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
   e = launch_pred_z(*layer, at<float>(ws, lay.u), batch, logit32(tau), mask, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pred_z launch");
+  return PI_OK;
+}
+
+pi_status pi_predict_noalloc(const pi_layer* layer, const float* xh, int batch, float tau,
+                             uint32_t* mask, void* stream) {
+  pi_status st = check_layer(layer, 0);
+  if (st != PI_OK) return st;
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID, "batch %d not in [1, 64]", batch);
+  if (!(tau > 0.f && tau < 1.f)) return fail(PI_ERR_INVALID, "tau must lie in (0, 1)");
+  if (!xh || !aligned(xh, 16)) return fail(PI_ERR_INVALID, "xh null or not 16-byte aligned");
+  if (!mask || !aligned(mask, 4)) return fail(PI_ERR_INVALID, "mask null or misaligned");
+  const long long need = (long long)batch * layer->rank;
+  if (need > PI_PREDICT_NOALLOC_MAX_FLOATS)
+    return fail(PI_ERR_INVALID,
+                "pi_predict_noalloc: batch * rank = %lld exceeds its static scratch of %d floats; "
+                "use pi_predict with a workspace",
+                need, PI_PREDICT_NOALLOC_MAX_FLOATS);
+  float* u = nullptr;
+  if ((st = predict_scratch(&u)) != PI_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = launch_pred_u(*layer, xh, batch, u, s);
+  if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
+  e = launch_pred_z(*layer, u, batch, logit32(tau), mask, s);
   if (e != cudaSuccess) return cuda_fail(e, "pred_z launch");
   return PI_OK;
 }

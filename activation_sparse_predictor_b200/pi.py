@@ -13,6 +13,7 @@ import re
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpi.so")
+PI_PREDICT_NOALLOC_MAX_FLOATS = 262144  # include/pi.h
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "pi.h")
 
 PI_OK, PI_ERR_INVALID, PI_ERR_UNSUPPORTED, PI_ERR_CUDA, PI_ERR_TIMEOUT, PI_ERR_DEVICE_CHECK = range(6)
@@ -53,6 +54,7 @@ def _load():
         "pi_workspace_bytes": (sz, [L, i32, i32]),
         "pi_workspace_init": (i32, [vp, sz, vp]),
         "pi_predict": (i32, [L, vp, i32, f32, vp, vp, sz, vp]),
+        "pi_predict_noalloc": (i32, [L, vp, i32, f32, vp, vp]),
         "pi_compact": (i32, [vp, i32, i32, i32, i32, vp, vp, vp]),
         "pi_sparse_ffn": (i32, [L, vp, i32, vp, vp, vp, i32, vp, vp, sz, vp]),
         "pi_ffn_stack": (i32, [L, i32, vp, i32, f32, i32, vp, vp, sz, vp]),
@@ -231,6 +233,16 @@ def pi_predict(layer: Layer, xh, tau: float, mask=None, ws=None, stream=None):
         ws = workspace([layer], batch, xh.device, stream)
     _check(_lib.pi_predict(ctypes.byref(layer.c), _ptr(xh), batch, tau, _ptr(mask), _ptr(ws),
                            ws.numel(), _stream(stream)))
+    return mask
+
+
+def pi_predict_noalloc(layer: Layer, xh, tau: float, mask, stream=None):
+    """pi_predict without a workspace: u lives in the library's static
+    per-device buffer (batch * rank <= PI_PREDICT_NOALLOC_MAX_FLOATS), so the
+    call allocates nothing; `mask` [batch][words] int32 is the caller's.
+    Calls whose GPU work overlaps on one device race on that buffer."""
+    _check(_lib.pi_predict_noalloc(ctypes.byref(layer.c), _ptr(xh), xh.shape[0], tau,
+                                   _ptr(mask), _stream(stream)))
     return mask
 
 

@@ -138,6 +138,29 @@ pi_status pi_workspace_init(void* ws, size_t ws_bytes, void* stream);
 pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float tau,
                      uint32_t* mask, void* ws, size_t ws_bytes, void* stream);
 
+/* pi_predict without a workspace: the same kernels, arguments and result
+ * (mask) as pi_predict, with u kept in a static buffer of the library, one
+ * per device, of PI_PREDICT_NOALLOC_MAX_FLOATS floats (1 MiB).  The method
+ * itself has no counterpart to this entry point; it exists for callers that
+ * must not allocate device memory: cudaMalloc and cudaFree synchronise the
+ * whole device (stalling every stream's work, which latency-bound serving
+ * loops avoid), and processes whose device memory is reserved up front by
+ * their own allocator have none to give to a workspace.
+ *   Limit: batch * rank <= PI_PREDICT_NOALLOC_MAX_FLOATS; larger calls
+ *          return PI_ERR_INVALID (use pi_predict with a workspace).
+ *   Set-up: the first call on each device, with that device current, looks
+ *          up the buffer's device address (cudaGetSymbolAddress); make that
+ *          first call before any stream capture.
+ *   Zeroing: nothing; every element of u is written before it is read.
+ *   Concurrency: the buffer is shared by all calls on a device, so calls
+ *          whose GPU work overlaps (e.g. on two streams with no ordering
+ *          between them) race on it and produce wrong masks; issue them on
+ *          one stream, or use pi_predict with a workspace per stream.
+ * Allocates nothing. */
+#define PI_PREDICT_NOALLOC_MAX_FLOATS 262144
+pi_status pi_predict_noalloc(const pi_layer* layer, const float* xh, int batch, float tau,
+                             uint32_t* mask, void* stream);
+
 /* Mask compaction: neuron ids j in [begin, d_ff) whose bit is set, in
  * ascending order, int32.  mask: [batch][ceil(d_ff/32)].
  *   PI_MASK_UNION    : one list over the OR of the batch's masks;
