@@ -21,9 +21,12 @@ layers, extrapolated to the whole stack.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import sys
 import threading
@@ -50,6 +53,8 @@ def parse():
     ap.add_argument("--mode", default="per_token", choices=["per_token", "union"])
     ap.add_argument("--cpu-sample-layers", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="run only the first N layers (profiling captures; 0 = all)")
     return ap.parse_args()
 
 
@@ -262,6 +267,36 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+PROFILES = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
+CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "activation_sparse_predictor_b200", "csrc")
+
+
+def kernel_source_sha256() -> str:
+    """Hash of the CUDA sources (csrc/*.cu, *.cuh) the library is built from."""
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
+        h.update(os.path.basename(f).encode())
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic_per_layer(workload: str):
+    """DRAM bytes (read + write) per layer of the fused kernel from the
+    committed ncu summary of this workload, or None when there is none or it
+    was taken on other kernel sources than the ones built now."""
+    path = os.path.join(PROFILES, f"fused_stack_{workload}_ncu.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        m = re.match(r"^- (source_sha256|dram_bytes_per_layer): `?([0-9a-fA-Fe.+]+)`?\s*$", line.strip())
+        if m:
+            vals[m.group(1)] = m.group(2)
+    if vals.get("source_sha256") != kernel_source_sha256() or "dram_bytes_per_layer" not in vals:
+        return None
+    return float(vals["dram_bytes_per_layer"])
+
+
 def workload_config(w, batch, mode):
     return {"workload": w.name, "layers": w.n_layers, "d_model": w.d_model, "d_ff": w.d_ff,
             "hot_prefix": w.hot, "predictor_rank": w.rank, "activation": w.act,
@@ -283,8 +318,9 @@ def run_pi(args, world, rank, local):
     w = synth.WORKLOADS[args.workload]
     B = args.batch
     mode = pi.MODES[args.mode]
+    nl = args.layers if 0 < args.layers < w.n_layers else w.n_layers
     layers = []
-    for l in range(w.n_layers):
+    for l in range(nl):
         t = synth.layer_device(w, l, dev)
         layers.append(pi.Layer.packed(
             w, {k: t[k] for k in ("w_gate", "w_up", "w_down_t", "bias", "p1", "p2", "p_bias")
@@ -335,7 +371,7 @@ def run_pi(args, world, rank, local):
     value = world * K * B / (ms_max / 1000.0)
 
     # bytes actually read per step (predictor + listed rows + nonzero down rows)
-    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * w.n_layers)
+    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * nl)
     step_bytes = sum(by.values()) / K
     peak, peak_kind = hbm_peak()
     step_gbs = step_bytes / (ms / K / 1000.0) / 1e9
@@ -345,15 +381,19 @@ def run_pi(args, world, rank, local):
     pi.pi_read_counters(ws, clear=True, stream=stream)
     prof = pi.pi_ffn_stack_profile(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
     pr_listed, pr_down = pi.pi_read_counters(ws, clear=True, stream=stream)
-    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, w.n_layers)
+    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, nl)
     pby["fused_stack"] = sum(pby.values())  # the fused kernel runs every step
     prof = {k: v for k, v in prof.items() if v[1] > 0}
     dom = max(prof, key=lambda k: prof[k][0])
     dom_ms, dom_n = prof[dom]
     achieved = pby[dom] / dom_n / (dom_ms / dom_n / 1000.0) / 1e9
+    # DRAM traffic per launch from the committed ncu capture of this kernel
+    # (per layer, scaled to the layers of an average launch); null when the
+    # capture was taken on other kernel sources
+    tpl = measured_traffic_per_layer(w.name) if dom == "fused_stack" else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
-                "traffic": None,
+                "traffic": tpl * nl / dom_n if tpl is not None else None,
                 "algorithmic_bytes_per_launch": pby[dom] / dom_n,
                 "avg_launch_us": 1000.0 * dom_ms / dom_n,
                 "per_kind_ms_per_step": {k: v[0] for k, v in prof.items()},
@@ -389,7 +429,8 @@ def run_pi(args, world, rank, local):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        tps, cores, s, desc = cpu_oracle_tokens_per_s(w, args.cpu_sample_layers, 2)
+        # ~10 s of oracle work: the sample layers, 24 passes
+        tps, cores, s, desc = cpu_oracle_tokens_per_s(w, args.cpu_sample_layers, 24)
         cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
 
     line = {
@@ -397,7 +438,7 @@ def run_pi(args, world, rank, local):
         "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded generator, weights generated on the GPU; no datasets)",
-        "config": dict(workload_config(w, B, args.mode),
+        "config": dict(workload_config(w, B, args.mode), layers=nl,
                        parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "hbm_gbs_actual": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
         "bytes_per_step": step_bytes,
