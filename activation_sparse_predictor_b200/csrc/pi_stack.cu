@@ -1,21 +1,22 @@
 // Persistent single-token decode kernel for the whole FFN stack (sm_100a).
 //
 // One cooperative launch runs a chunk of layers with one CTA per SM.  Each
-// CTA has four producer warps (one thread each) that stream every weight row
-// the CTA will use through a ring of shared-memory stages with 1-D bulk
+// CTA has three producer warps (one thread each) that stream every weight
+// row the CTA will use through a ring of shared-memory stages with 1-D bulk
 // copies (cp.async.bulk, completion counted on an mbarrier per stage; each
 // copy costs its thread a few hundred ns to issue, so the copies of
-// consecutive stages are issued by different threads), and sixteen consumer
-// warps in groups: a unit (stage) goes to one group, whose threads each take
-// a slice of its columns, so a stage is held only briefly and the ring keeps
-// many rows in flight.  Per layer:
+// consecutive stages are issued by different threads), a compaction warp,
+// and sixteen consumer warps in groups: a unit (stage) goes to one group,
+// whose threads each take a slice of its columns, so a stage is held only
+// briefly and the ring keeps many rows in flight.  Per layer:
 //
 //   x^  : every CTA normalises the full residual vector (rmsnorm) itself
 //   A   : predictor rows of P1 (a static share per CTA)   -> u      | grid barrier 1
 //   B   : predictor rows of P2 for the CTA's mask words   -> mask   | grid barrier 2 (arrive)
 //   C   : the CTA's hot neurons (j = s, s + SMs, ...)      -> h
-//         grid barrier 2 (wait), compaction of the mask in every CTA, the
-//         CTA's share of the ascending cold list (positions s, s + SMs, ...) -> h
+//         meanwhile the compaction warp waits for grid barrier 2 and builds
+//         the CTA's share of the ascending cold list (positions s, s + SMs, ...);
+//         then the cold neurons                            -> h
 //   D   : down rows of the CTA's neurons whose h != 0     -> partial y | grid barrier 3
 //   E   : fixed-order reduction of the CTA's column slice, residual add | grid barrier 4
 //
@@ -45,9 +46,8 @@ namespace {
 
 constexpr int NCW = 16;             // consumer warps
 constexpr int NCT = NCW * 32;       // consumer threads
-constexpr int NPMAX = 4;            // producer warps (after the consumers)
-constexpr int NTHR = NCT + 32 * NPMAX;
-static_assert((NPMAX & (NPMAX - 1)) == 0, "stage owner is st & (NPMAX - 1)");
+constexpr int NPMAX = 3;            // producer warps (after the consumers)
+constexpr int NTHR = NCT + 32 * (NPMAX + 1);  // + the compaction warp
 constexpr int NSMAX = 24;           // ring stages at most
 constexpr int MAXL = 24;            // layers per launch
 constexpr int GRP = 32;             // items per cross-warp finalisation group
@@ -464,7 +464,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   uint32_t l_uc0 = 0;  // first unit of the current layer
 
   // Stage st belongs to producer st % NPMAX.
-  auto mine = [&]() { return (cu.st & (NPMAX - 1)) == p; };
+  auto mine = [&]() { return cu.st % NPMAX == p; };
   // Claims the current unit's stage (one of ours) and arms its full barrier for `bytes`.
   auto claim = [&](uint32_t bytes) -> char* {
     const int st = cu.st;
@@ -609,6 +609,72 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         break;
       }
     }
+  }
+}
+
+// --------------------------------------------------------------- compaction
+
+// One warp: after grid barrier 2 of each layer (every CTA's mask words are
+// out), the CTA's share of the ascending cold list: list position p (the
+// p-th set cold bit over the whole mask) belongs to CTA p mod SMs, slot
+// p / SMs.  A mask word holds at most 32 < SMs positions, so it holds at most
+// one of this CTA's.  Runs while the consumers are still on the hot items,
+// so the producers can copy the first cold records as soon as stages free.
+template <int WT, int ACT, int PT>
+__device__ void compactor(const StackParams& P, const Smem& S) {
+  const Plan& pl = P.pl;
+  WsHeader* hdr = P.hdr;
+  const Ranges R = ranges(pl);
+  const int lane = threadIdx.x & 31, nS = gridDim.x, s = blockIdx.x;
+  const int per = (R.W - R.Wlo + 31) / 32;  // mask words per lane
+  const int wa = R.Wlo + lane * per, wb = min(wa + per, R.W);
+  for (int l = 0; l < P.n_layers; ++l) {
+    const LayerPtrs& L = P.L[l];
+    const uint32_t* mask = P.mask + (size_t)l * P.mask_stride;
+    int ok = 1;
+    if (lane == 0) ok = grid_wait(hdr, (uint32_t)(4 * l + 2) * (uint32_t)nS, S) ? 1 : 0;
+    __syncwarp();  // lane 0's acquire orders the mask reads below
+    if (!__shfl_sync(0xffffffffu, ok, 0)) return;
+    int cnt = 0;
+    for (int w = wa; w < wb; ++w) {
+      uint32_t m = __ldcg(mask + w);
+      const int lo = 32 * w;
+      if (pl.H > lo) m &= (pl.H - lo >= 32) ? 0u : (~0u << (pl.H - lo));
+      S.mw[w - R.Wlo] = m;
+      cnt += __popc(m);
+    }
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    const int p = incl - cnt;  // list position of this lane's first neuron
+    int r = p % nS, q = p / nS;
+    for (int w = wa; w < wb; ++w) {
+      uint32_t m = S.mw[w - R.Wlo];
+      const int c = __popc(m);
+      const int k = r <= s ? s - r : nS - r + s;  // offset of this CTA's position
+      if (k < c) {
+        for (int t = 0; t < k; ++t) m &= m - 1u;
+        const int j = 32 * w + __ffs(m) - 1;
+        const int slot = q + (r + k >= nS ? 1 : 0);
+        S.items[R.nh + slot] = j;
+        S.hbs[R.nh + slot] = L.bias ? L.bias[j] : 0.f;
+      }
+      r += c;
+      if (r >= nS) {
+        r -= nS;
+        ++q;
+      }
+    }
+    if (lane == 0) {
+      *S.nc = total > s ? (total - s + nS - 1) / nS : 0;
+      if (s == 0) __stcg(P.count, total);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(S.listbar, 1u);  // releases the list to the CTA
   }
 }
 
@@ -961,64 +1027,10 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     if (fin < R.nh) finalise(R.nh);
     if (tid == 0) tstamp(P, l, 5, gtime());
 
-    // ---- compaction (every CTA, after barrier 2): its share of the list
-    gsync_wait();
+    // ---- the CTA's share of the cold list, built by the compaction warp
+    // once every CTA's mask words are out (grid barrier 2)
+    const int nc = wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr) ? *S.nc : 0;
     if (tid == 0) tstamp(P, l, 6, gtime());
-    {
-      const int Wc = R.W - R.Wlo;
-      const int per = (Wc + NCT - 1) / NCT;
-      const int wa = R.Wlo + tid * per, wb = min(R.Wlo + (tid + 1) * per, R.W);
-      int cnt = 0;
-      for (int w = wa; w < wb; ++w) {
-        uint32_t m = __ldcg(mask + w);
-        const int lo = 32 * w;
-        if (pl.H > lo) m &= (pl.H - lo >= 32) ? 0u : (~0u << (pl.H - lo));
-        S.mw[w - R.Wlo] = m;
-        cnt += __popc(m);
-      }
-      int incl = cnt;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += t;
-      }
-      if (lane == 31) S.scan[warp] = incl;
-      csync();
-      int wpre = 0, total = 0;
-#pragma unroll
-      for (int w = 0; w < NCW; ++w) {
-        const int v = S.scan[w];
-        if (w < warp) wpre += v;
-        total += v;
-      }
-      // list position p = wpre + incl - cnt of this thread's first neuron goes
-      // to CTA p % nS, slot p / nS; both advance without dividing again
-      const int p = wpre + incl - cnt;
-      int r = p % nS, q = p / nS;
-      for (int w = wa; w < wb; ++w) {
-        uint32_t m = S.mw[w - R.Wlo];
-        while (m) {
-          const int bit = __ffs(m) - 1;
-          m &= m - 1u;
-          if (r == s) {
-            const int j = 32 * w + bit;
-            S.items[R.nh + q] = j;
-            S.hbs[R.nh + q] = L.bias ? L.bias[j] : 0.f;
-          }
-          if (++r == nS) {
-            r = 0;
-            ++q;
-          }
-        }
-      }
-      if (tid == 0) {
-        *S.nc = total > s ? (total - s + nS - 1) / nS : 0;
-        if (s == 0) __stcg(P.count, total);
-      }
-      csync();
-      if (lane == 0) mbar_arrive(S.listbar, 1u);
-    }
-    const int nc = *S.nc;
     for (int i = R.nh; i < R.nh + nc; ++i) unit_items(i, 1);
     if (fin < R.nh + nc) finalise(R.nh + nc);
     csync();
@@ -1219,7 +1231,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
       mbar_init(&S.full[i], 1u);
       mbar_init(&S.empty[i], (uint32_t)NCW);
     }
-    mbar_init(S.listbar, (uint32_t)NCW);
+    mbar_init(S.listbar, 1u);
     *S.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1233,7 +1245,11 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
   __syncthreads();
   if (threadIdx.x >= NCT) {
     const int p = (threadIdx.x - NCT) >> 5;
-    if ((threadIdx.x & 31) == 0 && p < P.pl.np) producer<WT, ACT, PT>(P, S, p);
+    if (p < P.pl.np) {
+      if ((threadIdx.x & 31) == 0) producer<WT, ACT, PT>(P, S, p);
+    } else if (p == NPMAX) {
+      compactor<WT, ACT, PT>(P, S);
+    }
     return;
   }
   consumers<WT, ACT, PT>(P, S);
@@ -1359,7 +1375,7 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   if (ns >= 8) ns -= ns % 4;
   else if (ns >= 4) ns -= ns % 2;
   pl.ns = ns;
-  pl.np = NPMAX;  // producer warp p owns the stages st with st % np == p
+  pl.np = NPMAX;  // producer warp p owns the stages st with st % NPMAX == p
   // consumer groups must divide the ring depth (a stage is always consumed
   // by the same group); the down phase also needs every column to fit one
   // group's accumulators (64 floats per thread)
