@@ -635,14 +635,25 @@ __device__ void compactor(const StackParams& P, const Smem& S) {
     if (lane == 0) ok = grid_wait(hdr, (uint32_t)(4 * l + 2) * (uint32_t)nS, S) ? 1 : 0;
     __syncwarp();  // lane 0's acquire orders the mask reads below
     if (!__shfl_sync(0xffffffffu, ok, 0)) return;
-    int cnt = 0;
-    for (int w = wa; w < wb; ++w) {
-      uint32_t m = __ldcg(mask + w);
-      const int lo = 32 * w;
-      if (pl.H > lo) m &= (pl.H - lo >= 32) ? 0u : (~0u << (pl.H - lo));
-      S.mw[w - R.Wlo] = m;
-      cnt += __popc(m);
+    // every cold mask word into shared memory: coalesced, 8 loads in flight per lane
+    const int Wc = R.W - R.Wlo;
+    for (int k0 = 0; k0 < Wc; k0 += 256) {
+      uint32_t v[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int k = k0 + 32 * t + lane;
+        v[t] = k < Wc ? __ldcg(mask + R.Wlo + k) : 0u;
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int k = k0 + 32 * t + lane;
+        const int lo = 32 * (R.Wlo + k);
+        if (k < Wc) S.mw[k] = pl.H > lo ? (pl.H - lo >= 32 ? 0u : v[t] & (~0u << (pl.H - lo))) : v[t];
+      }
     }
+    __syncwarp();
+    int cnt = 0;
+    for (int w = wa; w < wb; ++w) cnt += __popc(S.mw[w - R.Wlo]);
     int incl = cnt;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
