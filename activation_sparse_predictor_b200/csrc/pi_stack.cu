@@ -54,6 +54,7 @@ constexpr int GRP = 32;             // items per cross-warp finalisation group
 constexpr int MAXA = 16;            // P1 rows per CTA at most
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int UTR = 512;            // units per layer recorded by the unit trace
+constexpr int DRMAX = 16;           // down rows per unit at most
 
 struct LayerPtrs {
   const char* first;            // W_gate (ReGLU) or W_up (ReLU): codes / rows
@@ -76,7 +77,7 @@ struct Plan {
   int np;                           // producer warps
   int gw, gd;                       // consumer warp groups: up-projection / down phases
   int hp;                           // hot neurons per unit (adjacent records)
-  int dr;                           // down rows per unit at most (adjacent records)
+  int dr;                           // down rows per unit (the last one of a layer: fewer)
   int packed_up, packed_down;       // neuron records contiguous in memory
   long long up_stride, down_stride; // bytes between consecutive neurons' rows (codes)
   long long up_sstride, down_sstride; // the same for Q4_0 scales
@@ -86,7 +87,7 @@ struct Plan {
   uint32_t item_bytes, down_bytes;  // bytes copied per item / per down row
   uint32_t o_first_s, o_second, o_second_s, o_down_s;  // offsets inside a stage
   uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_mw, o_scan, o_items, o_hval, o_flag,
-      o_dlist, o_runs, o_pbs, o_hbs, o_redA, o_redC, o_redE, o_ring, total;
+      o_dlist, o_pbs, o_hbs, o_redA, o_redC, o_redE, o_ring, total;
 };
 
 struct StackParams {
@@ -293,7 +294,6 @@ struct Smem {
   float* hval;
   volatile int* flag;
   int* dlist;
-  int* runs;                  // down-row units: first dlist position, row count
   float* pbs;                 // predictor biases of the CTA's mask words
   float* hbs;                 // activation biases of the CTA's items
   float* redA;
@@ -322,7 +322,6 @@ __device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
   S.hval = reinterpret_cast<float*>(base + pl.o_hval);
   S.flag = reinterpret_cast<volatile int*>(base + pl.o_flag);
   S.dlist = reinterpret_cast<int*>(base + pl.o_dlist);
-  S.runs = reinterpret_cast<int*>(base + pl.o_runs);
   S.pbs = reinterpret_cast<float*>(base + pl.o_pbs);
   S.hbs = reinterpret_cast<float*>(base + pl.o_hbs);
   S.redA = reinterpret_cast<float*>(base + pl.o_redA);
@@ -440,12 +439,9 @@ struct Cursor {
   }
 };
 
-// Down-row units: runs of consecutive nonzero items whose neurons are
-// adjacent (when down records are packed), at most pl.dr rows each.  The
-// producers and the consumers apply this rule to the same sequence.
-__device__ __forceinline__ bool run_extends(int jprev, int jnext, int len, const Plan& pl) {
-  return pl.packed_down && jnext == jprev + 1 && len < pl.dr;
-}
+// Down-row units: the rows of consecutive nonzero items in item order, pl.dr
+// per unit (the last unit of a layer holds the rest).  The producers and the
+// consumers apply this rule to the same sequence.
 
 // ---------------------------------------------------------------- producer
 
@@ -509,18 +505,26 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
     }
     cu.next(pl.ns);
   };
-  // Down records of neurons j0 .. j0+n-1.
-  auto downs = [&](const LayerPtrs& L, int j0, int n) {
+  // Down records of the neurons uj[0 .. n) into one stage, row k at
+  // k * down_bytes; adjacent packed records share one copy.
+  auto downs = [&](const LayerPtrs& L, const int* uj, int n) {
     if (mine()) {
       char* dst = claim(pl.down_bytes * (uint32_t)n);
       if (dst) {
         uint64_t* b = bar_of();
-        if (pl.packed_down) {
-          bulk_g2s(dst, L.down + (size_t)j0 * pl.down_stride, pl.down_bytes * (uint32_t)n, b);
-        } else {
-          bulk_g2s(dst, L.down + (size_t)j0 * pl.down_stride, pl.rowb, b);
-          if constexpr (WT == PI_Q4_0)
-            bulk_g2s(dst + pl.o_down_s, L.down_scales + (size_t)j0 * pl.down_sstride, pl.scb, b);
+        for (int k = 0; k < n;) {
+          int m = 1;
+          if (pl.packed_down)
+            while (k + m < n && uj[k + m] == uj[k] + m) ++m;
+          char* d = dst + (size_t)k * pl.down_bytes;
+          if (pl.packed_down) {
+            bulk_g2s(d, L.down + (size_t)uj[k] * pl.down_stride, pl.down_bytes * (uint32_t)m, b);
+          } else {
+            bulk_g2s(d, L.down + (size_t)uj[k] * pl.down_stride, pl.rowb, b);
+            if constexpr (WT == PI_Q4_0)
+              bulk_g2s(d + pl.o_down_s, L.down_scales + (size_t)uj[k] * pl.down_sstride, pl.scb, b);
+          }
+          k += m;
         }
       }
     }
@@ -564,9 +568,9 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
     }
     const int nc = *S.nc;
     for (int i = 0; i < nc && ok; ++i) items(L, S.items[R.nh + i], 1);
-    // D: down rows of items whose h != 0, in item order, as runs
+    // D: down rows of items whose h != 0, in item order, pl.dr per unit
     const int tag = (l + 1) << 2;
-    int rj = -1, rlen = 0;  // open run: first neuron, rows
+    int uj[DRMAX], un = 0;  // the open unit's neurons
     for (int i = 0; i < R.nh + nc && ok; ++i) {
       int f = S.flag[i];
       if ((f & ~3) != tag) {
@@ -580,16 +584,13 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         if (!ok) break;
       }
       if ((f & 3) != 2) continue;
-      const int j = S.items[i];
-      if (rlen > 0 && run_extends(rj + rlen - 1, j, rlen, pl)) {
-        ++rlen;
-        continue;
+      uj[un++] = S.items[i];
+      if (un == pl.dr) {
+        downs(L, uj, un);
+        un = 0;
       }
-      if (rlen > 0) downs(L, rj, rlen);
-      rj = j;
-      rlen = 1;
     }
-    if (ok && rlen > 0) downs(L, rj, rlen);
+    if (ok && un > 0) downs(L, uj, un);
     if (P.trace && p == 0) {
       tstamp(P, l, 12, w_empty);
       tstamp(P, l, 13, w_list);
@@ -1047,9 +1048,9 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     csync();
     if (tid == 0) tstamp(P, l, 7, gtime());
 
-    // ---- D: down rows of items with h != 0; each unit (a run of adjacent
-    // neurons' rows) shared by one of GD warp groups, each group covering
-    // every column with its own accumulators
+    // ---- D: down rows of items with h != 0, pl.dr rows per unit, each unit
+    // shared by one of GD warp groups, each group covering every column with
+    // its own accumulators
     const int ni = R.nh + nc;
     if (warp == 0) {
       int base = 0;
@@ -1060,27 +1061,11 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         if (nz) S.dlist[base + __popc(bal & ((1u << lane) - 1u))] = i;
         base += __popc(bal);
       }
-      __syncwarp();
-      if (lane == 0) {
-        int nr = 0, jp = -1, len = 0;
-        for (int q = 0; q < base; ++q) {
-          const int j = S.items[S.dlist[q]];
-          if (len > 0 && run_extends(jp, j, len, pl)) {
-            ++len;
-          } else {
-            if (len > 0) S.runs[2 * nr++ + 1] = len;
-            S.runs[2 * nr] = q;
-            len = 1;
-          }
-          jp = j;
-        }
-        if (len > 0) S.runs[2 * nr++ + 1] = len;
-        S.scan[NCW] = base;
-        S.scan[NCW + 1] = nr;
-      }
+      if (lane == 0) S.scan[NCW] = base;
     }
     csync();
-    const int nd = S.scan[NCW], nruns = S.scan[NCW + 1];
+    const int nd = S.scan[NCW];
+    const int nruns = (nd + pl.dr - 1) / pl.dr;  // units of pl.dr rows
     if constexpr (WT == PI_Q4_0) {
       // one Q4_0 block (32 columns) per thread (the plan keeps d / 32 within
       // a group).  sum_j hs_j (q - 8), hs_j = h_j * scale, is accumulated as
@@ -1094,7 +1079,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
         if ((int)(cu.uc & gdm) != dgrp) continue;
         if (!ready()) continue;
-        const int q0 = S.runs[2 * q], len = S.runs[2 * q + 1];
+        const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
         if (c < nch) {
 #pragma unroll 2
           for (int rr = 0; rr < len; ++rr) {
@@ -1143,7 +1128,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
         if ((int)(cu.uc & gdm) != dgrp) continue;
         if (!ready()) continue;
-        const int q0 = S.runs[2 * q], len = S.runs[2 * q + 1];
+        const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
         for (int rr = 0; rr < len; ++rr) {
           const char* row = stage() + (size_t)rr * pl.down_bytes;
           const float hv = S.hval[S.dlist[q0 + rr]];
@@ -1347,7 +1332,8 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   sb = sb > pl.p2_row ? sb : pl.p2_row;
   sb = up128(sb);
   pl.sb = sb;
-  pl.dr = pl.packed_down ? (int)(sb / pl.down_bytes) : 1;
+  pl.dr = (int)(sb / pl.down_bytes);
+  if (pl.dr > DRMAX) pl.dr = DRMAX;
   if (pl.dr < 1) pl.dr = 1;
   int G = 32;
   while (G > 1 && (uint32_t)G * pl.p2_row > sb) G >>= 1;
@@ -1370,7 +1356,6 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.o_hval = o;       o = up16(o + 4u * pl.maxi);
   pl.o_flag = o;       o = up16(o + 4u * pl.maxi);
   pl.o_dlist = o;      o = up16(o + 4u * pl.maxi);
-  pl.o_runs = o;       o = up16(o + 8u * pl.maxi);
   pl.o_pbs = o;        o = up16(o + 4u * 32u * bw);
   pl.o_hbs = o;        o = up16(o + 4u * pl.maxi);
   pl.o_redA = o;       o = up16(o + 4u * (MAXA + MAXA * NCW));
