@@ -10,6 +10,7 @@
 #include "pi_common.cuh"
 #include "pi_kernels.cuh"
 #include "pi_stack.cuh"
+#include "pi_tc.cuh"
 
 namespace pi {
 namespace {
@@ -79,7 +80,7 @@ pi_status check_layer(const pi_layer* L, int i) {
   return PI_OK;
 }
 
-WsLayout layout_for(int d, int F, int r, int batch) {
+WsLayout layout_for(int d, int F, int r, int batch, int H) {
   WsLayout w{};
   size_t off = sizeof(WsHeader);
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
@@ -97,18 +98,20 @@ WsLayout layout_for(int d, int F, int r, int batch) {
                            : 2 * (size_t)device_sms();
   w.part = take(parts * d * 4);
   w.y = take((size_t)batch * d * 4);
+  w.tc = take(hot_tc_scratch_bytes(d, H, batch));
   w.total = off;
   return w;
 }
 
 WsLayout layout_for_layers(const pi_layer* layers, int n, int batch) {
-  int d = 0, F = 0, r = 0;
+  int d = 0, F = 0, r = 0, H = 0;
   for (int l = 0; l < n; ++l) {
     d = d > layers[l].d_model ? d : layers[l].d_model;
     F = F > layers[l].d_ff ? F : layers[l].d_ff;
     r = r > layers[l].rank ? r : layers[l].rank;
+    H = H > layers[l].hot ? H : layers[l].hot;
   }
-  return layout_for(d, F, r, batch);
+  return layout_for(d, F, r, batch, H);
 }
 
 pi_status check_ws(void* ws, size_t ws_bytes, const WsLayout& lay) {
@@ -152,8 +155,16 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
   Prof none;
   Prof& P = prof ? *prof : none;
   P.before(PI_KIND_FFN_UP);
-  cudaError_t e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h),
-                                header(ws), s);
+  cudaError_t e = cudaSuccess;
+  int n0 = 0;  // first list position left to the CUDA-core kernel
+  if (hot_tc_supported(L, batch)) {
+    // the dense hot prefix on the tensor cores, the listed cold rows after it
+    e = launch_hot_up_tc(L, xh, batch, at<float>(ws, lay.h), at<void>(ws, lay.tc), header(ws), s);
+    if (e != cudaSuccess) return cuda_fail(e, "hot prefix (tensor cores) launch");
+    n0 = L.hot;
+  }
+  e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h), header(ws), s,
+                    n0);
   P.after();
   if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
   const int S = down_splits(batch, L.d_model);

@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
                                                      int per_token, int words,
                                                      const int32_t* __restrict__ idx,
                                                      const int32_t* __restrict__ count,
-                                                     float* __restrict__ h, WsHeader* hdr) {
+                                                     float* __restrict__ h, WsHeader* hdr,
+                                                     int n0) {
   extern __shared__ __align__(16) float sx[];
   uint32_t* status = hdr ? &hdr->status : nullptr;
   const int d = L.d_model, F = L.d_ff, H = L.hot;
@@ -306,7 +307,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
   const int nch = d / CC;
   const int64_t rb = code_stride(WT, d, L.w_row_stride);
   const int64_t sbs = scale_stride(d, L.w_row_stride);
-  for (int n = blockIdx.x * kWarps + warp; n < N; n += gridDim.x * kWarps) {
+  // list positions n0 .. N-1 (n0 = H when the hot rows are computed elsewhere)
+  for (int n = n0 + blockIdx.x * kWarps + warp; n < N; n += gridDim.x * kWarps) {
     const int j = n < H ? n : idx[n - H];
     if (j < H && n >= H || j >= F || j < 0) {
       if (lane == 0) {
@@ -580,36 +582,36 @@ cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin,
 template <int WT, int ACT, int TB>
 static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                             int per_token, const int32_t* idx, const int32_t* count, float* h,
-                            WsHeader* status, cudaStream_t s) {
+                            WsHeader* status, cudaStream_t s, int n0) {
   const size_t smem = (size_t)TB * L.d_model * 4;
   auto kern = k_ffn_up<WT, ACT, TB>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(std::min((L.d_ff + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
   kern<<<grid, kThreads, smem, s>>>(L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
-                                    count, h, status);
+                                    count, h, status, n0);
   return cudaGetLastError();
 }
 
 template <int WT, int ACT>
 static cudaError_t ffn_up_a(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                             int per_token, const int32_t* idx, const int32_t* count, float* h,
-                            WsHeader* status, cudaStream_t s) {
+                            WsHeader* status, cudaStream_t s, int n0) {
   switch (pick_tb(batch, L.d_model)) {
-    case 1: return ffn_up_t<WT, ACT, 1>(L, xh, batch, mask, per_token, idx, count, h, status, s);
-    case 2: return ffn_up_t<WT, ACT, 2>(L, xh, batch, mask, per_token, idx, count, h, status, s);
-    case 4: return ffn_up_t<WT, ACT, 4>(L, xh, batch, mask, per_token, idx, count, h, status, s);
-    default: return ffn_up_t<WT, ACT, 8>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+    case 1: return ffn_up_t<WT, ACT, 1>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
+    case 2: return ffn_up_t<WT, ACT, 2>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
+    case 4: return ffn_up_t<WT, ACT, 4>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
+    default: return ffn_up_t<WT, ACT, 8>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
   }
 }
 
 cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                           int per_token, const int32_t* idx, const int32_t* count, float* h,
-                          WsHeader* status, cudaStream_t s) {
-#define PI_UP(WT)                                                                              \
-  return L.act == PI_REGLU                                                                     \
-             ? ffn_up_a<WT, PI_REGLU>(L, xh, batch, mask, per_token, idx, count, h, status, s) \
-             : ffn_up_a<WT, PI_RELU>(L, xh, batch, mask, per_token, idx, count, h, status, s);
+                          WsHeader* status, cudaStream_t s, int n0) {
+#define PI_UP(WT)                                                                                  \
+  return L.act == PI_REGLU                                                                         \
+             ? ffn_up_a<WT, PI_REGLU>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0) \
+             : ffn_up_a<WT, PI_RELU>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
   if (L.w_dtype == PI_F32) { PI_UP(PI_F32) }
   if (L.w_dtype == PI_F16) { PI_UP(PI_F16) }
   PI_UP(PI_Q4_0)

@@ -35,7 +35,7 @@ cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin,
 // h[n][b] for rows n of [0,hot) U idx[0..count)
 cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                           int per_token, const int32_t* idx, const int32_t* count, float* h,
-                          WsHeader* hdr, cudaStream_t s);
+                          WsHeader* hdr, cudaStream_t s, int n0 = 0);
 
 // part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n]
 cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,

@@ -1,0 +1,392 @@
+// Dense hot prefix at token batches on the tensor cores (sm_100a).
+//
+// The hot neurons [0, hot) run for every token, so at 16-64 tokens their
+// gate/up products are a real contraction: D[n][t] = sum_k W[n][k] xh[t][k]
+// for 128 hot neurons n per tile and all tokens t.  The weight rows are the
+// MMA's A operand exactly as stored (M = 128, K-major), an fp16 copy of the
+// normalised inputs is its B operand (N = tokens padded to 16, K-major), and
+// the fp32 accumulators live in tensor memory:
+//
+//   warp 0, one thread : TMA 2-D tile loads (128-byte swizzle) into a ring of
+//                        4 stages, completion on a full mbarrier per stage
+//   warp 1, one thread : tcgen05.mma (kind::f16, 4 per 64-wide stage), then
+//                        tcgen05.commit to the stage's empty mbarrier
+//   all 4 warps        : tcgen05.ld of their 32 accumulator lanes -> fp32
+//                        partial sums in the workspace
+//
+// d is split over up to 4 CTAs per tile so that about one CTA per SM
+// streams weights; a second kernel sums the splits in a fixed order, adds
+// the bias and applies ReLU / ReGLU, writing h as the CUDA-core kernels do.
+// Every mbarrier wait is bounded by %globaltimer (1 s): a wait that runs out
+// sets DEV_TIMEOUT in the workspace status word and a CTA abort flag, the
+// producer waits (bounded) for its own copies in flight, and the tensor
+// memory is always freed before the CTA exits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <mutex>
+
+#include "pi_kernels.cuh"
+#include "pi_tc.cuh"
+
+namespace pi {
+namespace {
+
+constexpr int TC_M = 128;        // hot neurons per tile (MMA M)
+constexpr int TC_BK = 64;        // k per stage: one 128-byte swizzle atom of fp16
+constexpr int TC_STAGES = 4;
+constexpr int TC_THREADS = 128;
+constexpr int TC_KSMAX = 4;      // CTAs sharing one tile's d at most
+constexpr int TC_TMAX = 64;      // tokens at most (MMA N)
+constexpr unsigned long long kTcTimeoutNs = 1000000000ull;
+
+__device__ __forceinline__ uint32_t tc_sa(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint64_t tc_time() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool tc_try(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(tc_sa(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of `bar`; false after an abort or a
+// timeout (which raises the abort and the status bit).
+__device__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, WsHeader* hdr) {
+  if (tc_try(bar, parity)) return true;
+  const uint64_t t0 = tc_time();
+  while (!tc_try(bar, parity)) {
+    if (*abort) return false;
+    if (tc_time() - t0 > kTcTimeoutNs) {
+      *abort = 1;
+      if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Shared-memory matrix descriptor of a K-major tile with 128-byte swizzle:
+// rows of 128 bytes, 8-row atoms 1024 bytes apart (stride byte offset),
+// leading byte offset unused (1), descriptor version 1, layout 2 (128B).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// D (tensor memory) [+]= A * B^T for one K = 16 slice, issued by one thread.
+__device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0));
+}
+
+// Arrives on `bar` once every tcgen05.mma this thread issued has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   tc_sa(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(tc_sa(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(tc_sa(bar))
+      : "memory");
+}
+
+// NR = 1: ReLU (W_up); NR = 2: ReGLU (W_gate, W_up).  Grid (hot / 128, ks).
+// part: [ks][NR][hot][nt] fp32.
+template <int NR>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_hot_up_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
+                const __grid_constant__ CUtensorMap mx, int nt, int nk, int ks, int H,
+                float* __restrict__ part, WsHeader* hdr) {
+  constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
+  constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB (nt rows used)
+  constexpr uint32_t STAGE = NR * A_BYTES + B_BYTES;
+  constexpr uint32_t NCOLS = NR == 1 ? 64u : 128u;   // >= NR * nt, a power of two
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = tc_sa(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // swizzle atoms: 1 KB aligned
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_STAGES * STAGE);
+  uint64_t* empty = full + TC_STAGES;
+  uint64_t* done = empty + TC_STAGES;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
+  const int nkt = kt1 - kt0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TC_STAGES; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(done)) : "memory");
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     tc_sa(tslot)),
+                 "r"(NCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0 && lane == 0) {
+    // producer: k tiles kt0 .. kt1-1 of the tile's weight rows and of xh16
+    const uint32_t tx = NR * A_BYTES + (uint32_t)nt * TC_BK * 2;
+    int last[TC_STAGES];
+    for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % TC_STAGES;
+      if (i >= TC_STAGES && !tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr)) break;
+      unsigned char* a = smem + st * STAGE;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
+                   "r"(tx)
+                   : "memory");
+      const int k = (kt0 + i) * TC_BK;
+      tma_load_2d(a, &mw0, k, tile * TC_M, &full[st]);
+      if constexpr (NR == 2) tma_load_2d(a + A_BYTES, &mw1, k, tile * TC_M, &full[st]);
+      tma_load_2d(a + NR * A_BYTES, &mx, k, 0, &full[st]);
+      last[st] = i;
+    }
+    // every copy issued here has landed before the CTA may exit (bounded)
+    for (int st = 0; st < TC_STAGES; ++st) {
+      if (last[st] < 0) continue;
+      const uint32_t par = (uint32_t)(last[st] / TC_STAGES) & 1u;
+      const uint64_t t0 = tc_time();
+      while (!tc_try(&full[st], par)) {
+        if (tc_time() - t0 > kTcTimeoutNs) {
+          if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer: kind::f16, fp16 A and B, fp32 D, both K-major, M = 128, N = nt
+    const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % TC_STAGES;
+      if (!tc_wait(&full[st], (uint32_t)(i / TC_STAGES) & 1u, abort, hdr)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = tc_sa(smem + st * STAGE), b = a + NR * A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk) {  // 32 bytes of K per MMA inside the atom
+        const uint64_t bd = sw128_desc(b + 32u * kk);
+        const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+        mma_f16(tmem, sw128_desc(a + 32u * kk), bd, idesc, acc);
+        if constexpr (NR == 2) mma_f16(tmem + (uint32_t)nt, sw128_desc(a + A_BYTES + 32u * kk), bd, idesc, acc);
+      }
+      mma_commit(&empty[st]);  // the stage is free once these products have read it
+    }
+    mma_commit(done);  // the accumulators are final (after an abort: quiescent)
+  }
+  __syncwarp();
+
+  // epilogue: warp w holds accumulator lanes [32w, 32w + 32) = hot neurons
+  // tile * 128 + 32w + lane, one column per token
+  // wait for `done` even after an abort: the MMA thread always commits it, so
+  // no product is still writing tensor memory when it is freed below
+  bool ok = tc_try(done, 0u);
+  if (!ok) {
+    const uint64_t t0 = tc_time();
+    while (!(ok = tc_try(done, 0u))) {
+      if (tc_time() - t0 > kTcTimeoutNs) {
+        if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
+        break;
+      }
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (ok) {
+    const int n = tile * TC_M + warp * 32 + lane;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      float* dst = part + ((size_t)(split * NR + r) * H + n) * nt;
+      for (int c0 = 0; c0 < nt; c0 += 16) {
+        uint32_t v[16];
+        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(r * nt + c0);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+            "%11, %12, %13, %14, %15}, [%16];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+              "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+              "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          __stcg(reinterpret_cast<float4*>(dst + c0) + q,
+                 make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS)
+                 : "memory");
+}
+
+// xh (fp32 [batch][d]) -> xh16 (fp16 [nt][d], rows >= batch zero); 8 per thread.
+__global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
+                       __half* __restrict__ xh16) {
+  const int n8 = d / 8;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt * n8; i += gridDim.x * blockDim.x) {
+    const int t = i / n8, c = i % n8;
+    uint4 o = make_uint4(0u, 0u, 0u, 0u);
+    if (t < batch) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(xh + (size_t)t * d) + 2 * c);
+      const float4 b = __ldg(reinterpret_cast<const float4*>(xh + (size_t)t * d) + 2 * c + 1);
+      const __half2 h0 = __floats2half2_rn(a.x, a.y), h1 = __floats2half2_rn(a.z, a.w);
+      const __half2 h2 = __floats2half2_rn(b.x, b.y), h3 = __floats2half2_rn(b.z, b.w);
+      o = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                     *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+    }
+    reinterpret_cast<uint4*>(xh16 + (size_t)t * d)[c] = o;
+  }
+}
+
+// h[n * batch + b] = act(sum over splits (fixed order) + bias) for n < H.
+template <int NR>
+__global__ void k_hot_finish(const float* __restrict__ part, int ks, int H, int nt, int batch,
+                             const float* __restrict__ bias, float* __restrict__ h) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H * batch; i += gridDim.x * blockDim.x) {
+    const int n = i / batch, b = i % batch;
+    float g = 0.f, u = 0.f;
+    for (int s = 0; s < ks; ++s) {
+      g += __ldcg(part + ((size_t)(s * NR) * H + n) * nt + b);
+      if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * H + n) * nt + b);
+    }
+    g += bias ? bias[n] : 0.f;
+    float hv = g > 0.f ? g : 0.f;
+    if constexpr (NR == 2) hv *= u;
+    h[(size_t)n * batch + b] = hv;
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static std::mutex mu;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D fp16 tensor [rows][inner] with `row_bytes` between rows; box
+// [box_rows][64], 128-byte swizzle.
+bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+            uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)TC_BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool tc_disabled() {
+  const char* e = getenv("PI_DISABLE_TC");
+  return e && e[0] && e[0] != '0';
+}
+
+size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+template <int NR>
+cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, void* scratch,
+                      WsHeader* hdr, cudaStream_t s) {
+  const int d = L.d_model, H = L.hot;
+  const int nt = (batch + 15) / 16 * 16;
+  __half* xh16 = static_cast<__half*>(scratch);
+  float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + up256((size_t)TC_TMAX * d * 2));
+  const int64_t rs = code_stride(PI_F16, d, L.w_row_stride);
+  CUtensorMap m0, m1, mx;
+  const void* w0 = NR == 2 ? L.w_gate : L.w_up;
+  if (!map_2d(&m0, w0, (uint64_t)d, (uint64_t)H, (uint64_t)rs, TC_M) ||
+      !map_2d(&m1, L.w_up, (uint64_t)d, (uint64_t)H, (uint64_t)rs, TC_M) ||
+      !map_2d(&mx, xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt))
+    return cudaErrorInvalidValue;
+  k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt, xh16);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int tiles = H / TC_M, nk = d / TC_BK;
+  int ks = device_sms() / tiles;
+  ks = ks < 1 ? 1 : (ks > TC_KSMAX ? TC_KSMAX : ks);
+  if (ks > nk) ks = nk;
+  constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
+  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
+  auto kern = k_hot_up_tc<NR>;
+  e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(m0, m1, mx, nt, nk, ks, H, part, hdr);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_hot_finish<NR><<<std::min((H * batch + 255) / 256, device_sms() * 4), 256, 0, s>>>(
+      part, ks, H, nt, batch, L.bias, h);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool hot_tc_supported(const pi_layer& L, int batch) {
+  if (tc_disabled()) return false;
+  if (L.w_dtype != PI_F16 || batch < 16 || batch > TC_TMAX) return false;
+  if (L.hot < TC_M || L.hot % TC_M != 0 || L.d_model % TC_BK != 0) return false;
+  const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
+  if (rs % 16 != 0) return false;
+  const uintptr_t bases = (uintptr_t)L.w_up | (uintptr_t)(L.act == PI_REGLU ? L.w_gate : L.w_up);
+  if (bases & 15u) return false;
+  return tensor_map_encoder() != nullptr;
+}
+
+size_t hot_tc_scratch_bytes(int d_model, int hot, int batch) {
+  if (batch < 16 || hot < TC_M) return 0;
+  return up256((size_t)TC_TMAX * d_model * 2) + (size_t)TC_KSMAX * 2 * hot * TC_TMAX * 4;
+}
+
+cudaError_t launch_hot_up_tc(const pi_layer& L, const float* xh, int batch, float* h,
+                             void* scratch, WsHeader* hdr, cudaStream_t s) {
+  return L.act == PI_REGLU ? launch_nr<2>(L, xh, batch, h, scratch, hdr, s)
+                           : launch_nr<1>(L, xh, batch, h, scratch, hdr, s);
+}
+
+}  // namespace pi

@@ -273,3 +273,36 @@ def test_stack_is_deterministic(pi, packed):
         pi.pi_ffn_stack(layers, x, 0.5, pi.PI_MASK_UNION)
         outs.append(x)
     assert torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("batch", [16, 20, 48, 64])
+def test_hot_prefix_on_tensor_cores(pi, orc, act, batch, monkeypatch):
+    """At 16-64 tokens the dense hot prefix (fp16) runs on the tensor cores
+    (fp16 inputs, fp32 accumulation): within the fp16 tolerance of the
+    oracle, close to the CUDA-core path, and not bitwise equal to it (so the
+    tensor-core path did run).  Batches 20 and 48 pad the token tile."""
+    w = _wl(act, "f16", (1024, 3001, 128, 640), seed=47)
+    L, _ = device_layer(w, 0, packed=(batch % 2 == 0))
+    H = synth.layer_host(w, 0)
+    xh = _xh(w.d_model, batch, 9)
+    masks, _ = _oracle_masks(orc, H, w, xh)
+    union = orc.compact(masks, w.d_ff, w.hot)
+    dev_idx = torch.zeros(w.d_ff, dtype=torch.int32, device="cuda")
+    dev_idx[: len(union)] = torch.from_numpy(union).cuda()
+    dev_cnt = torch.tensor([len(union)], dtype=torch.int32, device="cuda")
+    dxh = torch.from_numpy(xh).cuda()
+
+    def run():
+        return pi.pi_sparse_ffn(L, dxh, None, dev_idx, dev_cnt, pi.PI_MASK_UNION).cpu().numpy()
+
+    y_tc = run()
+    monkeypatch.setenv("PI_DISABLE_TC", "1")
+    y_cc = run()
+    monkeypatch.delenv("PI_DISABLE_TC")
+    assert not np.array_equal(y_tc, y_cc)
+    for b in range(batch):
+        ref = orc.sparse_ffn(H, xh[b].astype(np.float64), union)
+        assert rel_l2(y_tc[b], ref) <= TOL["f16"], b
+        assert rel_l2(y_tc[b], y_cc[b]) <= 2e-3, b
+    assert np.array_equal(run(), y_tc)  # deterministic
