@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
 }
 
 // Split-K gathered down projection.  Grid (column tiles, S, token chunks):
-// CTA (x, s, z) accumulates rows [s*N/S, (s+1)*N/S) of the list for 8
+// CTA (x, s, z) accumulates its slice s of the list positions [nb, N) for 8
 // columns per thread and TB tokens, skipping rows whose h is 0 for all of
 // its tokens, and writes its partial sums.
 template <int WT, int TB>
@@ -363,13 +363,13 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
                                                        const int32_t* __restrict__ count,
                                                        const float* __restrict__ h, int B,
                                                        int S, float* __restrict__ part,
-                                                       WsHeader* hdr, int64_t stride) {
+                                                       WsHeader* hdr, int64_t stride, int nb) {
   const int s = blockIdx.y, t0 = blockIdx.z * TB;
   const int col0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
   int cnt = *count;
   cnt = cnt < 0 ? 0 : (cnt > F - H ? F - H : cnt);
-  const int N = H + cnt;
-  const int n0 = (int)((int64_t)s * N / S), n1 = (int)((int64_t)(s + 1) * N / S);
+  const int N = H + cnt, M = N - nb;
+  const int n0 = nb + (int)((int64_t)s * M / S), n1 = nb + (int)((int64_t)(s + 1) * M / S);
   float acc[TB][8];
 #pragma unroll
   for (int b = 0; b < TB; ++b)
@@ -621,34 +621,34 @@ cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const u
 template <int WT, int TB>
 static cudaError_t ffn_down_t(const pi_layer& L, int batch, const int32_t* idx,
                               const int32_t* count, const float* h, float* part, int S,
-                              WsHeader* hdr, cudaStream_t s) {
+                              WsHeader* hdr, cudaStream_t s, int nb) {
   const int tiles = (L.d_model + 8 * kThreads - 1) / (8 * kThreads);
   dim3 grid(tiles, S, (batch + TB - 1) / TB);
   k_ffn_down<WT, TB><<<grid, kThreads, 0, s>>>((const char*)L.w_down_t,
                                               (const uint16_t*)L.w_down_t_scales, L.d_model,
                                               L.d_ff, L.hot, idx, count, h, batch, S, part, hdr,
-                                              L.w_down_row_stride);
+                                              L.w_down_row_stride, nb);
   return cudaGetLastError();
 }
 
 template <int WT>
 static cudaError_t ffn_down_w(const pi_layer& L, int batch, const int32_t* idx,
                               const int32_t* count, const float* h, float* part, int S,
-                              WsHeader* hdr, cudaStream_t s) {
+                              WsHeader* hdr, cudaStream_t s, int nb) {
   switch (down_tb(batch)) {
-    case 1: return ffn_down_t<WT, 1>(L, batch, idx, count, h, part, S, hdr, s);
-    case 2: return ffn_down_t<WT, 2>(L, batch, idx, count, h, part, S, hdr, s);
-    case 4: return ffn_down_t<WT, 4>(L, batch, idx, count, h, part, S, hdr, s);
-    default: return ffn_down_t<WT, 8>(L, batch, idx, count, h, part, S, hdr, s);
+    case 1: return ffn_down_t<WT, 1>(L, batch, idx, count, h, part, S, hdr, s, nb);
+    case 2: return ffn_down_t<WT, 2>(L, batch, idx, count, h, part, S, hdr, s, nb);
+    case 4: return ffn_down_t<WT, 4>(L, batch, idx, count, h, part, S, hdr, s, nb);
+    default: return ffn_down_t<WT, 8>(L, batch, idx, count, h, part, S, hdr, s, nb);
   }
 }
 
 cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,
                             const int32_t* count, const float* h, float* part, int splits,
-                            WsHeader* hdr, cudaStream_t s) {
-  if (L.w_dtype == PI_F32) return ffn_down_w<PI_F32>(L, batch, idx, count, h, part, splits, hdr, s);
-  if (L.w_dtype == PI_F16) return ffn_down_w<PI_F16>(L, batch, idx, count, h, part, splits, hdr, s);
-  return ffn_down_w<PI_Q4_0>(L, batch, idx, count, h, part, splits, hdr, s);
+                            WsHeader* hdr, cudaStream_t s, int nb) {
+  if (L.w_dtype == PI_F32) return ffn_down_w<PI_F32>(L, batch, idx, count, h, part, splits, hdr, s, nb);
+  if (L.w_dtype == PI_F16) return ffn_down_w<PI_F16>(L, batch, idx, count, h, part, splits, hdr, s, nb);
+  return ffn_down_w<PI_Q4_0>(L, batch, idx, count, h, part, splits, hdr, s, nb);
 }
 
 cudaError_t launch_delay(unsigned long long ns, cudaStream_t s) {

@@ -37,10 +37,11 @@ cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const u
                           int per_token, const int32_t* idx, const int32_t* count, float* h,
                           WsHeader* hdr, cudaStream_t s, int n0 = 0);
 
-// part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n]
+// part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n],
+// the list positions [nb, H + count) split into `splits` slices
 cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,
                             const int32_t* count, const float* h, float* part, int splits,
-                            WsHeader* hdr, cudaStream_t s);
+                            WsHeader* hdr, cudaStream_t s, int nb = 0);
 
 // out[b][i] = (resid ? resid[b][i] : 0) + sum_s part[s][b][i], s ascending.
 cudaError_t launch_reduce(const float* part, int splits, int batch, int d, const float* resid,

@@ -16,7 +16,15 @@
 //
 // d is split over up to 4 CTAs per tile so that about one CTA per SM
 // streams weights; a second kernel sums the splits in a fixed order, adds
-// the bias and applies ReLU / ReGLU, writing h as the CUDA-core kernels do.
+// the bias and applies ReLU / ReGLU, writing h (fp32, as the CUDA-core
+// kernels do, and an fp16 copy [tokens][hot]).
+//
+// The hot rows' down projection is the second contraction: D[c][t] =
+// sum_{j < hot} W_down^T[j][c] h[t][j] for 128 output columns c per tile.
+// W_down^T is stored neuron-major (c contiguous), so it is an MN-major A
+// operand: per stage two TMA boxes of 64 columns x 64 neurons (128-byte
+// swizzle); the fp16 h is the K-major B operand.  Its partial rows join the
+// CUDA-core kernel's split-K slices in the fixed-order reduction.
 // Every mbarrier wait is bounded by %globaltimer (1 s): a wait that runs out
 // sets DEV_TIMEOUT in the workspace status word and a CTA abort flag, the
 // producer waits (bounded) for its own copies in flight, and the tensor
@@ -85,6 +93,14 @@ __device__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, WsH
 // leading byte offset unused (1), descriptor version 1, layout 2 (128B).
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
   return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) |
+         ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Descriptor of an MN-major tile with 128-byte swizzle: 8 K-rows of 128
+// bytes (64 MN elements) per 1024-byte atom, K atoms 1024 bytes apart
+// (stride byte offset), MN atoms `mn_stride` bytes apart (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_mn_desc(uint32_t saddr, uint32_t mn_stride) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
@@ -277,22 +293,160 @@ __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
   }
 }
 
-// h[n * batch + b] = act(sum over splits (fixed order) + bias) for n < H.
+// h[n * batch + b] = act(sum over splits (fixed order) + bias) for n < H,
+// and its fp16 copy h16[b][n] (zero for the padding tokens b >= batch).
 template <int NR>
 __global__ void k_hot_finish(const float* __restrict__ part, int ks, int H, int nt, int batch,
-                             const float* __restrict__ bias, float* __restrict__ h) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H * batch; i += gridDim.x * blockDim.x) {
-    const int n = i / batch, b = i % batch;
-    float g = 0.f, u = 0.f;
-    for (int s = 0; s < ks; ++s) {
-      g += __ldcg(part + ((size_t)(s * NR) * H + n) * nt + b);
-      if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * H + n) * nt + b);
+                             const float* __restrict__ bias, float* __restrict__ h,
+                             __half* __restrict__ h16) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H * nt; i += gridDim.x * blockDim.x) {
+    const int b = i / H, n = i % H;
+    float hv = 0.f;
+    if (b < batch) {
+      float g = 0.f, u = 0.f;
+      for (int s = 0; s < ks; ++s) {
+        g += __ldcg(part + ((size_t)(s * NR) * H + n) * nt + b);
+        if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * H + n) * nt + b);
+      }
+      g += bias ? bias[n] : 0.f;
+      hv = g > 0.f ? g : 0.f;
+      if constexpr (NR == 2) hv *= u;
+      h[(size_t)n * batch + b] = hv;
     }
-    g += bias ? bias[n] : 0.f;
-    float hv = g > 0.f ? g : 0.f;
-    if constexpr (NR == 2) hv *= u;
-    h[(size_t)n * batch + b] = hv;
+    h16[(size_t)b * H + n] = __float2half_rn(hv);
   }
+}
+
+// Partial rows part[split][b][c] = sum over the split's hot neurons j of
+// W_down^T[j][c] h16[b][j], for the tile's 128 columns c.  Grid (d / 128, ks).
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_hot_down_tc(const __grid_constant__ CUtensorMap mwd, const __grid_constant__ CUtensorMap mh,
+                  int nt, int nk, int ks, int d, int batch, int H, float* __restrict__ part,
+                  WsHeader* hdr) {
+  constexpr uint32_t BOX = 64 * TC_BK * 2;             // 64 columns x 64 neurons: 8 KB
+  constexpr uint32_t A_BYTES = 2 * BOX;                // 128 columns
+  constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;    // 8 KB
+  constexpr uint32_t STAGE = A_BYTES + B_BYTES;
+  constexpr uint32_t NCOLS = 64u;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = tc_sa(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_STAGES * STAGE);
+  uint64_t* empty = full + TC_STAGES;
+  uint64_t* done = empty + TC_STAGES;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
+  const int nkt = kt1 - kt0;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TC_STAGES; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
+    }
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(done)) : "memory");
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)H);
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     tc_sa(tslot)),
+                 "r"(NCOLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0 && lane == 0) {
+    const uint32_t tx = A_BYTES + (uint32_t)nt * TC_BK * 2;
+    int last[TC_STAGES];
+    for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % TC_STAGES;
+      if (i >= TC_STAGES && !tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr)) break;
+      unsigned char* a = smem + st * STAGE;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
+                   "r"(tx)
+                   : "memory");
+      const int j = (kt0 + i) * TC_BK;  // first hot neuron of the stage
+      tma_load_2d(a, &mwd, tile * TC_M, j, &full[st]);
+      tma_load_2d(a + BOX, &mwd, tile * TC_M + 64, j, &full[st]);
+      tma_load_2d(a + A_BYTES, &mh, j, 0, &full[st]);
+      last[st] = i;
+    }
+    for (int st = 0; st < TC_STAGES; ++st) {
+      if (last[st] < 0) continue;
+      const uint32_t par = (uint32_t)(last[st] / TC_STAGES) & 1u;
+      const uint64_t t0 = tc_time();
+      while (!tc_try(&full[st], par)) {
+        if (tc_time() - t0 > kTcTimeoutNs) {
+          if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
+          break;
+        }
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // kind::f16, fp16 A (MN-major) and B (K-major), fp32 D, M = 128, N = nt
+    const uint32_t idesc = (1u << 4) | (1u << 15) | ((uint32_t)(nt >> 3) << 17) |
+                           ((uint32_t)(TC_M >> 4) << 24);
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % TC_STAGES;
+      if (!tc_wait(&full[st], (uint32_t)(i / TC_STAGES) & 1u, abort, hdr)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = tc_sa(smem + st * STAGE), b = a + A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk)  // 16 neurons = 2 K atoms of the A tile per MMA
+        mma_f16(tmem, sw128_mn_desc(a + 2048u * kk, BOX), sw128_desc(b + 32u * kk), idesc,
+                (i | kk) != 0 ? 1u : 0u);
+      mma_commit(&empty[st]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  bool ok = tc_try(done, 0u);
+  if (!ok) {
+    const uint64_t t0 = tc_time();
+    while (!(ok = tc_try(done, 0u))) {
+      if (tc_time() - t0 > kTcTimeoutNs) {
+        if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
+        break;
+      }
+    }
+  }
+  ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (ok) {
+    // accumulator lane = output column, accumulator column = token
+    const int c = tile * TC_M + warp * 32 + lane;
+    for (int c0 = 0; c0 < nt; c0 += 16) {
+      uint32_t v[16];
+      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+          "%11, %12, %13, %14, %15}, [%16];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+            "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+            "=r"(v[14]), "=r"(v[15])
+          : "r"(taddr));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int t = 0; t < 16; ++t)
+        if (c0 + t < batch) __stcg(part + ((size_t)split * batch + c0 + t) * d + c, __uint_as_float(v[t]));
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS)
+                 : "memory");
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -331,13 +485,38 @@ bool tc_disabled() {
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
+// Scratch: xh16 [64][d] fp16 | partial sums [4][2][hot][64] fp32 | h16 [64][hot] fp16.
+struct TcScratch {
+  __half* xh16;
+  float* part;
+  __half* h16;
+};
+
+TcScratch tc_scratch(void* base, int d, int H) {
+  char* p = static_cast<char*>(base);
+  TcScratch t;
+  t.xh16 = reinterpret_cast<__half*>(p);
+  p += up256((size_t)TC_TMAX * d * 2);
+  t.part = reinterpret_cast<float*>(p);
+  p += up256((size_t)TC_KSMAX * 2 * H * TC_TMAX * 4);
+  t.h16 = reinterpret_cast<__half*>(p);
+  return t;
+}
+
+int split_for(int tiles, int nk) {
+  int ks = device_sms() / tiles;
+  ks = ks < 1 ? 1 : (ks > TC_KSMAX ? TC_KSMAX : ks);
+  return ks > nk ? nk : ks;
+}
+
 template <int NR>
 cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, void* scratch,
                       WsHeader* hdr, cudaStream_t s) {
   const int d = L.d_model, H = L.hot;
   const int nt = (batch + 15) / 16 * 16;
-  __half* xh16 = static_cast<__half*>(scratch);
-  float* part = reinterpret_cast<float*>(static_cast<char*>(scratch) + up256((size_t)TC_TMAX * d * 2));
+  const TcScratch sc = tc_scratch(scratch, d, H);
+  __half* xh16 = sc.xh16;
+  float* part = sc.part;
   const int64_t rs = code_stride(PI_F16, d, L.w_row_stride);
   CUtensorMap m0, m1, mx;
   const void* w0 = NR == 2 ? L.w_gate : L.w_up;
@@ -349,9 +528,7 @@ cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, v
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int tiles = H / TC_M, nk = d / TC_BK;
-  int ks = device_sms() / tiles;
-  ks = ks < 1 ? 1 : (ks > TC_KSMAX ? TC_KSMAX : ks);
-  if (ks > nk) ks = nk;
+  const int ks = split_for(tiles, nk);
   constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
   const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
   auto kern = k_hot_up_tc<NR>;
@@ -360,8 +537,8 @@ cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, v
   kern<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(m0, m1, mx, nt, nk, ks, H, part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_hot_finish<NR><<<std::min((H * batch + 255) / 256, device_sms() * 4), 256, 0, s>>>(
-      part, ks, H, nt, batch, L.bias, h);
+  k_hot_finish<NR><<<std::min((H * nt + 255) / 256, device_sms() * 4), 256, 0, s>>>(
+      part, ks, H, nt, batch, L.bias, h, sc.h16);
   return cudaGetLastError();
 }
 
@@ -370,9 +547,10 @@ cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, v
 bool hot_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
   if (L.w_dtype != PI_F16 || batch < 16 || batch > TC_TMAX) return false;
-  if (L.hot < TC_M || L.hot % TC_M != 0 || L.d_model % TC_BK != 0) return false;
+  if (L.hot < TC_M || L.hot % TC_M != 0 || L.d_model % TC_M != 0) return false;
   const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
-  if (rs % 16 != 0) return false;
+  const int64_t rd = code_stride(PI_F16, L.d_model, L.w_down_row_stride);
+  if (rs % 16 != 0 || rd % 16 != 0 || ((uintptr_t)L.w_down_t & 15u)) return false;
   const uintptr_t bases = (uintptr_t)L.w_up | (uintptr_t)(L.act == PI_REGLU ? L.w_gate : L.w_up);
   if (bases & 15u) return false;
   return tensor_map_encoder() != nullptr;
@@ -380,7 +558,29 @@ bool hot_tc_supported(const pi_layer& L, int batch) {
 
 size_t hot_tc_scratch_bytes(int d_model, int hot, int batch) {
   if (batch < 16 || hot < TC_M) return 0;
-  return up256((size_t)TC_TMAX * d_model * 2) + (size_t)TC_KSMAX * 2 * hot * TC_TMAX * 4;
+  return up256((size_t)TC_TMAX * d_model * 2) + up256((size_t)TC_KSMAX * 2 * hot * TC_TMAX * 4) +
+         (size_t)TC_TMAX * hot * 2;
+}
+
+int hot_tc_down_splits(const pi_layer& L) { return split_for(L.d_model / TC_M, L.hot / TC_BK); }
+
+cudaError_t launch_hot_down_tc(const pi_layer& L, int batch, float* part, void* scratch,
+                               WsHeader* hdr, cudaStream_t s) {
+  const int d = L.d_model, H = L.hot;
+  const int nt = (batch + 15) / 16 * 16;
+  const TcScratch sc = tc_scratch(scratch, d, H);
+  const int64_t rd = code_stride(PI_F16, d, L.w_down_row_stride);
+  CUtensorMap mwd, mh;
+  if (!map_2d(&mwd, L.w_down_t, (uint64_t)d, (uint64_t)H, (uint64_t)rd, TC_BK) ||
+      !map_2d(&mh, sc.h16, (uint64_t)H, (uint64_t)nt, (uint64_t)H * 2, (uint32_t)nt))
+    return cudaErrorInvalidValue;
+  const int tiles = d / TC_M, nk = H / TC_BK, ks = hot_tc_down_splits(L);
+  constexpr uint32_t STAGE = 2 * 64 * TC_BK * 2 + TC_TMAX * TC_BK * 2;
+  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
+  cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_hot_down_tc), smem);
+  if (e != cudaSuccess) return e;
+  k_hot_down_tc<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(mwd, mh, nt, nk, ks, d, batch, H, part, hdr);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_hot_up_tc(const pi_layer& L, const float* xh, int batch, float* h,
