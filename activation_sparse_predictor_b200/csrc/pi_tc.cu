@@ -295,25 +295,37 @@ __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
 
 // h[n * batch + b] = act(sum over splits (fixed order) + bias) for n < H,
 // and its fp16 copy h16[b][n] (zero for the padding tokens b >= batch).
+// One block per 64 neurons: partial sums read and h16 written coalesced,
+// transposed through shared memory.
 template <int NR>
-__global__ void k_hot_finish(const float* __restrict__ part, int ks, int H, int nt, int batch,
-                             const float* __restrict__ bias, float* __restrict__ h,
-                             __half* __restrict__ h16) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < H * nt; i += gridDim.x * blockDim.x) {
-    const int b = i / H, n = i % H;
+__global__ void __launch_bounds__(256) k_hot_finish(const float* __restrict__ part, int ks, int H,
+                                                    int nt, int batch,
+                                                    const float* __restrict__ bias,
+                                                    float* __restrict__ h,
+                                                    __half* __restrict__ h16) {
+  __shared__ float sh[64][TC_TMAX + 1];
+  const int n0 = blockIdx.x * 64;
+  const int m = 64 * nt;  // this block's values per (split, matrix): contiguous
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    const int nn = i / nt, b = i % nt;
+    float g = 0.f, u = 0.f;
+    for (int s = 0; s < ks; ++s) {
+      g += __ldcg(part + ((size_t)(s * NR) * H + n0) * nt + i);
+      if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * H + n0) * nt + i);
+    }
     float hv = 0.f;
     if (b < batch) {
-      float g = 0.f, u = 0.f;
-      for (int s = 0; s < ks; ++s) {
-        g += __ldcg(part + ((size_t)(s * NR) * H + n) * nt + b);
-        if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * H + n) * nt + b);
-      }
-      g += bias ? bias[n] : 0.f;
+      g += bias ? bias[n0 + nn] : 0.f;
       hv = g > 0.f ? g : 0.f;
       if constexpr (NR == 2) hv *= u;
-      h[(size_t)n * batch + b] = hv;
+      h[(size_t)(n0 + nn) * batch + b] = hv;
     }
-    h16[(size_t)b * H + n] = __float2half_rn(hv);
+    sh[nn][b] = hv;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+    const int b = i / 64, nn = i % 64;
+    h16[(size_t)b * H + n0 + nn] = __float2half_rn(sh[nn][b]);
   }
 }
 
@@ -537,8 +549,7 @@ cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, v
   kern<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(m0, m1, mx, nt, nk, ks, H, part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_hot_finish<NR><<<std::min((H * nt + 255) / 256, device_sms() * 4), 256, 0, s>>>(
-      part, ks, H, nt, batch, L.bias, h, sc.h16);
+  k_hot_finish<NR><<<H / 64, 256, 0, s>>>(part, ks, H, nt, batch, L.bias, h, sc.h16);
   return cudaGetLastError();
 }
 

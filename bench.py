@@ -21,7 +21,6 @@ layers, extrapolated to the whole stack.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import math
@@ -271,12 +270,15 @@ PROFILES = os.path.join(os.path.dirname(os.path.abspath(__file__)), "profiles")
 CSRC = os.path.join(os.path.dirname(os.path.abspath(__file__)), "activation_sparse_predictor_b200", "csrc")
 
 
+FUSED_SOURCES = ("pi_stack.cu", "pi_stack.cuh", "pi_common.cuh")
+
+
 def kernel_source_sha256() -> str:
-    """Hash of the CUDA sources (csrc/*.cu, *.cuh) the library is built from."""
+    """Hash of the sources the fused single-token kernel is built from."""
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cuh"))):
-        h.update(os.path.basename(f).encode())
-        h.update(open(f, "rb").read())
+    for name in FUSED_SOURCES:
+        h.update(name.encode())
+        h.update(open(os.path.join(CSRC, name), "rb").read())
     return h.hexdigest()
 
 
