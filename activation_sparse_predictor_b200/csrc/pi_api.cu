@@ -474,6 +474,16 @@ pi_status pi_ffn_stack_timeline(const pi_layer* layers, int n_layers, float* x, 
 
 int pi_device_sms(void) { return device_sms(); }
 
+pi_status pi_wait_selftest(void* ws, size_t ws_bytes, int kind, unsigned timeout_us, void* stream) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < sizeof(WsHeader))
+    return fail(PI_ERR_INVALID, "workspace null, misaligned or smaller than its header");
+  if (kind != 0 && kind != 1) return fail(PI_ERR_INVALID, "kind %d not 0 (mbarrier) or 1 (grid)", kind);
+  if (timeout_us < 1 || timeout_us > 10000000u)
+    return fail(PI_ERR_INVALID, "timeout %u us not in [1, 1e7]", timeout_us);
+  cudaError_t e = launch_wait_selftest(ws, kind, 1000ull * timeout_us, (cudaStream_t)stream);
+  return e == cudaSuccess ? PI_OK : cuda_fail(e, "wait self-test launch");
+}
+
 pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {
   if (!ws || !aligned(ws, 256) || !out) return fail(PI_ERR_INVALID, "workspace or output null");
   cudaStream_t s = (cudaStream_t)stream;

@@ -342,14 +342,15 @@ __device__ void raise_abort(const Smem& S, WsHeader* hdr) {
 // The first try usually succeeds; the warp sleeps in the hardware wait
 // between later checks.
 __device__ __forceinline__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Smem& S,
-                                          WsHeader* hdr) {
+                                          WsHeader* hdr,
+                                          unsigned long long limit_ns = kTimeoutNs) {
   if (mbar_try(bar, parity)) return true;
   if (*S.abort) return false;
   const uint64_t t0 = gtime();
   while (true) {
     if (mbar_try_sleep(bar, parity, 50000u)) return true;
     if (*S.abort) return false;
-    if (gtime() - t0 > kTimeoutNs) {
+    if (gtime() - t0 > limit_ns) {
       raise_abort(S, hdr);
       return false;
     }
@@ -357,7 +358,8 @@ __device__ __forceinline__ bool wait_mbar(uint64_t* bar, uint32_t parity, const 
 }
 
 // Bounded grid-barrier wait by one thread: counter >= target.
-__device__ bool grid_wait(WsHeader* hdr, uint32_t target, const Smem& S) {
+__device__ bool grid_wait(WsHeader* hdr, uint32_t target, const Smem& S,
+                          unsigned long long limit_ns = kTimeoutNs) {
   if (*S.abort) return false;
   if (ld_acquire(&hdr->counters[0]) >= target) return true;
   const uint64_t t0 = gtime();
@@ -368,7 +370,7 @@ __device__ bool grid_wait(WsHeader* hdr, uint32_t target, const Smem& S) {
       *S.abort = 1;
       return false;
     }
-    if (gtime() - t0 > kTimeoutNs) {
+    if (gtime() - t0 > limit_ns) {
       raise_abort(S, hdr);
       return false;
     }
@@ -1435,7 +1437,37 @@ cudaError_t launch_any(const StackParams& P, int wt, int act, int pt, cudaStream
                          : launch_t<PI_F32, PI_RELU, PI_F32>(P, s);
 }
 
+// One CTA, one thread: the kernel's own bounded waits on state nothing
+// completes (kind 0: an mbarrier phase with no arrival; kind 1: a grid
+// barrier target no CTA reaches), ended by `limit_ns`.
+__global__ void k_wait_selftest(WsHeader* hdr, int kind, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  Smem S{};
+  S.abort = &abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1u);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (kind == 0)
+      (void)wait_mbar(&bar, 0u, S, hdr, limit_ns);
+    else
+      (void)grid_wait(hdr, 0xFFFFFFFFu, S, limit_ns);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(void* ws, int kind, unsigned long long limit_ns, cudaStream_t s) {
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+  cudaError_t e = cudaMemsetAsync(hdr->counters, 0, 2 * sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  k_wait_selftest<<<1, 32, 0, s>>>(hdr, kind, limit_ns);
+  return cudaGetLastError();
+}
 
 int stack1_chunk() { return MAXL; }
 int stack1_unit_trace_len() { return UTR; }

@@ -29,4 +29,8 @@ cudaError_t launch_stack1(const pi_layer* layers, int n_layers, float* x, uint32
 // Units per layer recorded by the unit trace (first CTA only).
 int stack1_unit_trace_len();
 
+// Runs the fused kernel's bounded-wait code on a wait nothing completes
+// (kind 0: mbarrier, kind 1: grid barrier), limited to limit_ns.
+cudaError_t launch_wait_selftest(void* ws, int kind, unsigned long long limit_ns, cudaStream_t s);
+
 }  // namespace pi

@@ -65,6 +65,7 @@ def _load():
         "pi_read_counters": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_uint64)]),
         "pi_ffn_stack_timeline": (i32, [L, i32, vp, f32, vp, sz, vp, vp, vp]),
         "pi_device_sms": (i32, []),
+        "pi_wait_selftest": (i32, [vp, sz, i32, ctypes.c_uint, vp]),
         "pi_status_string": (ctypes.c_char_p, [i32]),
         "pi_last_error": (ctypes.c_char_p, []),
         "pi_version": (i32, []),
@@ -339,6 +340,13 @@ def pi_get_device_status(ws, clear: bool = False, stream=None):
     word = ctypes.c_uint32(0)
     st = _lib.pi_get_device_status(_ptr(ws), _stream(stream), int(clear), ctypes.byref(word))
     return st, int(word.value)
+
+
+def pi_wait_selftest(ws, kind: int, timeout_us: int, stream=None) -> None:
+    """Runs the fused kernel's bounded wait on a wait nothing completes (kind
+    0: mbarrier, 1: grid barrier) for timeout_us; the timeout shows in
+    pi_get_device_status."""
+    _check(_lib.pi_wait_selftest(_ptr(ws), ws.numel(), kind, timeout_us, _stream(stream)))
 
 
 def pi_status_string(st: int) -> str:

@@ -149,7 +149,9 @@ def dist_setup(args):
         backend = "nccl" if (args.impl == "pi" and torch.cuda.is_available()) else "gloo"
         if backend == "nccl":
             torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+        # a short limit: a rank that waits for one that died ends with an error
+        limit = float(os.environ.get("PI_DIST_TIMEOUT_S", "180"))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=limit))
     return world, rank, local
 
 

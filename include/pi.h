@@ -273,6 +273,16 @@ pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out);
  * (nullable) receives the raw word; `clear` != 0 resets it. */
 pi_status pi_get_device_status(void* ws, void* stream, int clear, uint32_t* detail);
 
+/* Failure-detection self-test: runs, in one thread of a tiny kernel, the
+ * bounded waits the fused kernel uses, on a wait nothing can satisfy
+ * (kind 0: an mbarrier phase with no arrival; kind 1: the workspace's grid
+ * barrier counter against a target no CTA reaches), limited to timeout_us
+ * (1 .. 1e7) instead of the kernel's 1 s.  The wait runs out, records the
+ * timeout in the workspace status word (pi_get_device_status then returns
+ * PI_ERR_TIMEOUT) and the kernel returns normally: the context stays usable.
+ * Resets the workspace's grid-barrier counters.  Not part of the method. */
+pi_status pi_wait_selftest(void* ws, size_t ws_bytes, int kind, unsigned timeout_us, void* stream);
+
 const char* pi_status_string(int status);
 const char* pi_last_error(void);
 int pi_version(void);
