@@ -94,13 +94,13 @@ WsLayout layout_for(int d, int F, int r, int batch, int H) {
   // split-K partials: the multi-kernel split, or one slice per SM for the
   // fused single-token stack
   // (+ up to 4 slices of the tensor-core hot prefix at token batches)
-  const size_t tcp = hot_tc_scratch_bytes(d, H, batch) ? (size_t)4 * batch : 0;
+  const size_t tcp = ffn_tc_scratch_bytes(d, F, batch) ? (size_t)4 * batch : 0;
   const size_t parts = (size_t)w.splits * batch + tcp > 2 * (size_t)device_sms()
                            ? (size_t)w.splits * batch + tcp
                            : 2 * (size_t)device_sms();
   w.part = take(parts * d * 4);
   w.y = take((size_t)batch * d * 4);
-  w.tc = take(hot_tc_scratch_bytes(d, H, batch));
+  w.tc = take(ffn_tc_scratch_bytes(d, F, batch));
   w.total = off;
   return w;
 }
@@ -156,35 +156,33 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
                    Prof* prof = nullptr) {
   Prof none;
   Prof& P = prof ? *prof : none;
-  P.before(PI_KIND_FFN_UP);
-  cudaError_t e = cudaSuccess;
-  int n0 = 0;  // first list position left to the CUDA-core kernels
-  const bool tc = hot_tc_supported(L, batch);
-  if (tc) {
-    // the dense hot prefix on the tensor cores, the listed cold rows after it
-    e = launch_hot_up_tc(L, xh, batch, at<float>(ws, lay.h), at<void>(ws, lay.tc), header(ws), s);
-    if (e != cudaSuccess) return cuda_fail(e, "hot prefix (tensor cores) launch");
-    n0 = L.hot;
-  }
-  e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h), header(ws), s,
-                    n0);
-  P.after();
-  if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
   const int S = down_splits(batch, L.d_model);
   float* part = at<float>(ws, lay.part);
-  int St = 0;  // slices of the tensor-core hot rows, after the CUDA-core ones
-  P.before(PI_KIND_FFN_DOWN);
-  if (tc) {
-    St = hot_tc_down_splits(L);
-    e = launch_hot_down_tc(L, batch, part + (size_t)S * batch * L.d_model, at<void>(ws, lay.tc),
-                           header(ws), s);
-    if (e != cudaSuccess) return cuda_fail(e, "hot down projection (tensor cores) launch");
+  int St = S;  // split-K slices to reduce
+  cudaError_t e = cudaSuccess;
+  if (ffn_tc_supported(L, batch)) {
+    // token batches: both contractions over the listed rows on the tensor cores
+    P.before(PI_KIND_FFN_UP);
+    e = launch_ffn_up_tc(L, xh, batch, mask, idx, count, at<void>(ws, lay.tc), header(ws), s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "ffn up (tensor cores) launch");
+    P.before(PI_KIND_FFN_DOWN);
+    St = ffn_tc_down_splits(L);
+    e = launch_ffn_down_tc(L, batch, idx, count, part, at<void>(ws, lay.tc), header(ws), s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "ffn down (tensor cores) launch");
+  } else {
+    P.before(PI_KIND_FFN_UP);
+    e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h), header(ws), s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
+    P.before(PI_KIND_FFN_DOWN);
+    e = launch_ffn_down(L, batch, idx, count, at<float>(ws, lay.h), part, S, header(ws), s);
+    P.after();
+    if (e != cudaSuccess) return cuda_fail(e, "ffn_down launch");
   }
-  e = launch_ffn_down(L, batch, idx, count, at<float>(ws, lay.h), part, S, header(ws), s, n0);
-  P.after();
-  if (e != cudaSuccess) return cuda_fail(e, "ffn_down launch");
   P.before(PI_KIND_REDUCE);
-  e = launch_reduce(part, S + St, batch, L.d_model, resid, out, s);
+  e = launch_reduce(part, St, batch, L.d_model, resid, out, s);
   P.after();
   if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
   return PI_OK;

@@ -1,34 +1,29 @@
-// Dense hot prefix at token batches on the tensor cores (sm_100a).
+// The FFN of a layer at token batches on the tensor cores (sm_100a).
 //
-// The hot neurons [0, hot) run for every token, so at 16-64 tokens their
-// gate/up products are a real contraction: D[n][t] = sum_k W[n][k] xh[t][k]
-// for 128 hot neurons n per tile and all tokens t.  The weight rows are the
-// MMA's A operand exactly as stored (M = 128, K-major), an fp16 copy of the
-// normalised inputs is its B operand (N = tokens padded to 16, K-major), and
-// the fp32 accumulators live in tensor memory:
+// At 16-64 tokens the listed rows (the hot prefix [0, hot), then the cold
+// list idx) of every token batch form real contractions, both run as tcgen05
+// GEMMs over list positions p (row(p) = p for p < hot, idx[p - hot] after):
 //
-//   warp 0, one thread : TMA 2-D tile loads (128-byte swizzle) into a ring of
-//                        4 stages, completion on a full mbarrier per stage
-//   warp 1, one thread : tcgen05.mma (kind::f16, 4 per 64-wide stage), then
-//                        tcgen05.commit to the stage's empty mbarrier
-//   all 4 warps        : tcgen05.ld of their 32 accumulator lanes -> fp32
-//                        partial sums in the workspace
+//   up   : D[p][t] = sum_k W[row(p)][k] xh[t][k] for 128 list positions per
+//          tile (the MMA's A operand, K-major) and all tokens t (B: an fp16
+//          copy of the normalised inputs, tokens padded to 16); d split over
+//          up to 4 CTAs per tile; a second kernel sums the splits in a fixed
+//          order, adds the bias, applies ReLU / ReGLU and the per-token bits
+//          and writes an fp16 copy h16[t][p];
+//   down : D[c][t] = sum_p W_down^T[row(p)][c] h16[t][p] for 128 output
+//          columns per tile; W_down^T (columns contiguous) is an MN-major A
+//          operand; the list positions split over up to 4 CTAs; the partial
+//          rows go to the fixed-order split-K reduction.
 //
-// d is split over up to 4 CTAs per tile so that about one CTA per SM
-// streams weights; a second kernel sums the splits in a fixed order, adds
-// the bias and applies ReLU / ReGLU, writing h (fp32, as the CUDA-core
-// kernels do, and an fp16 copy [tokens][hot]).
-//
-// The hot rows' down projection is the second contraction: D[c][t] =
-// sum_{j < hot} W_down^T[j][c] h[t][j] for 128 output columns c per tile.
-// W_down^T is stored neuron-major (c contiguous), so it is an MN-major A
-// operand: per stage two TMA boxes of 64 columns x 64 neurons (128-byte
-// swizzle); the fp16 h is the K-major B operand.  Its partial rows join the
-// CUDA-core kernel's split-K slices in the fixed-order reduction.
-// Every mbarrier wait is bounded by %globaltimer (1 s): a wait that runs out
-// sets DEV_TIMEOUT in the workspace status word and a CTA abort flag, the
-// producer waits (bounded) for its own copies in flight, and the tensor
-// memory is always freed before the CTA exits.
+// A tile whose rows all lie in the hot prefix is one TMA box per operand
+// and stage; any other tile is gathered: each lane of the producer warp
+// issues one TMA tile::gather4 load (four rows, a one-row-high box) per
+// operand and stage.  128-byte swizzle throughout, a 4-stage mbarrier ring,
+// fp32 accumulators in tensor memory, one thread issuing the MMAs.  Every
+// mbarrier wait is bounded by %globaltimer (1 s): a wait that runs out sets
+// DEV_TIMEOUT in the workspace status word and a CTA abort flag; the
+// producer waits (bounded) for its copies in flight and the tensor memory
+// is always freed after the MMAs have completed.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -43,11 +38,11 @@
 namespace pi {
 namespace {
 
-constexpr int TC_M = 128;        // hot neurons per tile (MMA M)
+constexpr int TC_M = 128;        // list positions (up) / output columns (down) per tile
 constexpr int TC_BK = 64;        // k per stage: one 128-byte swizzle atom of fp16
 constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 128;
-constexpr int TC_KSMAX = 4;      // CTAs sharing one tile's d at most
+constexpr int TC_KSMAX = 4;      // CTAs sharing one tile's k range at most
 constexpr int TC_TMAX = 64;      // tokens at most (MMA N)
 constexpr unsigned long long kTcTimeoutNs = 1000000000ull;
 
@@ -81,6 +76,19 @@ __device__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, WsH
     if (*abort) return false;
     if (tc_time() - t0 > kTcTimeoutNs) {
       *abort = 1;
+      if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Bounded wait that ignores the abort flag (used before freeing resources).
+__device__ bool tc_wait_quiet(uint64_t* bar, uint32_t parity, WsHeader* hdr) {
+  if (tc_try(bar, parity)) return true;
+  const uint64_t t0 = tc_time();
+  while (!tc_try(bar, parity)) {
+    if (tc_time() - t0 > kTcTimeoutNs) {
       if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
       return false;
     }
@@ -130,12 +138,75 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
-// NR = 1: ReLU (W_up); NR = 2: ReGLU (W_gate, W_up).  Grid (hot / 128, ks).
-// part: [ks][NR][hot][nt] fp32.
+// Four rows y0..y3 (columns x .. x+63) of a map whose box is one row high,
+// to 4 consecutive 128-byte rows at dst.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, int x, int y0,
+                                            int y1, int y2, int y3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(tc_sa(dst)),
+      "l"(map), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(tc_sa(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_init(uint64_t* full, uint64_t* empty, uint64_t* done,
+                                        volatile int* abort) {
+  for (int i = 0; i < TC_STAGES; ++i) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
+  }
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(done)) : "memory");
+  *abort = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tc_sa(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+// 16 consecutive accumulator columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// List length hot + count with count clamped to [0, F - hot].
+__device__ __forceinline__ int list_len(const int32_t* count, int H, int F, WsHeader* hdr) {
+  int c = *count;
+  if (c < 0 || c > F - H) {
+    if (hdr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+      atomicOr(&hdr->status, DEV_BAD_COUNT);
+    c = c < 0 ? 0 : F - H;
+  }
+  return H + c;
+}
+
+// Weight row of list position p (a valid row for every p: positions beyond
+// the list and bad indices read row 0; their h is 0).
+__device__ __forceinline__ int list_row(int p, int H, int N, int F, const int32_t* idx) {
+  if (p < H) return p;
+  if (p >= N) return 0;
+  const int j = idx[p - H];
+  return (j >= H && j < F) ? j : 0;
+}
+
+// up: NR = 1 ReLU (W_up), NR = 2 ReGLU (W_gate, W_up).  Grid (Fp / 128, ks).
+// part: [ks][NR][Fp][nt] fp32.
 template <int NR>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    k_hot_up_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
-                const __grid_constant__ CUtensorMap mx, int nt, int nk, int ks, int H,
+    k_ffn_up_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
+                const __grid_constant__ CUtensorMap mg0, const __grid_constant__ CUtensorMap mg1,
+                const __grid_constant__ CUtensorMap mx, int nt, int nk, int ks, int H, int F, int Fp,
+                const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                 float* __restrict__ part, WsHeader* hdr) {
   constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB (nt rows used)
@@ -149,62 +220,63 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* done = empty + TC_STAGES;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+  int* rows = reinterpret_cast<int*>(tslot + 4);  // [128], 16-byte aligned
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, split = blockIdx.y;
+  const int N = list_len(count, H, F, hdr);
+  const int p0 = tile * TC_M;
+  if (p0 >= N) return;  // past the list: nothing of this tile is read
+  const bool dense = p0 + TC_M <= H;
   const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
   const int nkt = kt1 - kt0;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < TC_STAGES; ++i) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
-    }
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(done)) : "memory");
-    *abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     tc_sa(tslot)),
-                 "r"(NCOLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  rows[threadIdx.x] = list_row(p0 + threadIdx.x, H, N, F, idx);
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort);
+  if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tslot;
 
-  if (warp == 0 && lane == 0) {
-    // producer: k tiles kt0 .. kt1-1 of the tile's weight rows and of xh16
+  if (warp == 0) {
+    // producer warp: lane 0 arms the stage; in a gathered tile every lane
+    // then loads rows 4*lane .. 4*lane+3 of each weight operand
     const uint32_t tx = NR * A_BYTES + (uint32_t)nt * TC_BK * 2;
+    const int r = 4 * lane;
+    const int y0 = rows[r], y1 = rows[r + 1], y2 = rows[r + 2], y3 = rows[r + 3];
     int last[TC_STAGES];
     for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
       const int st = i % TC_STAGES;
-      if (i >= TC_STAGES && !tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr)) break;
+      int ok = 1;
+      if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       unsigned char* a = smem + st * STAGE;
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
-                   "r"(tx)
-                   : "memory");
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
+                     "r"(tx)
+                     : "memory");
+      __syncwarp();
       const int k = (kt0 + i) * TC_BK;
-      tma_load_2d(a, &mw0, k, tile * TC_M, &full[st]);
-      if constexpr (NR == 2) tma_load_2d(a + A_BYTES, &mw1, k, tile * TC_M, &full[st]);
-      tma_load_2d(a + NR * A_BYTES, &mx, k, 0, &full[st]);
-      last[st] = i;
-    }
-    // every copy issued here has landed before the CTA may exit (bounded)
-    for (int st = 0; st < TC_STAGES; ++st) {
-      if (last[st] < 0) continue;
-      const uint32_t par = (uint32_t)(last[st] / TC_STAGES) & 1u;
-      const uint64_t t0 = tc_time();
-      while (!tc_try(&full[st], par)) {
-        if (tc_time() - t0 > kTcTimeoutNs) {
-          if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
-          break;
+      if (dense) {
+        if (lane == 0) {
+          tma_load_2d(a, &mw0, k, p0, &full[st]);
+          if constexpr (NR == 2) tma_load_2d(a + A_BYTES, &mw1, k, p0, &full[st]);
         }
+      } else {
+        tma_gather4(a + 512u * lane, &mg0, k, y0, y1, y2, y3, &full[st]);
+        if constexpr (NR == 2)
+          tma_gather4(a + A_BYTES + 512u * lane, &mg1, k, y0, y1, y2, y3, &full[st]);
       }
+      if (lane == 0) {
+        tma_load_2d(a + NR * A_BYTES, &mx, k, 0, &full[st]);
+        last[st] = i;
+      }
+    }
+    if (lane == 0) {  // every copy of this CTA has landed before it may exit (bounded)
+      for (int st = 0; st < TC_STAGES; ++st)
+        if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer: kind::f16, fp16 A and B, fp32 D, both K-major, M = 128, N = nt
@@ -219,7 +291,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t bd = sw128_desc(b + 32u * kk);
         const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
         mma_f16(tmem, sw128_desc(a + 32u * kk), bd, idesc, acc);
-        if constexpr (NR == 2) mma_f16(tmem + (uint32_t)nt, sw128_desc(a + A_BYTES + 32u * kk), bd, idesc, acc);
+        if constexpr (NR == 2)
+          mma_f16(tmem + (uint32_t)nt, sw128_desc(a + A_BYTES + 32u * kk), bd, idesc, acc);
       }
       mma_commit(&empty[st]);  // the stage is free once these products have read it
     }
@@ -227,38 +300,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   __syncwarp();
 
-  // epilogue: warp w holds accumulator lanes [32w, 32w + 32) = hot neurons
-  // tile * 128 + 32w + lane, one column per token
-  // wait for `done` even after an abort: the MMA thread always commits it, so
-  // no product is still writing tensor memory when it is freed below
-  bool ok = tc_try(done, 0u);
-  if (!ok) {
-    const uint64_t t0 = tc_time();
-    while (!(ok = tc_try(done, 0u))) {
-      if (tc_time() - t0 > kTcTimeoutNs) {
-        if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
-        break;
-      }
-    }
-  }
+  // epilogue: warp w holds accumulator lanes [32w, 32w + 32) = list
+  // positions p0 + 32w + lane, one column per token.  `done` is awaited even
+  // after an abort, so no product still writes tensor memory when it is freed.
+  bool ok = tc_wait_quiet(done, 0u, hdr);
   ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   if (ok) {
-    const int n = tile * TC_M + warp * 32 + lane;
+    const int p = p0 + warp * 32 + lane;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-      float* dst = part + ((size_t)(split * NR + r) * H + n) * nt;
+      float* dst = part + ((size_t)(split * NR + r) * Fp + p) * nt;
       for (int c0 = 0; c0 < nt; c0 += 16) {
         uint32_t v[16];
-        const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(r * nt + c0);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-            "%11, %12, %13, %14, %15}, [%16];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-              "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-              "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(taddr));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(r * nt + c0), v);
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           __stcg(reinterpret_cast<float4*>(dst + c0) + q,
@@ -293,49 +348,60 @@ __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
   }
 }
 
-// h[n * batch + b] = act(sum over splits (fixed order) + bias) for n < H,
-// and its fp16 copy h16[b][n] (zero for the padding tokens b >= batch).
-// One block per 64 neurons: partial sums read and h16 written coalesced,
-// transposed through shared memory.
+// For list positions p of this block's 64: h = act(sum over splits (fixed
+// order) + bias), zero for a token whose own bit is 0 (per-token masks, cold
+// positions), for positions past the list and for bad list entries (which
+// also set DEV_BAD_INDEX); written as h16[t][p] (tokens t >= batch: 0).
+// Partial sums read and h16 written coalesced through shared memory.
 template <int NR>
-__global__ void __launch_bounds__(256) k_hot_finish(const float* __restrict__ part, int ks, int H,
-                                                    int nt, int batch,
+__global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ part, int ks,
+                                                    int H, int F, int Fp, int nt, int batch,
+                                                    const int32_t* __restrict__ idx,
+                                                    const int32_t* __restrict__ count,
                                                     const float* __restrict__ bias,
-                                                    float* __restrict__ h,
-                                                    __half* __restrict__ h16) {
+                                                    const uint32_t* __restrict__ mask, int words,
+                                                    __half* __restrict__ h16, WsHeader* hdr) {
   __shared__ float sh[64][TC_TMAX + 1];
+  const int N = list_len(count, H, F, hdr);
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&hdr->rows_listed, (unsigned long long)N);
   const int n0 = blockIdx.x * 64;
-  const int m = 64 * nt;  // this block's values per (split, matrix): contiguous
+  const int m = 64 * nt;
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
-    const int nn = i / nt, b = i % nt;
-    float g = 0.f, u = 0.f;
-    for (int s = 0; s < ks; ++s) {
-      g += __ldcg(part + ((size_t)(s * NR) * H + n0) * nt + i);
-      if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * H + n0) * nt + i);
-    }
+    const int nn = i / nt, b = i % nt, p = n0 + nn;
     float hv = 0.f;
-    if (b < batch) {
-      g += bias ? bias[n0 + nn] : 0.f;
-      hv = g > 0.f ? g : 0.f;
-      if constexpr (NR == 2) hv *= u;
-      h[(size_t)(n0 + nn) * batch + b] = hv;
+    if (p < N && b < batch) {
+      const int j = p < H ? p : idx[p - H];
+      if (p >= H && (j < H || j >= F)) {
+        if (b == 0 && hdr) atomicOr(&hdr->status, DEV_BAD_INDEX);
+      } else {
+        float g = 0.f, u = 0.f;
+        for (int s = 0; s < ks; ++s) {
+          g += __ldcg(part + ((size_t)(s * NR) * Fp + n0) * nt + i);
+          if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * Fp + n0) * nt + i);
+        }
+        g += bias ? bias[j] : 0.f;
+        hv = g > 0.f ? g : 0.f;
+        if constexpr (NR == 2) hv *= u;
+        if (mask && p >= H && !((mask[(size_t)b * words + (j >> 5)] >> (j & 31)) & 1u)) hv = 0.f;
+      }
     }
     sh[nn][b] = hv;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
     const int b = i / 64, nn = i % 64;
-    h16[(size_t)b * H + n0 + nn] = __float2half_rn(sh[nn][b]);
+    h16[(size_t)b * Fp + n0 + nn] = __float2half_rn(sh[nn][b]);
   }
 }
 
-// Partial rows part[split][b][c] = sum over the split's hot neurons j of
-// W_down^T[j][c] h16[b][j], for the tile's 128 columns c.  Grid (d / 128, ks).
+// down: part[split][b][c] = sum over the split's list positions p of
+// W_down^T[row(p)][c] h16[b][p], for the tile's 128 columns c.  Grid (d / 128, ks).
 __global__ void __launch_bounds__(TC_THREADS, 1)
-    k_hot_down_tc(const __grid_constant__ CUtensorMap mwd, const __grid_constant__ CUtensorMap mh,
-                  int nt, int nk, int ks, int d, int batch, int H, float* __restrict__ part,
-                  WsHeader* hdr) {
-  constexpr uint32_t BOX = 64 * TC_BK * 2;             // 64 columns x 64 neurons: 8 KB
+    k_ffn_down_tc(const __grid_constant__ CUtensorMap mwd, const __grid_constant__ CUtensorMap mwg,
+                  const __grid_constant__ CUtensorMap mh, int nt, int nk, int ks, int d, int batch,
+                  int H, int F, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
+                  float* __restrict__ part, WsHeader* hdr) {
+  constexpr uint32_t BOX = 64 * TC_BK * 2;             // 64 columns x 64 positions: 8 KB
   constexpr uint32_t A_BYTES = 2 * BOX;                // 128 columns
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;    // 8 KB
   constexpr uint32_t STAGE = A_BYTES + B_BYTES;
@@ -351,58 +417,60 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile = blockIdx.x, split = blockIdx.y;
-  const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
-  const int nkt = kt1 - kt0;
+  const int N = list_len(count, H, F, hdr);
+  const int nkN = (N + TC_BK - 1) / TC_BK;  // k tiles holding list positions
+  const int kt0 = (int)((long long)split * nk / ks);
+  int kt1 = (int)((long long)(split + 1) * nk / ks);
+  kt1 = kt1 < nkN ? kt1 : nkN;
+  const int nkt = kt1 > kt0 ? kt1 - kt0 : 0;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TC_STAGES; ++i) {
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
-    }
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(done)) : "memory");
-    *abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)H);
+    tc_init(full, empty, done, abort);
+    if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)N);
   }
-  if (warp == 0) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     tc_sa(tslot)),
-                 "r"(NCOLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tslot;
+  const int c0 = tile * TC_M;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     const uint32_t tx = A_BYTES + (uint32_t)nt * TC_BK * 2;
     int last[TC_STAGES];
     for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
       const int st = i % TC_STAGES;
-      if (i >= TC_STAGES && !tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr)) break;
+      int ok = 1;
+      if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       unsigned char* a = smem + st * STAGE;
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
-                   "r"(tx)
-                   : "memory");
-      const int j = (kt0 + i) * TC_BK;  // first hot neuron of the stage
-      tma_load_2d(a, &mwd, tile * TC_M, j, &full[st]);
-      tma_load_2d(a + BOX, &mwd, tile * TC_M + 64, j, &full[st]);
-      tma_load_2d(a + A_BYTES, &mh, j, 0, &full[st]);
-      last[st] = i;
-    }
-    for (int st = 0; st < TC_STAGES; ++st) {
-      if (last[st] < 0) continue;
-      const uint32_t par = (uint32_t)(last[st] / TC_STAGES) & 1u;
-      const uint64_t t0 = tc_time();
-      while (!tc_try(&full[st], par)) {
-        if (tc_time() - t0 > kTcTimeoutNs) {
-          if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
-          break;
+      if (lane == 0)
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
+                     "r"(tx)
+                     : "memory");
+      __syncwarp();
+      const int pk = (kt0 + i) * TC_BK;  // first list position of the stage
+      if (pk + TC_BK <= H) {
+        if (lane == 0) {
+          tma_load_2d(a, &mwd, c0, pk, &full[st]);
+          tma_load_2d(a + BOX, &mwd, c0 + 64, pk, &full[st]);
         }
+      } else {
+        // lanes 0..15: positions 4l .. 4l+3 of the first 64 columns; 16..31: of the next 64
+        const int half = lane >> 4, l = lane & 15, q = pk + 4 * l;
+        tma_gather4(a + half * BOX + 512u * l, &mwg, c0 + 64 * half, list_row(q, H, N, F, idx),
+                    list_row(q + 1, H, N, F, idx), list_row(q + 2, H, N, F, idx),
+                    list_row(q + 3, H, N, F, idx), &full[st]);
       }
+      if (lane == 0) {
+        tma_load_2d(a + A_BYTES, &mh, pk, 0, &full[st]);
+        last[st] = i;
+      }
+    }
+    if (lane == 0) {
+      for (int st = 0; st < TC_STAGES; ++st)
+        if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
     }
   } else if (warp == 1 && lane == 0) {
     // kind::f16, fp16 A (MN-major) and B (K-major), fp32 D, M = 128, N = nt
@@ -414,7 +482,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t a = tc_sa(smem + st * STAGE), b = a + A_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < TC_BK / 16; ++kk)  // 16 neurons = 2 K atoms of the A tile per MMA
+      for (int kk = 0; kk < TC_BK / 16; ++kk)  // 16 positions = 2 K atoms of the A tile per MMA
         mma_f16(tmem, sw128_mn_desc(a + 2048u * kk, BOX), sw128_desc(b + 32u * kk), idesc,
                 (i | kk) != 0 ? 1u : 0u);
       mma_commit(&empty[st]);
@@ -423,36 +491,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
   __syncwarp();
 
-  bool ok = tc_try(done, 0u);
-  if (!ok) {
-    const uint64_t t0 = tc_time();
-    while (!(ok = tc_try(done, 0u))) {
-      if (tc_time() - t0 > kTcTimeoutNs) {
-        if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
-        break;
-      }
-    }
-  }
-  ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
+  bool ok = tc_wait_quiet(done, 0u, hdr);
+  ok = __all_sync(0xffffffffu, ok && !*abort);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (ok) {
-    // accumulator lane = output column, accumulator column = token
-    const int c = tile * TC_M + warp * 32 + lane;
-    for (int c0 = 0; c0 < nt; c0 += 16) {
-      uint32_t v[16];
-      const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0;
-      asm volatile(
-          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
-          "%11, %12, %13, %14, %15}, [%16];"
-          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-            "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-            "=r"(v[14]), "=r"(v[15])
-          : "r"(taddr));
-      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  // accumulator lane = output column, accumulator column = token; a split
+  // with no list positions writes zeros (the reduction sums every slice)
+  const int c = c0 + warp * 32 + lane;
+  for (int t0 = 0; t0 < nt; t0 += 16) {
+    uint32_t v[16];
+    if (ok && nkt > 0) {
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)t0, v);
+    } else {
 #pragma unroll
-      for (int t = 0; t < 16; ++t)
-        if (c0 + t < batch) __stcg(part + ((size_t)split * batch + c0 + t) * d + c, __uint_as_float(v[t]));
+      for (int t = 0; t < 16; ++t) v[t] = 0u;
     }
+#pragma unroll
+    for (int t = 0; t < 16; ++t)
+      if (t0 + t < batch) __stcg(part + ((size_t)split * batch + t0 + t) * d + c, __uint_as_float(v[t]));
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -476,7 +531,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 }
 
 // 2-D fp16 tensor [rows][inner] with `row_bytes` between rows; box
-// [box_rows][64], 128-byte swizzle.
+// [box_rows][64], 128-byte swizzle (box_rows = 1 for gather4 maps).
 bool map_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
             uint32_t box_rows) {
   auto enc = tensor_map_encoder();
@@ -497,23 +552,7 @@ bool tc_disabled() {
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
-// Scratch: xh16 [64][d] fp16 | partial sums [4][2][hot][64] fp32 | h16 [64][hot] fp16.
-struct TcScratch {
-  __half* xh16;
-  float* part;
-  __half* h16;
-};
-
-TcScratch tc_scratch(void* base, int d, int H) {
-  char* p = static_cast<char*>(base);
-  TcScratch t;
-  t.xh16 = reinterpret_cast<__half*>(p);
-  p += up256((size_t)TC_TMAX * d * 2);
-  t.part = reinterpret_cast<float*>(p);
-  p += up256((size_t)TC_KSMAX * 2 * H * TC_TMAX * 4);
-  t.h16 = reinterpret_cast<__half*>(p);
-  return t;
-}
+int fpad(int F) { return (F + TC_M - 1) / TC_M * TC_M; }
 
 int split_for(int tiles, int nk) {
   int ks = device_sms() / tiles;
@@ -521,83 +560,115 @@ int split_for(int tiles, int nk) {
   return ks > nk ? nk : ks;
 }
 
+// splits of the up GEMM's d for a layer shape
+int up_splits(int d, int F) { return split_for(fpad(F) / TC_M, d / TC_BK); }
+
+// Scratch: xh16 [64][d] fp16 | up partial sums [ks][2][Fp][64] fp32 | h16 [64][Fp] fp16.
+struct TcScratch {
+  __half* xh16;
+  float* part;
+  __half* h16;
+};
+
+TcScratch tc_scratch(void* base, int d, int F) {
+  char* p = static_cast<char*>(base);
+  TcScratch t;
+  t.xh16 = reinterpret_cast<__half*>(p);
+  p += up256((size_t)TC_TMAX * d * 2);
+  t.part = reinterpret_cast<float*>(p);
+  p += up256((size_t)up_splits(d, F) * 2 * fpad(F) * TC_TMAX * 4);
+  t.h16 = reinterpret_cast<__half*>(p);
+  return t;
+}
+
 template <int NR>
-cudaError_t launch_nr(const pi_layer& L, const float* xh, int batch, float* h, void* scratch,
-                      WsHeader* hdr, cudaStream_t s) {
-  const int d = L.d_model, H = L.hot;
+cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                         const int32_t* idx, const int32_t* count, void* scratch, WsHeader* hdr,
+                         cudaStream_t s) {
+  const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
-  const TcScratch sc = tc_scratch(scratch, d, H);
-  __half* xh16 = sc.xh16;
-  float* part = sc.part;
+  const TcScratch sc = tc_scratch(scratch, d, F);
   const int64_t rs = code_stride(PI_F16, d, L.w_row_stride);
-  CUtensorMap m0, m1, mx;
   const void* w0 = NR == 2 ? L.w_gate : L.w_up;
-  if (!map_2d(&m0, w0, (uint64_t)d, (uint64_t)H, (uint64_t)rs, TC_M) ||
-      !map_2d(&m1, L.w_up, (uint64_t)d, (uint64_t)H, (uint64_t)rs, TC_M) ||
-      !map_2d(&mx, xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt))
+  CUtensorMap m0, m1, g0, g1, mx;
+  if (!map_2d(&m0, w0, (uint64_t)d, (uint64_t)F, (uint64_t)rs, TC_M) ||
+      !map_2d(&m1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs, TC_M) ||
+      !map_2d(&g0, w0, (uint64_t)d, (uint64_t)F, (uint64_t)rs, 1) ||
+      !map_2d(&g1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs, 1) ||
+      !map_2d(&mx, sc.xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt))
     return cudaErrorInvalidValue;
-  k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt, xh16);
+  k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt,
+                                                                              sc.xh16);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int tiles = H / TC_M, nk = d / TC_BK;
-  const int ks = split_for(tiles, nk);
+  const int tiles = Fp / TC_M, nk = d / TC_BK, ks = up_splits(d, F);
   constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
-  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
-  auto kern = k_hot_up_tc<NR>;
+  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16 + 4 * TC_M;
+  auto kern = k_ffn_up_tc<NR>;
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(m0, m1, mx, nt, nk, ks, H, part, hdr);
+  kern<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, ks, H, F, Fp, idx,
+                                                 count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_hot_finish<NR><<<H / 64, 256, 0, s>>>(part, ks, H, nt, batch, L.bias, h, sc.h16);
+  k_ffn_finish<NR><<<Fp / 64, 256, 0, s>>>(sc.part, ks, H, F, Fp, nt, batch, idx, count, L.bias,
+                                           mask, (F + 31) / 32, sc.h16, hdr);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-bool hot_tc_supported(const pi_layer& L, int batch) {
+bool ffn_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
   if (L.w_dtype != PI_F16 || batch < 16 || batch > TC_TMAX) return false;
-  if (L.hot < TC_M || L.hot % TC_M != 0 || L.d_model % TC_M != 0) return false;
+  if (L.d_model % TC_M != 0) return false;
   const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
   const int64_t rd = code_stride(PI_F16, L.d_model, L.w_down_row_stride);
-  if (rs % 16 != 0 || rd % 16 != 0 || ((uintptr_t)L.w_down_t & 15u)) return false;
-  const uintptr_t bases = (uintptr_t)L.w_up | (uintptr_t)(L.act == PI_REGLU ? L.w_gate : L.w_up);
+  if (rs % 16 != 0 || rd % 16 != 0) return false;
+  const uintptr_t bases = (uintptr_t)L.w_up | (uintptr_t)L.w_down_t |
+                          (uintptr_t)(L.act == PI_REGLU ? L.w_gate : L.w_up);
   if (bases & 15u) return false;
   return tensor_map_encoder() != nullptr;
 }
 
-size_t hot_tc_scratch_bytes(int d_model, int hot, int batch) {
-  if (batch < 16 || hot < TC_M) return 0;
-  return up256((size_t)TC_TMAX * d_model * 2) + up256((size_t)TC_KSMAX * 2 * hot * TC_TMAX * 4) +
-         (size_t)TC_TMAX * hot * 2;
+size_t ffn_tc_scratch_bytes(int d_model, int d_ff, int batch) {
+  if (batch < 16 || d_model % TC_M != 0) return 0;
+  return up256((size_t)TC_TMAX * d_model * 2) +
+         up256((size_t)up_splits(d_model, d_ff) * 2 * fpad(d_ff) * TC_TMAX * 4) +
+         (size_t)TC_TMAX * fpad(d_ff) * 2;
 }
 
-int hot_tc_down_splits(const pi_layer& L) { return split_for(L.d_model / TC_M, L.hot / TC_BK); }
+int ffn_tc_down_splits(const pi_layer& L) {
+  return split_for(L.d_model / TC_M, fpad(L.d_ff) / TC_BK);
+}
 
-cudaError_t launch_hot_down_tc(const pi_layer& L, int batch, float* part, void* scratch,
-                               WsHeader* hdr, cudaStream_t s) {
-  const int d = L.d_model, H = L.hot;
+cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                             const int32_t* idx, const int32_t* count, void* scratch,
+                             WsHeader* hdr, cudaStream_t s) {
+  return L.act == PI_REGLU ? launch_up_nr<2>(L, xh, batch, mask, idx, count, scratch, hdr, s)
+                           : launch_up_nr<1>(L, xh, batch, mask, idx, count, scratch, hdr, s);
+}
+
+cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
+                               const int32_t* count, float* part, void* scratch, WsHeader* hdr,
+                               cudaStream_t s) {
+  const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
-  const TcScratch sc = tc_scratch(scratch, d, H);
+  const TcScratch sc = tc_scratch(scratch, d, F);
   const int64_t rd = code_stride(PI_F16, d, L.w_down_row_stride);
-  CUtensorMap mwd, mh;
-  if (!map_2d(&mwd, L.w_down_t, (uint64_t)d, (uint64_t)H, (uint64_t)rd, TC_BK) ||
-      !map_2d(&mh, sc.h16, (uint64_t)H, (uint64_t)nt, (uint64_t)H * 2, (uint32_t)nt))
+  CUtensorMap mwd, mwg, mh;
+  if (!map_2d(&mwd, L.w_down_t, (uint64_t)d, (uint64_t)F, (uint64_t)rd, TC_BK) ||
+      !map_2d(&mwg, L.w_down_t, (uint64_t)d, (uint64_t)F, (uint64_t)rd, 1) ||
+      !map_2d(&mh, sc.h16, (uint64_t)Fp, (uint64_t)nt, (uint64_t)Fp * 2, (uint32_t)nt))
     return cudaErrorInvalidValue;
-  const int tiles = d / TC_M, nk = H / TC_BK, ks = hot_tc_down_splits(L);
+  const int tiles = d / TC_M, nk = Fp / TC_BK, ks = ffn_tc_down_splits(L);
   constexpr uint32_t STAGE = 2 * 64 * TC_BK * 2 + TC_TMAX * TC_BK * 2;
   const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
-  cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_hot_down_tc), smem);
+  cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_down_tc), smem);
   if (e != cudaSuccess) return e;
-  k_hot_down_tc<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(mwd, mh, nt, nk, ks, d, batch, H, part, hdr);
+  k_ffn_down_tc<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(mwd, mwg, mh, nt, nk, ks, d, batch, H, F,
+                                                          idx, count, part, hdr);
   return cudaGetLastError();
-}
-
-cudaError_t launch_hot_up_tc(const pi_layer& L, const float* xh, int batch, float* h,
-                             void* scratch, WsHeader* hdr, cudaStream_t s) {
-  return L.act == PI_REGLU ? launch_nr<2>(L, xh, batch, h, scratch, hdr, s)
-                           : launch_nr<1>(L, xh, batch, h, scratch, hdr, s);
 }
 
 }  // namespace pi

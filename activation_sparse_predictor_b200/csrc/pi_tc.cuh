@@ -1,5 +1,5 @@
-// Tensor-core (tcgen05) path for the dense hot prefix at token batches
-// (host interface, internal).
+// Tensor-core (tcgen05) path for the FFN at token batches (host interface,
+// internal).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -10,29 +10,30 @@
 
 namespace pi {
 
-// True when the hot prefix's gate/up products and down projection of this
-// layer at this batch run on tensor cores: fp16 weights, 16 <= batch <= 64,
-// hot % 128 == 0 and hot >= 128, d_model % 128 == 0 (and PI_DISABLE_TC unset).
-bool hot_tc_supported(const pi_layer& L, int batch);
+// True when this layer's listed rows (hot prefix, then the cold list) run
+// on the tensor cores at this batch: fp16 weights, 16 <= batch <= 64,
+// d_model % 128 == 0, 16-byte row strides (and PI_DISABLE_TC unset).
+bool ffn_tc_supported(const pi_layer& L, int batch);
 
-// Workspace bytes the path needs for a layer of this shape (0 if unused).
-size_t hot_tc_scratch_bytes(int d_model, int hot, int batch);
+// Workspace bytes the path needs for a layer shape at this batch (0: none).
+size_t ffn_tc_scratch_bytes(int d_model, int d_ff, int batch);
 
-// h[n * batch + b] for every hot row n < hot and token b < batch: the
-// activation of the hot neurons' gate/up products with xh [batch][d_model]
-// (fp32, rounded to fp16 for the tensor cores; fp32 accumulation).
-// `scratch`: hot_tc_scratch_bytes(...) bytes, 256-byte aligned.
-cudaError_t launch_hot_up_tc(const pi_layer& L, const float* xh, int batch, float* h,
-                             void* scratch, WsHeader* hdr, cudaStream_t s);
+// Up/gate products of list positions [0, hot + count) (row p for p < hot,
+// idx[p - hot] after) with xh [batch][d_model] (fp32, rounded to fp16 for
+// the tensor cores; fp32 accumulation), bias, ReLU / ReGLU, each token's own
+// mask bit for cold rows when `mask` ([batch][words]) is given; leaves the
+// fp16 activations in `scratch` for launch_ffn_down_tc.
+cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                             const int32_t* idx, const int32_t* count, void* scratch,
+                             WsHeader* hdr, cudaStream_t s);
 
-// Split-K slices the hot down projection writes (part[0 .. splits)).
-int hot_tc_down_splits(const pi_layer& L);
+// Split-K slices the down projection writes (part[0 .. splits)).
+int ffn_tc_down_splits(const pi_layer& L);
 
-// part[k][b][:] for k < hot_tc_down_splits(L): the hot rows' contribution
-// sum_{j < hot} h[j][b] * w_down_t[j] (from the fp16 h that
-// launch_hot_up_tc left in `scratch`), split over the hot rows in a fixed
-// order; adds hot to the workspace's down-row counter.
-cudaError_t launch_hot_down_tc(const pi_layer& L, int batch, float* part, void* scratch,
-                               WsHeader* hdr, cudaStream_t s);
+// part[k][b][:] for k < ffn_tc_down_splits(L): sum over the k-th share of
+// the list positions of h[p][b] * w_down_t[row(p)].
+cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
+                               const int32_t* count, float* part, void* scratch, WsHeader* hdr,
+                               cudaStream_t s);
 
 }  // namespace pi

@@ -275,15 +275,20 @@ def test_stack_is_deterministic(pi, packed):
     assert torch.equal(outs[0], outs[1])
 
 
+@pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0)])
 @pytest.mark.parametrize("act", ["relu", "reglu"])
-@pytest.mark.parametrize("batch", [16, 20, 48, 64])
-def test_hot_prefix_on_tensor_cores(pi, orc, act, batch, monkeypatch):
-    """At 16-64 tokens the dense hot prefix (fp16) runs on the tensor cores
-    (fp16 inputs, fp32 accumulation): within the fp16 tolerance of the
-    oracle, close to the CUDA-core path, and not bitwise equal to it (so the
-    tensor-core path did run).  Batches 20 and 48 pad the token tile."""
-    w = _wl(act, "f16", (1024, 3001, 128, 640), seed=47)
-    L, _ = device_layer(w, 0, packed=(batch % 2 == 0))
+@pytest.mark.parametrize("batch,mode", [(16, "per_token"), (20, "union"), (48, "per_token"),
+                                        (64, "union")])
+def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
+    """At 16-64 tokens an fp16 layer's listed rows (hot prefix and cold list;
+    whole-hot tiles loaded as boxes, the others gathered four rows per TMA
+    load) run on the tensor cores (fp16 inputs, fp32 accumulation): within
+    the fp16 tolerance of the oracle, close to the CUDA-core path, and not
+    bitwise equal to it (so the tensor-core path did run).  Shapes cover a
+    ragged d_ff, a hot prefix that ends inside a tile, and no hot prefix;
+    batches 20 and 48 pad the token tile."""
+    w = _wl(act, "f16", shape, seed=47)
+    L, _ = device_layer(w, 0, packed=(batch % 32 == 0))
     H = synth.layer_host(w, 0)
     xh = _xh(w.d_model, batch, 9)
     masks, _ = _oracle_masks(orc, H, w, xh)
@@ -292,9 +297,11 @@ def test_hot_prefix_on_tensor_cores(pi, orc, act, batch, monkeypatch):
     dev_idx[: len(union)] = torch.from_numpy(union).cuda()
     dev_cnt = torch.tensor([len(union)], dtype=torch.int32, device="cuda")
     dxh = torch.from_numpy(xh).cuda()
+    dmask = torch.from_numpy(masks.view(np.int32)).cuda()
+    m = pi.MODES[mode]
 
     def run():
-        return pi.pi_sparse_ffn(L, dxh, None, dev_idx, dev_cnt, pi.PI_MASK_UNION).cpu().numpy()
+        return pi.pi_sparse_ffn(L, dxh, dmask, dev_idx, dev_cnt, m).cpu().numpy()
 
     y_tc = run()
     monkeypatch.setenv("PI_DISABLE_TC", "1")
@@ -302,7 +309,11 @@ def test_hot_prefix_on_tensor_cores(pi, orc, act, batch, monkeypatch):
     monkeypatch.delenv("PI_DISABLE_TC")
     assert not np.array_equal(y_tc, y_cc)
     for b in range(batch):
-        ref = orc.sparse_ffn(H, xh[b].astype(np.float64), union)
+        own = orc.compact(masks[b], w.d_ff, w.hot) if mode == "per_token" else union
+        ref = orc.sparse_ffn(H, xh[b].astype(np.float64), own)
+        if np.linalg.norm(ref) == 0.0:
+            assert np.all(y_tc[b] == 0.0)
+            continue
         assert rel_l2(y_tc[b], ref) <= TOL["f16"], b
         assert rel_l2(y_tc[b], y_cc[b]) <= 2e-3, b
     assert np.array_equal(run(), y_tc)  # deterministic
