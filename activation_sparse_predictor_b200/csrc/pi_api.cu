@@ -94,13 +94,13 @@ WsLayout layout_for(int d, int F, int r, int batch, int H) {
   // split-K partials: the multi-kernel split, or one slice per SM for the
   // fused single-token stack
   // (+ up to 4 slices of the tensor-core hot prefix at token batches)
-  const size_t tcp = ffn_tc_scratch_bytes(d, F, batch) ? (size_t)4 * batch : 0;
+  const size_t tcp = tc_scratch_bytes(d, F, r, batch) ? (size_t)4 * batch : 0;
   const size_t parts = (size_t)w.splits * batch + tcp > 2 * (size_t)device_sms()
                            ? (size_t)w.splits * batch + tcp
                            : 2 * (size_t)device_sms();
   w.part = take(parts * d * 4);
   w.y = take((size_t)batch * d * 4);
-  w.tc = take(ffn_tc_scratch_bytes(d, F, batch));
+  w.tc = take(tc_scratch_bytes(d, F, r, batch));
   w.total = off;
   return w;
 }
@@ -188,6 +188,28 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
   return PI_OK;
 }
 
+// mask [batch][words] of xh: the predictor (tensor cores at token batches).
+pi_status predict_body(const pi_layer& L, const float* xh, int batch, float theta, uint32_t* mask,
+                       void* ws, const WsLayout& lay, cudaStream_t s, Prof* prof = nullptr) {
+  Prof none;
+  Prof& P = prof ? *prof : none;
+  cudaError_t e;
+  if (pred_tc_supported(L, batch)) {
+    P.before(PI_KIND_PRED_U);
+    e = launch_predict_tc(L, xh, batch, theta, mask, at<void>(ws, lay.tc), header(ws), s);
+    P.after();
+    return e == cudaSuccess ? PI_OK : cuda_fail(e, "predictor (tensor cores) launch");
+  }
+  P.before(PI_KIND_PRED_U);
+  e = launch_pred_u(L, xh, batch, at<float>(ws, lay.u), s);
+  P.after();
+  if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
+  P.before(PI_KIND_PRED_Z);
+  e = launch_pred_z(L, at<float>(ws, lay.u), batch, theta, mask, s);
+  P.after();
+  return e == cudaSuccess ? PI_OK : cuda_fail(e, "pred_z launch");
+}
+
 pi_status stack_check(const pi_layer* layers, int n_layers, float* x, int batch, float tau,
                       int mode, uint32_t* mask_trace, void* ws, size_t ws_bytes, WsLayout* lay) {
   if (!layers || n_layers < 1) return fail(PI_ERR_INVALID, "need at least one layer");
@@ -240,14 +262,7 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
     cudaError_t e = launch_rmsnorm(x, batch, d, xh, s);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
-    P.before(PI_KIND_PRED_U);
-    e = launch_pred_u(L, xh, batch, at<float>(ws, lay.u), s);
-    P.after();
-    if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
-    P.before(PI_KIND_PRED_Z);
-    e = launch_pred_z(L, at<float>(ws, lay.u), batch, theta, mask, s);
-    P.after();
-    if (e != cudaSuccess) return cuda_fail(e, "pred_z launch");
+    if ((st = predict_body(L, xh, batch, theta, mask, ws, lay, s, prof)) != PI_OK) return st;
     P.before(PI_KIND_COMPACT);
     e = launch_compact(mask, batch, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);
     P.after();
@@ -337,12 +352,7 @@ pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float ta
   if (!mask || !aligned(mask, 4)) return fail(PI_ERR_INVALID, "mask null or misaligned");
   const WsLayout lay = layout_for_layers(layer, 1, batch);
   if ((st = check_ws(ws, ws_bytes, lay)) != PI_OK) return st;
-  cudaStream_t s = (cudaStream_t)stream;
-  cudaError_t e = launch_pred_u(*layer, xh, batch, at<float>(ws, lay.u), s);
-  if (e != cudaSuccess) return cuda_fail(e, "pred_u launch");
-  e = launch_pred_z(*layer, at<float>(ws, lay.u), batch, logit32(tau), mask, s);
-  if (e != cudaSuccess) return cuda_fail(e, "pred_z launch");
-  return PI_OK;
+  return predict_body(*layer, xh, batch, logit32(tau), mask, ws, lay, (cudaStream_t)stream);
 }
 
 pi_status pi_predict_noalloc(const pi_layer* layer, const float* xh, int batch, float tau,

@@ -15,6 +15,13 @@
 //          operand; the list positions split over up to 4 CTAs; the partial
 //          rows go to the fixed-order split-K reduction.
 //
+// The predictor at token batches is two more contractions: u = P1 xh and
+// z = P2[H:] u.  Their results decide mask bits, so the fp32 vector operand
+// is split into two fp16 parts (hi + lo, ~22 bits) and both products
+// accumulate into the same fp32 accumulator; z's epilogue adds the bias,
+// compares with logit(tau) and turns each warp's 32 consecutive rows into
+// one mask word per token with a ballot.
+//
 // A tile whose rows all lie in the hot prefix is one TMA box per operand
 // and stage; any other tile is gathered: each lane of the producer warp
 // issues one TMA tile::gather4 load (four rows, a one-row-high box) per
@@ -516,6 +523,155 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                  : "memory");
 }
 
+constexpr int TC_KSMAX_U = 16;  // CTAs sharing one tile of P1's d at most
+
+// x (fp32 [batch][n]) -> hi = fp16(x), lo = fp16(x - hi), [nt][n] each
+// (rows >= batch zero).
+__global__ void k_split16(const float* __restrict__ x, int batch, int n, int nt,
+                          __half* __restrict__ hi, __half* __restrict__ lo) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt * n; i += gridDim.x * blockDim.x) {
+    const int t = i / n;
+    const float v = t < batch ? x[i] : 0.f;
+    const __half h = __float2half_rn(v);
+    hi[i] = h;
+    lo[i] = __float2half_rn(v - __half2float(h));
+  }
+}
+
+// MODE 0: D = P1 (x_hi + x_lo)^T for 128 predictor rows per tile, d split
+// over ks CTAs -> part[split][row][nt].  MODE 1: D = P2 (u_hi + u_lo)^T for
+// 128 neuron rows per tile from row0 (a multiple of 32, <= hot) -> mask
+// words: bit j of token t = (j < hot) or (z_j + c_j > theta) for j < d_ff.
+// Grid (tiles, ks).
+template <int MODE>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    k_pred_tc(const __grid_constant__ CUtensorMap ma, const __grid_constant__ CUtensorMap mbh,
+              const __grid_constant__ CUtensorMap mbl, int nt, int nk, int ks, int row0, int M,
+              float* __restrict__ part, const float* __restrict__ bias, float theta, int H,
+              uint32_t* __restrict__ mask, int words, int batch, WsHeader* hdr) {
+  constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
+  constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB per part
+  constexpr uint32_t STAGE = A_BYTES + 2 * B_BYTES;
+  constexpr uint32_t NCOLS = 64u;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = tc_sa(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_STAGES * STAGE);
+  uint64_t* empty = full + TC_STAGES;
+  uint64_t* done = empty + TC_STAGES;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int m0 = row0 + tile * TC_M;
+  const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
+  const int nkt = kt1 - kt0;
+
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort);
+  if (warp == 0) tmem_alloc(tslot, NCOLS);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tslot;
+
+  if (warp == 0 && lane == 0) {
+    const uint32_t tx = A_BYTES + 2u * (uint32_t)nt * TC_BK * 2;
+    int last[TC_STAGES];
+    for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % TC_STAGES;
+      if (i >= TC_STAGES && !tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr)) break;
+      unsigned char* a = smem + st * STAGE;
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
+                   "r"(tx)
+                   : "memory");
+      const int k = (kt0 + i) * TC_BK;
+      tma_load_2d(a, &ma, k, m0, &full[st]);  // rows past the matrix read zeros
+      tma_load_2d(a + A_BYTES, &mbh, k, 0, &full[st]);
+      tma_load_2d(a + A_BYTES + B_BYTES, &mbl, k, 0, &full[st]);
+      last[st] = i;
+    }
+    for (int st = 0; st < TC_STAGES; ++st)
+      if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
+  } else if (warp == 1 && lane == 0) {
+    const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % TC_STAGES;
+      if (!tc_wait(&full[st], (uint32_t)(i / TC_STAGES) & 1u, abort, hdr)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = tc_sa(smem + st * STAGE), bh = a + A_BYTES, bl = bh + B_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk) {
+        const uint64_t ad = sw128_desc(a + 32u * kk);
+        mma_f16(tmem, ad, sw128_desc(bh + 32u * kk), idesc, (i | kk) != 0 ? 1u : 0u);
+        mma_f16(tmem, ad, sw128_desc(bl + 32u * kk), idesc, 1u);
+      }
+      mma_commit(&empty[st]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  bool ok = tc_wait_quiet(done, 0u, hdr);
+  ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const int m = m0 + warp * 32 + lane;  // this thread's row
+  for (int c0 = 0; c0 < nt; c0 += 16) {
+    uint32_t v[16];
+    if (ok) {
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+    } else {
+#pragma unroll
+      for (int t = 0; t < 16; ++t) v[t] = 0u;
+    }
+    if constexpr (MODE == 0) {
+      if (m < M) {
+        float* dst = part + ((size_t)split * M + m) * nt + c0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          __stcg(reinterpret_cast<float4*>(dst) + q,
+                 make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+      }
+    } else {
+      const float cb = (bias && m < M) ? bias[m] : 0.f;
+      const int w = (m0 + warp * 32) >> 5;  // this warp's mask word
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const bool bit = m < H || (m < M && __uint_as_float(v[t]) + cb > theta);
+        const uint32_t word = __ballot_sync(0xffffffffu, bit);
+        if (lane == 0 && c0 + t < batch && w < words) mask[(size_t)(c0 + t) * words + w] = word;
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS)
+                 : "memory");
+}
+
+// u = sum over the splits (fixed order) -> u_hi, u_lo [nt][r] (tokens >= batch: 0).
+__global__ void k_pred_u_finish(const float* __restrict__ part, int ks, int r, int nt, int batch,
+                                __half* __restrict__ uhi, __half* __restrict__ ulo) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < r * nt; i += gridDim.x * blockDim.x) {
+    const int k = i / nt, t = i % nt;
+    float u = 0.f;
+    if (t < batch)
+      for (int s = 0; s < ks; ++s) u += __ldcg(part + ((size_t)s * r + k) * nt + t);
+    const __half h = __float2half_rn(u);
+    uhi[(size_t)t * r + k] = h;
+    ulo[(size_t)t * r + k] = __float2half_rn(u - __half2float(h));
+  }
+}
+
+// Mask words below the first evaluated row: all hot, all ones.
+__global__ void k_hot_words(uint32_t* __restrict__ mask, int words, int w0, int batch) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < batch * w0; i += gridDim.x * blockDim.x)
+    mask[(size_t)(i / w0) * words + i % w0] = 0xFFFFFFFFu;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static std::mutex mu;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -563,21 +719,45 @@ int split_for(int tiles, int nk) {
 // splits of the up GEMM's d for a layer shape
 int up_splits(int d, int F) { return split_for(fpad(F) / TC_M, d / TC_BK); }
 
-// Scratch: xh16 [64][d] fp16 | up partial sums [ks][2][Fp][64] fp32 | h16 [64][Fp] fp16.
+int pred_u_splits(int d, int r) {
+  int ks = device_sms() / (r / TC_M);
+  ks = ks < 1 ? 1 : (ks > TC_KSMAX_U ? TC_KSMAX_U : ks);
+  return ks > d / TC_BK ? d / TC_BK : ks;
+}
+
+// Scratch: xh16 [64][d] fp16 | up partial sums [ks][2][Fp][64] fp32 |
+// h16 [64][Fp] fp16 | predictor: xs_lo [64][d] fp16 | u partial sums
+// [ksu][r][64] fp32 | u_hi, u_lo [64][r] fp16 (xh16 doubles as xs_hi).
 struct TcScratch {
   __half* xh16;
   float* part;
   __half* h16;
+  __half* xlo;
+  float* upart;
+  __half* uhi;
+  __half* ulo;
+  size_t bytes;
 };
 
-TcScratch tc_scratch(void* base, int d, int F) {
-  char* p = static_cast<char*>(base);
+TcScratch tc_scratch(void* base, int d, int F, int r) {
+  char* p0 = static_cast<char*>(base);
+  char* p = p0;
   TcScratch t;
   t.xh16 = reinterpret_cast<__half*>(p);
   p += up256((size_t)TC_TMAX * d * 2);
   t.part = reinterpret_cast<float*>(p);
   p += up256((size_t)up_splits(d, F) * 2 * fpad(F) * TC_TMAX * 4);
   t.h16 = reinterpret_cast<__half*>(p);
+  p += up256((size_t)TC_TMAX * fpad(F) * 2);
+  t.xlo = reinterpret_cast<__half*>(p);
+  p += up256((size_t)TC_TMAX * d * 2);
+  t.upart = reinterpret_cast<float*>(p);
+  p += up256(r % TC_M == 0 ? (size_t)pred_u_splits(d, r) * r * TC_TMAX * 4 : 0);
+  t.uhi = reinterpret_cast<__half*>(p);
+  p += up256((size_t)TC_TMAX * r * 2);
+  t.ulo = reinterpret_cast<__half*>(p);
+  p += up256((size_t)TC_TMAX * r * 2);
+  t.bytes = (size_t)(p - p0);
   return t;
 }
 
@@ -587,7 +767,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
                          cudaStream_t s) {
   const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
-  const TcScratch sc = tc_scratch(scratch, d, F);
+  const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
   const int64_t rs = code_stride(PI_F16, d, L.w_row_stride);
   const void* w0 = NR == 2 ? L.w_gate : L.w_up;
   CUtensorMap m0, m1, g0, g1, mx;
@@ -631,11 +811,64 @@ bool ffn_tc_supported(const pi_layer& L, int batch) {
   return tensor_map_encoder() != nullptr;
 }
 
-size_t ffn_tc_scratch_bytes(int d_model, int d_ff, int batch) {
+size_t tc_scratch_bytes(int d_model, int d_ff, int rank, int batch) {
   if (batch < 16 || d_model % TC_M != 0) return 0;
-  return up256((size_t)TC_TMAX * d_model * 2) +
-         up256((size_t)up_splits(d_model, d_ff) * 2 * fpad(d_ff) * TC_TMAX * 4) +
-         (size_t)TC_TMAX * fpad(d_ff) * 2;
+  return tc_scratch(nullptr, d_model, d_ff, rank).bytes;
+}
+
+bool pred_tc_supported(const pi_layer& L, int batch) {
+  if (tc_disabled()) return false;
+  if (L.p_dtype != PI_F16 || batch < 16 || batch > TC_TMAX) return false;
+  if (L.rank % TC_M != 0 || L.d_model % TC_M != 0) return false;
+  if (((uintptr_t)L.p1 | (uintptr_t)L.p2) & 15u) return false;
+  return tensor_map_encoder() != nullptr;
+}
+
+cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, float theta,
+                              uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s) {
+  const int d = L.d_model, r = L.rank, F = L.d_ff, H = L.hot, words = (F + 31) / 32;
+  const int nt = (batch + 15) / 16 * 16;
+  const TcScratch sc = tc_scratch(scratch, d, F, r);
+  CUtensorMap m1, mxh, mxl, m2, muh, mul;
+  if (!map_2d(&m1, L.p1, (uint64_t)d, (uint64_t)r, (uint64_t)d * 2, TC_M) ||
+      !map_2d(&mxh, sc.xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt) ||
+      !map_2d(&mxl, sc.xlo, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt) ||
+      !map_2d(&m2, L.p2, (uint64_t)r, (uint64_t)F, (uint64_t)r * 2, TC_M) ||
+      !map_2d(&muh, sc.uhi, (uint64_t)r, (uint64_t)nt, (uint64_t)r * 2, (uint32_t)nt) ||
+      !map_2d(&mul, sc.ulo, (uint64_t)r, (uint64_t)nt, (uint64_t)r * 2, (uint32_t)nt))
+    return cudaErrorInvalidValue;
+  const int grid = device_sms() * 4;
+  k_split16<<<std::min((nt * d + 255) / 256, grid), 256, 0, s>>>(xh, batch, d, nt, sc.xh16, sc.xlo);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  constexpr uint32_t STAGE = TC_M * TC_BK * 2 + 2 * TC_TMAX * TC_BK * 2;
+  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
+  e = allow_smem_fn(reinterpret_cast<const void*>(k_pred_tc<0>), smem);
+  if (e == cudaSuccess) e = allow_smem_fn(reinterpret_cast<const void*>(k_pred_tc<1>), smem);
+  if (e != cudaSuccess) return e;
+  // u = P1 xh
+  const int ksu = pred_u_splits(d, r);
+  k_pred_tc<0><<<dim3(r / TC_M, ksu), TC_THREADS, smem, s>>>(m1, mxh, mxl, nt, d / TC_BK, ksu, 0, r,
+                                                             sc.upart, nullptr, 0.f, 0, nullptr, 0,
+                                                             batch, hdr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  k_pred_u_finish<<<std::min((r * nt + 255) / 256, grid), 256, 0, s>>>(sc.upart, ksu, r, nt, batch,
+                                                                       sc.uhi, sc.ulo);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // z = P2 u + c for rows from the word holding `hot`; the words below it are hot
+  const int w0 = H / 32, row0 = 32 * w0;
+  if (w0 > 0) {
+    k_hot_words<<<std::min((batch * w0 + 255) / 256, grid), 256, 0, s>>>(mask, words, w0, batch);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (row0 < F) {
+    const int tiles = (F - row0 + TC_M - 1) / TC_M;
+    k_pred_tc<1><<<dim3(tiles, 1), TC_THREADS, smem, s>>>(m2, muh, mul, nt, r / TC_BK, 1, row0, F,
+                                                          nullptr, L.p_bias, theta, H, mask, words,
+                                                          batch, hdr);
+    e = cudaGetLastError();
+  }
+  return e;
 }
 
 int ffn_tc_down_splits(const pi_layer& L) {
@@ -654,7 +887,7 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
                                cudaStream_t s) {
   const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
-  const TcScratch sc = tc_scratch(scratch, d, F);
+  const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
   const int64_t rd = code_stride(PI_F16, d, L.w_down_row_stride);
   CUtensorMap mwd, mwg, mh;
   if (!map_2d(&mwd, L.w_down_t, (uint64_t)d, (uint64_t)F, (uint64_t)rd, TC_BK) ||

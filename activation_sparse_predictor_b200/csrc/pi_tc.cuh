@@ -15,8 +15,19 @@ namespace pi {
 // d_model % 128 == 0, 16-byte row strides (and PI_DISABLE_TC unset).
 bool ffn_tc_supported(const pi_layer& L, int batch);
 
-// Workspace bytes the path needs for a layer shape at this batch (0: none).
-size_t ffn_tc_scratch_bytes(int d_model, int d_ff, int batch);
+// Workspace bytes the tensor-core paths (FFN and predictor) need for a layer
+// shape at this batch (0: none).
+size_t tc_scratch_bytes(int d_model, int d_ff, int rank, int batch);
+
+// True when this layer's predictor runs on the tensor cores at this batch:
+// fp16 predictor, 16 <= batch <= 64, rank % 128 == 0, d_model % 128 == 0.
+bool pred_tc_supported(const pi_layer& L, int batch);
+
+// mask [batch][words] of xh [batch][d_model]: u = P1 xh and z = P2[j] u + c
+// on the tensor cores with each fp32 vector split into two fp16 parts
+// (fp32 accumulation); bit j = j < hot or z_j > theta.
+cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, float theta,
+                              uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s);
 
 // Up/gate products of list positions [0, hot + count) (row p for p < hot,
 // idx[p - hot] after) with xh [batch][d_model] (fp32, rounded to fp16 for

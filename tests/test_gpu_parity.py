@@ -317,3 +317,28 @@ def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
         assert rel_l2(y_tc[b], ref) <= TOL["f16"], b
         assert rel_l2(y_tc[b], y_cc[b]) <= 2e-3, b
     assert np.array_equal(run(), y_tc)  # deterministic
+
+
+@pytest.mark.parametrize("shape", [(1024, 3001, 256, 640), (512, 2048, 128, 200)])
+@pytest.mark.parametrize("batch", [16, 20, 64])
+@pytest.mark.parametrize("tau", [0.5, 0.3])
+def test_predict_on_tensor_cores(pi, orc, shape, batch, tau, monkeypatch):
+    """At 16-64 tokens the fp16 predictor runs on the tensor cores with the
+    fp32 vectors split into fp16 hi + lo parts: masks equal the oracle's
+    outside the 1e-4 band (hot bits set, tail bits clear), including a hot
+    prefix that ends inside a mask word, and equal the CUDA-core path's
+    outside the band."""
+    w = _wl("relu", "f16", shape, seed=53)
+    L, _ = device_layer(w, 0)
+    H = synth.layer_host(w, 0)
+    xh = _xh(w.d_model, batch, 5)
+    dxh = torch.from_numpy(xh).cuda()
+    m_tc = words_np(pi.pi_predict(L, dxh, tau))
+    monkeypatch.setenv("PI_DISABLE_TC", "1")
+    m_cc = words_np(pi.pi_predict(L, dxh, tau))
+    monkeypatch.delenv("PI_DISABLE_TC")
+    theta = synth.threshold_logit(tau)
+    for b in range(batch):
+        _, z = orc.predict(H, xh[b].astype(np.float64))
+        check_mask(m_tc[b], z, w.d_ff, w.hot, theta)
+        check_mask(m_cc[b], z, w.d_ff, w.hot, theta)

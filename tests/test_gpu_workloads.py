@@ -68,16 +68,15 @@ def test_workload_layer_union(pi, orc, name):
     for batch in w.union_batches:
         x0 = synth.x_host(w, 1, batch)
         xg, tr = _run_layer_stack(pi, L, x0, pi.PI_MASK_UNION, words)
-        ms, xh, flips = [], [], 0
+        xh = []
         for b in range(batch):
             xhb = orc.rmsnorm(x0[b])
             _, z = orc.predict(H, xhb)
-            flips += check_mask(tr[b], z, w.d_ff, w.hot, 0.0)
-            ms.append(orc.mask(z, w.d_ff, w.hot, 0.0))
+            check_mask(tr[b], z, w.d_ff, w.hot, 0.0)  # exact outside the band
             xh.append(xhb)
-        union = orc.compact(np.stack(ms), w.d_ff, w.hot)
-        if flips:
-            pytest.skip("a band neuron decided differently; union set not comparable")
+        # teacher-forced: the FFN over the union of the masks the GPU decided
+        # (they differ from the oracle's only inside the band)
+        union = orc.compact(tr.copy(), w.d_ff, w.hot)
         for b in (0, batch // 2 + 5, batch - 1):
             ref = orc.sparse_ffn(H, xh[b], union)
             assert rel_l2(xg[b] - x0[b], ref) <= TOL[w.w_dtype], (name, b)
