@@ -35,6 +35,14 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-FFN decode tokens/s (Llama2-70B Q4_0 shape)"
+
+
+def metric_name(workload: str, batch: int) -> str:
+    """The headline metric for the headline workload at batch 1, else a
+    name that says which workload and batch the line measures."""
+    if workload == DEFAULT_WORKLOAD and batch == 1:
+        return METRIC
+    return f"sparse-FFN tokens/s ({workload}, batch {batch})"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "llama2_70b_reglu_8192x28672_q4_0"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -255,7 +263,8 @@ def run_reference(args, world, rank):
     sample = (f"each step: one token through {len(layers)} of {w.n_layers} layers "
               f"(host-generated, resident); tokens/s extrapolated to all {w.n_layers} layers")
     line = {
-        "impl": "reference", "metric": METRIC, "value": tps, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": metric_name(w.name, 1), "value": tps, "unit": UNIT,
+        "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * sec_per_layer * w.n_layers, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -438,7 +447,7 @@ def run_pi(args, world, rank, local):
         cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "metric": metric_name(w.name, B), "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded generator, weights generated on the GPU; no datasets)",
