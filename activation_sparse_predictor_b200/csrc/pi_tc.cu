@@ -710,8 +710,10 @@ size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 int fpad(int F) { return (F + TC_M - 1) / TC_M * TC_M; }
 
+// K splits per output tile so that tiles x splits fill every SM with the two
+// CTAs (about 100 KB of shared memory each) it can hold.
 int split_for(int tiles, int nk) {
-  int ks = device_sms() / tiles;
+  int ks = 2 * device_sms() / tiles;
   ks = ks < 1 ? 1 : (ks > TC_KSMAX ? TC_KSMAX : ks);
   return ks > nk ? nk : ks;
 }
