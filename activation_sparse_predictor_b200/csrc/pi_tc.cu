@@ -157,8 +157,8 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
 }
 
 __device__ __forceinline__ void tc_init(uint64_t* full, uint64_t* empty, uint64_t* done,
-                                        volatile int* abort) {
-  for (int i = 0; i < TC_STAGES; ++i) {
+                                        volatile int* abort, int stages = TC_STAGES) {
+  for (int i = 0; i < stages; ++i) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
   }
@@ -524,6 +524,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 }
 
 constexpr int TC_KSMAX_U = 16;  // CTAs sharing one tile of P1's d at most
+constexpr int TC_PSTAGES = 3;   // predictor ring stages: 97 KB, two CTAs per SM
 
 // x (fp32 [batch][n]) -> hi = fp16(x), lo = fp16(x - hi), [nt][n] each
 // (rows >= batch zero).
@@ -556,9 +557,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = tc_sa(smem_raw);
   unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_STAGES * STAGE);
-  uint64_t* empty = full + TC_STAGES;
-  uint64_t* done = empty + TC_STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_PSTAGES * STAGE);
+  uint64_t* empty = full + TC_PSTAGES;
+  uint64_t* done = empty + TC_PSTAGES;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
 
@@ -568,7 +569,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
   const int nkt = kt1 - kt0;
 
-  if (threadIdx.x == 0) tc_init(full, empty, done, abort);
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort, TC_PSTAGES);
   if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -577,11 +578,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == 0 && lane == 0) {
     const uint32_t tx = A_BYTES + 2u * (uint32_t)nt * TC_BK * 2;
-    int last[TC_STAGES];
-    for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
+    int last[TC_PSTAGES];
+    for (int i = 0; i < TC_PSTAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
-      const int st = i % TC_STAGES;
-      if (i >= TC_STAGES && !tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr)) break;
+      const int st = i % TC_PSTAGES;
+      if (i >= TC_PSTAGES && !tc_wait(&empty[st], ((i / TC_PSTAGES) - 1) & 1, abort, hdr)) break;
       unsigned char* a = smem + st * STAGE;
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
                    "r"(tx)
@@ -592,13 +593,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tma_load_2d(a + A_BYTES + B_BYTES, &mbl, k, 0, &full[st]);
       last[st] = i;
     }
-    for (int st = 0; st < TC_STAGES; ++st)
-      if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
+    for (int st = 0; st < TC_PSTAGES; ++st)
+      if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_PSTAGES) & 1u, hdr);
   } else if (warp == 1 && lane == 0) {
     const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
     for (int i = 0; i < nkt; ++i) {
-      const int st = i % TC_STAGES;
-      if (!tc_wait(&full[st], (uint32_t)(i / TC_STAGES) & 1u, abort, hdr)) break;
+      const int st = i % TC_PSTAGES;
+      if (!tc_wait(&full[st], (uint32_t)(i / TC_PSTAGES) & 1u, abort, hdr)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t a = tc_sa(smem + st * STAGE), bh = a + A_BYTES, bl = bh + B_BYTES;
 #pragma unroll
@@ -844,7 +845,7 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   constexpr uint32_t STAGE = TC_M * TC_BK * 2 + 2 * TC_TMAX * TC_BK * 2;
-  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
+  const size_t smem = 1024 + (size_t)TC_PSTAGES * STAGE + 8 * (2 * TC_PSTAGES + 1) + 16;
   e = allow_smem_fn(reinterpret_cast<const void*>(k_pred_tc<0>), smem);
   if (e == cudaSuccess) e = allow_smem_fn(reinterpret_cast<const void*>(k_pred_tc<1>), smem);
   if (e != cudaSuccess) return e;
