@@ -157,9 +157,11 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
 }
 
 __device__ __forceinline__ void tc_init(uint64_t* full, uint64_t* empty, uint64_t* done,
-                                        volatile int* abort, int stages = TC_STAGES) {
+                                        volatile int* abort, int stages = TC_STAGES,
+                                        uint32_t full_arrivals = 1u) {
   for (int i = 0; i < stages; ++i) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&full[i])) : "memory");
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(tc_sa(&full[i])), "r"(full_arrivals)
+                 : "memory");
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(&empty[i])) : "memory");
   }
   asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(tc_sa(done)) : "memory");
@@ -239,19 +241,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int nkt = kt1 - kt0;
 
   rows[threadIdx.x] = list_row(p0 + threadIdx.x, H, N, F, idx);
-  if (threadIdx.x == 0) tc_init(full, empty, done, abort);
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort, TC_STAGES, 2u);
   if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tslot;
 
-  if (warp == 0) {
-    // producer warp: lane 0 arms the stage; in a gathered tile every lane
-    // then loads rows 4*lane .. 4*lane+3 of each weight operand
-    const uint32_t tx = NR * A_BYTES + (uint32_t)nt * TC_BK * 2;
-    const int r = 4 * lane;
+  if (warp == 0 || warp == 2) {
+    // two producer warps, each arming its own bytes on the stage's full
+    // barrier (two arrivals per phase).  A dense tile is one TMA box per
+    // operand (warp 0).  In a gathered tile warp pw loads rows
+    // [64 pw, 64 pw + 64) of each weight operand as four-row gathers, one per
+    // lane (NR * 16 per warp), so the gathers of a stage issue from two warps.
+    const int pw = warp >> 1;
+    const int opnd = lane >> 4, g = lane & 15;  // operand, row group of this lane's gather
+    const bool gl = !dense && opnd < NR;
+    const int r = 64 * pw + 4 * g;
     const int y0 = rows[r], y1 = rows[r + 1], y2 = rows[r + 2], y3 = rows[r + 3];
+    const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
+    const uint32_t tx = dense ? (pw == 0 ? NR * A_BYTES + bx : 0u)
+                              : NR * (A_BYTES / 2) + (pw == 0 ? bx : 0u);
     int last[TC_STAGES];
     for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
@@ -267,19 +277,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       __syncwarp();
       const int k = (kt0 + i) * TC_BK;
       if (dense) {
-        if (lane == 0) {
+        if (pw == 0 && lane == 0) {
           tma_load_2d(a, &mw0, k, p0, &full[st]);
           if constexpr (NR == 2) tma_load_2d(a + A_BYTES, &mw1, k, p0, &full[st]);
         }
-      } else {
-        tma_gather4(a + 512u * lane, &mg0, k, y0, y1, y2, y3, &full[st]);
-        if constexpr (NR == 2)
-          tma_gather4(a + A_BYTES + 512u * lane, &mg1, k, y0, y1, y2, y3, &full[st]);
+      } else if (gl) {
+        tma_gather4(a + opnd * A_BYTES + 512u * (16 * pw + g), opnd == 0 ? &mg0 : &mg1, k, y0, y1, y2,
+                    y3, &full[st]);
       }
-      if (lane == 0) {
-        tma_load_2d(a + NR * A_BYTES, &mx, k, 0, &full[st]);
-        last[st] = i;
-      }
+      if (pw == 0 && lane == 0) tma_load_2d(a + NR * A_BYTES, &mx, k, 0, &full[st]);
+      if (lane == 0) last[st] = i;
     }
     if (lane == 0) {  // every copy of this CTA has landed before it may exit (bounded)
       for (int st = 0; st < TC_STAGES; ++st)
@@ -432,7 +439,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int nkt = kt1 > kt0 ? kt1 - kt0 : 0;
 
   if (threadIdx.x == 0) {
-    tc_init(full, empty, done, abort);
+    tc_init(full, empty, done, abort, TC_STAGES, 2u);
     if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)N);
   }
   if (warp == 0) tmem_alloc(tslot, NCOLS);
@@ -442,8 +449,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = *tslot;
   const int c0 = tile * TC_M;
 
-  if (warp == 0) {
-    const uint32_t tx = A_BYTES + (uint32_t)nt * TC_BK * 2;
+  if (warp == 0 || warp == 2) {
+    // two producer warps, each arming its own bytes on the stage's full
+    // barrier (two arrivals per phase).  A stage inside the hot prefix is two
+    // 64-column boxes (warp 0).  Otherwise warp pw gathers list positions
+    // [pk + 32 pw, pk + 32 pw + 32): lanes 0..7 four positions each of the
+    // first 64 columns, lanes 8..15 of the next 64.
+    const int pw = warp >> 1;
+    const int half = (lane >> 3) & 1, g = 8 * pw + (lane & 7);  // column half, position group
+    const uint32_t bx = (uint32_t)nt * TC_BK * 2;                 // the activation tile
     int last[TC_STAGES];
     for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
@@ -452,28 +466,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       unsigned char* a = smem + st * STAGE;
+      const int pk = (kt0 + i) * TC_BK;  // first list position of the stage
+      const bool boxed = pk + TC_BK <= H;
+      const uint32_t tx = boxed ? (pw == 0 ? A_BYTES + bx : 0u) : A_BYTES / 2 + (pw == 0 ? bx : 0u);
       if (lane == 0)
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
                      "r"(tx)
                      : "memory");
       __syncwarp();
-      const int pk = (kt0 + i) * TC_BK;  // first list position of the stage
-      if (pk + TC_BK <= H) {
-        if (lane == 0) {
+      if (boxed) {
+        if (pw == 0 && lane == 0) {
           tma_load_2d(a, &mwd, c0, pk, &full[st]);
           tma_load_2d(a + BOX, &mwd, c0 + 64, pk, &full[st]);
         }
-      } else {
-        // lanes 0..15: positions 4l .. 4l+3 of the first 64 columns; 16..31: of the next 64
-        const int half = lane >> 4, l = lane & 15, q = pk + 4 * l;
-        tma_gather4(a + half * BOX + 512u * l, &mwg, c0 + 64 * half, list_row(q, H, N, F, idx),
+      } else if (lane < 16) {
+        const int q = pk + 4 * g;
+        tma_gather4(a + half * BOX + 512u * g, &mwg, c0 + 64 * half, list_row(q, H, N, F, idx),
                     list_row(q + 1, H, N, F, idx), list_row(q + 2, H, N, F, idx),
                     list_row(q + 3, H, N, F, idx), &full[st]);
       }
-      if (lane == 0) {
-        tma_load_2d(a + A_BYTES, &mh, pk, 0, &full[st]);
-        last[st] = i;
-      }
+      if (pw == 0 && lane == 0) tma_load_2d(a + A_BYTES, &mh, pk, 0, &full[st]);
+      if (lane == 0) last[st] = i;
     }
     if (lane == 0) {
       for (int st = 0; st < TC_STAGES; ++st)
