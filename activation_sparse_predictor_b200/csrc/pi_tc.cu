@@ -49,6 +49,7 @@ constexpr int TC_M = 128;        // list positions (up) / output columns (down) 
 constexpr int TC_BK = 64;        // k per stage: one 128-byte swizzle atom of fp16
 constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 128;
+constexpr int TC_PW = 3;         // producer warps of the FFN kernels: 0, 2, 3 (warp 1 issues MMAs)
 constexpr int TC_KSMAX = 4;      // CTAs sharing one tile's k range at most
 constexpr int TC_TMAX = 64;      // tokens at most (MMA N)
 constexpr unsigned long long kTcTimeoutNs = 1000000000ull;
@@ -241,27 +242,28 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int nkt = kt1 - kt0;
 
   rows[threadIdx.x] = list_row(p0 + threadIdx.x, H, N, F, idx);
-  if (threadIdx.x == 0) tc_init(full, empty, done, abort, TC_STAGES, 2u);
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort, TC_STAGES, (uint32_t)TC_PW);
   if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tslot;
 
-  if (warp == 0 || warp == 2) {
-    // two producer warps, each arming its own bytes on the stage's full
-    // barrier (two arrivals per phase).  A dense tile is one TMA box per
-    // operand (warp 0).  In a gathered tile warp pw loads rows
-    // [64 pw, 64 pw + 64) of each weight operand as four-row gathers, one per
-    // lane (NR * 16 per warp), so the gathers of a stage issue from two warps.
-    const int pw = warp >> 1;
-    const int opnd = lane >> 4, g = lane & 15;  // operand, row group of this lane's gather
-    const bool gl = !dense && opnd < NR;
-    const int r = 64 * pw + 4 * g;
+  if (warp != 1) {
+    // TC_PW producer warps, each arming its own bytes on the stage's full
+    // barrier (TC_PW arrivals per phase).  A dense tile is one TMA box per
+    // operand (warp 0).  A gathered tile's NR * 32 four-row gathers (rows
+    // 4g .. 4g+3 of operand o / 32, g = o % 32) are dealt out round-robin,
+    // gather o = TC_PW * lane + pw, so a stage issues from every producer warp.
+    const int pw = warp == 0 ? 0 : warp - 1;
+    const int o = TC_PW * lane + pw;
+    const int opnd = o >> 5, g = o & 31;
+    const bool gl = !dense && o < NR * 32;
+    const int r = 4 * g;
     const int y0 = rows[r], y1 = rows[r + 1], y2 = rows[r + 2], y3 = rows[r + 3];
     const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
-    const uint32_t tx = dense ? (pw == 0 ? NR * A_BYTES + bx : 0u)
-                              : NR * (A_BYTES / 2) + (pw == 0 ? bx : 0u);
+    const uint32_t mine = (uint32_t)((NR * 32 - pw + TC_PW - 1) / TC_PW);  // gathers of this warp
+    const uint32_t tx = dense ? (pw == 0 ? NR * A_BYTES + bx : 0u) : 512u * mine + (pw == 0 ? bx : 0u);
     int last[TC_STAGES];
     for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
@@ -282,8 +284,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if constexpr (NR == 2) tma_load_2d(a + A_BYTES, &mw1, k, p0, &full[st]);
         }
       } else if (gl) {
-        tma_gather4(a + opnd * A_BYTES + 512u * (16 * pw + g), opnd == 0 ? &mg0 : &mg1, k, y0, y1, y2,
-                    y3, &full[st]);
+        tma_gather4(a + opnd * A_BYTES + 512u * g, opnd == 0 ? &mg0 : &mg1, k, y0, y1, y2, y3,
+                    &full[st]);
       }
       if (pw == 0 && lane == 0) tma_load_2d(a + NR * A_BYTES, &mx, k, 0, &full[st]);
       if (lane == 0) last[st] = i;
@@ -439,7 +441,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int nkt = kt1 > kt0 ? kt1 - kt0 : 0;
 
   if (threadIdx.x == 0) {
-    tc_init(full, empty, done, abort, TC_STAGES, 2u);
+    tc_init(full, empty, done, abort, TC_STAGES, (uint32_t)TC_PW);
     if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)N);
   }
   if (warp == 0) tmem_alloc(tslot, NCOLS);
@@ -449,15 +451,26 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem = *tslot;
   const int c0 = tile * TC_M;
 
-  if (warp == 0 || warp == 2) {
-    // two producer warps, each arming its own bytes on the stage's full
-    // barrier (two arrivals per phase).  A stage inside the hot prefix is two
-    // 64-column boxes (warp 0).  Otherwise warp pw gathers list positions
-    // [pk + 32 pw, pk + 32 pw + 32): lanes 0..7 four positions each of the
-    // first 64 columns, lanes 8..15 of the next 64.
-    const int pw = warp >> 1;
-    const int half = (lane >> 3) & 1, g = 8 * pw + (lane & 7);  // column half, position group
-    const uint32_t bx = (uint32_t)nt * TC_BK * 2;                 // the activation tile
+  if (warp != 1) {
+    // TC_PW producer warps, each arming its own bytes on the stage's full
+    // barrier (TC_PW arrivals per phase).  A stage inside the hot prefix is
+    // two 64-column boxes (warp 0).  Otherwise its 32 four-position gathers
+    // (positions pk + 4g .. pk + 4g + 3 of column half o / 16, g = o % 16)
+    // are dealt out round-robin, gather o = TC_PW * lane + pw; each lane
+    // loads the next stage's list rows while this one issues.
+    const int pw = warp == 0 ? 0 : warp - 1;
+    const int o = TC_PW * lane + pw;
+    const int half = o >> 4, g = o & 15;  // column half, position group
+    const bool gl = o < 32;
+    const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
+    const uint32_t mine = (uint32_t)((32 - pw + TC_PW - 1) / TC_PW);  // gathers of this warp
+    int y[4], ny[4];  // list rows of this lane's gather: this stage, the next
+    auto rows_at = [&](int i, int (&v)[4]) {
+      const int q = (kt0 + i) * TC_BK + 4 * g;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) v[t] = gl ? list_row(q + t, H, N, F, idx) : 0;
+    };
+    if (nkt > 0) rows_at(0, ny);
     int last[TC_STAGES];
     for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
@@ -468,7 +481,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       unsigned char* a = smem + st * STAGE;
       const int pk = (kt0 + i) * TC_BK;  // first list position of the stage
       const bool boxed = pk + TC_BK <= H;
-      const uint32_t tx = boxed ? (pw == 0 ? A_BYTES + bx : 0u) : A_BYTES / 2 + (pw == 0 ? bx : 0u);
+      const uint32_t tx = boxed ? (pw == 0 ? A_BYTES + bx : 0u) : 512u * mine + (pw == 0 ? bx : 0u);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) y[t] = ny[t];
+      if (i + 1 < nkt) rows_at(i + 1, ny);
       if (lane == 0)
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
                      "r"(tx)
@@ -479,11 +495,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tma_load_2d(a, &mwd, c0, pk, &full[st]);
           tma_load_2d(a + BOX, &mwd, c0 + 64, pk, &full[st]);
         }
-      } else if (lane < 16) {
-        const int q = pk + 4 * g;
-        tma_gather4(a + half * BOX + 512u * g, &mwg, c0 + 64 * half, list_row(q, H, N, F, idx),
-                    list_row(q + 1, H, N, F, idx), list_row(q + 2, H, N, F, idx),
-                    list_row(q + 3, H, N, F, idx), &full[st]);
+      } else if (gl) {
+        tma_gather4(a + half * BOX + 512u * g, &mwg, c0 + 64 * half, y[0], y[1], y[2], y[3], &full[st]);
       }
       if (pw == 0 && lane == 0) tma_load_2d(a + A_BYTES, &mh, pk, 0, &full[st]);
       if (lane == 0) last[st] = i;
