@@ -49,7 +49,8 @@ constexpr int TC_M = 128;        // list positions (up) / output columns (down) 
 constexpr int TC_BK = 64;        // k per stage: one 128-byte swizzle atom of fp16
 constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 128;
-constexpr int TC_PW = 3;         // producer warps of the FFN kernels: 0, 2, 3 (warp 1 issues MMAs)
+constexpr int TC_FFN_WARPS = 8;  // warps of the FFN kernels: warp 1 issues the MMAs, the rest
+constexpr int TC_PW = TC_FFN_WARPS - 1;  // load (warps 0-3 also drain the accumulators)
 constexpr int TC_KSMAX = 4;      // CTAs sharing one tile's k range at most
 constexpr int TC_TMAX = 64;      // tokens at most (MMA N)
 constexpr unsigned long long kTcTimeoutNs = 1000000000ull;
@@ -212,7 +213,7 @@ __device__ __forceinline__ int list_row(int p, int H, int N, int F, const int32_
 // up: NR = 1 ReLU (W_up), NR = 2 ReGLU (W_gate, W_up).  Grid (Fp / 128, ks).
 // part: [ks][NR][Fp][nt] fp32.
 template <int NR>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     k_ffn_up_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
                 const __grid_constant__ CUtensorMap mg0, const __grid_constant__ CUtensorMap mg1,
                 const __grid_constant__ CUtensorMap mx, int nt, int nk, int ks, int H, int F, int Fp,
@@ -241,7 +242,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
   const int nkt = kt1 - kt0;
 
-  rows[threadIdx.x] = list_row(p0 + threadIdx.x, H, N, F, idx);
+  if (threadIdx.x < TC_M) rows[threadIdx.x] = list_row(p0 + threadIdx.x, H, N, F, idx);
   if (threadIdx.x == 0) tc_init(full, empty, done, abort, TC_STAGES, (uint32_t)TC_PW);
   if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -322,7 +323,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   bool ok = tc_wait_quiet(done, 0u, hdr);
   ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (ok) {
+  if (ok && warp < 4) {
     const int p = p0 + warp * 32 + lane;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
@@ -412,7 +413,7 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
 
 // down: part[split][b][c] = sum over the split's list positions p of
 // W_down^T[row(p)][c] h16[b][p], for the tile's 128 columns c.  Grid (d / 128, ks).
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     k_ffn_down_tc(const __grid_constant__ CUtensorMap mwd, const __grid_constant__ CUtensorMap mwg,
                   const __grid_constant__ CUtensorMap mh, int nt, int nk, int ks, int d, int batch,
                   int H, int F, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
@@ -530,7 +531,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // accumulator lane = output column, accumulator column = token; a split
   // with no list positions writes zeros (the reduction sums every slice)
   const int c = c0 + warp * 32 + lane;
-  for (int t0 = 0; t0 < nt; t0 += 16) {
+  for (int t0 = 0; t0 < nt && warp < 4; t0 += 16) {
     uint32_t v[16];
     if (ok && nkt > 0) {
       tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)t0, v);
@@ -816,7 +817,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   auto kern = k_ffn_up_tc<NR>;
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, ks, H, F, Fp, idx,
+  kern<<<dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, ks, H, F, Fp, idx,
                                                  count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -928,7 +929,7 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
   const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
   cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_down_tc), smem);
   if (e != cudaSuccess) return e;
-  k_ffn_down_tc<<<dim3(tiles, ks), TC_THREADS, smem, s>>>(mwd, mwg, mh, nt, nk, ks, d, batch, H, F,
+  k_ffn_down_tc<<<dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s>>>(mwd, mwg, mh, nt, nk, ks, d, batch, H, F,
                                                           idx, count, part, hdr);
   return cudaGetLastError();
 }
