@@ -264,7 +264,15 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
     if ((st = predict_body(L, xh, batch, theta, mask, ws, lay, s, prof)) != PI_OK) return st;
     P.before(PI_KIND_COMPACT);
-    e = launch_compact(mask, batch, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);
+    if (batch > 1) {
+      // the tokens' union first, across many CTAs, into the activation
+      // buffer (free until the up projection), then one list from it
+      uint32_t* uni = at<uint32_t>(ws, lay.h);
+      e = launch_mask_union(mask, batch, words, uni, s);
+      if (e == cudaSuccess) e = launch_compact(uni, 1, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);
+    } else {
+      e = launch_compact(mask, batch, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);
+    }
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "compact launch");
     if ((st = ffn_body(L, xh, batch, per_token ? mask : nullptr, per_token, idx, cnt, x, x, ws,

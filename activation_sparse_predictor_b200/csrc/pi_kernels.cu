@@ -264,12 +264,14 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ m
       if (lane == 31) wsum[31] = vi;       // (nw <= 31 here) total of this tile
     }
     __syncthreads();
-    int pos = s_base + wsum[warp] + incl - c;
-    const int lo = w * 32;
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      out[pos++] = lo + bit;
-      m &= m - 1u;
+    // the warp's 32 words in order, lane t taking bit t of each: the
+    // entries of one word go to consecutive positions (coalesced stores)
+    int run = s_base + wsum[warp];
+    const int wfirst = w0 + warp * 32;
+    for (int i = 0; i < 32; ++i) {
+      const uint32_t mi = __shfl_sync(0xffffffffu, m, i);
+      if ((mi >> lane) & 1u) out[run + __popc(mi & ((1u << lane) - 1u))] = (wfirst + i) * 32 + lane;
+      run += __popc(mi);
     }
     const int tile_total = wsum[31];
     __syncthreads();
@@ -277,6 +279,39 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ m
     __syncthreads();
   }
   if (tid == 0) count[list] = s_base;
+}
+
+// out[w] = OR over tokens b < B of mask[b][w].  Block: 32 words x 8 token
+// groups (token b goes to group b % 8, eight loads in flight per thread),
+// the groups combined in shared memory.
+__global__ void __launch_bounds__(256) k_mask_union(const uint32_t* __restrict__ mask, int B,
+                                                    int words, uint32_t* __restrict__ out) {
+  __shared__ uint32_t sm[8][32];
+  const int wl = threadIdx.x & 31, tg = threadIdx.x >> 5;
+  const int w = blockIdx.x * 32 + wl;
+  uint32_t m = 0u;
+  if (w < words) {
+    uint32_t a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) a[k] = 0u;
+    for (int b0 = tg; b0 < B; b0 += 64) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int b = b0 + 8 * k;
+        if (b < B) a[k] |= mask[(size_t)b * words + w];
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m |= a[k];
+  }
+  sm[tg][wl] = m;
+  __syncthreads();
+  if (tg == 0 && w < words) {
+    uint32_t u = 0u;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) u |= sm[g][wl];
+    out[w] = u;
+  }
 }
 
 // Gathered up/gate rows + activation: one warp per listed row.
@@ -567,6 +602,12 @@ cudaError_t launch_pred_z(const pi_layer& L, const float* u, int batch, float th
   }
   if (L.p_dtype == PI_F32) { PI_PZ(PI_F32) } else { PI_PZ(PI_F16) }
 #undef PI_PZ
+}
+
+cudaError_t launch_mask_union(const uint32_t* mask, int batch, int words, uint32_t* out,
+                              cudaStream_t s) {
+  k_mask_union<<<(words + 31) / 32, 256, 0, s>>>(mask, batch, words, out);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,

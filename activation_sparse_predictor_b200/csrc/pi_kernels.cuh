@@ -28,6 +28,10 @@ cudaError_t launch_pred_u(const pi_layer& L, const float* xh, int batch, float* 
 cudaError_t launch_pred_z(const pi_layer& L, const float* u, int batch, float theta,
                           uint32_t* mask, cudaStream_t s);
 
+// out[w] = OR over b < batch of mask[b][w], w < words (many CTAs).
+cudaError_t launch_mask_union(const uint32_t* mask, int batch, int words, uint32_t* out,
+                              cudaStream_t s);
+
 // ascending set-bit lists (see pi_compact)
 cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,
                            int32_t* idx, int32_t* count, cudaStream_t s);

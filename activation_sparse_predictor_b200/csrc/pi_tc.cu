@@ -379,28 +379,47 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
                                                     const uint32_t* __restrict__ mask, int words,
                                                     __half* __restrict__ h16, WsHeader* hdr) {
   __shared__ float sh[64][TC_TMAX + 1];
+  __shared__ int sj[64];    // each row's neuron
+  __shared__ float sb[64];  // and bias
+  __shared__ int sv[64];    // 1: a listed row with a valid neuron
   const int N = list_len(count, H, F, hdr);
   if (hdr && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&hdr->rows_listed, (unsigned long long)N);
   const int n0 = blockIdx.x * 64;
   const int m = 64 * nt;
+  // per row once: neuron, index check, bias
+  if (threadIdx.x < 64) {
+    const int p = n0 + threadIdx.x;
+    int j = 0, v = 0;
+    float bb = 0.f;
+    if (p < N) {
+      j = p < H ? p : idx[p - H];
+      if (p >= H && (j < H || j >= F)) {
+        if (hdr) atomicOr(&hdr->status, DEV_BAD_INDEX);
+      } else {
+        v = 1;
+        bb = bias ? bias[j] : 0.f;
+      }
+    }
+    sj[threadIdx.x] = j;
+    sb[threadIdx.x] = bb;
+    sv[threadIdx.x] = v;
+  }
+  __syncthreads();
+#pragma unroll 4
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
     const int nn = i / nt, b = i % nt, p = n0 + nn;
     float hv = 0.f;
-    if (p < N && b < batch) {
-      const int j = p < H ? p : idx[p - H];
-      if (p >= H && (j < H || j >= F)) {
-        if (b == 0 && hdr) atomicOr(&hdr->status, DEV_BAD_INDEX);
-      } else {
-        float g = 0.f, u = 0.f;
-        for (int s = 0; s < ks; ++s) {
-          g += __ldcg(part + ((size_t)(s * NR) * Fp + n0) * nt + i);
-          if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * Fp + n0) * nt + i);
-        }
-        g += bias ? bias[j] : 0.f;
-        hv = g > 0.f ? g : 0.f;
-        if constexpr (NR == 2) hv *= u;
-        if (mask && p >= H && !((mask[(size_t)b * words + (j >> 5)] >> (j & 31)) & 1u)) hv = 0.f;
+    if (sv[nn] && b < batch) {
+      const int j = sj[nn];
+      float g = 0.f, u = 0.f;
+      for (int s = 0; s < ks; ++s) {
+        g += __ldcg(part + ((size_t)(s * NR) * Fp + n0) * nt + i);
+        if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * Fp + n0) * nt + i);
       }
+      g += sb[nn];
+      hv = g > 0.f ? g : 0.f;
+      if constexpr (NR == 2) hv *= u;
+      if (mask && p >= H && !((__ldg(mask + (size_t)b * words + (j >> 5)) >> (j & 31)) & 1u)) hv = 0.f;
     }
     sh[nn][b] = hv;
   }
