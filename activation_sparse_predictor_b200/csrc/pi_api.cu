@@ -247,6 +247,7 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
                                     utrace ? utrace + (size_t)l0 * stack1_unit_trace_len() * 4 : nullptr);
       P.after();
       if (e != cudaSuccess) return cuda_fail(e, "fused stack launch");
+      note_launch();
     }
     return PI_OK;
   }
@@ -490,6 +491,8 @@ pi_status pi_ffn_stack_timeline(const pi_layer* layers, int n_layers, float* x, 
 
 int pi_device_sms(void) { return device_sms(); }
 
+unsigned long long pi_kernel_launches(void) { return launches_so_far(); }
+
 pi_status pi_wait_selftest(void* ws, size_t ws_bytes, int kind, unsigned timeout_us, void* stream) {
   if (!ws || !aligned(ws, 256) || ws_bytes < sizeof(WsHeader))
     return fail(PI_ERR_INVALID, "workspace null, misaligned or smaller than its header");
@@ -497,7 +500,9 @@ pi_status pi_wait_selftest(void* ws, size_t ws_bytes, int kind, unsigned timeout
   if (timeout_us < 1 || timeout_us > 10000000u)
     return fail(PI_ERR_INVALID, "timeout %u us not in [1, 1e7]", timeout_us);
   cudaError_t e = launch_wait_selftest(ws, kind, 1000ull * timeout_us, (cudaStream_t)stream);
-  return e == cudaSuccess ? PI_OK : cuda_fail(e, "wait self-test launch");
+  if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
+  note_launch();
+  return PI_OK;
 }
 
 pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {

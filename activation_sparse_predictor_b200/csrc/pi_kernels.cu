@@ -10,6 +10,7 @@
 // with the reused vectors (xh, u) staged in shared memory.  Accumulation is
 // fp32 throughout.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <unordered_map>
 
@@ -514,6 +515,13 @@ cudaError_t allow_smem_fn(const void* fn, size_t bytes) {
 }
 
 
+namespace {
+std::atomic<unsigned long long> g_launches{0};  // kernels launched by this library
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1ull, std::memory_order_relaxed); }
+unsigned long long launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
+
 int device_sms() {
   static int cache[64] = {0};
   int dev = 0;
@@ -547,6 +555,7 @@ int down_splits(int batch, int d) {
 
 cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s) {
   k_rmsnorm<1><<<batch, 1024, 0, s>>>(x, d, xh);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -559,6 +568,7 @@ static cudaError_t pred_u_t(const pi_layer& L, const float* xh, int batch, float
   if (e != cudaSuccess) return e;
   dim3 grid(std::min((L.rank + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
   kern<<<grid, kThreads, smem, s>>>((const char*)L.p1, xh, batch, L.d_model, L.rank, u);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -587,6 +597,7 @@ static cudaError_t pred_z_t(const pi_layer& L, const float* u, int batch, float 
   dim3 grid(std::min((words + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
   kern<<<grid, kThreads, smem, s>>>((const char*)L.p2, L.p_bias, u, batch, L.rank, L.d_ff,
                                     L.hot, theta, mask, words);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -607,6 +618,7 @@ cudaError_t launch_pred_z(const pi_layer& L, const float* u, int batch, float th
 cudaError_t launch_mask_union(const uint32_t* mask, int batch, int words, uint32_t* out,
                               cudaStream_t s) {
   k_mask_union<<<(words + 31) / 32, 256, 0, s>>>(mask, batch, words, out);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -617,6 +629,7 @@ cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin,
   const int lists = unite ? 1 : batch;
   const int threads = std::min(992, std::max(32, ((words + 31) / 32) * 32));
   k_compact<<<lists, threads, 0, s>>>(mask, batch, words, d_ff, begin, unite, idx, d_ff, count);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -631,6 +644,7 @@ static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const
   dim3 grid(std::min((L.d_ff + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
   kern<<<grid, kThreads, smem, s>>>(L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
                                     count, h, status, n0);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -669,6 +683,7 @@ static cudaError_t ffn_down_t(const pi_layer& L, int batch, const int32_t* idx,
                                               (const uint16_t*)L.w_down_t_scales, L.d_model,
                                               L.d_ff, L.hot, idx, count, h, batch, S, part, hdr,
                                               L.w_down_row_stride, nb);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -694,6 +709,7 @@ cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,
 
 cudaError_t launch_delay(unsigned long long ns, cudaStream_t s) {
   k_delay<<<1, 32, 0, s>>>(ns);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -702,6 +718,7 @@ cudaError_t launch_reduce(const float* part, int splits, int batch, int d, const
   const int64_t n = (int64_t)batch * d;
   const int grid = (int)std::min<int64_t>((n + kThreads - 1) / kThreads, device_sms() * 8);
   k_reduce<<<grid, kThreads, 0, s>>>(part, splits, n, resid, out);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -10,6 +10,8 @@
 namespace pi {
 
 int device_sms();                 // SM count of the current device (cached)
+void note_launch();               // counts one kernel launch (pi_kernel_launches)
+unsigned long long launches_so_far();
 
 // Raises a kernel's dynamic shared-memory limit on the current device once.
 cudaError_t allow_smem_fn(const void* fn, size_t bytes);

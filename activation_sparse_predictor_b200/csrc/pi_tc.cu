@@ -828,6 +828,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
     return cudaErrorInvalidValue;
   k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt,
                                                                               sc.xh16);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int tiles = Fp / TC_M, nk = d / TC_BK, ks = up_splits(d, F);
@@ -838,10 +839,12 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   if (e != cudaSuccess) return e;
   kern<<<dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, ks, H, F, Fp, idx,
                                                  count, sc.part, hdr);
+  note_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_ffn_finish<NR><<<Fp / 64, 256, 0, s>>>(sc.part, ks, H, F, Fp, nt, batch, idx, count, L.bias,
                                            mask, (F + 31) / 32, sc.h16, hdr);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -888,6 +891,7 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
     return cudaErrorInvalidValue;
   const int grid = device_sms() * 4;
   k_split16<<<std::min((nt * d + 255) / 256, grid), 256, 0, s>>>(xh, batch, d, nt, sc.xh16, sc.xlo);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   constexpr uint32_t STAGE = TC_M * TC_BK * 2 + 2 * TC_TMAX * TC_BK * 2;
@@ -900,14 +904,17 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
   k_pred_tc<0><<<dim3(r / TC_M, ksu), TC_THREADS, smem, s>>>(m1, mxh, mxl, nt, d / TC_BK, ksu, 0, r,
                                                              sc.upart, nullptr, 0.f, 0, nullptr, 0,
                                                              batch, hdr);
+  note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   k_pred_u_finish<<<std::min((r * nt + 255) / 256, grid), 256, 0, s>>>(sc.upart, ksu, r, nt, batch,
                                                                        sc.uhi, sc.ulo);
+  note_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // z = P2 u + c for rows from the word holding `hot`; the words below it are hot
   const int w0 = H / 32, row0 = 32 * w0;
   if (w0 > 0) {
     k_hot_words<<<std::min((batch * w0 + 255) / 256, grid), 256, 0, s>>>(mask, words, w0, batch);
+    note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (row0 < F) {
@@ -915,6 +922,7 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
     k_pred_tc<1><<<dim3(tiles, 1), TC_THREADS, smem, s>>>(m2, muh, mul, nt, r / TC_BK, 1, row0, F,
                                                           nullptr, L.p_bias, theta, H, mask, words,
                                                           batch, hdr);
+    note_launch();
     e = cudaGetLastError();
   }
   return e;
@@ -950,6 +958,7 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
   if (e != cudaSuccess) return e;
   k_ffn_down_tc<<<dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s>>>(mwd, mwg, mh, nt, nk, ks, d, batch, H, F,
                                                           idx, count, part, hdr);
+  note_launch();
   return cudaGetLastError();
 }
 

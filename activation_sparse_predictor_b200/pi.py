@@ -65,6 +65,7 @@ def _load():
         "pi_read_counters": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_uint64)]),
         "pi_ffn_stack_timeline": (i32, [L, i32, vp, f32, vp, sz, vp, vp, vp]),
         "pi_device_sms": (i32, []),
+        "pi_kernel_launches": (ctypes.c_ulonglong, []),
         "pi_wait_selftest": (i32, [vp, sz, i32, ctypes.c_uint, vp]),
         "pi_status_string": (ctypes.c_char_p, [i32]),
         "pi_last_error": (ctypes.c_char_p, []),
@@ -329,6 +330,11 @@ def pi_ffn_stack_timeline(layers, x, tau: float, ws=None, stream=None, _arr=None
 
 def pi_device_sms() -> int:
     return int(_lib.pi_device_sms())
+
+
+def pi_kernel_launches() -> int:
+    """Kernels launched by the library in this process so far (include/pi.h)."""
+    return int(_lib.pi_kernel_launches())
 
 
 def pi_kind_name(kind: int) -> str:

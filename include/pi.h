@@ -259,6 +259,13 @@ pi_status pi_ffn_stack_timeline(const pi_layer* layers, int n_layers, float* x, 
 /* Number of SMs of the current device (the persistent kernel's grid). */
 int pi_device_sms(void);
 
+/* Number of kernels this library has launched in this process so far, over
+ * every entry point (a host-side count taken at each launch; a launch made
+ * while a stream is being captured into a CUDA graph counts once, at capture,
+ * so the difference across one captured call is the graph's kernel count).
+ * Never fails. */
+unsigned long long pi_kernel_launches(void);
+
 /* Synchronises `stream` and reads the workspace's two row counters, which
  * every FFN launch advances on the device: out[0] = neuron rows whose
  * gate/up (ReGLU) or up (ReLU) weights were read, out[1] = rows of w_down_t

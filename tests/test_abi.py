@@ -47,6 +47,12 @@ def test_status_strings_and_version(pi):
     assert pi.pi_status_string(99) == "PI_ERR_UNKNOWN"
 
 
+def test_kernel_launch_counter_without_gpu(pi):
+    a = pi.pi_kernel_launches()
+    b = pi.pi_kernel_launches()
+    assert isinstance(a, int) and 0 <= a <= b
+
+
 FAKE = 1 << 20  # an aligned, never-dereferenced address
 
 

@@ -275,6 +275,24 @@ def test_stack_is_deterministic(pi, packed):
     assert torch.equal(outs[0], outs[1])
 
 
+def test_kernel_launch_counter(pi):
+    """One fused launch per batch-1 stack call of at most 24 layers; the same
+    count on every repeat of a multi-kernel (batch 4) call."""
+    w = _wl("reglu", "q4_0", (512, 1500, 64, 256), seed=44).scaled(4)
+    layers = [device_layer(w, l, packed=True)[0] for l in range(4)]
+    x = torch.from_numpy(synth.x_host(w, 0, 1)).cuda()
+    n0 = pi.pi_kernel_launches()
+    pi.pi_ffn_stack(layers, x, 0.5, pi.PI_MASK_UNION)
+    assert pi.pi_kernel_launches() - n0 == 1
+    xb = torch.from_numpy(synth.x_host(w, 0, 4)).cuda()
+    counts = []
+    for _ in range(2):
+        n0 = pi.pi_kernel_launches()
+        pi.pi_ffn_stack(layers, xb, 0.5, pi.PI_MASK_PER_TOKEN)
+        counts.append(pi.pi_kernel_launches() - n0)
+    assert counts[0] == counts[1] >= 4 * 6  # per layer: norm, predictor, compaction, FFN, reduce
+
+
 @pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0)])
 @pytest.mark.parametrize("act", ["relu", "reglu"])
 @pytest.mark.parametrize("batch,mode", [(16, "per_token"), (20, "union"), (48, "per_token"),
