@@ -153,7 +153,7 @@ struct Prof {
 pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                    int per_token, const int32_t* idx, const int32_t* count, const float* resid,
                    float* out, void* ws, const WsLayout& lay, cudaStream_t s,
-                   Prof* prof = nullptr) {
+                   Prof* prof = nullptr, bool xh16_ready = false) {
   Prof none;
   Prof& P = prof ? *prof : none;
   const int S = down_splits(batch, L.d_model);
@@ -163,7 +163,8 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
   if (ffn_tc_supported(L, batch)) {
     // token batches: both contractions over the listed rows on the tensor cores
     P.before(PI_KIND_FFN_UP);
-    e = launch_ffn_up_tc(L, xh, batch, mask, idx, count, at<void>(ws, lay.tc), header(ws), s);
+    e = launch_ffn_up_tc(L, xh, batch, mask, idx, count, at<void>(ws, lay.tc), header(ws), s,
+                         xh16_ready);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn up (tensor cores) launch");
     P.before(PI_KIND_FFN_DOWN);
@@ -276,8 +277,9 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
     }
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "compact launch");
+    // the tensor-core predictor leaves the fp16 copy of xh the FFN reads
     if ((st = ffn_body(L, xh, batch, per_token ? mask : nullptr, per_token, idx, cnt, x, x, ws,
-                       lay, s, prof)) != PI_OK)
+                       lay, s, prof, pred_tc_supported(L, batch))) != PI_OK)
       return st;
   }
   return PI_OK;

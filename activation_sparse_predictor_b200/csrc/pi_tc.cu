@@ -813,7 +813,7 @@ TcScratch tc_scratch(void* base, int d, int F, int r) {
 template <int NR>
 cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                          const int32_t* idx, const int32_t* count, void* scratch, WsHeader* hdr,
-                         cudaStream_t s) {
+                         cudaStream_t s, bool xh16_ready) {
   const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
@@ -826,11 +826,13 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
       !map_2d(&g1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs, 1) ||
       !map_2d(&mx, sc.xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt))
     return cudaErrorInvalidValue;
-  k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt,
-                                                                              sc.xh16);
-  note_launch();
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!xh16_ready) {
+    k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt,
+                                                                                sc.xh16);
+    note_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   const int tiles = Fp / TC_M, nk = d / TC_BK, ks = up_splits(d, F);
   constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
   const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16 + 4 * TC_M;
@@ -934,9 +936,10 @@ int ffn_tc_down_splits(const pi_layer& L) {
 
 cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                              const int32_t* idx, const int32_t* count, void* scratch,
-                             WsHeader* hdr, cudaStream_t s) {
-  return L.act == PI_REGLU ? launch_up_nr<2>(L, xh, batch, mask, idx, count, scratch, hdr, s)
-                           : launch_up_nr<1>(L, xh, batch, mask, idx, count, scratch, hdr, s);
+                             WsHeader* hdr, cudaStream_t s, bool xh16_ready) {
+  return L.act == PI_REGLU
+             ? launch_up_nr<2>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready)
+             : launch_up_nr<1>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready);
 }
 
 cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,

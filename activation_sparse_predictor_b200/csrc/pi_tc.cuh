@@ -33,10 +33,12 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
 // idx[p - hot] after) with xh [batch][d_model] (fp32, rounded to fp16 for
 // the tensor cores; fp32 accumulation), bias, ReLU / ReGLU, each token's own
 // mask bit for cold rows when `mask` ([batch][words]) is given; leaves the
-// fp16 activations in `scratch` for launch_ffn_down_tc.
+// fp16 activations in `scratch` for launch_ffn_down_tc.  xh16_ready: the
+// fp16 copy of xh in `scratch` is already current (launch_predict_tc wrote
+// it from the same xh and batch), so it is not rebuilt.
 cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                              const int32_t* idx, const int32_t* count, void* scratch,
-                             WsHeader* hdr, cudaStream_t s);
+                             WsHeader* hdr, cudaStream_t s, bool xh16_ready = false);
 
 // Split-K slices the down projection writes (part[0 .. splits)).
 int ffn_tc_down_splits(const pi_layer& L);
