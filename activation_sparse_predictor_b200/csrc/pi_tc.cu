@@ -6,8 +6,9 @@
 //
 //   up   : D[p][t] = sum_k W[row(p)][k] xh[t][k] for 128 list positions per
 //          tile (the MMA's A operand, K-major) and all tokens t (B: an fp16
-//          copy of the normalised inputs, tokens padded to 16); d split over
-//          up to 4 CTAs per tile; a second kernel sums the splits in a fixed
+//          copy of the normalised inputs, tokens padded to 16, shared with
+//          the predictor); d split over up to 4 CTAs per tile; a second
+//          kernel sums the splits in a fixed
 //          order, adds the bias, applies ReLU / ReGLU and the per-token bits
 //          and writes an fp16 copy h16[t][p];
 //   down : D[c][t] = sum_p W_down^T[row(p)][c] h16[t][p] for 128 output
@@ -23,10 +24,15 @@
 // one mask word per token with a ballot.
 //
 // A tile whose rows all lie in the hot prefix is one TMA box per operand
-// and stage; any other tile is gathered: each lane of the producer warp
-// issues one TMA tile::gather4 load (four rows, a one-row-high box) per
-// operand and stage.  128-byte swizzle throughout, a 4-stage mbarrier ring,
-// fp32 accumulators in tensor memory, one thread issuing the MMAs.  Every
+// and stage; any other tile is gathered with TMA tile::gather4 loads (four
+// rows, a one-row-high box).  A gather costs its issuing lane a while, so
+// the FFN kernels run 8 warps: warp 1 issues the MMAs, the other seven deal
+// out a stage's gathers round-robin and each arms its own bytes on the
+// stage's mbarrier; warps 0-3 then drain the accumulators.  Two CTAs
+// (about 100 KB of shared memory each) fit per SM, and the K splits are
+// sized to fill them.  128-byte swizzle throughout, a 4-stage ring for the
+// FFN and a 3-stage one for the predictor, fp32 accumulators in tensor
+// memory, one thread issuing the MMAs.  Every
 // mbarrier wait is bounded by %globaltimer (1 s): a wait that runs out sets
 // DEV_TIMEOUT in the workspace status word and a CTA abort flag; the
 // producer waits (bounded) for its copies in flight and the tensor memory
