@@ -34,7 +34,7 @@
  *    a token's mask has ceil(d_ff / 32) words; bits at or beyond d_ff are 0.
  *  - Synchronous argument errors return PI_ERR_INVALID (null or misaligned
  *    pointer, bad size, workspace too small) or PI_ERR_UNSUPPORTED (a dtype /
- *    activation / size combination this build does not implement) before
+ *    activation / size combination the library does not implement) before
  *    anything is enqueued.  A failed launch returns PI_ERR_CUDA.  Problems
  *    only the device can see (an index out of range, a bounded wait that ran
  *    out) set sticky bits in the workspace's status word and skip the bad
