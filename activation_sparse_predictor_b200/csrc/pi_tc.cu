@@ -216,6 +216,10 @@ __device__ __forceinline__ int list_row(int p, int H, int N, int F, const int32_
   return (j >= H && j < F) ? j : 0;
 }
 
+// Ring stages of the up kernel: two operands (ReGLU) make a 40 KB stage, so
+// two stages keep two CTAs (80 KB each) on an SM.
+__host__ __device__ constexpr int up_stages(int nr) { return nr == 2 ? 2 : TC_STAGES; }
+
 // up: NR = 1 ReLU (W_up), NR = 2 ReGLU (W_gate, W_up).  Grid (Fp / 128, ks).
 // part: [ks][NR][Fp][nt] fp32.
 template <int NR>
@@ -229,12 +233,13 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB (nt rows used)
   constexpr uint32_t STAGE = NR * A_BYTES + B_BYTES;
   constexpr uint32_t NCOLS = NR == 1 ? 64u : 128u;   // >= NR * nt, a power of two
+  constexpr int NS = up_stages(NR);
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = tc_sa(smem_raw);
   unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // swizzle atoms: 1 KB aligned
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_STAGES * STAGE);
-  uint64_t* empty = full + TC_STAGES;
-  uint64_t* done = empty + TC_STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STAGE);
+  uint64_t* empty = full + NS;
+  uint64_t* done = empty + NS;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
   int* rows = reinterpret_cast<int*>(tslot + 4);  // [128], 16-byte aligned
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   const int nkt = kt1 - kt0;
 
   if (threadIdx.x < TC_M) rows[threadIdx.x] = list_row(p0 + threadIdx.x, H, N, F, idx);
-  if (threadIdx.x == 0) tc_init(full, empty, done, abort, TC_STAGES, (uint32_t)TC_PW);
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort, NS, (uint32_t)TC_PW);
   if (warp == 0) tmem_alloc(tslot, NCOLS);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -271,12 +276,12 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
     const uint32_t mine = (uint32_t)((NR * 32 - pw + TC_PW - 1) / TC_PW);  // gathers of this warp
     const uint32_t tx = dense ? (pw == 0 ? NR * A_BYTES + bx : 0u) : 512u * mine + (pw == 0 ? bx : 0u);
-    int last[TC_STAGES];
-    for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
+    int last[NS];
+    for (int i = 0; i < NS; ++i) last[i] = -1;
     for (int i = 0; i < nkt; ++i) {
-      const int st = i % TC_STAGES;
+      const int st = i % NS;
       int ok = 1;
-      if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
+      if (lane == 0 && i >= NS) ok = tc_wait(&empty[st], ((i / NS) - 1) & 1, abort, hdr);
       if (!__shfl_sync(0xffffffffu, ok, 0)) break;
       unsigned char* a = smem + st * STAGE;
       if (lane == 0)
@@ -298,15 +303,15 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
       if (lane == 0) last[st] = i;
     }
     if (lane == 0) {  // every copy of this CTA has landed before it may exit (bounded)
-      for (int st = 0; st < TC_STAGES; ++st)
-        if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
+      for (int st = 0; st < NS; ++st)
+        if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / NS) & 1u, hdr);
     }
   } else if (warp == 1 && lane == 0) {
     // MMA issuer: kind::f16, fp16 A and B, fp32 D, both K-major, M = 128, N = nt
     const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
     for (int i = 0; i < nkt; ++i) {
-      const int st = i % TC_STAGES;
-      if (!tc_wait(&full[st], (uint32_t)(i / TC_STAGES) & 1u, abort, hdr)) break;
+      const int st = i % NS;
+      if (!tc_wait(&full[st], (uint32_t)(i / NS) & 1u, abort, hdr)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t a = tc_sa(smem + st * STAGE), b = a + NR * A_BYTES;
 #pragma unroll
@@ -841,7 +846,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   }
   const int tiles = Fp / TC_M, nk = d / TC_BK, ks = up_splits(d, F);
   constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
-  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16 + 4 * TC_M;
+  const size_t smem = 1024 + (size_t)up_stages(NR) * STAGE + 8 * (2 * up_stages(NR) + 1) + 16 + 4 * TC_M;
   auto kern = k_ffn_up_tc<NR>;
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
