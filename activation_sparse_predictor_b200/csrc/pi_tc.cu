@@ -31,7 +31,8 @@
 // stage's mbarrier; warps 0-3 then drain the accumulators.  Two CTAs
 // (about 100 KB of shared memory each) fit per SM, and the K splits are
 // sized to fill them.  128-byte swizzle throughout, a 4-stage ring for the
-// FFN and a 3-stage one for the predictor, fp32 accumulators in tensor
+// FFN (2 for the ReGLU up kernel, whose stage carries two operands) and a
+// 3-stage one for the predictor, fp32 accumulators in tensor
 // memory, one thread issuing the MMAs.  Every
 // mbarrier wait is bounded by %globaltimer (1 s): a wait that runs out sets
 // DEV_TIMEOUT in the workspace status word and a CTA abort flag; the
