@@ -124,6 +124,35 @@ def test_call_validation(pi):
     assert lib.pi_workspace_init(FAKE + 8, 1024, None) == pi.PI_ERR_INVALID
 
 
+def test_newer_entry_points_validate_before_enqueuing(pi):
+    lib = pi._lib
+    L = _layer(pi)
+    # pi_predict_noalloc: its static scratch holds batch x rank <= 262144 floats
+    big = _layer(pi, rank=8192)
+    assert lib.pi_predict_noalloc(ctypes.byref(big), FAKE, 64, 0.5, FAKE, None) == pi.PI_ERR_INVALID
+    assert "static scratch" in pi.pi_last_error()
+    assert lib.pi_predict_noalloc(ctypes.byref(L), FAKE, 0, 0.5, FAKE, None) == pi.PI_ERR_INVALID
+    assert lib.pi_predict_noalloc(ctypes.byref(L), FAKE, 1, 0.0, FAKE, None) == pi.PI_ERR_INVALID
+    assert lib.pi_predict_noalloc(ctypes.byref(L), FAKE + 4, 1, 0.5, FAKE, None) == pi.PI_ERR_INVALID
+    assert lib.pi_predict_noalloc(ctypes.byref(L), FAKE, 1, 0.5, None, None) == pi.PI_ERR_INVALID
+    # pi_wait_selftest: workspace, wait kind and time limit
+    assert lib.pi_wait_selftest(None, 4096, 0, 2000, None) == pi.PI_ERR_INVALID
+    assert lib.pi_wait_selftest(FAKE + 8, 4096, 0, 2000, None) == pi.PI_ERR_INVALID
+    assert lib.pi_wait_selftest(FAKE, 16, 0, 2000, None) == pi.PI_ERR_INVALID
+    assert lib.pi_wait_selftest(FAKE, 4096, 2, 2000, None) == pi.PI_ERR_INVALID
+    assert lib.pi_wait_selftest(FAKE, 4096, 1, 0, None) == pi.PI_ERR_INVALID
+    assert lib.pi_wait_selftest(FAKE, 4096, 1, 20000000, None) == pi.PI_ERR_INVALID
+    # counters and the timeline need their buffers
+    out = (ctypes.c_uint64 * 2)()
+    assert lib.pi_read_counters(None, None, 0, out) == pi.PI_ERR_INVALID
+    assert lib.pi_read_counters(FAKE, None, 0, None) == pi.PI_ERR_INVALID
+    arr = (pi.pi_layer * 1)(L)
+    assert lib.pi_ffn_stack_timeline(arr, 1, FAKE, 0.5, FAKE, 1 << 30, None, None,
+                                     None) == pi.PI_ERR_INVALID
+    assert lib.pi_ffn_stack_timeline(arr, 0, FAKE, 0.5, FAKE, 1 << 30, None, FAKE,
+                                     None) == pi.PI_ERR_INVALID
+
+
 def test_workspace_grows_with_batch(pi):
     L = _layer(pi)
     arr = (pi.pi_layer * 1)(L)
