@@ -297,7 +297,9 @@ namespace pi {
 namespace {
 
 // Device address of g_predict_u on the current device.  Looked up once per
-// device, by the first pi_predict_noalloc call made with that device current.
+// device, by the first pi_predict_noalloc call made with that device current,
+// and kept for the life of the process (a cudaDeviceReset would make it stale;
+// the header tells callers not to use this entry point across one).
 pi_status predict_scratch(float** out) {
   static std::mutex mu;
   static float* addr[64] = {};
@@ -519,6 +521,36 @@ pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {
     return cuda_fail(e, "counter clear");
   out[0] = v[0];
   out[1] = v[1];
+  return PI_OK;
+}
+
+pi_status pi_read_list(const pi_layer* layers, int n_layers, int batch, void* ws,
+                       size_t ws_bytes, void* stream, int32_t* idx_out, int cap,
+                       int32_t* count_out) {
+  if (!layers || n_layers < 1) return fail(PI_ERR_INVALID, "need at least one layer");
+  if (batch < 1 || batch > PI_MAX_BATCH) return fail(PI_ERR_INVALID, "batch %d not in [1, 64]", batch);
+  pi_status st;
+  for (int l = 0; l < n_layers; ++l)
+    if ((st = check_layer(&layers[l], l)) != PI_OK) return st;
+  if (!count_out || cap < 0 || (cap > 0 && !idx_out))
+    return fail(PI_ERR_INVALID, "null count_out, negative cap or null idx_out");
+  const WsLayout lay = layout_for_layers(layers, n_layers, batch);
+  if ((st = check_ws(ws, ws_bytes, lay)) != PI_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int32_t n = 0;
+  e = cudaMemcpy(&n, at<int32_t>(ws, lay.count), sizeof n, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "list length read");
+  int maxn = 0;
+  for (int l = 0; l < n_layers; ++l)
+    maxn = maxn > layers[l].d_ff - layers[l].hot ? maxn : layers[l].d_ff - layers[l].hot;
+  if (n < 0 || n > maxn) return fail(PI_ERR_DEVICE_CHECK, "list length %d out of range", n);
+  *count_out = n;
+  const int k = n < cap ? n : cap;
+  if (k > 0 && (e = cudaMemcpy(idx_out, at<int32_t>(ws, lay.idx), sizeof(int32_t) * (size_t)k,
+                               cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "list read");
   return PI_OK;
 }
 

@@ -100,6 +100,7 @@ struct StackParams {
   float* u;              // [r]
   float* part;           // [nsms][d]
   int32_t* count;        // cold-list length of the last layer
+  int32_t* idx;          // [d_ff] the layer's ascending cold list (last layer's stays)
   WsHeader* hdr;
   unsigned long long* trace;  // nullable [n_layers][nsms][16] timeline
   unsigned long long* utrace; // nullable [n_layers][UTR][4]: CTA 0's units
@@ -676,6 +677,7 @@ __device__ void compactor(const StackParams& P, const Smem& S) {
         const int slot = q + (r + k >= nS ? 1 : 0);
         S.items[R.nh + slot] = j;
         S.hbs[R.nh + slot] = L.bias ? L.bias[j] : 0.f;
+        __stcg(P.idx + (size_t)slot * nS + s, j);  // the global list, for inspection
       }
       r += c;
       if (r >= nS) {
@@ -1518,6 +1520,7 @@ cudaError_t launch_stack1(const pi_layer* layers, int n_layers, float* x, uint32
   P.u = reinterpret_cast<float*>((char*)ws + lay.u);
   P.part = reinterpret_cast<float*>((char*)ws + lay.part);
   P.count = reinterpret_cast<int32_t*>((char*)ws + lay.count);
+  P.idx = reinterpret_cast<int32_t*>((char*)ws + lay.idx);
   P.hdr = hdr;
   P.trace = trace;
   P.utrace = utrace;

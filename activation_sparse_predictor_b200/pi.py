@@ -63,6 +63,8 @@ def _load():
                                        ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
         "pi_kind_name": (ctypes.c_char_p, [i32]),
         "pi_read_counters": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_uint64)]),
+        "pi_read_list": (i32, [L, i32, i32, vp, sz, vp, ctypes.POINTER(ctypes.c_int32), i32,
+                               ctypes.POINTER(ctypes.c_int32)]),
         "pi_ffn_stack_timeline": (i32, [L, i32, vp, f32, vp, sz, vp, vp, vp]),
         "pi_device_sms": (i32, []),
         "pi_kernel_launches": (ctypes.c_ulonglong, []),
@@ -239,11 +241,21 @@ def pi_predict(layer: Layer, xh, tau: float, mask=None, ws=None, stream=None):
 
 
 def pi_predict_noalloc(layer: Layer, xh, tau: float, mask, stream=None):
-    """pi_predict without a workspace: u lives in the library's static
+    """The predictor without a workspace: u lives in the library's static
     per-device buffer (batch * rank <= PI_PREDICT_NOALLOC_MAX_FLOATS), so the
     call allocates nothing; `mask` [batch][words] int32 is the caller's.
-    Calls whose GPU work overlaps on one device race on that buffer."""
-    _check(_lib.pi_predict_noalloc(ctypes.byref(layer.c), _ptr(xh), xh.shape[0], tau,
+    Always the CUDA-core predictor kernels (see include/pi.h).  Calls whose
+    GPU work overlaps on one device race on that buffer."""
+    import torch
+    batch = xh.shape[0]
+    if (tuple(mask.shape) != (batch, layer.words) or mask.dtype != torch.int32
+            or not mask.is_contiguous() or mask.device != xh.device):
+        raise ValueError(f"mask must be a contiguous int32 tensor of shape {(batch, layer.words)} "
+                         f"on {xh.device}")
+    if xh.dtype != torch.float32 or not xh.is_contiguous() or xh.dim() != 2 \
+            or xh.shape[1] != layer.d_model:
+        raise ValueError(f"xh must be a contiguous float32 tensor [batch][{layer.d_model}]")
+    _check(_lib.pi_predict_noalloc(ctypes.byref(layer.c), _ptr(xh), batch, tau,
                                    _ptr(mask), _stream(stream)))
     return mask
 
@@ -311,6 +323,20 @@ def pi_read_counters(ws, clear: bool = False, stream=None):
     out = (ctypes.c_uint64 * 2)()
     _check(_lib.pi_read_counters(_ptr(ws), _stream(stream), int(clear), out))
     return int(out[0]), int(out[1])
+
+
+def pi_read_list(layers, batch: int, ws, stream=None, _arr=None):
+    """The ascending cold list (numpy int32) of the last layer of the last
+    stack call on `ws` (include/pi.h); synchronises the stream."""
+    import numpy as np
+    layers = layers if isinstance(layers, (list, tuple)) else [layers]
+    arr = _arr if _arr is not None else _layer_array(layers)
+    cap = max(L.d_ff for L in layers)
+    out = (ctypes.c_int32 * cap)()
+    n = ctypes.c_int32(0)
+    _check(_lib.pi_read_list(arr, len(layers), batch, _ptr(ws), ws.numel(), _stream(stream),
+                             out, cap, ctypes.byref(n)))
+    return np.frombuffer(out, dtype=np.int32, count=int(n.value)).copy()
 
 
 def pi_ffn_stack_timeline(layers, x, tau: float, ws=None, stream=None, _arr=None):

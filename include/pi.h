@@ -138,19 +138,27 @@ pi_status pi_workspace_init(void* ws, size_t ws_bytes, void* stream);
 pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float tau,
                      uint32_t* mask, void* ws, size_t ws_bytes, void* stream);
 
-/* pi_predict without a workspace: the same kernels, arguments and result
- * (mask) as pi_predict, with u kept in a static buffer of the library, one
- * per device, of PI_PREDICT_NOALLOC_MAX_FLOATS floats (1 MiB).  The method
- * itself has no counterpart to this entry point; it exists for callers that
- * must not allocate device memory: cudaMalloc and cudaFree synchronise the
- * whole device (stalling every stream's work, which latency-bound serving
- * loops avoid), and processes whose device memory is reserved up front by
- * their own allocator have none to give to a workspace.
+/* pi_predict without a workspace, for callers that cannot allocate device
+ * memory: cudaMalloc and cudaFree synchronise the whole device (stalling
+ * every stream, which latency-bound serving loops avoid), and a process
+ * whose device memory is reserved up front by its own allocator has none
+ * left to give to a workspace.  The method itself has no counterpart to
+ * this entry point.  The hidden vector u lives in a static buffer of the
+ * library, one per device, of PI_PREDICT_NOALLOC_MAX_FLOATS floats (1 MiB).
+ *   Kernels: always the CUDA-core predictor pair (u = p1 xh, then logits,
+ *          threshold and mask), at every batch.  pi_predict takes the
+ *          tensor-core predictor for fp16 predictors at 16-64 tokens, so at
+ *          those batches the two calls may set different bits for neurons
+ *          whose logit lies within about 1e-4 of logit(tau); elsewhere they
+ *          agree.  At other batches and dtypes the kernels, and so the
+ *          masks, are the same as pi_predict's.
  *   Limit: batch * rank <= PI_PREDICT_NOALLOC_MAX_FLOATS; larger calls
  *          return PI_ERR_INVALID (use pi_predict with a workspace).
  *   Set-up: the first call on each device, with that device current, looks
- *          up the buffer's device address (cudaGetSymbolAddress); make that
- *          first call before any stream capture.
+ *          up the buffer's device address (cudaGetSymbolAddress) and keeps
+ *          it for the life of the process; make that first call before any
+ *          stream capture, and do not call this entry point again on a
+ *          device after cudaDeviceReset (the kept address would be stale).
  *   Zeroing: nothing; every element of u is written before it is read.
  *   Concurrency: the buffer is shared by all calls on a device, so calls
  *          whose GPU work overlaps (e.g. on two streams with no ordering
@@ -274,6 +282,19 @@ unsigned long long pi_kernel_launches(void);
  * predictor's fixed size they give the bytes the path actually read.
  * `clear` != 0 resets both. */
 pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out);
+
+/* Synchronises `stream` and copies to the host the ascending list of cold
+ * neurons (ids in [hot, d_ff)) that the LAST layer of the last
+ * pi_ffn_stack / pi_ffn_stack_profile / pi_ffn_stack_timeline call on this
+ * workspace ran over (batch > 1: the list of the batch's union mask):
+ * *count_out receives the list's length and idx_out (host, int32) its first
+ * min(length, cap) ids.  layers, n_layers and batch are that call's (they
+ * fix the workspace layout).  Inspection of the compaction step
+ * (QbitAI article, §"Что такое «разреженная активация»?": only the predicted
+ * neurons are computed; the list is that set), used by tests. */
+pi_status pi_read_list(const pi_layer* layers, int n_layers, int batch, void* ws,
+                       size_t ws_bytes, void* stream, int32_t* idx_out, int cap,
+                       int32_t* count_out);
 
 /* Synchronises `stream`, reads the workspace's status word and returns
  * PI_OK, PI_ERR_DEVICE_CHECK or PI_ERR_TIMEOUT (timeout wins).  `detail`

@@ -151,6 +151,17 @@ def test_newer_entry_points_validate_before_enqueuing(pi):
                                      None) == pi.PI_ERR_INVALID
     assert lib.pi_ffn_stack_timeline(arr, 0, FAKE, 0.5, FAKE, 1 << 30, None, FAKE,
                                      None) == pi.PI_ERR_INVALID
+    # pi_read_list: layers, batch, outputs and the workspace size
+    n = ctypes.c_int32(0)
+    idx = (ctypes.c_int32 * 8)()
+    assert lib.pi_read_list(arr, 0, 1, FAKE, 1 << 30, None, idx, 8, ctypes.byref(n)) == pi.PI_ERR_INVALID
+    assert lib.pi_read_list(arr, 1, 65, FAKE, 1 << 30, None, idx, 8, ctypes.byref(n)) == pi.PI_ERR_INVALID
+    assert lib.pi_read_list(arr, 1, 1, FAKE, 1 << 30, None, idx, 8, None) == pi.PI_ERR_INVALID
+    assert lib.pi_read_list(arr, 1, 1, FAKE, 1 << 30, None, None, 8, ctypes.byref(n)) == pi.PI_ERR_INVALID
+    assert lib.pi_read_list(arr, 1, 1, FAKE, 1 << 30, None, idx, -1, ctypes.byref(n)) == pi.PI_ERR_INVALID
+    assert lib.pi_read_list(arr, 1, 1, FAKE, 64, None, idx, 8, ctypes.byref(n)) == pi.PI_ERR_INVALID
+    assert "too small" in pi.pi_last_error()
+    assert lib.pi_read_list(arr, 1, 1, FAKE + 8, 1 << 30, None, idx, 8, ctypes.byref(n)) == pi.PI_ERR_INVALID
 
 
 def test_workspace_grows_with_batch(pi):

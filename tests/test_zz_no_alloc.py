@@ -1,6 +1,7 @@
 """pi_predict_noalloc: the predictor with its hidden vector u in the
-library's static per-device buffer instead of a workspace.  Named to be
-collected last, so it also runs after every other test in one process."""
+library's static per-device buffer instead of a workspace, for callers that
+cannot allocate device memory.  Named to be collected last, so it also runs
+after every other test in one process."""
 import ctypes
 
 import numpy as np
@@ -31,6 +32,8 @@ def test_noalloc_rejects_batch_times_rank_beyond_its_buffer():
 
 @pytest.mark.gpu
 def test_noalloc_matches_predict_on_consecutive_calls():
+    """Batch 4 (both entry points on the CUDA-core kernels): bit-identical
+    masks on two calls in a row, each on a fresh input."""
     torch = pytest.importorskip("torch")
     from gpu_helpers import device_layer, words_np
     pi = _pi()
@@ -38,10 +41,42 @@ def test_noalloc_matches_predict_on_consecutive_calls():
     L, _ = device_layer(w, 0)
     batch = 4
     words = (w.d_ff + 31) // 32
-    for call in range(2):  # two calls in a row, each on a fresh input
+    for call in range(2):
         xh = synth.x_device(w, 10 + call, batch)
         want = pi.pi_predict(L, xh, w.tau)
         got = torch.full((batch, words), -1, dtype=torch.int32, device="cuda")
         pi.pi_predict_noalloc(L, xh, w.tau, got)
         torch.cuda.synchronize()
         assert np.array_equal(words_np(got), words_np(want)), call
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("batch", [16, 64])
+def test_noalloc_matches_oracle_at_token_batches(orc, batch):
+    """At 16 and 64 tokens pi_predict runs the tensor-core predictor and
+    pi_predict_noalloc the CUDA-core one: both must match the oracle's mask
+    outside the 1e-4 logit band, so they agree there too; two calls in a row."""
+    torch = pytest.importorskip("torch")
+    from gpu_helpers import BAND, check_mask, device_layer, unpack_bits, words_np
+    pi = _pi()
+    w = synth.WORKLOADS["relullama7b_reglu_4096x11008_f16"]
+    L, _ = device_layer(w, 0)
+    H = synth.layer_host(w, 0)
+    words = (w.d_ff + 31) // 32
+    theta = synth.threshold_logit(w.tau)
+    for call in range(2):
+        x = synth.x_host(w, 20 + call, batch)
+        xh = torch.from_numpy(x).cuda()
+        got = torch.full((batch, words), -1, dtype=torch.int32, device="cuda")
+        pi.pi_predict_noalloc(L, xh, w.tau, got)
+        want = pi.pi_predict(L, xh, w.tau)
+        torch.cuda.synchronize()
+        g, t = words_np(got), words_np(want)
+        for b in range(0, batch, 5 if batch > 16 else 1):
+            _, z = orc.predict(H, x[b].astype(np.float64))
+            check_mask(g[b], z, w.d_ff, w.hot, theta)
+            check_mask(t[b], z, w.d_ff, w.hot, theta)
+            outside = np.abs(z - theta) > BAND
+            gb, _ = unpack_bits(g[b], w.d_ff)
+            tb, _ = unpack_bits(t[b], w.d_ff)
+            assert np.array_equal(gb[outside], tb[outside]), (call, b)
