@@ -1,6 +1,7 @@
 // C ABI of libpi (declared in include/pi.h): argument validation, workspace
 // layout and the stream-ordered launch sequences of each entry point.
 #include <cmath>
+#include <cstddef>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -41,7 +42,7 @@ pi_status check_layer(const pi_layer* L, int i) {
   if (F < 1 || F > PI_MAX_D_FF) return fail(PI_ERR_INVALID, "layer %d: d_ff %d out of range", i, F);
   if (r < 1 || r > PI_MAX_RANK) return fail(PI_ERR_INVALID, "layer %d: rank %d out of range", i, r);
   if (H < 0 || H > F) return fail(PI_ERR_INVALID, "layer %d: hot %d not in [0, d_ff]", i, H);
-  if (L->act != PI_RELU && L->act != PI_REGLU)
+  if (L->act != PI_RELU && L->act != PI_REGLU && L->act != PI_RELU2)
     return fail(PI_ERR_INVALID, "layer %d: unknown activation %d", i, L->act);
   if (L->w_dtype != PI_F32 && L->w_dtype != PI_F16 && L->w_dtype != PI_Q4_0)
     return fail(PI_ERR_INVALID, "layer %d: unknown weight dtype %d", i, L->w_dtype);
@@ -72,7 +73,9 @@ pi_status check_layer(const pi_layer* L, int i) {
   if ((L->bias && !aligned(L->bias, 4)) || (L->p_bias && !aligned(L->p_bias, 4)))
     return fail(PI_ERR_INVALID, "layer %d: bias pointer not 4-byte aligned", i);
   const int64_t codes = row_bytes(L->w_dtype, d);
-  const int64_t strides[2] = {L->w_row_stride, L->w_down_row_stride};
+  if (!reglu && L->w_up_row_stride)
+    return fail(PI_ERR_INVALID, "layer %d: w_up_row_stride is for ReGLU layers only", i);
+  const int64_t strides[3] = {L->w_row_stride, L->w_down_row_stride, L->w_up_row_stride};
   for (int64_t st : strides)
     if (st != 0 && (st < codes || st % 16 != 0))
       return fail(PI_ERR_INVALID, "layer %d: row stride %lld must be 0 or a multiple of 16 >= %lld",
@@ -514,13 +517,16 @@ pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-  unsigned long long v[2];
+  unsigned long long v[3];
+  static_assert(offsetof(WsHeader, rows_second) == offsetof(WsHeader, rows_listed) + 16,
+                "counters are adjacent");
   e = cudaMemcpy(v, &header(ws)->rows_listed, sizeof v, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "counter read");
   if (clear && (e = cudaMemset(&header(ws)->rows_listed, 0, sizeof v)) != cudaSuccess)
     return cuda_fail(e, "counter clear");
   out[0] = v[0];
   out[1] = v[1];
+  out[2] = v[2];
   return PI_OK;
 }
 

@@ -23,9 +23,10 @@ enum : uint32_t {
 struct WsHeader {
   uint32_t status;                   // sticky DEV_* bits
   uint32_t pad0[15];
-  unsigned long long rows_listed;    // up/gate neuron rows processed (x token passes)
-  unsigned long long rows_down;      // down-projection rows read (h != 0)
-  unsigned long long stats_pad[6];
+  unsigned long long rows_listed;    // first-matrix neuron rows processed (x token passes)
+  unsigned long long rows_down;      // down-projection rows read
+  unsigned long long rows_second;    // ReGLU W_up rows read
+  unsigned long long stats_pad[5];
   uint32_t counters[32];             // grid-barrier / arrival counters
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");

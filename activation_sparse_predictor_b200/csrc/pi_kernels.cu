@@ -336,13 +336,20 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
     cnt = cnt < 0 ? 0 : F - H;
   }
   const int N = H + cnt;
-  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&hdr->rows_listed, (unsigned long long)N);
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) {
+    atomicAdd(&hdr->rows_listed, (unsigned long long)(N - n0));
+    if (ACT == PI_REGLU) atomicAdd(&hdr->rows_second, (unsigned long long)(N - n0));
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool sq = L.act == PI_RELU2;
   constexpr int NR = (ACT == PI_REGLU) ? 2 : 1;
   constexpr int CC = WTraits<WT>::CHUNK_COLS;
   const int nch = d / CC;
   const int64_t rb = code_stride(WT, d, L.w_row_stride);
   const int64_t sbs = scale_stride(d, L.w_row_stride);
+  const int64_t up_rs = (ACT == PI_REGLU && L.w_up_row_stride) ? L.w_up_row_stride : L.w_row_stride;
+  const int64_t rb2 = code_stride(WT, d, up_rs);
+  const int64_t sbs2 = scale_stride(d, up_rs);
   // list positions n0 .. N-1 (n0 = H when the hot rows are computed elsewhere)
   for (int n = n0 + blockIdx.x * kWarps + warp; n < N; n += gridDim.x * kWarps) {
     const int j = n < H ? n : idx[n - H];
@@ -358,9 +365,9 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
     const uint16_t* sc[NR];
     if constexpr (ACT == PI_REGLU) {
       rows[0] = (const char*)L.w_gate + (size_t)j * rb;
-      rows[1] = (const char*)L.w_up + (size_t)j * rb;
+      rows[1] = (const char*)L.w_up + (size_t)j * rb2;
       sc[0] = (const uint16_t*)((const char*)L.w_gate_scales + (size_t)j * sbs);
-      sc[1] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs);
+      sc[1] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs2);
     } else {
       rows[0] = (const char*)L.w_up + (size_t)j * rb;
       sc[0] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs);
@@ -378,6 +385,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
       float g = warp_sum(acc[0][b]) + bj;
       float hv = g > 0.f ? g : 0.f;
       if constexpr (ACT == PI_REGLU) hv *= warp_sum(acc[NR - 1][b]);
+      else if (sq) hv *= hv;  // squared ReLU
       if (per_token && n >= H && mask && t0 + b < B) {
         const uint32_t bit = (mask[(size_t)(t0 + b) * words + (j >> 5)] >> (j & 31)) & 1u;
         if (!bit) hv = 0.f;

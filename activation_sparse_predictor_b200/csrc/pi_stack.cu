@@ -50,11 +50,11 @@ constexpr int NPMAX = 3;            // producer warps (after the consumers)
 constexpr int NTHR = NCT + 32 * (NPMAX + 1);  // + the compaction warp
 constexpr int NSMAX = 24;           // ring stages at most
 constexpr int MAXL = 24;            // layers per launch
-constexpr int GRP = 32;             // items per cross-warp finalisation group
 constexpr int MAXA = 16;            // P1 rows per CTA at most
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int UTR = 512;            // units per layer recorded by the unit trace
-constexpr int DRMAX = 16;           // down rows per unit at most
+constexpr int DRMAX = 16;           // D records per unit at most
+constexpr int DR2MAX = 4;           // D records per unit at most, ReGLU (W_up dot partials)
 
 struct LayerPtrs {
   const char* first;            // W_gate (ReGLU) or W_up (ReLU): codes / rows
@@ -71,23 +71,33 @@ struct LayerPtrs {
 static_assert(sizeof(LayerPtrs) == 80, "compact layer pointers");
 
 // Shape and shared-memory plan, identical for every CTA.
+//
+// Phase C streams "first" records (the matrix whose ReLU decides activity:
+// W_gate for ReGLU, W_up for ReLU): [codes | scales (Q4_0)], padded to 16
+// bytes.  Phase D streams, for the neurons whose first pre-activation is
+// positive, "D records": ReGLU [up codes | up scales | pad | down codes |
+// down scales | pad], ReLU [down codes | down scales | pad].
 struct Plan {
   int d, F, r, H;
   int ns, G, maxc, maxi, nsms;
   int np;                           // producer warps
-  int gw, gd;                       // consumer warp groups: up-projection / down phases
-  int hp;                           // hot neurons per unit (adjacent records)
-  int dr;                           // down rows per unit (the last one of a layer: fewer)
-  int packed_up, packed_down;       // neuron records contiguous in memory
-  long long up_stride, down_stride; // bytes between consecutive neurons' rows (codes)
-  long long up_sstride, down_sstride; // the same for Q4_0 scales
+  int gw, gd;                       // consumer warp groups: phases A-C / phase D
+  int hp;                           // first records per hot unit (adjacent neurons)
+  int cp;                           // first records per cold unit
+  int dr;                           // D records per unit (the last one of a layer: fewer)
+  int sq;                           // squared ReLU: h = max(0, g)^2
+  int first_packed, d2_packed;      // records contiguous in memory at their own size
+  int first_contig, second_contig, down_contig;  // a row's Q4_0 scales right behind its codes
+  long long first_stride, first_sstride;    // bytes between neurons: codes / Q4_0 scales
+  long long second_stride, second_sstride;  // ReGLU W_up
+  long long down_stride, down_sstride;
   uint32_t sb;                      // stage bytes
   uint32_t rowb, scb;               // weight row bytes (codes), Q4_0 scale row bytes
   uint32_t p1_bytes, p2_row;        // predictor row bytes
-  uint32_t item_bytes, down_bytes;  // bytes copied per item / per down row
-  uint32_t o_first_s, o_second, o_second_s, o_down_s;  // offsets inside a stage
+  uint32_t first_b;                 // a first record in a stage
+  uint32_t d2_bytes, o_d2_down;     // a D record in a stage; offset of its down row
   uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_mw, o_scan, o_items, o_hval, o_flag,
-      o_dlist, o_pbs, o_hbs, o_redA, o_redC, o_redE, o_ring, total;
+      o_dlist, o_pbs, o_hbs, o_redA, o_redC, o_redD, o_redE, o_ring, total;
 };
 
 struct StackParams {
@@ -298,7 +308,8 @@ struct Smem {
   float* pbs;                 // predictor biases of the CTA's mask words
   float* hbs;                 // activation biases of the CTA's items
   float* redA;
-  float* redC;
+  float* redC;                // [GW][2][8][WPG] first-record dot partials
+  float* redD;                // [GD][2][DR2MAX][WPD] W_up dot partials (ReGLU)
   float4* redE;
   char* ring;
 };
@@ -327,6 +338,7 @@ __device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
   S.hbs = reinterpret_cast<float*>(base + pl.o_hbs);
   S.redA = reinterpret_cast<float*>(base + pl.o_redA);
   S.redC = reinterpret_cast<float*>(base + pl.o_redC);
+  S.redD = reinterpret_cast<float*>(base + pl.o_redD);
   S.redE = reinterpret_cast<float4*>(base + pl.o_redE);
   S.ring = reinterpret_cast<char*>(base + pl.o_ring);
   return S;
@@ -486,46 +498,59 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   };
   auto bar_of = [&]() { return &S.full[cu.st]; };
 
-  // Up-projection records of neurons j0 .. j0+n-1 (n > 1 only when packed).
-  auto items = [&](const LayerPtrs& L, int j0, int n) {
+  // One row part (codes, then Q4_0 scales right behind them) of neuron j.
+  auto part = [&](char* o, const char* codes, const char* scales, size_t j, long long cs,
+                  long long ss, bool contig, uint64_t* b) {
+    if (contig) {
+      bulk_g2s(o, codes + j * cs, pl.rowb + pl.scb, b);
+    } else {
+      bulk_g2s(o, codes + j * cs, pl.rowb, b);
+      if constexpr (WT == PI_Q4_0) bulk_g2s(o + pl.rowb, scales + j * ss, pl.scb, b);
+    }
+  };
+  // First records of n neurons into one stage, record r at r * first_b:
+  // the adjacent neurons j0 .. j0+n-1 (one copy when packed) or jl[0 .. n).
+  auto firsts = [&](const LayerPtrs& L, const int* jl, int j0, int n) {
     if (mine()) {
-      char* dst = claim(pl.item_bytes * (uint32_t)n);
+      char* dst = claim(pl.first_b * (uint32_t)n);
       if (dst) {
         uint64_t* b = bar_of();
-        if (pl.packed_up) {
-          bulk_g2s(dst, L.first + (size_t)j0 * pl.up_stride, pl.item_bytes * (uint32_t)n, b);
+        if (!jl && pl.first_packed) {
+          bulk_g2s(dst, L.first + (size_t)j0 * pl.first_stride, pl.first_b * (uint32_t)n, b);
         } else {
-          bulk_g2s(dst, L.first + (size_t)j0 * pl.up_stride, pl.rowb, b);
-          if constexpr (WT == PI_Q4_0)
-            bulk_g2s(dst + pl.o_first_s, L.first_scales + (size_t)j0 * pl.up_sstride, pl.scb, b);
-          if constexpr (ACT == PI_REGLU) {
-            bulk_g2s(dst + pl.o_second, L.second + (size_t)j0 * pl.up_stride, pl.rowb, b);
-            if constexpr (WT == PI_Q4_0)
-              bulk_g2s(dst + pl.o_second_s, L.second_scales + (size_t)j0 * pl.up_sstride, pl.scb, b);
-          }
+          for (int r = 0; r < n; ++r)
+            part(dst + (size_t)r * pl.first_b, L.first, L.first_scales,
+                 (size_t)(jl ? jl[r] : j0 + r), pl.first_stride, pl.first_sstride,
+                 pl.first_contig, b);
         }
       }
     }
     cu.next(pl.ns);
   };
-  // Down records of the neurons uj[0 .. n) into one stage, row k at
-  // k * down_bytes; adjacent packed records share one copy.
-  auto downs = [&](const LayerPtrs& L, const int* uj, int n) {
+  // D records of the neurons uj[0 .. n) into one stage, record k at
+  // k * d2_bytes (ReGLU: W_up part, then the down part at o_d2_down);
+  // adjacent packed records share one copy.
+  auto d2s = [&](const LayerPtrs& L, const int* uj, int n) {
     if (mine()) {
-      char* dst = claim(pl.down_bytes * (uint32_t)n);
+      char* dst = claim(pl.d2_bytes * (uint32_t)n);
       if (dst) {
         uint64_t* b = bar_of();
         for (int k = 0; k < n;) {
           int m = 1;
-          if (pl.packed_down)
+          if (pl.d2_packed)
             while (k + m < n && uj[k + m] == uj[k] + m) ++m;
-          char* d = dst + (size_t)k * pl.down_bytes;
-          if (pl.packed_down) {
-            bulk_g2s(d, L.down + (size_t)uj[k] * pl.down_stride, pl.down_bytes * (uint32_t)m, b);
+          char* o = dst + (size_t)k * pl.d2_bytes;
+          const size_t j = (size_t)uj[k];
+          if (pl.d2_packed) {
+            const char* src = ACT == PI_REGLU ? L.second + j * pl.second_stride
+                                              : L.down + j * pl.down_stride;
+            bulk_g2s(o, src, pl.d2_bytes * (uint32_t)m, b);
           } else {
-            bulk_g2s(d, L.down + (size_t)uj[k] * pl.down_stride, pl.rowb, b);
-            if constexpr (WT == PI_Q4_0)
-              bulk_g2s(d + pl.o_down_s, L.down_scales + (size_t)uj[k] * pl.down_sstride, pl.scb, b);
+            if constexpr (ACT == PI_REGLU)
+              part(o, L.second, L.second_scales, j, pl.second_stride, pl.second_sstride,
+                   pl.second_contig, b);
+            part(o + pl.o_d2_down, L.down, L.down_scales, j, pl.down_stride, pl.down_sstride,
+                 pl.down_contig, b);
           }
           k += m;
         }
@@ -558,11 +583,11 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         }
       }
     }
-    // C: hot groups, then (after the consumers' compaction) cold neurons
+    // C: first records of the hot groups, then (after the compaction warp's
+    // list) of the cold neurons, pl.cp per unit
     for (int gi = 0; gi < R.ngh && ok; ++gi) {
       const int j0 = hot_group_first(gi, pl);
-      const int n = min(pl.hp, pl.H - j0);
-      items(L, j0, n);
+      firsts(L, nullptr, j0, min(pl.hp, pl.H - j0));
     }
     {
       const unsigned long long t0 = P.trace ? gtime() : 0ull;
@@ -570,8 +595,9 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       if (P.trace) w_list += gtime() - t0;
     }
     const int nc = *S.nc;
-    for (int i = 0; i < nc && ok; ++i) items(L, S.items[R.nh + i], 1);
-    // D: down rows of items whose h != 0, in item order, pl.dr per unit
+    for (int i = 0; i < nc && ok; i += pl.cp) firsts(L, S.items + R.nh + i, 0, min(pl.cp, nc - i));
+    // D: D records of items whose first pre-activation is positive, in item
+    // order, pl.dr per unit
     const int tag = (l + 1) << 2;
     int uj[DRMAX], un = 0;  // the open unit's neurons
     for (int i = 0; i < R.nh + nc && ok; ++i) {
@@ -589,11 +615,11 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       if ((f & 3) != 2) continue;
       uj[un++] = S.items[i];
       if (un == pl.dr) {
-        downs(L, uj, un);
+        d2s(L, uj, un);
         un = 0;
       }
     }
-    if (ok && un > 0) downs(L, uj, un);
+    if (ok && un > 0) d2s(L, uj, un);
     if (P.trace && p == 0) {
       tstamp(P, l, 12, w_empty);
       tstamp(P, l, 13, w_list);
@@ -938,39 +964,18 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     if (tid == 0) tstamp(P, l, 4, gtime());
     gsync_arrive();  // 2: mask complete (waited for after the hot items)
 
-    // ---- C: items (hot, then cold); each unit shared by one warp group,
-    // per-warp partial sums combined in fixed order per group of GRP items
-    int fin = 0;  // next item to finalise
-    auto finalise = [&](int upto) {  // items [fin, upto)
-      csync();
-      const int i = fin + tid;
-      if (i < upto) {
-        const float* r = S.redC + ((i / GRP) & 1) * (GRP * NCW * 2) + (i % GRP) * NCW * 2;
-        float a = 0.f, b = 0.f;
-        for (int w = 0; w < WPG; ++w) {
-          a += r[2 * w];
-          b += r[2 * w + 1];
-        }
-        if constexpr (WT == PI_Q4_0) {
-          a *= *S.xscale;
-          b *= *S.xscale;
-        }
-        const float g = a + S.hbs[i];
-        float h = g > 0.f ? g : 0.f;
-        if constexpr (two) h *= b;
-        S.hval[i] = h;
-        __threadfence_block();
-        S.flag[i] = tag | (h != 0.f ? 2 : 1);
-      }
-      fin = upto;
-    };
-    // one unit: items i0 .. i0+n-1, record r of the stage for item i0 + r
+    // ---- C: first records (hot units, then cold units); each unit shared
+    // by one warp group.  Right after a unit the group's per-warp partial
+    // sums are combined in fixed order (a named barrier per group, partial
+    // buffers alternating by the group's unit parity) and the items' flags
+    // are set, so the producers can fetch the D records at once.
+    int gk = 0;  // units this group has taken in this layer
     auto unit_items = [&](int i0, int n) {
       if ((int)(cu.uc & gwm) == grp) {
         const bool ok = ready();
-        float a[8], b[8];
+        float a[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) a[r] = b[r] = 0.f;
+        for (int r = 0; r < 8; ++r) a[r] = 0.f;
         if (ok) {
           const char* base = stage();
           if constexpr (WT == PI_Q4_0) {
@@ -983,15 +988,10 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
 #pragma unroll
               for (int r = 0; r < 8; ++r) {
                 if (r >= n) break;
-                const char* buf = base + (size_t)r * pl.item_bytes;
+                const char* buf = base + (size_t)r * pl.first_b;
                 const uint4 cf = lds128(buf + (size_t)k * 16);
-                const float sf = h2f(reinterpret_cast<const uint16_t*>(buf + pl.o_first_s)[k]);
+                const float sf = h2f(reinterpret_cast<const uint16_t*>(buf + pl.rowb)[k]);
                 a[r] = fmaf((float)q4_block_dot(cf, xw, bs), sf, a[r]);
-                if constexpr (two) {
-                  const uint4 cs = lds128(buf + pl.o_second + (size_t)k * 16);
-                  const float sg = h2f(reinterpret_cast<const uint16_t*>(buf + pl.o_second_s)[k]);
-                  b[r] = fmaf((float)q4_block_dot(cs, xw, bs), sg, b[r]);
-                }
               }
             }
           } else {
@@ -1001,60 +1001,73 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
 #pragma unroll
               for (int r = 0; r < 8; ++r) {
                 if (r >= n) break;
-                const char* buf = base + (size_t)r * pl.item_bytes;
-                a[r] += chunk_dot<WT>(lds128(buf + (size_t)c * 16), S.xf, c, d);
-                if constexpr (two)
-                  b[r] += chunk_dot<WT>(lds128(buf + pl.o_second + (size_t)c * 16), S.xf, c, d);
+                a[r] += chunk_dot<WT>(lds128(base + (size_t)r * pl.first_b + (size_t)c * 16), S.xf,
+                                      c, d);
               }
             }
           }
           release(WPG);
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
+        for (int r = 0; r < 8; ++r) {
+          if (r >= n) break;
+          a[r] = warp_sum(a[r]);
+        }
+        float* rc = S.redC + (size_t)((grp * 2 + (gk & 1)) * 8) * WPG;
+        if (lane == 0) {
 #pragma unroll
           for (int r = 0; r < 8; ++r) {
             if (r >= n) break;
-            a[r] += __shfl_xor_sync(0xffffffffu, a[r], o);
-            if constexpr (two) b[r] += __shfl_xor_sync(0xffffffffu, b[r], o);
-          }
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          if (r >= n) break;
-          const float av = a[r];
-          const float bv = two ? b[r] : 0.f;
-          if (lane == 0) {
-            const int i = i0 + r;
-            float* rr = S.redC + ((i / GRP) & 1) * (GRP * NCW * 2) + (i % GRP) * NCW * 2 + 2 * wg;
-            rr[0] = av;
-            rr[1] = bv;
+            rc[r * WPG + wg] = a[r];
           }
         }
+        // every warp of the group reaches this barrier for every unit the
+        // group owns, whether or not its wait succeeded
+        asm volatile("bar.sync %0, %1;" ::"r"(2 + grp), "r"(GT) : "memory");
+        if (wg == 0 && lane < n) {
+          const float* q = rc + lane * WPG;
+          float g = 0.f;
+          for (int w = 0; w < WPG; ++w) g += q[w];
+          if constexpr (WT == PI_Q4_0) g *= *S.xscale;
+          g += S.hbs[i0 + lane];
+          float h = g > 0.f ? g : 0.f;  // ReGLU: the gate's ReLU; W_up comes in phase D
+          if constexpr (!two) {
+            if (pl.sq) h *= h;  // squared ReLU
+          }
+          S.hval[i0 + lane] = h;
+          __threadfence_block();
+          S.flag[i0 + lane] = tag | (h != 0.f ? 2 : 1);
+        }
+        ++gk;
       }
       cu.next(pl.ns);
-      // finalise every group of GRP items completed by this unit
-      const int i1 = i0 + n;
-      if (i1 / GRP != i0 / GRP) finalise((i1 / GRP) * GRP);
     };
     for (int gi = 0; gi < R.ngh; ++gi) {
       const int j0 = hot_group_first(gi, pl);
       unit_items(gi * pl.hp, min(pl.hp, pl.H - j0));
     }
-    if (fin < R.nh) finalise(R.nh);
     if (tid == 0) tstamp(P, l, 5, gtime());
 
     // ---- the CTA's share of the cold list, built by the compaction warp
-    // once every CTA's mask words are out (grid barrier 2)
-    const int nc = wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr) ? *S.nc : 0;
-    if (tid == 0) tstamp(P, l, 6, gtime());
-    for (int i = R.nh; i < R.nh + nc; ++i) unit_items(i, 1);
-    if (fin < R.nh + nc) finalise(R.nh + nc);
+    // once every CTA's mask words are out (grid barrier 2).  One thread
+    // waits and publishes the count, so every warp of a group walks the same
+    // units and reaches its group barrier the same number of times.
+    if (tid == 0) {
+      S.scan[NCW + 1] = wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr) ? *S.nc : 0;
+      tstamp(P, l, 6, gtime());
+    }
+    csync();
+    const int nc = S.scan[NCW + 1];
+    for (int i = 0; i < nc; i += pl.cp) unit_items(R.nh + i, min(pl.cp, nc - i));
     csync();
     if (tid == 0) tstamp(P, l, 7, gtime());
 
-    // ---- D: down rows of items with h != 0, pl.dr rows per unit, each unit
-    // shared by one of GD warp groups, each group covering every column with
-    // its own accumulators
+    // ---- D: D records of the items whose first pre-activation is positive
+    // (hval != 0), pl.dr per unit, each unit shared by one of GD warp
+    // groups, each group covering every column with its own accumulators.
+    // ReGLU: the group first forms each record's W_up dot (per-warp partials
+    // combined in fixed order after a named barrier), h = gate * up, then
+    // accumulates h times the down row.
     const int ni = R.nh + nc;
     if (warp == 0) {
       int base = 0;
@@ -1069,7 +1082,18 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     }
     csync();
     const int nd = S.scan[NCW];
-    const int nruns = (nd + pl.dr - 1) / pl.dr;  // units of pl.dr rows
+    const int nruns = (nd + pl.dr - 1) / pl.dr;  // units of pl.dr records
+    const int wd = warp % WPD;
+    int dk = 0;  // D units this group has taken in this layer
+    // h of the unit's record rr (ReGLU: after the group's W_up dot)
+    auto unit_h = [&](int q0, int len, const float* part_up, int rr) -> float {
+      const float g = S.hval[S.dlist[q0 + rr]];
+      if constexpr (!two) return g;
+      float u = 0.f;
+      for (int w = 0; w < WPD; ++w) u += part_up[rr * WPD + w];
+      if constexpr (WT == PI_Q4_0) u *= *S.xscale;
+      return g * u;
+    };
     if constexpr (WT == PI_Q4_0) {
       // one Q4_0 block (32 columns) per thread (the plan keeps d / 32 within
       // a group).  sum_j hs_j (q - 8), hs_j = h_j * scale, is accumulated as
@@ -1082,15 +1106,34 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       float corr = 0.f;
       for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
         if ((int)(cu.uc & gdm) != dgrp) continue;
-        if (!ready()) continue;
+        const bool ok = ready();
         const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
-        if (c < nch) {
+        float* pu = S.redD + (size_t)((dgrp * 2 + (dk & 1)) * DR2MAX) * WPD;
+        if constexpr (two) {
+          // W_up dots of the unit's records
+          for (int rr = 0; rr < len; ++rr) {
+            float a = 0.f;
+            if (ok && c < nch) {
+              const char* row = stage() + (size_t)rr * pl.d2_bytes;
+              const int4* xb = reinterpret_cast<const int4*>(S.xi);
+              const int4 x0 = xb[c], x1 = xb[nch + c], x2 = xb[2 * nch + c], x3 = xb[3 * nch + c];
+              const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                  x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+              a = (float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]) *
+                  h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
+            }
+            a = warp_sum(a);
+            if (lane == 0) pu[rr * WPD + wd] = a;
+          }
+          asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
+        }
+        if (ok && c < nch) {
 #pragma unroll 2
           for (int rr = 0; rr < len; ++rr) {
-            const char* row = stage() + (size_t)rr * pl.down_bytes;
+            const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
             const uint4 v = lds128(row + (size_t)c * 16);
-            const float hs =
-                S.hval[S.dlist[q0 + rr]] * h2f(reinterpret_cast<const uint16_t*>(row + pl.o_down_s)[c]);
+            const float hs = unit_h(q0, len, pu, rr) *
+                             h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
             corr += hs;
             const float2 h2 = make_float2(16.f * hs, 16.f * hs);
             const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
@@ -1108,7 +1151,8 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
             }
           }
         }
-        release(WPD);
+        if (ok) release(WPD);
+        ++dk;
       }
       // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
       if (c < nch) {
@@ -1131,30 +1175,47 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         for (int e = 0; e < CC; ++e) acc[k][e] = 0.f;
       for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
         if ((int)(cu.uc & gdm) != dgrp) continue;
-        if (!ready()) continue;
+        const bool ok = ready();
         const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
-        for (int rr = 0; rr < len; ++rr) {
-          const char* row = stage() + (size_t)rr * pl.down_bytes;
-          const float hv = S.hval[S.dlist[q0 + rr]];
+        float* pu = S.redD + (size_t)((dgrp * 2 + (dk & 1)) * DR2MAX) * WPD;
+        if constexpr (two) {
+          for (int rr = 0; rr < len; ++rr) {
+            float a = 0.f;
+            if (ok) {
+              const char* row = stage() + (size_t)rr * pl.d2_bytes;
+              for (int c = dtid; c < nch; c += DT)
+                a += chunk_dot<WT>(lds128(row + (size_t)c * 16), S.xf, c, d);
+            }
+            a = warp_sum(a);
+            if (lane == 0) pu[rr * WPD + wd] = a;
+          }
+          asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
+        }
+        if (ok) {
+          for (int rr = 0; rr < len; ++rr) {
+            const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
+            const float hv = unit_h(q0, len, pu, rr);
 #pragma unroll
-          for (int k = 0; k < MAXK; ++k) {
-            const int c = dtid + k * DT;
-            if (c >= nch) break;
-            const uint4 v = lds128(row + (size_t)c * 16);
-            if constexpr (WT == PI_F16) {
-              float f[8];
-              f16x8_to_f32(v, f);
+            for (int k = 0; k < MAXK; ++k) {
+              const int c = dtid + k * DT;
+              if (c >= nch) break;
+              const uint4 v = lds128(row + (size_t)c * 16);
+              if constexpr (WT == PI_F16) {
+                float f[8];
+                f16x8_to_f32(v, f);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(hv, f[e], acc[k][e]);
-            } else {
-              acc[k][0] = fmaf(hv, __uint_as_float(v.x), acc[k][0]);
-              acc[k][1] = fmaf(hv, __uint_as_float(v.y), acc[k][1]);
-              acc[k][2] = fmaf(hv, __uint_as_float(v.z), acc[k][2]);
-              acc[k][3] = fmaf(hv, __uint_as_float(v.w), acc[k][3]);
+                for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(hv, f[e], acc[k][e]);
+              } else {
+                acc[k][0] = fmaf(hv, __uint_as_float(v.x), acc[k][0]);
+                acc[k][1] = fmaf(hv, __uint_as_float(v.y), acc[k][1]);
+                acc[k][2] = fmaf(hv, __uint_as_float(v.z), acc[k][2]);
+                acc[k][3] = fmaf(hv, __uint_as_float(v.w), acc[k][3]);
+              }
             }
           }
+          release(WPD);
         }
-        release(WPD);
+        ++dk;
       }
       // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
       float* part = P.part + ((size_t)s * GD + dgrp) * d;
@@ -1170,6 +1231,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     }
     if (tid == 0) {
       atomicAdd(&hdr->rows_listed, (unsigned long long)ni);
+      if constexpr (two) atomicAdd(&hdr->rows_second, (unsigned long long)nd);
       atomicAdd(&hdr->rows_down, (unsigned long long)nd);
       tstamp(P, l, 8, gtime());
     }
@@ -1272,27 +1334,36 @@ int smem_optin() {
 uint32_t up16(uint32_t v) { return (v + 15u) & ~15u; }
 uint32_t up128(uint32_t v) { return (v + 127u) & ~127u; }
 
-// Whether every layer stores each neuron's up-projection record (and each
-// down row with its scales) contiguously, with the record as row stride.
-void packing(const pi_layer* layers, int n, uint32_t rowb, uint32_t scb, int* up, int* down) {
-  *up = *down = 1;
+// Layout flags of the layers' weights (all layers must agree): whether a
+// row's Q4_0 scales sit right behind its codes ("contig"), and whether whole
+// records are contiguous at their own size, so adjacent neurons are one copy
+// ("packed").  First records: [codes | scales] of W_gate (ReGLU) / W_up
+// (ReLU).  D records: ReGLU [W_up codes | scales | W_down^T codes | scales],
+// ReLU [W_down^T codes | scales].
+void packing(const pi_layer* layers, int n, uint32_t rowb, uint32_t scb, Plan* pl) {
+  pl->first_packed = pl->d2_packed = pl->first_contig = pl->second_contig = pl->down_contig = 1;
+  const uintptr_t rec = (uintptr_t)rowb + scb;
   for (int l = 0; l < n; ++l) {
     const pi_layer& L = layers[l];
     const bool two = L.act == PI_REGLU, q4 = L.w_dtype == PI_Q4_0;
-    const uintptr_t rec = (uintptr_t)rowb + scb;
     const uintptr_t first = (uintptr_t)(two ? L.w_gate : L.w_up);
     const uintptr_t first_s = (uintptr_t)(two ? L.w_gate_scales : L.w_up_scales);
-    const int64_t item = (two ? 2 : 1) * (int64_t)rec;
-    bool ok = code_stride(L.w_dtype, L.d_model, L.w_row_stride) == item;
-    if (q4) ok = ok && first_s == first + rowb;
-    if (two) {
-      ok = ok && (uintptr_t)L.w_up == first + rec;
-      if (q4) ok = ok && (uintptr_t)L.w_up_scales == (uintptr_t)L.w_up + rowb;
-    }
-    if (!ok) *up = 0;
-    bool dk = code_stride(L.w_dtype, L.d_model, L.w_down_row_stride) == (int64_t)rec;
-    if (q4) dk = dk && (uintptr_t)L.w_down_t_scales == (uintptr_t)L.w_down_t + rowb;
-    if (!dk) *down = 0;
+    const int64_t up_rs = two && L.w_up_row_stride ? L.w_up_row_stride : L.w_row_stride;
+    if (q4 && first_s != first + rowb) pl->first_contig = 0;
+    if (q4 && two && (uintptr_t)L.w_up_scales != (uintptr_t)L.w_up + rowb) pl->second_contig = 0;
+    if (q4 && (uintptr_t)L.w_down_t_scales != (uintptr_t)L.w_down_t + rowb) pl->down_contig = 0;
+    if (!(pl->first_contig && code_stride(L.w_dtype, L.d_model, L.w_row_stride) == (int64_t)rec))
+      pl->first_packed = 0;
+    bool dk;
+    if (two)
+      dk = pl->second_contig && pl->down_contig &&
+           (uintptr_t)L.w_down_t == (uintptr_t)L.w_up + rec &&
+           code_stride(L.w_dtype, L.d_model, up_rs) == 2 * (int64_t)rec &&
+           code_stride(L.w_dtype, L.d_model, L.w_down_row_stride) == 2 * (int64_t)rec;
+    else
+      dk = pl->down_contig &&
+           code_stride(L.w_dtype, L.d_model, L.w_down_row_stride) == (int64_t)rec;
+    if (!dk) pl->d2_packed = 0;
   }
 }
 
@@ -1304,6 +1375,7 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.r = L0.rank;
   pl.H = L0.hot;
   pl.nsms = nsms;
+  pl.sq = L0.act == PI_RELU2;
   const int d = pl.d, F = pl.F, r = pl.r, H = pl.H;
   const bool q4 = L0.w_dtype == PI_Q4_0, two = L0.act == PI_REGLU;
   const uint32_t pb = L0.p_dtype == PI_F32 ? 4u : 2u;
@@ -1311,33 +1383,36 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.scb = q4 ? (uint32_t)(d / 32) * 2u : 0u;
   pl.p1_bytes = (uint32_t)d * pb;
   pl.p2_row = (uint32_t)r * pb;
-  // record layout inside a stage: [first codes | first scales | second codes | second scales]
-  pl.o_first_s = pl.rowb;
-  pl.o_second = pl.rowb + pl.scb;
-  pl.o_second_s = 2 * pl.rowb + pl.scb;
-  pl.item_bytes = (two ? 2u : 1u) * (pl.rowb + pl.scb);
-  pl.o_down_s = pl.rowb;
-  pl.down_bytes = pl.rowb + pl.scb;
-  packing(layers, n_layers, pl.rowb, pl.scb, &pl.packed_up, &pl.packed_down);
-  pl.up_stride = code_stride(L0.w_dtype, d, L0.w_row_stride);
-  pl.up_sstride = scale_stride(d, L0.w_row_stride);
+  const uint32_t rec = pl.rowb + pl.scb;
+  if (rec % 16 || pl.rowb % 16 || pl.scb % 16) return false;  // 16-byte bulk copies
+  pl.first_b = rec;
+  pl.o_d2_down = two ? rec : 0u;
+  pl.d2_bytes = two ? 2u * rec : rec;
+  packing(layers, n_layers, pl.rowb, pl.scb, &pl);
+  const int64_t up_rs = L0.w_up_row_stride ? L0.w_up_row_stride : L0.w_row_stride;
+  pl.first_stride = code_stride(L0.w_dtype, d, L0.w_row_stride);
+  pl.first_sstride = scale_stride(d, L0.w_row_stride);
+  pl.second_stride = code_stride(L0.w_dtype, d, up_rs);
+  pl.second_sstride = scale_stride(d, up_rs);
   pl.down_stride = code_stride(L0.w_dtype, d, L0.w_down_row_stride);
   pl.down_sstride = scale_stride(d, L0.w_down_row_stride);
   for (int l = 1; l < n_layers; ++l)
-    if (layers[l].w_row_stride != L0.w_row_stride || layers[l].w_down_row_stride != L0.w_down_row_stride)
+    if (layers[l].w_row_stride != L0.w_row_stride || layers[l].w_down_row_stride != L0.w_down_row_stride ||
+        layers[l].w_up_row_stride != L0.w_up_row_stride)
       return false;
-  // adjacent hot records per unit (packed): units of at least 16 KB
+  // first records per hot unit (adjacent neurons): units of at least 16 KB
   pl.hp = 1;
-  if (pl.packed_up)
-    while (pl.hp < 8 && (uint32_t)pl.hp * pl.item_bytes < 16384u) ++pl.hp;
+  while (pl.hp < 8 && (uint32_t)pl.hp * rec < 16384u) ++pl.hp;
+  pl.cp = pl.hp;
   uint32_t sb = pl.p1_bytes;
-  sb = sb > (uint32_t)pl.hp * pl.item_bytes ? sb : (uint32_t)pl.hp * pl.item_bytes;
-  sb = sb > pl.down_bytes ? sb : pl.down_bytes;
+  sb = sb > (uint32_t)pl.hp * rec ? sb : (uint32_t)pl.hp * rec;
+  sb = sb > pl.d2_bytes ? sb : pl.d2_bytes;
   sb = sb > pl.p2_row ? sb : pl.p2_row;
   sb = up128(sb);
   pl.sb = sb;
-  pl.dr = (int)(sb / pl.down_bytes);
-  if (pl.dr > DRMAX) pl.dr = DRMAX;
+  pl.dr = (int)(sb / pl.d2_bytes);
+  const int drmax = two ? DR2MAX : DRMAX;
+  if (pl.dr > drmax) pl.dr = drmax;
   if (pl.dr < 1) pl.dr = 1;
   int G = 32;
   while (G > 1 && (uint32_t)G * pl.p2_row > sb) G >>= 1;
@@ -1363,7 +1438,8 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.o_pbs = o;        o = up16(o + 4u * 32u * bw);
   pl.o_hbs = o;        o = up16(o + 4u * pl.maxi);
   pl.o_redA = o;       o = up16(o + 4u * (MAXA + MAXA * NCW));
-  pl.o_redC = o;       o = up16(o + 4u * (2 * GRP * NCW * 2));
+  pl.o_redC = o;       o = up16(o + 4u * (2 * 8 * NCW));
+  pl.o_redD = o;       o = up16(o + 4u * (2 * DR2MAX * NCW));
   pl.o_redE = o;       o = up16(o + 16u * NCT);
   pl.o_ring = up128(o);
   const int avail = smem_optin() - (int)pl.o_ring;

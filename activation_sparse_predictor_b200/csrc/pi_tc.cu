@@ -389,13 +389,17 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
                                                     const int32_t* __restrict__ count,
                                                     const float* __restrict__ bias,
                                                     const uint32_t* __restrict__ mask, int words,
-                                                    __half* __restrict__ h16, WsHeader* hdr) {
+                                                    __half* __restrict__ h16, WsHeader* hdr,
+                                                    int sq) {
   __shared__ float sh[64][TC_TMAX + 1];
   __shared__ int sj[64];    // each row's neuron
   __shared__ float sb[64];  // and bias
   __shared__ int sv[64];    // 1: a listed row with a valid neuron
   const int N = list_len(count, H, F, hdr);
-  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) atomicAdd(&hdr->rows_listed, (unsigned long long)N);
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0) {
+    atomicAdd(&hdr->rows_listed, (unsigned long long)N);
+    if (NR == 2) atomicAdd(&hdr->rows_second, (unsigned long long)N);
+  }
   const int n0 = blockIdx.x * 64;
   const int m = 64 * nt;
   // per row once: neuron, index check, bias
@@ -431,6 +435,7 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
       g += sb[nn];
       hv = g > 0.f ? g : 0.f;
       if constexpr (NR == 2) hv *= u;
+      else if (sq) hv *= hv;  // squared ReLU
       if (mask && p >= H && !((__ldg(mask + (size_t)b * words + (j >> 5)) >> (j & 31)) & 1u)) hv = 0.f;
     }
     sh[nn][b] = hv;
@@ -830,12 +835,14 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
   const int64_t rs = code_stride(PI_F16, d, L.w_row_stride);
+  const int64_t rs2 = code_stride(PI_F16, d, NR == 2 && L.w_up_row_stride ? L.w_up_row_stride
+                                                                           : L.w_row_stride);
   const void* w0 = NR == 2 ? L.w_gate : L.w_up;
   CUtensorMap m0, m1, g0, g1, mx;
   if (!map_2d(&m0, w0, (uint64_t)d, (uint64_t)F, (uint64_t)rs, TC_M) ||
-      !map_2d(&m1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs, TC_M) ||
+      !map_2d(&m1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs2, TC_M) ||
       !map_2d(&g0, w0, (uint64_t)d, (uint64_t)F, (uint64_t)rs, 1) ||
-      !map_2d(&g1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs, 1) ||
+      !map_2d(&g1, L.w_up, (uint64_t)d, (uint64_t)F, (uint64_t)rs2, 1) ||
       !map_2d(&mx, sc.xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaSuccess;
@@ -857,7 +864,8 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_ffn_finish<NR><<<Fp / 64, 256, 0, s>>>(sc.part, ks, H, F, Fp, nt, batch, idx, count, L.bias,
-                                           mask, (F + 31) / 32, sc.h16, hdr);
+                                           mask, (F + 31) / 32, sc.h16, hdr,
+                                           L.act == PI_RELU2 ? 1 : 0);
   note_launch();
   return cudaGetLastError();
 }
@@ -870,7 +878,9 @@ bool ffn_tc_supported(const pi_layer& L, int batch) {
   if (L.d_model % TC_M != 0) return false;
   const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
   const int64_t rd = code_stride(PI_F16, L.d_model, L.w_down_row_stride);
-  if (rs % 16 != 0 || rd % 16 != 0) return false;
+  const int64_t ru = code_stride(PI_F16, L.d_model, L.w_up_row_stride ? L.w_up_row_stride
+                                                                      : L.w_row_stride);
+  if (rs % 16 != 0 || rd % 16 != 0 || ru % 16 != 0) return false;
   const uintptr_t bases = (uintptr_t)L.w_up | (uintptr_t)L.w_down_t |
                           (uintptr_t)(L.act == PI_REGLU ? L.w_gate : L.w_up);
   if (bases & 15u) return false;

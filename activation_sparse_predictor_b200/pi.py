@@ -18,10 +18,10 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "pi.h")
 
 PI_OK, PI_ERR_INVALID, PI_ERR_UNSUPPORTED, PI_ERR_CUDA, PI_ERR_TIMEOUT, PI_ERR_DEVICE_CHECK = range(6)
 PI_F32, PI_F16, PI_Q4_0 = 0, 1, 2
-PI_RELU, PI_REGLU = 0, 1
+PI_RELU, PI_REGLU, PI_RELU2 = 0, 1, 2
 PI_MASK_PER_TOKEN, PI_MASK_UNION = 0, 1
 DTYPES = {"f32": PI_F32, "f16": PI_F16, "q4_0": PI_Q4_0}
-ACTS = {"relu": PI_RELU, "reglu": PI_REGLU}
+ACTS = {"relu": PI_RELU, "reglu": PI_REGLU, "relu2": PI_RELU2}
 MODES = {"per_token": PI_MASK_PER_TOKEN, "union": PI_MASK_UNION}
 
 
@@ -41,6 +41,7 @@ class pi_layer(ctypes.Structure):
         ("w_down_t_scales", ctypes.c_void_p), ("bias", ctypes.c_void_p),
         ("p1", ctypes.c_void_p), ("p2", ctypes.c_void_p), ("p_bias", ctypes.c_void_p),
         ("w_row_stride", ctypes.c_int64), ("w_down_row_stride", ctypes.c_int64),
+        ("w_up_row_stride", ctypes.c_int64),
     ]
 
 
@@ -118,7 +119,7 @@ class Layer:
     scales) pairs for q4_0), bias, p1, p2, p_bias."""
 
     def __init__(self, *, d_model, d_ff, rank, hot, act, w_dtype, p_dtype, tensors: dict,
-                 w_row_stride: int = 0, w_down_row_stride: int = 0):
+                 w_row_stride: int = 0, w_down_row_stride: int = 0, w_up_row_stride: int = 0):
         self.tensors = tensors
         self.d_model, self.d_ff, self.rank, self.hot = d_model, d_ff, rank, hot
         self.act, self.w_dtype, self.p_dtype = act, w_dtype, p_dtype
@@ -137,7 +138,7 @@ class Layer:
         self.c = pi_layer(d_model, d_ff, rank, hot, ACTS[act], DTYPES[w_dtype], DTYPES[p_dtype],
                           g, u, dn, gs, us, ds, _ptr(tensors.get("bias")), _ptr(tensors["p1"]),
                           _ptr(tensors["p2"]), _ptr(tensors.get("p_bias")), w_row_stride,
-                          w_down_row_stride)
+                          w_down_row_stride, w_up_row_stride)
 
     @classmethod
     def from_workload(cls, w, tensors: dict, **strides) -> "Layer":
@@ -146,9 +147,9 @@ class Layer:
 
     @classmethod
     def packed(cls, w, tensors: dict) -> "Layer":
-        """A layer whose neuron records are packed (see pack_records): each
-        neuron's gate/up weights, and each down row with its scales, are one
-        contiguous span.  Returns the Layer; the packed buffers live in it."""
+        """A layer whose neuron records are packed (see pack_records) the way
+        the single-token kernel reads them.  Returns the Layer; the packed
+        buffers live in it."""
         packed, strides = pack_records(w, tensors)
         return cls.from_workload(w, packed, **strides)
 
@@ -159,10 +160,12 @@ class Layer:
 
 def pack_records(w, tensors: dict):
     """Rearranges a layer's FFN weights (dense matrices as produced by the
-    input generator) into per-neuron records on the same device:
-      up record j  : [gate row j | up row j]  (ReGLU) or [up row j] (ReLU),
-                     Q4_0 rows as [codes (d/2 B) | scales (d/16 B)];
-      down record j: [w_down_t row j] (Q4_0: codes | scales).
+    input generator) into per-neuron records on the same device, each row as
+    [codes | scales] for Q4_0, padded to 16 bytes:
+      ReGLU : gate records one after another (a neuron's activity is decided
+              by its gate row alone), and per neuron [up row | down row] (read
+              together, only for neurons whose gate fires);
+      ReLU, squared ReLU: up records, and down records, one after another.
     Returns (tensor dict with views into the packed buffers, strides)."""
     import torch
     def q4rows(pair):
@@ -175,26 +178,26 @@ def pack_records(w, tensors: dict):
     def asbytes(t):
         b = q4rows(t) if isinstance(t, tuple) else t.contiguous().view(torch.uint8).reshape(t.shape[0], -1)
         return pad16(b)
-    F = tensors["w_up"][0].shape[0] if isinstance(tensors["w_up"], tuple) else tensors["w_up"].shape[0]
-    first = [tensors["w_gate"], tensors["w_up"]] if w.act == "reglu" else [tensors["w_up"]]
-    up = torch.cat([asbytes(t) for t in first], 1).contiguous()
-    down = asbytes(tensors["w_down_t"]).contiguous()
     out = {k: v for k, v in tensors.items() if k not in ("w_gate", "w_up", "w_down_t")}
     rb = {"f32": 4 * w.d_model, "f16": 2 * w.d_model, "q4_0": w.d_model // 2}[w.w_dtype]
     sc = w.d_model // 16 if w.w_dtype == "q4_0" else 0
     rec = rb + sc + (-(rb + sc)) % 16
-    def view(buf, off, n):
-        return buf[:, off:off + n]
-    names = ["w_gate", "w_up"] if w.act == "reglu" else ["w_up"]
-    for i, name in enumerate(names):
-        base = i * rec
+    def rows(buf, off):
         if w.w_dtype == "q4_0":
-            out[name] = (view(up, base, rb), view(up, base + rb, sc))
-        else:
-            out[name] = view(up, base, rb)
-    out["w_down_t"] = (view(down, 0, rb), view(down, rb, sc)) if w.w_dtype == "q4_0" else view(down, 0, rb)
-    out["_packed_up"], out["_packed_down"] = up, down
-    return out, {"w_row_stride": up.shape[1], "w_down_row_stride": down.shape[1]}
+            return (buf[:, off:off + rb], buf[:, off + rb:off + rb + sc])
+        return buf[:, off:off + rb]
+    if w.act == "reglu":
+        first = asbytes(tensors["w_gate"]).contiguous()
+        second = torch.cat([asbytes(tensors["w_up"]), asbytes(tensors["w_down_t"])], 1).contiguous()
+        out["w_gate"], out["w_up"], out["w_down_t"] = rows(first, 0), rows(second, 0), rows(second, rec)
+        strides = {"w_row_stride": rec, "w_up_row_stride": 2 * rec, "w_down_row_stride": 2 * rec}
+    else:
+        first = asbytes(tensors["w_up"]).contiguous()
+        second = asbytes(tensors["w_down_t"]).contiguous()
+        out["w_up"], out["w_down_t"] = rows(first, 0), rows(second, 0)
+        strides = {"w_row_stride": rec, "w_down_row_stride": rec}
+    out["_packed_first"], out["_packed_second"] = first, second
+    return out, strides
 
 
 def _layer_array(layers):
@@ -319,10 +322,11 @@ def pi_ffn_stack_profile(layers, x, tau: float, mode: int, mask_trace=None, ws=N
 
 
 def pi_read_counters(ws, clear: bool = False, stream=None):
-    """(rows whose up/gate weights were read, w_down_t rows read); syncs."""
-    out = (ctypes.c_uint64 * 2)()
+    """(first-matrix rows read, w_down_t rows read, ReGLU w_up rows read);
+    synchronises the stream (include/pi.h)."""
+    out = (ctypes.c_uint64 * 3)()
     _check(_lib.pi_read_counters(_ptr(ws), _stream(stream), int(clear), out))
-    return int(out[0]), int(out[1])
+    return int(out[0]), int(out[1]), int(out[2])
 
 
 def pi_read_list(layers, batch: int, ws, stream=None, _arr=None):

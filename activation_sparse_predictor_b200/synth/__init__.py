@@ -45,7 +45,7 @@ X_LAYER_BASE = 1_000_000  # key-space "layer" of the input of decode step s
 @dataclass(frozen=True)
 class Workload:
     name: str
-    act: str            # "relu" | "reglu"
+    act: str            # "relu" | "reglu" | "relu2" (squared ReLU)
     d_model: int
     d_ff: int
     rank: int
@@ -97,6 +97,16 @@ WORKLOADS = {
         "q4_0", "f16", seed=4, tau=0.5, p_rule=("mean", 0.15, 1.0), steps=64,
         description="Llama2-70B-shaped ReGLU stack, 80 layers, Q4_0 weights, fp16 "
                     "predictor, batch 1 decode"),
+    "prosparse13b_reglu_5120x13824_f16": Workload(
+        "prosparse13b_reglu_5120x13824_f16", "reglu", 5120, 13824, 1024, 40, _hot(13824),
+        "f16", "f16", seed=6, tau=0.5, p_rule=("mean", 0.10, 1.0), steps=64,
+        description="ProSparse-Llama2-13B-shaped ReGLU stack, 40 layers, fp16, ~90% "
+                    "sparse, batch 1 decode"),
+    "bamboo7b_relu2_4096x14336_f16": Workload(
+        "bamboo7b_relu2_4096x14336_f16", "relu2", 4096, 14336, 1024, 32, _hot(14336),
+        "f16", "f16", seed=7, tau=0.5, p_rule=("mean", 0.10, 1.0), steps=64,
+        description="Bamboo-7B-shaped squared-ReLU stack, 32 layers, fp16, ~90% sparse, "
+                    "batch 1 decode"),
     "opt175b_relu_12288x49152_f16": Workload(
         "opt175b_relu_12288x49152_f16", "relu", 12288, 49152, 1024, 12, _hot(49152),
         "f16", "f16", seed=5, tau=0.5, p_rule=("mean", 0.05, 1.1), steps=16,

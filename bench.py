@@ -190,20 +190,25 @@ def predictor_bytes(w) -> float:
     return (w.rank * w.d_model + (w.d_ff - w.hot) * w.rank) * pb + (w.d_ff - w.hot) * 4
 
 
-def layer_algorithmic_bytes(w, rows_listed: int, rows_down: int, n_layers: int) -> dict:
+def layer_algorithmic_bytes(w, rows_listed: int, rows_down: int, n_layers: int,
+                            rows_second: int | None = None) -> dict:
     """Algorithmic bytes of each kernel kind summed over a run in which the
-    FFN launches processed `rows_listed` up/gate rows and read `rows_down`
-    w_down_t rows, over `n_layers` layer evaluations (batch 1)."""
+    FFN launches read `rows_listed` first-matrix rows (W_gate for ReGLU,
+    W_up otherwise), `rows_second` W_up rows (ReGLU; None = one per listed
+    row, as the batch kernels read them) and `rows_down` w_down_t rows, over
+    `n_layers` layer evaluations (batch 1)."""
     rb = weight_row_bytes(w.w_dtype, w.d_model)
     d4 = 4.0 * w.d_model
     words = (w.d_ff + 31) // 32
+    if rows_second is None:
+        rows_second = rows_listed if w.act == "reglu" else 0
     return {
         "rmsnorm": n_layers * 2 * d4,
         "pred_u": n_layers * (w.rank * w.d_model * {"f32": 4, "f16": 2}[w.p_dtype] + d4 + 4 * w.rank),
         "pred_z": n_layers * ((w.d_ff - w.hot) * w.rank * {"f32": 4, "f16": 2}[w.p_dtype]
                               + (w.d_ff - w.hot) * 4 + 4 * w.rank + 4 * words),
         "compact": n_layers * 4.0 * words,
-        "ffn_up": rows_listed * ((w.nm - 1) * rb + 4 + 4) + n_layers * (d4 + 4 * words),
+        "ffn_up": rows_listed * (rb + 4 + 4) + rows_second * rb + n_layers * (d4 + 4 * words),
         "ffn_down": rows_down * rb,
         "reduce": 0.0,  # partials live in L2; counted as traffic only by ncu
     }
@@ -236,9 +241,55 @@ def cpu_oracle_tokens_per_s(w, n_sample_layers: int, reps: int, step0: int = 0):
     return tps, orc.num_threads(), s, desc
 
 
+def cpu_oracle_variants(w, budget_s: float = 12.0) -> dict:
+    """The oracle as it stands, on one token through one layer of the
+    workload, timed four ways: the sparse layer (predictor, compaction, FFN
+    over the predicted set: the method) and the dense FFN (every neuron), each
+    on all host threads and on one thread.  Repetitions stop once a variant
+    has used its share of `budget_s`.  Returns {variant: {...}}."""
+    from activation_sparse_predictor_b200 import synth
+    from oracle import Oracle
+    orc = Oracle()
+    all_threads = orc.num_threads()
+    L = synth.layer_host(w, 0)
+    x = synth.x_host(w, 0, 1)[0]
+    xh = orc.rmsnorm(x)
+
+    def sparse():
+        orc.layer_forward(L, x, w.tau)
+
+    def dense():
+        orc.dense_ffn(L, xh)
+
+    out = {}
+    share = budget_s / 4.0
+    try:
+        for name, fn in (("sparse", sparse), ("dense", dense)):
+            for threads in (all_threads, 1):
+                orc.set_num_threads(threads)
+                times = []
+                t_start = time.perf_counter()
+                while not times or (time.perf_counter() - t_start < share and len(times) < 5):
+                    t0 = time.perf_counter()
+                    fn()
+                    times.append(time.perf_counter() - t0)
+                s = statistics.median(times)
+                key = f"{name}_{'all_threads' if threads == all_threads else '1_thread'}"
+                out[key] = {"tokens_per_s": 1.0 / (s * w.n_layers), "seconds_per_layer": s,
+                            "threads": threads, "reps": len(times)}
+    finally:
+        orc.set_num_threads(all_threads)
+    return out
+
+
 def run_reference(args, world, rank):
     """CPU oracle arm: rank 0 only, bounded sample per step."""
     if rank != 0:
+        return
+    if args.batch != 1:
+        print(json.dumps({"impl": "reference",
+                          "unavailable": "the oracle arm times single-token decode (batch 1) only"}),
+              flush=True)
         return
     from activation_sparse_predictor_b200 import build, synth
     build.build_synth()
@@ -247,7 +298,8 @@ def run_reference(args, world, rank):
     from oracle.build import build as build_oracle
     build_oracle()
     orc = Oracle()
-    layers = [synth.layer_host(w, l) for l in range(args.cpu_sample_layers)]
+    n_sample = min(args.cpu_sample_layers, w.n_layers)
+    layers = [synth.layer_host(w, l) for l in range(n_sample)]
     per_step = []
     for step in range(args.warmup + args.steps):
         x = synth.x_host(w, step, 1)[0]
@@ -266,10 +318,16 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": metric_name(w.name, 1), "value": tps, "unit": UNIT,
         "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1000.0 * sec_per_layer * w.n_layers, "higher_is_better": True,
+        "ms_per_step": 1000.0 * sec_per_layer * w.n_layers,
+        "ms_per_step_basis": (f"extrapolated: measured {1000.0 * sec_per_layer:.1f} ms per layer "
+                              f"over {len(layers)} sampled layers x {args.steps} steps, times "
+                              f"{w.n_layers} layers"),
+        "ms_per_sampled_step": 1000.0 * sum(per_step) / len(per_step),
+        "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded generator; no weights or datasets)",
-        "config": workload_config(w, 1, "per_token"),
+        "config": run_config(w, args.batch, args.mode, w.n_layers, args.gpus,
+                             l2_mode_for(w, w.n_layers, B200_L2_BYTES)),
         "cpu_baseline": {"value": tps, "unit": UNIT, "cores": orc.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": tps, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -310,13 +368,35 @@ def measured_traffic_per_layer(workload: str):
     return float(vals["dram_bytes_per_layer"])
 
 
-def workload_config(w, batch, mode):
+def workload_config(w, batch, mode, l2="streamed"):
+    l2_text = {
+        "streamed": "inputs larger than L2: every step streams the whole stack's weights "
+                    "and predictors from HBM (no flush needed)",
+        "flushed": "weights fit in L2: a 2 x L2 buffer is written between timed steps, each "
+                   "step timed on its own (cold L2)",
+        "resident": "weights fit in L2 and stay resident across back-to-back steps "
+                    "(L2-resident figure)",
+    }[l2]
     return {"workload": w.name, "layers": w.n_layers, "d_model": w.d_model, "d_ff": w.d_ff,
             "hot_prefix": w.hot, "predictor_rank": w.rank, "activation": w.act,
             "weights": w.w_dtype, "predictor_weights": w.p_dtype, "batch": batch,
-            "mask_mode": mode, "tau": w.tau,
-            "l2": "inputs larger than L2: every step streams the whole stack's weights "
-                  "and predictors from HBM (no flush needed)"}
+            "mask_mode": mode, "tau": w.tau, "l2": l2_text}
+
+
+B200_L2_BYTES = 126 * 2 ** 20  # used where no device is at hand (the CPU arm)
+
+
+def l2_mode_for(w, n_layers: int, l2_bytes: int) -> str:
+    """'flushed' when the stack's weights would fit twice in L2 (then each
+    step is timed on its own after a 2 x L2 write), else 'streamed'."""
+    from activation_sparse_predictor_b200 import synth
+    return "flushed" if n_layers * synth.layer_nbytes(w) < 2 * l2_bytes else "streamed"
+
+
+def run_config(w, batch, mode, n_layers, world, l2="streamed"):
+    """The `config` object both arms print for a run (same keys)."""
+    return dict(workload_config(w, batch, mode, l2), layers=n_layers,
+                parallelism=f"replicas x{world}" if world > 1 else "single GPU")
 
 
 # ---------------------------------------------------------------- GPU leg
@@ -366,8 +446,16 @@ def run_pi(args, world, rank, local):
     assert st == pi.PI_OK, f"device status {word:#x} after warm-up"
     pi.pi_read_counters(ws, clear=True, stream=stream)
 
-    # ---- timed region: K graph replays, inputs already in HBM
+    # ---- timed region: K graph replays, inputs already in HBM.  A stack
+    # whose weights fit in L2 is timed step by step with a 2 x L2 write
+    # between steps (cold L2); larger stacks stream from HBM on every step.
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    l2_mode = l2_mode_for(w, nl, l2_bytes)
+    flush = (torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev)
+             if l2_mode == "flushed" else None)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(K)] if flush is not None else []
     sampler = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(dev)
@@ -376,17 +464,35 @@ def run_pi(args, world, rank, local):
             ev0.record(stream)
             for i in range(K):
                 x.copy_(xs[W + i])
+                if flush is not None:
+                    flush.fill_(float(i))
+                    step_ev[i][0].record(stream)
                 g.replay()
+                if flush is not None:
+                    step_ev[i][1].record(stream)
             ev1.record(stream)
         torch.cuda.synchronize(dev)
     barrier(world)
-    ms = ev0.elapsed_time(ev1)
-    rows_listed, rows_down = pi.pi_read_counters(ws, clear=True, stream=stream)
+    ms = ev0.elapsed_time(ev1) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
+    rows_listed, rows_down, rows_second = pi.pi_read_counters(ws, clear=True, stream=stream)
     ms_max = max_over_ranks(ms, world, dev)
     value = world * K * B / (ms_max / 1000.0)
+    resident = None
+    if flush is not None:
+        # the same steps back to back, weights left in L2 (reported beside the number)
+        r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            r0.record(stream)
+            for i in range(K):
+                x.copy_(xs[W + i])
+                g.replay()
+            r1.record(stream)
+        torch.cuda.synchronize(dev)
+        pi.pi_read_counters(ws, clear=True, stream=stream)
+        resident = K * B / (r0.elapsed_time(r1) / 1000.0)
 
     # bytes actually read per step (predictor + listed rows + nonzero down rows)
-    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * nl)
+    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * nl, rows_second)
     step_bytes = sum(by.values()) / K
     peak, peak_kind = hbm_peak()
     step_gbs = step_bytes / (ms / K / 1000.0) / 1e9
@@ -395,13 +501,22 @@ def run_pi(args, world, rank, local):
     x.copy_(xs[W])
     pi.pi_read_counters(ws, clear=True, stream=stream)
     prof = pi.pi_ffn_stack_profile(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
-    pr_listed, pr_down = pi.pi_read_counters(ws, clear=True, stream=stream)
-    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, nl)
+    pr_listed, pr_down, pr_second = pi.pi_read_counters(ws, clear=True, stream=stream)
+    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, nl, pr_second)
     pby["fused_stack"] = sum(pby.values())  # the fused kernel runs every step
     prof = {k: v for k, v in prof.items() if v[1] > 0}
     dom = max(prof, key=lambda k: prof[k][0])
     dom_ms, dom_n = prof[dom]
-    achieved = pby[dom] / dom_n / (dom_ms / dom_n / 1000.0) / 1e9
+    if len(prof) == 1:
+        # one kernel kind makes the whole step: take its launch time from the
+        # timed graph replays that give `value`, and its bytes from their counters
+        timing_source = "graph replays of the timed region (the same timing as value)"
+        dom_ms = ms / K * dom_n / prof[dom][1]
+        dom_bytes_per_launch = step_bytes / dom_n
+    else:
+        timing_source = "profiled eager pass with CUDA events around every launch"
+        dom_bytes_per_launch = pby[dom] / dom_n
+    achieved = dom_bytes_per_launch / (dom_ms / dom_n / 1000.0) / 1e9
     # DRAM traffic per launch from the committed ncu capture of this kernel
     # (per layer, scaled to the layers of an average launch); null when the
     # capture was taken on other kernel sources
@@ -409,8 +524,8 @@ def run_pi(args, world, rank, local):
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
                 "traffic": tpl * nl / dom_n if tpl is not None else None,
-                "algorithmic_bytes_per_launch": pby[dom] / dom_n,
-                "avg_launch_us": 1000.0 * dom_ms / dom_n,
+                "algorithmic_bytes_per_launch": dom_bytes_per_launch,
+                "avg_launch_us": 1000.0 * dom_ms / dom_n, "timing_source": timing_source,
                 "per_kind_ms_per_step": {k: v[0] for k, v in prof.items()},
                 "launches_per_step": {k: v[1] for k, v in prof.items()}}
 
@@ -444,20 +559,24 @@ def run_pi(args, world, rank, local):
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        # ~10 s of oracle work: the sample layers, 24 passes
+        # ~10 s of oracle work: the sample layers, 24 passes (the sparse layer
+        # on every host thread: the reported value), then the sparse and the
+        # dense layer on one thread and on all threads (~12 s)
         tps, cores, s, desc = cpu_oracle_tokens_per_s(w, args.cpu_sample_layers, 24)
-        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        cpu = {"value": tps, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc,
+               "variants": cpu_oracle_variants(w)}
 
     line = {
         "metric": metric_name(w.name, B), "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded generator, weights generated on the GPU; no datasets)",
-        "config": dict(workload_config(w, B, args.mode), layers=nl,
-                       parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "config": run_config(w, B, args.mode, nl, world, l2_mode),
         "hbm_gbs_actual": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
         "bytes_per_step": step_bytes,
-        "rows_per_step": {"listed": rows_listed / K, "down_read": rows_down / K},
+        "rows_per_step": {"first_read": rows_listed / K, "second_read": rows_second / K,
+                          "down_read": rows_down / K},
+        "l2_resident_value": resident,
         "clocks": sampler.summary(),
         "e2e": e2e,
         "gpu_launches": K * kernels_per_step,

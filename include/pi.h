@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define PI_VERSION 1
+#define PI_VERSION 2
 #define PI_MAX_BATCH 64        /* tokens per call                           */
 #define PI_MAX_D_MODEL 16384   /* d_model upper bound                       */
 #define PI_MAX_RANK 8192       /* predictor rank upper bound                */
@@ -67,7 +67,7 @@ typedef enum pi_status {
 } pi_status;
 
 typedef enum pi_dtype { PI_F32 = 0, PI_F16 = 1, PI_Q4_0 = 2 } pi_dtype;
-typedef enum pi_act { PI_RELU = 0, PI_REGLU = 1 } pi_act;
+typedef enum pi_act { PI_RELU = 0, PI_REGLU = 1, PI_RELU2 = 2 } pi_act;
 
 /* How a batch's tokens share the predicted neuron set.
  *  PER_TOKEN: each token's FFN runs over its own predicted set; rows
@@ -82,9 +82,14 @@ typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_m
  *                        always-active prefix [0, H) of the neuron order.
  *  act        : PI_RELU  h_j = max(0, w_up[j].xh + bias[j])
  *               PI_REGLU h_j = max(0, w_gate[j].xh + bias[j]) * (w_up[j].xh)
+ *               PI_RELU2 h_j = max(0, w_up[j].xh + bias[j])^2  (squared ReLU)
+ *               A neuron is active when its first matrix's pre-activation
+ *               (w_gate for ReGLU, w_up otherwise) plus bias is > 0; an
+ *               inactive neuron's h is 0 and its down row, and (ReGLU) its
+ *               w_up row, contribute nothing and need not be read.
  *  w_dtype    : PI_F32, PI_F16 or PI_Q4_0 for w_gate / w_up / w_down_t.
  *  p_dtype    : PI_F32 or PI_F16 for p1 / p2.
- *  w_gate     : [F][d] (ReGLU only; NULL for ReLU).   w_up : [F][d].
+ *  w_gate     : [F][d] (ReGLU only; NULL otherwise).   w_up : [F][d].
  *  w_down_t   : [F][d], row j = column j of W_down, so y = sum_j h_j w_down_t[j].
  *  *_scales   : Q4_0 only, [F][d/32] binary16; NULL otherwise.
  *  bias       : [F] fp32 on the first matrix (gate for ReGLU, up for ReLU); NULL = 0.
@@ -92,11 +97,19 @@ typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_m
  *  p_bias     : [F] fp32; NULL = 0.
  *  w_row_stride     : bytes from row j to row j+1 of w_gate and w_up, and (Q4_0)
  *                     of their scale arrays; 0 = dense rows (codes d/2 bytes,
- *                     scales d/16 bytes apart for Q4_0).  A stride lets one
- *                     buffer hold each neuron's record [gate | up] (Q4_0:
- *                     [gate codes | gate scales | up codes | up scales]) so the
- *                     neuron's up-projection weights are one contiguous read.
+ *                     scales d/16 bytes apart for Q4_0).
  *  w_down_row_stride: the same for w_down_t and its scales.
+ *  w_up_row_stride  : ReGLU only: the same for w_up, when it differs from
+ *                     w_row_stride (0 = w_row_stride).
+ *  Strides let neuron records share buffers so that what is read together
+ *  is one contiguous span.  The single-token kernel reads fastest from:
+ *    ReGLU: gate records [codes | scales] one after another (w_row_stride =
+ *           record size), and per neuron [up record | down record]
+ *           (w_up_row_stride = w_down_row_stride = 2 records, w_down_t =
+ *           w_up + one record), so an active neuron's up and down rows are
+ *           one read;
+ *    ReLU / squared ReLU: up records one after another, down records one
+ *           after another (Q4_0: each row's scales right behind its codes).
  * Alignment: every weight pointer 16-byte aligned; d % 8 (F32, F16),
  * d % 32 (Q4_0) == 0; r % 4 (F32 predictor) / r % 8 (F16 predictor) == 0;
  * strides multiples of 16 and at least one row's codes. */
@@ -115,6 +128,7 @@ typedef struct pi_layer {
   const float* p_bias;
   int64_t w_row_stride;
   int64_t w_down_row_stride;
+  int64_t w_up_row_stride;
 } pi_layer;
 
 /* Bytes of workspace the calls below need for these layers at this batch
@@ -274,13 +288,16 @@ int pi_device_sms(void);
  * Never fails. */
 unsigned long long pi_kernel_launches(void);
 
-/* Synchronises `stream` and reads the workspace's two row counters, which
- * every FFN launch advances on the device: out[0] = neuron rows whose
- * gate/up (ReGLU) or up (ReLU) weights were read, out[1] = rows of w_down_t
- * read (rows whose h was nonzero for some token).  Each pass over a row by a
- * token chunk of at most 8 tokens counts once.  Together with the
- * predictor's fixed size they give the bytes the path actually read.
- * `clear` != 0 resets both. */
+/* Synchronises `stream` and reads the workspace's three row counters, which
+ * every FFN launch advances on the device: out[0] = neuron rows whose first
+ * matrix (w_gate for ReGLU, w_up otherwise) was read, out[1] = rows of
+ * w_down_t read, out[2] = rows of w_up read for ReGLU (0 otherwise).  The
+ * single-token kernel reads w_up (ReGLU) and w_down_t rows only for neurons
+ * whose first pre-activation is positive; the batch kernels read w_up for
+ * every listed neuron and w_down_t rows whose h is nonzero for some token.
+ * Each pass over a row by a token chunk of at most 8 tokens counts once.
+ * Together with the predictor's fixed size they give the bytes the path
+ * actually read.  out: uint64_t[3].  `clear` != 0 resets all three. */
 pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out);
 
 /* Synchronises `stream` and copies to the host the ascending list of cold

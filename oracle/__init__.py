@@ -20,9 +20,9 @@ import numpy as np
 from .build import LIB_PATH, build as _build
 
 OR_F32, OR_F16, OR_Q4_0 = 0, 1, 2
-OR_RELU, OR_REGLU = 0, 1
+OR_RELU, OR_REGLU, OR_RELU2 = 0, 1, 2
 _DT = {"f32": OR_F32, "f16": OR_F16, "q4_0": OR_Q4_0}
-_ACT = {"relu": OR_RELU, "reglu": OR_REGLU}
+_ACT = {"relu": OR_RELU, "reglu": OR_REGLU, "relu2": OR_RELU2}
 
 
 class _Layer(ctypes.Structure):
@@ -53,6 +53,7 @@ def load(path: str | None = None):
     lib = ctypes.CDLL(path)
     vp, i32, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
     lib.or_num_threads.restype = i32
+    lib.or_set_num_threads.argtypes = [i32]
     lib.or_half_to_double.restype = dbl
     lib.or_half_to_double.argtypes = [ctypes.c_uint16]
     lib.or_q4_0_weight.restype = dbl
@@ -83,6 +84,9 @@ class Oracle:
 
     def num_threads(self) -> int:
         return int(self.lib.or_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.or_set_num_threads(int(n))
 
     # ----------------------------------------------------------- layer struct
     def _layer(self, L: dict):

@@ -17,7 +17,8 @@
  *    groups are summed (same article, §"Гибридный дизайн вывода CPU/GPU",
  *    the neurons 3, 4, 5 example; aibars.net "SJTU-IPADS/PowerInfer"
  *    §"Mecanismo de Neurônios Quentes e Frios");
- *  - activations are ReLU / ReGLU (hada.io summary, §"Hạn chế và FAQ");
+ *  - activations are ReLU / ReGLU / squared ReLU (hada.io summary,
+ *    §"Hạn chế và FAQ");
  *  - weights may be INT4 Q4_0 (hada.io summary, §"Lượng tử hóa và tương
  *    thích").
  * Readings where the pages are silent (predictor = two bias-free linear
@@ -38,7 +39,7 @@
 #endif
 
 enum { OR_F32 = 0, OR_F16 = 1, OR_Q4_0 = 2 };
-enum { OR_RELU = 0, OR_REGLU = 1 };
+enum { OR_RELU = 0, OR_REGLU = 1, OR_RELU2 = 2 };
 
 typedef struct {
   int32_t d, F, r, H, act, wdt, pdt;
@@ -54,6 +55,16 @@ int or_num_threads(void) {
   return omp_get_max_threads();
 #else
   return 1;
+#endif
+}
+
+/* Threads the parallel loops below use from now on (results do not depend
+ * on it: every output is summed in the same order whatever the count). */
+void or_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
 #endif
 }
 
@@ -159,6 +170,8 @@ int or_compact(const uint32_t* masks, int nmask, int F, int begin, int32_t* idx)
  * §"Гибридный дизайн вывода CPU/GPU" is the sum over S in ascending order):
  *   ReLU : h_j = max(0, W_up[j] . xh + b_j)
  *   ReGLU: h_j = max(0, W_gate[j] . xh + b_j) * (W_up[j] . xh)
+ *   squared ReLU (hada.io summary §"Hạn chế và FAQ" names the activation;
+ *   reading: applied where ReLU is, no gate): h_j = max(0, W_up[j] . xh + b_j)^2
  *   y_i  = sum over j in S, ascending, of h_j * W_down^T[j][i]
  * h_j = 0 for j not in S.  With S = all neurons this is the dense FFN. */
 void or_ffn(const or_layer* L, const double* xh, const uint8_t* rowset, double* h, double* y) {
@@ -168,11 +181,12 @@ void or_ffn(const or_layer* L, const double* xh, const uint8_t* rowset, double* 
     h[j] = 0.0;
     if (!rowset[j]) continue;
     double b = L->bias ? (double)L->bias[j] : 0.0;
-    if (L->act == OR_RELU) {
+    if (L->act != OR_REGLU) {
       double g = 0.0;
       for (int i = 0; i < d; ++i) g += weight(L->wdt, L->wu, L->su, d, j, i) * xh[i];
       g += b;
       h[j] = g > 0.0 ? g : 0.0;
+      if (L->act == OR_RELU2) h[j] = h[j] * h[j];
     } else {
       double g = 0.0, u = 0.0;
       for (int i = 0; i < d; ++i) g += weight(L->wdt, L->wg, L->sg, d, j, i) * xh[i];

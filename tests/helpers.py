@@ -50,6 +50,8 @@ def torch_dense_ffn(L: dict, xh: np.ndarray) -> np.ndarray:
     x = torch.from_numpy(np.asarray(xh, np.float64))
     if L["workload"].act == "relu":
         h = torch.relu(T["w_up"] @ x + T["bias"])
+    elif L["workload"].act == "relu2":
+        h = torch.relu(T["w_up"] @ x + T["bias"]) ** 2
     else:
         h = torch.relu(T["w_gate"] @ x + T["bias"]) * (T["w_up"] @ x)
     return (T["w_down_t"].T @ h).numpy()

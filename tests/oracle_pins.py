@@ -39,7 +39,7 @@ def _dyadic_layer(act: str) -> dict:
          "w_down_t": f32(g["w_down_t"]), "bias": f32(g["bias"]),
          "p1": np.zeros((1, 4), np.float32), "p2": np.zeros((4, 1), np.float32),
          "p_bias": None}
-    if act == "relu":
+    if act in ("relu", "relu2"):
         L["w_up"] = f32(g["first_matrix"])
     else:
         L["w_gate"] = f32(g["first_matrix"])
@@ -97,8 +97,8 @@ def pin_rmsnorm_closed_form(orc):
 # ---------------------------------------------------------------------- FFN
 
 def pin_dyadic_ffn(orc):
-    """Hand-computed ReLU and ReGLU layers: h and y exact."""
-    for act in ("relu", "reglu"):
+    """Hand-computed ReLU, ReGLU and squared ReLU layers: h and y exact."""
+    for act in ("relu", "reglu", "relu2"):
         L, g = _dyadic_layer(act)
         h, y = orc.ffn(L, np.array(g["xh"]), np.ones(4, np.uint8))
         assert list(h) == g[f"{act}_h"], (act, list(h))
@@ -106,9 +106,10 @@ def pin_dyadic_ffn(orc):
 
 
 def pin_dense_vs_torch_f64(orc):
-    """Dense FFN == torch float64 matmul + relu, tiny sizes, all weight dtypes."""
+    """Dense FFN == torch float64 matmul + relu (squared for squared ReLU),
+    tiny sizes, all weight dtypes."""
     rng = np.random.default_rng(3)
-    for act in ("relu", "reglu"):
+    for act in ("relu", "reglu", "relu2"):
         for wdt in ("f32", "f16", "q4_0"):
             w = small_workload(act, wdt, d=64, F=96, r=16, seed=21)
             L = synth.layer_host(w, 0)
@@ -126,7 +127,7 @@ def _true_set(orc, L, xh):
 def pin_sparse_true_mask_equals_dense(orc):
     """With S = {j : activation > 0}, sparse == dense bitwise."""
     rng = np.random.default_rng(4)
-    for act in ("relu", "reglu"):
+    for act in ("relu", "reglu", "relu2"):
         w = small_workload(act, "f16", d=64, F=256, r=16, seed=22)
         L = synth.layer_host(w, 0)
         xh = unit_rms(rng, w.d_model)
@@ -174,7 +175,7 @@ def pin_hot_prefix_invariance(orc):
 def pin_partition_additivity(orc):
     """y(S1 U S2) = y(S1) + y(S2) for disjoint S1, S2 (merge of partial sums)."""
     rng = np.random.default_rng(7)
-    for act in ("relu", "reglu"):
+    for act in ("relu", "reglu", "relu2"):
         w = small_workload(act, "f32", d=64, F=200, r=16, seed=25)
         L = synth.layer_host(w, 0)
         xh = unit_rms(rng, w.d_model)

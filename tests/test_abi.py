@@ -41,7 +41,7 @@ def test_library_is_sm100a_only(pi):
 
 
 def test_status_strings_and_version(pi):
-    assert pi.pi_version() == 1
+    assert pi.pi_version() == 2
     assert pi.pi_status_string(pi.PI_OK) == "PI_OK"
     assert pi.pi_status_string(pi.PI_ERR_TIMEOUT) == "PI_ERR_TIMEOUT"
     assert pi.pi_status_string(99) == "PI_ERR_UNKNOWN"
@@ -88,6 +88,9 @@ def _layer(pi, **over):
     (dict(w_up=FAKE + 4), "PI_ERR_INVALID"),    # misaligned weight
     (dict(act=1, w_gate=None), "PI_ERR_INVALID"),
     (dict(w_dtype=2, d_model=64, w_up_scales=None), "PI_ERR_INVALID"),
+    (dict(w_up_row_stride=256), "PI_ERR_INVALID"),        # a ReGLU-only field on ReLU
+    (dict(act=1, w_up_row_stride=100), "PI_ERR_INVALID"),  # not a multiple of 16
+    (dict(act=1, w_up_row_stride=64), "PI_ERR_INVALID"),   # shorter than one row (128 B)
 ])
 def test_layer_validation(pi, over, expect):
     L = _layer(pi, **over)

@@ -48,6 +48,12 @@ def test_headline_layer_bytes():
     # bytes scale with the layer evaluations and the rows actually read
     by2 = bench.layer_algorithmic_bytes(w, 2 * listed, 2 * down, 2)
     assert sum(by2.values()) == pytest.approx(2 * total)
+    # second-level sparsity (ReGLU): W_up rows only where the gate fired
+    by3 = bench.layer_algorithmic_bytes(w, listed, down, 1, rows_second=down)
+    assert total - sum(by3.values()) == pytest.approx((listed - down) * row)
+    relu = synth.WORKLOADS["falcon40b_relu_8192x32768_f16"]
+    by4 = bench.layer_algorithmic_bytes(relu, 1000, 100, 1)
+    assert by4["ffn_up"] == pytest.approx(1000 * (16384 + 8) + (4 * 8192 + 4 * 1024))
 
 
 def test_traffic_figure_follows_the_kernel_sources(tmp_path, monkeypatch):
@@ -119,3 +125,12 @@ def test_clock_summary_without_nvml(monkeypatch):
     assert not s.ok
     out = s.summary()
     assert out["sm_mhz"] is None and out["reasons"] == []
+
+
+def test_l2_mode_by_stack_size():
+    # the tiny workload (8.4 MB) fits in L2: timed step by step after a flush
+    assert bench.l2_mode_for(synth.WORKLOADS["tiny_relu_512x2048_f32"], 1,
+                             bench.B200_L2_BYTES) == "flushed"
+    w = synth.WORKLOADS[HEADLINE]
+    assert bench.l2_mode_for(w, w.n_layers, bench.B200_L2_BYTES) == "streamed"
+    assert "L2" in bench.run_config(w, 1, "per_token", 80, 1)["l2"]

@@ -24,7 +24,7 @@ SHAPES = [  # d, F, r, H   (F ragged; H not always a multiple of 32)
     (256, 1000, 64, 200),
     (1024, 3001, 128, 640),
 ]
-KINDS = [(act, wdt) for act in ("relu", "reglu") for wdt in ("f32", "f16", "q4_0")]
+KINDS = [(act, wdt) for act in ("relu", "reglu", "relu2") for wdt in ("f32", "f16", "q4_0")]
 
 
 def _wl(act, wdt, shape, seed=41, mean=0.2):
@@ -214,7 +214,8 @@ def test_device_checks_flag_bad_lists(pi, orc):
 # -------------------------------------------------------------------- stack
 
 @pytest.mark.parametrize("act,wdt", [("relu", "f32"), ("reglu", "f16"), ("reglu", "q4_0"),
-                                     ("relu", "q4_0"), ("relu", "f16")])
+                                     ("relu", "q4_0"), ("relu", "f16"), ("relu2", "f16"),
+                                     ("relu2", "q4_0"), ("reglu", "f32")])
 @pytest.mark.parametrize("batch,mode", [(1, "union"), (4, "per_token"), (8, "union")])
 @pytest.mark.parametrize("packed", [False, True])
 def test_stack(pi, orc, act, wdt, batch, mode, packed):
@@ -294,7 +295,7 @@ def test_kernel_launch_counter(pi):
 
 
 @pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0)])
-@pytest.mark.parametrize("act", ["relu", "reglu"])
+@pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
 @pytest.mark.parametrize("batch,mode", [(16, "per_token"), (20, "union"), (48, "per_token"),
                                         (64, "union")])
 def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):

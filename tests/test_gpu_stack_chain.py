@@ -37,14 +37,15 @@ def _workload(act, w_dtype, seed):
         seed=seed, tau=0.5, p_rule=("mean", 0.15, 1.0), steps=1)
 
 
-CASES = [("reglu", "q4_0", 31), ("relu", "f16", 32), ("reglu", "f16", 33), ("relu", "f32", 34)]
+CASES = [("reglu", "q4_0", 31), ("relu", "f16", 32), ("reglu", "f16", 33), ("relu", "f32", 34),
+         ("relu2", "q4_0", 35)]
 
 
 def _first_preact(H, xh):
     """First-matrix pre-activation (gate for ReGLU, up for ReLU) + bias, in
     float64 from numpy's own decode: decides which down rows are read."""
     w = H["workload"]
-    W = np_decode(H["w_gate"] if w.act == "reglu" else H["w_up"], w.w_dtype)
+    W = np_decode(H["w_gate"] if w.act == "reglu" else H["w_up"], w.w_dtype)  # relu2: up
     return W @ xh + np.asarray(H["bias"], np.float64)
 
 
@@ -76,7 +77,9 @@ def test_stack_prefixes_cross_launch_boundaries(orc, act, w_dtype, seed):
         pi.pi_read_counters(ws, clear=True)
         pi.pi_ffn_stack(layers[:n], x, w.tau, pi.PI_MASK_UNION, mask_trace=tr, ws=ws)
         lst = pi.pi_read_list(layers[:n], 1, ws)
-        listed, down = pi.pi_read_counters(ws, clear=True)
+        listed, down, second = pi.pi_read_counters(ws, clear=True)
+        # ReGLU reads W_up rows exactly where it reads down rows (gate > 0)
+        assert second == (down if act == "reglu" else 0)
         xn = x.cpu().numpy()[0]
         trn = words_np(tr)[:, 0]
         assert np.array_equal(trn, full_trace[:n]), f"prefix {n}: trace differs from the full run"
@@ -118,7 +121,8 @@ def test_single_layer_row_counters(orc, act, w_dtype, seed):
         tr = torch.zeros((1, 1, words), dtype=torch.int32, device="cuda")
         pi.pi_read_counters(ws, clear=True)
         pi.pi_ffn_stack([L], x, w.tau, pi.PI_MASK_UNION, mask_trace=tr, ws=ws)
-        listed, down = pi.pi_read_counters(ws, clear=True)
+        listed, down, second = pi.pi_read_counters(ws, clear=True)
+        assert second == (down if act == "reglu" else 0)
         lst = orc.compact(words_np(tr)[0, 0], w.d_ff, w.hot)
         assert listed == w.hot + len(lst)
         xh = orc.rmsnorm(x0[0])

@@ -94,3 +94,9 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the same config object (keys and values) the GPU arm prints for this run
+    import bench
+    from activation_sparse_predictor_b200 import synth
+    w = synth.WORKLOADS["tiny_relu_512x2048_f32"]
+    assert d["config"] == bench.run_config(w, 1, "per_token", w.n_layers, 2, "flushed")
+    assert "extrapolated" in d["ms_per_step_basis"]

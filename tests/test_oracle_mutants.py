@@ -29,6 +29,9 @@ MUTANTS = [
     ("p1_transposed_scale", "acc += weight(L->pdt, L->p1, NULL, d, k, i) * xh[i];",
      "acc += weight(L->pdt, L->p1, NULL, d, k, i) * xh[d - 1 - i];"),
     ("predict_evaluates_hot_as_cold", "if (j < L->H) { z[j] = INFINITY; continue; }", ""),
+    ("relu2_not_squared", "if (L->act == OR_RELU2) h[j] = h[j] * h[j];", ""),
+    ("relu2_squares_before_relu", "h[j] = g > 0.0 ? g : 0.0;\n      if (L->act == OR_RELU2) h[j] = h[j] * h[j];",
+     "h[j] = g > 0.0 ? g : 0.0;\n      if (L->act == OR_RELU2) h[j] = g * g;"),
 ]
 
 
