@@ -90,20 +90,21 @@ WsLayout layout_for(int d, int F, int r, int batch, int H) {
   w.splits = down_splits(batch, d);
   w.xh = take((size_t)batch * d * 4);
   w.u = take((size_t)batch * r * 4);
-  w.mask = take((size_t)batch * words_of(F) * 4);
+  w.mask = take((size_t)(batch > 2 ? batch : 2) * words_of(F) * 4);
   w.idx = take((size_t)F * 4);
   w.count = take(16);
   w.h = take((size_t)F * batch * 4);
-  // split-K partials: the multi-kernel split, or one slice per SM for the
+  // split-K partials: the multi-kernel split, or one row per SM for the
   // fused single-token stack
   // (+ up to 4 slices of the tensor-core hot prefix at token batches)
   const size_t tcp = tc_scratch_bytes(d, F, r, batch) ? (size_t)4 * batch : 0;
-  const size_t parts = (size_t)w.splits * batch + tcp > 2 * (size_t)device_sms()
+  const size_t parts = (size_t)w.splits * batch + tcp > (size_t)device_sms()
                            ? (size_t)w.splits * batch + tcp
-                           : 2 * (size_t)device_sms();
+                           : (size_t)device_sms();
   w.part = take(parts * d * 4);
   w.y = take((size_t)batch * d * 4);
   w.tc = take(tc_scratch_bytes(d, F, r, batch));
+  w.cta = take(4 * (size_t)device_sms());
   w.total = off;
   return w;
 }

@@ -55,6 +55,7 @@ constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int UTR = 512;            // units per layer recorded by the unit trace
 constexpr int DRMAX = 16;           // D records per unit at most
 constexpr int DR2MAX = 4;           // D records per unit at most, ReGLU (W_up dot partials)
+constexpr int kQ4Blocks = 1;        // Q4_0 blocks per thread in phase D
 
 struct LayerPtrs {
   const char* first;            // W_gate (ReGLU) or W_up (ReLU): codes / rows
@@ -96,7 +97,7 @@ struct Plan {
   uint32_t p1_bytes, p2_row;        // predictor row bytes
   uint32_t first_b;                 // a first record in a stage
   uint32_t d2_bytes, o_d2_down;     // a D record in a stage; offset of its down row
-  uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_mw, o_scan, o_items, o_hval, o_flag,
+  uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_scan, o_items, o_hval, o_flag,
       o_dlist, o_pbs, o_hbs, o_redA, o_redC, o_redD, o_redE, o_ring, total;
 };
 
@@ -106,11 +107,13 @@ struct StackParams {
   float theta;
   float* x;              // [d] residual stream, in/out
   uint32_t* mask;        // this chunk's first layer's mask words
-  long long mask_stride; // words between consecutive layers' masks (0: reused)
+  long long mask_stride; // words between consecutive layers' masks (0: two alternating slots)
+  long long mask_words;  // words per mask
   float* u;              // [r]
   float* part;           // [nsms][d]
   int32_t* count;        // cold-list length of the last layer
   int32_t* idx;          // [d_ff] the layer's ascending cold list (last layer's stays)
+  uint32_t* cta_counts;  // [SMs] per-CTA cold-list lengths of the current layer (tagged)
   WsHeader* hdr;
   unsigned long long* trace;  // nullable [n_layers][nsms][16] timeline
   unsigned long long* utrace; // nullable [n_layers][UTR][4]: CTA 0's units
@@ -205,16 +208,14 @@ __device__ __forceinline__ float4 f4add(float4 a, float4 b) {
 // so the two float4 halves of 16-byte chunk c are float4 number c and
 // n/8 + c, and consecutive threads read consecutive 16-byte words (no bank
 // conflicts).  fp32 rows use the natural order.  The int16 copy of x^ for
-// Q4_0 rows is sub-chunk-major: element 32k + 8q + o at (q * nb + k) * 8 + o.
+// Q4_0 rows is sub-chunk-major: element 32k + 8q + o at (q * nb + k) * 8 + o
+// (nb = d / 32 blocks).
 template <int DT>
 __device__ __forceinline__ int vpos(int i, int n) {
   if constexpr (DT == PI_F16) return ((i & 7) >> 2) * (n >> 1) + ((i >> 3) << 2) + (i & 3);
   return i;
 }
 
-__device__ __forceinline__ int qpos(int i, int nb) {
-  return ((((i >> 3) & 3) * nb + (i >> 5)) << 3) + (i & 7);
-}
 
 // The staged-vector elements that chunk c of a DT row multiplies.
 struct VFrag {
@@ -290,7 +291,8 @@ __device__ __forceinline__ int q4_block_dot(const uint4 v, const int (&xw)[16], 
 struct Smem {
   uint64_t* full;
   uint64_t* empty;
-  uint64_t* listbar;
+  uint64_t* listbar;          // the CTA's cold list of the layer is ready
+  uint64_t* listdone;         // the list warp is done with it
   volatile int* abort;        // CTA-wide: stop waiting and computing
   volatile int* nc;           // this CTA's cold items (current layer)
   float* xscale;              // int16 scale of xh (Q4_0)
@@ -299,7 +301,6 @@ struct Smem {
   int* bsum;
   float* us;
   uint32_t* bw;
-  uint32_t* mw;
   int* scan;
   int* items;                 // neuron of each item: hot items, then this layer's cold list
   float* hval;
@@ -319,6 +320,7 @@ __device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
   S.full = reinterpret_cast<uint64_t*>(base);
   S.empty = S.full + NSMAX;
   S.listbar = S.empty + NSMAX;
+  S.listdone = S.listbar + 1;
   int* misc = reinterpret_cast<int*>(base + pl.o_misc);
   S.abort = misc;
   S.nc = misc + 1;
@@ -328,7 +330,6 @@ __device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
   S.bsum = reinterpret_cast<int*>(base + pl.o_bsum);
   S.us = reinterpret_cast<float*>(base + pl.o_u);
   S.bw = reinterpret_cast<uint32_t*>(base + pl.o_bw);
-  S.mw = reinterpret_cast<uint32_t*>(base + pl.o_mw);
   S.scan = reinterpret_cast<int*>(base + pl.o_scan);
   S.items = reinterpret_cast<int*>(base + pl.o_items);
   S.hval = reinterpret_cast<float*>(base + pl.o_hval);
@@ -390,6 +391,12 @@ __device__ bool grid_wait(WsHeader* hdr, uint32_t target, const Smem& S,
   }
 }
 
+// The mask words of layer l: its slot of the caller's trace, or one of two
+// alternating workspace slots.
+__device__ __forceinline__ uint32_t* layer_mask(const StackParams& P, int l) {
+  return P.mask + (P.mask_stride ? (size_t)l * P.mask_stride : (size_t)(l & 1) * P.mask_words);
+}
+
 // Timeline stamp, when a trace buffer is given.
 __device__ __forceinline__ void tstamp(const StackParams& P, int l, int slot,
                                        unsigned long long v) {
@@ -408,7 +415,7 @@ __device__ __forceinline__ void utstamp(const StackParams& P, int l, uint32_t u,
 
 struct Ranges {
   int kA0, kA1;   // P1 rows
-  int wB0, wB1;   // mask words evaluated here
+  int nw;         // mask words evaluated here: Wlo + s + k * SMs, k < nw
   int Wlo, W;     // first word holding a cold neuron, words per mask
   int ngh;        // hot groups g = s, s + SMs, ... of hp adjacent neurons
   int nh;         // hot neurons in them
@@ -422,8 +429,9 @@ __device__ __forceinline__ Ranges ranges(const Plan& pl) {
   R.W = (pl.F + 31) / 32;
   R.Wlo = pl.H / 32;
   const int Wc = R.W - R.Wlo;
-  R.wB0 = R.Wlo + (int)((long long)s * Wc / S);
-  R.wB1 = R.Wlo + (int)((long long)(s + 1) * Wc / S);
+  // interleaved, so that every CTA's words sample the whole cold range
+  // (the predicted density falls along the frequency-sorted order)
+  R.nw = Wc > s ? (Wc - 1 - s) / S + 1 : 0;
   const int G = (pl.H + pl.hp - 1) / pl.hp;
   R.ngh = s < G ? (G - 1 - s) / S + 1 : 0;
   R.nh = 0;
@@ -572,7 +580,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       }
     }
     // B: predictor rows of P2, G per unit
-    for (int w = R.wB0; w < R.wB1 && ok; ++w) {
+    for (int k = 0, w = R.Wlo + (int)blockIdx.x; k < R.nw && ok; ++k, w += (int)gridDim.x) {
       for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F && ok; ja += pl.G, cu.next(pl.ns)) {
         const int jb = min(ja + pl.G, pl.F);
         const uint32_t bytes = (uint32_t)(jb - ja) * pl.p2_row;
@@ -583,8 +591,9 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
         }
       }
     }
-    // C: first records of the hot groups, then (after the compaction warp's
-    // list) of the cold neurons, pl.cp per unit
+    // C: first records of the hot groups, then (once the consumers have
+    // listed the cold neurons of the CTA's own mask words) of the cold
+    // neurons, pl.cp per unit
     for (int gi = 0; gi < R.ngh && ok; ++gi) {
       const int j0 = hot_group_first(gi, pl);
       firsts(L, nullptr, j0, min(pl.hp, pl.H - j0));
@@ -642,81 +651,63 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   }
 }
 
-// --------------------------------------------------------------- compaction
+// --------------------------------------------------------------- list warp
 
-// One warp: after grid barrier 2 of each layer (every CTA's mask words are
-// out), the CTA's share of the ascending cold list: list position p (the
-// p-th set cold bit over the whole mask) belongs to CTA p mod SMs, slot
-// p / SMs.  A mask word holds at most 32 < SMs positions, so it holds at most
-// one of this CTA's.  Runs while the consumers are still on the hot items,
-// so the producers can copy the first cold records as soon as stages free.
+// One warp, off the critical path: once the CTA's mask words of a layer are
+// out (right after its phase B), it tags its slot of the per-CTA array,
+// waits (bounded) until every CTA has, then walks the layer's cold mask
+// words in order with a running count and writes the neurons of the CTA's
+// own words at their positions of the global ascending list (CTA 0 also
+// writes its length).  The computation never reads this list; it is there
+// for inspection (pi_read_list).  A wait that gives up leaves the list
+// incomplete and records the timeout.
 template <int WT, int ACT, int PT>
-__device__ void compactor(const StackParams& P, const Smem& S) {
+__device__ void list_writer(const StackParams& P, const Smem& S) {
   const Plan& pl = P.pl;
   WsHeader* hdr = P.hdr;
   const Ranges R = ranges(pl);
   const int lane = threadIdx.x & 31, nS = gridDim.x, s = blockIdx.x;
-  const int per = (R.W - R.Wlo + 31) / 32;  // mask words per lane
-  const int wa = R.Wlo + lane * per, wb = min(wa + per, R.W);
   for (int l = 0; l < P.n_layers; ++l) {
-    const LayerPtrs& L = P.L[l];
-    const uint32_t* mask = P.mask + (size_t)l * P.mask_stride;
     int ok = 1;
-    if (lane == 0) ok = grid_wait(hdr, (uint32_t)(4 * l + 2) * (uint32_t)nS, S) ? 1 : 0;
-    __syncwarp();  // lane 0's acquire orders the mask reads below
+    if (lane == 0) ok = wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr) ? 1 : 0;
     if (!__shfl_sync(0xffffffffu, ok, 0)) return;
-    // every cold mask word into shared memory: coalesced, 8 loads in flight per lane
-    const int Wc = R.W - R.Wlo;
-    for (int k0 = 0; k0 < Wc; k0 += 256) {
-      uint32_t v[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int k = k0 + 32 * t + lane;
-        v[t] = k < Wc ? __ldcg(mask + R.Wlo + k) : 0u;
-      }
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const int k = k0 + 32 * t + lane;
-        const int lo = 32 * (R.Wlo + k);
-        if (k < Wc) S.mw[k] = pl.H > lo ? (pl.H - lo >= 32 ? 0u : v[t] & (~0u << (pl.H - lo))) : v[t];
+    const uint32_t tag = (uint32_t)(l + 1);  // the array is zeroed before each launch
+    if (lane == 0)
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(P.cta_counts + s), "r"(tag) : "memory");
+    const uint64_t t0 = gtime();
+    for (int c = lane; c < nS && ok; c += 32) {
+      while (ld_acquire(P.cta_counts + c) != tag) {
+        if (*S.abort || gtime() - t0 > kTimeoutNs) { ok = 0; break; }
+        __nanosleep(256);
       }
     }
-    __syncwarp();
-    int cnt = 0;
-    for (int w = wa; w < wb; ++w) cnt += __popc(S.mw[w - R.Wlo]);
-    int incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) atomicOr(&hdr->status, DEV_TIMEOUT);
+      return;
     }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    const int p = incl - cnt;  // list position of this lane's first neuron
-    int r = p % nS, q = p / nS;
-    for (int w = wa; w < wb; ++w) {
-      uint32_t m = S.mw[w - R.Wlo];
+    const uint32_t* mask = layer_mask(P, l);
+    int base = 0;
+    for (int w0 = R.Wlo; w0 < R.W; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t m = w < R.W ? __ldcg(mask + w) : 0u;
+      const int lo = 32 * w;
+      if (pl.H > lo) m = pl.H - lo >= 32 ? 0u : m & (~0u << (pl.H - lo));  // hot bits
       const int c = __popc(m);
-      const int k = r <= s ? s - r : nS - r + s;  // offset of this CTA's position
-      if (k < c) {
-        for (int t = 0; t < k; ++t) m &= m - 1u;
-        const int j = 32 * w + __ffs(m) - 1;
-        const int slot = q + (r + k >= nS ? 1 : 0);
-        S.items[R.nh + slot] = j;
-        S.hbs[R.nh + slot] = L.bias ? L.bias[j] : 0.f;
-        __stcg(P.idx + (size_t)slot * nS + s, j);  // the global list, for inspection
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
       }
-      r += c;
-      if (r >= nS) {
-        r -= nS;
-        ++q;
+      if (w < R.W && (w - R.Wlo) % nS == s) {
+        int pos = base + incl - c;
+        for (; m; m &= m - 1u, ++pos) __stcg(P.idx + pos, lo + __ffs(m) - 1);
       }
+      base += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (lane == 0) {
-      *S.nc = total > s ? (total - s + nS - 1) / nS : 0;
-      if (s == 0) __stcg(P.count, total);
-    }
+    if (lane == 0 && s == 0) __stcg(P.count, base);
     __syncwarp();
-    if (lane == 0) mbar_arrive(S.listbar, 1u);  // releases the list to the CTA
+    if (lane == 0) mbar_arrive(S.listdone, 1u);  // done with this layer's mask
   }
 }
 
@@ -771,7 +762,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
 
   for (int l = 0; l < P.n_layers; ++l) {
     const LayerPtrs& L = P.L[l];
-    uint32_t* mask = P.mask + (size_t)l * P.mask_stride;
+    uint32_t* mask = layer_mask(P, l);
     const int tag = (l + 1) << 2;
     cur_l = l;
     l_uc0 = cu.uc;
@@ -898,8 +889,8 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     if (tid == 0) tstamp(P, l, 2, gtime());
     gsync_arrive();  // 1: u complete
     // biases used later in this layer: their load latency overlaps the barrier
-    for (int k = tid; k < (R.wB1 - R.wB0) * 32; k += NCT) {
-      const int j = 32 * R.wB0 + k;
+    for (int k = tid; k < R.nw * 32; k += NCT) {
+      const int j = 32 * (R.Wlo + s + (k >> 5) * nS) + (k & 31);
       S.pbs[k] = (L.pbias && j < pl.F) ? L.pbias[j] : 0.f;
     }
     for (int i = tid; i < R.nh; i += NCT) S.hbs[i] = L.bias ? L.bias[S.items[i]] : 0.f;
@@ -908,12 +899,12 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
 
     // ---- B: logits of the CTA's mask words; the group's warps take the rows
     for (int k = tid; k < pl.r; k += NCT) S.us[vpos<PT>(k, pl.r)] = __ldcg(P.u + k);
-    for (int k = tid; k < R.wB1 - R.wB0; k += NCT) S.bw[k] = 0u;
+    for (int k = tid; k < R.nw; k += NCT) S.bw[k] = 0u;
     csync();
     {
       constexpr int CCP = WTraits<PT>::CHUNK_COLS;
       const int nch = pl.r / CCP;
-      for (int w = R.wB0; w < R.wB1; ++w) {
+      for (int kw = 0, w = R.Wlo + s; kw < R.nw; ++kw, w += nS) {
         for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F; ja += pl.G, cu.next(pl.ns)) {
           if ((int)(cu.uc & gwm) != grp) continue;
           if (!ready()) continue;
@@ -938,21 +929,21 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
               z0 += __shfl_xor_sync(0xffffffffu, z0, o);
               z1 += __shfl_xor_sync(0xffffffffu, z1, o);
             }
-            const float za = z0 + S.pbs[j - 32 * R.wB0];
+            const float za = z0 + S.pbs[32 * kw + (j & 31)];
             if (j >= pl.H && za > P.theta) bits |= 1u << (j & 31);
             if (pair) {
-              const float zb = z1 + S.pbs[j2 - 32 * R.wB0];
+              const float zb = z1 + S.pbs[32 * kw + (j2 & 31)];
               if (j2 >= pl.H && zb > P.theta) bits |= 1u << (j2 & 31);
             }
           }
           release(WPG);
-          if (lane == 0 && bits) atomicOr(&S.bw[w - R.wB0], bits);
+          if (lane == 0 && bits) atomicOr(&S.bw[kw], bits);
         }
       }
     }
     csync();
-    for (int k = tid; k < R.wB1 - R.wB0; k += NCT) {
-      const int w = R.wB0 + k;
+    for (int k = tid; k < R.nw; k += NCT) {
+      const int w = R.Wlo + s + k * nS;
       uint32_t word = S.bw[k];
       const int lo = 32 * w;
       if (pl.H > lo) word |= (pl.H - lo >= 32) ? 0xFFFFFFFFu : ((1u << (pl.H - lo)) - 1u);
@@ -961,8 +952,35 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     for (int w = (int)((long long)s * R.Wlo / nS) + tid; w < (int)((long long)(s + 1) * R.Wlo / nS);
          w += NCT)
       __stcg(mask + w, 0xFFFFFFFFu);
+    // the CTA's cold list: the predicted cold neurons of its own mask words,
+    // ascending (one lane per word), published to the producers at once; no
+    // grid barrier is needed, the CTAs' word shares being disjoint
+    if (warp == 0) {
+      if (l > 0 && lane == 0) (void)wait_mbar(S.listdone, (uint32_t)(l - 1) & 1u, S, hdr);
+      __syncwarp();
+      const int nw = R.nw;  // <= 32 (plan)
+      const uint32_t word = lane < nw ? S.bw[lane] : 0u;
+      const int cnt = __popc(word);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += t;
+      }
+      const int total = __shfl_sync(0xffffffffu, incl, 31);
+      int pos = R.nh + incl - cnt;
+      for (uint32_t m = word; m; m &= m - 1u, ++pos) {
+        const int j = 32 * (R.Wlo + s + lane * nS) + __ffs(m) - 1;
+        S.items[pos] = j;
+        S.hbs[pos] = L.bias ? L.bias[j] : 0.f;
+      }
+      if (lane == 0) *S.nc = total;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(S.listbar, 1u);  // releases the list to the producers
+    }
     if (tid == 0) tstamp(P, l, 4, gtime());
-    gsync_arrive();  // 2: mask complete (waited for after the hot items)
+    csync();
+    const int nc = *S.nc;
 
     // ---- C: first records (hot units, then cold units); each unit shared
     // by one warp group.  Right after a unit the group's per-warp partial
@@ -1048,16 +1066,10 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     }
     if (tid == 0) tstamp(P, l, 5, gtime());
 
-    // ---- the CTA's share of the cold list, built by the compaction warp
-    // once every CTA's mask words are out (grid barrier 2).  One thread
-    // waits and publishes the count, so every warp of a group walks the same
-    // units and reaches its group barrier the same number of times.
-    if (tid == 0) {
-      S.scan[NCW + 1] = wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr) ? *S.nc : 0;
-      tstamp(P, l, 6, gtime());
-    }
-    csync();
-    const int nc = S.scan[NCW + 1];
+    // ---- then the CTA's cold neurons (nc was read after the barrier that
+    // follows the list, so every warp of a group walks the same units and
+    // reaches its group barrier the same number of times)
+    if (tid == 0) tstamp(P, l, 6, gtime());
     for (int i = 0; i < nc; i += pl.cp) unit_items(R.nh + i, min(pl.cp, nc - i));
     csync();
     if (tid == 0) tstamp(P, l, 7, gtime());
@@ -1095,15 +1107,21 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       return g * u;
     };
     if constexpr (WT == PI_Q4_0) {
-      // one Q4_0 block (32 columns) per thread (the plan keeps d / 32 within
-      // a group).  sum_j hs_j (q - 8), hs_j = h_j * scale, is accumulated as
-      // sum_j 16 hs_j (1 + q/16) with packed fp32x2 FMAs on floats built from
-      // the nibbles by byte permutes, minus 24 sum_j hs_j at the end.
-      const int nch = d / 32, c = dtid;
-      float2 acc[16];
+      // QB Q4_0 blocks (32 columns each) per thread (the plan keeps d / 32
+      // within a group's QB * DT).  sum_j hs_j (q - 8), hs_j = h_j * scale,
+      // is accumulated as sum_j 16 hs_j (1 + q/16) with packed fp32x2 FMAs on
+      // floats built from the nibbles by byte permutes, minus 24 sum_j hs_j
+      // at the end.
+      constexpr int QB = kQ4Blocks;
+      const int nch = d / 32;
+      float2 acc[QB][16];
+      float corr[QB];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) acc[e] = make_float2(0.f, 0.f);
-      float corr = 0.f;
+      for (int kb = 0; kb < QB; ++kb) {
+        corr[kb] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[kb][e] = make_float2(0.f, 0.f);
+      }
       for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
         if ((int)(cu.uc & gdm) != dgrp) continue;
         const bool ok = ready();
@@ -1113,60 +1131,94 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
           // W_up dots of the unit's records
           for (int rr = 0; rr < len; ++rr) {
             float a = 0.f;
-            if (ok && c < nch) {
+            if (ok) {
               const char* row = stage() + (size_t)rr * pl.d2_bytes;
               const int4* xb = reinterpret_cast<const int4*>(S.xi);
-              const int4 x0 = xb[c], x1 = xb[nch + c], x2 = xb[2 * nch + c], x3 = xb[3 * nch + c];
-              const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
-                                  x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-              a = (float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]) *
-                  h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
+              for (int c = dtid; c < nch; c += DT) {
+                const int4 x0 = xb[c], x1 = xb[nch + c], x2 = xb[2 * nch + c], x3 = xb[3 * nch + c];
+                const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                    x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+                a = fmaf((float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]),
+                         h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]), a);
+              }
             }
             a = warp_sum(a);
             if (lane == 0) pu[rr * WPD + wd] = a;
           }
           asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
         }
-        if (ok && c < nch) {
+        if (ok) {
 #pragma unroll 2
           for (int rr = 0; rr < len; ++rr) {
             const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
-            const uint4 v = lds128(row + (size_t)c * 16);
-            const float hs = unit_h(q0, len, pu, rr) *
-                             h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
-            corr += hs;
-            const float2 h2 = make_float2(16.f * hs, 16.f * hs);
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            const float hv = unit_h(q0, len, pu, rr);
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              // byte b: 0x80 | q << 3 for element 4m + b (low nibbles) / 16 + 4m + b (high)
-              const uint32_t lo = ((wv[m] << 3) & 0x78787878u) | 0x80808080u;
-              const uint32_t hi = ((wv[m] >> 1) & 0x78787878u) | 0x80808080u;
+            for (int kb = 0; kb < QB; ++kb) {
+              const int c = dtid + kb * DT;
+              if (c >= nch) break;
+              const uint4 v = lds128(row + (size_t)c * 16);
+              const float hs = hv * h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
+              corr[kb] += hs;
+              const float2 h2 = make_float2(16.f * hs, 16.f * hs);
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-              for (int b = 0; b < 4; b += 2) {
-                acc[(4 * m + b) >> 1] = __ffma2_rn(nib_pair(lo, b), h2, acc[(4 * m + b) >> 1]);
-                acc[(16 + 4 * m + b) >> 1] =
-                    __ffma2_rn(nib_pair(hi, b), h2, acc[(16 + 4 * m + b) >> 1]);
+              for (int m = 0; m < 4; ++m) {
+                // byte b: 0x80 | q << 3 for element 4m + b (low nibbles) / 16 + 4m + b (high)
+                const uint32_t lo = ((wv[m] << 3) & 0x78787878u) | 0x80808080u;
+                const uint32_t hi = ((wv[m] >> 1) & 0x78787878u) | 0x80808080u;
+#pragma unroll
+                for (int b = 0; b < 4; b += 2) {
+                  acc[kb][(4 * m + b) >> 1] =
+                      __ffma2_rn(nib_pair(lo, b), h2, acc[kb][(4 * m + b) >> 1]);
+                  acc[kb][(16 + 4 * m + b) >> 1] =
+                      __ffma2_rn(nib_pair(hi, b), h2, acc[kb][(16 + 4 * m + b) >> 1]);
+                }
               }
             }
           }
+          release(WPD);
         }
-        if (ok) release(WPD);
         ++dk;
       }
-      // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
-      if (c < nch) {
-        float* part = P.part + ((size_t)s * GD + dgrp) * d + (size_t)c * 32;
-        const float k24 = 24.f * corr;
+      // the CTA's partial row s: group GD-1 leaves its sums in shared memory
+      // (the fp32 copy of x^, free until the next layer), group 0 adds them
+      // to its own in a fixed order and writes the row
+      float4* xs4 = reinterpret_cast<float4*>(S.xf);
+      csync();
+      if (GD > 1 && dgrp == GD - 1) {
 #pragma unroll
-        for (int e = 0; e < 16; e += 2)
-          __stcg(reinterpret_cast<float4*>(part + 2 * e),
-                 make_float4(acc[e].x - k24, acc[e].y - k24, acc[e + 1].x - k24, acc[e + 1].y - k24));
+        for (int kb = 0; kb < QB; ++kb) {
+          const int c = dtid + kb * DT;
+          if (c >= nch) break;
+          const float k24 = 24.f * corr[kb];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2)
+            xs4[c * 8 + e / 2] = make_float4(acc[kb][e].x - k24, acc[kb][e].y - k24,
+                                             acc[kb][e + 1].x - k24, acc[kb][e + 1].y - k24);
+        }
+      }
+      csync();
+      if (dgrp == 0) {
+#pragma unroll
+        for (int kb = 0; kb < QB; ++kb) {
+          const int c = dtid + kb * DT;
+          if (c >= nch) break;
+          float* part = P.part + (size_t)s * d + (size_t)c * 32;
+          const float k24 = 24.f * corr[kb];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float4 v = make_float4(acc[kb][e].x - k24, acc[kb][e].y - k24, acc[kb][e + 1].x - k24,
+                                   acc[kb][e + 1].y - k24);
+            if (GD > 1) v = f4add(v, xs4[c * 8 + e / 2]);
+            __stcg(reinterpret_cast<float4*>(part + 2 * e), v);
+          }
+        }
       }
     } else {
-      // fp16 / fp32 rows: up to 48 columns per thread
+      // fp16 / fp32 rows: up to 48 columns per thread (32 for ReGLU, whose
+      // D phase also forms the W_up dots)
       constexpr int CC = WTraits<WT>::CHUNK_COLS;
-      constexpr int MAXK = 48 / CC;  // chunks per thread of a D group
+      constexpr int MAXK = (two ? 32 : 48) / CC;  // chunks per thread of a D group
       const int nch = d / CC;
       float acc[MAXK][CC];
 #pragma unroll
@@ -1217,16 +1269,35 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         }
         ++dk;
       }
-      // partial of (CTA s, group dgrp) -> partial row s * GD + dgrp
-      float* part = P.part + ((size_t)s * GD + dgrp) * d;
+      // the CTA's partial row s: group GD-1 leaves its sums in shared memory
+      // (the fp32 copy of x^, free until the next layer), group 0 adds them
+      // to its own in a fixed order and writes the row
+      float4* xs4 = reinterpret_cast<float4*>(S.xf);
+      csync();
+      if (GD > 1 && dgrp == GD - 1) {
 #pragma unroll
-      for (int k = 0; k < MAXK; ++k) {
-        const int c = dtid + k * DT;
-        if (c >= nch) break;
+        for (int k = 0; k < MAXK; ++k) {
+          const int c = dtid + k * DT;
+          if (c >= nch) break;
 #pragma unroll
-        for (int e = 0; e < CC; e += 4)
-          __stcg(reinterpret_cast<float4*>(part + c * CC + e),
-                 make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]));
+          for (int e = 0; e < CC; e += 4)
+            xs4[(c * CC + e) / 4] = make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]);
+        }
+      }
+      csync();
+      if (dgrp == 0) {
+        float* part = P.part + (size_t)s * d;
+#pragma unroll
+        for (int k = 0; k < MAXK; ++k) {
+          const int c = dtid + k * DT;
+          if (c >= nch) break;
+#pragma unroll
+          for (int e = 0; e < CC; e += 4) {
+            float4 v = make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]);
+            if (GD > 1) v = f4add(v, xs4[(c * CC + e) / 4]);
+            __stcg(reinterpret_cast<float4*>(part + c * CC + e), v);
+          }
+        }
       }
     }
     if (tid == 0) {
@@ -1239,11 +1310,11 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     gsync_wait();
     if (tid == 0) tstamp(P, l, 9, gtime());
 
-    // ---- E: reduce this CTA's float4 column slice over the nS * GD partial
-    // rows in a fixed order (rows in interleaved groups, then the groups in
+    // ---- E: reduce this CTA's float4 column slice over the nS partial rows
+    // in a fixed order (rows in interleaved groups, then the groups in
     // order), residual add.
     {
-      const int q4n = d / 4, nP = nS * GD;
+      const int q4n = d / 4, nP = nS;
       const int cq0 = (int)((long long)s * q4n / nS), cq1 = (int)((long long)(s + 1) * q4n / nS);
       const int nq = cq1 - cq0;  // <= 32
       const int g = nq > 0 ? NCT / nq : 0;
@@ -1294,6 +1365,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
       mbar_init(&S.empty[i], (uint32_t)NCW);
     }
     mbar_init(S.listbar, 1u);
+    mbar_init(S.listdone, 1u);
     *S.abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -1310,7 +1382,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
     if (p < P.pl.np) {
       if ((threadIdx.x & 31) == 0) producer<WT, ACT, PT>(P, S, p);
     } else if (p == NPMAX) {
-      compactor<WT, ACT, PT>(P, S);
+      list_writer<WT, ACT, PT>(P, S);
     }
     return;
   }
@@ -1418,10 +1490,14 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   while (G > 1 && (uint32_t)G * pl.p2_row > sb) G >>= 1;
   pl.G = G;
   const int W = (F + 31) / 32, Wlo = H / 32, Wc = W - Wlo;
-  pl.maxc = (F - H + nsms - 1) / nsms + 1;
+  // a CTA's cold neurons come from its own share of the mask words (one
+  // warp lane per word): up to 32 per word
+  const int wpc = (Wc + nsms - 1) / nsms;  // mask words per CTA at most
+  if (wpc > 32) return false;
+  pl.maxc = 32 * wpc;
   pl.maxi = (H + nsms - 1) / nsms + pl.hp + pl.maxc + 1;
-  const int bw = Wc / nsms + 2;
-  uint32_t o = 8 * (2 * NSMAX + 1);  // mbarriers
+  const int bw = wpc + 2;
+  uint32_t o = 8 * (2 * NSMAX + 2);  // mbarriers
   o = up16(o);
   pl.o_misc = o;       o = up16(o + 16);
   pl.o_xf = o;         o = up16(o + 4u * d);
@@ -1429,7 +1505,6 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.o_bsum = o;       o = up16(o + (q4 ? 4u * (d / 32) : 0u));
   pl.o_u = o;          o = up16(o + 4u * r);
   pl.o_bw = o;         o = up16(o + 4u * bw);
-  pl.o_mw = o;         o = up16(o + 4u * Wc);
   pl.o_scan = o;       o = up16(o + 4u * (NCW + 4));
   pl.o_items = o;      o = up16(o + 4u * pl.maxi);
   pl.o_hval = o;       o = up16(o + 4u * pl.maxi);
@@ -1460,7 +1535,7 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
     // chunks per consumer thread in the down phase must fit its accumulators
     // (one Q4_0 block, or 48 fp16 / fp32 values)
     const int cc = L0.w_dtype == PI_Q4_0 ? 32 : (L0.w_dtype == PI_F16 ? 8 : 4);
-    const int cap = cc == 32 ? 1 : 48 / cc;
+    const int cap = cc == 32 ? kQ4Blocks : (two ? 32 : 48) / cc;
     const int per2 = (d / cc + NCT / 2 - 1) / (NCT / 2);
     const int per1 = (d / cc + NCT - 1) / NCT;
     if (ns % 2 == 0 && per2 <= cap) pl.gd = 2;
@@ -1597,10 +1672,12 @@ cudaError_t launch_stack1(const pi_layer* layers, int n_layers, float* x, uint32
   P.part = reinterpret_cast<float*>((char*)ws + lay.part);
   P.count = reinterpret_cast<int32_t*>((char*)ws + lay.count);
   P.idx = reinterpret_cast<int32_t*>((char*)ws + lay.idx);
+  P.cta_counts = reinterpret_cast<uint32_t*>((char*)ws + lay.cta);
   P.hdr = hdr;
   P.trace = trace;
   P.utrace = utrace;
   P.n_layers = n_layers;
+  P.mask_words = words;
   if (mask_trace) {
     P.mask = mask_trace;
     P.mask_stride = words;
@@ -1624,6 +1701,7 @@ cudaError_t launch_stack1(const pi_layer* layers, int n_layers, float* x, uint32
     p.pbias = L.p_bias;
   }
   cudaError_t e = cudaMemsetAsync(hdr->counters, 0, 2 * sizeof(uint32_t), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(P.cta_counts, 0, sizeof(uint32_t) * (size_t)nsms, s);
   if (e != cudaSuccess) return e;
   return launch_any(P, a.w_dtype, a.act, a.p_dtype, s);
 }
