@@ -5,31 +5,41 @@
 // row the CTA will use through a ring of shared-memory stages with 1-D bulk
 // copies (cp.async.bulk, completion counted on an mbarrier per stage; each
 // copy costs its thread a few hundred ns to issue, so the copies of
-// consecutive stages are issued by different threads), a compaction warp,
-// and sixteen consumer warps in groups: a unit (stage) goes to one group,
-// whose threads each take a slice of its columns, so a stage is held only
-// briefly and the ring keeps many rows in flight.  Per layer:
+// consecutive stages are issued by different threads), a list warp, and
+// sixteen consumer warps in groups: a unit (stage) goes to one group, whose
+// threads each take a slice of its columns, so a stage is held only briefly
+// and the ring keeps many rows in flight.  Per layer:
 //
 //   x^  : every CTA normalises the full residual vector (rmsnorm) itself
 //   A   : predictor rows of P1 (a static share per CTA)   -> u      | grid barrier 1
-//   B   : predictor rows of P2 for the CTA's mask words   -> mask   | grid barrier 2 (arrive)
-//   C   : the CTA's hot neurons (j = s, s + SMs, ...)      -> h
-//         meanwhile the compaction warp waits for grid barrier 2 and builds
-//         the CTA's share of the ascending cold list (positions s, s + SMs, ...);
-//         then the cold neurons                            -> h
-//   D   : down rows of the CTA's neurons whose h != 0     -> partial y | grid barrier 3
+//   B   : predictor rows of P2 for the CTA's mask words (words s, s + SMs, ...
+//         of the cold range) -> mask words; the CTA lists the predicted cold
+//         neurons of its own words at once (no grid barrier)
+//   C   : first matrix (W_gate for ReGLU, W_up otherwise) of the CTA's hot
+//         neurons (j = s, s + SMs, ... in groups of adjacent neurons), then
+//         of its cold neurons; each unit is finalised as soon as it is
+//         consumed: the neuron's first pre-activation + bias and its flag
+//   D   : ReLU / squared ReLU: down rows of the neurons whose h != 0.
+//         ReGLU (second-level sparsity): [W_up | W_down^T] of the neurons
+//         whose gate fired, read only for those; two up groups of consumer
+//         warps form the W_up dots and h = gate * up of alternate units while
+//         a down group accumulates h times the down rows of the unit before
+//                                                          -> partial y | grid barrier 3
 //   E   : fixed-order reduction of the CTA's column slice, residual add | grid barrier 4
 //
 // The producers run ahead across phases for every row whose address does
 // not depend on this layer's data (P1, P2, hot rows, the next layer's rows);
-// only cold rows wait for the compaction and down rows for their h.  (L2
-// prefetching of the static rows ahead of the ring, by bulk or per-line
-// prefetches, measured slower at every distance tried, 256 KB to 1 MB per
-// CTA, and is not used.)  Every wait (mbarrier, grid barrier, flag) is
-// bounded by %globaltimer; a wait that runs out sets
-// DEV_TIMEOUT and an abort flag, after which every thread runs the rest of
-// its loops without waiting or computing and the producer waits (bounded)
-// for its own copies in flight before exiting.
+// cold rows wait for the CTA's list and the rows of phase D for their
+// neuron's flag.  (L2 prefetching of the static rows ahead of the ring, by
+// bulk or per-line prefetches, measured slower at every distance tried,
+// 256 KB to 1 MB per CTA, and is not used.)  The kernel is bound by latency
+// more than by issue: its instruction footprint counts (instruction-fetch
+// stalls), so the timeline instrumentation is a separate instantiation and
+// the per-unit loops are unrolled only as far as a unit's records go.
+// Every wait (mbarrier, grid barrier, flag) is bounded by %globaltimer; a
+// wait that runs out sets DEV_TIMEOUT and an abort flag, after which every
+// thread runs the rest of its loops without waiting or computing and the
+// producer waits (bounded) for its own copies in flight before exiting.
 //
 // Q4_0 gate/up dot products are exact integer sums: the normalised input is
 // rounded once per layer to int16 on a per-vector scale, each block's
@@ -54,6 +64,8 @@ constexpr int MAXA = 16;            // P1 rows per CTA at most
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int UTR = 512;            // units per layer recorded by the unit trace
 constexpr int DRMAX = 16;           // D records per unit at most
+constexpr int HQ = 32;              // ReGLU down-phase unit flags (a ring, >= ring depth)
+constexpr int kMaxRec = 4;          // first records per C unit at most
 constexpr int DR2MAX = 4;           // D records per unit at most, ReGLU (W_up dot partials)
 constexpr int kQ4Blocks = 1;        // Q4_0 blocks per thread in phase D
 
@@ -98,7 +110,7 @@ struct Plan {
   uint32_t first_b;                 // a first record in a stage
   uint32_t d2_bytes, o_d2_down;     // a D record in a stage; offset of its down row
   uint32_t o_misc, o_xf, o_xi, o_bsum, o_u, o_bw, o_scan, o_items, o_hval, o_flag,
-      o_dlist, o_pbs, o_hbs, o_redA, o_redC, o_redD, o_redE, o_ring, total;
+      o_dlist, o_pbs, o_hbs, o_redA, o_redC, o_redD, o_hflag, o_redE, o_ring, total;
 };
 
 struct StackParams {
@@ -305,6 +317,7 @@ struct Smem {
   int* items;                 // neuron of each item: hot items, then this layer's cold list
   float* hval;
   volatile int* flag;
+  volatile int* hflag;        // [HQ] ReGLU down phase: unit q's h is ready (tag | q + 1)
   int* dlist;
   float* pbs;                 // predictor biases of the CTA's mask words
   float* hbs;                 // activation biases of the CTA's items
@@ -334,6 +347,7 @@ __device__ __forceinline__ Smem carve(unsigned char* base, const Plan& pl) {
   S.items = reinterpret_cast<int*>(base + pl.o_items);
   S.hval = reinterpret_cast<float*>(base + pl.o_hval);
   S.flag = reinterpret_cast<volatile int*>(base + pl.o_flag);
+  S.hflag = reinterpret_cast<volatile int*>(base + pl.o_hflag);
   S.dlist = reinterpret_cast<int*>(base + pl.o_dlist);
   S.pbs = reinterpret_cast<float*>(base + pl.o_pbs);
   S.hbs = reinterpret_cast<float*>(base + pl.o_hbs);
@@ -398,17 +412,23 @@ __device__ __forceinline__ uint32_t* layer_mask(const StackParams& P, int l) {
 }
 
 // Timeline stamp, when a trace buffer is given.
+template <bool TR>
 __device__ __forceinline__ void tstamp(const StackParams& P, int l, int slot,
                                        unsigned long long v) {
-  if (P.trace) P.trace[((size_t)l * gridDim.x + blockIdx.x) * 16 + slot] = v;
+  if constexpr (TR) {
+    if (TR && P.trace) P.trace[((size_t)l * gridDim.x + blockIdx.x) * 16 + slot] = v;
+  }
 }
 
 // Unit trace of CTA 0 (slot 0 armed, 1 data seen by consumer warp 0,
 // 2 released by consumer warp 0, 3 bytes).
+template <bool TR>
 __device__ __forceinline__ void utstamp(const StackParams& P, int l, uint32_t u, int slot,
                                         unsigned long long v) {
-  if (P.utrace && blockIdx.x == 0 && u < (uint32_t)UTR)
-    P.utrace[((size_t)l * UTR + u) * 4 + slot] = v;
+  if constexpr (TR) {
+    if (P.utrace && blockIdx.x == 0 && u < (uint32_t)UTR)
+      P.utrace[((size_t)l * UTR + u) * 4 + slot] = v;
+  }
 }
 
 // ------------------------------------------------------------ per-CTA shares
@@ -468,7 +488,7 @@ struct Cursor {
 
 // ---------------------------------------------------------------- producer
 
-template <int WT, int ACT, int PT>
+template <int WT, int ACT, int PT, bool TR>
 __device__ void producer(const StackParams& P, const Smem& S, const int p) {
   const Plan& pl = P.pl;
   WsHeader* hdr = P.hdr;
@@ -489,18 +509,18 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
     const int st = cu.st;
     const uint32_t k = cu.gen;
     if (k > 0 && !mbar_try(&S.empty[st], (k - 1) & 1u)) {
-      const unsigned long long t0 = P.trace ? gtime() : 0ull;
+      const unsigned long long t0 = (TR && P.trace) ? gtime() : 0ull;
       if (!wait_mbar(&S.empty[st], (k - 1) & 1u, S, hdr)) {
         ok = false;
         return nullptr;
       }
-      if (P.trace) w_empty += gtime() - t0;
+      if (TR && P.trace) w_empty += gtime() - t0;
     }
     mbar_arrive_tx(&S.full[st], bytes);
     last[st] = k;
-    if (P.utrace) {
-      utstamp(P, cur_l, cu.uc - l_uc0, 0, gtime());
-      utstamp(P, cur_l, cu.uc - l_uc0, 3, bytes);
+    if (TR && P.utrace) {
+      utstamp<TR>(P, cur_l, cu.uc - l_uc0, 0, gtime());
+      utstamp<TR>(P, cur_l, cu.uc - l_uc0, 3, bytes);
     }
     return S.ring + (size_t)st * pl.sb;
   };
@@ -599,9 +619,9 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       firsts(L, nullptr, j0, min(pl.hp, pl.H - j0));
     }
     {
-      const unsigned long long t0 = P.trace ? gtime() : 0ull;
+      const unsigned long long t0 = (TR && P.trace) ? gtime() : 0ull;
       if (!ok || !wait_mbar(S.listbar, (uint32_t)l & 1u, S, hdr)) break;
-      if (P.trace) w_list += gtime() - t0;
+      if (TR && P.trace) w_list += gtime() - t0;
     }
     const int nc = *S.nc;
     for (int i = 0; i < nc && ok; i += pl.cp) firsts(L, S.items + R.nh + i, 0, min(pl.cp, nc - i));
@@ -618,7 +638,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
           if (gtime() - t0 > kTimeoutNs) { raise_abort(S, hdr); ok = false; break; }
           __nanosleep(128);
         }
-        if (P.trace) w_flag += gtime() - t0;
+        if (TR && P.trace) w_flag += gtime() - t0;
         if (!ok) break;
       }
       if ((f & 3) != 2) continue;
@@ -629,11 +649,11 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       }
     }
     if (ok && un > 0) d2s(L, uj, un);
-    if (P.trace && p == 0) {
-      tstamp(P, l, 12, w_empty);
-      tstamp(P, l, 13, w_list);
-      tstamp(P, l, 14, w_flag);
-      tstamp(P, l, 15, gtime());
+    if (TR && P.trace && p == 0) {
+      tstamp<TR>(P, l, 12, w_empty);
+      tstamp<TR>(P, l, 13, w_list);
+      tstamp<TR>(P, l, 14, w_flag);
+      tstamp<TR>(P, l, 15, gtime());
       w_empty = w_list = w_flag = 0;
     }
   }
@@ -661,7 +681,7 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
 // writes its length).  The computation never reads this list; it is there
 // for inspection (pi_read_list).  A wait that gives up leaves the list
 // incomplete and records the timeout.
-template <int WT, int ACT, int PT>
+template <int WT, int ACT, int PT, bool TR>
 __device__ void list_writer(const StackParams& P, const Smem& S) {
   const Plan& pl = P.pl;
   WsHeader* hdr = P.hdr;
@@ -713,7 +733,7 @@ __device__ void list_writer(const StackParams& P, const Smem& S) {
 
 // ---------------------------------------------------------------- consumers
 
-template <int WT, int ACT, int PT>
+template <int WT, int ACT, int PT, bool TR>
 __device__ void consumers(const StackParams& P, const Smem& S) {
   constexpr bool two = (ACT == PI_REGLU);
   const Plan& pl = P.pl;
@@ -740,7 +760,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
   // the current unit's data has landed (false on abort / timeout)
   auto ready = [&]() -> bool {
     const bool ok = wait_mbar(&S.full[cu.st], cu.gen & 1u, S, hdr);
-    if (P.utrace && tid == 0) utstamp(P, cur_l, cu.uc - l_uc0, 1, gtime());
+    if (TR && P.utrace && tid == 0) utstamp<TR>(P, cur_l, cu.uc - l_uc0, 1, gtime());
     return __all_sync(0xffffffffu, ok);
   };
   auto stage = [&]() { return S.ring + (size_t)cu.st * pl.sb; };
@@ -748,7 +768,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
   auto release = [&](int warps) {
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.empty[cu.st], (uint32_t)(NCW / warps));
-    if (P.utrace && tid == 0) utstamp(P, cur_l, cu.uc - l_uc0, 2, gtime());
+    if (TR && P.utrace && tid == 0) utstamp<TR>(P, cur_l, cu.uc - l_uc0, 2, gtime());
   };
   auto gsync_arrive = [&]() {
     csync();
@@ -771,7 +791,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     // chunks c = tid, tid + NCT, ... (all loads issued at once); one CTA-wide
     // reduction gives sum(x^2) and max|x|; 16-byte stores of x^ (and of its
     // int16 copy) are conflict-free
-    if (tid == 0) tstamp(P, l, 0, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 0, gtime());
     {
       constexpr int MC = 3;  // chunks per thread, d <= 12288
       const int nc8 = d / 8;
@@ -854,7 +874,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       }
       csync();
     }
-    if (tid == 0) tstamp(P, l, 1, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 1, gtime());
 
     // ---- A: u = P1 xh; each row shared by one warp group
     const int nA = R.kA1 - R.kA0;
@@ -886,7 +906,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         __stcg(P.u + R.kA0 + a, v);
       }
     }
-    if (tid == 0) tstamp(P, l, 2, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 2, gtime());
     gsync_arrive();  // 1: u complete
     // biases used later in this layer: their load latency overlaps the barrier
     for (int k = tid; k < R.nw * 32; k += NCT) {
@@ -895,7 +915,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     }
     for (int i = tid; i < R.nh; i += NCT) S.hbs[i] = L.bias ? L.bias[S.items[i]] : 0.f;
     gsync_wait();
-    if (tid == 0) tstamp(P, l, 3, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 3, gtime());
 
     // ---- B: logits of the CTA's mask words; the group's warps take the rows
     for (int k = tid; k < pl.r; k += NCT) S.us[vpos<PT>(k, pl.r)] = __ldcg(P.u + k);
@@ -918,7 +938,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
             const char* row = buf + (size_t)(j - ja) * pl.p2_row;
             const char* row2 = row + (size_t)WPG * pl.p2_row;
             float z0 = 0.f, z1 = 0.f;
-#pragma unroll 4
+#pragma unroll 2
             for (int c = lane; c < nch; c += 32) {
               const VFrag uf = vfrag<PT>(S.us, c, pl.r);
               z0 += frag_dot<PT>(lds128(row + (size_t)c * 16), uf);
@@ -978,7 +998,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       __syncwarp();
       if (lane == 0) mbar_arrive(S.listbar, 1u);  // releases the list to the producers
     }
-    if (tid == 0) tstamp(P, l, 4, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 4, gtime());
     csync();
     const int nc = *S.nc;
 
@@ -991,9 +1011,9 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     auto unit_items = [&](int i0, int n) {
       if ((int)(cu.uc & gwm) == grp) {
         const bool ok = ready();
-        float a[8];
+        float a[kMaxRec];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) a[r] = 0.f;
+        for (int r = 0; r < kMaxRec; ++r) a[r] = 0.f;
         if (ok) {
           const char* base = stage();
           if constexpr (WT == PI_Q4_0) {
@@ -1004,7 +1024,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
                                   x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
               const int bs = -8 * S.bsum[k];
 #pragma unroll
-              for (int r = 0; r < 8; ++r) {
+              for (int r = 0; r < kMaxRec; ++r) {
                 if (r >= n) break;
                 const char* buf = base + (size_t)r * pl.first_b;
                 const uint4 cf = lds128(buf + (size_t)k * 16);
@@ -1017,7 +1037,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
             const int nch = d / CCW;
             for (int c = gtid; c < nch; c += GT) {
 #pragma unroll
-              for (int r = 0; r < 8; ++r) {
+              for (int r = 0; r < kMaxRec; ++r) {
                 if (r >= n) break;
                 a[r] += chunk_dot<WT>(lds128(base + (size_t)r * pl.first_b + (size_t)c * 16), S.xf,
                                       c, d);
@@ -1027,14 +1047,14 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
           release(WPG);
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
+        for (int r = 0; r < kMaxRec; ++r) {
           if (r >= n) break;
           a[r] = warp_sum(a[r]);
         }
-        float* rc = S.redC + (size_t)((grp * 2 + (gk & 1)) * 8) * WPG;
+        float* rc = S.redC + (size_t)((grp * 2 + (gk & 1)) * kMaxRec) * WPG;
         if (lane == 0) {
 #pragma unroll
-          for (int r = 0; r < 8; ++r) {
+          for (int r = 0; r < kMaxRec; ++r) {
             if (r >= n) break;
             rc[r * WPG + wg] = a[r];
           }
@@ -1064,15 +1084,15 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       const int j0 = hot_group_first(gi, pl);
       unit_items(gi * pl.hp, min(pl.hp, pl.H - j0));
     }
-    if (tid == 0) tstamp(P, l, 5, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 5, gtime());
 
     // ---- then the CTA's cold neurons (nc was read after the barrier that
     // follows the list, so every warp of a group walks the same units and
     // reaches its group barrier the same number of times)
-    if (tid == 0) tstamp(P, l, 6, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 6, gtime());
     for (int i = 0; i < nc; i += pl.cp) unit_items(R.nh + i, min(pl.cp, nc - i));
     csync();
-    if (tid == 0) tstamp(P, l, 7, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 7, gtime());
 
     // ---- D: D records of the items whose first pre-activation is positive
     // (hval != 0), pl.dr per unit, each unit shared by one of GD warp
@@ -1106,209 +1126,387 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       if constexpr (WT == PI_Q4_0) u *= *S.xscale;
       return g * u;
     };
-    if constexpr (WT == PI_Q4_0) {
-      // QB Q4_0 blocks (32 columns each) per thread (the plan keeps d / 32
-      // within a group's QB * DT).  sum_j hs_j (q - 8), hs_j = h_j * scale,
-      // is accumulated as sum_j 16 hs_j (1 + q/16) with packed fp32x2 FMAs on
-      // floats built from the nibbles by byte permutes, minus 24 sum_j hs_j
-      // at the end.
-      constexpr int QB = kQ4Blocks;
-      const int nch = d / 32;
-      float2 acc[QB][16];
-      float corr[QB];
-#pragma unroll
-      for (int kb = 0; kb < QB; ++kb) {
-        corr[kb] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[kb][e] = make_float2(0.f, 0.f);
-      }
-      for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
-        if ((int)(cu.uc & gdm) != dgrp) continue;
-        const bool ok = ready();
-        const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
-        float* pu = S.redD + (size_t)((dgrp * 2 + (dk & 1)) * DR2MAX) * WPD;
-        if constexpr (two) {
-          // W_up dots of the unit's records
-          for (int rr = 0; rr < len; ++rr) {
-            float a = 0.f;
-            if (ok) {
-              const char* row = stage() + (size_t)rr * pl.d2_bytes;
-              const int4* xb = reinterpret_cast<const int4*>(S.xi);
-              for (int c = dtid; c < nch; c += DT) {
-                const int4 x0 = xb[c], x1 = xb[nch + c], x2 = xb[2 * nch + c], x3 = xb[3 * nch + c];
-                const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
-                                    x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-                a = fmaf((float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]),
-                         h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]), a);
-              }
-            }
-            a = warp_sum(a);
-            if (lane == 0) pu[rr * WPD + wd] = a;
-          }
-          asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
+    if constexpr (!two) {
+      if constexpr (WT == PI_Q4_0) {
+        // QB Q4_0 blocks (32 columns each) per thread (the plan keeps d / 32
+        // within a group's QB * DT).  sum_j hs_j (q - 8), hs_j = h_j * scale,
+        // is accumulated as sum_j 16 hs_j (1 + q/16) with packed fp32x2 FMAs on
+        // floats built from the nibbles by byte permutes, minus 24 sum_j hs_j
+        // at the end.
+        constexpr int QB = kQ4Blocks;
+        const int nch = d / 32;
+        float2 acc[QB][16];
+        float corr[QB];
+  #pragma unroll
+        for (int kb = 0; kb < QB; ++kb) {
+          corr[kb] = 0.f;
+  #pragma unroll
+          for (int e = 0; e < 16; ++e) acc[kb][e] = make_float2(0.f, 0.f);
         }
-        if (ok) {
-#pragma unroll 2
-          for (int rr = 0; rr < len; ++rr) {
-            const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
-            const float hv = unit_h(q0, len, pu, rr);
-#pragma unroll
-            for (int kb = 0; kb < QB; ++kb) {
-              const int c = dtid + kb * DT;
-              if (c >= nch) break;
-              const uint4 v = lds128(row + (size_t)c * 16);
-              const float hs = hv * h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
-              corr[kb] += hs;
-              const float2 h2 = make_float2(16.f * hs, 16.f * hs);
-              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int m = 0; m < 4; ++m) {
-                // byte b: 0x80 | q << 3 for element 4m + b (low nibbles) / 16 + 4m + b (high)
-                const uint32_t lo = ((wv[m] << 3) & 0x78787878u) | 0x80808080u;
-                const uint32_t hi = ((wv[m] >> 1) & 0x78787878u) | 0x80808080u;
-#pragma unroll
-                for (int b = 0; b < 4; b += 2) {
-                  acc[kb][(4 * m + b) >> 1] =
-                      __ffma2_rn(nib_pair(lo, b), h2, acc[kb][(4 * m + b) >> 1]);
-                  acc[kb][(16 + 4 * m + b) >> 1] =
-                      __ffma2_rn(nib_pair(hi, b), h2, acc[kb][(16 + 4 * m + b) >> 1]);
+        for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+          if ((int)(cu.uc & gdm) != dgrp) continue;
+          const bool ok = ready();
+          const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
+          float* pu = S.redD + (size_t)((dgrp * 2 + (dk & 1)) * DR2MAX) * WPD;
+          if constexpr (two) {
+            // W_up dots of the unit's records
+            for (int rr = 0; rr < len; ++rr) {
+              float a = 0.f;
+              if (ok) {
+                const char* row = stage() + (size_t)rr * pl.d2_bytes;
+                const int4* xb = reinterpret_cast<const int4*>(S.xi);
+                for (int c = dtid; c < nch; c += DT) {
+                  const int4 x0 = xb[c], x1 = xb[nch + c], x2 = xb[2 * nch + c], x3 = xb[3 * nch + c];
+                  const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                      x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+                  a = fmaf((float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]),
+                           h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]), a);
+                }
+              }
+              a = warp_sum(a);
+              if (lane == 0) pu[rr * WPD + wd] = a;
+            }
+            asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
+          }
+          if (ok) {
+  #pragma unroll 1
+            for (int rr = 0; rr < len; ++rr) {
+              const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
+              const float hv = unit_h(q0, len, pu, rr);
+  #pragma unroll
+              for (int kb = 0; kb < QB; ++kb) {
+                const int c = dtid + kb * DT;
+                if (c >= nch) break;
+                const uint4 v = lds128(row + (size_t)c * 16);
+                const float hs = hv * h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
+                corr[kb] += hs;
+                const float2 h2 = make_float2(16.f * hs, 16.f * hs);
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+  #pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                  // byte b: 0x80 | q << 3 for element 4m + b (low nibbles) / 16 + 4m + b (high)
+                  const uint32_t lo = ((wv[m] << 3) & 0x78787878u) | 0x80808080u;
+                  const uint32_t hi = ((wv[m] >> 1) & 0x78787878u) | 0x80808080u;
+  #pragma unroll
+                  for (int b = 0; b < 4; b += 2) {
+                    acc[kb][(4 * m + b) >> 1] =
+                        __ffma2_rn(nib_pair(lo, b), h2, acc[kb][(4 * m + b) >> 1]);
+                    acc[kb][(16 + 4 * m + b) >> 1] =
+                        __ffma2_rn(nib_pair(hi, b), h2, acc[kb][(16 + 4 * m + b) >> 1]);
+                  }
                 }
               }
             }
+            release(WPD);
           }
-          release(WPD);
+          ++dk;
         }
-        ++dk;
-      }
-      // the CTA's partial row s: group GD-1 leaves its sums in shared memory
-      // (the fp32 copy of x^, free until the next layer), group 0 adds them
-      // to its own in a fixed order and writes the row
-      float4* xs4 = reinterpret_cast<float4*>(S.xf);
-      csync();
-      if (GD > 1 && dgrp == GD - 1) {
-#pragma unroll
-        for (int kb = 0; kb < QB; ++kb) {
-          const int c = dtid + kb * DT;
-          if (c >= nch) break;
-          const float k24 = 24.f * corr[kb];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2)
-            xs4[c * 8 + e / 2] = make_float4(acc[kb][e].x - k24, acc[kb][e].y - k24,
-                                             acc[kb][e + 1].x - k24, acc[kb][e + 1].y - k24);
+        // the CTA's partial row s: group GD-1 leaves its sums in shared memory
+        // (the fp32 copy of x^, free until the next layer), group 0 adds them
+        // to its own in a fixed order and writes the row
+        float4* xs4 = reinterpret_cast<float4*>(S.xf);
+        csync();
+        if (GD > 1 && dgrp == GD - 1) {
+  #pragma unroll
+          for (int kb = 0; kb < QB; ++kb) {
+            const int c = dtid + kb * DT;
+            if (c >= nch) break;
+            const float k24 = 24.f * corr[kb];
+  #pragma unroll
+            for (int e = 0; e < 16; e += 2)
+              xs4[c * 8 + e / 2] = make_float4(acc[kb][e].x - k24, acc[kb][e].y - k24,
+                                               acc[kb][e + 1].x - k24, acc[kb][e + 1].y - k24);
+          }
         }
-      }
-      csync();
-      if (dgrp == 0) {
-#pragma unroll
-        for (int kb = 0; kb < QB; ++kb) {
-          const int c = dtid + kb * DT;
-          if (c >= nch) break;
-          float* part = P.part + (size_t)s * d + (size_t)c * 32;
-          const float k24 = 24.f * corr[kb];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float4 v = make_float4(acc[kb][e].x - k24, acc[kb][e].y - k24, acc[kb][e + 1].x - k24,
-                                   acc[kb][e + 1].y - k24);
-            if (GD > 1) v = f4add(v, xs4[c * 8 + e / 2]);
-            __stcg(reinterpret_cast<float4*>(part + 2 * e), v);
+        csync();
+        if (dgrp == 0) {
+  #pragma unroll
+          for (int kb = 0; kb < QB; ++kb) {
+            const int c = dtid + kb * DT;
+            if (c >= nch) break;
+            float* part = P.part + (size_t)s * d + (size_t)c * 32;
+            const float k24 = 24.f * corr[kb];
+  #pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+              float4 v = make_float4(acc[kb][e].x - k24, acc[kb][e].y - k24, acc[kb][e + 1].x - k24,
+                                     acc[kb][e + 1].y - k24);
+              if (GD > 1) v = f4add(v, xs4[c * 8 + e / 2]);
+              __stcg(reinterpret_cast<float4*>(part + 2 * e), v);
+            }
+          }
+        }
+      } else {
+        // fp16 / fp32 rows: up to 48 columns per thread (32 for ReGLU, whose
+        // D phase also forms the W_up dots)
+        constexpr int CC = WTraits<WT>::CHUNK_COLS;
+        constexpr int MAXK = (two ? 32 : 48) / CC;  // chunks per thread of a D group
+        const int nch = d / CC;
+        float acc[MAXK][CC];
+  #pragma unroll
+        for (int k = 0; k < MAXK; ++k)
+  #pragma unroll
+          for (int e = 0; e < CC; ++e) acc[k][e] = 0.f;
+        for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+          if ((int)(cu.uc & gdm) != dgrp) continue;
+          const bool ok = ready();
+          const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
+          float* pu = S.redD + (size_t)((dgrp * 2 + (dk & 1)) * DR2MAX) * WPD;
+          if constexpr (two) {
+            for (int rr = 0; rr < len; ++rr) {
+              float a = 0.f;
+              if (ok) {
+                const char* row = stage() + (size_t)rr * pl.d2_bytes;
+                for (int c = dtid; c < nch; c += DT)
+                  a += chunk_dot<WT>(lds128(row + (size_t)c * 16), S.xf, c, d);
+              }
+              a = warp_sum(a);
+              if (lane == 0) pu[rr * WPD + wd] = a;
+            }
+            asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
+          }
+          if (ok) {
+            for (int rr = 0; rr < len; ++rr) {
+              const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
+              const float hv = unit_h(q0, len, pu, rr);
+  #pragma unroll
+              for (int k = 0; k < MAXK; ++k) {
+                const int c = dtid + k * DT;
+                if (c >= nch) break;
+                const uint4 v = lds128(row + (size_t)c * 16);
+                if constexpr (WT == PI_F16) {
+                  float f[8];
+                  f16x8_to_f32(v, f);
+  #pragma unroll
+                  for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(hv, f[e], acc[k][e]);
+                } else {
+                  acc[k][0] = fmaf(hv, __uint_as_float(v.x), acc[k][0]);
+                  acc[k][1] = fmaf(hv, __uint_as_float(v.y), acc[k][1]);
+                  acc[k][2] = fmaf(hv, __uint_as_float(v.z), acc[k][2]);
+                  acc[k][3] = fmaf(hv, __uint_as_float(v.w), acc[k][3]);
+                }
+              }
+            }
+            release(WPD);
+          }
+          ++dk;
+        }
+        // the CTA's partial row s: group GD-1 leaves its sums in shared memory
+        // (the fp32 copy of x^, free until the next layer), group 0 adds them
+        // to its own in a fixed order and writes the row
+        float4* xs4 = reinterpret_cast<float4*>(S.xf);
+        csync();
+        if (GD > 1 && dgrp == GD - 1) {
+  #pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int c = dtid + k * DT;
+            if (c >= nch) break;
+  #pragma unroll
+            for (int e = 0; e < CC; e += 4)
+              xs4[(c * CC + e) / 4] = make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]);
+          }
+        }
+        csync();
+        if (dgrp == 0) {
+          float* part = P.part + (size_t)s * d;
+  #pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int c = dtid + k * DT;
+            if (c >= nch) break;
+  #pragma unroll
+            for (int e = 0; e < CC; e += 4) {
+              float4 v = make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]);
+              if (GD > 1) v = f4add(v, xs4[(c * CC + e) / 4]);
+              __stcg(reinterpret_cast<float4*>(part + c * CC + e), v);
+            }
           }
         }
       }
     } else {
-      // fp16 / fp32 rows: up to 48 columns per thread (32 for ReGLU, whose
-      // D phase also forms the W_up dots)
-      constexpr int CC = WTraits<WT>::CHUNK_COLS;
-      constexpr int MAXK = (two ? 32 : 48) / CC;  // chunks per thread of a D group
-      const int nch = d / CC;
-      float acc[MAXK][CC];
-#pragma unroll
-      for (int k = 0; k < MAXK; ++k)
-#pragma unroll
-        for (int e = 0; e < CC; ++e) acc[k][e] = 0.f;
-      for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
-        if ((int)(cu.uc & gdm) != dgrp) continue;
-        const bool ok = ready();
-        const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
-        float* pu = S.redD + (size_t)((dgrp * 2 + (dk & 1)) * DR2MAX) * WPD;
-        if constexpr (two) {
+      // ReGLU: a two-role pipeline over the D units ([W_up | W_down^T]
+      // records of the items whose gate fired, pl.dr per unit).  Warps
+      // 0 .. NCW/2-1 form two up groups; group q & 1 forms unit q's W_up dots
+      // (per-warp partials combined in fixed order after a named barrier),
+      // h = gate * up for its records, and raises the unit's flag.  Warps
+      // NCW/2 .. NCW-1 take every unit in order once its flag is up and
+      // accumulate h times the down rows over all columns (one partial row
+      // per CTA).  The two roles work on consecutive units at once.
+      constexpr int UW = NCW / 4;              // warps per up group
+      constexpr int UT = UW * 32, VT = NCT / 2;
+      const bool vrole = warp >= NCW / 2;
+      const int ug = warp / UW;                // up group (up role)
+      const int uw = warp % UW, ut = uw * 32 + lane;
+      const int vt = tid - NCT / 2;            // thread of the down role
+      const int ntag = (l + 1) << 16;
+      if (!vrole) {
+        int uk = 0;  // units this up group has taken in this layer
+        for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+          if ((q & 1) != ug) continue;
+          const bool ok = ready();
+          const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
+          float* pu = S.redD + (size_t)((ug * 2 + (uk & 1)) * DR2MAX) * UW;
           for (int rr = 0; rr < len; ++rr) {
             float a = 0.f;
             if (ok) {
               const char* row = stage() + (size_t)rr * pl.d2_bytes;
-              for (int c = dtid; c < nch; c += DT)
-                a += chunk_dot<WT>(lds128(row + (size_t)c * 16), S.xf, c, d);
+              if constexpr (WT == PI_Q4_0) {
+                const int4* xb = reinterpret_cast<const int4*>(S.xi);
+                for (int c = ut; c < nb; c += UT) {
+                  const int4 x0 = xb[c], x1 = xb[nb + c], x2 = xb[2 * nb + c], x3 = xb[3 * nb + c];
+                  const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                      x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+                  a = fmaf((float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]),
+                           h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]), a);
+                }
+              } else {
+                constexpr int CCW = WTraits<WT>::CHUNK_COLS;
+                for (int c = ut; c < d / CCW; c += UT)
+                  a += chunk_dot<WT>(lds128(row + (size_t)c * 16), S.xf, c, d);
+              }
             }
             a = warp_sum(a);
-            if (lane == 0) pu[rr * WPD + wd] = a;
+            if (lane == 0) pu[rr * UW + uw] = a;
           }
-          asm volatile("bar.sync %0, %1;" ::"r"(6 + dgrp), "r"(DT) : "memory");
+          // every warp of the up group reaches this barrier for every unit it owns
+          asm volatile("bar.sync %0, %1;" ::"r"(2 + ug), "r"(UT) : "memory");
+          if (uw == 0) {
+            if (lane < len) {
+              float u = 0.f;
+              for (int w = 0; w < UW; ++w) u += pu[lane * UW + w];
+              if constexpr (WT == PI_Q4_0) u *= *S.xscale;
+              const int i = S.dlist[q0 + lane];
+              S.hval[i] = S.hval[i] * u;  // gate (after its ReLU) * up
+            }
+            __syncwarp();
+            __threadfence_block();
+            if (lane == 0) S.hflag[q & (HQ - 1)] = ntag | (q + 1);
+          }
+          if (ok) release(NCW / 2);
+          ++uk;
         }
-        if (ok) {
-          for (int rr = 0; rr < len; ++rr) {
-            const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
-            const float hv = unit_h(q0, len, pu, rr);
-#pragma unroll
-            for (int k = 0; k < MAXK; ++k) {
-              const int c = dtid + k * DT;
-              if (c >= nch) break;
-              const uint4 v = lds128(row + (size_t)c * 16);
-              if constexpr (WT == PI_F16) {
-                float f[8];
-                f16x8_to_f32(v, f);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(hv, f[e], acc[k][e]);
-              } else {
-                acc[k][0] = fmaf(hv, __uint_as_float(v.x), acc[k][0]);
-                acc[k][1] = fmaf(hv, __uint_as_float(v.y), acc[k][1]);
-                acc[k][2] = fmaf(hv, __uint_as_float(v.z), acc[k][2]);
-                acc[k][3] = fmaf(hv, __uint_as_float(v.w), acc[k][3]);
+      } else {
+        // the unit's flag, by one lane per warp (bounded)
+        auto hready = [&](int q) -> bool {
+          int okf = 1;
+          if (lane == 0) {
+            const int want = ntag | (q + 1);
+            if (S.hflag[q & (HQ - 1)] != want) {
+              const uint64_t t0 = gtime();
+              while (S.hflag[q & (HQ - 1)] != want) {
+                if (*S.abort) { okf = 0; break; }
+                if (gtime() - t0 > kTimeoutNs) { raise_abort(S, hdr); okf = 0; break; }
+                __nanosleep(32);
               }
             }
           }
-          release(WPD);
-        }
-        ++dk;
-      }
-      // the CTA's partial row s: group GD-1 leaves its sums in shared memory
-      // (the fp32 copy of x^, free until the next layer), group 0 adds them
-      // to its own in a fixed order and writes the row
-      float4* xs4 = reinterpret_cast<float4*>(S.xf);
-      csync();
-      if (GD > 1 && dgrp == GD - 1) {
-#pragma unroll
-        for (int k = 0; k < MAXK; ++k) {
-          const int c = dtid + k * DT;
-          if (c >= nch) break;
-#pragma unroll
-          for (int e = 0; e < CC; e += 4)
-            xs4[(c * CC + e) / 4] = make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]);
-        }
-      }
-      csync();
-      if (dgrp == 0) {
+          __syncwarp();
+          return __shfl_sync(0xffffffffu, okf, 0) != 0;
+        };
         float* part = P.part + (size_t)s * d;
+        if constexpr (WT == PI_Q4_0) {
+          // one Q4_0 block (32 columns) per thread, accumulated as in the
+          // ReLU branch above
+          const int nch = d / 32, c = vt;
+          float2 acc[16];
 #pragma unroll
-        for (int k = 0; k < MAXK; ++k) {
-          const int c = dtid + k * DT;
-          if (c >= nch) break;
+          for (int e = 0; e < 16; ++e) acc[e] = make_float2(0.f, 0.f);
+          float corr = 0.f;
+          for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+            const bool ok = ready();
+            const bool hk = hready(q);
+            const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
+            if (ok && hk && c < nch) {
+#pragma unroll 1
+              for (int rr = 0; rr < len; ++rr) {
+                const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
+                const uint4 v = lds128(row + (size_t)c * 16);
+                const float hs = S.hval[S.dlist[q0 + rr]] *
+                                 h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]);
+                corr += hs;
+                const float2 h2 = make_float2(16.f * hs, 16.f * hs);
+                const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < CC; e += 4) {
-            float4 v = make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]);
-            if (GD > 1) v = f4add(v, xs4[(c * CC + e) / 4]);
-            __stcg(reinterpret_cast<float4*>(part + c * CC + e), v);
+                for (int m = 0; m < 4; ++m) {
+                  const uint32_t lo = ((wv[m] << 3) & 0x78787878u) | 0x80808080u;
+                  const uint32_t hi = ((wv[m] >> 1) & 0x78787878u) | 0x80808080u;
+#pragma unroll
+                  for (int b2 = 0; b2 < 4; b2 += 2) {
+                    acc[(4 * m + b2) >> 1] = __ffma2_rn(nib_pair(lo, b2), h2, acc[(4 * m + b2) >> 1]);
+                    acc[(16 + 4 * m + b2) >> 1] =
+                        __ffma2_rn(nib_pair(hi, b2), h2, acc[(16 + 4 * m + b2) >> 1]);
+                  }
+                }
+              }
+            }
+            if (ok) release(NCW);
+          }
+          if (c < nch) {
+            const float k24 = 24.f * corr;
+#pragma unroll
+            for (int e = 0; e < 16; e += 2)
+              __stcg(reinterpret_cast<float4*>(part + (size_t)c * 32 + 2 * e),
+                     make_float4(acc[e].x - k24, acc[e].y - k24, acc[e + 1].x - k24,
+                                 acc[e + 1].y - k24));
+          }
+        } else {
+          constexpr int CC = WTraits<WT>::CHUNK_COLS;
+          constexpr int MAXK = 48 / CC;
+          const int nch = d / CC;
+          float acc[MAXK][CC];
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k)
+#pragma unroll
+            for (int e = 0; e < CC; ++e) acc[k][e] = 0.f;
+          for (int q = 0; q < nruns; ++q, cu.next(pl.ns)) {
+            const bool ok = ready();
+            const bool hk = hready(q);
+            const int q0 = q * pl.dr, len = min(pl.dr, nd - q0);
+            if (ok && hk) {
+              for (int rr = 0; rr < len; ++rr) {
+                const char* row = stage() + (size_t)rr * pl.d2_bytes + pl.o_d2_down;
+                const float hv = S.hval[S.dlist[q0 + rr]];
+#pragma unroll
+                for (int k = 0; k < MAXK; ++k) {
+                  const int c = vt + k * VT;
+                  if (c >= nch) break;
+                  const uint4 v = lds128(row + (size_t)c * 16);
+                  if constexpr (WT == PI_F16) {
+                    float f[8];
+                    f16x8_to_f32(v, f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(hv, f[e], acc[k][e]);
+                  } else {
+                    acc[k][0] = fmaf(hv, __uint_as_float(v.x), acc[k][0]);
+                    acc[k][1] = fmaf(hv, __uint_as_float(v.y), acc[k][1]);
+                    acc[k][2] = fmaf(hv, __uint_as_float(v.z), acc[k][2]);
+                    acc[k][3] = fmaf(hv, __uint_as_float(v.w), acc[k][3]);
+                  }
+                }
+              }
+            }
+            if (ok) release(NCW);
+          }
+#pragma unroll
+          for (int k = 0; k < MAXK; ++k) {
+            const int c = vt + k * VT;
+            if (c >= nch) break;
+#pragma unroll
+            for (int e = 0; e < CC; e += 4)
+              __stcg(reinterpret_cast<float4*>(part + c * CC + e),
+                     make_float4(acc[k][e], acc[k][e + 1], acc[k][e + 2], acc[k][e + 3]));
           }
         }
       }
+      csync();
     }
     if (tid == 0) {
       atomicAdd(&hdr->rows_listed, (unsigned long long)ni);
       if constexpr (two) atomicAdd(&hdr->rows_second, (unsigned long long)nd);
       atomicAdd(&hdr->rows_down, (unsigned long long)nd);
-      tstamp(P, l, 8, gtime());
+      tstamp<TR>(P, l, 8, gtime());
     }
     gsync_arrive();  // 3: partials complete
     gsync_wait();
-    if (tid == 0) tstamp(P, l, 9, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 9, gtime());
 
     // ---- E: reduce this CTA's float4 column slice over the nS partial rows
     // in a fixed order (rows in interleaved groups, then the groups in
@@ -1323,7 +1521,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       const float4 xo = tid < nq ? __ldcg(x4) : make_float4(0.f, 0.f, 0.f, 0.f);
       if (nq > 0 && tid < nq * g) {
         // rows gi, gi + g, ... summed in that order; 12 loads in flight
-        constexpr int ER = 12;
+        constexpr int ER = 8;
         const int q = tid % nq, gi = tid / nq;
         float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int sp0 = gi; sp0 < nP; sp0 += ER * g) {
@@ -1346,16 +1544,16 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       }
     }
     csync();
-    if (tid == 0) tstamp(P, l, 10, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 10, gtime());
     if (l + 1 < P.n_layers) {
       gsync_arrive();  // 4: x complete
       gsync_wait();
     }
-    if (tid == 0) tstamp(P, l, 11, gtime());
+    if (tid == 0) tstamp<TR>(P, l, 11, gtime());
   }
 }
 
-template <int WT, int ACT, int PT>
+template <int WT, int ACT, int PT, bool TR>
 __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ StackParams P) {
   extern __shared__ __align__(128) unsigned char smem[];
   const Smem S = carve(smem, P.pl);
@@ -1370,6 +1568,7 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (int i = threadIdx.x; i < P.pl.maxi; i += NTHR) S.flag[i] = 0;
+  for (int i = threadIdx.x; i < HQ; i += NTHR) S.hflag[i] = 0;
   {
     // the CTA's hot items: groups g = s, s + SMs, ... of hp adjacent neurons
     const Ranges R = ranges(P.pl);
@@ -1380,13 +1579,13 @@ __global__ void __launch_bounds__(NTHR, 1) k_stack1(const __grid_constant__ Stac
   if (threadIdx.x >= NCT) {
     const int p = (threadIdx.x - NCT) >> 5;
     if (p < P.pl.np) {
-      if ((threadIdx.x & 31) == 0) producer<WT, ACT, PT>(P, S, p);
+      if ((threadIdx.x & 31) == 0) producer<WT, ACT, PT, TR>(P, S, p);
     } else if (p == NPMAX) {
-      list_writer<WT, ACT, PT>(P, S);
+      list_writer<WT, ACT, PT, TR>(P, S);
     }
     return;
   }
-  consumers<WT, ACT, PT>(P, S);
+  consumers<WT, ACT, PT, TR>(P, S);
 }
 
 // ------------------------------------------------------------------- host
@@ -1472,9 +1671,10 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
     if (layers[l].w_row_stride != L0.w_row_stride || layers[l].w_down_row_stride != L0.w_down_row_stride ||
         layers[l].w_up_row_stride != L0.w_up_row_stride)
       return false;
-  // first records per hot unit (adjacent neurons): units of at least 16 KB
+  // first records per hot unit (adjacent neurons): units of at least 16 KB,
+  // at most kMaxRec records
   pl.hp = 1;
-  while (pl.hp < 8 && (uint32_t)pl.hp * rec < 16384u) ++pl.hp;
+  while (pl.hp < kMaxRec && (uint32_t)pl.hp * rec < 16384u) ++pl.hp;
   pl.cp = pl.hp;
   uint32_t sb = pl.p1_bytes;
   sb = sb > (uint32_t)pl.hp * rec ? sb : (uint32_t)pl.hp * rec;
@@ -1515,6 +1715,7 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   pl.o_redA = o;       o = up16(o + 4u * (MAXA + MAXA * NCW));
   pl.o_redC = o;       o = up16(o + 4u * (2 * 8 * NCW));
   pl.o_redD = o;       o = up16(o + 4u * (2 * DR2MAX * NCW));
+  pl.o_hflag = o;      o = up16(o + 4u * HQ);
   pl.o_redE = o;       o = up16(o + 16u * NCT);
   pl.o_ring = up128(o);
   const int avail = smem_optin() - (int)pl.o_ring;
@@ -1542,6 +1743,15 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
     else if (per1 <= cap) pl.gd = 1;
     else return false;
   }
+  if (two) {
+    // the ReGLU down phase: its up groups alternate units (an even ring keeps
+    // each stage with one group) and its down group covers every column
+    // with one Q4_0 block or at most 48 fp16 / fp32 values per thread
+    if (ns % 2) return false;
+    const int cc = L0.w_dtype == PI_Q4_0 ? 32 : (L0.w_dtype == PI_F16 ? 8 : 4);
+    const int per = (d / cc + NCT / 2 - 1) / (NCT / 2);
+    if (per > (cc == 32 ? 1 : 48 / cc)) return false;
+  }
   pl.total = pl.o_ring + (uint32_t)ns * sb;
   *out = pl;
   return true;
@@ -1558,7 +1768,9 @@ bool fused_disabled() {
 
 template <int WT, int ACT, int PT>
 cudaError_t launch_t(const StackParams& P, cudaStream_t s) {
-  auto kern = k_stack1<WT, ACT, PT>;
+  // the timeline instrumentation lives in its own instantiation, so the
+  // kernel that normally runs carries none of it
+  auto kern = (P.trace || P.utrace) ? k_stack1<WT, ACT, PT, true> : k_stack1<WT, ACT, PT, false>;
   cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(kern), P.pl.total);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
