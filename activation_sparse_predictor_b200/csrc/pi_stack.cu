@@ -441,6 +441,26 @@ struct Ranges {
   int nh;         // hot neurons in them
 };
 
+// The k-th of CTA s's items dealt round by round over S CTAs, every other
+// round in reverse ("snake"): where the items' expected work falls along
+// the order (the frequency-sorted neurons), every CTA gets the same share.
+__device__ __forceinline__ int snake(int k, int s, int S) {
+  return k * S + ((k & 1) ? S - 1 - s : s);
+}
+
+// The CTA that owns item i of a snake deal over S CTAs.
+__device__ __forceinline__ int snake_owner(int i, int S) {
+  const int k = i / S, p = i - k * S;
+  return (k & 1) ? S - 1 - p : p;
+}
+
+// Items of a snake deal of n items that CTA s owns.
+__device__ __forceinline__ int snake_count(int n, int s, int S) {
+  const int full = n / S, rem = n - full * S;
+  const int pos = (full & 1) ? S - 1 - s : s;
+  return full + (rem > 0 && pos < rem ? 1 : 0);
+}
+
 __device__ __forceinline__ Ranges ranges(const Plan& pl) {
   Ranges R;
   const int S = gridDim.x, s = blockIdx.x;
@@ -449,22 +469,25 @@ __device__ __forceinline__ Ranges ranges(const Plan& pl) {
   R.W = (pl.F + 31) / 32;
   R.Wlo = pl.H / 32;
   const int Wc = R.W - R.Wlo;
-  // interleaved, so that every CTA's words sample the whole cold range
-  // (the predicted density falls along the frequency-sorted order)
-  R.nw = Wc > s ? (Wc - 1 - s) / S + 1 : 0;
+  // the cold mask words Wlo + snake(k): every CTA's words sample the whole
+  // cold range (the predicted density falls along the order)
+  R.nw = snake_count(Wc, s, S);
+  // the hot groups snake(gi) of hp adjacent neurons (the last one shorter)
   const int G = (pl.H + pl.hp - 1) / pl.hp;
-  R.ngh = s < G ? (G - 1 - s) / S + 1 : 0;
-  R.nh = 0;
-  if (R.ngh > 0) {
-    const int gl = s + S * (R.ngh - 1);
-    R.nh = (R.ngh - 1) * pl.hp + min(pl.hp, pl.H - gl * pl.hp);
-  }
+  R.ngh = snake_count(G, s, S);
+  R.nh = R.ngh * pl.hp;
+  if (R.ngh > 0 && snake(R.ngh - 1, s, S) == G - 1) R.nh -= G * pl.hp - pl.H;
   return R;
 }
 
 // First neuron of this CTA's hot group gi.
 __device__ __forceinline__ int hot_group_first(int gi, const Plan& pl) {
-  return ((int)blockIdx.x + (int)gridDim.x * gi) * pl.hp;
+  return snake(gi, (int)blockIdx.x, (int)gridDim.x) * pl.hp;
+}
+
+// This CTA's k-th cold mask word.
+__device__ __forceinline__ int cold_word(int k, const Ranges& R) {
+  return R.Wlo + snake(k, (int)blockIdx.x, (int)gridDim.x);
 }
 
 // Position in the unit sequence: unit number, its stage (uc % ns) and the
@@ -600,7 +623,8 @@ __device__ void producer(const StackParams& P, const Smem& S, const int p) {
       }
     }
     // B: predictor rows of P2, G per unit
-    for (int k = 0, w = R.Wlo + (int)blockIdx.x; k < R.nw && ok; ++k, w += (int)gridDim.x) {
+    for (int k = 0; k < R.nw && ok; ++k) {
+      const int w = cold_word(k, R);
       for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F && ok; ja += pl.G, cu.next(pl.ns)) {
         const int jb = min(ja + pl.G, pl.F);
         const uint32_t bytes = (uint32_t)(jb - ja) * pl.p2_row;
@@ -719,7 +743,7 @@ __device__ void list_writer(const StackParams& P, const Smem& S) {
         const int t = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += t;
       }
-      if (w < R.W && (w - R.Wlo) % nS == s) {
+      if (w < R.W && snake_owner(w - R.Wlo, nS) == s) {
         int pos = base + incl - c;
         for (; m; m &= m - 1u, ++pos) __stcg(P.idx + pos, lo + __ffs(m) - 1);
       }
@@ -910,7 +934,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     gsync_arrive();  // 1: u complete
     // biases used later in this layer: their load latency overlaps the barrier
     for (int k = tid; k < R.nw * 32; k += NCT) {
-      const int j = 32 * (R.Wlo + s + (k >> 5) * nS) + (k & 31);
+      const int j = 32 * cold_word(k >> 5, R) + (k & 31);
       S.pbs[k] = (L.pbias && j < pl.F) ? L.pbias[j] : 0.f;
     }
     for (int i = tid; i < R.nh; i += NCT) S.hbs[i] = L.bias ? L.bias[S.items[i]] : 0.f;
@@ -924,7 +948,8 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     {
       constexpr int CCP = WTraits<PT>::CHUNK_COLS;
       const int nch = pl.r / CCP;
-      for (int kw = 0, w = R.Wlo + s; kw < R.nw; ++kw, w += nS) {
+      for (int kw = 0; kw < R.nw; ++kw) {
+        const int w = cold_word(kw, R);
         for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F; ja += pl.G, cu.next(pl.ns)) {
           if ((int)(cu.uc & gwm) != grp) continue;
           if (!ready()) continue;
@@ -963,7 +988,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     }
     csync();
     for (int k = tid; k < R.nw; k += NCT) {
-      const int w = R.Wlo + s + k * nS;
+      const int w = cold_word(k, R);
       uint32_t word = S.bw[k];
       const int lo = 32 * w;
       if (pl.H > lo) word |= (pl.H - lo >= 32) ? 0xFFFFFFFFu : ((1u << (pl.H - lo)) - 1u);
@@ -990,7 +1015,7 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
       const int total = __shfl_sync(0xffffffffu, incl, 31);
       int pos = R.nh + incl - cnt;
       for (uint32_t m = word; m; m &= m - 1u, ++pos) {
-        const int j = 32 * (R.Wlo + s + lane * nS) + __ffs(m) - 1;
+        const int j = 32 * cold_word(lane, R) + __ffs(m) - 1;
         S.items[pos] = j;
         S.hbs[pos] = L.bias ? L.bias[j] : 0.f;
       }
