@@ -947,7 +947,19 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     csync();
     {
       constexpr int CCP = WTraits<PT>::CHUNK_COLS;
-      const int nch = pl.r / CCP;
+      const int nch = pl.r / CCP;  // <= 32 * MU (plan)
+      // the lane's u chunks, kept in registers for the whole phase
+      constexpr int MU = 4;
+      VFrag ur[MU];
+#pragma unroll
+      for (int m = 0; m < MU; ++m) {
+        const int c = lane + 32 * m;
+        if (c < nch) {
+          ur[m] = vfrag<PT>(S.us, c, pl.r);
+        } else {
+          ur[m].lo = ur[m].hi = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
       for (int kw = 0; kw < R.nw; ++kw) {
         const int w = cold_word(kw, R);
         for (int ja = 32 * w; ja < 32 * w + 32 && ja < pl.F; ja += pl.G, cu.next(pl.ns)) {
@@ -963,11 +975,12 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
             const char* row = buf + (size_t)(j - ja) * pl.p2_row;
             const char* row2 = row + (size_t)WPG * pl.p2_row;
             float z0 = 0.f, z1 = 0.f;
-#pragma unroll 2
-            for (int c = lane; c < nch; c += 32) {
-              const VFrag uf = vfrag<PT>(S.us, c, pl.r);
-              z0 += frag_dot<PT>(lds128(row + (size_t)c * 16), uf);
-              if (pair) z1 += frag_dot<PT>(lds128(row2 + (size_t)c * 16), uf);
+#pragma unroll
+            for (int m = 0; m < MU; ++m) {
+              const int c = lane + 32 * m;
+              if (c >= nch) break;
+              z0 += frag_dot<PT>(lds128(row + (size_t)c * 16), ur[m]);
+              if (pair) z1 += frag_dot<PT>(lds128(row2 + (size_t)c * 16), ur[m]);
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -1033,6 +1046,31 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
     // buffers alternating by the group's unit parity) and the items' flags
     // are set, so the producers can fetch the D records at once.
     int gk = 0;  // units this group has taken in this layer
+    // Q4_0: the thread's int16 x^ blocks (k = gtid + GT m) in registers for
+    // phase C and the ReGLU up groups of phase D (same thread-to-block map)
+    constexpr int MQ = 2;  // d / 32 <= MQ * GT (plan)
+    int xq[MQ][16], bq[MQ];
+#pragma unroll
+    for (int m = 0; m < MQ; ++m) {
+      bq[m] = 0;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) xq[m][e] = 0;
+    }
+    if constexpr (WT == PI_Q4_0) {
+      const int4* xb = reinterpret_cast<const int4*>(S.xi);
+#pragma unroll
+      for (int m = 0; m < MQ; ++m) {
+        const int k = gtid + GT * m;
+        if (k < nb) {
+          const int4 x0 = xb[k], x1 = xb[nb + k], x2 = xb[2 * nb + k], x3 = xb[3 * nb + k];
+          const int v[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                             x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
+#pragma unroll
+          for (int e = 0; e < 16; ++e) xq[m][e] = v[e];
+          bq[m] = -8 * S.bsum[k];
+        }
+      }
+    }
     auto unit_items = [&](int i0, int n) {
       if ((int)(cu.uc & gwm) == grp) {
         const bool ok = ready();
@@ -1042,19 +1080,17 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
         if (ok) {
           const char* base = stage();
           if constexpr (WT == PI_Q4_0) {
-            const int4* xb = reinterpret_cast<const int4*>(S.xi);
-            for (int k = gtid; k < nb; k += GT) {
-              const int4 x0 = xb[k], x1 = xb[nb + k], x2 = xb[2 * nb + k], x3 = xb[3 * nb + k];
-              const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
-                                  x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-              const int bs = -8 * S.bsum[k];
+#pragma unroll
+            for (int m = 0; m < MQ; ++m) {
+              const int k = gtid + GT * m;
+              if (k >= nb) break;
 #pragma unroll
               for (int r = 0; r < kMaxRec; ++r) {
                 if (r >= n) break;
                 const char* buf = base + (size_t)r * pl.first_b;
                 const uint4 cf = lds128(buf + (size_t)k * 16);
                 const float sf = h2f(reinterpret_cast<const uint16_t*>(buf + pl.rowb)[k]);
-                a[r] = fmaf((float)q4_block_dot(cf, xw, bs), sf, a[r]);
+                a[r] = fmaf((float)q4_block_dot(cf, xq[m], bq[m]), sf, a[r]);
               }
             }
           } else {
@@ -1374,12 +1410,12 @@ __device__ void consumers(const StackParams& P, const Smem& S) {
             if (ok) {
               const char* row = stage() + (size_t)rr * pl.d2_bytes;
               if constexpr (WT == PI_Q4_0) {
-                const int4* xb = reinterpret_cast<const int4*>(S.xi);
-                for (int c = ut; c < nb; c += UT) {
-                  const int4 x0 = xb[c], x1 = xb[nb + c], x2 = xb[2 * nb + c], x3 = xb[3 * nb + c];
-                  const int xw[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
-                                      x2.x, x2.y, x2.z, x2.w, x3.x, x3.y, x3.z, x3.w};
-                  a = fmaf((float)q4_block_dot(lds128(row + (size_t)c * 16), xw, -8 * S.bsum[c]),
+                static_assert(UT == NCT / 4, "up-group threads map to the phase-C blocks");
+#pragma unroll
+                for (int m = 0; m < MQ; ++m) {
+                  const int c = ut + UT * m;
+                  if (c >= nb) break;
+                  a = fmaf((float)q4_block_dot(lds128(row + (size_t)c * 16), xq[m], bq[m]),
                            h2f(reinterpret_cast<const uint16_t*>(row + pl.rowb)[c]), a);
                 }
               } else {
@@ -1771,8 +1807,9 @@ bool make_plan(const pi_layer* layers, int n_layers, int nsms, Plan* out) {
   if (two) {
     // the ReGLU down phase: its up groups alternate units (an even ring keeps
     // each stage with one group) and its down group covers every column
-    // with one Q4_0 block or at most 48 fp16 / fp32 values per thread
-    if (ns % 2) return false;
+    // with one Q4_0 block or at most 48 fp16 / fp32 values per thread; its
+    // up groups reuse the phase-C threads' x^ blocks (four groups in C)
+    if (ns % 2 || pl.gw != 4) return false;
     const int cc = L0.w_dtype == PI_Q4_0 ? 32 : (L0.w_dtype == PI_F16 ? 8 : 4);
     const int per = (d / cc + NCT / 2 - 1) / (NCT / 2);
     if (per > (cc == 32 ? 1 : 48 / cc)) return false;
@@ -1874,7 +1911,9 @@ bool stack1_supported(const pi_layer* layers, int n_layers, int batch) {
   // fp16 weights go with an fp16 predictor, fp32 with fp32 (one staged layout)
   if ((a.w_dtype == PI_F16 && a.p_dtype != PI_F16) || (a.w_dtype == PI_F32 && a.p_dtype != PI_F32))
     return false;
-  if (a.d_model > 12288 || a.rank > 2048) return false;
+  // the predictor's u and (Q4_0) x^ stay in consumer registers
+  if (a.d_model > 12288 || a.rank > (a.p_dtype == PI_F16 ? 1024 : 512)) return false;
+  if (a.w_dtype == PI_Q4_0 && a.d_model > 8192) return false;
   if (a.w_dtype == PI_Q4_0) {
     if (a.d_model % 256) return false;
     for (int l = 0; l < n_layers; ++l) {

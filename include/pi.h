@@ -217,7 +217,8 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch,
  *   x  = x + FFN_S(xh)
  * (the pre-norm residual chaining is this library's reading; the pages do
  * not describe how layers chain).  With batch 1 and layers of one shape
- * (d_model <= 12288, rank <= 2048; Q4_0 also d_model % 256 == 0 and 16-byte
+ * (d_model <= 12288, rank <= 1024 for an fp16 predictor and <= 512 for an
+ * fp32 one; Q4_0 also d_model <= 8192, d_model % 256 == 0 and 16-byte
  * aligned scale arrays) the whole stack runs in one persistent cooperative
  * kernel per 24 layers; otherwise as a sequence of per-step kernels.
  * Setting the environment variable PI_DISABLE_FUSED=1 forces the sequence.  All layers must share d_model and d_ff;
