@@ -22,6 +22,13 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
+// Kernels that stage the inputs of a token chunk in shared memory (up to
+// 200 KB, one CTA per SM) run wider CTAs, so more warps share one staged copy
+// and more weight rows stream at once.
+constexpr int kWideThreads = 512;
+constexpr int kWideWarps = kWideThreads / 32;
+// (Q4_0 rows keep the narrow CTA: their decode needs the registers)
+template <int WT> constexpr int up_threads() { return WT == PI_Q4_0 ? kThreads : kWideThreads; }
 
 __device__ __forceinline__ void flag(uint32_t* status, uint32_t bit) {
   if (status) atomicOr(status, bit);
@@ -139,7 +146,7 @@ __global__ void __launch_bounds__(1024) k_rmsnorm(const float* __restrict__ x, i
 
 // u[b][k] = p1[k] . xh[b]; one warp per predictor row.
 template <int PT, int TB>
-__global__ void __launch_bounds__(kThreads) k_pred_u(const char* __restrict__ p1,
+__global__ void __launch_bounds__(kWideThreads) k_pred_u(const char* __restrict__ p1,
                                                      const float* __restrict__ xh, int B,
                                                      int d, int r, float* __restrict__ u) {
   extern __shared__ __align__(16) float sx[];
@@ -150,13 +157,13 @@ __global__ void __launch_bounds__(kThreads) k_pred_u(const char* __restrict__ p1
   constexpr int CC = WTraits<PT>::CHUNK_COLS;
   const int nch = d / CC;
   const int64_t rb = row_bytes(PT, d);
-  for (int k = blockIdx.x * kWarps + warp; k < r; k += gridDim.x * kWarps) {
+  for (int k = blockIdx.x * kWideWarps + warp; k < r; k += gridDim.x * kWideWarps) {
     float acc[1][TB];
 #pragma unroll
     for (int b = 0; b < TB; ++b) acc[0][b] = 0.f;
     const char* rows[1] = {p1 + (size_t)k * rb};
     const uint16_t* sc[1] = {nullptr};
-#pragma unroll 4
+#pragma unroll 8
     for (int c = lane; c < nch; c += 32) RowDot<PT, 1, TB>::chunk(rows, sc, c, sx, d, acc);
 #pragma unroll
     for (int b = 0; b < TB; ++b) {
@@ -197,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) k_pred_z(const char* __restrict__ p2
         for (int b = 0; b < TB; ++b) acc[0][b] = acc[1][b] = 0.f;
         const char* rows[2] = {p2 + (size_t)(va ? ja : jb) * rb, p2 + (size_t)(vb ? jb : ja) * rb};
         const uint16_t* sc[2] = {nullptr, nullptr};
-#pragma unroll 2
+#pragma unroll 4
         for (int c = lane; c < nch; c += 32) RowDot<PT, 2, TB>::chunk(rows, sc, c, su, r, acc);
 #pragma unroll
         for (int b = 0; b < TB; ++b) {
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(256) k_mask_union(const uint32_t* __restrict__
 
 // Gathered up/gate rows + activation: one warp per listed row.
 template <int WT, int ACT, int TB>
-__global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __restrict__ xh,
+__global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const float* __restrict__ xh,
                                                      int B, const uint32_t* __restrict__ mask,
                                                      int per_token, int words,
                                                      const int32_t* __restrict__ idx,
@@ -351,7 +358,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
   const int64_t rb2 = code_stride(WT, d, up_rs);
   const int64_t sbs2 = scale_stride(d, up_rs);
   // list positions n0 .. N-1 (n0 = H when the hot rows are computed elsewhere)
-  for (int n = n0 + blockIdx.x * kWarps + warp; n < N; n += gridDim.x * kWarps) {
+  constexpr int UPW = up_threads<WT>() / 32;
+  for (int n = n0 + blockIdx.x * UPW + warp; n < N; n += gridDim.x * UPW) {
     const int j = n < H ? n : idx[n - H];
     if (j < H && n >= H || j >= F || j < 0) {
       if (lane == 0) {
@@ -377,7 +385,9 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
     for (int r = 0; r < NR; ++r)
 #pragma unroll
       for (int b = 0; b < TB; ++b) acc[r][b] = 0.f;
-#pragma unroll 2
+    // several 16-byte loads per lane in flight: one row per warp, so the
+    // warp's memory parallelism comes from unrolling along the row
+#pragma unroll (8 / NR)
     for (int c = lane; c < nch; c += 32) RowDot<WT, NR, TB>::chunk(rows, sc, c, sx, d, acc);
     const float bj = L.bias ? L.bias[j] : 0.f;
 #pragma unroll
@@ -398,7 +408,12 @@ __global__ void __launch_bounds__(kThreads) k_ffn_up(pi_layer L, const float* __
 // Split-K gathered down projection.  Grid (column tiles, S, token chunks):
 // CTA (x, s, z) accumulates its slice s of the list positions [nb, N) for 8
 // columns per thread and TB tokens, skipping rows whose h is 0 for all of
-// its tokens, and writes its partial sums.
+// its tokens, and writes its partial sums.  The slice is taken in passes of
+// kDownStage positions: the CTA first lists the pass's rows with a nonzero
+// h (row id and the tokens' h, in position order) in shared memory, then
+// streams just those rows, several loads in flight per thread.
+constexpr int kDownStage = 512;
+
 template <int WT, int TB>
 __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ wd,
                                                        const uint16_t* __restrict__ wsc, int d,
@@ -408,8 +423,12 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
                                                        const float* __restrict__ h, int B,
                                                        int S, float* __restrict__ part,
                                                        WsHeader* hdr, int64_t stride, int nb) {
+  __shared__ int srow[kDownStage];
+  __shared__ float sh[kDownStage][TB];
+  __shared__ int swarp[kWarps + 1];
   const int s = blockIdx.y, t0 = blockIdx.z * TB;
-  const int col0 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int col0 = (blockIdx.x * blockDim.x + tid) * 8;
   int cnt = *count;
   cnt = cnt < 0 ? 0 : (cnt > F - H ? F - H : cnt);
   const int N = H + cnt, M = N - nb;
@@ -422,47 +441,84 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
   const int64_t rb = code_stride(WT, d, stride);
   const int64_t sbs = scale_stride(d, stride);
   unsigned long long nread = 0;
-  if (col0 < d) {
-#pragma unroll 4
-    for (int n = n0; n < n1; ++n) {
+  for (int p0 = n0; p0 < n1; p0 += kDownStage) {
+    const int pn = min(kDownStage, n1 - p0);
+    // the pass's rows with a nonzero h for some token of the chunk, in order
+    int base = 0;
+    for (int r0 = 0; r0 < pn; r0 += kThreads) {
+      const int q = r0 + tid;
+      const int n = p0 + q;
       float hv[TB];
-      bool any = false;
+      bool keep = false;
+      int j = 0;
+      if (q < pn) {
 #pragma unroll
-      for (int b = 0; b < TB; ++b) {
-        hv[b] = (t0 + b < B) ? h[(size_t)n * B + t0 + b] : 0.f;
-        any |= hv[b] != 0.f;
+        for (int b = 0; b < TB; ++b) {
+          hv[b] = (t0 + b < B) ? h[(size_t)n * B + t0 + b] : 0.f;
+          keep |= hv[b] != 0.f;
+        }
+        j = n < H ? n : idx[n - H];
+        keep = keep && j >= 0 && j < F;
       }
-      if (!any) continue;
-      const int j = n < H ? n : idx[n - H];
-      if (j < 0 || j >= F) continue;
-      ++nread;
-      float w[8];
-      const char* row = wd + (size_t)j * rb;
-      if constexpr (WT == PI_F32) {
-        const uint4 a = ld_stream16(row + (size_t)col0 * 4);
-        const uint4 c = ld_stream16(row + (size_t)col0 * 4 + 16);
-        w[0] = __uint_as_float(a.x); w[1] = __uint_as_float(a.y);
-        w[2] = __uint_as_float(a.z); w[3] = __uint_as_float(a.w);
-        w[4] = __uint_as_float(c.x); w[5] = __uint_as_float(c.y);
-        w[6] = __uint_as_float(c.z); w[7] = __uint_as_float(c.w);
-      } else if constexpr (WT == PI_F16) {
-        f16x8_to_f32(ld_stream16(row + (size_t)col0 * 2), w);
-      } else {
-        const int blk = col0 >> 5, k0 = col0 & 31;
-        const uint2 q = *reinterpret_cast<const uint2*>(row + (size_t)blk * 16 + (k0 & 15));
-        const float sc = h2f(reinterpret_cast<const uint16_t*>(
-            reinterpret_cast<const char*>(wsc) + (size_t)j * sbs)[blk]);
-        const int sh = k0 >= 16 ? 4 : 0;
-        const uint32_t qq[2] = {q.x, q.y};
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          w[e] = q4_centered((qq[e >> 2] >> (8 * (e & 3) + sh)) & 0xFu) * sc;
+      const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) swarp[warp] = __popc(bal);
+      __syncthreads();
+      if (tid == 0) {
+        int t = base;
+        for (int w = 0; w < kWarps; ++w) {
+          const int c = swarp[w];
+          swarp[w] = t;
+          t += c;
+        }
+        swarp[kWarps] = t;
       }
+      __syncthreads();
+      if (keep) {
+        const int pos = swarp[warp] + __popc(bal & ((1u << lane) - 1u));
+        srow[pos] = j;
 #pragma unroll
-      for (int b = 0; b < TB; ++b)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(hv[b], w[e], acc[b][e]);
+        for (int b = 0; b < TB; ++b) sh[pos][b] = hv[b];
+      }
+      base = swarp[kWarps];
+      __syncthreads();
     }
+    nread += (unsigned long long)base;
+    if (col0 < d) {
+#pragma unroll (WT == PI_Q4_0 ? 4 : 8)
+      for (int q = 0; q < base; ++q) {
+        const int j = srow[q];
+        float w[8];
+        const char* row = wd + (size_t)j * rb;
+        if constexpr (WT == PI_F32) {
+          const uint4 a = ld_stream16(row + (size_t)col0 * 4);
+          const uint4 c = ld_stream16(row + (size_t)col0 * 4 + 16);
+          w[0] = __uint_as_float(a.x); w[1] = __uint_as_float(a.y);
+          w[2] = __uint_as_float(a.z); w[3] = __uint_as_float(a.w);
+          w[4] = __uint_as_float(c.x); w[5] = __uint_as_float(c.y);
+          w[6] = __uint_as_float(c.z); w[7] = __uint_as_float(c.w);
+        } else if constexpr (WT == PI_F16) {
+          f16x8_to_f32(ld_stream16(row + (size_t)col0 * 2), w);
+        } else {
+          const int blk = col0 >> 5, k0 = col0 & 31;
+          const uint2 qv = *reinterpret_cast<const uint2*>(row + (size_t)blk * 16 + (k0 & 15));
+          const float sc = h2f(reinterpret_cast<const uint16_t*>(
+              reinterpret_cast<const char*>(wsc) + (size_t)j * sbs)[blk]);
+          const int sh4 = k0 >= 16 ? 4 : 0;
+          const uint32_t qq[2] = {qv.x, qv.y};
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            w[e] = q4_centered((qq[e >> 2] >> (8 * (e & 3) + sh4)) & 0xFu) * sc;
+        }
+#pragma unroll
+        for (int b = 0; b < TB; ++b) {
+          const float hb = sh[q][b];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[b][e] = fmaf(hb, w[e], acc[b][e]);
+        }
+      }
+    }
+  }
+  if (col0 < d) {
 #pragma unroll
     for (int b = 0; b < TB; ++b) {
       if (t0 + b >= B) continue;
@@ -471,7 +527,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
       reinterpret_cast<float4*>(o)[1] = make_float4(acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
     }
   }
-  if (hdr && blockIdx.x == 0 && threadIdx.x == 0 && nread) atomicAdd(&hdr->rows_down, nread);
+  if (hdr && blockIdx.x == 0 && tid == 0 && nread) atomicAdd(&hdr->rows_down, nread);
 }
 
 __global__ void __launch_bounds__(kThreads) k_reduce(const float* __restrict__ part, int S,
@@ -574,8 +630,8 @@ static cudaError_t pred_u_t(const pi_layer& L, const float* xh, int batch, float
   auto kern = k_pred_u<PT, TB>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(std::min((L.rank + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
-  kern<<<grid, kThreads, smem, s>>>((const char*)L.p1, xh, batch, L.d_model, L.rank, u);
+  dim3 grid(std::min((L.rank + kWideWarps - 1) / kWideWarps, device_sms() * 2), (batch + TB - 1) / TB);
+  kern<<<grid, kWideThreads, smem, s>>>((const char*)L.p1, xh, batch, L.d_model, L.rank, u);
   note_launch();
   return cudaGetLastError();
 }
@@ -649,8 +705,9 @@ static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const
   auto kern = k_ffn_up<WT, ACT, TB>;
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(std::min((L.d_ff + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
-  kern<<<grid, kThreads, smem, s>>>(L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
+  constexpr int T = up_threads<WT>();
+  dim3 grid(std::min((L.d_ff + T / 32 - 1) / (T / 32), device_sms() * (1024 / T)), (batch + TB - 1) / TB);
+  kern<<<grid, T, smem, s>>>(L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
                                     count, h, status, n0);
   note_launch();
   return cudaGetLastError();
