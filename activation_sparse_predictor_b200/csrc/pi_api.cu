@@ -96,8 +96,8 @@ WsLayout layout_for(int d, int F, int r, int batch, int H) {
   w.h = take((size_t)F * batch * 4);
   // split-K partials: the multi-kernel split, or one row per SM for the
   // fused single-token stack
-  // (+ up to 4 slices of the tensor-core hot prefix at token batches)
-  const size_t tcp = tc_scratch_bytes(d, F, r, batch) ? (size_t)4 * batch : 0;
+  // (+ up to 8 slices of the tensor-core down projection at token batches)
+  const size_t tcp = tc_scratch_bytes(d, F, r, batch) ? (size_t)8 * batch : 0;
   const size_t parts = (size_t)w.splits * batch + tcp > (size_t)device_sms()
                            ? (size_t)w.splits * batch + tcp
                            : (size_t)device_sms();

@@ -7,14 +7,18 @@
 //   up   : D[p][t] = sum_k W[row(p)][k] xh[t][k] for 128 list positions per
 //          tile (the MMA's A operand, K-major) and all tokens t (B: an fp16
 //          copy of the normalised inputs, tokens padded to 16, shared with
-//          the predictor); d split over up to 4 CTAs per tile; a second
+//          the predictor); the tiles that hold list positions, and the
+//          share of d each CTA takes, are sized on the device from the list
+//          length so that the CTAs fill the SMs; a second
 //          kernel sums the splits in a fixed
 //          order, adds the bias, applies ReLU / ReGLU and the per-token bits
-//          and writes an fp16 copy h16[t][p];
-//   down : D[c][t] = sum_p W_down^T[row(p)][c] h16[t][p] for 128 output
+//          and writes an fp16 copy h16 of h, tile-major: the 64 positions
+//          of k tile kt for token t at h16[(kt * nt + t) * 64 ..];
+//   down : D[c][t] = sum_p W_down^T[row(p)][c] h[t][p] for 128 output
 //          columns per tile; W_down^T (columns contiguous) is an MN-major A
-//          operand; the list positions split over up to 4 CTAs; the partial
-//          rows go to the fixed-order split-K reduction.
+//          operand; the k tiles that hold list positions split evenly over
+//          up to 8 CTAs; the partial rows go to the fixed-order split-K
+//          reduction.
 //
 // The predictor at token batches is two more contractions: u = P1 xh and
 // z = P2[H:] u.  Their results decide mask bits, so the fp32 vector operand
@@ -58,7 +62,7 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_THREADS = 128;
 constexpr int TC_FFN_WARPS = 8;  // warps of the FFN kernels: warp 1 issues the MMAs, the rest
 constexpr int TC_PW = TC_FFN_WARPS - 1;  // load (warps 0-3 also drain the accumulators)
-constexpr int TC_KSMAX = 4;      // CTAs sharing one tile's k range at most
+constexpr int TC_KSMAX_D = 8;    // CTAs sharing one down tile's list positions at most
 constexpr int TC_TMAX = 64;      // tokens at most (MMA N)
 constexpr unsigned long long kTcTimeoutNs = 1000000000ull;
 
@@ -221,13 +225,33 @@ __device__ __forceinline__ int list_row(int p, int H, int N, int F, const int32_
 // two stages keep two CTAs (80 KB each) on an SM.
 __host__ __device__ constexpr int up_stages(int nr) { return nr == 2 ? 2 : TC_STAGES; }
 
-// up: NR = 1 ReLU (W_up), NR = 2 ReGLU (W_gate, W_up).  Grid (Fp / 128, ks).
-// part: [ks][NR][Fp][nt] fp32.
+// Work of the up kernel for a list of N positions: nT = ceil(N / 128) row
+// tiles, each split over ks shares of d (nk k tiles) so that nT * ks CTAs
+// fill the g CTA slots of the grid.  A split costs a 32 KB fp32 partial
+// tile per operand, written here and read back by the finish kernel, about
+// 4 ks / nk of the tile's weight bytes; ks <= nk / 32 keeps that near 1/8.
+// Partial sums are laid out [ks][NR][nT * 128][nt].  The same function
+// sizes the work on both sides of the finish kernel.
+struct UpShare {
+  int nT, ks;
+};
+__host__ __device__ inline UpShare up_share(int N, int g, int nk) {
+  UpShare u;
+  u.nT = (N + TC_M - 1) / TC_M;
+  int ks = u.nT > 0 ? g / u.nT : 1;
+  const int cap = nk / 32 > 1 ? nk / 32 : 1;
+  u.ks = ks < 1 ? 1 : (ks > cap ? cap : ks);
+  return u;
+}
+
+// up: NR = 1 ReLU (W_up), NR = 2 ReGLU (W_gate, W_up).  One-dimensional
+// grid of at least g CTAs; CTA b takes tile b / ks, share b % ks of
+// up_share(N, g, nk) and exits past nT * ks.  part: [ks][NR][nT * 128][nt] fp32.
 template <int NR>
 __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     k_ffn_up_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
                 const __grid_constant__ CUtensorMap mg0, const __grid_constant__ CUtensorMap mg1,
-                const __grid_constant__ CUtensorMap mx, int nt, int nk, int ks, int H, int F, int Fp,
+                const __grid_constant__ CUtensorMap mx, int nt, int nk, int g, int H, int F,
                 const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                 float* __restrict__ part, WsHeader* hdr) {
   constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
@@ -246,10 +270,12 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   int* rows = reinterpret_cast<int*>(tslot + 4);  // [128], 16-byte aligned
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tile = blockIdx.x, split = blockIdx.y;
   const int N = list_len(count, H, F, hdr);
+  const UpShare us = up_share(N, g, nk);
+  const int ks = us.ks, Np = us.nT * TC_M;
+  if ((int)blockIdx.x >= us.nT * ks) return;  // no share of the list for this CTA
+  const int tile = blockIdx.x / ks, split = blockIdx.x % ks;
   const int p0 = tile * TC_M;
-  if (p0 >= N) return;  // past the list: nothing of this tile is read
   const bool dense = p0 + TC_M <= H;
   const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
   const int nkt = kt1 - kt0;
@@ -339,7 +365,7 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     const int p = p0 + warp * 32 + lane;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-      float* dst = part + ((size_t)(split * NR + r) * Fp + p) * nt;
+      float* dst = part + ((size_t)(split * NR + r) * Np + p) * nt;
       for (int c0 = 0; c0 < nt; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(r * nt + c0), v);
@@ -380,10 +406,16 @@ __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
 // For list positions p of this block's 64: h = act(sum over splits (fixed
 // order) + bias), zero for a token whose own bit is 0 (per-token masks, cold
 // positions), for positions past the list and for bad list entries (which
-// also set DEV_BAD_INDEX); written as h16[t][p] (tokens t >= batch: 0).
+// also set DEV_BAD_INDEX); written to h16 tile-major, [Fp / 64][nt][64]
+// (tokens t >= batch: 0), so that the down kernel's activation tile of a
+// stage is one contiguous 8 KB block: every column tile loads the same
+// tile at about the same time, and 64 rows a whole d_ff apart would
+// gather those loads on a few L2 slices.
+// Blocks wholly past the list write nothing: the down kernel reads h16 only
+// in 64-position tiles that hold list positions.
 // Partial sums read and h16 written coalesced through shared memory.
 template <int NR>
-__global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ part, int ks,
+__global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ part, int g, int nk,
                                                     int H, int F, int Fp, int nt, int batch,
                                                     const int32_t* __restrict__ idx,
                                                     const int32_t* __restrict__ count,
@@ -401,6 +433,9 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
     if (NR == 2) atomicAdd(&hdr->rows_second, (unsigned long long)N);
   }
   const int n0 = blockIdx.x * 64;
+  if (n0 >= N) return;
+  const UpShare us = up_share(N, g, nk);
+  const int ks = us.ks, Np = us.nT * TC_M;
   const int m = 64 * nt;
   // per row once: neuron, index check, bias
   if (threadIdx.x < 64) {
@@ -429,8 +464,8 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
       const int j = sj[nn];
       float g = 0.f, u = 0.f;
       for (int s = 0; s < ks; ++s) {
-        g += __ldcg(part + ((size_t)(s * NR) * Fp + n0) * nt + i);
-        if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * Fp + n0) * nt + i);
+        g += __ldcg(part + ((size_t)(s * NR) * Np + n0) * nt + i);
+        if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * Np + n0) * nt + i);
       }
       g += sb[nn];
       hv = g > 0.f ? g : 0.f;
@@ -443,12 +478,12 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
   __syncthreads();
   for (int i = threadIdx.x; i < m; i += blockDim.x) {
     const int b = i / 64, nn = i % 64;
-    h16[(size_t)b * Fp + n0 + nn] = __float2half_rn(sh[nn][b]);
+    h16[((size_t)(n0 / 64) * nt + b) * 64 + nn] = __float2half_rn(sh[nn][b]);
   }
 }
 
 // down: part[split][b][c] = sum over the split's list positions p of
-// W_down^T[row(p)][c] h16[b][p], for the tile's 128 columns c.  Grid (d / 128, ks).
+// W_down^T[row(p)][c] h[b][p], for the tile's 128 columns c.  Grid (d / 128, ks).
 __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     k_ffn_down_tc(const __grid_constant__ CUtensorMap mwd, const __grid_constant__ CUtensorMap mwg,
                   const __grid_constant__ CUtensorMap mh, int nt, int nk, int ks, int d, int batch,
@@ -472,9 +507,11 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   const int tile = blockIdx.x, split = blockIdx.y;
   const int N = list_len(count, H, F, hdr);
   const int nkN = (N + TC_BK - 1) / TC_BK;  // k tiles holding list positions
-  const int kt0 = (int)((long long)split * nk / ks);
-  int kt1 = (int)((long long)(split + 1) * nk / ks);
-  kt1 = kt1 < nkN ? kt1 : nkN;
+  // the splits share the k tiles that hold list positions, not all of d_ff
+  // (the list is usually much shorter), so no split idles
+  (void)nk;
+  const int kt0 = (int)((long long)split * nkN / ks);
+  const int kt1 = (int)((long long)(split + 1) * nkN / ks);
   const int nkt = kt1 > kt0 ? kt1 - kt0 : 0;
 
   if (threadIdx.x == 0) {
@@ -493,52 +530,66 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     // barrier (TC_PW arrivals per phase).  A stage inside the hot prefix is
     // two 64-column boxes (warp 0).  Otherwise its 32 four-position gathers
     // (positions pk + 4g .. pk + 4g + 3 of column half o / 16, g = o % 16)
-    // are dealt out round-robin, gather o = TC_PW * lane + pw; each lane
-    // loads the next stage's list rows while this one issues.
+    // are dealt out round-robin, gather o = TC_PW * lane + pw.  Each lane
+    // holds the list rows of its gather for as many stages ahead as the ring
+    // is deep, so the list loads of a stage are in flight a whole ring ahead
+    // of its gathers (the loop runs the ring's slots unrolled, and the row
+    // registers are indexed statically).
     const int pw = warp == 0 ? 0 : warp - 1;
     const int o = TC_PW * lane + pw;
     const int half = o >> 4, g = o & 15;  // column half, position group
     const bool gl = o < 32;
     const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
     const uint32_t mine = (uint32_t)((32 - pw + TC_PW - 1) / TC_PW);  // gathers of this warp
-    int y[4], ny[4];  // list rows of this lane's gather: this stage, the next
+    int yr[TC_STAGES][4];  // list rows of this lane's gather, one set per ring slot
     auto rows_at = [&](int i, int (&v)[4]) {
       const int q = (kt0 + i) * TC_BK + 4 * g;
 #pragma unroll
       for (int t = 0; t < 4; ++t) v[t] = gl ? list_row(q + t, H, N, F, idx) : 0;
     };
-    if (nkt > 0) rows_at(0, ny);
-    int last[TC_STAGES];
-    for (int i = 0; i < TC_STAGES; ++i) last[i] = -1;
-    for (int i = 0; i < nkt; ++i) {
-      const int st = i % TC_STAGES;
-      int ok = 1;
-      if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      unsigned char* a = smem + st * STAGE;
-      const int pk = (kt0 + i) * TC_BK;  // first list position of the stage
-      const bool boxed = pk + TC_BK <= H;
-      const uint32_t tx = boxed ? (pw == 0 ? A_BYTES + bx : 0u) : 512u * mine + (pw == 0 ? bx : 0u);
 #pragma unroll
-      for (int t = 0; t < 4; ++t) y[t] = ny[t];
-      if (i + 1 < nkt) rows_at(i + 1, ny);
-      if (lane == 0)
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
-                     "r"(tx)
-                     : "memory");
-      __syncwarp();
-      if (boxed) {
-        if (pw == 0 && lane == 0) {
-          tma_load_2d(a, &mwd, c0, pk, &full[st]);
-          tma_load_2d(a + BOX, &mwd, c0 + 64, pk, &full[st]);
+    for (int u = 0; u < TC_STAGES; ++u)
+      if (u < nkt) rows_at(u, yr[u]);
+    int last[TC_STAGES];
+#pragma unroll
+    for (int u = 0; u < TC_STAGES; ++u) last[u] = -1;
+    bool stop = false;
+    for (int i0 = 0; i0 < nkt && !stop; i0 += TC_STAGES) {
+#pragma unroll
+      for (int st = 0; st < TC_STAGES; ++st) {  // ring slot st = i % TC_STAGES
+        const int i = i0 + st;
+        if (i >= nkt) break;
+        int ok = 1;
+        if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
         }
-      } else if (gl) {
-        tma_gather4(a + half * BOX + 512u * g, &mwg, c0 + 64 * half, y[0], y[1], y[2], y[3], &full[st]);
+        unsigned char* a = smem + st * STAGE;
+        const int pk = (kt0 + i) * TC_BK;  // first list position of the stage
+        const bool boxed = pk + TC_BK <= H;
+        const uint32_t tx = boxed ? (pw == 0 ? A_BYTES + bx : 0u) : 512u * mine + (pw == 0 ? bx : 0u);
+        const int y0 = yr[st][0], y1 = yr[st][1], y2 = yr[st][2], y3 = yr[st][3];
+        if (i + TC_STAGES < nkt) rows_at(i + TC_STAGES, yr[st]);
+        if (lane == 0)
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
+                       "r"(tx)
+                       : "memory");
+        __syncwarp();
+        if (boxed) {
+          if (pw == 0 && lane == 0) {
+            tma_load_2d(a, &mwd, c0, pk, &full[st]);
+            tma_load_2d(a + BOX, &mwd, c0 + 64, pk, &full[st]);
+          }
+        } else if (gl) {
+          tma_gather4(a + half * BOX + 512u * g, &mwg, c0 + 64 * half, y0, y1, y2, y3, &full[st]);
+        }
+        if (pw == 0 && lane == 0) tma_load_2d(a + A_BYTES, &mh, 0, (pk / TC_BK) * nt, &full[st]);
+        last[st] = i;
       }
-      if (pw == 0 && lane == 0) tma_load_2d(a + A_BYTES, &mh, pk, 0, &full[st]);
-      if (lane == 0) last[st] = i;
     }
     if (lane == 0) {
+#pragma unroll
       for (int st = 0; st < TC_STAGES; ++st)
         if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
     }
@@ -774,16 +825,10 @@ size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 int fpad(int F) { return (F + TC_M - 1) / TC_M * TC_M; }
 
-// K splits per output tile so that tiles x splits fill every SM with the two
-// CTAs (about 100 KB of shared memory each) it can hold.
-int split_for(int tiles, int nk) {
-  int ks = 2 * device_sms() / tiles;
-  ks = ks < 1 ? 1 : (ks > TC_KSMAX ? TC_KSMAX : ks);
-  return ks > nk ? nk : ks;
-}
-
-// splits of the up GEMM's d for a layer shape
-int up_splits(int d, int F) { return split_for(fpad(F) / TC_M, d / TC_BK); }
+// CTA slots of the up kernel's grid (two CTAs per SM), and its length:
+// every row tile of the longest list (ks = 1) or the slots, whichever is more.
+int up_slots() { return 2 * device_sms(); }
+int up_grid(int F) { return std::max(up_slots(), fpad(F) / TC_M); }
 
 int pred_u_splits(int d, int r) {
   int ks = device_sms() / (r / TC_M);
@@ -792,7 +837,7 @@ int pred_u_splits(int d, int r) {
 }
 
 // Scratch: xh16 [64][d] fp16 | up partial sums [ks][2][Fp][64] fp32 |
-// h16 [64][Fp] fp16 | predictor: xs_lo [64][d] fp16 | u partial sums
+// h16 [Fp / 64][64][64] fp16 | predictor: xs_lo [64][d] fp16 | u partial sums
 // [ksu][r][64] fp32 | u_hi, u_lo [64][r] fp16 (xh16 doubles as xs_hi).
 struct TcScratch {
   __half* xh16;
@@ -812,7 +857,8 @@ TcScratch tc_scratch(void* base, int d, int F, int r) {
   t.xh16 = reinterpret_cast<__half*>(p);
   p += up256((size_t)TC_TMAX * d * 2);
   t.part = reinterpret_cast<float*>(p);
-  p += up256((size_t)up_splits(d, F) * 2 * fpad(F) * TC_TMAX * 4);
+  // nT * ks <= up_grid(F) partial row tiles of two operands
+  p += up256((size_t)up_grid(F) * TC_M * 2 * TC_TMAX * 4);
   t.h16 = reinterpret_cast<__half*>(p);
   p += up256((size_t)TC_TMAX * fpad(F) * 2);
   t.xlo = reinterpret_cast<__half*>(p);
@@ -852,18 +898,18 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
     note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const int tiles = Fp / TC_M, nk = d / TC_BK, ks = up_splits(d, F);
+  const int nk = d / TC_BK, g = up_slots();
   constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
   const size_t smem = 1024 + (size_t)up_stages(NR) * STAGE + 8 * (2 * up_stages(NR) + 1) + 16 + 4 * TC_M;
   auto kern = k_ffn_up_tc<NR>;
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, ks, H, F, Fp, idx,
-                                                 count, sc.part, hdr);
+  kern<<<up_grid(F), 32 * TC_FFN_WARPS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, g, H, F, idx, count,
+                                            sc.part, hdr);
   note_launch();
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_ffn_finish<NR><<<Fp / 64, 256, 0, s>>>(sc.part, ks, H, F, Fp, nt, batch, idx, count, L.bias,
+  k_ffn_finish<NR><<<Fp / 64, 256, 0, s>>>(sc.part, g, nk, H, F, Fp, nt, batch, idx, count, L.bias,
                                            mask, (F + 31) / 32, sc.h16, hdr,
                                            L.act == PI_RELU2 ? 1 : 0);
   note_launch();
@@ -953,7 +999,11 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
 }
 
 int ffn_tc_down_splits(const pi_layer& L) {
-  return split_for(L.d_model / TC_M, fpad(L.d_ff) / TC_BK);
+  // up to TC_KSMAX_D list shares per 128-column tile, to fill two CTAs per SM
+  int ks = 2 * device_sms() / (L.d_model / TC_M);
+  ks = ks < 1 ? 1 : (ks > TC_KSMAX_D ? TC_KSMAX_D : ks);
+  const int nk = fpad(L.d_ff) / TC_BK;
+  return ks > nk ? nk : ks;
 }
 
 cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
@@ -974,7 +1024,8 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
   CUtensorMap mwd, mwg, mh;
   if (!map_2d(&mwd, L.w_down_t, (uint64_t)d, (uint64_t)F, (uint64_t)rd, TC_BK) ||
       !map_2d(&mwg, L.w_down_t, (uint64_t)d, (uint64_t)F, (uint64_t)rd, 1) ||
-      !map_2d(&mh, sc.h16, (uint64_t)Fp, (uint64_t)nt, (uint64_t)Fp * 2, (uint32_t)nt))
+      !map_2d(&mh, sc.h16, (uint64_t)TC_BK, (uint64_t)(Fp / TC_BK) * nt, (uint64_t)TC_BK * 2,
+              (uint32_t)nt))
     return cudaErrorInvalidValue;
   const int tiles = d / TC_M, nk = Fp / TC_BK, ks = ffn_tc_down_splits(L);
   constexpr uint32_t STAGE = 2 * 64 * TC_BK * 2 + TC_TMAX * TC_BK * 2;

@@ -216,7 +216,8 @@ def test_device_checks_flag_bad_lists(pi, orc):
 @pytest.mark.parametrize("act,wdt", [("relu", "f32"), ("reglu", "f16"), ("reglu", "q4_0"),
                                      ("relu", "q4_0"), ("relu", "f16"), ("relu2", "f16"),
                                      ("relu2", "q4_0"), ("reglu", "f32")])
-@pytest.mark.parametrize("batch,mode", [(1, "union"), (4, "per_token"), (8, "union")])
+@pytest.mark.parametrize("batch,mode", [(1, "union"), (2, "per_token"), (4, "per_token"),
+                                        (8, "per_token"), (8, "union")])
 @pytest.mark.parametrize("packed", [False, True])
 def test_stack(pi, orc, act, wdt, batch, mode, packed):
     w = _wl(act, wdt, (512, 1500, 64, 256), seed=43, mean=0.15).scaled(3)
@@ -294,7 +295,8 @@ def test_kernel_launch_counter(pi):
     assert counts[0] == counts[1] >= 4 * 6  # per layer: norm, predictor, compaction, FFN, reduce
 
 
-@pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0)])
+@pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0),
+                                   (4096, 1500, 64, 256), (8192, 1000, 64, 640)])
 @pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
 @pytest.mark.parametrize("batch,mode", [(16, "per_token"), (20, "union"), (48, "per_token"),
                                         (64, "union")])
@@ -305,7 +307,9 @@ def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
     the fp16 tolerance of the oracle, close to the CUDA-core path, and not
     bitwise equal to it (so the tensor-core path did run).  Shapes cover a
     ragged d_ff, a hot prefix that ends inside a tile, and no hot prefix;
-    batches 20 and 48 pad the token tile."""
+    batches 20 and 48 pad the token tile.  At d = 4096 and 8192 the up
+    kernel splits d over 2 and 4 CTAs per row tile, and the down kernel
+    splits a short list over 8 and 4 CTAs per column tile."""
     w = _wl(act, "f16", shape, seed=47)
     L, _ = device_layer(w, 0, packed=(batch % 32 == 0))
     H = synth.layer_host(w, 0)
