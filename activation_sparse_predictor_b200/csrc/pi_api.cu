@@ -194,14 +194,20 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
 }
 
 // mask [batch][words] of xh: the predictor (tensor cores at token batches).
+// `uni` (optional): the tensor-core predictor also writes there the OR of
+// the tokens' words from the word holding `hot` on; *uni_done says whether
+// it did.
 pi_status predict_body(const pi_layer& L, const float* xh, int batch, float theta, uint32_t* mask,
-                       void* ws, const WsLayout& lay, cudaStream_t s, Prof* prof = nullptr) {
+                       void* ws, const WsLayout& lay, cudaStream_t s, Prof* prof = nullptr,
+                       uint32_t* uni = nullptr, bool* uni_done = nullptr) {
   Prof none;
   Prof& P = prof ? *prof : none;
   cudaError_t e;
+  if (uni_done) *uni_done = false;
   if (pred_tc_supported(L, batch)) {
     P.before(PI_KIND_PRED_U);
-    e = launch_predict_tc(L, xh, batch, theta, mask, at<void>(ws, lay.tc), header(ws), s);
+    e = launch_predict_tc(L, xh, batch, theta, mask, at<void>(ws, lay.tc), header(ws), s, uni);
+    if (uni_done) *uni_done = uni != nullptr;
     P.after();
     return e == cudaSuccess ? PI_OK : cuda_fail(e, "predictor (tensor cores) launch");
   }
@@ -268,13 +274,16 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
     cudaError_t e = launch_rmsnorm(x, batch, d, xh, s);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
-    if ((st = predict_body(L, xh, batch, theta, mask, ws, lay, s, prof)) != PI_OK) return st;
+    // at token batches the tokens' union goes into the activation buffer
+    // (free until the up projection): from the tensor-core predictor's
+    // epilogue, else from a union kernel; then one list from it
+    uint32_t* uni = batch > 1 ? at<uint32_t>(ws, lay.h) : nullptr;
+    bool uni_done = false;
+    if ((st = predict_body(L, xh, batch, theta, mask, ws, lay, s, prof, uni, &uni_done)) != PI_OK)
+      return st;
     P.before(PI_KIND_COMPACT);
     if (batch > 1) {
-      // the tokens' union first, across many CTAs, into the activation
-      // buffer (free until the up projection), then one list from it
-      uint32_t* uni = at<uint32_t>(ws, lay.h);
-      e = launch_mask_union(mask, batch, words, uni, s);
+      e = uni_done ? cudaSuccess : launch_mask_union(mask, batch, words, uni, s);
       if (e == cudaSuccess) e = launch_compact(uni, 1, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);
     } else {
       e = launch_compact(mask, batch, L.d_ff, L.hot, PI_MASK_UNION, idx, cnt, s);

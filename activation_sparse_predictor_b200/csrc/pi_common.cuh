@@ -31,6 +31,21 @@ struct WsHeader {
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");
 
+// ------------------------------------------------ dependent launches
+// The per-step kernels are launched with programmatic stream serialization
+// (launch_dep): a kernel's CTAs may be scheduled while the previous kernel
+// on the stream drains.  Each such kernel calls pdl_wait() before its first
+// access to global memory that another kernel writes or reads (it returns
+// once the previous kernel has completed and its writes are visible; a
+// no-op when the kernel was launched without the attribute), and then
+// pdl_trigger(), which lets the next kernel's CTAs be scheduled once every
+// CTA of this one has started.  Since each kernel waits for the one before
+// it, every earlier kernel has completed by then too.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- loads
 // 16-byte streaming load of data read once per kernel (weights): no L1
 // allocation, so the reused vectors in L1/shared memory are not evicted.

@@ -10,6 +10,7 @@
 // with the reused vectors (xh, u) staged in shared memory.  Accumulation is
 // fp32 throughout.
 #include <algorithm>
+#include <cstdlib>
 #include <atomic>
 #include <mutex>
 #include <unordered_map>
@@ -124,24 +125,43 @@ struct RowDot {
 };
 
 // ---------------------------------------------------------------------------
-template <int TB>
+// One CTA per row (d <= 16384, d % 4 == 0): the row is read once into
+// registers (up to four float4 per thread), its mean square reduced across
+// the CTA, and the scaled row written from the registers.
 __global__ void __launch_bounds__(1024) k_rmsnorm(const float* __restrict__ x, int d,
                                                   float* __restrict__ xh) {
-  const float* xr = x + (size_t)blockIdx.x * d;
+  pdl_wait();
+  pdl_trigger();
+  const float4* xr = reinterpret_cast<const float4*>(x + (size_t)blockIdx.x * d);
+  float4* yr = reinterpret_cast<float4*>(xh + (size_t)blockIdx.x * d);
+  const int n4 = d >> 2;
+  float4 v[4];
   float ss = 0.f;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) ss = fmaf(xr[i], xr[i], ss);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = threadIdx.x + k * blockDim.x;
+    v[k] = i < n4 ? xr[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    ss = fmaf(v[k].x, v[k].x, ss);
+    ss = fmaf(v[k].y, v[k].y, ss);
+    ss = fmaf(v[k].z, v[k].z, ss);
+    ss = fmaf(v[k].w, v[k].w, ss);
+  }
   ss = warp_sum(ss);
   __shared__ float red[32];
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
   if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-    v = warp_sum(v);
-    if (threadIdx.x == 0) red[0] = v;
+    float t = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    t = warp_sum(t);
+    if (threadIdx.x == 0) red[0] = t;
   }
   __syncthreads();
   const float inv = 1.0f / sqrtf(red[0] / (float)d + 1e-6f);
-  for (int i = threadIdx.x; i < d; i += blockDim.x) xh[(size_t)blockIdx.x * d + i] = xr[i] * inv;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int i = threadIdx.x + k * blockDim.x;
+    if (i < n4) yr[i] = make_float4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
+  }
 }
 
 // u[b][k] = p1[k] . xh[b]; one warp per predictor row.
@@ -149,6 +169,7 @@ template <int PT, int TB>
 __global__ void __launch_bounds__(kWideThreads) k_pred_u(const char* __restrict__ p1,
                                                      const float* __restrict__ xh, int B,
                                                      int d, int r, float* __restrict__ u) {
+  pdl_wait();
   extern __shared__ __align__(16) float sx[];
   const int t0 = blockIdx.y * TB;
   stage_x<TB>(sx, xh, B, d, t0);
@@ -180,6 +201,7 @@ __global__ void __launch_bounds__(kThreads) k_pred_z(const char* __restrict__ p2
                                                      const float* __restrict__ u, int B, int r,
                                                      int F, int H, float theta,
                                                      uint32_t* __restrict__ mask, int words) {
+  pdl_wait();
   extern __shared__ __align__(16) float su[];
   const int t0 = blockIdx.y * TB;
   stage_x<TB>(su, u, B, r, t0);
@@ -225,68 +247,89 @@ __global__ void __launch_bounds__(kThreads) k_pred_z(const char* __restrict__ p2
   }
 }
 
-// Compaction: one CTA per list; block-wide exclusive scan of per-word
-// popcounts, each thread then writes its word's set bits in order.
-__global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ mask, int B,
-                                                  int words, int F, int begin, int unite,
-                                                  int32_t* __restrict__ idx, int idx_stride,
-                                                  int32_t* __restrict__ count) {
-  __shared__ int wsum[32];
+// Compaction.  Grid (chunks, lists): CTA x of list l takes the
+// kCompactWords mask words [x * kCompactWords, ...) of the list, one word
+// per thread.  Its first output position is the number of set bits in the
+// list's words before the chunk, which the CTA counts itself (a few KB of
+// mask words at most); then a scan of its words' popcounts places every
+// word's bits, and each warp writes its 32 words' entries in order, lane t
+// taking bit t of each word (the entries of one word go to consecutive
+// positions).  The last chunk's CTA writes the count.  Bits below `begin`
+// and from F on are cleared; `unite` ORs the B tokens' words first.
+constexpr int kCompactWords = 256;
+
+__device__ __forceinline__ uint32_t compact_word(const uint32_t* __restrict__ mask, int B,
+                                                 int words, int F, int begin, int unite, int list,
+                                                 int w) {
+  uint32_t m = 0u;
+  if (unite) {
+#pragma unroll 8
+    for (int b = 0; b < B; ++b) m |= mask[(size_t)b * words + w];
+  } else {
+    m = mask[(size_t)list * words + w];
+  }
+  const int lo = w * 32;
+  if (begin > lo) m = (begin - lo >= 32) ? 0u : (m & (~0u << (begin - lo)));
+  if (F < lo + 32) m = (F <= lo) ? 0u : (m & ((1u << (F - lo)) - 1u));
+  return m;
+}
+
+__global__ void __launch_bounds__(kCompactWords) k_compact(const uint32_t* __restrict__ mask, int B,
+                                                           int words, int F, int begin, int unite,
+                                                           int32_t* __restrict__ idx, int idx_stride,
+                                                           int32_t* __restrict__ count) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NW = kCompactWords / 32;
+  __shared__ int wsum[NW + 1];
   __shared__ int s_base;
-  const int list = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  if (tid == 0) s_base = 0;
+  const int list = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int w_lo = blockIdx.x * kCompactWords;
+  // set bits of the list's words before this chunk (words below `begin`
+  // are empty and skipped)
+  int before = 0;
+  for (int w = max(begin >> 5, 0) + tid; w < w_lo; w += kCompactWords)
+    before += __popc(compact_word(mask, B, words, F, begin, unite, list, w));
+  before = __reduce_add_sync(0xffffffffu, before);
+  if (lane == 0) wsum[warp] = before;
+  __syncthreads();
+  if (tid == 0) {
+    int t = 0;
+    for (int k = 0; k < NW; ++k) t += wsum[k];
+    s_base = t;
+  }
+  __syncthreads();
+  const int w = w_lo + tid;
+  const uint32_t m = w < words ? compact_word(mask, B, words, F, begin, unite, list, w) : 0u;
+  const int c = __popc(m);
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int k = 0; k < NW; ++k) {
+      const int t = wsum[k];
+      wsum[k] = run;
+      run += t;
+    }
+    wsum[NW] = run;
+  }
   __syncthreads();
   int32_t* out = idx + (size_t)list * idx_stride;
-  for (int w0 = 0; w0 < words; w0 += blockDim.x) {
-    const int w = w0 + tid;
-    uint32_t m = 0;
-    if (w < words) {
-      if (unite) {
-        for (int b = 0; b < B; ++b) m |= mask[(size_t)b * words + w];
-      } else {
-        m = mask[(size_t)list * words + w];
-      }
-      const int lo = w * 32;
-      if (begin > lo) m = (begin - lo >= 32) ? 0u : (m & (~0u << (begin - lo)));
-      if (F < lo + 32) m = (F <= lo) ? 0u : (m & ((1u << (F - lo)) - 1u));
-    }
-    const int c = __popc(m);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-      int v = lane < nw ? wsum[lane] : 0;
-      int vi = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, vi, o);
-        if (lane >= o) vi += t;
-      }
-      if (lane < nw) wsum[lane] = vi - v;  // exclusive warp offsets
-      if (lane == 31) wsum[31] = vi;       // (nw <= 31 here) total of this tile
-    }
-    __syncthreads();
-    // the warp's 32 words in order, lane t taking bit t of each: the
-    // entries of one word go to consecutive positions (coalesced stores)
-    int run = s_base + wsum[warp];
-    const int wfirst = w0 + warp * 32;
-    for (int i = 0; i < 32; ++i) {
-      const uint32_t mi = __shfl_sync(0xffffffffu, m, i);
-      if ((mi >> lane) & 1u) out[run + __popc(mi & ((1u << lane) - 1u))] = (wfirst + i) * 32 + lane;
-      run += __popc(mi);
-    }
-    const int tile_total = wsum[31];
-    __syncthreads();
-    if (tid == 0) s_base += tile_total;
-    __syncthreads();
+  int run = s_base + wsum[warp];
+  const int wfirst = w_lo + warp * 32;
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t mi = __shfl_sync(0xffffffffu, m, i);
+    if ((mi >> lane) & 1u) out[run + __popc(mi & ((1u << lane) - 1u))] = (wfirst + i) * 32 + lane;
+    run += __popc(mi);
   }
-  if (tid == 0) count[list] = s_base;
+  if (blockIdx.x == gridDim.x - 1 && tid == 0) count[list] = s_base + wsum[NW];
 }
 
 // out[w] = OR over tokens b < B of mask[b][w].  Block: 32 words x 8 token
@@ -294,6 +337,7 @@ __global__ void __launch_bounds__(1024) k_compact(const uint32_t* __restrict__ m
 // the groups combined in shared memory.
 __global__ void __launch_bounds__(256) k_mask_union(const uint32_t* __restrict__ mask, int B,
                                                     int words, uint32_t* __restrict__ out) {
+  pdl_wait();
   __shared__ uint32_t sm[8][32];
   const int wl = threadIdx.x & 31, tg = threadIdx.x >> 5;
   const int w = blockIdx.x * 32 + wl;
@@ -331,6 +375,7 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
                                                      const int32_t* __restrict__ count,
                                                      float* __restrict__ h, WsHeader* hdr,
                                                      int n0) {
+  pdl_wait();
   extern __shared__ __align__(16) float sx[];
   uint32_t* status = hdr ? &hdr->status : nullptr;
   const int d = L.d_model, F = L.d_ff, H = L.hot;
@@ -423,6 +468,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
                                                        const float* __restrict__ h, int B,
                                                        int S, float* __restrict__ part,
                                                        WsHeader* hdr, int64_t stride, int nb) {
+  pdl_wait();
   __shared__ int srow[kDownStage];
   __shared__ float sh[kDownStage][TB];
   __shared__ int swarp[kWarps + 1];
@@ -530,14 +576,32 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
   if (hdr && blockIdx.x == 0 && tid == 0 && nread) atomicAdd(&hdr->rows_down, nread);
 }
 
+// out = resid + (sum over the S slices in order), four floats per thread
+// (n % 4 == 0; part, resid and out 16-byte aligned); the slices' loads are
+// unrolled so that several are in flight at once.
 __global__ void __launch_bounds__(kThreads) k_reduce(const float* __restrict__ part, int S,
                                                      int64_t n, const float* resid,
                                                      float* out) {
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
+  pdl_wait();
+  pdl_trigger();
+  const int64_t n4 = n >> 2;
+  const float4* p4 = reinterpret_cast<const float4*>(part);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n4;
        e += (int64_t)gridDim.x * blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < S; ++s) acc += part[(size_t)s * n + e];
-    out[e] = (resid ? resid[e] : 0.f) + acc;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int s = 0; s < S; ++s) {
+      const float4 v = __ldcg(p4 + (size_t)s * n4 + e);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if (resid) {
+      const float4 r = reinterpret_cast<const float4*>(resid)[e];
+      acc = make_float4(r.x + acc.x, r.y + acc.y, r.z + acc.z, r.w + acc.w);
+    }
+    reinterpret_cast<float4*>(out)[e] = acc;
   }
 }
 
@@ -586,6 +650,14 @@ std::atomic<unsigned long long> g_launches{0};  // kernels launched by this libr
 void note_launch() { g_launches.fetch_add(1ull, std::memory_order_relaxed); }
 unsigned long long launches_so_far() { return g_launches.load(std::memory_order_relaxed); }
 
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("PI_NO_PDL");
+    return !(e && e[0] && e[0] != '0');
+  }();
+  return on;
+}
+
 int device_sms() {
   static int cache[64] = {0};
   int dev = 0;
@@ -618,8 +690,9 @@ int down_splits(int batch, int d) {
 // ---------------------------------------------------------------- launches
 
 cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s) {
-  k_rmsnorm<1><<<batch, 1024, 0, s>>>(x, d, xh);
-  note_launch();
+  // one float4 per thread up to d = 4096, then 1024 threads with up to four
+  const int n4 = d / 4, threads = std::min(1024, (n4 + 31) / 32 * 32);
+  (void)launch_dep(k_rmsnorm, batch, threads, 0, s, x, d, xh);
   return cudaGetLastError();
 }
 
@@ -631,8 +704,8 @@ static cudaError_t pred_u_t(const pi_layer& L, const float* xh, int batch, float
   cudaError_t e = allow_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid(std::min((L.rank + kWideWarps - 1) / kWideWarps, device_sms() * 2), (batch + TB - 1) / TB);
-  kern<<<grid, kWideThreads, smem, s>>>((const char*)L.p1, xh, batch, L.d_model, L.rank, u);
-  note_launch();
+  (void)launch_plain(kern, grid, kWideThreads, smem, s, (const char*)L.p1, xh, batch, L.d_model,
+                     L.rank, u);
   return cudaGetLastError();
 }
 
@@ -659,9 +732,8 @@ static cudaError_t pred_z_t(const pi_layer& L, const float* u, int batch, float 
   if (e != cudaSuccess) return e;
   const int words = (L.d_ff + 31) / 32;
   dim3 grid(std::min((words + kWarps - 1) / kWarps, device_sms() * 4), (batch + TB - 1) / TB);
-  kern<<<grid, kThreads, smem, s>>>((const char*)L.p2, L.p_bias, u, batch, L.rank, L.d_ff,
-                                    L.hot, theta, mask, words);
-  note_launch();
+  (void)launch_plain(kern, grid, kThreads, smem, s, (const char*)L.p2, L.p_bias, u, batch, L.rank,
+                     L.d_ff, L.hot, theta, mask, words);
   return cudaGetLastError();
 }
 
@@ -681,8 +753,7 @@ cudaError_t launch_pred_z(const pi_layer& L, const float* u, int batch, float th
 
 cudaError_t launch_mask_union(const uint32_t* mask, int batch, int words, uint32_t* out,
                               cudaStream_t s) {
-  k_mask_union<<<(words + 31) / 32, 256, 0, s>>>(mask, batch, words, out);
-  note_launch();
+  (void)launch_plain(k_mask_union, (words + 31) / 32, 256, 0, s, mask, batch, words, out);
   return cudaGetLastError();
 }
 
@@ -691,9 +762,9 @@ cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin,
   const int words = (d_ff + 31) / 32;
   const int unite = (mode == PI_MASK_UNION);
   const int lists = unite ? 1 : batch;
-  const int threads = std::min(992, std::max(32, ((words + 31) / 32) * 32));
-  k_compact<<<lists, threads, 0, s>>>(mask, batch, words, d_ff, begin, unite, idx, d_ff, count);
-  note_launch();
+  const dim3 grid((words + kCompactWords - 1) / kCompactWords, lists);
+  (void)launch_dep(k_compact, grid, kCompactWords, 0, s, mask, batch, words, d_ff, begin, unite,
+                   idx, d_ff, count);
   return cudaGetLastError();
 }
 
@@ -707,9 +778,8 @@ static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const
   if (e != cudaSuccess) return e;
   constexpr int T = up_threads<WT>();
   dim3 grid(std::min((L.d_ff + T / 32 - 1) / (T / 32), device_sms() * (1024 / T)), (batch + TB - 1) / TB);
-  kern<<<grid, T, smem, s>>>(L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
-                                    count, h, status, n0);
-  note_launch();
+  (void)launch_plain(kern, grid, T, smem, s, L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
+                     count, h, status, n0);
   return cudaGetLastError();
 }
 
@@ -744,11 +814,9 @@ static cudaError_t ffn_down_t(const pi_layer& L, int batch, const int32_t* idx,
                               WsHeader* hdr, cudaStream_t s, int nb) {
   const int tiles = (L.d_model + 8 * kThreads - 1) / (8 * kThreads);
   dim3 grid(tiles, S, (batch + TB - 1) / TB);
-  k_ffn_down<WT, TB><<<grid, kThreads, 0, s>>>((const char*)L.w_down_t,
-                                              (const uint16_t*)L.w_down_t_scales, L.d_model,
-                                              L.d_ff, L.hot, idx, count, h, batch, S, part, hdr,
-                                              L.w_down_row_stride, nb);
-  note_launch();
+  (void)launch_plain(k_ffn_down<WT, TB>, grid, kThreads, 0, s, (const char*)L.w_down_t,
+                     (const uint16_t*)L.w_down_t_scales, L.d_model, L.d_ff, L.hot, idx, count, h,
+                     batch, S, part, hdr, L.w_down_row_stride, nb);
   return cudaGetLastError();
 }
 
@@ -780,10 +848,9 @@ cudaError_t launch_delay(unsigned long long ns, cudaStream_t s) {
 
 cudaError_t launch_reduce(const float* part, int splits, int batch, int d, const float* resid,
                           float* out, cudaStream_t s) {
-  const int64_t n = (int64_t)batch * d;
-  const int grid = (int)std::min<int64_t>((n + kThreads - 1) / kThreads, device_sms() * 8);
-  k_reduce<<<grid, kThreads, 0, s>>>(part, splits, n, resid, out);
-  note_launch();
+  const int64_t n = (int64_t)batch * d;  // d % 4 == 0
+  const int grid = (int)std::min<int64_t>((n / 4 + kThreads - 1) / kThreads, device_sms() * 8);
+  (void)launch_dep(k_reduce, grid, kThreads, 0, s, part, splits, n, resid, out);
   return cudaGetLastError();
 }
 

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "pi.h"
 #include "pi_common.cuh"
 
@@ -15,6 +17,46 @@ unsigned long long launches_so_far();
 
 // Raises a kernel's dynamic shared-memory limit on the current device once.
 cudaError_t allow_smem_fn(const void* fn, size_t bytes);
+
+// Whether launch_dep sets programmatic stream serialization (on unless the
+// environment variable PI_NO_PDL is set to a value other than 0).
+bool pdl_enabled();
+
+// Launches kernel k like k<<<grid, block, smem, s>>>(args...) and counts
+// the launch; with dep, and when pdl_enabled(), with programmatic stream
+// serialization (the kernel must call pdl_wait() before touching global
+// memory another kernel uses).  The CUDA-core kernels of small token
+// batches, whose grids are sized to the SM count, are launched without it
+// (and do not trigger their dependents early): CTAs scheduled while the
+// previous kernel still holds SMs would be placed unevenly.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool dep, void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                     cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dep && pdl_enabled() ? 1 : 0;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, k, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dep(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  return launch_k(true, k, grid, block, smem, s, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_plain(void (*k)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                         Args&&... args) {
+  return launch_k(false, k, grid, block, smem, s, std::forward<Args>(args)...);
+}
 int pick_tb(int batch, int d);    // tokens per pass of the x-staged kernels
 int down_tb(int batch);           // tokens per pass of the down projection
 int down_splits(int batch, int d);// split-K slices of the down projection

@@ -254,6 +254,8 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
                 const __grid_constant__ CUtensorMap mx, int nt, int nk, int g, int H, int F,
                 const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                 float* __restrict__ part, WsHeader* hdr) {
+  pdl_wait();
+  pdl_trigger();
   constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB (nt rows used)
   constexpr uint32_t STAGE = NR * A_BYTES + B_BYTES;
@@ -387,6 +389,8 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
 // xh (fp32 [batch][d]) -> xh16 (fp16 [nt][d], rows >= batch zero); 8 per thread.
 __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
                        __half* __restrict__ xh16) {
+  pdl_wait();
+  pdl_trigger();
   const int n8 = d / 8;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt * n8; i += gridDim.x * blockDim.x) {
     const int t = i / n8, c = i % n8;
@@ -423,6 +427,8 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
                                                     const uint32_t* __restrict__ mask, int words,
                                                     __half* __restrict__ h16, WsHeader* hdr,
                                                     int sq) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float sh[64][TC_TMAX + 1];
   __shared__ int sj[64];    // each row's neuron
   __shared__ float sb[64];  // and bias
@@ -456,20 +462,36 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
     sv[threadIdx.x] = v;
   }
   __syncthreads();
-#pragma unroll 4
-  for (int i = threadIdx.x; i < m; i += blockDim.x) {
+  // this thread's elements i = threadIdx.x + 256 e of the block's 64 x nt:
+  // the sums over the splits stay in registers, and each split's loads of
+  // all of them are in flight together
+  constexpr int EPT = 64 * TC_TMAX / 256;
+  float gs[EPT], ua[EPT];
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) gs[e] = ua[e] = 0.f;
+  for (int s = 0; s < ks; ++s) {
+    const float* pg = part + ((size_t)(s * NR) * Np + n0) * nt;
+    const float* pu = part + ((size_t)(s * NR + 1) * Np + n0) * nt;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const int i = threadIdx.x + 256 * e;
+      if (i < m) {
+        gs[e] += __ldcg(pg + i);
+        if constexpr (NR == 2) ua[e] += __ldcg(pu + i);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const int i = threadIdx.x + 256 * e;
+    if (i >= m) break;
     const int nn = i / nt, b = i % nt, p = n0 + nn;
     float hv = 0.f;
     if (sv[nn] && b < batch) {
       const int j = sj[nn];
-      float g = 0.f, u = 0.f;
-      for (int s = 0; s < ks; ++s) {
-        g += __ldcg(part + ((size_t)(s * NR) * Np + n0) * nt + i);
-        if constexpr (NR == 2) u += __ldcg(part + ((size_t)(s * NR + 1) * Np + n0) * nt + i);
-      }
-      g += sb[nn];
-      hv = g > 0.f ? g : 0.f;
-      if constexpr (NR == 2) hv *= u;
+      const float gv = gs[e] + sb[nn];
+      hv = gv > 0.f ? gv : 0.f;
+      if constexpr (NR == 2) hv *= ua[e];
       else if (sq) hv *= hv;  // squared ReLU
       if (mask && p >= H && !((__ldg(mask + (size_t)b * words + (j >> 5)) >> (j & 31)) & 1u)) hv = 0.f;
     }
@@ -489,6 +511,8 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
                   const __grid_constant__ CUtensorMap mh, int nt, int nk, int ks, int d, int batch,
                   int H, int F, const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
                   float* __restrict__ part, WsHeader* hdr) {
+  pdl_wait();
+  pdl_trigger();
   constexpr uint32_t BOX = 64 * TC_BK * 2;             // 64 columns x 64 positions: 8 KB
   constexpr uint32_t A_BYTES = 2 * BOX;                // 128 columns
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;    // 8 KB
@@ -641,29 +665,50 @@ constexpr int TC_KSMAX_U = 16;  // CTAs sharing one tile of P1's d at most
 constexpr int TC_PSTAGES = 3;   // predictor ring stages: 97 KB, two CTAs per SM
 
 // x (fp32 [batch][n]) -> hi = fp16(x), lo = fp16(x - hi), [nt][n] each
-// (rows >= batch zero).
+// (rows >= batch zero); eight elements per thread (n % 8 == 0).
 __global__ void k_split16(const float* __restrict__ x, int batch, int n, int nt,
                           __half* __restrict__ hi, __half* __restrict__ lo) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt * n; i += gridDim.x * blockDim.x) {
-    const int t = i / n;
-    const float v = t < batch ? x[i] : 0.f;
-    const __half h = __float2half_rn(v);
-    hi[i] = h;
-    lo[i] = __float2half_rn(v - __half2float(h));
+  pdl_wait();
+  pdl_trigger();
+  const int n8 = n / 8;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt * n8; i += gridDim.x * blockDim.x) {
+    const int t = i / n8;
+    float v[8];
+    if (t < batch) {
+      const float4 a = __ldg(reinterpret_cast<const float4*>(x) + 2 * (size_t)i);
+      const float4 b = __ldg(reinterpret_cast<const float4*>(x) + 2 * (size_t)i + 1);
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+      v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) v[k] = 0.f;
+    }
+    __align__(16) __half h[8], l[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      h[k] = __float2half_rn(v[k]);
+      l[k] = __float2half_rn(v[k] - __half2float(h[k]));
+    }
+    reinterpret_cast<uint4*>(hi)[i] = *reinterpret_cast<const uint4*>(h);
+    reinterpret_cast<uint4*>(lo)[i] = *reinterpret_cast<const uint4*>(l);
   }
 }
 
 // MODE 0: D = P1 (x_hi + x_lo)^T for 128 predictor rows per tile, d split
-// over ks CTAs -> part[split][row][nt].  MODE 1: D = P2 (u_hi + u_lo)^T for
-// 128 neuron rows per tile from row0 (a multiple of 32, <= hot) -> mask
-// words: bit j of token t = (j < hot) or (z_j + c_j > theta) for j < d_ff.
-// Grid (tiles, ks).
+// over ks CTAs -> part[split][token][row] (token-major, so the finish
+// kernel reads and writes along the rows).  MODE 1: D = P2 (u_hi + u_lo)^T
+// for 128 neuron rows per tile from row0 (a multiple of 32, <= hot) -> mask
+// words: bit j of token t = (j < hot) or (z_j + c_j > theta) for j < d_ff;
+// the words below row0 (all hot) are written all ones by the CTAs in turn,
+// and `uni`, when given, gets each word's OR over the batch's tokens (each
+// warp holds one word of every token).  Grid (tiles, ks).
 template <int MODE>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     k_pred_tc(const __grid_constant__ CUtensorMap ma, const __grid_constant__ CUtensorMap mbh,
               const __grid_constant__ CUtensorMap mbl, int nt, int nk, int ks, int row0, int M,
               float* __restrict__ part, const float* __restrict__ bias, float theta, int H,
-              uint32_t* __restrict__ mask, int words, int batch, WsHeader* hdr) {
+              uint32_t* __restrict__ mask, int words, int batch, WsHeader* hdr,
+              uint32_t* __restrict__ uni) {
   constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB per part
   constexpr uint32_t STAGE = A_BYTES + 2 * B_BYTES;
@@ -689,6 +734,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tslot;
+  pdl_wait();  // the prologue above touches no global memory
+  pdl_trigger();
 
   if (warp == 0 && lane == 0) {
     const uint32_t tx = A_BYTES + 2u * (uint32_t)nt * TC_BK * 2;
@@ -732,6 +779,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const int m = m0 + warp * 32 + lane;  // this thread's row
+  uint32_t any = 0u;                     // MODE 1: OR of this warp's word over the tokens
   for (int c0 = 0; c0 < nt; c0 += 16) {
     uint32_t v[16];
     if (ok) {
@@ -742,12 +790,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     if constexpr (MODE == 0) {
       if (m < M) {
-        float* dst = part + ((size_t)split * M + m) * nt + c0;
+        float* dst = part + ((size_t)split * nt + c0) * M + m;
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          __stcg(reinterpret_cast<float4*>(dst) + q,
-                 make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
-                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+        for (int t = 0; t < 16; ++t) __stcg(dst + (size_t)t * M, __uint_as_float(v[t]));
       }
     } else {
       const float cb = (bias && m < M) ? bias[m] : 0.f;
@@ -756,9 +801,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int t = 0; t < 16; ++t) {
         const bool bit = m < H || (m < M && __uint_as_float(v[t]) + cb > theta);
         const uint32_t word = __ballot_sync(0xffffffffu, bit);
+        if (c0 + t < batch) any |= word;
         if (lane == 0 && c0 + t < batch && w < words) mask[(size_t)(c0 + t) * words + w] = word;
       }
     }
+  }
+  if constexpr (MODE == 1) {
+    const int w = (m0 + warp * 32) >> 5;
+    if (uni && lane == 0 && w < words) uni[w] = any;
+    const int w0 = row0 >> 5;  // hot words, all ones
+    for (int i = (blockIdx.x * gridDim.y + blockIdx.y) * TC_THREADS + threadIdx.x; i < batch * w0;
+         i += gridDim.x * gridDim.y * TC_THREADS)
+      mask[(size_t)(i / w0) * words + i % w0] = 0xFFFFFFFFu;
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
@@ -767,22 +821,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                  : "memory");
 }
 
-// u = sum over the splits (fixed order) -> u_hi, u_lo [nt][r] (tokens >= batch: 0).
+// u = sum over the splits (fixed order) of part[split][t][k] -> u_hi,
+// u_lo [nt][r] (tokens >= batch: 0); four rows k per thread (r % 4 == 0),
+// every split's load issued before the sums (ks <= TC_KSMAX_U).
 __global__ void k_pred_u_finish(const float* __restrict__ part, int ks, int r, int nt, int batch,
                                 __half* __restrict__ uhi, __half* __restrict__ ulo) {
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < r * nt; i += gridDim.x * blockDim.x) {
-    const int k = i / nt, t = i % nt;
-    float u = 0.f;
-    if (t < batch)
-      for (int s = 0; s < ks; ++s) u += __ldcg(part + ((size_t)s * r + k) * nt + t);
-    const __half h = __float2half_rn(u);
-    uhi[(size_t)t * r + k] = h;
-    ulo[(size_t)t * r + k] = __float2half_rn(u - __half2float(h));
+  pdl_wait();
+  pdl_trigger();
+  const int r4 = r / 4;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nt * r4; i += gridDim.x * blockDim.x) {
+    const int t = i / r4;
+    float4 u = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (t < batch) {
+      float4 v[TC_KSMAX_U];
+#pragma unroll
+      for (int s = 0; s < TC_KSMAX_U; ++s)
+        if (s < ks) v[s] = __ldcg(reinterpret_cast<const float4*>(part + (size_t)s * nt * r) + i);
+#pragma unroll
+      for (int s = 0; s < TC_KSMAX_U; ++s)
+        if (s < ks) {
+          u.x += v[s].x;
+          u.y += v[s].y;
+          u.z += v[s].z;
+          u.w += v[s].w;
+        }
+    }
+    const float uu[4] = {u.x, u.y, u.z, u.w};
+    __align__(8) __half h[4], l[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      h[k] = __float2half_rn(uu[k]);
+      l[k] = __float2half_rn(uu[k] - __half2float(h[k]));
+    }
+    reinterpret_cast<uint2*>(uhi)[i] = *reinterpret_cast<const uint2*>(h);
+    reinterpret_cast<uint2*>(ulo)[i] = *reinterpret_cast<const uint2*>(l);
   }
 }
 
 // Mask words below the first evaluated row: all hot, all ones.
 __global__ void k_hot_words(uint32_t* __restrict__ mask, int words, int w0, int batch) {
+  pdl_wait();
+  pdl_trigger();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < batch * w0; i += gridDim.x * blockDim.x)
     mask[(size_t)(i / w0) * words + i % w0] = 0xFFFFFFFFu;
 }
@@ -893,9 +972,8 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
     return cudaErrorInvalidValue;
   cudaError_t e = cudaSuccess;
   if (!xh16_ready) {
-    k_xh16<<<std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s>>>(xh, batch, d, nt,
-                                                                                sc.xh16);
-    note_launch();
+    (void)launch_dep(k_xh16, std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s, xh,
+                     batch, d, nt, sc.xh16);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int nk = d / TC_BK, g = up_slots();
@@ -904,15 +982,12 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   auto kern = k_ffn_up_tc<NR>;
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  kern<<<up_grid(F), 32 * TC_FFN_WARPS, smem, s>>>(m0, m1, g0, g1, mx, nt, nk, g, H, F, idx, count,
-                                            sc.part, hdr);
-  note_launch();
+  (void)launch_dep(kern, up_grid(F), 32 * TC_FFN_WARPS, smem, s, m0, m1, g0, g1, mx, nt, nk, g, H,
+                   F, idx, count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  k_ffn_finish<NR><<<Fp / 64, 256, 0, s>>>(sc.part, g, nk, H, F, Fp, nt, batch, idx, count, L.bias,
-                                           mask, (F + 31) / 32, sc.h16, hdr,
-                                           L.act == PI_RELU2 ? 1 : 0);
-  note_launch();
+  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, H, F, Fp, nt, batch, idx,
+                   count, L.bias, mask, (F + 31) / 32, sc.h16, hdr, L.act == PI_RELU2 ? 1 : 0);
   return cudaGetLastError();
 }
 
@@ -947,7 +1022,8 @@ bool pred_tc_supported(const pi_layer& L, int batch) {
 }
 
 cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, float theta,
-                              uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s) {
+                              uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s,
+                              uint32_t* uni) {
   const int d = L.d_model, r = L.rank, F = L.d_ff, H = L.hot, words = (F + 31) / 32;
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, r);
@@ -960,8 +1036,8 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
       !map_2d(&mul, sc.ulo, (uint64_t)r, (uint64_t)nt, (uint64_t)r * 2, (uint32_t)nt))
     return cudaErrorInvalidValue;
   const int grid = device_sms() * 4;
-  k_split16<<<std::min((nt * d + 255) / 256, grid), 256, 0, s>>>(xh, batch, d, nt, sc.xh16, sc.xlo);
-  note_launch();
+  (void)launch_dep(k_split16, std::min((nt * d / 8 + 255) / 256, grid), 256, 0, s, xh, batch, d, nt,
+                   sc.xh16, sc.xlo);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   constexpr uint32_t STAGE = TC_M * TC_BK * 2 + 2 * TC_TMAX * TC_BK * 2;
@@ -971,28 +1047,24 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
   if (e != cudaSuccess) return e;
   // u = P1 xh
   const int ksu = pred_u_splits(d, r);
-  k_pred_tc<0><<<dim3(r / TC_M, ksu), TC_THREADS, smem, s>>>(m1, mxh, mxl, nt, d / TC_BK, ksu, 0, r,
-                                                             sc.upart, nullptr, 0.f, 0, nullptr, 0,
-                                                             batch, hdr);
-  note_launch();
+  (void)launch_dep(k_pred_tc<0>, dim3(r / TC_M, ksu), TC_THREADS, smem, s, m1, mxh, mxl, nt,
+                   d / TC_BK, ksu, 0, r, sc.upart, nullptr, 0.f, 0, nullptr, 0, batch, hdr,
+                   nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  k_pred_u_finish<<<std::min((r * nt + 255) / 256, grid), 256, 0, s>>>(sc.upart, ksu, r, nt, batch,
-                                                                       sc.uhi, sc.ulo);
-  note_launch();
+  (void)launch_dep(k_pred_u_finish, std::min((r / 4 * nt + 255) / 256, grid), 256, 0, s, sc.upart,
+                   ksu, r, nt, batch, sc.uhi, sc.ulo);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // z = P2 u + c for rows from the word holding `hot`; the words below it are hot
+  // z = P2 u + c for rows from the word holding `hot`; the words below it
+  // are hot (written by the z kernel, or here when every row is hot)
   const int w0 = H / 32, row0 = 32 * w0;
-  if (w0 > 0) {
-    k_hot_words<<<std::min((batch * w0 + 255) / 256, grid), 256, 0, s>>>(mask, words, w0, batch);
-    note_launch();
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
   if (row0 < F) {
     const int tiles = (F - row0 + TC_M - 1) / TC_M;
-    k_pred_tc<1><<<dim3(tiles, 1), TC_THREADS, smem, s>>>(m2, muh, mul, nt, r / TC_BK, 1, row0, F,
-                                                          nullptr, L.p_bias, theta, H, mask, words,
-                                                          batch, hdr);
-    note_launch();
+    (void)launch_dep(k_pred_tc<1>, dim3(tiles, 1), TC_THREADS, smem, s, m2, muh, mul, nt, r / TC_BK,
+                     1, row0, F, nullptr, L.p_bias, theta, H, mask, words, batch, hdr, uni);
+    e = cudaGetLastError();
+  } else {
+    (void)launch_dep(k_hot_words, std::min((batch * w0 + 255) / 256, grid), 256, 0, s, mask, words,
+                     w0, batch);
     e = cudaGetLastError();
   }
   return e;
@@ -1032,9 +1104,8 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
   const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
   cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_down_tc), smem);
   if (e != cudaSuccess) return e;
-  k_ffn_down_tc<<<dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s>>>(mwd, mwg, mh, nt, nk, ks, d, batch, H, F,
-                                                          idx, count, part, hdr);
-  note_launch();
+  (void)launch_dep(k_ffn_down_tc, dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s, mwd, mwg, mh, nt, nk,
+                   ks, d, batch, H, F, idx, count, part, hdr);
   return cudaGetLastError();
 }
 

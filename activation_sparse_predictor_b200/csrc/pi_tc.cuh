@@ -25,9 +25,12 @@ bool pred_tc_supported(const pi_layer& L, int batch);
 
 // mask [batch][words] of xh [batch][d_model]: u = P1 xh and z = P2[j] u + c
 // on the tensor cores with each fp32 vector split into two fp16 parts
-// (fp32 accumulation); bit j = j < hot or z_j > theta.
+// (fp32 accumulation); bit j = j < hot or z_j > theta.  `uni` (optional,
+// [words]): the OR of the tokens' words, written for the words from the
+// one holding `hot` on (the words below are not written).
 cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, float theta,
-                              uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s);
+                              uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s,
+                              uint32_t* uni = nullptr);
 
 // Up/gate products of list positions [0, hot + count) (row p for p < hot,
 // idx[p - hot] after) with xh [batch][d_model] (fp32, rounded to fp16 for
