@@ -121,7 +121,7 @@ struct WsLayout {
   size_t h;         // fp32 [F][B]        activations of listed rows
   size_t part;      // fp32 [S][B][d]     split-K partials
   size_t y;         // fp32 [B][d]        FFN output (stack)
-  size_t tc;        // tensor-core hot-prefix scratch (batches >= 16)
+  size_t tc;        // tensor-core scratch (fp16 layers at 2-64 tokens)
   size_t cta;       // u32  [SMs]         per-CTA list lengths (single-token kernel)
   size_t total;
   int splits;       // S

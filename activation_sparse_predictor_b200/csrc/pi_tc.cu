@@ -1,6 +1,6 @@
 // The FFN of a layer at token batches on the tensor cores (sm_100a).
 //
-// At 16-64 tokens the listed rows (the hot prefix [0, hot), then the cold
+// At 2-64 tokens the listed rows (the hot prefix [0, hot), then the cold
 // list idx) of every token batch form real contractions, both run as tcgen05
 // GEMMs over list positions p (row(p) = p for p < hot, idx[p - hot] after):
 //
@@ -64,6 +64,10 @@ constexpr int TC_FFN_WARPS = 8;  // warps of the FFN kernels: warp 1 issues the 
 constexpr int TC_PW = TC_FFN_WARPS - 1;  // load (warps 0-3 also drain the accumulators)
 constexpr int TC_KSMAX_D = 8;    // CTAs sharing one down tile's list positions at most
 constexpr int TC_TMAX = 64;      // tokens at most (MMA N)
+// Tokens at least: from two tokens on, one pass over the listed rows on the
+// tensor cores (the token tile padded to 16 with zero rows) costs less than
+// the CUDA-core kernels' passes; one token takes the CUDA-core kernels.
+constexpr int TC_MIN_BATCH = 2;
 constexpr unsigned long long kTcTimeoutNs = 1000000000ull;
 
 __device__ __forceinline__ uint32_t tc_sa(const void* p) {
@@ -995,7 +999,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
 
 bool ffn_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
-  if (L.w_dtype != PI_F16 || batch < 16 || batch > TC_TMAX) return false;
+  if (L.w_dtype != PI_F16 || batch < TC_MIN_BATCH || batch > TC_TMAX) return false;
   if (L.d_model % TC_M != 0) return false;
   const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
   const int64_t rd = code_stride(PI_F16, L.d_model, L.w_down_row_stride);
@@ -1009,13 +1013,13 @@ bool ffn_tc_supported(const pi_layer& L, int batch) {
 }
 
 size_t tc_scratch_bytes(int d_model, int d_ff, int rank, int batch) {
-  if (batch < 16 || d_model % TC_M != 0) return 0;
+  if (batch < TC_MIN_BATCH || d_model % TC_M != 0) return 0;
   return tc_scratch(nullptr, d_model, d_ff, rank).bytes;
 }
 
 bool pred_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
-  if (L.p_dtype != PI_F16 || batch < 16 || batch > TC_TMAX) return false;
+  if (L.p_dtype != PI_F16 || batch < TC_MIN_BATCH || batch > TC_TMAX) return false;
   if (L.rank % TC_M != 0 || L.d_model % TC_M != 0) return false;
   if (((uintptr_t)L.p1 | (uintptr_t)L.p2) & 15u) return false;
   return tensor_map_encoder() != nullptr;

@@ -161,7 +161,7 @@ pi_status pi_predict(const pi_layer* layer, const float* xh, int batch, float ta
  * library, one per device, of PI_PREDICT_NOALLOC_MAX_FLOATS floats (1 MiB).
  *   Kernels: always the CUDA-core predictor pair (u = p1 xh, then logits,
  *          threshold and mask), at every batch.  pi_predict takes the
- *          tensor-core predictor for fp16 predictors at 16-64 tokens, so at
+ *          tensor-core predictor for fp16 predictors at 2-64 tokens, so at
  *          those batches the two calls may set different bits for neurons
  *          whose logit lies within about 1e-4 of logit(tau); elsewhere they
  *          agree.  At other batches and dtypes the kernels, and so the

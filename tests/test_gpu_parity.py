@@ -154,6 +154,15 @@ def test_sparse_ffn(pi, orc, shape, act, wdt, batch, mode, packed):
         assert err <= TOL[wdt], (b, err)
 
 
+@pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
+@pytest.mark.parametrize("batch,mode", [(3, "per_token"), (5, "union"), (8, "per_token")])
+def test_sparse_ffn_cuda_cores_fp16(pi, orc, act, batch, mode, monkeypatch):
+    """fp16 layers at 2-15 tokens take the tensor cores; the CUDA-core
+    kernels (the path when those are unavailable) still match the oracle."""
+    monkeypatch.setenv("PI_DISABLE_TC", "1")
+    test_sparse_ffn(pi, orc, (1024, 3001, 128, 640), act, "f16", batch, mode, batch % 2 == 0)
+
+
 @pytest.mark.parametrize("act,wdt", KINDS)
 def test_sparse_ffn_edges(pi, orc, act, wdt):
     """Empty set (y == 0 exactly), everything cold listed, everything hot."""
@@ -298,16 +307,16 @@ def test_kernel_launch_counter(pi):
 @pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0),
                                    (4096, 1500, 64, 256), (8192, 1000, 64, 640)])
 @pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
-@pytest.mark.parametrize("batch,mode", [(16, "per_token"), (20, "union"), (48, "per_token"),
-                                        (64, "union")])
+@pytest.mark.parametrize("batch,mode", [(2, "per_token"), (5, "union"), (16, "per_token"),
+                                        (20, "union"), (48, "per_token"), (64, "union")])
 def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
-    """At 16-64 tokens an fp16 layer's listed rows (hot prefix and cold list;
+    """At 2-64 tokens an fp16 layer's listed rows (hot prefix and cold list;
     whole-hot tiles loaded as boxes, the others gathered four rows per TMA
     load) run on the tensor cores (fp16 inputs, fp32 accumulation): within
     the fp16 tolerance of the oracle, close to the CUDA-core path, and not
     bitwise equal to it (so the tensor-core path did run).  Shapes cover a
     ragged d_ff, a hot prefix that ends inside a tile, and no hot prefix;
-    batches 20 and 48 pad the token tile.  At d = 4096 and 8192 the up
+    batches 2, 5, 20 and 48 pad the token tile.  At d = 4096 and 8192 the up
     kernel splits d over 2 and 4 CTAs per row tile, and the down kernel
     splits a short list over 8 and 4 CTAs per column tile."""
     w = _wl(act, "f16", shape, seed=47)
@@ -343,10 +352,10 @@ def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
 
 
 @pytest.mark.parametrize("shape", [(1024, 3001, 256, 640), (512, 2048, 128, 200)])
-@pytest.mark.parametrize("batch", [16, 20, 64])
+@pytest.mark.parametrize("batch", [2, 7, 16, 20, 64])
 @pytest.mark.parametrize("tau", [0.5, 0.3])
 def test_predict_on_tensor_cores(pi, orc, shape, batch, tau, monkeypatch):
-    """At 16-64 tokens the fp16 predictor runs on the tensor cores with the
+    """At 2-64 tokens the fp16 predictor runs on the tensor cores with the
     fp32 vectors split into fp16 hi + lo parts: masks equal the oracle's
     outside the 1e-4 band (hot bits set, tail bits clear), including a hot
     prefix that ends inside a mask word, and equal the CUDA-core path's
