@@ -225,9 +225,13 @@ __device__ __forceinline__ int list_row(int p, int H, int N, int F, const int32_
   return (j >= H && j < F) ? j : 0;
 }
 
-// Ring stages of the up kernel: two operands (ReGLU) make a 40 KB stage, so
-// two stages keep two CTAs (80 KB each) on an SM.
-__host__ __device__ constexpr int up_stages(int nr) { return nr == 2 ? 2 : TC_STAGES; }
+// Ring stages of the up kernel by operand count and token tile, as many as
+// keep two CTAs (under 113 KB of shared memory each) on an SM: a stage is
+// NR 16 KB weight tiles and the activation tile (nt x 128 bytes, rounded to
+// the 1 KB swizzle atom).
+__host__ __device__ constexpr int up_stages(int nr, int nt) {
+  return nr == 1 ? (nt <= 32 ? 5 : 4) : (nt <= 32 ? 3 : 2);
+}
 
 // Work of the up kernel for a list of N positions: nT = ceil(N / 128) row
 // tiles, each split over ks shares of d (nk k tiles) so that nT * ks CTAs
@@ -251,7 +255,7 @@ __host__ __device__ inline UpShare up_share(int N, int g, int nk) {
 // up: NR = 1 ReLU (W_up), NR = 2 ReGLU (W_gate, W_up).  One-dimensional
 // grid of at least g CTAs; CTA b takes tile b / ks, share b % ks of
 // up_share(N, g, nk) and exits past nT * ks.  part: [ks][NR][nT * 128][nt] fp32.
-template <int NR>
+template <int NR, int NS>
 __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     k_ffn_up_tc(const __grid_constant__ CUtensorMap mw0, const __grid_constant__ CUtensorMap mw1,
                 const __grid_constant__ CUtensorMap mg0, const __grid_constant__ CUtensorMap mg1,
@@ -261,10 +265,8 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   pdl_wait();
   pdl_trigger();
   constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
-  constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;  // 8 KB (nt rows used)
-  constexpr uint32_t STAGE = NR * A_BYTES + B_BYTES;
+  const uint32_t STAGE = NR * A_BYTES + (((uint32_t)nt * TC_BK * 2 + 1023u) & ~1023u);
   constexpr uint32_t NCOLS = NR == 1 ? 64u : 128u;   // >= NR * nt, a power of two
-  constexpr int NS = up_stages(NR);
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = tc_sa(smem_raw);
   unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // swizzle atoms: 1 KB aligned
@@ -981,9 +983,11 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   const int nk = d / TC_BK, g = up_slots();
-  constexpr uint32_t STAGE = NR * TC_M * TC_BK * 2 + TC_TMAX * TC_BK * 2;
-  const size_t smem = 1024 + (size_t)up_stages(NR) * STAGE + 8 * (2 * up_stages(NR) + 1) + 16 + 4 * TC_M;
-  auto kern = k_ffn_up_tc<NR>;
+  const int NS = up_stages(NR, nt);
+  const uint32_t stage = NR * TC_M * TC_BK * 2 + (((uint32_t)nt * TC_BK * 2 + 1023u) & ~1023u);
+  const size_t smem = 1024 + (size_t)NS * stage + 8 * (2 * NS + 1) + 16 + 4 * TC_M;
+  auto kern = NS == up_stages(NR, 64) ? k_ffn_up_tc<NR, up_stages(NR, 64)>
+                                      : k_ffn_up_tc<NR, up_stages(NR, 16)>;
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   (void)launch_dep(kern, up_grid(F), 32 * TC_FFN_WARPS, smem, s, m0, m1, g0, g1, mx, nt, nk, g, H,
