@@ -491,20 +491,24 @@ def run_pi(args, world, rank, local):
         pi.pi_read_counters(ws, clear=True, stream=stream)
         resident = K * B / (r0.elapsed_time(r1) / 1000.0)
 
-    # bytes actually read per step (predictor + listed rows + nonzero down rows)
-    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * nl, rows_second)
-    step_bytes = sum(by.values()) / K
-    peak, peak_kind = hbm_peak()
-    step_gbs = step_bytes / (ms / K / 1000.0) / 1e9
-
     # ---- per-kernel device times: one profiled pass over the same step inputs
     x.copy_(xs[W])
     pi.pi_read_counters(ws, clear=True, stream=stream)
     prof = pi.pi_ffn_stack_profile(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
     pr_listed, pr_down, pr_second = pi.pi_read_counters(ws, clear=True, stream=stream)
-    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, nl, pr_second)
-    pby["fused_stack"] = sum(pby.values())  # the fused kernel runs every step
     prof = {k: v for k, v in prof.items() if v[1] > 0}
+    # the persistent kernel alone at several tokens (Q4_0 stacks with
+    # per-token masks) makes one pass over the stack per token, so the
+    # predictor and the per-layer vectors are read once per layer and token
+    passes = B if (B > 1 and set(prof) == {"fused_stack"}) else 1
+
+    # bytes actually read per step (predictor + listed rows + nonzero down rows)
+    by = layer_algorithmic_bytes(w, rows_listed, rows_down, K * nl * passes, rows_second)
+    step_bytes = sum(by.values()) / K
+    peak, peak_kind = hbm_peak()
+    step_gbs = step_bytes / (ms / K / 1000.0) / 1e9
+    pby = layer_algorithmic_bytes(w, pr_listed, pr_down, nl * passes, pr_second)
+    pby["fused_stack"] = sum(pby.values())  # the fused kernel runs every step
     dom = max(prof, key=lambda k: prof[k][0])
     dom_ms, dom_n = prof[dom]
     if len(prof) == 1:
@@ -523,7 +527,7 @@ def run_pi(args, world, rank, local):
     tpl = measured_traffic_per_layer(w.name) if dom == "fused_stack" else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peak,
                 "unit": "GB/s", "frac": achieved / peak, "peak_source": peak_kind,
-                "traffic": tpl * nl / dom_n if tpl is not None else None,
+                "traffic": tpl * nl * passes / dom_n if tpl is not None else None,
                 "algorithmic_bytes_per_launch": dom_bytes_per_launch,
                 "avg_launch_us": 1000.0 * dom_ms / dom_n, "timing_source": timing_source,
                 "per_kind_ms_per_step": {k: v[0] for k, v in prof.items()},

@@ -288,7 +288,7 @@ def test_stack_is_deterministic(pi, packed):
 
 def test_kernel_launch_counter(pi):
     """One fused launch per batch-1 stack call of at most 24 layers; the same
-    count on every repeat of a multi-kernel (batch 4) call."""
+    count on every repeat of a multi-kernel (batch 4, union) call."""
     w = _wl("reglu", "q4_0", (512, 1500, 64, 256), seed=44).scaled(4)
     layers = [device_layer(w, l, packed=True)[0] for l in range(4)]
     x = torch.from_numpy(synth.x_host(w, 0, 1)).cuda()
@@ -299,9 +299,30 @@ def test_kernel_launch_counter(pi):
     counts = []
     for _ in range(2):
         n0 = pi.pi_kernel_launches()
-        pi.pi_ffn_stack(layers, xb, 0.5, pi.PI_MASK_PER_TOKEN)
+        pi.pi_ffn_stack(layers, xb, 0.5, pi.PI_MASK_UNION)
         counts.append(pi.pi_kernel_launches() - n0)
     assert counts[0] == counts[1] >= 4 * 6  # per layer: norm, predictor, compaction, FFN, reduce
+
+
+@pytest.mark.parametrize("act", ["reglu", "relu2"])
+@pytest.mark.parametrize("batch", [2, 5])
+def test_q4_per_token_stack_is_one_fused_pass_per_token(pi, act, batch):
+    """A Q4_0 stack at 2-15 tokens with per-token masks (no mask trace) runs
+    one persistent single-token pass per token: one launch per token, and
+    every token's result bit-identical to a batch-1 call on it (the batched
+    kernels, taken when a mask trace is asked for, are checked against the
+    oracle by test_stack)."""
+    w = _wl(act, "q4_0", (512, 1500, 64, 256), seed=45, mean=0.15).scaled(4)
+    layers = [device_layer(w, l, packed=True)[0] for l in range(4)]
+    x0 = torch.from_numpy(synth.x_host(w, 0, batch)).cuda()
+    x = x0.clone()
+    n0 = pi.pi_kernel_launches()
+    pi.pi_ffn_stack(layers, x, 0.5, pi.PI_MASK_PER_TOKEN)
+    assert pi.pi_kernel_launches() - n0 == batch
+    for b in range(batch):
+        xb = x0[b:b + 1].clone()
+        pi.pi_ffn_stack(layers, xb, 0.5, pi.PI_MASK_PER_TOKEN)
+        assert torch.equal(xb[0], x[b]), b
 
 
 @pytest.mark.parametrize("shape", [(1024, 3001, 128, 640), (256, 1000, 64, 200), (512, 2048, 64, 0),
