@@ -392,6 +392,386 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
                  : "memory");
 }
 
+// ------------------------------------------------------------------ Q4_0
+// Q4_0 weights on the tensor cores.  The listed rows' codes and scales are
+// loaded by 256 threads with vector loads, TC_Q4_PRE stages ahead in
+// registers, decoded to fp16 (q - 8) * s and stored into the 128-byte
+// swizzled operand tile of the ring; each thread fences its stores for
+// the tensor cores' (async) proxy and arrives on the stage's barrier, which
+// completes when all 256 have arrived and the activation tile's TMA bytes
+// have landed.  Warp 8 issues the MMAs; warps 8-11 drain the accumulators.
+constexpr int TC_Q4_WARPS = 12;
+constexpr int TC_Q4_LOADERS = 256;  // threads 0..255 load and decode
+constexpr int TC_Q4_PRE = 4;        // stages of codes each loader holds ahead
+
+// Elements 8c .. 8c+7 of a Q4_0 block (16 code bytes: byte k holds element
+// k in its low nibble and element k + 16 in its high nibble) as eight fp16
+// values (q - 8) * s: c = 0, 1 take the low nibbles of bytes 8c .. 8c+7,
+// c = 2, 3 the high nibbles of bytes 8(c-2) ..  A nibble n becomes the
+// fp16 number 1024 + n (0x6400 | n) by a byte permute, from which 1032 is
+// subtracted exactly; the product with the scale is rounded once.
+__device__ __forceinline__ uint4 q4_chunk_f16(uint32_t w0, uint32_t w1, bool high, __half2 s2) {
+  if (high) {
+    w0 >>= 4;
+    w1 >>= 4;
+  }
+  w0 &= 0x0F0F0F0Fu;
+  w1 &= 0x0F0F0F0Fu;
+  const uint32_t p[4] = {__byte_perm(w0, 0x64u, 0x4140), __byte_perm(w0, 0x64u, 0x4342),
+                         __byte_perm(w1, 0x64u, 0x4140), __byte_perm(w1, 0x64u, 0x4342)};
+  const __half2 off = __half2half2(__ushort_as_half((unsigned short)0x6408u));  // 1032
+  uint32_t r[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 v = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&p[k]), off), s2);
+    r[k] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+  return make_uint4(r[0], r[1], r[2], r[3]);
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(tc_sa(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_release(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(tc_sa(bar)) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Q4_0 up/gate: as k_ffn_up_tc (grid, work shares, part layout), with
+// K = 128 per stage (two 64-column atoms) and NS = 2 ring stages.  Loader
+// thread t decodes blocks 2h, 2h + 1 of row t / 2 (h = t % 2) in each
+// operand: 32 contiguous code bytes and two scales per operand and stage.
+template <int NR>
+__global__ void __launch_bounds__(32 * TC_Q4_WARPS, NR == 1 ? 2 : 1)
+    k_ffn_up_q4tc(const __grid_constant__ CUtensorMap mx, const char* __restrict__ cw0,
+                  const char* __restrict__ sw0, int64_t cst0, int64_t sst0,
+                  const char* __restrict__ cw1, const char* __restrict__ sw1, int64_t cst1,
+                  int64_t sst1, int nt, int nk, int g, int H, int F,
+                  const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
+                  float* __restrict__ part, WsHeader* hdr) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NS = 2;
+  constexpr uint32_t AT = TC_M * 128;  // one 64-column atom of a 128-row tile: 16 KB
+  constexpr uint32_t NCOLS = NR == 1 ? 64u : 128u;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = tc_sa(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t batom = (uint32_t)nt * 128u;  // one 64-column atom of the activation tile
+  const uint32_t STAGE = NR * 2 * AT + ((2 * batom + 1023u) & ~1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STAGE);
+  uint64_t* empty = full + NS;
+  uint64_t* done = empty + NS;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int N = list_len(count, H, F, hdr);
+  const UpShare us = up_share(N, g, nk);
+  const int ks = us.ks, Np = us.nT * TC_M;
+  if ((int)blockIdx.x >= us.nT * ks) return;
+  const int tile = blockIdx.x / ks, split = blockIdx.x % ks;
+  const int p0 = tile * TC_M;
+  const int kt0 = (int)((long long)split * nk / ks), kt1 = (int)((long long)(split + 1) * nk / ks);
+  const int nkt = kt1 - kt0;
+
+  if (threadIdx.x == 0) tc_init(full, empty, done, abort, NS, (uint32_t)TC_Q4_LOADERS);
+  if (warp == 0) tmem_alloc(tslot, NCOLS);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tslot;
+
+  if (threadIdx.x < TC_Q4_LOADERS) {
+    const int t = threadIdx.x, m = t >> 1, h = t & 1;
+    const int row = list_row(p0 + m, H, N, F, idx);
+    const char* cp[2] = {cw0 + (size_t)row * cst0, NR == 2 ? cw1 + (size_t)row * cst1 : nullptr};
+    const char* sp[2] = {sw0 + (size_t)row * sst0, NR == 2 ? sw1 + (size_t)row * sst1 : nullptr};
+    uint4 cq[TC_Q4_PRE][NR][2];
+    uint32_t sq[TC_Q4_PRE][NR];
+    // codes and scales of stage i into register slot u
+    auto fetch = [&](int i, int u) {
+      if (i < nkt) {
+        const size_t kb = (size_t)(kt0 + i) * 64 + (size_t)h * 32;  // code bytes
+        const size_t sb = (size_t)(kt0 + i) * 8 + (size_t)h * 4;    // scale bytes
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          cq[u][r][0] = ld_stream16(cp[r] + kb);
+          cq[u][r][1] = ld_stream16(cp[r] + kb + 16);
+          sq[u][r] = __ldg(reinterpret_cast<const uint32_t*>(sp[r] + sb));
+        }
+      }
+    };
+#pragma unroll
+    for (int u = 0; u < TC_Q4_PRE; ++u) fetch(u, u);
+    const uint32_t sm0 = tc_sa(smem);
+    bool stop = false;
+    int last = -1;  // thread 0: the last stage whose activation tile it loaded
+    for (int i0 = 0; i0 < nkt && !stop; i0 += TC_Q4_PRE) {
+#pragma unroll
+      for (int u = 0; u < TC_Q4_PRE; ++u) {
+        const int i = i0 + u;
+        if (i >= nkt) break;
+        const int st = u % NS;  // i % NS (TC_Q4_PRE is a multiple of NS)
+        int ok = 1;
+        if (lane == 0 && i >= NS) ok = tc_wait(&empty[st], ((i / NS) - 1) & 1, abort, hdr);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        unsigned char* a = smem + st * STAGE;
+        if (t == 0) {
+          mbar_expect_tx(&full[st], 2 * batom);
+          const int k = (kt0 + i) * 128;
+          tma_load_2d(a + NR * 2 * AT, &mx, k, 0, &full[st]);
+          tma_load_2d(a + NR * 2 * AT + batom, &mx, k + 64, 0, &full[st]);
+          last = i;
+        }
+        const uint32_t abase = sm0 + (uint32_t)st * STAGE + (uint32_t)h * AT + (uint32_t)m * 128u;
+#pragma unroll
+        for (int r = 0; r < NR; ++r) {
+          const uint32_t ar = abase + (uint32_t)r * 2 * AT;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t sbits = q ? (sq[u][r] >> 16) : (sq[u][r] & 0xFFFFu);
+            const __half2 s2 = __half2half2(__ushort_as_half((unsigned short)sbits));
+            const uint4 v = cq[u][r][q];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 o = q4_chunk_f16(c & 1 ? v.z : v.x, c & 1 ? v.w : v.y, c >= 2, s2);
+              const uint32_t cc = (uint32_t)(4 * q + c);
+              sts128(ar + ((cc ^ (uint32_t)(m & 7)) << 4), o);
+            }
+          }
+        }
+        fence_async_smem();
+        mbar_arrive_release(&full[st]);
+        fetch(i + TC_Q4_PRE, u);
+      }
+    }
+    if (t == 0 && last >= 0) {  // the activation tiles it loaded have landed (bounded)
+      for (int i = last; i >= 0 && i > last - NS; --i)
+        (void)tc_wait_quiet(&full[i % NS], (uint32_t)(i / NS) & 1u, hdr);
+    }
+  } else if (warp == 8 && lane == 0) {
+    // kind::f16, fp16 A and B, both K-major, M = 128, N = nt
+    const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % NS;
+      if (!tc_wait(&full[st], (uint32_t)(i / NS) & 1u, abort, hdr)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = tc_sa(smem + st * STAGE), b = a + NR * 2 * AT;
+#pragma unroll
+      for (int at = 0; at < 2; ++at)
+#pragma unroll
+        for (int kk = 0; kk < TC_BK / 16; ++kk) {
+          const uint64_t bd = sw128_desc(b + (uint32_t)at * batom + 32u * kk);
+          const uint32_t acc = (i | at | kk) != 0 ? 1u : 0u;
+#pragma unroll
+          for (int r = 0; r < NR; ++r)
+            mma_f16(tmem + (uint32_t)(r * nt), sw128_desc(a + (uint32_t)(r * 2 + at) * AT + 32u * kk),
+                    bd, idesc, acc);
+        }
+      mma_commit(&empty[st]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  bool ok = tc_wait_quiet(done, 0u, hdr);
+  ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (ok && warp >= 8) {
+    const int e = warp - 8;
+    const int p = p0 + e * 32 + lane;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      float* dst = part + ((size_t)(split * NR + r) * Np + p) * nt;
+      for (int c0 = 0; c0 < nt; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(e * 32) << 16) + (uint32_t)(r * nt + c0), v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          __stcg(reinterpret_cast<float4*>(dst + c0) + q,
+                 make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                             __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS)
+                 : "memory");
+}
+
+// Q4_0 down: as k_ffn_down_tc (grid (d / 128, ks), the k tiles that hold
+// list positions split evenly over the ks CTAs of a column tile, part rows
+// [split][b][c]), with the MN-major operand tile decoded from W_down^T's
+// Q4_0 rows: loader t takes list position t / 4 of the stage's 64 and
+// columns c0 + 32 (t % 4) .. +31 of it (one block: 16 code bytes and a
+// scale).  The list rows are loaded one stage before
+// the codes that depend on them, the codes TC_Q4_PRE - 1 stages ahead.
+__global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
+    k_ffn_down_q4tc(const __grid_constant__ CUtensorMap mh, const char* __restrict__ cw,
+                    const char* __restrict__ sw, int64_t cst, int64_t sst, int nt, int ks, int d,
+                    int batch, int H, int F, const int32_t* __restrict__ idx,
+                    const int32_t* __restrict__ count, float* __restrict__ part, WsHeader* hdr) {
+  pdl_wait();
+  pdl_trigger();
+  constexpr int NS = 4;
+  constexpr uint32_t BOX = 64 * TC_BK * 2;  // 64 columns x 64 positions: 8 KB
+  constexpr uint32_t A_BYTES = 2 * BOX;     // 128 columns
+  constexpr uint32_t NCOLS = 64u;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = tc_sa(smem_raw);
+  unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
+  const uint32_t STAGE = A_BYTES + ((bx + 1023u) & ~1023u);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STAGE);
+  uint64_t* empty = full + NS;
+  uint64_t* done = empty + NS;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const int N = list_len(count, H, F, hdr);
+  const int nkN = (N + TC_BK - 1) / TC_BK;  // k tiles holding list positions
+  const int kt0 = (int)((long long)split * nkN / ks);
+  const int kt1 = (int)((long long)(split + 1) * nkN / ks);
+  const int nkt = kt1 > kt0 ? kt1 - kt0 : 0;
+  const int c0 = tile * TC_M;
+
+  if (threadIdx.x == 0) {
+    tc_init(full, empty, done, abort, NS, (uint32_t)TC_Q4_LOADERS);
+    if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)N);
+  }
+  if (warp == 0) tmem_alloc(tslot, NCOLS);
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tslot;
+
+  if (threadIdx.x < TC_Q4_LOADERS) {
+    const int t = threadIdx.x, k = t >> 2, q = t & 3;  // position in the stage, column block
+    const size_t cb = (size_t)(c0 + 32 * q) / 2;       // code bytes of the block in a row
+    const size_t sb = (size_t)(c0 + 32 * q) / 32 * 2;  // scale bytes
+    int rq[TC_Q4_PRE];       // list rows, one slot per stage
+    uint4 cq[TC_Q4_PRE];     // codes
+    uint16_t sq[TC_Q4_PRE];  // scales
+    auto row_of = [&](int i) { return i < nkt ? list_row((kt0 + i) * TC_BK + k, H, N, F, idx) : 0; };
+    auto fetch = [&](int i, int u) {
+      if (i < nkt) {
+        cq[u] = ld_stream16(cw + (size_t)rq[u] * cst + cb);
+        sq[u] = __ldg(reinterpret_cast<const unsigned short*>(sw + (size_t)rq[u] * sst + sb));
+      }
+    };
+#pragma unroll
+    for (int u = 0; u < TC_Q4_PRE; ++u) rq[u] = row_of(u);
+#pragma unroll
+    for (int u = 0; u < TC_Q4_PRE - 1; ++u) fetch(u, u);
+    const uint32_t sm0 = tc_sa(smem);
+    const uint32_t h = (uint32_t)(q >> 1), cbase = (uint32_t)(4 * (q & 1));
+    bool stop = false;
+    int last = -1;
+    for (int i0 = 0; i0 < nkt && !stop; i0 += TC_Q4_PRE) {
+#pragma unroll
+      for (int u = 0; u < TC_Q4_PRE; ++u) {
+        const int i = i0 + u;
+        if (i >= nkt) break;
+        // the codes of stage i + PRE - 1 (their row came one stage ago), then
+        // the row of stage i + PRE into the slot this stage frees
+        const int un = (u + TC_Q4_PRE - 1) % TC_Q4_PRE;
+        fetch(i + TC_Q4_PRE - 1, un);
+        const int st = u % NS;
+        int ok = 1;
+        if (lane == 0 && i >= NS) ok = tc_wait(&empty[st], ((i / NS) - 1) & 1, abort, hdr);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
+        unsigned char* a = smem + st * STAGE;
+        if (t == 0) {
+          mbar_expect_tx(&full[st], bx);
+          tma_load_2d(a + A_BYTES, &mh, 0, (kt0 + i) * nt, &full[st]);
+          last = i;
+        }
+        const __half2 s2 = __half2half2(__ushort_as_half(sq[u]));
+        const uint4 v = cq[u];
+        const uint32_t ab = sm0 + (uint32_t)st * STAGE + h * BOX + (uint32_t)k * 128u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 o = q4_chunk_f16(c & 1 ? v.z : v.x, c & 1 ? v.w : v.y, c >= 2, s2);
+          sts128(ab + (((cbase + (uint32_t)c) ^ (uint32_t)(k & 7)) << 4), o);
+        }
+        fence_async_smem();
+        mbar_arrive_release(&full[st]);
+        rq[u] = row_of(i + TC_Q4_PRE);
+      }
+    }
+    if (t == 0 && last >= 0) {
+      for (int i = last; i >= 0 && i > last - NS; --i)
+        (void)tc_wait_quiet(&full[i % NS], (uint32_t)(i / NS) & 1u, hdr);
+    }
+  } else if (warp == 8 && lane == 0) {
+    // kind::f16, fp16 A (MN-major) and B (K-major), fp32 D, M = 128, N = nt
+    const uint32_t idesc = (1u << 4) | (1u << 15) | ((uint32_t)(nt >> 3) << 17) |
+                           ((uint32_t)(TC_M >> 4) << 24);
+    for (int i = 0; i < nkt; ++i) {
+      const int st = i % NS;
+      if (!tc_wait(&full[st], (uint32_t)(i / NS) & 1u, abort, hdr)) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t a = tc_sa(smem + st * STAGE), b = a + A_BYTES;
+#pragma unroll
+      for (int kk = 0; kk < TC_BK / 16; ++kk)
+        mma_f16(tmem, sw128_mn_desc(a + 2048u * kk, BOX), sw128_desc(b + 32u * kk), idesc,
+                (i | kk) != 0 ? 1u : 0u);
+      mma_commit(&empty[st]);
+    }
+    mma_commit(done);
+  }
+  __syncwarp();
+
+  bool ok = tc_wait_quiet(done, 0u, hdr);
+  ok = __all_sync(0xffffffffu, ok && !*abort);
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  // accumulator lane = output column, accumulator column = token; a split
+  // with no list positions writes zeros (the reduction sums every slice)
+  if (warp >= 8) {
+    const int e = warp - 8;
+    const int c = c0 + e * 32 + lane;
+    for (int t0 = 0; t0 < nt; t0 += 16) {
+      uint32_t v[16];
+      if (ok && nkt > 0) {
+        tmem_ld16(tmem + ((uint32_t)(e * 32) << 16) + (uint32_t)t0, v);
+      } else {
+#pragma unroll
+        for (int tt = 0; tt < 16; ++tt) v[tt] = 0u;
+      }
+#pragma unroll
+      for (int tt = 0; tt < 16; ++tt)
+        if (t0 + tt < batch) __stcg(part + ((size_t)split * batch + t0 + tt) * d + c, __uint_as_float(v[tt]));
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NCOLS)
+                 : "memory");
+}
+
 // xh (fp32 [batch][d]) -> xh16 (fp16 [nt][d], rows >= batch zero); 8 per thread.
 __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
                        __half* __restrict__ xh16) {
@@ -999,12 +1379,68 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   return cudaGetLastError();
 }
 
+// Q4_0 up/gate (k_ffn_up_q4tc) and the same finish kernel.  CTA slots: two
+// per SM for one operand (two 48 KB stages at most), one for two (160 KB).
+template <int NR>
+cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
+                         const int32_t* idx, const int32_t* count, void* scratch, WsHeader* hdr,
+                         cudaStream_t s, bool xh16_ready) {
+  const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
+  const int nt = (batch + 15) / 16 * 16;
+  const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
+  const int64_t ur = NR == 2 && L.w_up_row_stride ? L.w_up_row_stride : L.w_row_stride;
+  const char* cw0 = static_cast<const char*>(NR == 2 ? L.w_gate : L.w_up);
+  const char* sw0 = static_cast<const char*>(NR == 2 ? L.w_gate_scales : L.w_up_scales);
+  CUtensorMap mx;
+  if (!map_2d(&mx, sc.xh16, (uint64_t)d, (uint64_t)nt, (uint64_t)d * 2, (uint32_t)nt))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaSuccess;
+  if (!xh16_ready) {
+    (void)launch_dep(k_xh16, std::min((nt * d / 8 + 255) / 256, device_sms() * 4), 256, 0, s, xh,
+                     batch, d, nt, sc.xh16);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const int nk = d / 128, g = (NR == 1 ? 2 : 1) * device_sms();
+  const uint32_t stage = NR * 2 * TC_M * 128 + (((uint32_t)nt * 256 + 1023u) & ~1023u);
+  const size_t smem = 1024 + 2 * (size_t)stage + 8 * (2 * 2 + 1) + 16;
+  e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_up_q4tc<NR>), smem);
+  if (e != cudaSuccess) return e;
+  (void)launch_dep(k_ffn_up_q4tc<NR>, std::max(g, Fp / TC_M), 32 * TC_Q4_WARPS, smem, s, mx, cw0,
+                   sw0, code_stride(PI_Q4_0, d, L.w_row_stride), scale_stride(d, L.w_row_stride),
+                   static_cast<const char*>(L.w_up), static_cast<const char*>(L.w_up_scales),
+                   code_stride(PI_Q4_0, d, ur), scale_stride(d, ur), nt, nk, g, H, F, idx, count,
+                   sc.part, hdr);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, H, F, Fp, nt, batch, idx,
+                   count, L.bias, mask, (F + 31) / 32, sc.h16, hdr, L.act == PI_RELU2 ? 1 : 0);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool ffn_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
-  if (L.w_dtype != PI_F16 || batch < TC_MIN_BATCH || batch > TC_TMAX) return false;
+  if ((L.w_dtype != PI_F16 && L.w_dtype != PI_Q4_0) || batch < TC_MIN_BATCH || batch > TC_TMAX)
+    return false;
   if (L.d_model % TC_M != 0) return false;
+  if (L.w_dtype == PI_Q4_0) {
+    // 16-byte code loads, 4-byte scale loads (two scales at a time)
+    const int d = L.d_model;
+    const int64_t ur = L.act == PI_REGLU && L.w_up_row_stride ? L.w_up_row_stride : L.w_row_stride;
+    const int64_t cs[3] = {code_stride(PI_Q4_0, d, L.w_row_stride), code_stride(PI_Q4_0, d, ur),
+                           code_stride(PI_Q4_0, d, L.w_down_row_stride)};
+    const int64_t ss[3] = {scale_stride(d, L.w_row_stride), scale_stride(d, ur),
+                           scale_stride(d, L.w_down_row_stride)};
+    for (int k = 0; k < 3; ++k)
+      if (cs[k] % 16 != 0 || ss[k] % 4 != 0) return false;
+    const uintptr_t codes = (uintptr_t)L.w_up | (uintptr_t)L.w_down_t |
+                            (uintptr_t)(L.act == PI_REGLU ? L.w_gate : L.w_up);
+    const uintptr_t scales = (uintptr_t)L.w_up_scales | (uintptr_t)L.w_down_t_scales |
+                             (uintptr_t)(L.act == PI_REGLU ? L.w_gate_scales : L.w_up_scales);
+    if ((codes & 15u) || (scales & 3u)) return false;
+    return tensor_map_encoder() != nullptr;
+  }
   const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
   const int64_t rd = code_stride(PI_F16, L.d_model, L.w_down_row_stride);
   const int64_t ru = code_stride(PI_F16, L.d_model, L.w_up_row_stride ? L.w_up_row_stride
@@ -1089,6 +1525,10 @@ int ffn_tc_down_splits(const pi_layer& L) {
 cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                              const int32_t* idx, const int32_t* count, void* scratch,
                              WsHeader* hdr, cudaStream_t s, bool xh16_ready) {
+  if (L.w_dtype == PI_Q4_0)
+    return L.act == PI_REGLU
+               ? launch_up_q4<2>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready)
+               : launch_up_q4<1>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready);
   return L.act == PI_REGLU
              ? launch_up_nr<2>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready)
              : launch_up_nr<1>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready);
@@ -1100,6 +1540,24 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
   const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
+  if (L.w_dtype == PI_Q4_0) {
+    CUtensorMap mh;
+    if (!map_2d(&mh, sc.h16, (uint64_t)TC_BK, (uint64_t)(Fp / TC_BK) * nt, (uint64_t)TC_BK * 2,
+                (uint32_t)nt))
+      return cudaErrorInvalidValue;
+    const int tiles = d / TC_M, ks = ffn_tc_down_splits(L);
+    const uint32_t stage = 2 * 64 * TC_BK * 2 + (((uint32_t)nt * TC_BK * 2 + 1023u) & ~1023u);
+    const size_t smem = 1024 + 4 * (size_t)stage + 8 * (2 * 4 + 1) + 16;
+    cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_down_q4tc), smem);
+    if (e != cudaSuccess) return e;
+    (void)launch_dep(k_ffn_down_q4tc, dim3(tiles, ks), 32 * TC_Q4_WARPS, smem, s, mh,
+                     static_cast<const char*>(L.w_down_t),
+                     static_cast<const char*>(L.w_down_t_scales),
+                     code_stride(PI_Q4_0, d, L.w_down_row_stride),
+                     scale_stride(d, L.w_down_row_stride), nt, ks, d, batch, H, F, idx, count,
+                     part, hdr);
+    return cudaGetLastError();
+  }
   const int64_t rd = code_stride(PI_F16, d, L.w_down_row_stride);
   CUtensorMap mwd, mwg, mh;
   if (!map_2d(&mwd, L.w_down_t, (uint64_t)d, (uint64_t)F, (uint64_t)rd, TC_BK) ||

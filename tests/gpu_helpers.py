@@ -32,14 +32,15 @@ def unpack_bits(words: np.ndarray, n: int) -> np.ndarray:
     return bits[:n].astype(bool), bits[n:]
 
 
-def check_mask(gpu_words: np.ndarray, z_ref: np.ndarray, F: int, H: int, theta: float):
+def check_mask(gpu_words: np.ndarray, z_ref: np.ndarray, F: int, H: int, theta: float,
+               band: float = BAND):
     """GPU mask == oracle decision outside the band; tail bits zero.
     Returns the number of (allowed) disagreements inside the band."""
     got, tail = unpack_bits(gpu_words, F)
     j = np.arange(F)
     want = (j < H) | ((j >= H) & (z_ref > theta))
     diff = got != want
-    allowed = (j >= H) & (np.abs(z_ref - theta) <= BAND)
+    allowed = (j >= H) & (np.abs(z_ref - theta) <= band)
     bad = diff & ~allowed
     assert not bad.any(), f"mask mismatch outside the band at neurons {np.flatnonzero(bad)[:10]}"
     assert not tail.any(), "bits beyond d_ff must be 0"

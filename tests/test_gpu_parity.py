@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 
 from activation_sparse_predictor_b200 import synth
-from gpu_helpers import TOL, check_mask, device_layer, pi_mod, unpack_bits, words_np
+from gpu_helpers import BAND, TOL, check_mask, device_layer, pi_mod, unpack_bits, words_np
 from helpers import small_workload
 from oracle import rel_l2
 
@@ -229,6 +229,13 @@ def test_device_checks_flag_bad_lists(pi, orc):
                                         (8, "per_token"), (8, "union")])
 @pytest.mark.parametrize("packed", [False, True])
 def test_stack(pi, orc, act, wdt, batch, mode, packed):
+    """Stacks of 3 layers against the oracle, layer by layer.  The oracle
+    runs each layer on the GPU's own masks (from the mask trace), so the
+    final x checks the FFN arithmetic of the whole chain; each GPU mask is
+    checked against the oracle's logits, exactly outside the 1e-4 band in
+    the first layer (same inputs) and outside a band scaled to the path's
+    tolerance in later layers, whose inputs differ by the earlier layers'
+    rounding (fp16 operands on the tensor cores from 2 tokens on)."""
     w = _wl(act, wdt, (512, 1500, 64, 256), seed=43, mean=0.15).scaled(3)
     dev = [device_layer(w, l, packed=packed) for l in range(w.n_layers)]
     host = [synth.layer_host(w, l) for l in range(w.n_layers)]
@@ -239,38 +246,19 @@ def test_stack(pi, orc, act, wdt, batch, mode, packed):
     pi.pi_ffn_stack([L for L, _ in dev], x, 0.5, pi.MODES[mode], mask_trace=trace)
     xg = x.cpu().numpy()
     tr = trace.cpu().numpy().view(np.uint32)
-    for b in range(batch):
-        if mode == "union" and batch > 1:
-            continue  # union chains couple tokens; checked token-coupled below
-        xr = x0[b].astype(np.float64)
-        for l in range(w.n_layers):
-            xo, m, z = orc.layer_forward(host[l], xr.astype(np.float32), 0.5)
-            flips = check_mask(tr[l, b], z, w.d_ff, w.hot, 0.0)
-            assert flips == 0, "a band flip makes the chains diverge; pick another seed"
-            xr = xo
-        assert rel_l2(xg[b] - x0[b], xr - x0[b]) <= TOL[wdt]
-    if mode == "union" and batch > 1:
-        _check_union_stack(orc, host, x0, xg, tr, w)
-
-
-def _check_union_stack(orc, host, x0, xg, tr, w):
-    """Union chains: every token's FFN runs over the union of the batch's sets."""
-    B = x0.shape[0]
+    union = mode == "union" and batch > 1
     xs = x0.astype(np.float64)
     for l, H in enumerate(host):
-        ms = []
-        xh = []
-        for b in range(B):
-            xhb = orc.rmsnorm(xs[b].astype(np.float32))
-            _, z = orc.predict(H, xhb)
-            assert check_mask(tr[l, b], z, w.d_ff, w.hot, 0.0) == 0
-            ms.append(orc.mask(z, w.d_ff, w.hot, 0.0))
-            xh.append(xhb)
-        union = orc.compact(np.stack(ms), w.d_ff, w.hot)
+        band = BAND if l == 0 else max(BAND, 4 * TOL[wdt])
+        xh = [orc.rmsnorm(xs[b].astype(np.float32)) for b in range(batch)]
+        for b in range(batch):
+            _, z = orc.predict(H, xh[b])
+            check_mask(tr[l, b], z, w.d_ff, w.hot, 0.0, band)
+        lists = [orc.compact(tr[l] if union else tr[l, b], w.d_ff, w.hot) for b in range(batch)]
         xs = np.stack([xs[b].astype(np.float32).astype(np.float64) +
-                       orc.sparse_ffn(H, xh[b], union) for b in range(B)])
-    for b in range(B):
-        assert rel_l2(xg[b] - x0[b], xs[b] - x0[b]) <= TOL[w.w_dtype]
+                       orc.sparse_ffn(H, xh[b], lists[b]) for b in range(batch)])
+    for b in range(batch):
+        assert rel_l2(xg[b] - x0[b], xs[b] - x0[b]) <= TOL[wdt], b
 
 
 @pytest.mark.parametrize("packed", [False, True])
@@ -307,7 +295,7 @@ def test_kernel_launch_counter(pi):
 @pytest.mark.parametrize("act", ["reglu", "relu2"])
 @pytest.mark.parametrize("batch", [2, 5])
 def test_q4_per_token_stack_is_one_fused_pass_per_token(pi, act, batch):
-    """A Q4_0 stack at 2-15 tokens with per-token masks (no mask trace) runs
+    """A Q4_0 stack at several tokens with per-token masks (no mask trace) runs
     one persistent single-token pass per token: one launch per token, and
     every token's result bit-identical to a batch-1 call on it (the batched
     kernels, taken when a mask trace is asked for, are checked against the
@@ -330,7 +318,8 @@ def test_q4_per_token_stack_is_one_fused_pass_per_token(pi, act, batch):
 @pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
 @pytest.mark.parametrize("batch,mode", [(2, "per_token"), (5, "union"), (16, "per_token"),
                                         (20, "union"), (48, "per_token"), (64, "union")])
-def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
+@pytest.mark.parametrize("wdt", ["f16", "q4_0"])
+def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, wdt, monkeypatch):
     """At 2-64 tokens an fp16 layer's listed rows (hot prefix and cold list;
     whole-hot tiles loaded as boxes, the others gathered four rows per TMA
     load) run on the tensor cores (fp16 inputs, fp32 accumulation): within
@@ -339,8 +328,10 @@ def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
     ragged d_ff, a hot prefix that ends inside a tile, and no hot prefix;
     batches 2, 5, 20 and 48 pad the token tile.  At d = 4096 and 8192 the up
     kernel splits d over 2 and 4 CTAs per row tile, and the down kernel
-    splits a short list over 8 and 4 CTAs per column tile."""
-    w = _wl(act, "f16", shape, seed=47)
+    splits a short list over 8 and 4 CTAs per column tile.  Q4_0 layers take
+    the same path with their rows decoded to fp16 in shared memory (within
+    the Q4_0 tolerance; 4e-3 of the CUDA-core path, which decodes to fp32)."""
+    w = _wl(act, wdt, shape, seed=47)
     L, _ = device_layer(w, 0, packed=(batch % 32 == 0))
     H = synth.layer_host(w, 0)
     xh = _xh(w.d_model, batch, 9)
@@ -367,8 +358,8 @@ def test_ffn_on_tensor_cores(pi, orc, shape, act, batch, mode, monkeypatch):
         if np.linalg.norm(ref) == 0.0:
             assert np.all(y_tc[b] == 0.0)
             continue
-        assert rel_l2(y_tc[b], ref) <= TOL["f16"], b
-        assert rel_l2(y_tc[b], y_cc[b]) <= 2e-3, b
+        assert rel_l2(y_tc[b], ref) <= TOL[wdt], b
+        assert rel_l2(y_tc[b], y_cc[b]) <= (2e-3 if wdt == "f16" else 4e-3), b
     assert np.array_equal(run(), y_tc)  # deterministic
 
 
