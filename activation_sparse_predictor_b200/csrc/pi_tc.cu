@@ -107,11 +107,27 @@ __device__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile int* abort, WsH
   return true;
 }
 
-// Bounded wait that ignores the abort flag (used before freeing resources).
+// try_wait with a suspend-time hint: the thread may sleep in hardware
+// until the phase completes (or the hint elapses) instead of spinning.
+__device__ __forceinline__ bool tc_try_sleep(uint64_t* b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(tc_sa(b)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait that ignores the abort flag (used before freeing resources,
+// and by warps with nothing else to do until a kernel's products are
+// final): it sleeps between tries, so waiting warps take no issue slots
+// from the working ones.
 __device__ bool tc_wait_quiet(uint64_t* bar, uint32_t parity, WsHeader* hdr) {
   if (tc_try(bar, parity)) return true;
   const uint64_t t0 = tc_time();
-  while (!tc_try(bar, parity)) {
+  while (!tc_try_sleep(bar, parity, 100000u)) {
     if (tc_time() - t0 > kTcTimeoutNs) {
       if (hdr) atomicOr(&hdr->status, DEV_TIMEOUT);
       return false;
@@ -397,9 +413,11 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
 // loaded by 256 threads with vector loads, TC_Q4_PRE stages ahead in
 // registers, decoded to fp16 (q - 8) * s and stored into the 128-byte
 // swizzled operand tile of the ring; each thread fences its stores for
-// the tensor cores' (async) proxy and arrives on the stage's barrier, which
-// completes when all 256 have arrived and the activation tile's TMA bytes
-// have landed.  Warp 8 issues the MMAs; warps 8-11 drain the accumulators.
+// the tensor cores' (async) proxy and arrives on the stage's barrier,
+// which completes when all 256 have arrived and the activation tile's TMA
+// bytes have landed (one arrival per warp after a warp barrier measured
+// slower: the warp then waits for its slowest lane).  Warp 8 issues the
+// MMAs; warps 8-11 drain the accumulators.
 constexpr int TC_Q4_WARPS = 12;
 constexpr int TC_Q4_LOADERS = 256;  // threads 0..255 load and decode
 constexpr int TC_Q4_PRE = 4;        // stages of codes each loader holds ahead
@@ -429,6 +447,29 @@ __device__ __forceinline__ uint4 q4_chunk_f16(uint32_t w0, uint32_t w1, bool hig
   return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
+// Read-only loads of Q4_0 codes and scales that ask L2 to fetch the whole
+// 256-byte block around them: a row's next stages (and, for the down
+// projection, the neighbouring column tiles, which read the same rows at
+// the same time) then hit L2, so DRAM sees 256-byte requests instead of
+// the 64 bytes one stage takes from a row.
+__device__ __forceinline__ uint4 ld_q4_codes(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_q4_scales2(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L2::256B.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint16_t ld_q4_scale(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L2::256B.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
 __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)
@@ -449,11 +490,14 @@ __device__ __forceinline__ void fence_async_smem() {
 }
 
 // Q4_0 up/gate: as k_ffn_up_tc (grid, work shares, part layout), with
-// K = 128 per stage (two 64-column atoms) and NS = 2 ring stages.  Loader
-// thread t decodes blocks 2h, 2h + 1 of row t / 2 (h = t % 2) in each
-// operand: 32 contiguous code bytes and two scales per operand and stage.
-template <int NR>
-__global__ void __launch_bounds__(32 * TC_Q4_WARPS, NR == 1 ? 2 : 1)
+// K = 64 KB per stage (KB 64-column atoms) and NS = 2 ring stages, two CTAs
+// per SM (a separate, deeper ring for the activation tiles, loaded ahead
+// by an idle warp, measured slower).  Loader thread t
+// decodes blocks KB h .. KB h + KB - 1 of the stage in row t / 2 (h = t %
+// 2) of each operand: 16 KB contiguous code bytes and KB scales per
+// operand and stage.
+template <int NR, int KB>
+__global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
     k_ffn_up_q4tc(const __grid_constant__ CUtensorMap mx, const char* __restrict__ cw0,
                   const char* __restrict__ sw0, int64_t cst0, int64_t sst0,
                   const char* __restrict__ cw1, const char* __restrict__ sw1, int64_t cst1,
@@ -469,7 +513,7 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, NR == 1 ? 2 : 1)
   const uint32_t raw = tc_sa(smem_raw);
   unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const uint32_t batom = (uint32_t)nt * 128u;  // one 64-column atom of the activation tile
-  const uint32_t STAGE = NR * 2 * AT + ((2 * batom + 1023u) & ~1023u);
+  const uint32_t STAGE = NR * KB * AT + ((KB * batom + 1023u) & ~1023u);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + NS * STAGE);
   uint64_t* empty = full + NS;
   uint64_t* done = empty + NS;
@@ -498,18 +542,18 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, NR == 1 ? 2 : 1)
     const int row = list_row(p0 + m, H, N, F, idx);
     const char* cp[2] = {cw0 + (size_t)row * cst0, NR == 2 ? cw1 + (size_t)row * cst1 : nullptr};
     const char* sp[2] = {sw0 + (size_t)row * sst0, NR == 2 ? sw1 + (size_t)row * sst1 : nullptr};
-    uint4 cq[TC_Q4_PRE][NR][2];
+    uint4 cq[TC_Q4_PRE][NR][KB];
     uint32_t sq[TC_Q4_PRE][NR];
     // codes and scales of stage i into register slot u
     auto fetch = [&](int i, int u) {
       if (i < nkt) {
-        const size_t kb = (size_t)(kt0 + i) * 64 + (size_t)h * 32;  // code bytes
-        const size_t sb = (size_t)(kt0 + i) * 8 + (size_t)h * 4;    // scale bytes
+        const size_t kb = (size_t)(kt0 + i) * 32 * KB + (size_t)h * 16 * KB;  // code bytes
+        const size_t sb = (size_t)(kt0 + i) * 4 * KB + (size_t)h * 2 * KB;    // scale bytes
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-          cq[u][r][0] = ld_stream16(cp[r] + kb);
-          cq[u][r][1] = ld_stream16(cp[r] + kb + 16);
-          sq[u][r] = __ldg(reinterpret_cast<const uint32_t*>(sp[r] + sb));
+#pragma unroll
+          for (int q = 0; q < KB; ++q) cq[u][r][q] = ld_q4_codes(cp[r] + kb + 16 * q);
+          sq[u][r] = KB == 2 ? ld_q4_scales2(sp[r] + sb) : (uint32_t)ld_q4_scale(sp[r] + sb);
         }
       }
     };
@@ -532,25 +576,28 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, NR == 1 ? 2 : 1)
         }
         unsigned char* a = smem + st * STAGE;
         if (t == 0) {
-          mbar_expect_tx(&full[st], 2 * batom);
-          const int k = (kt0 + i) * 128;
-          tma_load_2d(a + NR * 2 * AT, &mx, k, 0, &full[st]);
-          tma_load_2d(a + NR * 2 * AT + batom, &mx, k + 64, 0, &full[st]);
+          mbar_expect_tx(&full[st], KB * batom);
+          const int k = (kt0 + i) * 64 * KB;
+#pragma unroll
+          for (int at = 0; at < KB; ++at)
+            tma_load_2d(a + NR * KB * AT + at * batom, &mx, k + 64 * at, 0, &full[st]);
           last = i;
         }
-        const uint32_t abase = sm0 + (uint32_t)st * STAGE + (uint32_t)h * AT + (uint32_t)m * 128u;
+        // block h KB + q of the stage: atom (h KB + q) / 2, chunks 4 ((h KB + q) % 2) ..
+        const uint32_t srow = sm0 + (uint32_t)st * STAGE + (uint32_t)m * 128u;
 #pragma unroll
         for (int r = 0; r < NR; ++r) {
-          const uint32_t ar = abase + (uint32_t)r * 2 * AT;
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {
+          for (int q = 0; q < KB; ++q) {
+            const int blk = h * KB + q;
+            const uint32_t ar = srow + (uint32_t)(r * KB + blk / 2) * AT;
             const uint32_t sbits = q ? (sq[u][r] >> 16) : (sq[u][r] & 0xFFFFu);
             const __half2 s2 = __half2half2(__ushort_as_half((unsigned short)sbits));
             const uint4 v = cq[u][r][q];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
               const uint4 o = q4_chunk_f16(c & 1 ? v.z : v.x, c & 1 ? v.w : v.y, c >= 2, s2);
-              const uint32_t cc = (uint32_t)(4 * q + c);
+              const uint32_t cc = (uint32_t)(4 * (blk & 1) + c);
               sts128(ar + ((cc ^ (uint32_t)(m & 7)) << 4), o);
             }
           }
@@ -571,16 +618,16 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, NR == 1 ? 2 : 1)
       const int st = i % NS;
       if (!tc_wait(&full[st], (uint32_t)(i / NS) & 1u, abort, hdr)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const uint32_t a = tc_sa(smem + st * STAGE), b = a + NR * 2 * AT;
+      const uint32_t a = tc_sa(smem + st * STAGE), b = a + NR * KB * AT;
 #pragma unroll
-      for (int at = 0; at < 2; ++at)
+      for (int at = 0; at < KB; ++at)
 #pragma unroll
         for (int kk = 0; kk < TC_BK / 16; ++kk) {
           const uint64_t bd = sw128_desc(b + (uint32_t)at * batom + 32u * kk);
           const uint32_t acc = (i | at | kk) != 0 ? 1u : 0u;
 #pragma unroll
           for (int r = 0; r < NR; ++r)
-            mma_f16(tmem + (uint32_t)(r * nt), sw128_desc(a + (uint32_t)(r * 2 + at) * AT + 32u * kk),
+            mma_f16(tmem + (uint32_t)(r * nt), sw128_desc(a + (uint32_t)(r * KB + at) * AT + 32u * kk),
                     bd, idesc, acc);
         }
       mma_commit(&empty[st]);
@@ -674,8 +721,8 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
     auto row_of = [&](int i) { return i < nkt ? list_row((kt0 + i) * TC_BK + k, H, N, F, idx) : 0; };
     auto fetch = [&](int i, int u) {
       if (i < nkt) {
-        cq[u] = ld_stream16(cw + (size_t)rq[u] * cst + cb);
-        sq[u] = __ldg(reinterpret_cast<const unsigned short*>(sw + (size_t)rq[u] * sst + sb));
+        cq[u] = ld_q4_codes(cw + (size_t)rq[u] * cst + cb);
+        sq[u] = ld_q4_scale(sw + (size_t)rq[u] * sst + sb);
       }
     };
 #pragma unroll
@@ -1379,8 +1426,9 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   return cudaGetLastError();
 }
 
-// Q4_0 up/gate (k_ffn_up_q4tc) and the same finish kernel.  CTA slots: two
-// per SM for one operand (two 48 KB stages at most), one for two (160 KB).
+// Q4_0 up/gate (k_ffn_up_q4tc) and the same finish kernel, two CTAs per
+// SM: one operand takes K = 128 per stage (two 48 KB stages at most), two
+// operands K = 64 (two 40 KB stages).
 template <int NR>
 cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                          const int32_t* idx, const int32_t* count, void* scratch, WsHeader* hdr,
@@ -1400,12 +1448,13 @@ cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const ui
                      batch, d, nt, sc.xh16);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const int nk = d / 128, g = (NR == 1 ? 2 : 1) * device_sms();
-  const uint32_t stage = NR * 2 * TC_M * 128 + (((uint32_t)nt * 256 + 1023u) & ~1023u);
+  constexpr int KB = NR == 1 ? 2 : 1;
+  const int nk = d / (64 * KB), g = 2 * device_sms();
+  const uint32_t stage = NR * KB * TC_M * 128 + (((uint32_t)nt * 128 * KB + 1023u) & ~1023u);
   const size_t smem = 1024 + 2 * (size_t)stage + 8 * (2 * 2 + 1) + 16;
-  e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_up_q4tc<NR>), smem);
+  e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_up_q4tc<NR, KB>), smem);
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_up_q4tc<NR>, std::max(g, Fp / TC_M), 32 * TC_Q4_WARPS, smem, s, mx, cw0,
+  (void)launch_dep(k_ffn_up_q4tc<NR, KB>, std::max(g, Fp / TC_M), 32 * TC_Q4_WARPS, smem, s, mx, cw0,
                    sw0, code_stride(PI_Q4_0, d, L.w_row_stride), scale_stride(d, L.w_row_stride),
                    static_cast<const char*>(L.w_up), static_cast<const char*>(L.w_up_scales),
                    code_stride(PI_Q4_0, d, ur), scale_stride(d, ur), nt, nk, g, H, F, idx, count,

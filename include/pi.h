@@ -221,14 +221,13 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch,
  * fp32 one; Q4_0 also d_model <= 8192, d_model % 256 == 0 and 16-byte
  * aligned scale arrays) the whole stack runs in one persistent cooperative
  * kernel per 24 layers; otherwise as a sequence of per-step kernels (fp16
- * layers at 2-64 tokens on the tensor cores).  Q4_0 stacks that meet the
- * single-token conditions run at any batch with PI_MASK_PER_TOKEN and no
- * mask_trace as one persistent pass per token, which gives each token its
- * per-token FFN exactly.  Setting the environment variable
- * PI_DISABLE_FUSED=1 forces the sequence.  All layers must share d_model
- * and d_ff;
- * `layers`
- * is a HOST array of n_layers descriptors.  mode: PI_MASK_PER_TOKEN or
+ * and Q4_0 layers at 2-64 tokens on the tensor cores).  Q4_0 stacks that
+ * meet the single-token conditions run below 8 tokens with
+ * PI_MASK_PER_TOKEN and no mask_trace as one persistent pass per token,
+ * which gives each token its per-token FFN exactly.  Setting the
+ * environment variable PI_DISABLE_FUSED=1 forces the sequence.  All layers
+ * must share d_model and d_ff; `layers` is a HOST array of n_layers
+ * descriptors.  mode: PI_MASK_PER_TOKEN or
  * PI_MASK_UNION as in pi_sparse_ffn.  mask_trace: NULL, or device
  * [n_layers][batch][ceil(d_ff/32)] receiving every layer's predicted masks
  * (d_ff of the largest layer).  No host synchronisation; capturable in a
