@@ -938,7 +938,11 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
 }
 
 // down: part[split][b][c] = sum over the split's list positions p of
-// W_down^T[row(p)][c] h[b][p], for the tile's 128 columns c.  Grid (d / 128, ks).
+// W_down^T[row(p)][c] h[b][p], for the tile's 128 CH columns c (CH M = 128
+// operands and accumulators; CH = 2 reads each listed row in 512-byte
+// pieces from half as many CTAs, with a 2-stage ring).  Grid
+// (d / (128 CH), ks).
+template <int CH>
 __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     k_ffn_down_tc(const __grid_constant__ CUtensorMap mwd, const __grid_constant__ CUtensorMap mwg,
                   const __grid_constant__ CUtensorMap mh, int nt, int nk, int ks, int d, int batch,
@@ -947,16 +951,17 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   pdl_wait();
   pdl_trigger();
   constexpr uint32_t BOX = 64 * TC_BK * 2;             // 64 columns x 64 positions: 8 KB
-  constexpr uint32_t A_BYTES = 2 * BOX;                // 128 columns
+  constexpr uint32_t A_BYTES = 2 * CH * BOX;           // 128 CH columns
   constexpr uint32_t B_BYTES = TC_TMAX * TC_BK * 2;    // 8 KB
   constexpr uint32_t STAGE = A_BYTES + B_BYTES;
-  constexpr uint32_t NCOLS = 64u;
+  constexpr uint32_t NCOLS = 64u * CH;
+  constexpr int DS = CH == 1 ? TC_STAGES : 2;  // ring stages
   extern __shared__ unsigned char smem_raw[];
   const uint32_t raw = tc_sa(smem_raw);
   unsigned char* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + TC_STAGES * STAGE);
-  uint64_t* empty = full + TC_STAGES;
-  uint64_t* done = empty + TC_STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + DS * STAGE);
+  uint64_t* empty = full + DS;
+  uint64_t* done = empty + DS;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
 
@@ -972,7 +977,7 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   const int nkt = kt1 > kt0 ? kt1 - kt0 : 0;
 
   if (threadIdx.x == 0) {
-    tc_init(full, empty, done, abort, TC_STAGES, (uint32_t)TC_PW);
+    tc_init(full, empty, done, abort, DS, (uint32_t)TC_PW);
     if (hdr && tile == 0 && split == 0) atomicAdd(&hdr->rows_down, (unsigned long long)N);
   }
   if (warp == 0) tmem_alloc(tslot, NCOLS);
@@ -980,13 +985,13 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tslot;
-  const int c0 = tile * TC_M;
+  const int c0 = tile * TC_M * CH;
 
   if (warp != 1) {
     // TC_PW producer warps, each arming its own bytes on the stage's full
     // barrier (TC_PW arrivals per phase).  A stage inside the hot prefix is
     // two 64-column boxes (warp 0).  Otherwise its 32 four-position gathers
-    // (positions pk + 4g .. pk + 4g + 3 of column half o / 16, g = o % 16)
+    // (positions pk + 4g .. pk + 4g + 3 of 64-column part o / 16, g = o % 16)
     // are dealt out round-robin, gather o = TC_PW * lane + pw.  Each lane
     // holds the list rows of its gather for as many stages ahead as the ring
     // is deep, so the list loads of a stage are in flight a whole ring ahead
@@ -994,30 +999,30 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     // registers are indexed statically).
     const int pw = warp == 0 ? 0 : warp - 1;
     const int o = TC_PW * lane + pw;
-    const int half = o >> 4, g = o & 15;  // column half, position group
-    const bool gl = o < 32;
+    const int part64 = o >> 4, g = o & 15;  // 64-column part, position group
+    const bool gl = o < 32 * CH;
     const uint32_t bx = (uint32_t)nt * TC_BK * 2;  // the activation tile
-    const uint32_t mine = (uint32_t)((32 - pw + TC_PW - 1) / TC_PW);  // gathers of this warp
-    int yr[TC_STAGES][4];  // list rows of this lane's gather, one set per ring slot
+    const uint32_t mine = (uint32_t)((32 * CH - pw + TC_PW - 1) / TC_PW);  // gathers of this warp
+    int yr[DS][4];  // list rows of this lane's gather, one set per ring slot
     auto rows_at = [&](int i, int (&v)[4]) {
       const int q = (kt0 + i) * TC_BK + 4 * g;
 #pragma unroll
       for (int t = 0; t < 4; ++t) v[t] = gl ? list_row(q + t, H, N, F, idx) : 0;
     };
 #pragma unroll
-    for (int u = 0; u < TC_STAGES; ++u)
+    for (int u = 0; u < DS; ++u)
       if (u < nkt) rows_at(u, yr[u]);
-    int last[TC_STAGES];
+    int last[DS];
 #pragma unroll
-    for (int u = 0; u < TC_STAGES; ++u) last[u] = -1;
+    for (int u = 0; u < DS; ++u) last[u] = -1;
     bool stop = false;
-    for (int i0 = 0; i0 < nkt && !stop; i0 += TC_STAGES) {
+    for (int i0 = 0; i0 < nkt && !stop; i0 += DS) {
 #pragma unroll
-      for (int st = 0; st < TC_STAGES; ++st) {  // ring slot st = i % TC_STAGES
+      for (int st = 0; st < DS; ++st) {  // ring slot st = i % DS
         const int i = i0 + st;
         if (i >= nkt) break;
         int ok = 1;
-        if (lane == 0 && i >= TC_STAGES) ok = tc_wait(&empty[st], ((i / TC_STAGES) - 1) & 1, abort, hdr);
+        if (lane == 0 && i >= DS) ok = tc_wait(&empty[st], ((i / DS) - 1) & 1, abort, hdr);
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
           stop = true;
           break;
@@ -1027,7 +1032,7 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
         const bool boxed = pk + TC_BK <= H;
         const uint32_t tx = boxed ? (pw == 0 ? A_BYTES + bx : 0u) : 512u * mine + (pw == 0 ? bx : 0u);
         const int y0 = yr[st][0], y1 = yr[st][1], y2 = yr[st][2], y3 = yr[st][3];
-        if (i + TC_STAGES < nkt) rows_at(i + TC_STAGES, yr[st]);
+        if (i + DS < nkt) rows_at(i + DS, yr[st]);
         if (lane == 0)
           asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tc_sa(&full[st])),
                        "r"(tx)
@@ -1035,11 +1040,12 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
         __syncwarp();
         if (boxed) {
           if (pw == 0 && lane == 0) {
-            tma_load_2d(a, &mwd, c0, pk, &full[st]);
-            tma_load_2d(a + BOX, &mwd, c0 + 64, pk, &full[st]);
+#pragma unroll
+            for (int q = 0; q < 2 * CH; ++q) tma_load_2d(a + q * BOX, &mwd, c0 + 64 * q, pk, &full[st]);
           }
         } else if (gl) {
-          tma_gather4(a + half * BOX + 512u * g, &mwg, c0 + 64 * half, y0, y1, y2, y3, &full[st]);
+          tma_gather4(a + part64 * BOX + 512u * g, &mwg, c0 + 64 * part64, y0, y1, y2, y3,
+                      &full[st]);
         }
         if (pw == 0 && lane == 0) tma_load_2d(a + A_BYTES, &mh, 0, (pk / TC_BK) * nt, &full[st]);
         last[st] = i;
@@ -1047,22 +1053,26 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
     }
     if (lane == 0) {
 #pragma unroll
-      for (int st = 0; st < TC_STAGES; ++st)
-        if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / TC_STAGES) & 1u, hdr);
+      for (int st = 0; st < DS; ++st)
+        if (last[st] >= 0) (void)tc_wait_quiet(&full[st], (uint32_t)(last[st] / DS) & 1u, hdr);
     }
   } else if (warp == 1 && lane == 0) {
     // kind::f16, fp16 A (MN-major) and B (K-major), fp32 D, M = 128, N = nt
     const uint32_t idesc = (1u << 4) | (1u << 15) | ((uint32_t)(nt >> 3) << 17) |
                            ((uint32_t)(TC_M >> 4) << 24);
     for (int i = 0; i < nkt; ++i) {
-      const int st = i % TC_STAGES;
-      if (!tc_wait(&full[st], (uint32_t)(i / TC_STAGES) & 1u, abort, hdr)) break;
+      const int st = i % DS;
+      if (!tc_wait(&full[st], (uint32_t)(i / DS) & 1u, abort, hdr)) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t a = tc_sa(smem + st * STAGE), b = a + A_BYTES;
 #pragma unroll
-      for (int kk = 0; kk < TC_BK / 16; ++kk)  // 16 positions = 2 K atoms of the A tile per MMA
-        mma_f16(tmem, sw128_mn_desc(a + 2048u * kk, BOX), sw128_desc(b + 32u * kk), idesc,
-                (i | kk) != 0 ? 1u : 0u);
+      for (int kk = 0; kk < TC_BK / 16; ++kk) {  // 16 positions = 2 K atoms of the A tile per MMA
+        const uint64_t bd = sw128_desc(b + 32u * kk);
+#pragma unroll
+        for (int hh = 0; hh < CH; ++hh)
+          mma_f16(tmem + 64u * hh, sw128_mn_desc(a + 2 * hh * BOX + 2048u * kk, BOX), bd, idesc,
+                  (i | kk) != 0 ? 1u : 0u);
+      }
       mma_commit(&empty[st]);
     }
     mma_commit(done);
@@ -1074,11 +1084,12 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   // accumulator lane = output column, accumulator column = token; a split
   // with no list positions writes zeros (the reduction sums every slice)
-  const int c = c0 + warp * 32 + lane;
+  for (int hh = 0; hh < CH; ++hh)
   for (int t0 = 0; t0 < nt && warp < 4; t0 += 16) {
+    const int c = c0 + 128 * hh + warp * 32 + lane;
     uint32_t v[16];
     if (ok && nkt > 0) {
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)t0, v);
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(64 * hh + t0), v);
     } else {
 #pragma unroll
       for (int t = 0; t < 16; ++t) v[t] = 0u;
@@ -1563,9 +1574,15 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
   return e;
 }
 
+// Columns per down tile, in units of 128: 256 where d_model / 256 tiles
+// still fill the SMs with up to TC_KSMAX_D splits each (d_model >= 8192).
+int down_ch(const pi_layer& L) {
+  return (L.w_dtype == PI_F16 && L.d_model >= 8192 && L.d_model % 256 == 0) ? 2 : 1;
+}
+
 int ffn_tc_down_splits(const pi_layer& L) {
-  // up to TC_KSMAX_D list shares per 128-column tile, to fill two CTAs per SM
-  int ks = 2 * device_sms() / (L.d_model / TC_M);
+  // up to TC_KSMAX_D list shares per column tile, to fill two CTAs per SM
+  int ks = 2 * device_sms() / (L.d_model / (TC_M * down_ch(L)));
   ks = ks < 1 ? 1 : (ks > TC_KSMAX_D ? TC_KSMAX_D : ks);
   const int nk = fpad(L.d_ff) / TC_BK;
   return ks > nk ? nk : ks;
@@ -1614,13 +1631,15 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
       !map_2d(&mh, sc.h16, (uint64_t)TC_BK, (uint64_t)(Fp / TC_BK) * nt, (uint64_t)TC_BK * 2,
               (uint32_t)nt))
     return cudaErrorInvalidValue;
-  const int tiles = d / TC_M, nk = Fp / TC_BK, ks = ffn_tc_down_splits(L);
-  constexpr uint32_t STAGE = 2 * 64 * TC_BK * 2 + TC_TMAX * TC_BK * 2;
-  const size_t smem = 1024 + (size_t)TC_STAGES * STAGE + 8 * (2 * TC_STAGES + 1) + 16;
-  cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_down_tc), smem);
+  const int ch = down_ch(L), ds = ch == 1 ? TC_STAGES : 2;
+  const int tiles = d / (TC_M * ch), nk = Fp / TC_BK, ks = ffn_tc_down_splits(L);
+  const uint32_t stage = 2 * ch * 64 * TC_BK * 2 + TC_TMAX * TC_BK * 2;
+  const size_t smem = 1024 + (size_t)ds * stage + 8 * (2 * ds + 1) + 16;
+  auto kern = ch == 2 ? k_ffn_down_tc<2> : k_ffn_down_tc<1>;
+  cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_down_tc, dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s, mwd, mwg, mh, nt, nk,
-                   ks, d, batch, H, F, idx, count, part, hdr);
+  (void)launch_dep(kern, dim3(tiles, ks), 32 * TC_FFN_WARPS, smem, s, mwd, mwg, mh, nt, nk, ks, d,
+                   batch, H, F, idx, count, part, hdr);
   return cudaGetLastError();
 }
 
