@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "pi.h"
 #include "pi_common.cuh"
@@ -33,6 +34,11 @@ pi_status cuda_fail(cudaError_t e, const char* what) {
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 int words_of(int F) { return (F + 31) / 32; }
+
+bool has_cold(const pi_layer& L) {
+  return L.w_gate_cold || L.w_up_cold || L.w_down_t_cold || L.w_gate_cold_scales ||
+         L.w_up_cold_scales || L.w_down_t_cold_scales;
+}
 
 // Validates one layer descriptor.
 pi_status check_layer(const pi_layer* L, int i) {
@@ -80,6 +86,52 @@ pi_status check_layer(const pi_layer* L, int i) {
     if (st != 0 && (st < codes || st % 16 != 0))
       return fail(PI_ERR_INVALID, "layer %d: row stride %lld must be 0 or a multiple of 16 >= %lld",
                   i, (long long)st, (long long)codes);
+  if (has_cold(*L)) {
+    if (!L->w_up_cold || !L->w_down_t_cold || (reglu && !L->w_gate_cold))
+      return fail(PI_ERR_INVALID, "layer %d: cold tier needs w_up_cold, w_down_t_cold%s", i,
+                  reglu ? " and w_gate_cold" : "");
+    if (q4 && (!L->w_up_cold_scales || !L->w_down_t_cold_scales || (reglu && !L->w_gate_cold_scales)))
+      return fail(PI_ERR_INVALID, "layer %d: Q4_0 cold tier needs its scale arrays", i);
+    if (!aligned(L->w_up_cold, 16) || !aligned(L->w_down_t_cold, 16) || !aligned(L->w_gate_cold, 16))
+      return fail(PI_ERR_INVALID, "layer %d: cold-tier pointer not 16-byte aligned", i);
+    if (!aligned(L->w_up_cold_scales, 2) || !aligned(L->w_down_t_cold_scales, 2) ||
+        !aligned(L->w_gate_cold_scales, 2))
+      return fail(PI_ERR_INVALID, "layer %d: cold-tier scale pointer not 2-byte aligned", i);
+  }
+  return PI_OK;
+}
+
+// The layers as the kernels read them: a layer with a host-memory cold tier
+// gets the device addresses of its cold rows (cudaPointerGetAttributes;
+// page-locked memory the current device can address, else PI_ERR_INVALID).
+// Layers without one are passed through untouched (*out = in, no copy).
+pi_status cold_resolve(const pi_layer* in, int n, std::vector<pi_layer>& store,
+                       const pi_layer** out) {
+  *out = in;
+  bool any = false;
+  for (int l = 0; l < n; ++l) any = any || has_cold(in[l]);
+  if (!any) return PI_OK;
+  store.assign(in, in + n);
+  for (int l = 0; l < n; ++l) {
+    pi_layer& L = store[l];
+    const void** ptrs[6] = {&L.w_gate_cold, &L.w_up_cold, &L.w_down_t_cold,
+                            &L.w_gate_cold_scales, &L.w_up_cold_scales, &L.w_down_t_cold_scales};
+    for (const void** p : ptrs) {
+      if (!*p) continue;
+      cudaPointerAttributes a{};
+      const cudaError_t e = cudaPointerGetAttributes(&a, *p);
+      if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return fail(PI_ERR_INVALID, "layer %d: cold-tier pointer %p: %s", l, *p, cudaGetErrorString(e));
+      }
+      if (a.type != cudaMemoryTypeHost || !a.devicePointer)
+        return fail(PI_ERR_INVALID,
+                    "layer %d: cold-tier pointer %p is not page-locked host memory mapped for "
+                    "this device", l, *p);
+      *p = a.devicePointer;
+    }
+  }
+  *out = store.data();
   return PI_OK;
 }
 
@@ -451,7 +503,10 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch, const
     return fail(PI_ERR_INVALID, "per-token mode with batch > 1 needs the mask");
   const WsLayout lay = layout_for_layers(layer, 1, batch);
   if ((st = check_ws(ws, ws_bytes, lay)) != PI_OK) return st;
-  return ffn_body(*layer, xh, batch, per_token ? mask : nullptr, per_token, idx, count, nullptr, y,
+  std::vector<pi_layer> store;
+  const pi_layer* kl;
+  if ((st = cold_resolve(layer, 1, store, &kl)) != PI_OK) return st;
+  return ffn_body(*kl, xh, batch, per_token ? mask : nullptr, per_token, idx, count, nullptr, y,
                   ws, lay, (cudaStream_t)stream);
 }
 
@@ -460,8 +515,11 @@ pi_status pi_ffn_stack(const pi_layer* layers, int n_layers, float* x, int batch
   WsLayout lay;
   pi_status st = stack_check(layers, n_layers, x, batch, tau, mode, mask_trace, ws, ws_bytes, &lay);
   if (st != PI_OK) return st;
-  return stack_run(layers, n_layers, x, batch, tau, mode, mask_trace, ws, lay,
-                   (cudaStream_t)stream, nullptr);
+  std::vector<pi_layer> store;
+  const pi_layer* kl;
+  if ((st = cold_resolve(layers, n_layers, store, &kl)) != PI_OK) return st;
+  return stack_run(kl, n_layers, x, batch, tau, mode, mask_trace, ws, lay, (cudaStream_t)stream,
+                   nullptr);
 }
 
 const char* pi_kind_name(int kind) {
@@ -477,6 +535,10 @@ pi_status pi_ffn_stack_profile(const pi_layer* layers, int n_layers, float* x, i
   WsLayout lay;
   pi_status st = stack_check(layers, n_layers, x, batch, tau, mode, mask_trace, ws, ws_bytes, &lay);
   if (st != PI_OK) return st;
+  std::vector<pi_layer> store;
+  const pi_layer* kl;
+  if ((st = cold_resolve(layers, n_layers, store, &kl)) != PI_OK) return st;
+  layers = kl;
   cudaStream_t s = (cudaStream_t)stream;
   Prof P;
   P.cap = n_layers * 8;
@@ -555,6 +617,22 @@ pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out) {
   out[0] = v[0];
   out[1] = v[1];
   out[2] = v[2];
+  return PI_OK;
+}
+
+pi_status pi_read_cold_counters(void* ws, void* stream, int clear, uint64_t* out) {
+  if (!ws || !aligned(ws, 256) || !out) return fail(PI_ERR_INVALID, "workspace or output null");
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned long long v[3];
+  static_assert(offsetof(WsHeader, cold_second) == offsetof(WsHeader, cold_listed) + 16,
+                "counters are adjacent");
+  e = cudaMemcpy(v, &header(ws)->cold_listed, sizeof v, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "counter read");
+  if (clear && (e = cudaMemset(&header(ws)->cold_listed, 0, sizeof v)) != cudaSuccess)
+    return cuda_fail(e, "counter clear");
+  for (int k = 0; k < 3; ++k) out[k] = v[k];
   return PI_OK;
 }
 

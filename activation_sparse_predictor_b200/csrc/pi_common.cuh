@@ -26,7 +26,10 @@ struct WsHeader {
   unsigned long long rows_listed;    // first-matrix neuron rows processed (x token passes)
   unsigned long long rows_down;      // down-projection rows read
   unsigned long long rows_second;    // ReGLU W_up rows read
-  unsigned long long stats_pad[5];
+  unsigned long long cold_listed;    // the three counts above, for rows read
+  unsigned long long cold_down;      //   from a host-memory cold tier
+  unsigned long long cold_second;
+  unsigned long long stats_pad[2];
   uint32_t counters[32];             // grid-barrier / arrival counters
 };
 static_assert(sizeof(WsHeader) == 256, "workspace header is 256 bytes");

@@ -366,6 +366,14 @@ __global__ void __launch_bounds__(256) k_mask_union(const uint32_t* __restrict__
   }
 }
 
+// Row j of a weight matrix whose rows [H, F) may live in a host-memory cold
+// tier (`cold` != null): those rows are read over the host link from there.
+__device__ __forceinline__ const char* wrow(const void* hot, const void* cold, int j, int H,
+                                            int64_t stride) {
+  return cold && j >= H ? (const char*)cold + (size_t)(j - H) * stride
+                        : (const char*)hot + (size_t)j * stride;
+}
+
 // Gathered up/gate rows + activation: one warp per listed row.
 template <int WT, int ACT, int TB>
 __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const float* __restrict__ xh,
@@ -391,6 +399,11 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
   if (hdr && blockIdx.x == 0 && threadIdx.x == 0) {
     atomicAdd(&hdr->rows_listed, (unsigned long long)(N - n0));
     if (ACT == PI_REGLU) atomicAdd(&hdr->rows_second, (unsigned long long)(N - n0));
+    const int nc = N - (n0 > H ? n0 : H);  // list positions >= H hold the cold rows
+    if (L.w_up_cold && nc > 0) {
+      atomicAdd(&hdr->cold_listed, (unsigned long long)nc);
+      if (ACT == PI_REGLU) atomicAdd(&hdr->cold_second, (unsigned long long)nc);
+    }
   }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool sq = L.act == PI_RELU2;
@@ -417,13 +430,13 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
     const char* rows[NR];
     const uint16_t* sc[NR];
     if constexpr (ACT == PI_REGLU) {
-      rows[0] = (const char*)L.w_gate + (size_t)j * rb;
-      rows[1] = (const char*)L.w_up + (size_t)j * rb2;
-      sc[0] = (const uint16_t*)((const char*)L.w_gate_scales + (size_t)j * sbs);
-      sc[1] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs2);
+      rows[0] = wrow(L.w_gate, L.w_gate_cold, j, H, rb);
+      rows[1] = wrow(L.w_up, L.w_up_cold, j, H, rb2);
+      sc[0] = (const uint16_t*)wrow(L.w_gate_scales, L.w_gate_cold_scales, j, H, sbs);
+      sc[1] = (const uint16_t*)wrow(L.w_up_scales, L.w_up_cold_scales, j, H, sbs2);
     } else {
-      rows[0] = (const char*)L.w_up + (size_t)j * rb;
-      sc[0] = (const uint16_t*)((const char*)L.w_up_scales + (size_t)j * sbs);
+      rows[0] = wrow(L.w_up, L.w_up_cold, j, H, rb);
+      sc[0] = (const uint16_t*)wrow(L.w_up_scales, L.w_up_cold_scales, j, H, sbs);
     }
     float acc[NR][TB];
 #pragma unroll
@@ -456,12 +469,15 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
 // its tokens, and writes its partial sums.  The slice is taken in passes of
 // kDownStage positions: the CTA first lists the pass's rows with a nonzero
 // h (row id and the tokens' h, in position order) in shared memory, then
-// streams just those rows, several loads in flight per thread.
+// streams just those rows, several loads in flight per thread.  Rows j >= H
+// come from `wdc` / `wscc` when those are set (a host-memory cold tier).
 constexpr int kDownStage = 512;
 
 template <int WT, int TB>
 __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ wd,
-                                                       const uint16_t* __restrict__ wsc, int d,
+                                                       const uint16_t* __restrict__ wsc,
+                                                       const char* __restrict__ wdc,
+                                                       const uint16_t* __restrict__ wscc, int d,
                                                        int F, int H,
                                                        const int32_t* __restrict__ idx,
                                                        const int32_t* __restrict__ count,
@@ -486,7 +502,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
     for (int e = 0; e < 8; ++e) acc[b][e] = 0.f;
   const int64_t rb = code_stride(WT, d, stride);
   const int64_t sbs = scale_stride(d, stride);
-  unsigned long long nread = 0;
+  unsigned long long nread = 0, ncold = 0;
   for (int p0 = n0; p0 < n1; p0 += kDownStage) {
     const int pn = min(kDownStage, n1 - p0);
     // the pass's rows with a nonzero h for some token of the chunk, in order
@@ -507,6 +523,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
         keep = keep && j >= 0 && j < F;
       }
       const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+      const uint32_t cbal = __ballot_sync(0xffffffffu, keep && j >= H);
+      if (lane == 0) ncold += __popc(cbal);  // this warp's cold rows
       if (lane == 0) swarp[warp] = __popc(bal);
       __syncthreads();
       if (tid == 0) {
@@ -534,7 +552,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
       for (int q = 0; q < base; ++q) {
         const int j = srow[q];
         float w[8];
-        const char* row = wd + (size_t)j * rb;
+        const char* row = wrow(wd, wdc, j, H, rb);
         if constexpr (WT == PI_F32) {
           const uint4 a = ld_stream16(row + (size_t)col0 * 4);
           const uint4 c = ld_stream16(row + (size_t)col0 * 4 + 16);
@@ -547,8 +565,8 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
         } else {
           const int blk = col0 >> 5, k0 = col0 & 31;
           const uint2 qv = *reinterpret_cast<const uint2*>(row + (size_t)blk * 16 + (k0 & 15));
-          const float sc = h2f(reinterpret_cast<const uint16_t*>(
-              reinterpret_cast<const char*>(wsc) + (size_t)j * sbs)[blk]);
+          const float sc =
+              h2f(reinterpret_cast<const uint16_t*>(wrow(wsc, wscc, j, H, sbs))[blk]);
           const int sh4 = k0 >= 16 ? 4 : 0;
           const uint32_t qq[2] = {qv.x, qv.y};
 #pragma unroll
@@ -574,6 +592,7 @@ __global__ void __launch_bounds__(kThreads) k_ffn_down(const char* __restrict__ 
     }
   }
   if (hdr && blockIdx.x == 0 && tid == 0 && nread) atomicAdd(&hdr->rows_down, nread);
+  if (hdr && wdc && blockIdx.x == 0 && lane == 0 && ncold) atomicAdd(&hdr->cold_down, ncold);
 }
 
 // out = resid + (sum over the S slices in order), four floats per thread
@@ -815,7 +834,8 @@ static cudaError_t ffn_down_t(const pi_layer& L, int batch, const int32_t* idx,
   const int tiles = (L.d_model + 8 * kThreads - 1) / (8 * kThreads);
   dim3 grid(tiles, S, (batch + TB - 1) / TB);
   (void)launch_plain(k_ffn_down<WT, TB>, grid, kThreads, 0, s, (const char*)L.w_down_t,
-                     (const uint16_t*)L.w_down_t_scales, L.d_model, L.d_ff, L.hot, idx, count, h,
+                     (const uint16_t*)L.w_down_t_scales, (const char*)L.w_down_t_cold,
+                     (const uint16_t*)L.w_down_t_cold_scales, L.d_model, L.d_ff, L.hot, idx, count, h,
                      batch, S, part, hdr, L.w_down_row_stride, nb);
   return cudaGetLastError();
 }

@@ -1901,6 +1901,9 @@ int stack1_unit_trace_len() { return UTR; }
 
 bool stack1_supported(const pi_layer* layers, int n_layers, int batch) {
   if (batch != 1 || n_layers < 1 || fused_disabled()) return false;
+  // rows in a host-memory cold tier are read by the CUDA-core kernels only
+  for (int l = 0; l < n_layers; ++l)
+    if (layers[l].w_up_cold) return false;
   const pi_layer& a = layers[0];
   for (int l = 1; l < n_layers; ++l) {
     const pi_layer& b = layers[l];

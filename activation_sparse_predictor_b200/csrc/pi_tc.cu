@@ -1483,7 +1483,7 @@ bool ffn_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
   if ((L.w_dtype != PI_F16 && L.w_dtype != PI_Q4_0) || batch < TC_MIN_BATCH || batch > TC_TMAX)
     return false;
-  if (L.d_model % TC_M != 0) return false;
+  if (L.d_model % TC_M != 0 || L.w_up_cold) return false;  // no host-memory cold tier
   if (L.w_dtype == PI_Q4_0) {
     // 16-byte code loads, 4-byte scale loads (two scales at a time)
     const int d = L.d_model;

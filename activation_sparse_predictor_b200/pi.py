@@ -42,6 +42,9 @@ class pi_layer(ctypes.Structure):
         ("p1", ctypes.c_void_p), ("p2", ctypes.c_void_p), ("p_bias", ctypes.c_void_p),
         ("w_row_stride", ctypes.c_int64), ("w_down_row_stride", ctypes.c_int64),
         ("w_up_row_stride", ctypes.c_int64),
+        ("w_gate_cold", ctypes.c_void_p), ("w_up_cold", ctypes.c_void_p),
+        ("w_down_t_cold", ctypes.c_void_p), ("w_gate_cold_scales", ctypes.c_void_p),
+        ("w_up_cold_scales", ctypes.c_void_p), ("w_down_t_cold_scales", ctypes.c_void_p),
     ]
 
 
@@ -64,6 +67,7 @@ def _load():
                                        ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]),
         "pi_kind_name": (ctypes.c_char_p, [i32]),
         "pi_read_counters": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_uint64)]),
+        "pi_read_cold_counters": (i32, [vp, vp, i32, ctypes.POINTER(ctypes.c_uint64)]),
         "pi_read_list": (i32, [L, i32, i32, vp, sz, vp, ctypes.POINTER(ctypes.c_int32), i32,
                                ctypes.POINTER(ctypes.c_int32)]),
         "pi_ffn_stack_timeline": (i32, [L, i32, vp, f32, vp, sz, vp, vp, vp]),
@@ -156,6 +160,58 @@ class Layer:
     @property
     def words(self) -> int:
         return (self.d_ff + 31) // 32
+
+    def with_host_cold_tier(self) -> "Layer":
+        """The same layer with rows [hot, d_ff) of w_gate / w_up / w_down_t
+        (and their Q4_0 scales) read from page-locked host memory: each
+        weight buffer's rows from `hot` on are copied to a pinned host
+        buffer with the same row layout, and the descriptor's cold pointers
+        point into it (see pi_layer).  The device tensors are shared with
+        this layer; the returned layer never reads their rows >= hot."""
+        import torch
+        bufs, host = {}, {}
+
+        def base_of(t):  # the row-major buffer a weight view lives in
+            b = t
+            while b._base is not None:
+                b = b._base
+            return b
+
+        def cold_ptr(t):
+            if t is None:
+                return None
+            b = base_of(t)
+            rows = b.reshape(self.d_ff, -1)
+            assert rows.shape[0] == self.d_ff and b.is_contiguous(), "one row per neuron"
+            key = b.data_ptr()
+            if key not in host:
+                h = torch.empty((rows.shape[0] - self.hot, rows.shape[1]), dtype=rows.dtype,
+                                pin_memory=True)
+                h.copy_(rows[self.hot:])
+                host[key] = h
+                bufs[key] = rows
+            rs = bufs[key].stride(0) * bufs[key].element_size()
+            off = t.data_ptr() - key  # offset inside the first row
+            assert 0 <= off < rs and t.stride(0) * t.element_size() == rs, "rows must share the buffer's stride"
+            return host[key].data_ptr() + off
+
+        out = Layer.__new__(Layer)
+        out.__dict__.update(self.__dict__)
+        c = pi_layer()
+        ctypes.pointer(c)[0] = self.c
+        for name, fld, sfld in (("w_gate", "w_gate_cold", "w_gate_cold_scales"),
+                                ("w_up", "w_up_cold", "w_up_cold_scales"),
+                                ("w_down_t", "w_down_t_cold", "w_down_t_cold_scales")):
+            v = self.tensors.get(name)
+            if v is None:
+                continue
+            codes, scales = v if isinstance(v, tuple) else (v, None)
+            setattr(c, fld, cold_ptr(codes))
+            if scales is not None:
+                setattr(c, sfld, cold_ptr(scales))
+        out.c = c
+        out.cold_host = host  # keeps the pinned buffers alive
+        return out
 
 
 def pack_records(w, tensors: dict):
@@ -319,6 +375,13 @@ def pi_ffn_stack_profile(layers, x, tau: float, mode: int, mask_trace=None, ws=N
                                      _ptr(mask_trace), _ptr(ws), ws.numel(), _stream(stream),
                                      ms, n))
     return {_lib.pi_kind_name(k).decode(): (float(ms[k]), int(n[k])) for k in range(PI_KINDS)}
+
+
+def pi_read_cold_counters(ws, clear: bool = False, stream=None):
+    """(first-matrix rows, w_down_t rows, ReGLU w_up rows) read from a host-memory cold tier."""
+    out = (ctypes.c_uint64 * 3)()
+    _check(_lib.pi_read_cold_counters(_ptr(ws), _stream(stream), int(clear), out))
+    return int(out[0]), int(out[1]), int(out[2])
 
 
 def pi_read_counters(ws, clear: bool = False, stream=None):

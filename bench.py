@@ -62,6 +62,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=0,
                     help="run only the first N layers (profiling captures; 0 = all)")
+    ap.add_argument("--cold-tier", default="none", choices=["none", "host"],
+                    help="host: every layer's cold rows (neurons >= hot) in page-locked host "
+                         "memory, read by the GPU over the host link")
     return ap.parse_args()
 
 
@@ -393,10 +396,33 @@ def l2_mode_for(w, n_layers: int, l2_bytes: int) -> str:
     return "flushed" if n_layers * synth.layer_nbytes(w) < 2 * l2_bytes else "streamed"
 
 
-def run_config(w, batch, mode, n_layers, world, l2="streamed"):
+def run_config(w, batch, mode, n_layers, world, l2="streamed", cold_tier="none"):
     """The `config` object both arms print for a run (same keys)."""
-    return dict(workload_config(w, batch, mode, l2), layers=n_layers,
-                parallelism=f"replicas x{world}" if world > 1 else "single GPU")
+    c = dict(workload_config(w, batch, mode, l2), layers=n_layers,
+             parallelism=f"replicas x{world}" if world > 1 else "single GPU")
+    if cold_tier == "host":
+        c["cold_tier"] = "rows of neurons >= hot in page-locked host memory"
+    return c
+
+
+def host_link_peak(dev, stream) -> float:
+    """GB/s of a 1 GiB copy from page-locked host memory to the device (the
+    best of 3), the bound for rows read from a host-memory cold tier."""
+    import torch
+    n = 1 << 30
+    h = torch.empty(n, dtype=torch.uint8).pin_memory()
+    d = torch.empty(n, dtype=torch.uint8, device=dev)
+    best = 0.0
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            d.copy_(h, non_blocking=True)
+            b.record(stream)
+            b.synchronize()
+            best = max(best, n / (a.elapsed_time(b) / 1000.0) / 1e9)
+    del h, d
+    return best
 
 
 # ---------------------------------------------------------------- GPU leg
@@ -419,6 +445,8 @@ def run_pi(args, world, rank, local):
             w, {k: t[k] for k in ("w_gate", "w_up", "w_down_t", "bias", "p1", "p2", "p_bias")
                 if k in t}))
         del t
+    if args.cold_tier == "host":
+        layers = [L.with_host_cold_tier() for L in layers]
     arr = pi.layer_array(layers)
     K, W = args.steps, max(3, args.warmup)
     xs = torch.stack([synth.x_device(w, rank * 1_000_003 + s, B, dev) for s in range(K + W)])
@@ -435,7 +463,9 @@ def run_pi(args, world, rank, local):
         stream.synchronize()
         g = torch.cuda.CUDAGraph()
         n_before = pi.pi_kernel_launches()
-        with torch.cuda.graph(g, stream=stream):
+        # (relaxed: the cold tier's host pointers are looked up at the call)
+        with torch.cuda.graph(g, stream=stream,
+                              capture_error_mode="relaxed" if args.cold_tier == "host" else "global"):
             pi.pi_ffn_stack(layers, x, w.tau, mode, ws=ws, stream=stream, _arr=arr)
         kernels_per_step = pi.pi_kernel_launches() - n_before  # what one replay launches
         for i in range(W):
@@ -445,6 +475,7 @@ def run_pi(args, world, rank, local):
     st, word = pi.pi_get_device_status(ws, stream=stream)
     assert st == pi.PI_OK, f"device status {word:#x} after warm-up"
     pi.pi_read_counters(ws, clear=True, stream=stream)
+    pi.pi_read_cold_counters(ws, clear=True, stream=stream)
 
     # ---- timed region: K graph replays, inputs already in HBM.  A stack
     # whose weights fit in L2 is timed step by step with a 2 x L2 write
@@ -475,6 +506,7 @@ def run_pi(args, world, rank, local):
     barrier(world)
     ms = ev0.elapsed_time(ev1) if flush is None else sum(a.elapsed_time(b) for a, b in step_ev)
     rows_listed, rows_down, rows_second = pi.pi_read_counters(ws, clear=True, stream=stream)
+    cold_rows = pi.pi_read_cold_counters(ws, clear=True, stream=stream)
     ms_max = max_over_ranks(ms, world, dev)
     value = world * K * B / (ms_max / 1000.0)
     resident = None
@@ -532,6 +564,23 @@ def run_pi(args, world, rank, local):
                 "avg_launch_us": 1000.0 * dom_ms / dom_n, "timing_source": timing_source,
                 "per_kind_ms_per_step": {k: v[0] for k, v in prof.items()},
                 "launches_per_step": {k: v[1] for k, v in prof.items()}}
+    if args.cold_tier == "host":
+        # the rows read from host memory bound the step: bytes that crossed
+        # the host link per step over the step time, against a pinned copy
+        cold_bytes = sum(cold_rows) * weight_row_bytes(w.w_dtype, w.d_model) / K
+        link = host_link_peak(dev, stream)
+        achieved = cold_bytes / (ms / K / 1000.0) / 1e9
+        roofline = {"bound": "host_link", "kernel": "ffn_up + ffn_down (rows >= hot)",
+                    "achieved": achieved, "peak": link, "unit": "GB/s", "frac": achieved / link,
+                    "peak_source": "page-locked host-to-device copy of 1 GiB, measured in this run",
+                    "traffic": None, "host_bytes_per_step": cold_bytes,
+                    "host_rows_per_step": {"first_read": cold_rows[0] / K,
+                                           "down_read": cold_rows[1] / K,
+                                           "second_read": cold_rows[2] / K},
+                    "device_bytes_per_step": step_bytes - cold_bytes,
+                    "timing_source": "graph replays of the timed region (the same timing as value)",
+                    "per_kind_ms_per_step": {k: v[0] for k, v in prof.items()},
+                    "launches_per_step": {k: v[1] for k, v in prof.items()}}
 
     # ---- end to end through the C ABI with host buffers: pinned H2D of the
     # step's input, the stack, D2H of the step's output, every step
@@ -575,7 +624,7 @@ def run_pi(args, world, rank, local):
         "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded generator, weights generated on the GPU; no datasets)",
-        "config": run_config(w, B, args.mode, nl, world, l2_mode),
+        "config": run_config(w, B, args.mode, nl, world, l2_mode, args.cold_tier),
         "hbm_gbs_actual": step_gbs, "hbm_frac_of_peak": step_gbs / peak,
         "bytes_per_step": step_bytes,
         "rows_per_step": {"first_read": rows_listed / K, "second_read": rows_second / K,

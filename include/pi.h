@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-#define PI_VERSION 2
+#define PI_VERSION 3
 #define PI_MAX_BATCH 64        /* tokens per call                           */
 #define PI_MAX_D_MODEL 16384   /* d_model upper bound                       */
 #define PI_MAX_RANK 8192       /* predictor rank upper bound                */
@@ -77,7 +77,8 @@ typedef enum pi_act { PI_RELU = 0, PI_REGLU = 1, PI_RELU2 = 2 } pi_act;
  *             predicted sets (prefill). */
 typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_mode;
 
-/* One FFN layer and its predictor.  All pointers are device pointers.
+/* One FFN layer and its predictor.  All pointers are device pointers, except
+ * the optional cold-tier pointers at the end (page-locked host memory).
  *  d_model, d_ff, rank : sizes d, F, r.  hot : H, 0 <= H <= F, the
  *                        always-active prefix [0, H) of the neuron order.
  *  act        : PI_RELU  h_j = max(0, w_up[j].xh + bias[j])
@@ -112,7 +113,27 @@ typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_m
  *           after another (Q4_0: each row's scales right behind its codes).
  * Alignment: every weight pointer 16-byte aligned; d % 8 (F32, F16),
  * d % 32 (Q4_0) == 0; r % 4 (F32 predictor) / r % 8 (F16 predictor) == 0;
- * strides multiples of 16 and at least one row's codes. */
+ * strides multiples of 16 and at least one row's codes.
+ *
+ * Hybrid cold tier (optional; the QbitAI article, §"Гибридный дизайн вывода
+ * CPU/GPU": hot neurons stay in GPU memory, cold ones in host memory, and
+ * the partial results are merged on the GPU).  When w_up_cold is not NULL,
+ * rows [hot, d_ff) of w_gate, w_up and w_down_t, and of their Q4_0 scale
+ * arrays, are read from the *_cold pointers instead: row j >= hot of w_up
+ * is at w_up_cold + (j - hot) * stride, with the same strides as the device
+ * rows (so packed records keep their layout), and rows [hot, d_ff) of the
+ * device pointers are never read (they may be left unallocated past row
+ * hot - 1).  The cold pointers must point into page-locked host memory
+ * that the current device can address (cudaHostAlloc / cudaMallocHost, or
+ * cudaHostRegister with cudaHostRegisterMapped); anything else returns
+ * PI_ERR_INVALID.  All cold pointers a layer needs must be set together
+ * (w_gate_cold for ReGLU, the scale arrays for Q4_0), with the alignment of
+ * their device counterparts.  The GPU reads the cold rows over the host
+ * link (PCIe or C2C) and merges them in the same kernels as the hot rows:
+ * the result is the same as with every row in device memory.  Such layers
+ * always take the multi-kernel CUDA-core path (batch 1 included), and their
+ * host memory must stay allocated and unchanged until the stream has run
+ * the call. */
 typedef struct pi_layer {
   int32_t d_model, d_ff, rank, hot;
   int32_t act, w_dtype, p_dtype;
@@ -129,6 +150,12 @@ typedef struct pi_layer {
   int64_t w_row_stride;
   int64_t w_down_row_stride;
   int64_t w_up_row_stride;
+  const void* w_gate_cold;
+  const void* w_up_cold;
+  const void* w_down_t_cold;
+  const void* w_gate_cold_scales;
+  const void* w_up_cold_scales;
+  const void* w_down_t_cold_scales;
 } pi_layer;
 
 /* Bytes of workspace the calls below need for these layers at this batch
@@ -304,6 +331,13 @@ unsigned long long pi_kernel_launches(void);
  * Together with the predictor's fixed size they give the bytes the path
  * actually read.  out: uint64_t[3].  `clear` != 0 resets all three. */
 pi_status pi_read_counters(void* ws, void* stream, int clear, uint64_t* out);
+
+/* The same three counts restricted to rows read from a hybrid cold tier
+ * (host memory, see pi_layer): out[0] first-matrix rows, out[1] w_down_t
+ * rows, out[2] ReGLU w_up rows.  Multiplied by the row bytes they give the
+ * bytes that crossed the host link.  out: uint64_t[3].  `clear` != 0 resets
+ * all three. */
+pi_status pi_read_cold_counters(void* ws, void* stream, int clear, uint64_t* out);
 
 /* Synchronises `stream` and copies to the host the ascending list of cold
  * neurons (ids in [hot, d_ff)) that the LAST layer of the last

@@ -41,7 +41,7 @@ def test_library_is_sm100a_only(pi):
 
 
 def test_status_strings_and_version(pi):
-    assert pi.pi_version() == 2
+    assert pi.pi_version() == 3
     assert pi.pi_status_string(pi.PI_OK) == "PI_OK"
     assert pi.pi_status_string(pi.PI_ERR_TIMEOUT) == "PI_ERR_TIMEOUT"
     assert pi.pi_status_string(99) == "PI_ERR_UNKNOWN"
@@ -174,3 +174,37 @@ def test_workspace_grows_with_batch(pi):
     b = pi._lib.pi_workspace_bytes(arr, 1, 16)
     assert 0 < a < b
     assert a % 256 == 0
+
+
+def test_layer_struct_matches_the_header(pi, tmp_path):
+    """ctypes' pi_layer has the C struct's size and field offsets (the
+    cold-tier pointers at the end included)."""
+    import os
+    fields = [f for f, _ in pi.pi_layer._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text("#include <stdio.h>\n#include <stddef.h>\n#include \"pi.h\"\nint main(void) {\n"
+                   "  printf(\"%zu\\n\", sizeof(pi_layer));\n" +
+                   "".join(f"  printf(\"%zu\\n\", offsetof(pi_layer, {f}));\n" for f in fields) +
+                   "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(pi.HEADER))
+    subprocess.run(["gcc", "-std=c11", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert got[0] == ctypes.sizeof(pi.pi_layer)
+    for f, off in zip(fields, got[1:]):
+        assert getattr(pi.pi_layer, f).offset == off, f
+
+
+def test_cold_tier_validation(pi):
+    """A cold tier must be complete (w_gate_cold for ReGLU, scales for Q4_0)
+    and aligned; checked before any device call."""
+    for over in (dict(w_up_cold=FAKE),                                   # no w_down_t_cold
+                 dict(act=1, w_up_cold=FAKE, w_down_t_cold=FAKE),        # ReGLU without gate
+                 dict(w_dtype=2, d_model=64, w_up_cold=FAKE, w_down_t_cold=FAKE),  # no scales
+                 dict(w_up_cold=FAKE + 4, w_down_t_cold=FAKE),           # misaligned
+                 dict(w_up_cold_scales=FAKE)):                           # scales alone
+        L = _layer(pi, **over)
+        st = pi._lib.pi_predict(ctypes.byref(L), FAKE, 1, 0.5, FAKE, FAKE, 1 << 30, None)
+        assert pi.pi_status_string(st) == "PI_ERR_INVALID", (over, pi.pi_last_error())
+        assert "cold" in pi.pi_last_error()

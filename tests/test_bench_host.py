@@ -134,3 +134,12 @@ def test_l2_mode_by_stack_size():
     w = synth.WORKLOADS[HEADLINE]
     assert bench.l2_mode_for(w, w.n_layers, bench.B200_L2_BYTES) == "streamed"
     assert "L2" in bench.run_config(w, 1, "per_token", 80, 1)["l2"]
+
+
+def test_cold_tier_is_named_in_the_config():
+    w = synth.WORKLOADS["llama2_70b_reglu_8192x28672_q4_0"]
+    plain = bench.run_config(w, 1, "per_token", 8, 1)
+    cold = bench.run_config(w, 1, "per_token", 8, 1, cold_tier="host")
+    assert "cold_tier" not in plain
+    assert "host memory" in cold["cold_tier"]
+    assert {k: v for k, v in cold.items() if k != "cold_tier"} == plain
