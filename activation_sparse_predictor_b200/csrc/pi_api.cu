@@ -135,7 +135,7 @@ pi_status cold_resolve(const pi_layer* in, int n, std::vector<pi_layer>& store,
   return PI_OK;
 }
 
-WsLayout layout_for(int d, int F, int r, int batch, int H) {
+WsLayout layout_for(int d, int F, int r, int batch, int H, size_t stage_bytes = 0) {
   WsLayout w{};
   size_t off = sizeof(WsHeader);
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
@@ -157,19 +157,24 @@ WsLayout layout_for(int d, int F, int r, int batch, int H) {
   w.y = take((size_t)batch * d * 4);
   w.tc = take(tc_scratch_bytes(d, F, r, batch));
   w.cta = take(4 * (size_t)device_sms());
+  w.stage_bytes = stage_bytes;
+  w.stage = take(stage_bytes);
   w.total = off;
   return w;
 }
 
 WsLayout layout_for_layers(const pi_layer* layers, int n, int batch) {
   int d = 0, F = 0, r = 0, H = 0;
+  size_t stage = 0;
   for (int l = 0; l < n; ++l) {
+    const size_t sb = cold_stage_bytes(layers[l], batch);
+    stage = stage > sb ? stage : sb;
     d = d > layers[l].d_model ? d : layers[l].d_model;
     F = F > layers[l].d_ff ? F : layers[l].d_ff;
     r = r > layers[l].rank ? r : layers[l].rank;
     H = H > layers[l].hot ? H : layers[l].hot;
   }
-  return layout_for(d, F, r, batch, H);
+  return layout_for(d, F, r, batch, H, stage);
 }
 
 pi_status check_ws(void* ws, size_t ws_bytes, const WsLayout& lay) {
@@ -230,7 +235,8 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
     if (e != cudaSuccess) return cuda_fail(e, "ffn down (tensor cores) launch");
   } else {
     P.before(PI_KIND_FFN_UP);
-    e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h), header(ws), s);
+    e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h), header(ws), s,
+                      0, lay.stage_bytes ? at<char>(ws, lay.stage) : nullptr);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
     P.before(PI_KIND_FFN_DOWN);

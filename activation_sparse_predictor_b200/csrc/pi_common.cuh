@@ -105,6 +105,12 @@ __host__ __device__ __forceinline__ int64_t row_bytes(int dt, int d) {
   return dt == PI_F32 ? 4LL * d : (dt == PI_F16 ? 2LL * d : (int64_t)d / 2);
 }
 
+// Bytes of one staged row: its codes, then (Q4_0) its scales, padded to 16.
+__host__ __device__ __forceinline__ int64_t stage_row_bytes(int dt, int d) {
+  const int64_t b = row_bytes(dt, d) + (dt == PI_Q4_0 ? d / 16 : 0);
+  return (b + 15) & ~(int64_t)15;
+}
+
 // Row-to-row distance of a weight matrix's codes, and of its Q4_0 scales.
 __host__ __device__ __forceinline__ int64_t code_stride(int dt, int d, int64_t stride) {
   return stride ? stride : row_bytes(dt, d);
@@ -126,6 +132,8 @@ struct WsLayout {
   size_t y;         // fp32 [B][d]        FFN output (stack)
   size_t tc;        // tensor-core scratch (fp16 layers at 2-64 tokens)
   size_t cta;       // u32  [SMs]         per-CTA list lengths (single-token kernel)
+  size_t stage;     // listed cold rows of a host-memory cold tier, staged (token batches)
+  size_t stage_bytes;
   size_t total;
   int splits;       // S
 };

@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
                                                      const int32_t* __restrict__ idx,
                                                      const int32_t* __restrict__ count,
                                                      float* __restrict__ h, WsHeader* hdr,
-                                                     int n0) {
+                                                     int n0, const char* __restrict__ stg) {
   pdl_wait();
   extern __shared__ __align__(16) float sx[];
   uint32_t* status = hdr ? &hdr->status : nullptr;
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
     atomicAdd(&hdr->rows_listed, (unsigned long long)(N - n0));
     if (ACT == PI_REGLU) atomicAdd(&hdr->rows_second, (unsigned long long)(N - n0));
     const int nc = N - (n0 > H ? n0 : H);  // list positions >= H hold the cold rows
-    if (L.w_up_cold && nc > 0) {
+    if (L.w_up_cold && !stg && nc > 0) {  // (staged rows were counted when staged)
       atomicAdd(&hdr->cold_listed, (unsigned long long)nc);
       if (ACT == PI_REGLU) atomicAdd(&hdr->cold_second, (unsigned long long)nc);
     }
@@ -429,7 +429,14 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
     }
     const char* rows[NR];
     const uint16_t* sc[NR];
-    if constexpr (ACT == PI_REGLU) {
+    if (stg && n >= H) {  // a cold row staged in device memory at its list position
+      const int64_t srb = stage_row_bytes(WT, d), cb = row_bytes(WT, d);
+#pragma unroll
+      for (int r = 0; r < NR; ++r) {
+        rows[r] = stg + ((size_t)r * (F - H) + (n - H)) * srb;
+        sc[r] = (const uint16_t*)(rows[r] + cb);
+      }
+    } else if constexpr (ACT == PI_REGLU) {
       rows[0] = wrow(L.w_gate, L.w_gate_cold, j, H, rb);
       rows[1] = wrow(L.w_up, L.w_up_cold, j, H, rb2);
       sc[0] = (const uint16_t*)wrow(L.w_gate_scales, L.w_gate_cold_scales, j, H, sbs);
@@ -459,6 +466,53 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
         if (!bit) hv = 0.f;
       }
       if (lane == 0 && t0 + b < B) h[(size_t)n * B + t0 + b] = hv;
+    }
+  }
+}
+
+// Copies the listed cold rows of the first matrix (and ReGLU's W_up) from a
+// host-memory cold tier into device memory, at their list positions
+// (stage_row_bytes each: codes, then Q4_0 scales), so that the up kernel's
+// token chunks read them from HBM and each row crosses the host link once.
+// One warp per list position; positions holding an id outside [H, F) are
+// skipped (the up kernel flags them and never reads their stage).
+template <int WT, int NR>
+__global__ void __launch_bounds__(kThreads) k_stage_cold(pi_layer L, const int32_t* __restrict__ idx,
+                                                         const int32_t* __restrict__ count,
+                                                         char* __restrict__ stg, WsHeader* hdr) {
+  pdl_wait();
+  const int d = L.d_model, F = L.d_ff, H = L.hot;
+  int cnt = *count;
+  cnt = cnt < 0 ? 0 : (cnt > F - H ? F - H : cnt);
+  if (hdr && blockIdx.x == 0 && threadIdx.x == 0 && cnt > 0) {
+    atomicAdd(&hdr->cold_listed, (unsigned long long)cnt);
+    if (NR == 2) atomicAdd(&hdr->cold_second, (unsigned long long)cnt);
+  }
+  const int64_t srb = stage_row_bytes(WT, d), cb = row_bytes(WT, d);
+  const int nsc = WT == PI_Q4_0 ? d / 32 : 0;
+  const int64_t up_rs = (NR == 2 && L.w_up_row_stride) ? L.w_up_row_stride : L.w_row_stride;
+  const int64_t rs[2] = {code_stride(WT, d, L.w_row_stride), code_stride(WT, d, up_rs)};
+  const int64_t ss[2] = {scale_stride(d, L.w_row_stride), scale_stride(d, up_rs)};
+  const void* hot[2] = {NR == 2 ? L.w_gate : L.w_up, L.w_up};
+  const void* cold[2] = {NR == 2 ? L.w_gate_cold : L.w_up_cold, L.w_up_cold};
+  const void* shot[2] = {NR == 2 ? L.w_gate_scales : L.w_up_scales, L.w_up_scales};
+  const void* scold[2] = {NR == 2 ? L.w_gate_cold_scales : L.w_up_cold_scales, L.w_up_cold_scales};
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int p = blockIdx.x * wpb + (threadIdx.x >> 5); p < cnt; p += gridDim.x * wpb) {
+    const int j = idx[p];
+    if (j < H || j >= F) continue;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      const char* src = wrow(hot[r], cold[r], j, H, rs[r]);
+      char* dst = stg + ((size_t)r * (F - H) + p) * srb;
+      for (int64_t c = lane; c < cb / 16; c += 32)
+        *reinterpret_cast<uint4*>(dst + 16 * c) = ld_stream16(src + 16 * c);
+      if (nsc) {
+        const uint16_t* ssrc = (const uint16_t*)wrow(shot[r], scold[r], j, H, ss[r]);
+        for (int e = lane; e < nsc; e += 32)
+          reinterpret_cast<uint16_t*>(dst + cb)[e] = ld_stream_u16(ssrc + e);
+      }
     }
   }
 }
@@ -698,6 +752,14 @@ int pick_tb(int batch, int d) {
 
 int down_tb(int batch) { return batch <= 1 ? 1 : (batch <= 2 ? 2 : (batch <= 4 ? 4 : 8)); }
 
+size_t cold_stage_bytes(const pi_layer& L, int batch) {
+  const int tb = pick_tb(batch, L.d_model);
+  if (!L.w_up_cold || (batch + tb - 1) / tb <= 1) return 0;  // one token chunk: read once anyway
+  return (size_t)(L.d_ff - L.hot) * (size_t)stage_row_bytes(L.w_dtype, L.d_model) *
+         (L.act == PI_REGLU ? 2u : 1u);
+}
+
+
 int down_splits(int batch, int d) {
   const int sms = device_sms();
   const int tiles = (d + 8 * kThreads - 1) / (8 * kThreads);
@@ -790,7 +852,7 @@ cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin,
 template <int WT, int ACT, int TB>
 static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                             int per_token, const int32_t* idx, const int32_t* count, float* h,
-                            WsHeader* status, cudaStream_t s, int n0) {
+                            WsHeader* status, cudaStream_t s, int n0, const char* stg) {
   const size_t smem = (size_t)TB * L.d_model * 4;
   auto kern = k_ffn_up<WT, ACT, TB>;
   cudaError_t e = allow_smem(kern, smem);
@@ -798,29 +860,40 @@ static cudaError_t ffn_up_t(const pi_layer& L, const float* xh, int batch, const
   constexpr int T = up_threads<WT>();
   dim3 grid(std::min((L.d_ff + T / 32 - 1) / (T / 32), device_sms() * (1024 / T)), (batch + TB - 1) / TB);
   (void)launch_plain(kern, grid, T, smem, s, L, xh, batch, mask, per_token, (L.d_ff + 31) / 32, idx,
-                     count, h, status, n0);
+                     count, h, status, n0, stg);
   return cudaGetLastError();
 }
 
 template <int WT, int ACT>
 static cudaError_t ffn_up_a(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                             int per_token, const int32_t* idx, const int32_t* count, float* h,
-                            WsHeader* status, cudaStream_t s, int n0) {
+                            WsHeader* status, cudaStream_t s, int n0, char* stage) {
+  const char* stg = nullptr;
+  if (stage && cold_stage_bytes(L, batch)) {
+    constexpr int NR = ACT == PI_REGLU ? 2 : 1;
+    const int grid = std::min((L.d_ff - L.hot + kWarps - 1) / kWarps, device_sms() * 4);
+    (void)launch_plain(k_stage_cold<WT, NR>, std::max(grid, 1), kThreads, 0, s, L, idx, count,
+                       stage, status);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    stg = stage;
+  }
   switch (pick_tb(batch, L.d_model)) {
-    case 1: return ffn_up_t<WT, ACT, 1>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
-    case 2: return ffn_up_t<WT, ACT, 2>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
-    case 4: return ffn_up_t<WT, ACT, 4>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
-    default: return ffn_up_t<WT, ACT, 8>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
+    case 1: return ffn_up_t<WT, ACT, 1>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0, stg);
+    case 2: return ffn_up_t<WT, ACT, 2>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0, stg);
+    case 4: return ffn_up_t<WT, ACT, 4>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0, stg);
+    default: return ffn_up_t<WT, ACT, 8>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0, stg);
   }
 }
 
 cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                           int per_token, const int32_t* idx, const int32_t* count, float* h,
-                          WsHeader* status, cudaStream_t s, int n0) {
-#define PI_UP(WT)                                                                                  \
-  return L.act == PI_REGLU                                                                         \
-             ? ffn_up_a<WT, PI_REGLU>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0) \
-             : ffn_up_a<WT, PI_RELU>(L, xh, batch, mask, per_token, idx, count, h, status, s, n0);
+                          WsHeader* status, cudaStream_t s, int n0, char* stage) {
+#define PI_UP(WT)                                                                          \
+  return L.act == PI_REGLU ? ffn_up_a<WT, PI_REGLU>(L, xh, batch, mask, per_token, idx,   \
+                                                    count, h, status, s, n0, stage)       \
+                           : ffn_up_a<WT, PI_RELU>(L, xh, batch, mask, per_token, idx,    \
+                                                   count, h, status, s, n0, stage);
   if (L.w_dtype == PI_F32) { PI_UP(PI_F32) }
   if (L.w_dtype == PI_F16) { PI_UP(PI_F16) }
   PI_UP(PI_Q4_0)

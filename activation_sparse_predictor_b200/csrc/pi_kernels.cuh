@@ -80,10 +80,17 @@ cudaError_t launch_mask_union(const uint32_t* mask, int batch, int words, uint32
 cudaError_t launch_compact(const uint32_t* mask, int batch, int d_ff, int begin, int mode,
                            int32_t* idx, int32_t* count, cudaStream_t s);
 
-// h[n][b] for rows n of [0,hot) U idx[0..count)
+// h[n][b] for rows n of [0,hot) U idx[0..count).  `stage` (optional, at
+// least cold_stage_bytes(L, batch)): a layer with a host-memory cold tier
+// first copies its listed cold rows there, so that every token chunk reads
+// them from device memory.
 cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                           int per_token, const int32_t* idx, const int32_t* count, float* h,
-                          WsHeader* hdr, cudaStream_t s, int n0 = 0);
+                          WsHeader* hdr, cudaStream_t s, int n0 = 0, char* stage = nullptr);
+
+// Device bytes launch_ffn_up stages a host-memory cold tier's listed rows in
+// (0: the layer has none, or its tokens fit one chunk and read each row once).
+size_t cold_stage_bytes(const pi_layer& L, int batch);
 
 // part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n],
 // the list positions [nb, H + count) split into `splits` slices

@@ -715,7 +715,7 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
     const int t = threadIdx.x, k = t >> 2, q = t & 3;  // position in the stage, column block
     const size_t cb = (size_t)(c0 + 32 * q) / 2;       // code bytes of the block in a row
     const size_t sb = (size_t)(c0 + 32 * q) / 32 * 2;  // scale bytes
-    int rq[TC_Q4_PRE];       // list rows, one slot per stage
+    int rq[TC_Q4_PRE] = {};  // list rows, one slot per stage
     uint4 cq[TC_Q4_PRE];     // codes
     uint16_t sq[TC_Q4_PRE];  // scales
     auto row_of = [&](int i) { return i < nkt ? list_row((kt0 + i) * TC_BK + k, H, N, F, idx) : 0; };

@@ -102,6 +102,10 @@ def test_cold_tier_sparse_ffn(pi, orc, act, wdt, batch, mode, packed, monkeypatc
         ref = orc.sparse_ffn(H, xh[b].astype(np.float64), own)
         assert rel_l2(yn[b], ref) <= TOL[wdt], b
     listed, down, second = pi.pi_read_cold_counters(ws)
+    # each listed cold row crossed the host link once: at token batches of
+    # several chunks the up kernel reads them from their device stage
+    assert listed == len(union)
+    assert second == (len(union) if act == "reglu" else 0)
     if batch == 1:
         # every listed neuron is cold; its first matrix (and ReGLU's W_up) came
         # over the host link, and its down row when its h was nonzero
@@ -111,7 +115,7 @@ def test_cold_tier_sparse_ffn(pi, orc, act, wdt, batch, mode, packed, monkeypatc
         nz = int(np.count_nonzero(h[union]))
         assert down <= listed and abs(down - nz) <= max(2, len(union) // 100), (down, nz)
     else:
-        assert listed >= len(union) and down <= listed
+        assert down <= listed * ((batch + 7) // 8)  # down rows: once per chunk of <= 8 tokens
 
 
 @pytest.mark.parametrize("act,wdt", [("reglu", "q4_0"), ("relu", "f16"), ("relu2", "f32")])
