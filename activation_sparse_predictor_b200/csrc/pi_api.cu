@@ -240,7 +240,8 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
     P.before(PI_KIND_FFN_DOWN);
-    e = launch_ffn_down(L, batch, idx, count, at<float>(ws, lay.h), part, S, header(ws), s);
+    e = launch_ffn_down(L, batch, idx, count, at<float>(ws, lay.h), part, S, header(ws), s, 0,
+                        lay.stage_bytes ? at<char>(ws, lay.stage) : nullptr);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn_down launch");
   }

@@ -88,15 +88,19 @@ cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const u
                           int per_token, const int32_t* idx, const int32_t* count, float* h,
                           WsHeader* hdr, cudaStream_t s, int n0 = 0, char* stage = nullptr);
 
-// Device bytes launch_ffn_up stages a host-memory cold tier's listed rows in
-// (0: the layer has none, or its tokens fit one chunk and read each row once).
+// Device bytes launch_ffn_up and launch_ffn_down stage a host-memory cold
+// tier's listed rows in (0: the layer has none, or its tokens fit one chunk
+// of each kernel and read each row once).
 size_t cold_stage_bytes(const pi_layer& L, int batch);
 
 // part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n],
 // the list positions [nb, H + count) split into `splits` slices
+// `stage`: as for launch_ffn_up (the same buffer); a cold-tier layer's down
+// rows that some token needs are staged there first when the tokens take
+// four chunks or more.
 cudaError_t launch_ffn_down(const pi_layer& L, int batch, const int32_t* idx,
                             const int32_t* count, const float* h, float* part, int splits,
-                            WsHeader* hdr, cudaStream_t s, int nb = 0);
+                            WsHeader* hdr, cudaStream_t s, int nb = 0, char* stage = nullptr);
 
 // out[b][i] = (resid ? resid[b][i] : 0) + sum_s part[s][b][i], s ascending.
 cudaError_t launch_reduce(const float* part, int splits, int batch, int d, const float* resid,
