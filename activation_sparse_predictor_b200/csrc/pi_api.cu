@@ -167,7 +167,8 @@ WsLayout layout_for_layers(const pi_layer* layers, int n, int batch) {
   int d = 0, F = 0, r = 0, H = 0;
   size_t stage = 0;
   for (int l = 0; l < n; ++l) {
-    const size_t sb = cold_stage_bytes(layers[l], batch);
+    const size_t sb = ffn_tc_supported(layers[l], batch) ? tc_cold_stage_bytes(layers[l])
+                                                         : cold_stage_bytes(layers[l], batch);
     stage = stage > sb ? stage : sb;
     d = d > layers[l].d_model ? d : layers[l].d_model;
     F = F > layers[l].d_ff ? F : layers[l].d_ff;
@@ -221,27 +222,31 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
   float* part = at<float>(ws, lay.part);
   int St = S;  // split-K slices to reduce
   cudaError_t e = cudaSuccess;
-  if (ffn_tc_supported(L, batch)) {
+  // a host-memory cold tier's rows are staged in the workspace when it has
+  // room for them (it does when sized by pi_workspace_bytes for these layers)
+  char* stage = lay.stage_bytes ? at<char>(ws, lay.stage) : nullptr;
+  if (ffn_tc_supported(L, batch) && lay.stage_bytes >= tc_cold_stage_bytes(L)) {
     // token batches: both contractions over the listed rows on the tensor cores
     P.before(PI_KIND_FFN_UP);
     e = launch_ffn_up_tc(L, xh, batch, mask, idx, count, at<void>(ws, lay.tc), header(ws), s,
-                         xh16_ready);
+                         xh16_ready, stage);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn up (tensor cores) launch");
     P.before(PI_KIND_FFN_DOWN);
     St = ffn_tc_down_splits(L);
-    e = launch_ffn_down_tc(L, batch, idx, count, part, at<void>(ws, lay.tc), header(ws), s);
+    e = launch_ffn_down_tc(L, batch, idx, count, part, at<void>(ws, lay.tc), header(ws), s, stage);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn down (tensor cores) launch");
   } else {
     P.before(PI_KIND_FFN_UP);
+    if (lay.stage_bytes < cold_stage_bytes(L, batch)) stage = nullptr;  // read the host rows directly
     e = launch_ffn_up(L, xh, batch, mask, per_token, idx, count, at<float>(ws, lay.h), header(ws), s,
-                      0, lay.stage_bytes ? at<char>(ws, lay.stage) : nullptr);
+                      0, stage);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn_up launch");
     P.before(PI_KIND_FFN_DOWN);
     e = launch_ffn_down(L, batch, idx, count, at<float>(ws, lay.h), part, S, header(ws), s, 0,
-                        lay.stage_bytes ? at<char>(ws, lay.stage) : nullptr);
+                        stage);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "ffn_down launch");
   }

@@ -474,8 +474,9 @@ __global__ void __launch_bounds__(up_threads<WT>()) k_ffn_up(pi_layer L, const f
 // host-memory cold tier into device memory, at their list positions
 // (stage_row_bytes each: codes, then Q4_0 scales), so that the up kernel's
 // token chunks read them from HBM and each row crosses the host link once.
-// One warp per list position; positions holding an id outside [H, F) are
-// skipped (the up kernel flags them and never reads their stage).
+// One warp per list position; a position holding an id outside [H, F) gets
+// a zero row (the up kernels flag such ids; the tensor-core kernels read
+// every staged position, so none may hold stale bytes).
 template <int WT, int NR>
 __global__ void __launch_bounds__(kThreads) k_stage_cold(pi_layer L, const int32_t* __restrict__ idx,
                                                          const int32_t* __restrict__ count,
@@ -501,28 +502,30 @@ __global__ void __launch_bounds__(kThreads) k_stage_cold(pi_layer L, const int32
   const int wpb = blockDim.x >> 5;
   for (int p = blockIdx.x * wpb + (threadIdx.x >> 5); p < cnt; p += gridDim.x * wpb) {
     const int j = idx[p];
-    if (j < H || j >= F) continue;
+    const bool ok = j >= H && j < F;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
-      const char* src = wrow(hot[r], cold[r], j, H, rs[r]);
+      const char* src = ok ? wrow(hot[r], cold[r], j, H, rs[r]) : nullptr;
       char* dst = stg + ((size_t)r * (F - H) + p) * srb;
       for (int64_t c = lane; c < cb / 16; c += 32)
-        *reinterpret_cast<uint4*>(dst + 16 * c) = ld_stream16(src + 16 * c);
+        *reinterpret_cast<uint4*>(dst + 16 * c) = ok ? ld_stream16(src + 16 * c) : make_uint4(0, 0, 0, 0);
       if (nsc) {
-        const uint16_t* ssrc = (const uint16_t*)wrow(shot[r], scold[r], j, H, ss[r]);
+        const uint16_t* ssrc = ok ? (const uint16_t*)wrow(shot[r], scold[r], j, H, ss[r]) : nullptr;
         for (int e = lane; e < nsc; e += 32)
-          reinterpret_cast<uint16_t*>(dst + cb)[e] = ld_stream_u16(ssrc + e);
+          reinterpret_cast<uint16_t*>(dst + cb)[e] = ok ? ld_stream_u16(ssrc + e) : (uint16_t)0;
       }
     }
   }
 }
 
-// Copies the w_down_t rows of the listed cold neurons whose h is nonzero for
-// some token from the host-memory cold tier into device memory at their
-// list positions (one warp per position), so that the down kernel's token
-// chunks read them from HBM; the rows with h = 0 for every token are never
-// read.  Ids outside [H, F) are skipped (the down kernel reads those, if in
-// range, from the device rows).
+// Copies w_down_t rows of listed cold neurons from the host-memory cold tier
+// into device memory at their list positions (one warp per position), so
+// that the down kernel reads them from HBM.  With h (the CUDA-core path:
+// h[n][b]) only rows whose h is nonzero for some token are copied, the rows
+// the down kernel reads; ids outside [H, F) are skipped (it reads those, if
+// in range, from the device rows).  Without h (the tensor-core path, which
+// reads every listed position) every row is copied, and a bad id gets a
+// zero row.
 template <int WT>
 __global__ void __launch_bounds__(kThreads) k_stage_cold_down(pi_layer L,
                                                               const int32_t* __restrict__ idx,
@@ -542,19 +545,23 @@ __global__ void __launch_bounds__(kThreads) k_stage_cold_down(pi_layer L,
   unsigned long long copied = 0;
   for (int p = blockIdx.x * wpb + (threadIdx.x >> 5); p < cnt; p += gridDim.x * wpb) {
     const int j = idx[p];
-    if (j < H || j >= F) continue;
-    bool nz = false;
-    for (int b = lane; b < B; b += 32) nz |= h[(size_t)(H + p) * B + b] != 0.f;
-    if (!__any_sync(0xffffffffu, nz)) continue;
-    ++copied;
-    const char* src = wrow(L.w_down_t, L.w_down_t_cold, j, H, rs);
+    const bool ok = j >= H && j < F;
+    if (h) {
+      if (!ok) continue;
+      bool nz = false;
+      for (int b = lane; b < B; b += 32) nz |= h[(size_t)(H + p) * B + b] != 0.f;
+      if (!__any_sync(0xffffffffu, nz)) continue;
+    }
+    copied += ok;
+    const char* src = ok ? wrow(L.w_down_t, L.w_down_t_cold, j, H, rs) : nullptr;
     char* dst = stg + (size_t)p * srb;
     for (int64_t c = lane; c < cb / 16; c += 32)
-      *reinterpret_cast<uint4*>(dst + 16 * c) = ld_stream16(src + 16 * c);
+      *reinterpret_cast<uint4*>(dst + 16 * c) = ok ? ld_stream16(src + 16 * c) : make_uint4(0, 0, 0, 0);
     if (nsc) {
-      const uint16_t* ssrc = (const uint16_t*)wrow(L.w_down_t_scales, L.w_down_t_cold_scales, j, H, ss);
+      const uint16_t* ssrc =
+          ok ? (const uint16_t*)wrow(L.w_down_t_scales, L.w_down_t_cold_scales, j, H, ss) : nullptr;
       for (int e = lane; e < nsc; e += 32)
-        reinterpret_cast<uint16_t*>(dst + cb)[e] = ld_stream_u16(ssrc + e);
+        reinterpret_cast<uint16_t*>(dst + cb)[e] = ok ? ld_stream_u16(ssrc + e) : (uint16_t)0;
     }
   }
   if (hdr && lane == 0 && copied) atomicAdd(&hdr->cold_down, copied);
@@ -821,6 +828,32 @@ size_t cold_stage_bytes(const pi_layer& L, int batch) {
   return stage_up_bytes(L, batch) + stage_down_bytes(L, batch);
 }
 
+cudaError_t launch_stage_cold(const pi_layer& L, const int32_t* idx, const int32_t* count,
+                              char* stage, WsHeader* hdr, cudaStream_t s) {
+  const int grid = std::max(1, std::min((L.d_ff - L.hot + kWarps - 1) / kWarps, device_sms() * 4));
+  const bool two = L.act == PI_REGLU;
+  if (L.w_dtype == PI_F32)
+    (void)launch_plain(two ? k_stage_cold<PI_F32, 2> : k_stage_cold<PI_F32, 1>, grid, kThreads, 0,
+                       s, L, idx, count, stage, hdr);
+  else if (L.w_dtype == PI_F16)
+    (void)launch_plain(two ? k_stage_cold<PI_F16, 2> : k_stage_cold<PI_F16, 1>, grid, kThreads, 0,
+                       s, L, idx, count, stage, hdr);
+  else
+    (void)launch_plain(two ? k_stage_cold<PI_Q4_0, 2> : k_stage_cold<PI_Q4_0, 1>, grid, kThreads, 0,
+                       s, L, idx, count, stage, hdr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stage_cold_down(const pi_layer& L, int batch, const int32_t* idx,
+                                   const int32_t* count, const float* h, char* stage,
+                                   WsHeader* hdr, cudaStream_t s) {
+  const int grid = std::max(1, std::min((L.d_ff - L.hot + kWarps - 1) / kWarps, device_sms() * 4));
+  auto kern = L.w_dtype == PI_F32 ? k_stage_cold_down<PI_F32>
+              : L.w_dtype == PI_F16 ? k_stage_cold_down<PI_F16> : k_stage_cold_down<PI_Q4_0>;
+  (void)launch_plain(kern, grid, kThreads, 0, s, L, idx, count, h, batch, stage, hdr);
+  return cudaGetLastError();
+}
+
 
 int down_splits(int batch, int d) {
   const int sms = device_sms();
@@ -931,12 +964,8 @@ static cudaError_t ffn_up_a(const pi_layer& L, const float* xh, int batch, const
                             int per_token, const int32_t* idx, const int32_t* count, float* h,
                             WsHeader* status, cudaStream_t s, int n0, char* stage) {
   const char* stg = nullptr;
-  if (stage && cold_stage_bytes(L, batch)) {
-    constexpr int NR = ACT == PI_REGLU ? 2 : 1;
-    const int grid = std::min((L.d_ff - L.hot + kWarps - 1) / kWarps, device_sms() * 4);
-    (void)launch_plain(k_stage_cold<WT, NR>, std::max(grid, 1), kThreads, 0, s, L, idx, count,
-                       stage, status);
-    const cudaError_t e = cudaGetLastError();
+  if (stage && stage_up_bytes(L, batch)) {
+    const cudaError_t e = launch_stage_cold(L, idx, count, stage, status, s);
     if (e != cudaSuccess) return e;
     stg = stage;
   }
@@ -982,10 +1011,7 @@ static cudaError_t ffn_down_w(const pi_layer& L, int batch, const int32_t* idx,
   const char* stg = nullptr;
   if (stage && stage_down_bytes(L, batch)) {
     char* dst = stage + stage_up_bytes(L, batch);
-    const int grid = std::min((L.d_ff - L.hot + kWarps - 1) / kWarps, device_sms() * 4);
-    (void)launch_plain(k_stage_cold_down<WT>, std::max(grid, 1), kThreads, 0, s, L, idx, count, h,
-                       batch, dst, hdr);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_stage_cold_down(L, batch, idx, count, h, dst, hdr, s);
     if (e != cudaSuccess) return e;
     stg = dst;
   }

@@ -93,6 +93,17 @@ cudaError_t launch_ffn_up(const pi_layer& L, const float* xh, int batch, const u
 // of each kernel and read each row once).
 size_t cold_stage_bytes(const pi_layer& L, int batch);
 
+// Copies the first matrix's (and ReGLU's W_up) rows of a host-memory cold
+// tier's listed neurons to stage[r][p] (row bytes stage_row_bytes, r the
+// matrix, p the list position; zeros for an id outside [hot, d_ff)).
+cudaError_t launch_stage_cold(const pi_layer& L, const int32_t* idx, const int32_t* count,
+                              char* stage, WsHeader* hdr, cudaStream_t s);
+// Copies their w_down_t rows to stage[p]: with h ([n][batch] fp32), only the
+// rows whose h is nonzero for some token; without, every listed row.
+cudaError_t launch_stage_cold_down(const pi_layer& L, int batch, const int32_t* idx,
+                                   const int32_t* count, const float* h, char* stage,
+                                   WsHeader* hdr, cudaStream_t s);
+
 // part[s][b][:] = sum over the slice's rows of h[n][b] * w_down_t[row n],
 // the list positions [nb, H + count) split into `splits` slices
 // `stage`: as for launch_ffn_up (the same buffer); a cold-tier layer's down

@@ -501,9 +501,10 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
     k_ffn_up_q4tc(const __grid_constant__ CUtensorMap mx, const char* __restrict__ cw0,
                   const char* __restrict__ sw0, int64_t cst0, int64_t sst0,
                   const char* __restrict__ cw1, const char* __restrict__ sw1, int64_t cst1,
-                  int64_t sst1, int nt, int nk, int g, int H, int F,
-                  const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
-                  float* __restrict__ part, WsHeader* hdr) {
+                  int64_t sst1, const char* __restrict__ cc0, const char* __restrict__ cc1,
+                  int64_t cstr, int cscb, int nt, int nk,
+                  int g, int H, int F, const int32_t* __restrict__ idx,
+                  const int32_t* __restrict__ count, float* __restrict__ part, WsHeader* hdr) {
   pdl_wait();
   pdl_trigger();
   constexpr int NS = 2;
@@ -539,9 +540,17 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
 
   if (threadIdx.x < TC_Q4_LOADERS) {
     const int t = threadIdx.x, m = t >> 1, h = t & 1;
-    const int row = list_row(p0 + m, H, N, F, idx);
-    const char* cp[2] = {cw0 + (size_t)row * cst0, NR == 2 ? cw1 + (size_t)row * cst1 : nullptr};
-    const char* sp[2] = {sw0 + (size_t)row * sst0, NR == 2 ? sw1 + (size_t)row * sst1 : nullptr};
+    const int p = p0 + m, row = list_row(p, H, N, F, idx);
+    // a host-memory cold tier's listed rows were staged in device memory at
+    // their list positions (cc0 / cc1: codes, scales cscb bytes behind; a
+    // bad id staged as zeros); positions past the list read staged row 0
+    // when there is no hot row 0 to read
+    const bool cold = cc0 && p >= H && (p < N || H == 0);
+    const size_t cq0 = (size_t)(p < N ? p - H : 0) * cstr;
+    const char* cp[2] = {cold ? cc0 + cq0 : cw0 + (size_t)row * cst0,
+                         NR == 2 ? (cold ? cc1 + cq0 : cw1 + (size_t)row * cst1) : nullptr};
+    const char* sp[2] = {cold ? cc0 + cq0 + cscb : sw0 + (size_t)row * sst0,
+                         NR == 2 ? (cold ? cc1 + cq0 + cscb : sw1 + (size_t)row * sst1) : nullptr};
     uint4 cq[TC_Q4_PRE][NR][KB];
     uint32_t sq[TC_Q4_PRE][NR];
     // codes and scales of stage i into register slot u
@@ -672,7 +681,8 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
 // the codes that depend on them, the codes TC_Q4_PRE - 1 stages ahead.
 __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
     k_ffn_down_q4tc(const __grid_constant__ CUtensorMap mh, const char* __restrict__ cw,
-                    const char* __restrict__ sw, int64_t cst, int64_t sst, int nt, int ks, int d,
+                    const char* __restrict__ sw, int64_t cst, int64_t sst,
+                    const char* __restrict__ cwc, int64_t cstr, int cscb, int nt, int ks, int d,
                     int batch, int H, int F, const int32_t* __restrict__ idx,
                     const int32_t* __restrict__ count, float* __restrict__ part, WsHeader* hdr) {
   pdl_wait();
@@ -721,8 +731,13 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
     auto row_of = [&](int i) { return i < nkt ? list_row((kt0 + i) * TC_BK + k, H, N, F, idx) : 0; };
     auto fetch = [&](int i, int u) {
       if (i < nkt) {
-        cq[u] = ld_q4_codes(cw + (size_t)rq[u] * cst + cb);
-        sq[u] = ld_q4_scale(sw + (size_t)rq[u] * sst + sb);
+        // a host-memory cold tier's listed rows, staged at their list
+        // positions (as in the up kernel)
+        const int pos = (kt0 + i) * TC_BK + k;
+        const bool cold = cwc && pos >= H && (pos < N || H == 0);
+        const size_t cq0 = (size_t)(pos < N ? pos - H : 0) * cstr;
+        cq[u] = ld_q4_codes(cold ? cwc + cq0 + cb : cw + (size_t)rq[u] * cst + cb);
+        sq[u] = ld_q4_scale(cold ? cwc + cq0 + cscb + sb : sw + (size_t)rq[u] * sst + sb);
       }
     };
 #pragma unroll
@@ -1443,7 +1458,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
 template <int NR>
 cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                          const int32_t* idx, const int32_t* count, void* scratch, WsHeader* hdr,
-                         cudaStream_t s, bool xh16_ready) {
+                         cudaStream_t s, bool xh16_ready, char* cold_stage) {
   const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
@@ -1459,6 +1474,15 @@ cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const ui
                      batch, d, nt, sc.xh16);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  // a host-memory cold tier: its listed rows first, once, into the stage
+  const int64_t srb = stage_row_bytes(PI_Q4_0, d);
+  const char *cc0 = nullptr, *cc1 = nullptr;
+  if (L.w_up_cold) {
+    if (!cold_stage) return cudaErrorInvalidValue;
+    if ((e = launch_stage_cold(L, idx, count, cold_stage, hdr, s)) != cudaSuccess) return e;
+    cc0 = cold_stage;
+    cc1 = cold_stage + (size_t)(F - H) * srb;
+  }
   constexpr int KB = NR == 1 ? 2 : 1;
   const int nk = d / (64 * KB), g = 2 * device_sms();
   const uint32_t stage = NR * KB * TC_M * 128 + (((uint32_t)nt * 128 * KB + 1023u) & ~1023u);
@@ -1468,8 +1492,8 @@ cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const ui
   (void)launch_dep(k_ffn_up_q4tc<NR, KB>, std::max(g, Fp / TC_M), 32 * TC_Q4_WARPS, smem, s, mx, cw0,
                    sw0, code_stride(PI_Q4_0, d, L.w_row_stride), scale_stride(d, L.w_row_stride),
                    static_cast<const char*>(L.w_up), static_cast<const char*>(L.w_up_scales),
-                   code_stride(PI_Q4_0, d, ur), scale_stride(d, ur), nt, nk, g, H, F, idx, count,
-                   sc.part, hdr);
+                   code_stride(PI_Q4_0, d, ur), scale_stride(d, ur),
+                   cc0, cc1, srb, d / 2, nt, nk, g, H, F, idx, count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, H, F, Fp, nt, batch, idx,
@@ -1483,7 +1507,10 @@ bool ffn_tc_supported(const pi_layer& L, int batch) {
   if (tc_disabled()) return false;
   if ((L.w_dtype != PI_F16 && L.w_dtype != PI_Q4_0) || batch < TC_MIN_BATCH || batch > TC_TMAX)
     return false;
-  if (L.d_model % TC_M != 0 || L.w_up_cold) return false;  // no host-memory cold tier
+  if (L.d_model % TC_M != 0) return false;
+  // a host-memory cold tier: the Q4_0 kernels' loaders read its rows with
+  // plain loads; the fp16 kernels' TMA loads read device memory only
+  if (L.w_up_cold && L.w_dtype != PI_Q4_0) return false;
   if (L.w_dtype == PI_Q4_0) {
     // 16-byte code loads, 4-byte scale loads (two scales at a time)
     const int d = L.d_model;
@@ -1499,6 +1526,11 @@ bool ffn_tc_supported(const pi_layer& L, int batch) {
     const uintptr_t scales = (uintptr_t)L.w_up_scales | (uintptr_t)L.w_down_t_scales |
                              (uintptr_t)(L.act == PI_REGLU ? L.w_gate_scales : L.w_up_scales);
     if ((codes & 15u) || (scales & 3u)) return false;
+    const uintptr_t ccodes = (uintptr_t)L.w_up_cold | (uintptr_t)L.w_down_t_cold |
+                             (uintptr_t)L.w_gate_cold;
+    const uintptr_t cscales = (uintptr_t)L.w_up_cold_scales | (uintptr_t)L.w_down_t_cold_scales |
+                              (uintptr_t)L.w_gate_cold_scales;
+    if ((ccodes & 15u) || (cscales & 3u)) return false;
     return tensor_map_encoder() != nullptr;
   }
   const int64_t rs = code_stride(PI_F16, L.d_model, L.w_row_stride);
@@ -1590,19 +1622,25 @@ int ffn_tc_down_splits(const pi_layer& L) {
 
 cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                              const int32_t* idx, const int32_t* count, void* scratch,
-                             WsHeader* hdr, cudaStream_t s, bool xh16_ready) {
+                             WsHeader* hdr, cudaStream_t s, bool xh16_ready, char* stage) {
   if (L.w_dtype == PI_Q4_0)
     return L.act == PI_REGLU
-               ? launch_up_q4<2>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready)
-               : launch_up_q4<1>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready);
+               ? launch_up_q4<2>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready, stage)
+               : launch_up_q4<1>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready, stage);
   return L.act == PI_REGLU
              ? launch_up_nr<2>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready)
              : launch_up_nr<1>(L, xh, batch, mask, idx, count, scratch, hdr, s, xh16_ready);
 }
 
+size_t tc_cold_stage_bytes(const pi_layer& L) {
+  if (!L.w_up_cold || L.w_dtype != PI_Q4_0) return 0;
+  return (size_t)(L.d_ff - L.hot) * (size_t)stage_row_bytes(PI_Q4_0, L.d_model) *
+         (L.act == PI_REGLU ? 3u : 2u);
+}
+
 cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
                                const int32_t* count, float* part, void* scratch, WsHeader* hdr,
-                               cudaStream_t s) {
+                               cudaStream_t s, char* cold_stage) {
   const int d = L.d_model, H = L.hot, F = L.d_ff, Fp = fpad(F);
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, L.rank);
@@ -1616,12 +1654,22 @@ cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
     const size_t smem = 1024 + 4 * (size_t)stage + 8 * (2 * 4 + 1) + 16;
     cudaError_t e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_down_q4tc), smem);
     if (e != cudaSuccess) return e;
+    // a host-memory cold tier: every listed down row, once, into the stage
+    // behind the up kernel's (the kernel reads every listed position)
+    const int64_t srb = stage_row_bytes(PI_Q4_0, d);
+    char* cwc = nullptr;
+    if (L.w_up_cold) {
+      if (!cold_stage) return cudaErrorInvalidValue;
+      cwc = cold_stage + (size_t)(F - H) * srb * (L.act == PI_REGLU ? 2u : 1u);
+      if ((e = launch_stage_cold_down(L, batch, idx, count, nullptr, cwc, hdr, s)) != cudaSuccess)
+        return e;
+    }
     (void)launch_dep(k_ffn_down_q4tc, dim3(tiles, ks), 32 * TC_Q4_WARPS, smem, s, mh,
                      static_cast<const char*>(L.w_down_t),
                      static_cast<const char*>(L.w_down_t_scales),
                      code_stride(PI_Q4_0, d, L.w_down_row_stride),
-                     scale_stride(d, L.w_down_row_stride), nt, ks, d, batch, H, F, idx, count,
-                     part, hdr);
+                     scale_stride(d, L.w_down_row_stride),
+                     cwc, srb, d / 2, nt, ks, d, batch, H, F, idx, count, part, hdr);
     return cudaGetLastError();
   }
   const int64_t rd = code_stride(PI_F16, d, L.w_down_row_stride);

@@ -39,9 +39,16 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
 // fp16 activations in `scratch` for launch_ffn_down_tc.  xh16_ready: the
 // fp16 copy of xh in `scratch` is already current (launch_predict_tc wrote
 // it from the same xh and batch), so it is not rebuilt.
+// cold_stage (at least tc_cold_stage_bytes(L)): a Q4_0 layer with a
+// host-memory cold tier copies its listed cold rows there first, once.
 cudaError_t launch_ffn_up_tc(const pi_layer& L, const float* xh, int batch, const uint32_t* mask,
                              const int32_t* idx, const int32_t* count, void* scratch,
-                             WsHeader* hdr, cudaStream_t s, bool xh16_ready = false);
+                             WsHeader* hdr, cudaStream_t s, bool xh16_ready = false,
+                             char* cold_stage = nullptr);
+
+// Device bytes the tensor-core kernels stage a Q4_0 cold tier's listed rows
+// in (0: no cold tier).
+size_t tc_cold_stage_bytes(const pi_layer& L);
 
 // Split-K slices the down projection writes (part[0 .. splits)).
 int ffn_tc_down_splits(const pi_layer& L);
@@ -50,6 +57,6 @@ int ffn_tc_down_splits(const pi_layer& L);
 // the list positions of h[p][b] * w_down_t[row(p)].
 cudaError_t launch_ffn_down_tc(const pi_layer& L, int batch, const int32_t* idx,
                                const int32_t* count, float* part, void* scratch, WsHeader* hdr,
-                               cudaStream_t s);
+                               cudaStream_t s, char* cold_stage = nullptr);
 
 }  // namespace pi

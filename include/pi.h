@@ -130,10 +130,14 @@ typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_m
  * (w_gate_cold for ReGLU, the scale arrays for Q4_0), with the alignment of
  * their device counterparts.  The GPU reads the cold rows over the host
  * link (PCIe or C2C) and merges them in the same kernels as the hot rows:
- * the result is the same as with every row in device memory.  Such layers
- * always take the multi-kernel CUDA-core path (batch 1 included), and their
- * host memory must stay allocated and unchanged until the stream has run
- * the call. */
+ * the result is the same as with every row in device memory on those
+ * kernels.  Such layers take the multi-kernel path (batch 1 included): the
+ * CUDA-core kernels, or for Q4_0 layers at 2-64 tokens the tensor-core
+ * kernels.  Where those kernels would read a row more than once (several
+ * token chunks, or the tensor cores' tiles), each call first copies the
+ * listed cold rows into the workspace once (pi_workspace_bytes counts that
+ * stage).  The host memory must stay allocated and unchanged until the
+ * stream has run the call. */
 typedef struct pi_layer {
   int32_t d_model, d_ff, rank, hot;
   int32_t act, w_dtype, p_dtype;

@@ -122,6 +122,53 @@ def test_cold_tier_sparse_ffn(pi, orc, act, wdt, batch, mode, packed, monkeypatc
         assert down <= (listed if chunks >= 4 else listed * chunks)
 
 
+@pytest.mark.parametrize("act", ["relu", "reglu", "relu2"])
+@pytest.mark.parametrize("batch,mode,packed", [(2, "per_token", True), (5, "union", False),
+                                               (16, "per_token", True), (64, "union", True),
+                                               (64, "per_token", False)])
+def test_cold_tier_q4_on_tensor_cores(pi, orc, act, batch, mode, packed):
+    """Q4_0 layers at token batches take the tensor-core kernels with a cold
+    tier too: the listed cold rows (and every listed down row) are staged in
+    device memory once, then read by the same kernels, so the result equals
+    the device-resident layer's bit for bit."""
+    w = _wl(act, "q4_0", (1024, 3001, 128, 640), seed=49)
+    L, _ = device_layer(w, 0, packed=packed)
+    H = synth.layer_host(w, 0)
+    xh = _xh(w.d_model, batch, 8)
+    masks, union = _list_and_masks(orc, w, H, xh)
+    m = pi.MODES[mode]
+    idx = torch.zeros(w.d_ff, dtype=torch.int32, device="cuda")
+    idx[: len(union)] = torch.from_numpy(union).cuda()
+    cnt = torch.tensor([len(union)], dtype=torch.int32, device="cuda")
+    xd = torch.from_numpy(xh).cuda()
+    md = torch.from_numpy(masks.view(np.int32)).cuda()
+    n0 = pi.pi_kernel_launches()
+    y_dev = pi.pi_sparse_ffn(L, xd, md, idx, cnt, m).clone()
+    launches_dev = pi.pi_kernel_launches() - n0
+    Lc = L.with_host_cold_tier()
+    _poison_cold_rows(L)
+    ws = pi.workspace([Lc], batch)
+    pi.pi_read_cold_counters(ws, clear=True)
+    pi.pi_read_counters(ws, clear=True)
+    n0 = pi.pi_kernel_launches()
+    y = pi.pi_sparse_ffn(Lc, xd, md, idx, cnt, m, ws=ws)
+    launches = pi.pi_kernel_launches() - n0
+    torch.cuda.synchronize()
+    assert torch.equal(y, y_dev)
+    yn = y.cpu().numpy()
+    for b in range(batch):
+        own = orc.compact(masks[b], w.d_ff, w.hot) if mode == "per_token" else union
+        ref = orc.sparse_ffn(H, xh[b].astype(np.float64), own)
+        assert rel_l2(yn[b], ref) <= TOL["q4_0"], b
+    listed, down, second = pi.pi_read_cold_counters(ws)
+    assert listed == len(union) and down == len(union)
+    assert second == (len(union) if act == "reglu" else 0)
+    # the tensor-core path read every listed row once (its own counters)
+    rows_listed, rows_down, _ = pi.pi_read_counters(ws)
+    assert rows_listed == w.hot + len(union) and rows_down == w.hot + len(union)
+    assert launches == launches_dev + 2  # the two staging kernels, then the same FFN kernels
+
+
 @pytest.mark.parametrize("act,wdt", [("reglu", "q4_0"), ("relu", "f16"), ("relu2", "f32")])
 @pytest.mark.parametrize("batch,mode", [(1, "union"), (4, "per_token"), (8, "union")])
 def test_cold_tier_stack(pi, orc, act, wdt, batch, mode, monkeypatch):
