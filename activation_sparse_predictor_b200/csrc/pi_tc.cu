@@ -256,14 +256,37 @@ __host__ __device__ constexpr int up_stages(int nr, int nt) {
 // 4 ks / nk of the tile's weight bytes; ks <= nk / 32 keeps that near 1/8.
 // Partial sums are laid out [ks][NR][nT * 128][nt].  The same function
 // sizes the work on both sides of the finish kernel.
+//
+// fit (the Q4_0 kernel, bound by its loaders rather than by HBM, two CTAs
+// per SM): g is the number of resident CTA slots and ks the split, up to
+// the cap, that fills the last wave of nT * ks CTAs best (the largest
+// split within 2 % of the best fill: more, shorter CTAs balance the SMs
+// better), so that few SMs run one CTA while others run two.  (Llama2-70B
+// shape, tokens/s: 8 tokens 402 -> 472, 16 tokens 578 -> 759, 64 tokens
+// 1892 -> 2167 against ks = g / nT.)
 struct UpShare {
   int nT, ks;
 };
-__host__ __device__ inline UpShare up_share(int N, int g, int nk) {
+__host__ __device__ inline UpShare up_share(int N, int g, int nk, bool fit = false) {
   UpShare u;
   u.nT = (N + TC_M - 1) / TC_M;
-  int ks = u.nT > 0 ? g / u.nT : 1;
   const int cap = nk / 32 > 1 ? nk / 32 : 1;
+  if (fit && u.nT > 0) {
+    auto fill = [&](int k) {
+      const int c = u.nT * k, w = (c + g - 1) / g;
+      return (float)c / (float)(w * g);
+    };
+    float be = 0.f;
+    for (int k = 1; k <= cap; ++k) be = fmaxf(be, fill(k));
+    u.ks = 1;
+    for (int k = cap; k >= 1; --k)
+      if (fill(k) >= be - 0.02f) {
+        u.ks = k;
+        break;
+      }
+    return u;
+  }
+  int ks = u.nT > 0 ? g / u.nT : 1;
   u.ks = ks < 1 ? 1 : (ks > cap ? cap : ks);
   return u;
 }
@@ -523,7 +546,7 @@ __global__ void __launch_bounds__(32 * TC_Q4_WARPS, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int N = list_len(count, H, F, hdr);
-  const UpShare us = up_share(N, g, nk);
+  const UpShare us = up_share(N, g, nk, true);
   const int ks = us.ks, Np = us.nT * TC_M;
   if ((int)blockIdx.x >= us.nT * ks) return;
   const int tile = blockIdx.x / ks, split = blockIdx.x % ks;
@@ -868,7 +891,7 @@ __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
 // Partial sums read and h16 written coalesced through shared memory.
 template <int NR>
 __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ part, int g, int nk,
-                                                    int H, int F, int Fp, int nt, int batch,
+                                                    int fit, int H, int F, int Fp, int nt, int batch,
                                                     const int32_t* __restrict__ idx,
                                                     const int32_t* __restrict__ count,
                                                     const float* __restrict__ bias,
@@ -888,7 +911,7 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
   }
   const int n0 = blockIdx.x * 64;
   if (n0 >= N) return;
-  const UpShare us = up_share(N, g, nk);
+  const UpShare us = up_share(N, g, nk, fit != 0);
   const int ks = us.ks, Np = us.nT * TC_M;
   const int m = 64 * nt;
   // per row once: neuron, index check, bias
@@ -1395,8 +1418,10 @@ TcScratch tc_scratch(void* base, int d, int F, int r) {
   t.xh16 = reinterpret_cast<__half*>(p);
   p += up256((size_t)TC_TMAX * d * 2);
   t.part = reinterpret_cast<float*>(p);
-  // nT * ks <= up_grid(F) partial row tiles of two operands
-  p += up256((size_t)up_grid(F) * TC_M * 2 * TC_TMAX * 4);
+  // nT * ks <= up_grid(F) partial row tiles of two operands (fp16), or
+  // (Fp / 128) * (d / 2048) (Q4_0: up to nk / 32 shares per tile, nk <= d / 64)
+  const size_t ptiles = std::max((size_t)up_grid(F), (size_t)(fpad(F) / TC_M) * std::max(1, d / 2048));
+  p += up256(ptiles * TC_M * 2 * TC_TMAX * 4);
   t.h16 = reinterpret_cast<__half*>(p);
   p += up256((size_t)TC_TMAX * fpad(F) * 2);
   t.xlo = reinterpret_cast<__half*>(p);
@@ -1447,7 +1472,7 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
                    F, idx, count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, H, F, Fp, nt, batch, idx,
+  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, 0, H, F, Fp, nt, batch, idx,
                    count, L.bias, mask, (F + 31) / 32, sc.h16, hdr, L.act == PI_RELU2 ? 1 : 0);
   return cudaGetLastError();
 }
@@ -1489,14 +1514,16 @@ cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const ui
   const size_t smem = 1024 + 2 * (size_t)stage + 8 * (2 * 2 + 1) + 16;
   e = allow_smem_fn(reinterpret_cast<const void*>(k_ffn_up_q4tc<NR, KB>), smem);
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_up_q4tc<NR, KB>, std::max(g, Fp / TC_M), 32 * TC_Q4_WARPS, smem, s, mx, cw0,
+  // up to nk / 32 shares of each of at most Fp / 128 row tiles (up_share, fit)
+  const int grid = std::max(g, (Fp / TC_M) * std::max(1, nk / 32));
+  (void)launch_dep(k_ffn_up_q4tc<NR, KB>, grid, 32 * TC_Q4_WARPS, smem, s, mx, cw0,
                    sw0, code_stride(PI_Q4_0, d, L.w_row_stride), scale_stride(d, L.w_row_stride),
                    static_cast<const char*>(L.w_up), static_cast<const char*>(L.w_up_scales),
                    code_stride(PI_Q4_0, d, ur), scale_stride(d, ur),
                    cc0, cc1, srb, d / 2, nt, nk, g, H, F, idx, count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, H, F, Fp, nt, batch, idx,
+  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, 1, H, F, Fp, nt, batch, idx,
                    count, L.bias, mask, (F + 31) / 32, sc.h16, hdr, L.act == PI_RELU2 ? 1 : 0);
   return cudaGetLastError();
 }
