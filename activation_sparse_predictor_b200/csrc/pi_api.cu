@@ -328,16 +328,17 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
     return PI_OK;
   };
   if (stack1_supported(layers, n_layers, batch)) return fused(x, mask_trace);
-  // Q4_0 stacks with per-token masks below 8 tokens (or where the layers
+  // Q4_0 stacks with per-token masks below 5 tokens (or where the layers
   // do not qualify for the tensor cores): each token's per-token FFN is the
   // single-token computation on that token, and one fused pass per token
-  // (Llama2-70B shape: 3.5 ms) costs less than a batched step there (16 ms
-  // at 4 tokens on the tensor cores, 41 ms on the CUDA-core kernels, which
-  // dequantize every weight block to fp32 for every token).  A mask trace
+  // (Llama2-70B shape: 3.5 ms, 286 tokens/s) costs less than a batched step
+  // there (262 tokens/s at 4 tokens on the tensor cores, 377 at 6; 97 at 4
+  // on the CUDA-core kernels, which dequantize every weight block to fp32
+  // for every token).  A mask trace
   // keeps the batched path, whose trace layout is [layer][token][word].
   if (batch > 1 && mode == PI_MASK_PER_TOKEN && !mask_trace && !trace &&
       layers[0].w_dtype == PI_Q4_0 && stack1_supported(layers, n_layers, 1) &&
-      (batch < 8 || !ffn_tc_supported(layers[0], batch))) {
+      (batch < 5 || !ffn_tc_supported(layers[0], batch))) {
     const int d = layers[0].d_model;
     for (int b = 0; b < batch; ++b) {
       if ((st = fused(x + (size_t)b * d, nullptr)) != PI_OK) return st;

@@ -253,7 +253,7 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch,
  * aligned scale arrays) the whole stack runs in one persistent cooperative
  * kernel per 24 layers; otherwise as a sequence of per-step kernels (fp16
  * and Q4_0 layers at 2-64 tokens on the tensor cores).  Q4_0 stacks that
- * meet the single-token conditions run below 8 tokens with
+ * meet the single-token conditions run below 5 tokens with
  * PI_MASK_PER_TOKEN and no mask_trace as one persistent pass per token,
  * which gives each token its per-token FFN exactly.  Setting the
  * environment variable PI_DISABLE_FUSED=1 forces the sequence.  All layers
