@@ -59,7 +59,7 @@ constexpr int NCT = NCW * 32;       // consumer threads
 constexpr int NPMAX = 3;            // producer warps (after the consumers)
 constexpr int NTHR = NCT + 32 * (NPMAX + 1);  // + the compaction warp
 constexpr int NSMAX = 24;           // ring stages at most
-constexpr int MAXL = 24;            // layers per launch
+constexpr int MAXL = 40;            // layers per launch (the parameter block stays under 4 KB)
 constexpr int MAXA = 16;            // P1 rows per CTA at most
 constexpr unsigned long long kTimeoutNs = 1000000000ull;  // 1 s per wait
 constexpr int UTR = 512;            // units per layer recorded by the unit trace

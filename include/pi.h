@@ -251,7 +251,7 @@ pi_status pi_sparse_ffn(const pi_layer* layer, const float* xh, int batch,
  * (d_model <= 12288, rank <= 1024 for an fp16 predictor and <= 512 for an
  * fp32 one; Q4_0 also d_model <= 8192, d_model % 256 == 0 and 16-byte
  * aligned scale arrays) the whole stack runs in one persistent cooperative
- * kernel per 24 layers; otherwise as a sequence of per-step kernels (fp16
+ * kernel per 40 layers; otherwise as a sequence of per-step kernels (fp16
  * and Q4_0 layers at 2-64 tokens on the tensor cores).  Q4_0 stacks that
  * meet the single-token conditions run below 5 tokens with
  * PI_MASK_PER_TOKEN and no mask_trace as one persistent pass per token,

@@ -275,7 +275,7 @@ def test_stack_is_deterministic(pi, packed):
 
 
 def test_kernel_launch_counter(pi):
-    """One fused launch per batch-1 stack call of at most 24 layers; the same
+    """One fused launch per batch-1 stack call of at most 40 layers; the same
     count on every repeat of a multi-kernel (batch 4, union) call."""
     w = _wl("reglu", "q4_0", (512, 1500, 64, 256), seed=44).scaled(4)
     layers = [device_layer(w, l, packed=True)[0] for l in range(4)]

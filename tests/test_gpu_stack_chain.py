@@ -1,7 +1,7 @@
 """The benchmarked batch-1 path end to end: stacks deeper than one launch of
-the persistent kernel (it runs at most 24 layers per launch), checked layer
+the persistent kernel (it runs at most 40 layers per launch), checked layer
 by layer against the oracle, so the hand-off of x, of the mask trace and of
-the layer pointers at the launch boundaries (layers 24 and 48) is pinned.
+the layer pointers at the launch boundaries (layers 40 and 80) is pinned.
 
 For every prefix length n the stack is run from the same x0 on the GPU; by
 determinism the prefix's output is the full stack's x after n layers (this
@@ -27,7 +27,7 @@ from oracle import rel_l2
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-N_LAYERS = 52  # crosses the persistent kernel's launch boundaries at 24 and 48
+N_LAYERS = 84  # crosses the persistent kernel's launch boundaries at 40 and 80
 
 
 def _workload(act, w_dtype, seed):
