@@ -263,14 +263,15 @@ pi_status ffn_body(const pi_layer& L, const float* xh, int batch, const uint32_t
 // it did.
 pi_status predict_body(const pi_layer& L, const float* xh, int batch, float theta, uint32_t* mask,
                        void* ws, const WsLayout& lay, cudaStream_t s, Prof* prof = nullptr,
-                       uint32_t* uni = nullptr, bool* uni_done = nullptr) {
+                       uint32_t* uni = nullptr, bool* uni_done = nullptr, bool split_ready = false) {
   Prof none;
   Prof& P = prof ? *prof : none;
   cudaError_t e;
   if (uni_done) *uni_done = false;
   if (pred_tc_supported(L, batch)) {
     P.before(PI_KIND_PRED_U);
-    e = launch_predict_tc(L, xh, batch, theta, mask, at<void>(ws, lay.tc), header(ws), s, uni);
+    e = launch_predict_tc(L, xh, batch, theta, mask, at<void>(ws, lay.tc), header(ws), s, uni,
+                          split_ready);
     if (uni_done) *uni_done = uni != nullptr;
     P.after();
     return e == cudaSuccess ? PI_OK : cuda_fail(e, "predictor (tensor cores) launch");
@@ -353,8 +354,12 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
   for (int l = 0; l < n_layers; ++l) {
     const pi_layer& L = layers[l];
     uint32_t* mask = mask_trace ? mask_trace + (size_t)l * batch * words : at<uint32_t>(ws, lay.mask);
+    // with the tensor-core predictor, the RMSNorm also writes its fp16 operands
+    const bool ptc = pred_tc_supported(L, batch);
+    void *hi = nullptr, *lo = nullptr;
+    if (ptc) tc_split_buffers(L, at<void>(ws, lay.tc), &hi, &lo);
     P.before(PI_KIND_RMSNORM);
-    cudaError_t e = launch_rmsnorm(x, batch, d, xh, s);
+    cudaError_t e = launch_rmsnorm(x, batch, d, xh, s, hi, lo, (batch + 15) / 16 * 16);
     P.after();
     if (e != cudaSuccess) return cuda_fail(e, "rmsnorm launch");
     // at token batches the tokens' union goes into the activation buffer
@@ -362,7 +367,7 @@ pi_status stack_run(const pi_layer* layers, int n_layers, float* x, int batch, f
     // epilogue, else from a union kernel; then one list from it
     uint32_t* uni = batch > 1 ? at<uint32_t>(ws, lay.h) : nullptr;
     bool uni_done = false;
-    if ((st = predict_body(L, xh, batch, theta, mask, ws, lay, s, prof, uni, &uni_done)) != PI_OK)
+    if ((st = predict_body(L, xh, batch, theta, mask, ws, lay, s, prof, uni, &uni_done, ptc)) != PI_OK)
       return st;
     P.before(PI_KIND_COMPACT);
     if (batch > 1) {

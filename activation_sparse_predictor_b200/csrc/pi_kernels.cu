@@ -128,10 +128,23 @@ struct RowDot {
 // One CTA per row (d <= 16384, d % 4 == 0): the row is read once into
 // registers (up to four float4 per thread), its mean square reduced across
 // the CTA, and the scaled row written from the registers.
+// xh = x / sqrt(mean(x^2) + 1e-6), one CTA per token.  With hi / lo (the
+// tensor-core predictor's operands, [nt][d] fp16), also hi = fp16(xh) and
+// lo = fp16(xh - hi), and zero rows for the padding tokens batch .. nt-1
+// (CTAs past the batch), which the predictor would otherwise build in a
+// kernel of its own.
 __global__ void __launch_bounds__(1024) k_rmsnorm(const float* __restrict__ x, int d,
-                                                  float* __restrict__ xh) {
+                                                  float* __restrict__ xh, int batch,
+                                                  __half* __restrict__ hi, __half* __restrict__ lo) {
   pdl_wait();
   pdl_trigger();
+  if ((int)blockIdx.x >= batch) {  // a padding token of the fp16 operands
+    for (int i = threadIdx.x; i < d / 4; i += blockDim.x) {
+      reinterpret_cast<uint2*>(hi + (size_t)blockIdx.x * d)[i] = make_uint2(0u, 0u);
+      reinterpret_cast<uint2*>(lo + (size_t)blockIdx.x * d)[i] = make_uint2(0u, 0u);
+    }
+    return;
+  }
   const float4* xr = reinterpret_cast<const float4*>(x + (size_t)blockIdx.x * d);
   float4* yr = reinterpret_cast<float4*>(xh + (size_t)blockIdx.x * d);
   const int n4 = d >> 2;
@@ -160,7 +173,20 @@ __global__ void __launch_bounds__(1024) k_rmsnorm(const float* __restrict__ x, i
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int i = threadIdx.x + k * blockDim.x;
-    if (i < n4) yr[i] = make_float4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
+    if (i >= n4) continue;
+    const float4 y = make_float4(v[k].x * inv, v[k].y * inv, v[k].z * inv, v[k].w * inv);
+    yr[i] = y;
+    if (hi) {
+      const float e[4] = {y.x, y.y, y.z, y.w};
+      __align__(8) __half h[4], l[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        h[m] = __float2half_rn(e[m]);
+        l[m] = __float2half_rn(e[m] - __half2float(h[m]));
+      }
+      reinterpret_cast<uint2*>(hi + (size_t)blockIdx.x * d)[i] = *reinterpret_cast<const uint2*>(h);
+      reinterpret_cast<uint2*>(lo + (size_t)blockIdx.x * d)[i] = *reinterpret_cast<const uint2*>(l);
+    }
   }
 }
 
@@ -865,10 +891,12 @@ int down_splits(int batch, int d) {
 
 // ---------------------------------------------------------------- launches
 
-cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s) {
+cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s,
+                           void* hi, void* lo, int nt) {
   // one float4 per thread up to d = 4096, then 1024 threads with up to four
   const int n4 = d / 4, threads = std::min(1024, (n4 + 31) / 32 * 32);
-  (void)launch_dep(k_rmsnorm, batch, threads, 0, s, x, d, xh);
+  (void)launch_dep(k_rmsnorm, hi ? nt : batch, threads, 0, s, x, d, xh, batch,
+                   static_cast<__half*>(hi), static_cast<__half*>(lo));
   return cudaGetLastError();
 }
 

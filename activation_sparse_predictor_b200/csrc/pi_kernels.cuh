@@ -62,7 +62,10 @@ int down_tb(int batch);           // tokens per pass of the down projection
 int down_splits(int batch, int d);// split-K slices of the down projection
 
 // xh[b] = x[b] / sqrt(mean(x[b]^2) + 1e-6), b < batch.
-cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s);
+// xh = rmsnorm(x) per token; with hi / lo ([nt][d] fp16, nt >= batch) also
+// the split hi = fp16(xh), lo = fp16(xh - hi), zero rows past the batch.
+cudaError_t launch_rmsnorm(const float* x, int batch, int d, float* xh, cudaStream_t s,
+                           void* hi = nullptr, void* lo = nullptr, int nt = 0);
 
 // u[b][k] = p1[k] . xh[b]
 cudaError_t launch_pred_u(const pi_layer& L, const float* xh, int batch, float* u,

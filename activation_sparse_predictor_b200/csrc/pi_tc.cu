@@ -1584,9 +1584,15 @@ bool pred_tc_supported(const pi_layer& L, int batch) {
   return tensor_map_encoder() != nullptr;
 }
 
+void tc_split_buffers(const pi_layer& L, void* scratch, void** hi, void** lo) {
+  const TcScratch sc = tc_scratch(scratch, L.d_model, L.d_ff, L.rank);
+  *hi = sc.xh16;
+  *lo = sc.xlo;
+}
+
 cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, float theta,
                               uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s,
-                              uint32_t* uni) {
+                              uint32_t* uni, bool split_ready) {
   const int d = L.d_model, r = L.rank, F = L.d_ff, H = L.hot, words = (F + 31) / 32;
   const int nt = (batch + 15) / 16 * 16;
   const TcScratch sc = tc_scratch(scratch, d, F, r);
@@ -1599,10 +1605,12 @@ cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, flo
       !map_2d(&mul, sc.ulo, (uint64_t)r, (uint64_t)nt, (uint64_t)r * 2, (uint32_t)nt))
     return cudaErrorInvalidValue;
   const int grid = device_sms() * 4;
-  (void)launch_dep(k_split16, std::min((nt * d / 8 + 255) / 256, grid), 256, 0, s, xh, batch, d, nt,
-                   sc.xh16, sc.xlo);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!split_ready) {
+    (void)launch_dep(k_split16, std::min((nt * d / 8 + 255) / 256, grid), 256, 0, s, xh, batch, d,
+                     nt, sc.xh16, sc.xlo);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   constexpr uint32_t STAGE = TC_M * TC_BK * 2 + 2 * TC_TMAX * TC_BK * 2;
   const size_t smem = 1024 + (size_t)TC_PSTAGES * STAGE + 8 * (2 * TC_PSTAGES + 1) + 16;
   e = allow_smem_fn(reinterpret_cast<const void*>(k_pred_tc<0>), smem);

@@ -28,9 +28,15 @@ bool pred_tc_supported(const pi_layer& L, int batch);
 // (fp32 accumulation); bit j = j < hot or z_j > theta.  `uni` (optional,
 // [words]): the OR of the tokens' words, written for the words from the
 // one holding `hot` on (the words below are not written).
+// split_ready: the fp16 hi / lo split of xh in `scratch` (tc_split_buffers)
+// is already current (the stack's RMSNorm wrote it), so it is not rebuilt.
 cudaError_t launch_predict_tc(const pi_layer& L, const float* xh, int batch, float theta,
                               uint32_t* mask, void* scratch, WsHeader* hdr, cudaStream_t s,
-                              uint32_t* uni = nullptr);
+                              uint32_t* uni = nullptr, bool split_ready = false);
+
+// The predictor's fp16 operands of xh in `scratch`: hi and lo, [nt][d_model]
+// each, nt = batch rounded up to 16.
+void tc_split_buffers(const pi_layer& L, void* scratch, void** hi, void** lo);
 
 // Up/gate products of list positions [0, hot + count) (row p for p < hot,
 // idx[p - hot] after) with xh [batch][d_model] (fp32, rounded to fp16 for
