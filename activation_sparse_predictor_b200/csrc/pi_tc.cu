@@ -300,7 +300,9 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
                 const __grid_constant__ CUtensorMap mg0, const __grid_constant__ CUtensorMap mg1,
                 const __grid_constant__ CUtensorMap mx, int nt, int nk, int g, int H, int F,
                 const int32_t* __restrict__ idx, const int32_t* __restrict__ count,
-                float* __restrict__ part, WsHeader* hdr) {
+                float* __restrict__ part, WsHeader* hdr, const float* __restrict__ bias,
+                const uint32_t* __restrict__ mask, int words, __half* __restrict__ h16,
+                int batch, int sq) {
   pdl_wait();
   pdl_trigger();
   constexpr uint32_t A_BYTES = TC_M * TC_BK * 2;     // 16 KB
@@ -408,7 +410,44 @@ __global__ void __launch_bounds__(32 * TC_FFN_WARPS, 1)
   bool ok = tc_wait_quiet(done, 0u, hdr);
   ok = __all_sync(0xffffffffu, ok && !*abort && nkt > 0);
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-  if (ok && warp < 4) {
+  if (ok && warp < 4 && ks == 1) {
+    // one share of d per row tile: the accumulators are the pre-activations,
+    // so the activation is applied here, with the arithmetic of k_ffn_finish
+    // for one split (which then skips this layer), and h16 written directly
+    const int p = p0 + warp * 32 + lane;
+    int j = 0;
+    bool valid = false;
+    float bb = 0.f;
+    if (p < N) {
+      j = p < H ? p : idx[p - H];
+      if (p >= H && (j < H || j >= F)) {
+        if (hdr) atomicOr(&hdr->status, DEV_BAD_INDEX);
+      } else {
+        valid = true;
+        bb = bias ? bias[j] : 0.f;
+      }
+    }
+    __half* hrow = h16 + (size_t)(p / 64) * nt * 64 + (p % 64);
+    for (int c0 = 0; c0 < nt; c0 += 16) {
+      uint32_t gv16[16], uv16[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, gv16);
+      if constexpr (NR == 2) tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(nt + c0), uv16);
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int b = c0 + q;
+        float hv = 0.f;
+        if (valid && b < batch) {
+          const float gv = (0.f + __uint_as_float(gv16[q])) + bb;
+          hv = gv > 0.f ? gv : 0.f;
+          if constexpr (NR == 2) hv *= 0.f + __uint_as_float(uv16[q]);
+          else if (sq) hv *= hv;  // squared ReLU
+          if (mask && p >= H && !((__ldg(mask + (size_t)b * words + (j >> 5)) >> (j & 31)) & 1u))
+            hv = 0.f;
+        }
+        hrow[(size_t)b * 64] = __float2half_rn(hv);
+      }
+    }
+  } else if (ok && warp < 4) {
     const int p = p0 + warp * 32 + lane;
 #pragma unroll
     for (int r = 0; r < NR; ++r) {
@@ -891,7 +930,8 @@ __global__ void k_xh16(const float* __restrict__ xh, int batch, int d, int nt,
 // Partial sums read and h16 written coalesced through shared memory.
 template <int NR>
 __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ part, int g, int nk,
-                                                    int fit, int H, int F, int Fp, int nt, int batch,
+                                                    int fit, int direct, int H, int F, int Fp,
+                                                    int nt, int batch,
                                                     const int32_t* __restrict__ idx,
                                                     const int32_t* __restrict__ count,
                                                     const float* __restrict__ bias,
@@ -912,6 +952,7 @@ __global__ void __launch_bounds__(256) k_ffn_finish(const float* __restrict__ pa
   const int n0 = blockIdx.x * 64;
   if (n0 >= N) return;
   const UpShare us = up_share(N, g, nk, fit != 0);
+  if (direct && us.ks == 1) return;  // the up kernel applied the activation itself
   const int ks = us.ks, Np = us.nT * TC_M;
   const int m = 64 * nt;
   // per row once: neuron, index check, bias
@@ -1469,10 +1510,11 @@ cudaError_t launch_up_nr(const pi_layer& L, const float* xh, int batch, const ui
   e = allow_smem_fn(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   (void)launch_dep(kern, up_grid(F), 32 * TC_FFN_WARPS, smem, s, m0, m1, g0, g1, mx, nt, nk, g, H,
-                   F, idx, count, sc.part, hdr);
+                   F, idx, count, sc.part, hdr, L.bias, mask, (F + 31) / 32, sc.h16, batch,
+                   L.act == PI_RELU2 ? 1 : 0);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, 0, H, F, Fp, nt, batch, idx,
+  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, 0, 1, H, F, Fp, nt, batch, idx,
                    count, L.bias, mask, (F + 31) / 32, sc.h16, hdr, L.act == PI_RELU2 ? 1 : 0);
   return cudaGetLastError();
 }
@@ -1523,7 +1565,7 @@ cudaError_t launch_up_q4(const pi_layer& L, const float* xh, int batch, const ui
                    cc0, cc1, srb, d / 2, nt, nk, g, H, F, idx, count, sc.part, hdr);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, 1, H, F, Fp, nt, batch, idx,
+  (void)launch_dep(k_ffn_finish<NR>, Fp / 64, 256, 0, s, sc.part, g, nk, 1, 0, H, F, Fp, nt, batch, idx,
                    count, L.bias, mask, (F + 31) / 32, sc.h16, hdr, L.act == PI_RELU2 ? 1 : 0);
   return cudaGetLastError();
 }
