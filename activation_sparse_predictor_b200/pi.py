@@ -161,14 +161,18 @@ class Layer:
     def words(self) -> int:
         return (self.d_ff + 31) // 32
 
-    def with_host_cold_tier(self) -> "Layer":
+    def with_host_cold_tier(self, pin: bool = True) -> "Layer":
         """The same layer with rows [hot, d_ff) of w_gate / w_up / w_down_t
         (and their Q4_0 scales) read from page-locked host memory: each
         weight buffer's rows from `hot` on are copied to a pinned host
         buffer with the same row layout, and the descriptor's cold pointers
         point into it (see pi_layer).  The device tensors are shared with
-        this layer; the returned layer never reads their rows >= hot."""
+        this layer; the returned layer never reads their rows >= hot.
+        (pin=False leaves the copies in pageable memory, which the library
+        rejects: for checking the layout without a GPU.)"""
         import torch
+        if self.hot >= self.d_ff:
+            return self  # no cold rows: nothing to move
         bufs, host = {}, {}
 
         def base_of(t):  # the row-major buffer a weight view lives in
@@ -186,7 +190,7 @@ class Layer:
             key = b.data_ptr()
             if key not in host:
                 h = torch.empty((rows.shape[0] - self.hot, rows.shape[1]), dtype=rows.dtype,
-                                pin_memory=True)
+                                pin_memory=pin)
                 h.copy_(rows[self.hot:])
                 host[key] = h
                 bufs[key] = rows
