@@ -136,8 +136,10 @@ typedef enum pi_mask_mode { PI_MASK_PER_TOKEN = 0, PI_MASK_UNION = 1 } pi_mask_m
  * kernels.  Where those kernels would read a row more than once (several
  * token chunks, or the tensor cores' tiles), each call first copies the
  * listed cold rows into the workspace once (pi_workspace_bytes counts that
- * stage).  The host memory must stay allocated and unchanged until the
- * stream has run the call. */
+ * stage).  Each call looks the cold pointers up (cudaPointerGetAttributes,
+ * a few microseconds per layer on the host; also legal inside a stream
+ * capture in cudaStreamCaptureModeRelaxed).  The host memory must stay
+ * allocated and unchanged until the stream has run the call. */
 typedef struct pi_layer {
   int32_t d_model, d_ff, rank, hot;
   int32_t act, w_dtype, p_dtype;
