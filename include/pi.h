@@ -166,7 +166,9 @@ typedef struct pi_layer {
 
 /* Bytes of workspace the calls below need for these layers at this batch
  * size, on the current CUDA device (the split of the down projection
- * follows the device's SM count).  Returns 0 on invalid arguments. */
+ * follows the device's SM count; layers with a host-memory cold tier add
+ * the stage of their listed cold rows where the kernels use one).  Returns
+ * 0 on invalid arguments. */
 size_t pi_workspace_bytes(const pi_layer* layers, int n_layers, int batch);
 
 /* Clears the workspace's status word and wait counters; call once after
